@@ -1,0 +1,221 @@
+"""CPU oracle for reciprocal nearest-neighbour matching (MASt3R).
+
+TEST INFRASTRUCTURE ONLY. The tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg may import this package; the product path
+(``reciprocal_nearest_neighbours_b200``) never imports it, and this package
+imports nothing from the product path. The two share no code: only the seeded
+input generators in ``synth`` serve both.
+
+What the oracle computes, step by step, in the pages' order:
+
+* ``nn`` -- the nearest neighbour of each query descriptor in a database by
+  dot product, argmax_k <q, DB_k>, lowest index on ties ("MASt3R dissection",
+  section 3 Napkin Formula, the inference-time reciprocal matching set). The
+  scan itself is the plain C loop in ``oracle.c``.
+* ``dense_mutual`` -- the reciprocal (mutual nearest-neighbour) set
+  M = {(i, j) : NN(D1[i], D2) = j and NN(D2[j], D1) = i}
+  ("MASt3R dissection", section 1 architecture diagram and section 3; "DUSt3R
+  / MASt3R explained", the paragraph on fast reciprocal matching, which names
+  this the naive all-pixels computation).
+* ``fast_reciprocal`` -- MASt3R's fast reciprocal matching ("DUSt3R / MASt3R
+  explained", fast-matching paragraph): seeds on a sparse pixel grid of image
+  1; each is mapped to its best match in image 2 and that match is mapped back
+  to image 1; pixels that return to themselves are kept; the others continue
+  from where they landed, for at most ``max_iter`` rounds.
+
+Readings taken where the pages are silent (each listed in the design notes):
+dot-product similarity for unnormalised integer descriptors; lowest index on
+ties; grid origin (0, 0) with step ``subsample`` in x and y; convergence means
+u' == u; non-converged walks are dropped after ``max_iter`` rounds; the output
+is a set, unique by the image-1 pixel.
+
+Parity pins: every function here is checked in ``tests/test_oracle_*.py``
+against things other than itself (a library argmax over a matrix product,
+hand-worked fixtures in ``tests/golden``, closed-form special cases, brute
+force on tiny maps, and invariants the definition implies).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass, field
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``oracle.c`` into ``liboracle.so`` next to it (gcc, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-march=native", "-fopenmp", "-fPIC", "-shared",
+               "-std=c11", "-Wall", "-o", _LIB, _SRC]
+        try:
+            subprocess.run(cmd, check=True, capture_output=True, text=True)
+        except subprocess.CalledProcessError:
+            # -march=native can fail under some emulators; retry portable.
+            cmd.remove("-march=native")
+            subprocess.run(cmd, check=True, capture_output=True, text=True)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        I64 = ctypes.c_int64
+        lib.oracle_nn_i8.argtypes = [P, I64, P, I64, ctypes.c_int, P, P, ctypes.c_int]
+        lib.oracle_nn_i8.restype = ctypes.c_int
+        lib.oracle_nn_bf16.argtypes = [P, I64, P, I64, ctypes.c_int, P, P, P, ctypes.c_int]
+        lib.oracle_nn_bf16.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def default_threads() -> int:
+    return max(1, len(os.sched_getaffinity(0)))
+
+
+def _ptr(a: np.ndarray) -> int:
+    return a.ctypes.data
+
+
+@dataclass
+class NNResult:
+    idx: np.ndarray  # int32 [nq]
+    score: np.ndarray  # int64 (int8 descriptors) or float64 (bf16) [nq]
+    second: np.ndarray | None = None  # float64 runner-up score (bf16 only)
+
+
+def nn(q: np.ndarray, db: np.ndarray, dtype: str, nthreads: int | None = None) -> NNResult:
+    """Nearest neighbour of every row of ``q`` among the rows of ``db``.
+
+    ``q`` is [nq, d], ``db`` is [ndb, d]; int8 arrays for ``dtype == "i8"``,
+    uint16 bfloat16 bit patterns for ``dtype == "bf16"``.
+    """
+    lib = _load()
+    nthreads = default_threads() if nthreads is None else nthreads
+    q = np.ascontiguousarray(q)
+    db = np.ascontiguousarray(db)
+    nq, d = q.shape
+    ndb = db.shape[0]
+    assert db.shape[1] == d and ndb > 0
+    idx = np.empty(nq, dtype=np.int32)
+    if dtype == "i8":
+        assert q.dtype == np.int8 and db.dtype == np.int8
+        score = np.empty(nq, dtype=np.int64)
+        rc = lib.oracle_nn_i8(_ptr(q), nq, _ptr(db), ndb, d, _ptr(idx), _ptr(score), nthreads)
+        assert rc == 0
+        return NNResult(idx, score)
+    if dtype == "bf16":
+        assert q.dtype == np.uint16 and db.dtype == np.uint16
+        score = np.empty(nq, dtype=np.float64)
+        second = np.empty(nq, dtype=np.float64)
+        rc = lib.oracle_nn_bf16(_ptr(q), nq, _ptr(db), ndb, d, _ptr(idx), _ptr(score),
+                                _ptr(second), nthreads)
+        assert rc == 0
+        return NNResult(idx, score, second)
+    raise ValueError(dtype)
+
+
+def score_of(D1: np.ndarray, i: np.ndarray, D2: np.ndarray, j: np.ndarray, dtype: str) -> np.ndarray:
+    """Exact scores <D1[i], D2[j]> for paired index arrays (int64 or float64)."""
+    if dtype == "i8":
+        return (D1[i].astype(np.int64) * D2[j].astype(np.int64)).sum(axis=1)
+    a = (D1[i].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    b = (D2[j].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return (a * b).sum(axis=1)
+
+
+def grid_seeds(H: int, W: int, step: int) -> np.ndarray:
+    """Seed pixels y*W + x for x in {0, step, 2 step, ...} < W, y likewise < H."""
+    ys = np.arange(0, H, step, dtype=np.int64)
+    xs = np.arange(0, W, step, dtype=np.int64)
+    return (ys[:, None] * W + xs[None, :]).ravel()
+
+
+@dataclass
+class DenseResult:
+    pairs: np.ndarray  # int64 [m, 2] (i, j), ascending i
+    score: np.ndarray  # [m]
+    nn12: NNResult = None
+    nn21: NNResult = None
+
+
+def dense_mutual(D1: np.ndarray, D2: np.ndarray, dtype: str, nthreads: int | None = None) -> DenseResult:
+    """All mutual nearest-neighbour pairs between flattened maps D1 [N1,d], D2 [N2,d]."""
+    r12 = nn(D1, D2, dtype, nthreads)
+    r21 = nn(D2, D1, dtype, nthreads)
+    i = np.arange(D1.shape[0])
+    keep = r21.idx[r12.idx] == i
+    pairs = np.stack([i[keep], r12.idx[keep].astype(np.int64)], axis=1)
+    return DenseResult(pairs, r12.score[keep], r12, r21)
+
+
+@dataclass
+class FastResult:
+    pairs: np.ndarray  # int64 [m, 2] (u, v), sorted by u
+    score: np.ndarray  # [m]
+    frontier_sizes: list = field(default_factory=list)  # |F_t| per round run
+    first_seen: list = field(default_factory=list)  # new pixels per round run
+    min_gap: dict = field(default_factory=dict)  # bf16: kept pixel -> best walk's min top-2 gap
+
+
+def fast_reciprocal(D1: np.ndarray, H1: int, W1: int, D2: np.ndarray, H2: int, W2: int,
+                    dtype: str, subsample: int, max_iter: int,
+                    nthreads: int | None = None, track_gaps: bool = False) -> FastResult:
+    """MASt3R fast reciprocal matching from a sparse seed grid.
+
+    F_1 = grid seeds of image 1. Round t (t = 1 .. max_iter, while F_t is not
+    empty): for each u in F_t, v = NN(D1[u], D2) and u' = NN(D2[v], D1). If
+    u' == u the pair (u, v) is kept; otherwise u' joins F_{t+1}, which is
+    taken as a set. Walks still open after ``max_iter`` rounds are dropped.
+
+    ``first_seen[t-1]`` counts the members of F_t that appear in no earlier
+    frontier. With ``track_gaps`` (bf16), ``min_gap[u]`` for a kept pixel u
+    is, over all walks that end at u, the largest value of the smallest top-2
+    score gap met on that walk (forward and backward steps, u's own included):
+    when it is below a tolerance, every walk to u passes a near-tie.
+    """
+    D1 = D1.reshape(H1 * W1, -1)
+    D2 = D2.reshape(H2 * W2, -1)
+    F = [int(u) for u in grid_seeds(H1, W1, subsample)]
+    chain_gap = {u: np.inf for u in F}
+    kept = {}
+    kept_gap = {}
+    sizes, first = [], []
+    seen: set = set()
+    for _ in range(max_iter):
+        if not F:
+            break
+        sizes.append(len(F))
+        first.append(sum(1 for u in F if u not in seen))
+        seen.update(F)
+        fwd = nn(D1[np.array(F)], D2, dtype, nthreads)
+        bwd = nn(D2[fwd.idx], D1, dtype, nthreads)
+        nxt_gap = {}
+        for k, u in enumerate(F):
+            v = int(fwd.idx[k])
+            u2 = int(bwd.idx[k])
+            g = np.inf
+            if track_gaps:
+                g = min(chain_gap[u], fwd.score[k] - fwd.second[k],
+                        bwd.score[k] - bwd.second[k])
+            if u2 == u:
+                kept[u] = (v, fwd.score[k])
+                kept_gap[u] = max(kept_gap.get(u, -np.inf), g)
+            else:
+                nxt_gap[u2] = max(nxt_gap.get(u2, -np.inf), g)
+        F = sorted(nxt_gap)
+        chain_gap = nxt_gap
+    us = sorted(kept)
+    pairs = np.array([[u, kept[u][0]] for u in us], dtype=np.int64).reshape(-1, 2)
+    sc = np.array([kept[u][1] for u in us], dtype=np.float64 if dtype == "bf16" else np.int64)
+    return FastResult(pairs, sc, sizes, first, kept_gap if track_gaps else {})

@@ -1,0 +1,71 @@
+"""Brute-force restatements used to pin the oracle (pure Python, tiny inputs).
+
+Each function states the definition in a different form from the oracle's
+running scan, so that a slip in one is caught by the other:
+
+* ``nn_by_definition``: the lowest index k whose score equals the row maximum
+  (the argmax set first, then its minimum).
+* ``mutual_by_quantifiers``: (i, j) is kept iff j beats every k < j strictly
+  and ties-or-beats every k > j in row i, and i does the same in column j.
+* ``walks``: follows every seed's walk u -> NN21(NN12(u)) on its own, without
+  frontiers or sets, and reads the fast scheme's result off the walks.
+"""
+
+from __future__ import annotations
+
+
+def dot(a, b):
+    return sum(int(x) * int(y) for x, y in zip(a, b))
+
+
+def nn_by_definition(q, db):
+    scores = [dot(q, row) for row in db]
+    m = max(scores)
+    return min(k for k, s in enumerate(scores) if s == m), m
+
+
+def mutual_by_quantifiers(D1, D2):
+    n1, n2 = len(D1), len(D2)
+    S = [[dot(D1[i], D2[j]) for j in range(n2)] for i in range(n1)]
+    out = []
+    for i in range(n1):
+        for j in range(n2):
+            row_ok = all(S[i][j] > S[i][k] for k in range(j)) and \
+                all(S[i][j] >= S[i][k] for k in range(j + 1, n2))
+            col_ok = all(S[i][j] > S[k][j] for k in range(i)) and \
+                all(S[i][j] >= S[k][j] for k in range(i + 1, n1))
+            if row_ok and col_ok:
+                out.append((i, j, S[i][j]))
+    return out
+
+
+def walk_step(u, D1, D2):
+    v, s = nn_by_definition(D1[u], D2)
+    u2, _ = nn_by_definition(D2[v], D1)
+    return v, s, u2
+
+
+def walks(seeds, D1, D2, max_iter):
+    """Per-seed walks. Returns (kept set of (u, v, s), list of walks).
+
+    A seed's walk visits u_0 = seed, u_1, ... with u_{t+1} = NN21(NN12(u_t));
+    it is kept iff some u_t with t <= max_iter - 1 is a fixed point (it stops
+    there). Each walk is returned as (nodes, scores, fixed_or_None).
+    """
+    kept = set()
+    info = []
+    for s0 in seeds:
+        u = s0
+        nodes, scores = [u], []
+        fixed = None
+        for t in range(max_iter):
+            v, s, u2 = walk_step(u, D1, D2)
+            scores.append(s)
+            if u2 == u:
+                fixed = (u, v, s)
+                kept.add(fixed)
+                break
+            u = u2
+            nodes.append(u)
+        info.append((nodes, scores, fixed))
+    return kept, info
