@@ -1,0 +1,159 @@
+/*
+ * fastnn.h -- C ABI of the B200 (sm_100a) reciprocal nearest-neighbour
+ * matcher for dense per-pixel descriptor maps (MASt3R's matching step).
+ *
+ * What is computed
+ *   Similarity of two descriptors is their dot product; the nearest
+ *   neighbour of a query in a database is argmax_k <q, db_k>, the LOWEST k
+ *   among equal scores ("MASt3R dissection", section 3 Napkin Formula: the
+ *   inference-time reciprocal set is written with argmax of dot products).
+ *   A reciprocal match is a pair (i, j) with NN(D1[i], D2) = j and
+ *   NN(D2[j], D1) = i ("MASt3R dissection", section 1 architecture diagram
+ *   and section 3).
+ *
+ * Conventions shared by every entry point
+ *   - Every data pointer is a DEVICE pointer owned by the caller. The library
+ *     allocates no memory: scratch lives in a caller-provided workspace whose
+ *     size comes from fastnn_workspace_size(). Workspace and descriptor
+ *     pointers must be 256-byte aligned.
+ *   - Descriptor maps are row-major [rows][d] (an image is [H][W][d], pixel
+ *     index p = y * W + x); batches are [batch][rows][d].
+ *   - dtype FASTNN_I8: int8 descriptors, int32 scores (exact).
+ *     dtype FASTNN_BF16: bfloat16 descriptors (raw 16-bit patterns), float32
+ *     scores (fp32 accumulation of exact bf16 products).
+ *     1 <= d <= 32 for both.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream). The host blocks only in fastnn_device_status().
+ *   - Return value: FASTNN_OK, or a negative fastnn_status describing an
+ *     argument or launch error detected on the host; nothing has been
+ *     enqueued when an argument error is returned. Errors found on the
+ *     device (a bounded wait that ran out) are recorded in the workspace and
+ *     read with fastnn_device_status().
+ *   - Calls that share a workspace must be ordered (same stream or events);
+ *     overlapping calls on one workspace race.
+ */
+#ifndef FASTNN_H_
+#define FASTNN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *fastnn_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    FASTNN_OK = 0,
+    FASTNN_ERR_INVALID = -1,     /* bad pointer, size, alignment or argument */
+    FASTNN_ERR_UNSUPPORTED = -2, /* d or dtype outside what the kernels take */
+    FASTNN_ERR_CAPACITY = -3,    /* output capacity or workspace too small */
+    FASTNN_ERR_CUDA = -4,        /* a CUDA runtime call or launch failed */
+    FASTNN_ERR_TIMEOUT = -5      /* a device-side bounded wait ran out */
+} fastnn_status;
+
+typedef enum { FASTNN_I8 = 0, FASTNN_BF16 = 1 } fastnn_dtype;
+
+typedef enum { FASTNN_OP_NN = 0, FASTNN_OP_RECIPROCAL = 1, FASTNN_OP_MUTUAL_DENSE = 2 } fastnn_op;
+
+/*
+ * Workspace bytes one call needs.
+ *   FASTNN_OP_NN:           n1 = nq, n2 = ndb (batch and max_queries unused)
+ *   FASTNN_OP_RECIPROCAL:   n1 = H1*W1, n2 = H2*W2, max_queries = number of
+ *                           grid seeds per pair, batch = pairs
+ *   FASTNN_OP_MUTUAL_DENSE: n1, n2 = pixel counts (batch, max_queries unused)
+ * Returns 0 for arguments no call would accept.
+ */
+size_t fastnn_workspace_size(int op, int64_t n1, int64_t n2, int d, int dtype,
+                             int batch, int64_t max_queries);
+
+/*
+ * fastnn_nn -- nearest neighbour of every query row in a database.
+ *   For i < nq: out_idx[i] = argmax_k <q[i], db[k]> (lowest k on ties),
+ *   out_score[i] = that score (int32 for FASTNN_I8, float for FASTNN_BF16;
+ *   out_score may be NULL). This is the primitive of both matching schemes
+ *   ("MASt3R dissection", section 3, argmax of dot products).
+ *   q: [nq][d], db: [ndb][d]; nq >= 0, ndb >= 1; nq == 0 is a no-op.
+ */
+int fastnn_nn(const void *q, int64_t nq, const void *db, int64_t ndb, int d,
+              int dtype, int32_t *out_idx, void *out_score, void *workspace,
+              size_t workspace_bytes, fastnn_stream_t stream);
+
+/*
+ * fastnn_reciprocal -- MASt3R fast reciprocal matching ("DUSt3R / MASt3R
+ * explained", the paragraph on fast reciprocal matching: seeds on a sparse
+ * grid of image 1 are mapped to their best match in image 2 and back; pixels
+ * that map onto themselves are kept; the others walk on).
+ *   Seeds: pixels (x, y) of image 1 with x, y multiples of `subsample`
+ *   (origin 0), S = ceil(H1/subsample) * ceil(W1/subsample) per pair.
+ *   Round t = 1..max_iter while the frontier is non-empty: for u in the
+ *   frontier, v = NN(D1[u], D2), u' = NN(D2[v], D1); u' == u keeps (u, v);
+ *   otherwise u' joins the next frontier unless it was already in any
+ *   frontier of this call (a pruning that leaves the kept set unchanged: the
+ *   walk from a pixel is deterministic, and its first visit is the furthest
+ *   ahead). Walks still open after max_iter rounds are dropped.
+ *   desc1: [batch][H1][W1][d], desc2: [batch][H2][W2][d]; pairs independent.
+ *   out_pairs: [batch][capacity][2] int32 (u, v) pixel indices in order of
+ *   discovery (round, then frontier position); out_score: [batch][capacity]
+ *   (int32 or float) or NULL; out_count: [batch] int32 pairs written per
+ *   pair; out_iters: [batch] int32 rounds run with a non-empty frontier, or
+ *   NULL; out_frontier: [batch][max_iter] int32 frontier size of each round
+ *   (0 for rounds not run), or NULL. capacity must be >= S (at most one pair
+ *   per seed), else
+ *   FASTNN_ERR_CAPACITY. 1 <= subsample, 1 <= max_iter <= 255, S < 2^24.
+ */
+int fastnn_reciprocal(const void *desc1, int H1, int W1, const void *desc2,
+                      int H2, int W2, int d, int dtype, int subsample,
+                      int max_iter, int batch, int32_t *out_pairs,
+                      void *out_score, int64_t capacity, int32_t *out_count,
+                      int32_t *out_iters, int32_t *out_frontier,
+                      void *workspace, size_t workspace_bytes,
+                      fastnn_stream_t stream);
+
+/*
+ * fastnn_mutual_dense -- every mutual nearest-neighbour pair of two maps,
+ * the brute-force reciprocal set ("MASt3R dissection", section 1 and section
+ * 3; "DUSt3R / MASt3R explained" calls it the naive every-pixel-against-
+ * every-pixel comparison that the fast scheme avoids).
+ *   desc1: [n1][d], desc2: [n2][d]. Output pairs (i, j) in ascending i into
+ *   out_pairs [capacity][2] int32 and out_score [capacity] (or NULL);
+ *   *out_count (device int32) = number of pairs. capacity must be
+ *   >= min(n1, n2), else FASTNN_ERR_CAPACITY.
+ */
+int fastnn_mutual_dense(const void *desc1, int64_t n1, const void *desc2,
+                        int64_t n2, int d, int dtype, int32_t *out_pairs,
+                        void *out_score, int64_t capacity, int32_t *out_count,
+                        void *workspace, size_t workspace_bytes,
+                        fastnn_stream_t stream);
+
+/*
+ * fastnn_device_status -- synchronise `stream` and read the device status
+ * word of the last call that used `workspace`: FASTNN_OK, or
+ * FASTNN_ERR_TIMEOUT when a kernel's bounded wait ran out (its outputs are
+ * then invalid). Blocks the host.
+ */
+int fastnn_device_status(const void *workspace, fastnn_stream_t stream);
+
+/*
+ * Benchmark instrumentation (not needed for matching). After
+ * fastnn_kernel_timer_enable(capacity > 0), each of the next `capacity`
+ * launches of the tensor-core nearest-neighbour kernel is bracketed by two
+ * CUDA events recorded on the launching stream (events are created here, once,
+ * not per call). fastnn_kernel_timer_read() waits for the recorded events,
+ * returns the number of timed launches and their summed device time in
+ * milliseconds, and starts a new count. fastnn_kernel_timer_enable(0)
+ * destroys the events. Process-wide state: not for concurrent use from
+ * several host threads.
+ */
+int fastnn_kernel_timer_enable(int capacity);
+int fastnn_kernel_timer_read(int *launches, double *total_ms);
+
+/* Human-readable name of a fastnn_status value (static string). */
+const char *fastnn_status_str(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FASTNN_H_ */

@@ -170,7 +170,8 @@ class FastResult:
 
 def fast_reciprocal(D1: np.ndarray, H1: int, W1: int, D2: np.ndarray, H2: int, W2: int,
                     dtype: str, subsample: int, max_iter: int,
-                    nthreads: int | None = None, track_gaps: bool = False) -> FastResult:
+                    nthreads: int | None = None, track_gaps: bool = False,
+                    seeds: np.ndarray | None = None) -> FastResult:
     """MASt3R fast reciprocal matching from a sparse seed grid.
 
     F_1 = grid seeds of image 1. Round t (t = 1 .. max_iter, while F_t is not
@@ -186,7 +187,9 @@ def fast_reciprocal(D1: np.ndarray, H1: int, W1: int, D2: np.ndarray, H2: int, W
     """
     D1 = D1.reshape(H1 * W1, -1)
     D2 = D2.reshape(H2 * W2, -1)
-    F = [int(u) for u in grid_seeds(H1, W1, subsample)]
+    if seeds is None:
+        seeds = grid_seeds(H1, W1, subsample)
+    F = [int(u) for u in seeds]
     chain_gap = {u: np.inf for u in F}
     kept = {}
     kept_gap = {}

@@ -1,0 +1,31 @@
+"""B200-native reciprocal nearest-neighbour matching of dense descriptor maps.
+
+Python binding of ``libfastnn.so`` (declared in ``include/fastnn.h``). The
+functions here only marshal arguments: they take CUDA tensors, allocate the
+outputs and the workspace with PyTorch when the caller does not pass them, and
+call the C ABI on the current CUDA stream. Every step of the matching runs in
+the library's sm_100a kernels; there is no other implementation to fall back
+to, and loading fails loudly when the library is missing.
+"""
+
+from __future__ import annotations
+
+from ._lib import (  # noqa: F401
+    FASTNN_BF16,
+    FASTNN_I8,
+    FASTNN_OP_MUTUAL_DENSE,
+    FASTNN_OP_NN,
+    FASTNN_OP_RECIPROCAL,
+    FastNNError,
+    fastnn_device_status,
+    fastnn_kernel_timer_enable,
+    fastnn_kernel_timer_read,
+    fastnn_mutual_dense,
+    fastnn_nn,
+    fastnn_reciprocal,
+    fastnn_status_str,
+    fastnn_workspace_size,
+    library,
+    library_path,
+    seed_count,
+)

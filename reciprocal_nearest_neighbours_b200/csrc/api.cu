@@ -1,0 +1,326 @@
+// C ABI entry points (declared in include/fastnn.h): argument checks,
+// workspace carving and the launch sequence of each operation. No memory is
+// allocated here; every launch goes on the caller's stream.
+#include <cstring>
+
+#include "common.cuh"
+#include "frontier.cuh"
+#include "nn_tc.cuh"
+
+using namespace fastnn;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr int kPadRows = 256;  // zero rows after each repacked database (one TMA box)
+constexpr int kMaxIter = 255;
+constexpr int64_t kMaxSeeds = (int64_t{1} << 24) - 1;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+// Bump allocator over the caller's workspace (or a size-only dry run).
+struct Carver {
+  uint8_t* base;
+  size_t off = 0;
+  template <typename T>
+  T* take(size_t count) {
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off = align_up(off + count * sizeof(T));
+    return p;
+  }
+};
+
+bool dtype_ok(int dtype) { return dtype == FASTNN_I8 || dtype == FASTNN_BF16; }
+
+struct NNLayout {
+  int* status;
+  uint8_t* qrep;
+  uint8_t* dbrep;
+  uint64_t* keys;
+};
+NNLayout carve_nn(Carver& c, int64_t nq, int64_t ndb, int dtype) {
+  NNLayout L;
+  const int rb = row_bytes(dtype);
+  L.status = c.take<int>(64);
+  L.qrep = c.take<uint8_t>(static_cast<size_t>(nq) * rb);
+  L.dbrep = c.take<uint8_t>(static_cast<size_t>(ndb + kPadRows) * rb);
+  L.keys = c.take<uint64_t>(static_cast<size_t>(nq));
+  return L;
+}
+
+struct RecLayout {
+  int* status;
+  uint8_t* d1rep;
+  uint8_t* d2rep;
+  int32_t* F[2];
+  uint64_t* fwd;
+  uint64_t* bwd;
+  uint32_t* claim;
+  int32_t* cnt[2];
+};
+RecLayout carve_rec(Carver& c, int64_t N1, int64_t N2, int dtype, int batch, int64_t S) {
+  RecLayout L;
+  const int rb = row_bytes(dtype);
+  L.status = c.take<int>(64);
+  L.d1rep = c.take<uint8_t>(static_cast<size_t>(batch * N1 + kPadRows) * rb);
+  L.d2rep = c.take<uint8_t>(static_cast<size_t>(batch * N2 + kPadRows) * rb);
+  L.F[0] = c.take<int32_t>(static_cast<size_t>(batch) * S);
+  L.F[1] = c.take<int32_t>(static_cast<size_t>(batch) * S);
+  L.fwd = c.take<uint64_t>(static_cast<size_t>(batch) * S);
+  L.bwd = c.take<uint64_t>(static_cast<size_t>(batch) * S);
+  L.claim = c.take<uint32_t>(static_cast<size_t>(batch) * N1);
+  L.cnt[0] = c.take<int32_t>(static_cast<size_t>(batch));
+  L.cnt[1] = c.take<int32_t>(static_cast<size_t>(batch));
+  return L;
+}
+
+struct MutLayout {
+  int* status;
+  uint8_t* d1rep;
+  uint8_t* d2rep;
+  uint64_t* k12;
+  uint64_t* k21;
+  int32_t* blocks;
+};
+MutLayout carve_mut(Carver& c, int64_t n1, int64_t n2, int dtype) {
+  MutLayout L;
+  const int rb = row_bytes(dtype);
+  L.status = c.take<int>(64);
+  L.d1rep = c.take<uint8_t>(static_cast<size_t>(n1 + kPadRows) * rb);
+  L.d2rep = c.take<uint8_t>(static_cast<size_t>(n2 + kPadRows) * rb);
+  L.k12 = c.take<uint64_t>(static_cast<size_t>(n1));
+  L.k21 = c.take<uint64_t>(static_cast<size_t>(n2));
+  L.blocks = c.take<int32_t>(static_cast<size_t>(mutual_blocks(n1)));
+  return L;
+}
+
+int64_t seed_count(int H, int W, int sub) {
+  return static_cast<int64_t>((H + sub - 1) / sub) * ((W + sub - 1) / sub);
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+#define FASTNN_TRY(expr)              \
+  do {                                \
+    int rc_ = (expr);                 \
+    if (rc_ != FASTNN_OK) return rc_; \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+size_t fastnn_workspace_size(int op, int64_t n1, int64_t n2, int d, int dtype, int batch,
+                             int64_t max_queries) {
+  if (!dtype_ok(dtype) || d < 1 || d > 32 || n1 < 0 || n2 < 1) return 0;
+  Carver c{nullptr};
+  switch (op) {
+    case FASTNN_OP_NN:
+      carve_nn(c, n1, n2, dtype);
+      break;
+    case FASTNN_OP_RECIPROCAL:
+      if (batch < 1 || max_queries < 1 || n1 < 1) return 0;
+      carve_rec(c, n1, n2, dtype, batch, max_queries);
+      break;
+    case FASTNN_OP_MUTUAL_DENSE:
+      if (n1 < 1) return 0;
+      carve_mut(c, n1, n2, dtype);
+      break;
+    default:
+      return 0;
+  }
+  return c.off;
+}
+
+int fastnn_nn(const void* q, int64_t nq, const void* db, int64_t ndb, int d, int dtype,
+              int32_t* out_idx, void* out_score, void* workspace, size_t workspace_bytes,
+              fastnn_stream_t stream) {
+  if (!dtype_ok(dtype) || d < 1 || d > 32) return FASTNN_ERR_UNSUPPORTED;
+  if (nq < 0 || ndb < 1 || nq > INT32_MAX || ndb > INT32_MAX - kPadRows) return FASTNN_ERR_INVALID;
+  if (nq == 0) return FASTNN_OK;
+  if (!q || !db || !out_idx || !workspace || !aligned(workspace, kAlign)) return FASTNN_ERR_INVALID;
+  if (workspace_bytes < fastnn_workspace_size(FASTNN_OP_NN, nq, ndb, d, dtype, 1, 0))
+    return FASTNN_ERR_CAPACITY;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  Carver c{static_cast<uint8_t*>(workspace)};
+  NNLayout L = carve_nn(c, nq, ndb, dtype);
+  FASTNN_CUDA_TRY(cudaMemsetAsync(L.status, 0, sizeof(int), st));
+  FASTNN_CUDA_TRY(cudaMemsetAsync(L.keys, 0, static_cast<size_t>(nq) * sizeof(uint64_t), st));
+  FASTNN_TRY(launch_repack(q, nq, d, dtype, L.qrep, 0, st));
+  FASTNN_TRY(launch_repack(db, ndb, d, dtype, L.dbrep, kPadRows, st));
+  NNArgs a{};
+  a.q_rows = L.qrep;
+  a.q_rows_per_pair = nq;
+  a.q_cap = nq;
+  a.nq_static = nq;
+  a.db_rows = L.dbrep;
+  a.ndb = ndb;
+  a.out_key = L.keys;
+  a.batch = 1;
+  a.status = L.status;
+  FASTNN_TRY(launch_nn_tc(a, dtype, ndb + kPadRows, st));
+  return launch_decode(L.keys, nq, dtype, out_idx, out_score, st);
+}
+
+int fastnn_reciprocal(const void* desc1, int H1, int W1, const void* desc2, int H2, int W2, int d,
+                      int dtype, int subsample, int max_iter, int batch, int32_t* out_pairs,
+                      void* out_score, int64_t capacity, int32_t* out_count, int32_t* out_iters,
+                      int32_t* out_frontier, void* workspace, size_t workspace_bytes,
+                      fastnn_stream_t stream) {
+  if (!dtype_ok(dtype) || d < 1 || d > 32) return FASTNN_ERR_UNSUPPORTED;
+  if (H1 < 1 || W1 < 1 || H2 < 1 || W2 < 1 || subsample < 1 || max_iter < 1 ||
+      max_iter > kMaxIter || batch < 1 || batch > nn_tc_max_batch())
+    return FASTNN_ERR_INVALID;
+  const int64_t N1 = static_cast<int64_t>(H1) * W1;
+  const int64_t N2 = static_cast<int64_t>(H2) * W2;
+  if (batch * N1 > INT32_MAX - kPadRows || batch * N2 > INT32_MAX - kPadRows)
+    return FASTNN_ERR_INVALID;
+  const int64_t S = seed_count(H1, W1, subsample);
+  if (S > kMaxSeeds) return FASTNN_ERR_INVALID;
+  if (!desc1 || !desc2 || !out_pairs || !out_count || !workspace || !aligned(workspace, kAlign))
+    return FASTNN_ERR_INVALID;
+  if (capacity < S) return FASTNN_ERR_CAPACITY;
+  if (workspace_bytes <
+      fastnn_workspace_size(FASTNN_OP_RECIPROCAL, N1, N2, d, dtype, batch, S))
+    return FASTNN_ERR_CAPACITY;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  Carver c{static_cast<uint8_t*>(workspace)};
+  RecLayout L = carve_rec(c, N1, N2, dtype, batch, S);
+
+  FASTNN_CUDA_TRY(cudaMemsetAsync(L.status, 0, sizeof(int), st));
+  FASTNN_CUDA_TRY(cudaMemsetAsync(L.fwd, 0, static_cast<size_t>(batch) * S * 8, st));
+  FASTNN_CUDA_TRY(cudaMemsetAsync(L.bwd, 0, static_cast<size_t>(batch) * S * 8, st));
+  FASTNN_CUDA_TRY(cudaMemsetAsync(L.claim, 0xFF, static_cast<size_t>(batch) * N1 * 4, st));
+  FASTNN_CUDA_TRY(cudaMemsetAsync(out_count, 0, static_cast<size_t>(batch) * 4, st));
+  if (out_iters) FASTNN_CUDA_TRY(cudaMemsetAsync(out_iters, 0, static_cast<size_t>(batch) * 4, st));
+  if (out_frontier)
+    FASTNN_CUDA_TRY(cudaMemsetAsync(out_frontier, 0, static_cast<size_t>(batch) * max_iter * 4, st));
+  FASTNN_TRY(launch_repack(desc1, batch * N1, d, dtype, L.d1rep, kPadRows, st));
+  FASTNN_TRY(launch_repack(desc2, batch * N2, d, dtype, L.d2rep, kPadRows, st));
+  FASTNN_TRY(launch_seed(L.F[0], S, L.claim, N1, L.cnt[0], H1, W1, subsample,
+                         static_cast<int>(S), batch, st));
+
+  for (int t = 1; t <= max_iter; ++t) {
+    const int cur = (t - 1) & 1, nxt = t & 1;
+    NNArgs fwd{};
+    fwd.q_rows = L.d1rep;
+    fwd.q_rows_per_pair = N1;
+    fwd.q_index = L.F[cur];
+    fwd.q_cap = S;
+    fwd.q_count = L.cnt[cur];
+    fwd.db_rows = L.d2rep;
+    fwd.ndb = N2;
+    fwd.out_key = L.fwd;
+    fwd.batch = batch;
+    fwd.status = L.status;
+    FASTNN_TRY(launch_nn_tc(fwd, dtype, batch * N2 + kPadRows, st));
+
+    NNArgs bwd{};
+    bwd.q_rows = L.d2rep;
+    bwd.q_rows_per_pair = N2;
+    bwd.q_key = L.fwd;
+    bwd.q_cap = S;
+    bwd.q_count = L.cnt[cur];
+    bwd.db_rows = L.d1rep;
+    bwd.ndb = N1;
+    bwd.out_key = L.bwd;
+    bwd.batch = batch;
+    bwd.status = L.status;
+    FASTNN_TRY(launch_nn_tc(bwd, dtype, batch * N1 + kPadRows, st));
+
+    CompactArgs ca{};
+    ca.F_cur = L.F[cur];
+    ca.F_next = L.F[nxt];
+    ca.S_cap = S;
+    ca.cnt_cur = L.cnt[cur];
+    ca.cnt_next = L.cnt[nxt];
+    ca.fwd_key = L.fwd;
+    ca.bwd_key = L.bwd;
+    ca.claim = L.claim;
+    ca.N1 = N1;
+    ca.out_pairs = out_pairs;
+    ca.out_score = out_score;
+    ca.cap = capacity;
+    ca.out_count = out_count;
+    ca.out_iters = out_iters;
+    ca.out_frontier = out_frontier;
+    ca.max_iter = max_iter;
+    FASTNN_TRY(launch_check_compact(ca, dtype, t, t == max_iter, batch, st));
+  }
+  return FASTNN_OK;
+}
+
+int fastnn_mutual_dense(const void* desc1, int64_t n1, const void* desc2, int64_t n2, int d,
+                        int dtype, int32_t* out_pairs, void* out_score, int64_t capacity,
+                        int32_t* out_count, void* workspace, size_t workspace_bytes,
+                        fastnn_stream_t stream) {
+  if (!dtype_ok(dtype) || d < 1 || d > 32) return FASTNN_ERR_UNSUPPORTED;
+  if (n1 < 1 || n2 < 1 || n1 > INT32_MAX - kPadRows || n2 > INT32_MAX - kPadRows)
+    return FASTNN_ERR_INVALID;
+  if (!desc1 || !desc2 || !out_pairs || !out_count || !workspace || !aligned(workspace, kAlign))
+    return FASTNN_ERR_INVALID;
+  if (capacity < (n1 < n2 ? n1 : n2)) return FASTNN_ERR_CAPACITY;
+  if (workspace_bytes < fastnn_workspace_size(FASTNN_OP_MUTUAL_DENSE, n1, n2, d, dtype, 1, 0))
+    return FASTNN_ERR_CAPACITY;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  Carver c{static_cast<uint8_t*>(workspace)};
+  MutLayout L = carve_mut(c, n1, n2, dtype);
+  FASTNN_CUDA_TRY(cudaMemsetAsync(L.status, 0, sizeof(int), st));
+  FASTNN_CUDA_TRY(cudaMemsetAsync(L.k12, 0, static_cast<size_t>(n1) * 8, st));
+  FASTNN_CUDA_TRY(cudaMemsetAsync(L.k21, 0, static_cast<size_t>(n2) * 8, st));
+  FASTNN_TRY(launch_repack(desc1, n1, d, dtype, L.d1rep, kPadRows, st));
+  FASTNN_TRY(launch_repack(desc2, n2, d, dtype, L.d2rep, kPadRows, st));
+  NNArgs a{};
+  a.q_rows = L.d1rep;
+  a.q_rows_per_pair = n1;
+  a.q_cap = n1;
+  a.nq_static = n1;
+  a.db_rows = L.d2rep;
+  a.ndb = n2;
+  a.out_key = L.k12;
+  a.batch = 1;
+  a.status = L.status;
+  FASTNN_TRY(launch_nn_tc(a, dtype, n2 + kPadRows, st));
+  NNArgs r{};
+  r.q_rows = L.d2rep;
+  r.q_rows_per_pair = n2;
+  r.q_cap = n2;
+  r.nq_static = n2;
+  r.db_rows = L.d1rep;
+  r.ndb = n1;
+  r.out_key = L.k21;
+  r.batch = 1;
+  r.status = L.status;
+  FASTNN_TRY(launch_nn_tc(r, dtype, n1 + kPadRows, st));
+  return launch_mutual(L.k12, L.k21, n1, n2, L.blocks, dtype, out_pairs, out_score, capacity,
+                       out_count, st);
+}
+
+int fastnn_device_status(const void* workspace, fastnn_stream_t stream) {
+  if (!workspace) return FASTNN_ERR_INVALID;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int h = 0;
+  FASTNN_CUDA_TRY(cudaMemcpyAsync(&h, workspace, sizeof(int), cudaMemcpyDeviceToHost, st));
+  FASTNN_CUDA_TRY(cudaStreamSynchronize(st));
+  return (h & kStatusTimeout) ? FASTNN_ERR_TIMEOUT : FASTNN_OK;
+}
+
+int fastnn_kernel_timer_enable(int capacity) { return kernel_timer_enable(capacity); }
+
+int fastnn_kernel_timer_read(int* launches, double* total_ms) {
+  return kernel_timer_read(launches, total_ms);
+}
+
+const char* fastnn_status_str(int status) {
+  switch (status) {
+    case FASTNN_OK: return "FASTNN_OK";
+    case FASTNN_ERR_INVALID: return "FASTNN_ERR_INVALID";
+    case FASTNN_ERR_UNSUPPORTED: return "FASTNN_ERR_UNSUPPORTED";
+    case FASTNN_ERR_CAPACITY: return "FASTNN_ERR_CAPACITY";
+    case FASTNN_ERR_CUDA: return "FASTNN_ERR_CUDA";
+    case FASTNN_ERR_TIMEOUT: return "FASTNN_ERR_TIMEOUT";
+    default: return "FASTNN_UNKNOWN_STATUS";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,88 @@
+// Shared device helpers for the fastnn kernels (sm_100a).
+//
+// Score/index packing: a nearest-neighbour result is carried as one 64-bit
+// key whose unsigned order is (score ascending, index descending):
+//   key = (ordered_bits(score) << 32) | (0xFFFFFFFF - index)
+// so the maximum key over a set of candidates is the highest score with the
+// LOWEST index among equal scores, and partial results from any number of
+// CTAs merge with one 64-bit atomicMax in any order, deterministically.
+// key == 0 means "no candidate yet".
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "../../include/fastnn.h"
+
+namespace fastnn {
+
+constexpr int kStatusTimeout = 1;  // bit set in the device status word
+
+__host__ __device__ __forceinline__ uint32_t ord_i32(int32_t s) {
+  return static_cast<uint32_t>(s) ^ 0x80000000u;
+}
+__host__ __device__ __forceinline__ int32_t unord_i32(uint32_t h) {
+  return static_cast<int32_t>(h ^ 0x80000000u);
+}
+__device__ __forceinline__ uint32_t ord_f32(float s) {
+  s += 0.0f;  // -0 -> +0 so that equal scores share one key
+  uint32_t u = __float_as_uint(s);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float unord_f32(uint32_t h) {
+  uint32_t u = (h & 0x80000000u) ? (h & 0x7FFFFFFFu) : ~h;
+  return __uint_as_float(u);
+}
+__host__ __device__ __forceinline__ uint64_t make_key(uint32_t ord_score, uint32_t idx) {
+  return (static_cast<uint64_t>(ord_score) << 32) | static_cast<uint64_t>(0xFFFFFFFFu - idx);
+}
+__host__ __device__ __forceinline__ uint32_t key_index(uint64_t key) {
+  return 0xFFFFFFFFu - static_cast<uint32_t>(key);
+}
+__host__ __device__ __forceinline__ uint32_t key_score_bits(uint64_t key) {
+  return static_cast<uint32_t>(key >> 32);
+}
+
+// Bytes of one repacked descriptor row: d <= 32 elements zero-padded to 32.
+__host__ __device__ constexpr int row_bytes(int dtype) { return dtype == FASTNN_I8 ? 32 : 64; }
+
+// Where the query rows of one nearest-neighbour pass come from.
+//   row id of slot k of pair b:
+//     q_index != nullptr : q_index[b * q_cap + k]
+//     q_key   != nullptr : key_index(q_key[b * q_cap + k])   (chained pass)
+//     otherwise          : k
+//   rows live in q_rows + (b * q_rows_per_pair + row) * row_bytes.
+//   Active slots of pair b: q_count ? q_count[b] : nq_static.
+struct NNArgs {
+  const uint8_t* q_rows;
+  int64_t q_rows_per_pair;
+  const int32_t* q_index;
+  const uint64_t* q_key;
+  int64_t q_cap;
+  const int32_t* q_count;
+  int64_t nq_static;
+  const uint8_t* db_rows;  // repacked database rows [batch][ndb][row_bytes]
+  int64_t ndb;
+  uint64_t* out_key;       // [batch][q_cap], merged with atomicMax
+  int batch;
+  int* status;
+};
+
+__device__ __forceinline__ int64_t nn_count(const NNArgs& a, int b) {
+  return a.q_count ? static_cast<int64_t>(a.q_count[b]) : a.nq_static;
+}
+
+__device__ __forceinline__ int64_t nn_query_row(const NNArgs& a, int b, int64_t k) {
+  if (a.q_index) return a.q_index[b * a.q_cap + k];
+  if (a.q_key) return key_index(a.q_key[b * a.q_cap + k]);
+  return k;
+}
+
+}  // namespace fastnn
+
+#define FASTNN_CUDA_TRY(expr)                              \
+  do {                                                     \
+    cudaError_t e_ = (expr);                               \
+    if (e_ != cudaSuccess) return FASTNN_ERR_CUDA;         \
+  } while (0)

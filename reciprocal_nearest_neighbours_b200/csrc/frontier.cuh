@@ -1,0 +1,41 @@
+// Launchers of the memory-bound kernels (frontier.cu).
+#pragma once
+
+#include "common.cuh"
+
+namespace fastnn {
+
+// Per-round state of the fast scheme, all device pointers.
+struct CompactArgs {
+  const int32_t* F_cur;   // [batch][S_cap] frontier of this round
+  int32_t* F_next;        // [batch][S_cap] frontier of the next round
+  int64_t S_cap;
+  const int32_t* cnt_cur; // [batch]
+  int32_t* cnt_next;      // [batch]
+  uint64_t* fwd_key;      // [batch][S_cap] NN12 of the frontier (reset to 0 here)
+  uint64_t* bwd_key;      // [batch][S_cap] NN21 of those matches (reset to 0 here)
+  uint32_t* claim;        // [batch][N1] first-visit stamps (round << 24 | slot)
+  int64_t N1;
+  int32_t* out_pairs;     // [batch][cap][2]
+  void* out_score;        // [batch][cap] or nullptr
+  int64_t cap;
+  int32_t* out_count;     // [batch]
+  int32_t* out_iters;     // [batch] or nullptr
+  int32_t* out_frontier;  // [batch][max_iter] or nullptr
+  int max_iter;
+};
+
+int launch_repack(const void* src, int64_t rows, int d, int dtype, void* dst, int64_t pad_rows,
+                  cudaStream_t st);
+int launch_seed(int32_t* F0, int64_t S_cap, uint32_t* claim, int64_t N1, int32_t* cnt0, int H1,
+                int W1, int sub, int S, int batch, cudaStream_t st);
+int launch_check_compact(const CompactArgs& c, int dtype, int t, bool last_round, int batch,
+                         cudaStream_t st);
+int mutual_blocks(int64_t n1);
+int launch_mutual(const uint64_t* k12, const uint64_t* k21, int64_t n1, int64_t n2,
+                  int32_t* block_scratch, int dtype, int32_t* out_pairs, void* out_score,
+                  int64_t cap, int32_t* out_count, cudaStream_t st);
+int launch_decode(const uint64_t* key, int64_t n, int dtype, int32_t* out_idx, void* out_score,
+                  cudaStream_t st);
+
+}  // namespace fastnn

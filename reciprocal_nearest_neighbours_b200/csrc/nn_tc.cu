@@ -1,0 +1,516 @@
+// Nearest neighbour by dot product on the 5th-generation tensor cores.
+//
+// For every active query slot k of every pair b:
+//     out_key[b][k] = max over db rows j of key(<q_k, db_j>, j)
+// i.e. the highest score with the lowest index among ties ("MASt3R
+// dissection", section 3 Napkin Formula: argmax of dot products, the
+// primitive of both the dense reciprocal set and the fast scheme).
+//
+// Design (one persistent CTA per SM, warp-specialised):
+//   warps 0..7  epilogue: tcgen05.ld the 128 x 256 score tile from TMEM and
+//               fold it into a running (max score, lowest index) per query
+//               row; warpgroup 0 takes columns 0..127, warpgroup 1 128..255.
+//               The score matrix never leaves the SM.
+//   warp 8      producer: gathers the 128 query rows of a tile into shared
+//               memory (swizzled, K-major) and streams 256-row database tiles
+//               with TMA (cp.async.bulk.tensor, no multicast) into a
+//               kStages-deep ring.
+//   warp 9      MMA issuer (one thread): tcgen05.mma kind::i8 (int8 -> int32,
+//               K = 32) or kind::f16 (bf16 -> fp32, 2 x K = 16) into one of
+//               two 256-column TMEM accumulators, tcgen05.commit to free the
+//               database stage and to hand the accumulator to the epilogue.
+// Work: units (pair, 128-query tile, 256-row database tile) in row-major
+// order, split into contiguous ranges over the CTAs; a CTA merges each
+// query tile's partial result with one 64-bit atomicMax per row, which is
+// order independent. Descriptors are zero-padded to 32 elements (32 B int8
+// rows, 64 B bf16 rows) by the repack kernel, so the padding adds nothing.
+// Every mbarrier wait is bounded; on expiry the kernel records
+// FASTNN_ERR_TIMEOUT in the status word, drains what it issued and exits.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "nn_tc.cuh"
+#include "ptx.cuh"
+
+namespace fastnn {
+
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kBN = 256;
+constexpr int kStages = 6;
+constexpr int kAcc = 2;
+constexpr int kEpiWarps = 8;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kThreads = 320;
+constexpr int kMaxBatch = 1024;
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+
+// Barrier slots inside the barrier block.
+constexpr int kBarBFull = 0;
+constexpr int kBarBEmpty = kBarBFull + kStages;
+constexpr int kBarAFull = kBarBEmpty + kStages;
+constexpr int kBarAEmpty = kBarAFull + 2;
+constexpr int kBarAccFull = kBarAEmpty + 2;
+constexpr int kBarAccEmpty = kBarAccFull + kAcc;
+constexpr int kBarDone = kBarAccEmpty + kAcc;
+constexpr int kNumBars = kBarDone + 1;
+
+struct Ctl {
+  uint64_t bars[kNumBars];
+  uint32_t tmem_base;
+  int abort_flag;
+  int b0;
+  int64_t m0, n0, u0, u1, nt;
+  int mt[kMaxBatch];
+  int cnt[kMaxBatch];
+};
+
+__host__ __device__ constexpr size_t tile_bytes_a(int rb) { return static_cast<size_t>(kBM) * rb; }
+__host__ __device__ constexpr size_t tile_bytes_b(int rb) { return static_cast<size_t>(kBN) * rb; }
+
+size_t smem_bytes(int rb) {
+  return 1024 /* alignment slack */ + 2 * tile_bytes_a(rb) + kStages * tile_bytes_b(rb) +
+         sizeof(Ctl);
+}
+
+// Bounded wait on an mbarrier phase. Returns false (and raises the abort flag
+// and the device status) if the phase did not complete within kTimeoutNs, or
+// if another role already aborted.
+__device__ bool wait_bounded(uint32_t bar, uint32_t parity, Ctl* ctl, int* status) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer_ns();
+  while (true) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (*reinterpret_cast<volatile int*>(&ctl->abort_flag)) return false;
+    if (ptx::globaltimer_ns() - t0 > kTimeoutNs) {
+      *reinterpret_cast<volatile int*>(&ctl->abort_flag) = 1;
+      atomicOr(status, kStatusTimeout);
+      return false;
+    }
+  }
+}
+
+// Warp-uniform bounded wait: every lane polls, the warp proceeds only if all
+// lanes saw the phase complete.
+__device__ bool warp_wait_bounded(uint32_t bar, uint32_t parity, Ctl* ctl, int* status) {
+  const bool ok = wait_bounded(bar, parity, ctl, status);
+  return __all_sync(0xffffffffu, ok);
+}
+
+struct Pos {
+  int b;
+  int64_t m, n;
+};
+
+__device__ __forceinline__ void advance(Pos& p, const Ctl* ctl, int batch) {
+  if (++p.n == ctl->nt) {
+    p.n = 0;
+    if (++p.m == ctl->mt[p.b]) {
+      p.m = 0;
+      do {
+        ++p.b;
+      } while (p.b < batch && ctl->mt[p.b] == 0);
+    }
+  }
+}
+
+// Query-tile gather: 32 lanes copy 128 rows of `rb` bytes into a K-major tile
+// with the 32B (rb = 32) or 64B (rb = 64) swizzle the MMA descriptor names:
+// the 16-byte chunk c of row r lands at r * rb + 16 * (c ^ swz(r)).
+template <int RB>
+__device__ __forceinline__ void gather_a(uint8_t* tile, const NNArgs& a, int b, int64_t m,
+                                         int cnt, int lane) {
+  constexpr int kChunks = RB / 16;
+#pragma unroll
+  for (int i = 0; i < kBM / 32; ++i) {
+    const int r = lane + 32 * i;
+    const int64_t k = m * kBM + r;
+    uint4 v[kChunks];
+    const int64_t row = k < cnt ? nn_query_row(a, b, k) : -1;
+    // Rows outside the query source (never produced by a healthy pipeline)
+    // read as zeros instead of faulting.
+    if (row >= 0 && row < a.q_rows_per_pair) {
+      const uint4* src = reinterpret_cast<const uint4*>(
+          a.q_rows + (static_cast<int64_t>(b) * a.q_rows_per_pair + row) * RB);
+#pragma unroll
+      for (int c = 0; c < kChunks; ++c) v[c] = __ldg(src + c);
+    } else {
+#pragma unroll
+      for (int c = 0; c < kChunks; ++c) v[c] = make_uint4(0, 0, 0, 0);
+    }
+    const int swz = RB == 32 ? ((r >> 2) & 1) : ((r >> 1) & 3);
+#pragma unroll
+    for (int c = 0; c < kChunks; ++c)
+      *reinterpret_cast<uint4*>(tile + r * RB + 16 * (c ^ swz)) = v[c];
+  }
+}
+
+template <int DT>
+struct Epi;
+
+// int8 descriptors: int32 scores.
+template <>
+struct Epi<FASTNN_I8> {
+  using S = int32_t;
+  static __device__ __forceinline__ S lowest() { return INT32_MIN; }
+  static __device__ __forceinline__ S as_score(uint32_t r) { return static_cast<int32_t>(r); }
+  static __device__ __forceinline__ S mx(S x, S y) { return max(x, y); }
+  static __device__ __forceinline__ uint32_t ord(S s) { return ord_i32(s); }
+};
+
+// bf16 descriptors: fp32 scores.
+template <>
+struct Epi<FASTNN_BF16> {
+  using S = float;
+  static __device__ __forceinline__ S lowest() { return -INFINITY; }
+  static __device__ __forceinline__ S as_score(uint32_t r) { return __uint_as_float(r); }
+  static __device__ __forceinline__ S mx(S x, S y) { return fmaxf(x, y); }
+  static __device__ __forceinline__ uint32_t ord(S s) { return ord_f32(s); }
+};
+
+// Fold 32 consecutive columns (global index col0 + j) into (best, bidx).
+// The chunk maximum is taken first; only when it beats the running best
+// strictly is the chunk rescanned for the first column holding it, so the
+// lowest index among equal scores survives. `valid` < 32 masks a ragged
+// database tail.
+template <int DT>
+__device__ __forceinline__ void fold32(const uint32_t (&r)[32], uint32_t col0, int valid,
+                                       typename Epi<DT>::S& best, uint32_t& bidx) {
+  using E = Epi<DT>;
+  using S = typename E::S;
+  S v[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = (j < valid) ? E::as_score(r[j]) : E::lowest();
+  S m = v[0];
+#pragma unroll
+  for (int j = 1; j < 32; ++j) m = E::mx(m, v[j]);
+  if (m > best) {
+    int first = 31;
+#pragma unroll
+    for (int j = 31; j >= 0; --j)
+      if (v[j] == m) first = j;
+    best = m;
+    bidx = col0 + first;
+  }
+}
+
+template <int DT>
+__global__ void __launch_bounds__(kThreads, 1)
+    nn_tc_kernel(const __grid_constant__ CUtensorMap tmap_db, NNArgs a) {
+  constexpr int RB = row_bytes(DT);
+  using E = Epi<DT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* tileA = smem;                              // 2 x kBM x RB
+  uint8_t* tileB = tileA + 2 * tile_bytes_a(RB);      // kStages x kBN x RB
+  Ctl* ctl = reinterpret_cast<Ctl*>(tileB + kStages * tile_bytes_b(RB));
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int batch = a.batch;
+
+  // ---- work range of this CTA (thread 0), barrier init --------------------
+  if (threadIdx.x == 0) {
+    const int64_t nt = (a.ndb + kBN - 1) / kBN;
+    int64_t total = 0;
+    for (int b = 0; b < batch; ++b) {
+      const int64_t c = nn_count(a, b);
+      ctl->cnt[b] = static_cast<int>(c);
+      ctl->mt[b] = static_cast<int>((c + kBM - 1) / kBM);
+      total += static_cast<int64_t>(ctl->mt[b]) * nt;
+    }
+    const int64_t G = gridDim.x;
+    const int64_t u0 = total * blockIdx.x / G;
+    const int64_t u1 = total * (blockIdx.x + 1) / G;
+    ctl->nt = nt;
+    ctl->u0 = u0;
+    ctl->u1 = u1;
+    ctl->abort_flag = 0;
+    int64_t acc = 0;
+    int b = 0;
+    while (b < batch && acc + static_cast<int64_t>(ctl->mt[b]) * nt <= u0) {
+      acc += static_cast<int64_t>(ctl->mt[b]) * nt;
+      ++b;
+    }
+    ctl->b0 = b;
+    const int64_t rem = u0 - acc;
+    ctl->m0 = nt > 0 ? rem / nt : 0;
+    ctl->n0 = nt > 0 ? rem % nt : 0;
+    for (int i = 0; i < kNumBars; ++i) {
+      uint32_t count = 1;
+      if (i >= kBarAFull && i < kBarAFull + 2) count = 32;        // producer lanes
+      if (i >= kBarAccEmpty && i < kBarAccEmpty + kAcc) count = kEpiWarps;
+      ptx::mbar_init(ptx::smem_u32(&ctl->bars[i]), count);
+    }
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+  const int64_t u0 = ctl->u0, u1 = ctl->u1;
+  if (u0 >= u1) return;  // uniform over the CTA: nothing was allocated yet
+
+  if (warp == 0) {
+    ptx::tmem_alloc(ptx::smem_u32(&ctl->tmem_base), 512);
+    ptx::tmem_relinquish();
+  }
+  if (warp == kProducerWarp && lane == 0) ptx::prefetch_tmap(&tmap_db);
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+
+  auto bar = [&](int i) { return ptx::smem_u32(&ctl->bars[i]); };
+  const Pos start{ctl->b0, ctl->m0, ctl->n0};
+  const int64_t nt = ctl->nt;
+
+  if (warp == kProducerWarp) {
+    // ---------------------------------------------------------------- producer
+    Pos p = start;
+    int64_t it = 0, seg = 0;
+    int64_t last_issue[kStages];
+#pragma unroll
+    for (int s = 0; s < kStages; ++s) last_issue[s] = -1;
+    for (int64_t u = u0; u < u1; ++u) {
+      if (u == u0 || p.n == 0) {
+        const int as = static_cast<int>(seg & 1);
+        if (!warp_wait_bounded(bar(kBarAEmpty + as), static_cast<uint32_t>(((seg >> 1) & 1) ^ 1),
+                               ctl, a.status))
+          break;
+        gather_a<RB>(tileA + as * tile_bytes_a(RB), a, p.b, p.m, ctl->cnt[p.b], lane);
+        ptx::fence_proxy_async_smem();
+        ptx::mbar_arrive(bar(kBarAFull + as));
+        ++seg;
+      }
+      const int s = static_cast<int>(it % kStages);
+      const uint32_t ph = static_cast<uint32_t>((it / kStages) & 1);
+      bool ok = true;
+      if (lane == 0) {
+        ok = wait_bounded(bar(kBarBEmpty + s), ph ^ 1, ctl, a.status);
+        if (ok) {
+          ptx::mbar_arrive_expect_tx(bar(kBarBFull + s), static_cast<uint32_t>(tile_bytes_b(RB)));
+          ptx::tma_load_2d(ptx::smem_u32(tileB + s * tile_bytes_b(RB)), &tmap_db, 0,
+                           static_cast<int32_t>(static_cast<int64_t>(p.b) * a.ndb + p.n * kBN),
+                           bar(kBarBFull + s));
+          last_issue[s] = it;
+        }
+      }
+      if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
+      ++it;
+      advance(p, ctl, batch);
+    }
+    // Drain: every TMA load this warp issued must land before smem is freed.
+    if (lane == 0) {
+      for (int s = 0; s < kStages; ++s)
+        if (last_issue[s] >= 0)
+          wait_bounded(bar(kBarBFull + s), static_cast<uint32_t>((last_issue[s] / kStages) & 1),
+                       ctl, a.status);
+    }
+  } else if (warp == kMmaWarp) {
+    // --------------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      constexpr uint32_t kIdesc =
+          DT == FASTNN_I8
+              ? ((2u << 4) | (1u << 7) | (1u << 10) | ((kBN >> 3) << 17) | ((kBM >> 4) << 24))
+              : ((1u << 4) | (1u << 7) | (1u << 10) | ((kBN >> 3) << 17) | ((kBM >> 4) << 24));
+      Pos p = start;
+      int64_t it = 0, seg = 0;
+      int as = 0;
+      for (int64_t u = u0; u < u1; ++u) {
+        if (u == u0 || p.n == 0) {
+          as = static_cast<int>(seg & 1);
+          if (!wait_bounded(bar(kBarAFull + as), static_cast<uint32_t>((seg >> 1) & 1), ctl,
+                            a.status))
+            break;
+          ptx::tc_fence_after();
+          ++seg;
+        }
+        const int acc = static_cast<int>(it & 1);
+        if (!wait_bounded(bar(kBarAccEmpty + acc), static_cast<uint32_t>(((it >> 1) & 1) ^ 1), ctl,
+                          a.status))
+          break;
+        ptx::tc_fence_after();
+        const int s = static_cast<int>(it % kStages);
+        if (!wait_bounded(bar(kBarBFull + s), static_cast<uint32_t>((it / kStages) & 1), ctl,
+                          a.status))
+          break;
+        ptx::tc_fence_after();
+        const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * kBN);
+        const uint64_t adesc =
+            ptx::smem_desc_kmajor(ptx::smem_u32(tileA + as * tile_bytes_a(RB)), RB);
+        const uint64_t bdesc =
+            ptx::smem_desc_kmajor(ptx::smem_u32(tileB + s * tile_bytes_b(RB)), RB);
+        if constexpr (DT == FASTNN_I8) {
+          ptx::mma_i8(d_tmem, adesc, bdesc, kIdesc, 0u);
+        } else {
+          // K = 32 bf16 = two K = 16 steps; the second starts 32 bytes in.
+          ptx::mma_bf16(d_tmem, adesc, bdesc, kIdesc, 0u);
+          ptx::mma_bf16(d_tmem, adesc + 2, bdesc + 2, kIdesc, 1u);
+        }
+        ptx::mma_commit(bar(kBarBEmpty + s));
+        ptx::mma_commit(bar(kBarAccFull + acc));
+        const bool seg_end = (u + 1 == u1) || (p.n == nt - 1);
+        if (seg_end) ptx::mma_commit(bar(kBarAEmpty + as));
+        ++it;
+        advance(p, ctl, batch);
+      }
+      // Every MMA issued above completes before TMEM is released.
+      ptx::mma_commit(bar(kBarDone));
+      wait_bounded(bar(kBarDone), 0, ctl, a.status);
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int lg = warp & 3;  // TMEM lane quarter this warp may access
+    const int h = warp >> 2;  // column half of the 256-wide tile
+    Pos p = start;
+    int64_t it = 0;
+    typename E::S best = E::lowest();
+    uint32_t bidx = 0xFFFFFFFFu;
+    const int tail = static_cast<int>(a.ndb - (nt - 1) * kBN);  // valid columns, last tile
+    for (int64_t u = u0; u < u1; ++u) {
+      const int acc = static_cast<int>(it & 1);
+      if (!warp_wait_bounded(bar(kBarAccFull + acc), static_cast<uint32_t>((it >> 1) & 1), ctl,
+                             a.status))
+        break;
+      ptx::tc_fence_after();
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(lg * 32) << 16) +
+                             static_cast<uint32_t>(acc * kBN + h * (kBN / 2));
+      const uint32_t colbase = static_cast<uint32_t>(p.n * kBN + h * (kBN / 2));
+      const int valid_tile = (p.n == nt - 1) ? tail - h * (kBN / 2) : kBN / 2;
+#pragma unroll
+      for (int c = 0; c < (kBN / 2) / 32; ++c) {
+        uint32_t r[32];
+        ptx::tmem_ld32(taddr + c * 32, r);
+        ptx::tmem_ld_wait();
+        const int valid = min(32, max(0, valid_tile - c * 32));
+        fold32<DT>(r, colbase + c * 32, valid, best, bidx);
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(kBarAccEmpty + acc));
+      const bool seg_end = (u + 1 == u1) || (p.n == nt - 1);
+      if (seg_end) {
+        const int64_t k = p.m * kBM + lg * 32 + lane;
+        if (k < ctl->cnt[p.b] && bidx != 0xFFFFFFFFu)
+          atomicMax(reinterpret_cast<unsigned long long*>(&a.out_key[p.b * a.q_cap + k]),
+                    static_cast<unsigned long long>(make_key(E::ord(best), bidx)));
+        best = E::lowest();
+        bidx = 0xFFFFFFFFu;
+      }
+      ++it;
+      advance(p, ctl, batch);
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  if (warp == 0) ptx::tmem_dealloc(tmem, 512);
+}
+
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                              const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                              const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn get_encode() {
+  static EncodeFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(p);
+  }
+  return fn;
+}
+
+// Optional event pairs around launches (benchmark instrumentation).
+struct KernelTimer {
+  cudaEvent_t* ev = nullptr;  // 2 * cap events
+  int cap = 0;
+  int used = 0;
+};
+KernelTimer g_timer;
+
+}  // namespace
+
+int kernel_timer_enable(int capacity) {
+  if (g_timer.ev) {
+    for (int i = 0; i < 2 * g_timer.cap; ++i) cudaEventDestroy(g_timer.ev[i]);
+    delete[] g_timer.ev;
+    g_timer = KernelTimer{};
+  }
+  if (capacity <= 0) return FASTNN_OK;
+  g_timer.ev = new cudaEvent_t[2 * capacity];
+  for (int i = 0; i < 2 * capacity; ++i)
+    if (cudaEventCreate(&g_timer.ev[i]) != cudaSuccess) {
+      for (int j = 0; j < i; ++j) cudaEventDestroy(g_timer.ev[j]);
+      delete[] g_timer.ev;
+      g_timer = KernelTimer{};
+      return FASTNN_ERR_CUDA;
+    }
+  g_timer.cap = capacity;
+  return FASTNN_OK;
+}
+
+int kernel_timer_read(int* launches, double* total_ms) {
+  double ms = 0.0;
+  for (int i = 0; i < g_timer.used; ++i) {
+    FASTNN_CUDA_TRY(cudaEventSynchronize(g_timer.ev[2 * i + 1]));
+    float x = 0.f;
+    FASTNN_CUDA_TRY(cudaEventElapsedTime(&x, g_timer.ev[2 * i], g_timer.ev[2 * i + 1]));
+    ms += x;
+  }
+  if (launches) *launches = g_timer.used;
+  if (total_ms) *total_ms = ms;
+  g_timer.used = 0;
+  return FASTNN_OK;
+}
+
+int nn_tc_min_rows() { return kBN; }
+int nn_tc_max_batch() { return kMaxBatch; }
+
+int launch_nn_tc(const NNArgs& a, int dtype, int64_t db_total_rows, cudaStream_t stream) {
+  const int rb = row_bytes(dtype);
+  if (db_total_rows < kBN || a.batch < 1 || a.batch > kMaxBatch) return FASTNN_ERR_INVALID;
+  EncodeFn encode = get_encode();
+  if (!encode) return FASTNN_ERR_CUDA;
+  CUtensorMap tm;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(rb), static_cast<cuuint64_t>(db_total_rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(rb)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(rb), static_cast<cuuint32_t>(kBN)};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a.db_rows), dims,
+                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      rb == 32 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return FASTNN_ERR_INVALID;
+
+  int dev = 0, sms = 0;
+  FASTNN_CUDA_TRY(cudaGetDevice(&dev));
+  FASTNN_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  const size_t smem = smem_bytes(rb);
+  const int slot = (g_timer.ev && g_timer.used < g_timer.cap) ? g_timer.used++ : -1;
+  if (slot >= 0) FASTNN_CUDA_TRY(cudaEventRecord(g_timer.ev[2 * slot], stream));
+  if (dtype == FASTNN_I8) {
+    FASTNN_CUDA_TRY(cudaFuncSetAttribute(nn_tc_kernel<FASTNN_I8>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem)));
+    nn_tc_kernel<FASTNN_I8><<<sms, kThreads, smem, stream>>>(tm, a);
+  } else {
+    FASTNN_CUDA_TRY(cudaFuncSetAttribute(nn_tc_kernel<FASTNN_BF16>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem)));
+    nn_tc_kernel<FASTNN_BF16><<<sms, kThreads, smem, stream>>>(tm, a);
+  }
+  FASTNN_CUDA_TRY(cudaGetLastError());
+  if (slot >= 0) FASTNN_CUDA_TRY(cudaEventRecord(g_timer.ev[2 * slot + 1], stream));
+  return FASTNN_OK;
+}
+
+}  // namespace fastnn

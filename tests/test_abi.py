@@ -1,0 +1,110 @@
+"""Host-side checks of the C ABI (no GPU, no compute calls).
+
+The library must load, export every function include/fastnn.h declares, size
+workspaces consistently, and reject bad arguments on the host before it
+touches the device.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import reciprocal_nearest_neighbours_b200 as fnn
+from reciprocal_nearest_neighbours_b200 import build as fnn_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include"))
+           if f.endswith(".h")]
+
+
+@pytest.fixture(scope="module")
+def lib():
+    fnn_build.build()
+    return fnn.library()
+
+
+def _declared():
+    names = []
+    for h in HEADERS:
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names += re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(fastnn_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert {"fastnn_nn", "fastnn_reciprocal", "fastnn_mutual_dense",
+            "fastnn_workspace_size", "fastnn_device_status", "fastnn_status_str"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+        assert ctypes.cast(getattr(lib, n), ctypes.c_void_p).value
+
+
+def test_status_strings(lib):
+    assert fnn.fastnn_status_str(0) == "FASTNN_OK"
+    assert fnn.fastnn_status_str(-3) == "FASTNN_ERR_CAPACITY"
+    assert fnn.fastnn_status_str(-5) == "FASTNN_ERR_TIMEOUT"
+    assert fnn.fastnn_status_str(42) == "FASTNN_UNKNOWN_STATUS"
+
+
+def test_workspace_sizes(lib):
+    ws = fnn.fastnn_workspace_size
+    a = ws(fnn.FASTNN_OP_RECIPROCAL, 196608, 196608, 24, fnn.FASTNN_I8, 1, 3072)
+    b = ws(fnn.FASTNN_OP_RECIPROCAL, 196608, 196608, 24, fnn.FASTNN_BF16, 1, 3072)
+    c = ws(fnn.FASTNN_OP_RECIPROCAL, 147456, 147456, 32, fnn.FASTNN_I8, 16, 9216)
+    assert 0 < a < b and c > 16 * a // 2
+    assert a % 256 == 0
+    # int8 repacked maps: 2 x (N + 256) rows x 32 B, plus claims and frontier state
+    assert a >= 2 * (196608 + 256) * 32 + 196608 * 4
+    assert ws(fnn.FASTNN_OP_NN, 10, 1000, 24, fnn.FASTNN_I8) > 1000 * 32
+    assert ws(fnn.FASTNN_OP_MUTUAL_DENSE, 3072, 3072, 24, fnn.FASTNN_I8) > 2 * 3072 * 40
+    # unsupported arguments size to 0
+    assert ws(fnn.FASTNN_OP_NN, 10, 10, 33, fnn.FASTNN_I8) == 0
+    assert ws(fnn.FASTNN_OP_NN, 10, 10, 0, fnn.FASTNN_I8) == 0
+    assert ws(fnn.FASTNN_OP_NN, 10, 10, 24, 7) == 0
+    assert ws(7, 10, 10, 24, fnn.FASTNN_I8) == 0
+    assert ws(fnn.FASTNN_OP_RECIPROCAL, 10, 10, 24, fnn.FASTNN_I8, 0, 5) == 0
+
+
+def test_argument_errors_are_reported_on_the_host(lib):
+    """Every call here fails validation before any CUDA API is reached."""
+    P = ctypes.c_void_p
+    fake = P(1 << 20)  # never dereferenced: validation rejects first
+    big = 1 << 30
+    I8 = fnn.FASTNN_I8
+    # unsupported d / dtype
+    assert lib.fastnn_nn(fake, 4, fake, 4, 33, I8, fake, None, fake, big, None) == -2
+    assert lib.fastnn_nn(fake, 4, fake, 4, 24, 5, fake, None, fake, big, None) == -2
+    # empty query set is a no-op, even with null pointers
+    assert lib.fastnn_nn(None, 0, None, 4, 24, I8, None, None, None, 0, None) == 0
+    # empty database, null output, misaligned workspace, small workspace
+    assert lib.fastnn_nn(fake, 4, fake, 0, 24, I8, fake, None, fake, big, None) == -1
+    assert lib.fastnn_nn(fake, 4, fake, 4, 24, I8, None, None, fake, big, None) == -1
+    assert lib.fastnn_nn(fake, 4, fake, 4, 24, I8, fake, None, P((1 << 20) + 8), big, None) == -1
+    assert lib.fastnn_nn(fake, 4, fake, 4, 24, I8, fake, None, fake, 16, None) == -3
+    # reciprocal: capacity below the seed count, bad rounds, bad batch
+    rec = lib.fastnn_reciprocal
+    S = fnn.seed_count(48, 64, 8)
+    assert S == 48
+    assert rec(fake, 48, 64, fake, 48, 64, 24, I8, 8, 10, 1, fake, None, S - 1, fake, None,
+               None, fake, big, None) == -3
+    assert rec(fake, 48, 64, fake, 48, 64, 24, I8, 8, 0, 1, fake, None, S, fake, None,
+               None, fake, big, None) == -1
+    assert rec(fake, 48, 64, fake, 48, 64, 24, I8, 8, 256, 1, fake, None, S, fake, None,
+               None, fake, big, None) == -1
+    assert rec(fake, 48, 64, fake, 48, 64, 24, I8, 0, 10, 1, fake, None, S, fake, None,
+               None, fake, big, None) == -1
+    assert rec(fake, 48, 64, fake, 48, 64, 24, I8, 8, 10, 0, fake, None, S, fake, None,
+               None, fake, big, None) == -1
+    assert rec(fake, 48, 64, fake, 48, 64, 24, I8, 8, 10, 1, fake, None, S, fake, None,
+               None, fake, 64, None) == -3
+    # dense: capacity below min(n1, n2)
+    mut = lib.fastnn_mutual_dense
+    assert mut(fake, 100, fake, 50, 24, I8, fake, None, 49, fake, fake, big, None) == -3
+    assert mut(fake, 0, fake, 50, 24, I8, fake, None, 49, fake, fake, big, None) == -1
+    assert mut(fake, 100, fake, 50, 24, I8, None, None, 50, fake, fake, big, None) == -1

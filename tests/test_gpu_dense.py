@@ -1,0 +1,110 @@
+"""GPU parity of fastnn_mutual_dense (all mutual nearest-neighbour pairs)."""
+
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from reciprocal_nearest_neighbours_b200 import fastnn_mutual_dense, fastnn_reciprocal
+from tests._dev import BF16_TOL, gpu_pairs, require_cuda, to_dev
+from tests.test_oracle import _load_golden
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _cuda():
+    require_cuda()
+
+
+def run_dense(D1, D2):
+    pairs, score, count = fastnn_mutual_dense(to_dev(D1), to_dev(D2))
+    torch.cuda.synchronize()
+    return gpu_pairs(pairs, score, count)
+
+
+def check_dense_int8(D1, D2):
+    p, s = run_dense(D1, D2)
+    ref = oracle.dense_mutual(D1, D2, "i8")
+    assert np.array_equal(p, ref.pairs)  # same pairs, same (ascending) order
+    assert np.array_equal(s.astype(np.int64), ref.score)
+    return p
+
+
+def test_golden_fixture():
+    fx = _load_golden("chain_2x2_1x3_d2.txt")
+    _, _, m1 = fx["image1"]
+    _, _, m2 = fx["image2"]
+    p, s = run_dense(m1.reshape(-1, 2), m2.reshape(-1, 2))
+    exp = fx["dense"]
+    assert [(int(a), int(b), int(c)) for (a, b), c in zip(p.tolist(), s.tolist())] == \
+        [tuple(exp[k:k + 3]) for k in range(0, len(exp), 3)]
+
+
+def test_tiny_config_exact():
+    w = synth.make_workload("tiny_64x48_d24_i8")
+    p = w.pairs[0]
+    got = check_dense_int8(p.desc1.reshape(-1, 24), p.desc2.reshape(-1, 24))
+    # the tiny pair's planted correspondences are largely mutual
+    assert len(got) > 1000
+
+
+@pytest.mark.parametrize("n1,n2,d,amp", [(1000, 777, 24, 8), (1, 1, 3, 2), (300, 5000, 7, 1),
+                                         (2049, 4095, 32, 16), (513, 129, 1, 3)])
+def test_random_ragged_sizes(n1, n2, d, amp):
+    rng = np.random.default_rng(n1 + n2 + d)
+    D1 = rng.integers(-amp, amp + 1, size=(n1, d)).astype(np.int8)
+    D2 = rng.integers(-amp, amp + 1, size=(n2, d)).astype(np.int8)
+    check_dense_int8(D1, D2)
+
+
+def test_bf16_small_within_tolerance():
+    m = synth.warped_pair_bf16(31, H=48, W=64)
+    D1 = m.desc1.reshape(-1, 24)
+    D2 = m.desc2.reshape(-1, 24)
+    p, s = run_dense(D1, D2)
+    exact = oracle.score_of(D1, p[:, 0], D2, p[:, 1], "bf16")
+    assert np.all(np.abs(s - exact) <= BF16_TOL)
+    ref = oracle.dense_mutual(D1, D2, "bf16")
+    got = set(map(tuple, p.tolist()))
+    exp = set(map(tuple, ref.pairs.tolist()))
+    for i, j in got ^ exp:
+        # a disagreement needs a near-tie in row i or in the column of its partner
+        g12 = ref.nn12.score[i] - ref.nn12.second[i]
+        jj = ref.nn12.idx[i]
+        g21 = ref.nn21.score[jj] - ref.nn21.second[jj]
+        g21b = ref.nn21.score[j] - ref.nn21.second[j]
+        assert min(g12, g21, g21b) < BF16_TOL
+
+
+def test_dense_512x384_full_size_sampled():
+    """The 196,608 x 196,608 workload: structure of the whole output, and the
+    oracle's verdict on sampled pixels and on sampled output pairs."""
+    m = synth.make_workload("dense_512x384_d24_i8").pairs[0]
+    D1 = m.desc1.reshape(-1, 24)
+    D2 = m.desc2.reshape(-1, 24)
+    p, s = run_dense(D1, D2)
+    assert len(p) > 10000
+    assert np.all(np.diff(p[:, 0]) > 0)  # ascending, unique i
+    assert len(np.unique(p[:, 1])) == len(p)  # unique j
+    assert np.array_equal(s.astype(np.int64), oracle.score_of(D1, p[:, 0], D2, p[:, 1], "i8"))
+    rng = np.random.default_rng(4)
+    # sampled output pairs are mutual
+    sel = p[rng.choice(len(p), size=400, replace=False)]
+    assert np.array_equal(oracle.nn(D1[sel[:, 0]], D2, "i8").idx, sel[:, 1])
+    assert np.array_equal(oracle.nn(D2[sel[:, 1]], D1, "i8").idx, sel[:, 0])
+    # sampled pixels: in the output exactly when the oracle says mutual
+    probe = np.sort(rng.choice(D1.shape[0], size=400, replace=False))
+    v = oracle.nn(D1[probe], D2, "i8").idx
+    back = oracle.nn(D2[v], D1, "i8").idx
+    mutual = {int(i): int(j) for i, j, b in zip(probe, v, back) if b == i}
+    out = dict(map(tuple, p.tolist()))
+    for i in probe.tolist():
+        assert out.get(i) == mutual.get(i)
+    # the fast scheme on the same maps keeps a subset of the dense set
+    fp, fs, fc, _ = fastnn_reciprocal(to_dev(m.desc1), to_dev(m.desc2), 8, 10)
+    fast, _ = gpu_pairs(fp, fs, fc)
+    assert set(map(tuple, fast.tolist())) <= set(map(tuple, p.tolist()))
