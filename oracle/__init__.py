@@ -51,16 +51,12 @@ _lib = None
 
 
 def build(force: bool = False) -> str:
-    """Compile ``oracle.c`` into ``liboracle.so`` next to it (gcc, OpenMP)."""
+    """Compile ``oracle.c`` into ``liboracle.so`` next to it (gcc -O2, OpenMP)."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        cmd = ["gcc", "-O2", "-march=native", "-fopenmp", "-fPIC", "-shared",
+        cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared",
                "-std=c11", "-Wall", "-o", _LIB, _SRC]
-        try:
-            subprocess.run(cmd, check=True, capture_output=True, text=True)
-        except subprocess.CalledProcessError:
-            # -march=native can fail under some emulators; retry portable.
-            cmd.remove("-march=native")
-            subprocess.run(cmd, check=True, capture_output=True, text=True)
+        # Portable x86-64 code: the built library travels to other hosts.
+        subprocess.run(cmd, check=True, capture_output=True, text=True)
     return _LIB
 
 
