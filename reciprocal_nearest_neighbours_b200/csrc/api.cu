@@ -14,6 +14,9 @@ namespace {
 constexpr size_t kAlign = 256;
 constexpr int kPadRows = 256;  // zero rows after each repacked database (one TMA box)
 constexpr int kMaxIter = 255;
+// Status block at the head of every workspace: [0] device status word,
+// [1] / [2] max |element| of the first / second int8 map.
+constexpr size_t kStatusBytes = 64 * sizeof(int);
 constexpr int64_t kMaxSeeds = (int64_t{1} << 24) - 1;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -144,10 +147,10 @@ int fastnn_nn(const void* q, int64_t nq, const void* db, int64_t ndb, int d, int
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   Carver c{static_cast<uint8_t*>(workspace)};
   NNLayout L = carve_nn(c, nq, ndb, dtype);
-  FASTNN_CUDA_TRY(cudaMemsetAsync(L.status, 0, sizeof(int), st));
+  FASTNN_CUDA_TRY(cudaMemsetAsync(L.status, 0, kStatusBytes, st));
   FASTNN_CUDA_TRY(cudaMemsetAsync(L.keys, 0, static_cast<size_t>(nq) * sizeof(uint64_t), st));
-  FASTNN_TRY(launch_repack(q, nq, d, dtype, L.qrep, 0, st));
-  FASTNN_TRY(launch_repack(db, ndb, d, dtype, L.dbrep, kPadRows, st));
+  FASTNN_TRY(launch_repack(q, nq, d, dtype, L.qrep, 0, L.status + 1, st));
+  FASTNN_TRY(launch_repack(db, ndb, d, dtype, L.dbrep, kPadRows, L.status + 2, st));
   NNArgs a{};
   a.q_rows = L.qrep;
   a.q_rows_per_pair = nq;
@@ -158,6 +161,9 @@ int fastnn_nn(const void* q, int64_t nq, const void* db, int64_t ndb, int d, int
   a.out_key = L.keys;
   a.batch = 1;
   a.status = L.status;
+  a.d = d;
+  a.q_absmax = L.status + 1;
+  a.db_absmax = L.status + 2;
   FASTNN_TRY(launch_nn_tc(a, dtype, ndb + kPadRows, st));
   return launch_decode(L.keys, nq, dtype, out_idx, out_score, st);
 }
@@ -187,7 +193,7 @@ int fastnn_reciprocal(const void* desc1, int H1, int W1, const void* desc2, int 
   Carver c{static_cast<uint8_t*>(workspace)};
   RecLayout L = carve_rec(c, N1, N2, dtype, batch, S);
 
-  FASTNN_CUDA_TRY(cudaMemsetAsync(L.status, 0, sizeof(int), st));
+  FASTNN_CUDA_TRY(cudaMemsetAsync(L.status, 0, kStatusBytes, st));
   FASTNN_CUDA_TRY(cudaMemsetAsync(L.fwd, 0, static_cast<size_t>(batch) * S * 8, st));
   FASTNN_CUDA_TRY(cudaMemsetAsync(L.bwd, 0, static_cast<size_t>(batch) * S * 8, st));
   FASTNN_CUDA_TRY(cudaMemsetAsync(L.claim, 0xFF, static_cast<size_t>(batch) * N1 * 4, st));
@@ -195,8 +201,8 @@ int fastnn_reciprocal(const void* desc1, int H1, int W1, const void* desc2, int 
   if (out_iters) FASTNN_CUDA_TRY(cudaMemsetAsync(out_iters, 0, static_cast<size_t>(batch) * 4, st));
   if (out_frontier)
     FASTNN_CUDA_TRY(cudaMemsetAsync(out_frontier, 0, static_cast<size_t>(batch) * max_iter * 4, st));
-  FASTNN_TRY(launch_repack(desc1, batch * N1, d, dtype, L.d1rep, kPadRows, st));
-  FASTNN_TRY(launch_repack(desc2, batch * N2, d, dtype, L.d2rep, kPadRows, st));
+  FASTNN_TRY(launch_repack(desc1, batch * N1, d, dtype, L.d1rep, kPadRows, L.status + 1, st));
+  FASTNN_TRY(launch_repack(desc2, batch * N2, d, dtype, L.d2rep, kPadRows, L.status + 2, st));
   FASTNN_TRY(launch_seed(L.F[0], S, L.claim, N1, L.cnt[0], H1, W1, subsample,
                          static_cast<int>(S), batch, st));
 
@@ -213,6 +219,9 @@ int fastnn_reciprocal(const void* desc1, int H1, int W1, const void* desc2, int 
     fwd.out_key = L.fwd;
     fwd.batch = batch;
     fwd.status = L.status;
+    fwd.d = d;
+    fwd.q_absmax = L.status + 1;
+    fwd.db_absmax = L.status + 2;
     FASTNN_TRY(launch_nn_tc(fwd, dtype, batch * N2 + kPadRows, st));
 
     NNArgs bwd{};
@@ -226,6 +235,9 @@ int fastnn_reciprocal(const void* desc1, int H1, int W1, const void* desc2, int 
     bwd.out_key = L.bwd;
     bwd.batch = batch;
     bwd.status = L.status;
+    bwd.d = d;
+    bwd.q_absmax = L.status + 2;
+    bwd.db_absmax = L.status + 1;
     FASTNN_TRY(launch_nn_tc(bwd, dtype, batch * N1 + kPadRows, st));
 
     CompactArgs ca{};
@@ -265,11 +277,11 @@ int fastnn_mutual_dense(const void* desc1, int64_t n1, const void* desc2, int64_
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   Carver c{static_cast<uint8_t*>(workspace)};
   MutLayout L = carve_mut(c, n1, n2, dtype);
-  FASTNN_CUDA_TRY(cudaMemsetAsync(L.status, 0, sizeof(int), st));
+  FASTNN_CUDA_TRY(cudaMemsetAsync(L.status, 0, kStatusBytes, st));
   FASTNN_CUDA_TRY(cudaMemsetAsync(L.k12, 0, static_cast<size_t>(n1) * 8, st));
   FASTNN_CUDA_TRY(cudaMemsetAsync(L.k21, 0, static_cast<size_t>(n2) * 8, st));
-  FASTNN_TRY(launch_repack(desc1, n1, d, dtype, L.d1rep, kPadRows, st));
-  FASTNN_TRY(launch_repack(desc2, n2, d, dtype, L.d2rep, kPadRows, st));
+  FASTNN_TRY(launch_repack(desc1, n1, d, dtype, L.d1rep, kPadRows, L.status + 1, st));
+  FASTNN_TRY(launch_repack(desc2, n2, d, dtype, L.d2rep, kPadRows, L.status + 2, st));
   NNArgs a{};
   a.q_rows = L.d1rep;
   a.q_rows_per_pair = n1;
@@ -280,6 +292,9 @@ int fastnn_mutual_dense(const void* desc1, int64_t n1, const void* desc2, int64_
   a.out_key = L.k12;
   a.batch = 1;
   a.status = L.status;
+  a.d = d;
+  a.q_absmax = L.status + 1;
+  a.db_absmax = L.status + 2;
   FASTNN_TRY(launch_nn_tc(a, dtype, n2 + kPadRows, st));
   NNArgs r{};
   r.q_rows = L.d2rep;
@@ -291,6 +306,9 @@ int fastnn_mutual_dense(const void* desc1, int64_t n1, const void* desc2, int64_
   r.out_key = L.k21;
   r.batch = 1;
   r.status = L.status;
+  r.d = d;
+  r.q_absmax = L.status + 2;
+  r.db_absmax = L.status + 1;
   FASTNN_TRY(launch_nn_tc(r, dtype, n1 + kPadRows, st));
   return launch_mutual(L.k12, L.k21, n1, n2, L.blocks, dtype, out_pairs, out_score, capacity,
                        out_count, st);

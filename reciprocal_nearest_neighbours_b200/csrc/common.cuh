@@ -67,6 +67,9 @@ struct NNArgs {
   uint64_t* out_key;       // [batch][q_cap], merged with atomicMax
   int batch;
   int* status;
+  int d;                   // descriptor length (<= 32)
+  const int* q_absmax;     // int8: max |element| of the query map (or nullptr)
+  const int* db_absmax;    // int8: max |element| of the database map (or nullptr)
 };
 
 __device__ __forceinline__ int64_t nn_count(const NNArgs& a, int b) {

@@ -15,13 +15,17 @@ namespace {
 // One thread per output row. Source rows of d elements (esize bytes each) are
 // copied into 32-element rows (32 B int8 / 64 B bf16) with zero padding, so
 // every row is 16-byte aligned for TMA and the MMA's K extent is exactly 32.
+// For int8 maps, `absmax` (if given) receives max |element| over the map
+// (atomicMax), which tells the nearest-neighbour kernel whether every score
+// fits in 16 bits.
 template <int ESIZE>
 __global__ void repack_kernel(const uint8_t* __restrict__ src, int64_t rows, int d,
-                              uint8_t* __restrict__ dst, int64_t pad_rows) {
+                              uint8_t* __restrict__ dst, int64_t pad_rows, int* absmax) {
   constexpr int RB = 32 * ESIZE;
   constexpr int NW = RB / 4;
   const int nbytes = d * ESIZE;
   const bool words = (nbytes % 4) == 0 && (reinterpret_cast<uintptr_t>(src) % 4) == 0;
+  int amax = 0;
   for (int64_t row = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
        row < rows + pad_rows; row += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     uint32_t w[NW];
@@ -40,9 +44,22 @@ __global__ void repack_kernel(const uint8_t* __restrict__ src, int64_t rows, int
           if (i < nbytes) w[i / 4] |= static_cast<uint32_t>(__ldg(s + i)) << (8 * (i % 4));
       }
     }
+    if (ESIZE == 1 && absmax) {
+#pragma unroll
+      for (int i = 0; i < NW; ++i) {
+        const uint32_t x = w[i];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) amax = max(amax, abs(static_cast<int>(static_cast<int8_t>(x >> (8 * k)))));
+      }
+    }
     uint4* o = reinterpret_cast<uint4*>(dst + row * RB);
 #pragma unroll
     for (int i = 0; i < RB / 16; ++i) o[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+  }
+  if (ESIZE == 1 && absmax) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if ((threadIdx.x & 31) == 0 && amax > 0) atomicMax(absmax, amax);
   }
 }
 
@@ -285,15 +302,16 @@ int grid_for(int64_t n, int threads, int max_blocks = 148 * 16) {
 }  // namespace
 
 int launch_repack(const void* src, int64_t rows, int d, int dtype, void* dst, int64_t pad_rows,
-                  cudaStream_t st) {
+                  int* absmax, cudaStream_t st) {
   const int64_t total = rows + pad_rows;
   if (total <= 0) return FASTNN_OK;
   if (dtype == FASTNN_I8)
     repack_kernel<1><<<grid_for(total, 256), 256, 0, st>>>(static_cast<const uint8_t*>(src), rows,
-                                                            d, static_cast<uint8_t*>(dst), pad_rows);
+                                                            d, static_cast<uint8_t*>(dst), pad_rows, absmax);
   else
     repack_kernel<2><<<grid_for(total, 256), 256, 0, st>>>(static_cast<const uint8_t*>(src), rows,
-                                                            d, static_cast<uint8_t*>(dst), pad_rows);
+                                                            d, static_cast<uint8_t*>(dst), pad_rows,
+                                                            nullptr);
   FASTNN_CUDA_TRY(cudaGetLastError());
   return FASTNN_OK;
 }

@@ -46,6 +46,7 @@ constexpr int kMmaWarp = 9;
 constexpr int kThreads = 320;
 constexpr int kMaxBatch = 1024;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
+constexpr int kStashBytes = kEpiWarps * 32 * 32;  // 32 B per epilogue thread
 
 // Barrier slots inside the barrier block.
 constexpr int kBarBFull = 0;
@@ -61,6 +62,7 @@ struct Ctl {
   uint64_t bars[kNumBars];
   uint32_t tmem_base;
   int abort_flag;
+  int pack16;
   int b0;
   int64_t m0, n0, u0, u1, nt;
   int mt[kMaxBatch];
@@ -72,7 +74,7 @@ __host__ __device__ constexpr size_t tile_bytes_b(int rb) { return static_cast<s
 
 size_t smem_bytes(int rb) {
   return 1024 /* alignment slack */ + 2 * tile_bytes_a(rb) + kStages * tile_bytes_b(rb) +
-         sizeof(Ctl);
+         ((sizeof(Ctl) + 15) & ~static_cast<size_t>(15)) + kStashBytes;
 }
 
 // Bounded wait on an mbarrier phase. Returns false (and raises the abort flag
@@ -196,6 +198,125 @@ __device__ __forceinline__ void fold32(const uint32_t (&r)[32], uint32_t col0, i
   }
 }
 
+// ---- fast epilogue for full 256-column tiles ------------------------------
+// Each thread owns one query row and 128 columns of the tile. The maximum of
+// those columns is formed with a reduction tree; only when it beats the
+// running best strictly (a new record for this row) is the first column
+// holding it searched for: the 16-column group (8 registers) holding it is
+// found from the tree's group maxima, staged to this thread's 32-byte slot in
+// shared memory, and scanned there, so the search needs no dynamic register
+// indexing. The lowest index among equal scores survives.
+
+__device__ __forceinline__ uint32_t vmax3_s16x2(uint32_t a, uint32_t b, uint32_t c) {
+  return ptx::vmax_s16x2(ptx::vmax_s16x2(a, b), c);
+}
+
+// Tree maximum of 8 packed registers starting at r[o].
+template <int N>
+__device__ __forceinline__ uint32_t tree8_s16x2(const uint32_t (&r)[N], int o) {
+  const uint32_t x = vmax3_s16x2(r[o], r[o + 1], r[o + 2]);
+  const uint32_t y = vmax3_s16x2(r[o + 3], r[o + 4], r[o + 5]);
+  const uint32_t z = ptx::vmax_s16x2(r[o + 6], r[o + 7]);
+  return vmax3_s16x2(x, y, z);
+}
+
+__device__ __forceinline__ int lo16(uint32_t x) { return static_cast<int>(static_cast<int16_t>(x & 0xFFFFu)); }
+__device__ __forceinline__ int hi16(uint32_t x) { return static_cast<int>(x) >> 16; }
+
+__device__ __forceinline__ void stash8(uint4* slot, const uint32_t* r) {
+  slot[0] = make_uint4(r[0], r[1], r[2], r[3]);
+  slot[1] = make_uint4(r[4], r[5], r[6], r[7]);
+}
+
+// int8 scores that fit in 16 bits: r[c][i] holds columns 32c + 2i (low half)
+// and 32c + 2i + 1 (high half) of this thread's 128-column block.
+__device__ __forceinline__ void fold128_pack16(const uint32_t (&r0)[16], const uint32_t (&r1)[16],
+                                               const uint32_t (&r2)[16], const uint32_t (&r3)[16],
+                                               uint32_t colbase, int& best, uint32_t& bidx,
+                                               uint4* slot) {
+  uint32_t g[8];
+  g[0] = tree8_s16x2(r0, 0);
+  g[1] = tree8_s16x2(r0, 8);
+  g[2] = tree8_s16x2(r1, 0);
+  g[3] = tree8_s16x2(r1, 8);
+  g[4] = tree8_s16x2(r2, 0);
+  g[5] = tree8_s16x2(r2, 8);
+  g[6] = tree8_s16x2(r3, 0);
+  g[7] = tree8_s16x2(r3, 8);
+  const uint32_t u = tree8_s16x2(g, 0);
+  const int m = max(lo16(u), hi16(u));
+  if (m > best) {
+    best = m;
+    int gi = 7;
+#pragma unroll
+    for (int i = 7; i >= 0; --i)
+      if (lo16(g[i]) == m || hi16(g[i]) == m) gi = i;
+    switch (gi) {
+      case 0: stash8(slot, r0); break;
+      case 1: stash8(slot, r0 + 8); break;
+      case 2: stash8(slot, r1); break;
+      case 3: stash8(slot, r1 + 8); break;
+      case 4: stash8(slot, r2); break;
+      case 5: stash8(slot, r2 + 8); break;
+      case 6: stash8(slot, r3); break;
+      default: stash8(slot, r3 + 8); break;
+    }
+    const uint4 a = slot[0], b = slot[1];
+    const uint32_t x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    int w = 15;
+#pragma unroll
+    for (int j = 7; j >= 0; --j) {
+      if (hi16(x[j]) == m) w = 2 * j + 1;
+      if (lo16(x[j]) == m) w = 2 * j;
+    }
+    bidx = colbase + 16 * gi + w;
+  }
+}
+
+// 32-bit scores (int32, or fp32 for bf16 descriptors): 64 columns in r.
+template <int DT>
+__device__ __forceinline__ void fold64_wide(const uint32_t (&r)[64], uint32_t colbase,
+                                            typename Epi<DT>::S& best, uint32_t& bidx,
+                                            uint4* slot) {
+  using E = Epi<DT>;
+  using S = typename E::S;
+  S g[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const S a0 = E::mx(E::as_score(r[8 * i]), E::as_score(r[8 * i + 1]));
+    const S a1 = E::mx(E::as_score(r[8 * i + 2]), E::as_score(r[8 * i + 3]));
+    const S a2 = E::mx(E::as_score(r[8 * i + 4]), E::as_score(r[8 * i + 5]));
+    const S a3 = E::mx(E::as_score(r[8 * i + 6]), E::as_score(r[8 * i + 7]));
+    g[i] = E::mx(E::mx(a0, a1), E::mx(a2, a3));
+  }
+  const S m = E::mx(E::mx(E::mx(g[0], g[1]), E::mx(g[2], g[3])),
+                    E::mx(E::mx(g[4], g[5]), E::mx(g[6], g[7])));
+  if (m > best) {
+    best = m;
+    int gi = 7;
+#pragma unroll
+    for (int i = 7; i >= 0; --i)
+      if (g[i] == m) gi = i;
+    switch (gi) {
+      case 0: stash8(slot, r); break;
+      case 1: stash8(slot, r + 8); break;
+      case 2: stash8(slot, r + 16); break;
+      case 3: stash8(slot, r + 24); break;
+      case 4: stash8(slot, r + 32); break;
+      case 5: stash8(slot, r + 40); break;
+      case 6: stash8(slot, r + 48); break;
+      default: stash8(slot, r + 56); break;
+    }
+    const uint4 a = slot[0], b = slot[1];
+    const uint32_t x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    int w = 7;
+#pragma unroll
+    for (int j = 7; j >= 0; --j)
+      if (E::as_score(x[j]) == m) w = j;
+    bidx = colbase + 8 * gi + w;
+  }
+}
+
 template <int DT>
 __global__ void __launch_bounds__(kThreads, 1)
     nn_tc_kernel(const __grid_constant__ CUtensorMap tmap_db, NNArgs a) {
@@ -207,6 +328,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* tileA = smem;                              // 2 x kBM x RB
   uint8_t* tileB = tileA + 2 * tile_bytes_a(RB);      // kStages x kBN x RB
   Ctl* ctl = reinterpret_cast<Ctl*>(tileB + kStages * tile_bytes_b(RB));
+  uint4* stash = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(ctl) +
+                                          ((sizeof(Ctl) + 15) & ~static_cast<size_t>(15)));
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -229,6 +352,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     ctl->u0 = u0;
     ctl->u1 = u1;
     ctl->abort_flag = 0;
+    // int8 scores fit in 16 bits when d * max|q| * max|db| < 2^15; the repack
+    // pass measured both maxima.
+    ctl->pack16 = (DT == FASTNN_I8 && a.q_absmax && a.db_absmax &&
+                   static_cast<int64_t>(*a.q_absmax) * (*a.db_absmax) * a.d <= 32767)
+                      ? 1
+                      : 0;
     int64_t acc = 0;
     int b = 0;
     while (b < batch && acc + static_cast<int64_t>(ctl->mt[b]) * nt <= u0) {
@@ -368,6 +497,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     typename E::S best = E::lowest();
     uint32_t bidx = 0xFFFFFFFFu;
     const int tail = static_cast<int>(a.ndb - (nt - 1) * kBN);  // valid columns, last tile
+    const bool pack16 = ctl->pack16 != 0;
+    uint4* slot = stash + 2 * threadIdx.x;
     for (int64_t u = u0; u < u1; ++u) {
       const int acc = static_cast<int>(it & 1);
       if (!warp_wait_bounded(bar(kBarAccFull + acc), static_cast<uint32_t>((it >> 1) & 1), ctl,
@@ -377,18 +508,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t taddr = tmem + (static_cast<uint32_t>(lg * 32) << 16) +
                              static_cast<uint32_t>(acc * kBN + h * (kBN / 2));
       const uint32_t colbase = static_cast<uint32_t>(p.n * kBN + h * (kBN / 2));
-      const int valid_tile = (p.n == nt - 1) ? tail - h * (kBN / 2) : kBN / 2;
-#pragma unroll
-      for (int c = 0; c < (kBN / 2) / 32; ++c) {
-        uint32_t r[32];
-        ptx::tmem_ld32(taddr + c * 32, r);
+      if (p.n == nt - 1 && tail < kBN) {
+        // Ragged last tile of the database: column-masked fold.
+        const int valid_tile = tail - h * (kBN / 2);
+#pragma unroll 1
+        for (int c = 0; c < (kBN / 2) / 32; ++c) {
+          uint32_t r[32];
+          ptx::tmem_ld32(taddr + c * 32, r);
+          ptx::tmem_ld_wait();
+          const int valid = min(32, max(0, valid_tile - c * 32));
+          fold32<DT>(r, colbase + c * 32, valid, best, bidx);
+        }
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(kBarAccEmpty + acc));
+      } else if (DT == FASTNN_I8 && pack16) {
+        uint32_t r0[16], r1[16], r2[16], r3[16];
+        ptx::tmem_ld16_pack(taddr, r0);
+        ptx::tmem_ld16_pack(taddr + 32, r1);
+        ptx::tmem_ld16_pack(taddr + 64, r2);
+        ptx::tmem_ld16_pack(taddr + 96, r3);
         ptx::tmem_ld_wait();
-        const int valid = min(32, max(0, valid_tile - c * 32));
-        fold32<DT>(r, colbase + c * 32, valid, best, bidx);
+        // The accumulator is free for the next MMA as soon as it is in registers.
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(kBarAccEmpty + acc));
+        if constexpr (DT == FASTNN_I8) fold128_pack16(r0, r1, r2, r3, colbase, best, bidx, slot);
+      } else {
+        uint32_t r0[64], r1[64];
+        ptx::tmem_ld64(taddr, r0);
+        ptx::tmem_ld64(taddr + 64, r1);
+        ptx::tmem_ld_wait();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(kBarAccEmpty + acc));
+        fold64_wide<DT>(r0, colbase, best, bidx, slot);
+        fold64_wide<DT>(r1, colbase + 64, best, bidx, slot);
       }
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(bar(kBarAccEmpty + acc));
       const bool seg_end = (u + 1 == u1) || (p.n == nt - 1);
       if (seg_end) {
         const int64_t k = p.m * kBM + lg * 32 + lane;

@@ -37,6 +37,9 @@ I8_CASES = [
     (200, 513, 24, -128, 127),  # extreme int8 values
     (4000, 2000, 1, -5, 5),    # d = 1: massive ties
     (333, 4099, 17, -16, 16),
+    (300, 1024, 32, -31, 31),   # 32 * 31 * 31 < 2^15: 16-bit packed epilogue, near its limit
+    (300, 1024, 32, -32, 31),   # 32 * 32 * 32 = 2^15: 32-bit epilogue
+    (256, 8192, 24, 0, 1),      # non-negative 0/1 values: long runs of equal maxima
 ]
 
 
