@@ -7,15 +7,15 @@
 // primitive of both the dense reciprocal set and the fast scheme).
 //
 // Design (one persistent CTA per SM, warp-specialised):
-//   warps 0..7  epilogue: tcgen05.ld the 128 x 256 score tile from TMEM and
+//   warps 0..15 epilogue: tcgen05.ld the 128 x 256 score tile from TMEM and
 //               fold it into a running (max score, lowest index) per query
-//               row; warpgroup 0 takes columns 0..127, warpgroup 1 128..255.
-//               The score matrix never leaves the SM.
-//   warp 8      producer: gathers the 128 query rows of a tile into shared
+//               row; warp w reads TMEM lanes 32 (w mod 4) .. +31 and columns
+//               64 (w div 4) .. +63. The score matrix never leaves the SM.
+//   warp 16     producer: gathers the 128 query rows of a tile into shared
 //               memory (swizzled, K-major) and streams 256-row database tiles
 //               with TMA (cp.async.bulk.tensor, no multicast) into a
 //               kStages-deep ring.
-//   warp 9      MMA issuer (one thread): tcgen05.mma kind::i8 (int8 -> int32,
+//   warp 17     MMA issuer (one thread): tcgen05.mma kind::i8 (int8 -> int32,
 //               K = 32) or kind::f16 (bf16 -> fp32, 2 x K = 16) into one of
 //               two 256-column TMEM accumulators, tcgen05.commit to free the
 //               database stage and to hand the accumulator to the epilogue.
@@ -40,10 +40,11 @@ constexpr int kBM = 128;
 constexpr int kBN = 256;
 constexpr int kStages = 6;
 constexpr int kAcc = 2;
-constexpr int kEpiWarps = 8;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kThreads = 320;
+constexpr int kEpiWarps = 16;
+constexpr int kProducerWarp = 16;
+constexpr int kMmaWarp = 17;
+constexpr int kThreads = 576;
+constexpr int kEpiCols = kBN / (kEpiWarps / 4);  // columns of a tile per epilogue thread
 constexpr int kMaxBatch = 1024;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr int kStashBytes = kEpiWarps * 32 * 32;  // 32 B per epilogue thread
@@ -159,6 +160,7 @@ struct Epi<FASTNN_I8> {
   static __device__ __forceinline__ S lowest() { return INT32_MIN; }
   static __device__ __forceinline__ S as_score(uint32_t r) { return static_cast<int32_t>(r); }
   static __device__ __forceinline__ S mx(S x, S y) { return max(x, y); }
+  static __device__ __forceinline__ S mx3(S x, S y, S z) { return max(max(x, y), z); }
   static __device__ __forceinline__ uint32_t ord(S s) { return ord_i32(s); }
 };
 
@@ -169,6 +171,11 @@ struct Epi<FASTNN_BF16> {
   static __device__ __forceinline__ S lowest() { return -INFINITY; }
   static __device__ __forceinline__ S as_score(uint32_t r) { return __uint_as_float(r); }
   static __device__ __forceinline__ S mx(S x, S y) { return fmaxf(x, y); }
+  static __device__ __forceinline__ S mx3(S x, S y, S z) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(x), "f"(y), "f"(z));
+    return r;
+  }
   static __device__ __forceinline__ uint32_t ord(S s) { return ord_f32(s); }
 };
 
@@ -229,37 +236,28 @@ __device__ __forceinline__ void stash8(uint4* slot, const uint32_t* r) {
 }
 
 // int8 scores that fit in 16 bits: r[c][i] holds columns 32c + 2i (low half)
-// and 32c + 2i + 1 (high half) of this thread's 128-column block.
-__device__ __forceinline__ void fold128_pack16(const uint32_t (&r0)[16], const uint32_t (&r1)[16],
-                                               const uint32_t (&r2)[16], const uint32_t (&r3)[16],
-                                               uint32_t colbase, int& best, uint32_t& bidx,
-                                               uint4* slot) {
-  uint32_t g[8];
+// and 32c + 2i + 1 (high half) of this thread's 64-column block.
+__device__ __forceinline__ void fold64_pack16(const uint32_t (&r0)[16], const uint32_t (&r1)[16],
+                                              uint32_t colbase, int& best, uint32_t& bidx,
+                                              uint4* slot) {
+  uint32_t g[4];
   g[0] = tree8_s16x2(r0, 0);
   g[1] = tree8_s16x2(r0, 8);
   g[2] = tree8_s16x2(r1, 0);
   g[3] = tree8_s16x2(r1, 8);
-  g[4] = tree8_s16x2(r2, 0);
-  g[5] = tree8_s16x2(r2, 8);
-  g[6] = tree8_s16x2(r3, 0);
-  g[7] = tree8_s16x2(r3, 8);
-  const uint32_t u = tree8_s16x2(g, 0);
+  const uint32_t u = ptx::vmax_s16x2(ptx::vmax_s16x2(g[0], g[1]), ptx::vmax_s16x2(g[2], g[3]));
   const int m = max(lo16(u), hi16(u));
   if (m > best) {
     best = m;
-    int gi = 7;
+    int gi = 3;
 #pragma unroll
-    for (int i = 7; i >= 0; --i)
+    for (int i = 3; i >= 0; --i)
       if (lo16(g[i]) == m || hi16(g[i]) == m) gi = i;
     switch (gi) {
       case 0: stash8(slot, r0); break;
       case 1: stash8(slot, r0 + 8); break;
       case 2: stash8(slot, r1); break;
-      case 3: stash8(slot, r1 + 8); break;
-      case 4: stash8(slot, r2); break;
-      case 5: stash8(slot, r2 + 8); break;
-      case 6: stash8(slot, r3); break;
-      default: stash8(slot, r3 + 8); break;
+      default: stash8(slot, r1 + 8); break;
     }
     const uint4 a = slot[0], b = slot[1];
     const uint32_t x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
@@ -283,14 +281,11 @@ __device__ __forceinline__ void fold64_wide(const uint32_t (&r)[64], uint32_t co
   S g[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const S a0 = E::mx(E::as_score(r[8 * i]), E::as_score(r[8 * i + 1]));
-    const S a1 = E::mx(E::as_score(r[8 * i + 2]), E::as_score(r[8 * i + 3]));
-    const S a2 = E::mx(E::as_score(r[8 * i + 4]), E::as_score(r[8 * i + 5]));
-    const S a3 = E::mx(E::as_score(r[8 * i + 6]), E::as_score(r[8 * i + 7]));
-    g[i] = E::mx(E::mx(a0, a1), E::mx(a2, a3));
+    const S a0 = E::mx3(E::as_score(r[8 * i]), E::as_score(r[8 * i + 1]), E::as_score(r[8 * i + 2]));
+    const S a1 = E::mx3(E::as_score(r[8 * i + 3]), E::as_score(r[8 * i + 4]), E::as_score(r[8 * i + 5]));
+    g[i] = E::mx3(a0, a1, E::mx(E::as_score(r[8 * i + 6]), E::as_score(r[8 * i + 7])));
   }
-  const S m = E::mx(E::mx(E::mx(g[0], g[1]), E::mx(g[2], g[3])),
-                    E::mx(E::mx(g[4], g[5]), E::mx(g[6], g[7])));
+  const S m = E::mx3(E::mx3(g[0], g[1], g[2]), E::mx3(g[3], g[4], g[5]), E::mx(g[6], g[7]));
   if (m > best) {
     best = m;
     int gi = 7;
@@ -491,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ---------------------------------------------------------------- epilogue
     const int lg = warp & 3;  // TMEM lane quarter this warp may access
-    const int h = warp >> 2;  // column half of the 256-wide tile
+    const int h = warp >> 2;  // column block (of kEpiCols) of the 256-wide tile
     Pos p = start;
     int64_t it = 0;
     typename E::S best = E::lowest();
@@ -506,44 +501,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       ptx::tc_fence_after();
       const uint32_t taddr = tmem + (static_cast<uint32_t>(lg * 32) << 16) +
-                             static_cast<uint32_t>(acc * kBN + h * (kBN / 2));
-      const uint32_t colbase = static_cast<uint32_t>(p.n * kBN + h * (kBN / 2));
+                             static_cast<uint32_t>(acc * kBN + h * kEpiCols);
+      const uint32_t colbase = static_cast<uint32_t>(p.n * kBN + h * kEpiCols);
       if (p.n == nt - 1 && tail < kBN) {
         // Ragged last tile of the database: column-masked fold.
-        const int valid_tile = tail - h * (kBN / 2);
+        const int valid_blk = tail - h * kEpiCols;
 #pragma unroll 1
-        for (int c = 0; c < (kBN / 2) / 32; ++c) {
+        for (int c = 0; c < kEpiCols / 32; ++c) {
           uint32_t r[32];
           ptx::tmem_ld32(taddr + c * 32, r);
           ptx::tmem_ld_wait();
-          const int valid = min(32, max(0, valid_tile - c * 32));
+          const int valid = min(32, max(0, valid_blk - c * 32));
           fold32<DT>(r, colbase + c * 32, valid, best, bidx);
         }
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(bar(kBarAccEmpty + acc));
       } else if (DT == FASTNN_I8 && pack16) {
-        uint32_t r0[16], r1[16], r2[16], r3[16];
+        uint32_t r0[16], r1[16];
         ptx::tmem_ld16_pack(taddr, r0);
         ptx::tmem_ld16_pack(taddr + 32, r1);
-        ptx::tmem_ld16_pack(taddr + 64, r2);
-        ptx::tmem_ld16_pack(taddr + 96, r3);
         ptx::tmem_ld_wait();
         // The accumulator is free for the next MMA as soon as it is in registers.
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(bar(kBarAccEmpty + acc));
-        if constexpr (DT == FASTNN_I8) fold128_pack16(r0, r1, r2, r3, colbase, best, bidx, slot);
+        if constexpr (DT == FASTNN_I8) fold64_pack16(r0, r1, colbase, best, bidx, slot);
       } else {
-        uint32_t r0[64], r1[64];
+        uint32_t r0[64];
         ptx::tmem_ld64(taddr, r0);
-        ptx::tmem_ld64(taddr + 64, r1);
         ptx::tmem_ld_wait();
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(bar(kBarAccEmpty + acc));
         fold64_wide<DT>(r0, colbase, best, bidx, slot);
-        fold64_wide<DT>(r1, colbase + 64, best, bidx, slot);
       }
       const bool seg_end = (u + 1 == u1) || (p.n == nt - 1);
       if (seg_end) {
