@@ -7,23 +7,23 @@
 // primitive of both the dense reciprocal set and the fast scheme).
 //
 // Design (one persistent CTA per SM, warp-specialised):
-//   warps 0..15 epilogue: tcgen05.ld the 128 x 256 score tile from TMEM and
-//               fold it into a running (max score, lowest index) per query
-//               row; warp w reads TMEM lanes 32 (w mod 4) .. +31 and columns
-//               64 (w div 4) .. +63. The score matrix never leaves the SM.
-//   warp 16     producer: gathers the 128 query rows of a tile into shared
-//               memory (swizzled, K-major) and streams 256-row database tiles
-//               with TMA (cp.async.bulk.tensor, no multicast) into a
-//               kStages-deep ring.
-//   warp 17     MMA issuer (one thread): tcgen05.mma kind::i8 (int8 -> int32,
-//               K = 32) or kind::f16 (bf16 -> fp32, 2 x K = 16) into one of
-//               two 256-column TMEM accumulators, tcgen05.commit to free the
-//               database stage and to hand the accumulator to the epilogue.
-// Work: units (pair, 128-query tile, 256-row database tile) in row-major
-// order, split into contiguous ranges over the CTAs; a CTA merges each
-// query tile's partial result with one 64-bit atomicMax per row, which is
-// order independent. Descriptors are zero-padded to 32 elements (32 B int8
-// rows, 64 B bf16 rows) by the repack kernel, so the padding adds nothing.
+//   epilogue warps (kEpiWarps): tcgen05.ld score tiles from TMEM and fold
+//       them into a running (max score, lowest index) per query row; warp w
+//       reads TMEM lanes 32 (w mod 4) .. +31 and a block of kEpiCols columns.
+//       The score matrix never leaves the SM.
+//   producer warp: gathers the 128 query rows of a tile into shared memory
+//       (swizzled, K-major) and streams kBN-row database tiles with TMA
+//       (cp.async.bulk.tensor, no multicast) into a kStages-deep ring.
+//   MMA warp (one thread): tcgen05.mma kind::i8 (int8 -> int32, K = 32) or
+//       kind::f16 (bf16 -> fp32, 2 x K = 16) into a ring of kAcc TMEM
+//       accumulators of kBN columns; tcgen05.commit frees the database stage
+//       and hands the accumulator to the epilogue.
+// Work: units (pair, 128-query tile, kBN-row database tile) in row-major
+// order, split into contiguous ranges over the CTAs. A run of units that
+// share a query tile is a segment; at its end the CTA merges each row's
+// partial result with one 64-bit atomicMax, which is order independent.
+// Descriptors are zero-padded to 32 elements (32 B int8 rows, 64 B bf16 rows)
+// by the repack kernel, so the padding adds nothing to any score.
 // Every mbarrier wait is bounded; on expiry the kernel records
 // FASTNN_ERR_TIMEOUT in the status word, drains what it issued and exits.
 #include <cuda.h>
@@ -32,22 +32,34 @@
 #include "nn_tc.cuh"
 #include "ptx.cuh"
 
+#ifndef FASTNN_BN
+#define FASTNN_BN 128
+#endif
+#ifndef FASTNN_EPI_WARPS
+#define FASTNN_EPI_WARPS 16
+#endif
+
 namespace fastnn {
 
 namespace {
 
 constexpr int kBM = 128;
-constexpr int kBN = 256;
-constexpr int kStages = 6;
-constexpr int kAcc = 2;
-constexpr int kEpiWarps = 16;
-constexpr int kProducerWarp = 16;
-constexpr int kMmaWarp = 17;
-constexpr int kThreads = 576;
+constexpr int kBN = FASTNN_BN;                  // database rows per unit = accumulator columns
+constexpr int kAcc = 512 / kBN;                 // TMEM accumulator ring (512 columns)
+constexpr int kStages = 49152 / (kBN * 32);     // database ring: 48 KB (int8) / 96 KB (bf16)
+constexpr int kEpiWarps = FASTNN_EPI_WARPS;
+constexpr int kProducerWarp = kEpiWarps;
+constexpr int kMmaWarp = kEpiWarps + 1;
+constexpr int kThreads = 32 * (kEpiWarps + 2);
 constexpr int kEpiCols = kBN / (kEpiWarps / 4);  // columns of a tile per epilogue thread
+constexpr int kChunks = kEpiCols / 32;           // 32-column TMEM loads per unit and thread
 constexpr int kMaxBatch = 1024;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr int kStashBytes = kEpiWarps * 32 * 32;  // 32 B per epilogue thread
+
+static_assert(kBN == 128 || kBN == 256, "tile width");
+static_assert(kEpiWarps == 8 || kEpiWarps == 16, "epilogue warps");
+static_assert(kChunks >= 1 && kChunks <= 4, "columns per epilogue thread");
 
 // Barrier slots inside the barrier block.
 constexpr int kBarBFull = 0;
@@ -72,10 +84,11 @@ struct Ctl {
 
 __host__ __device__ constexpr size_t tile_bytes_a(int rb) { return static_cast<size_t>(kBM) * rb; }
 __host__ __device__ constexpr size_t tile_bytes_b(int rb) { return static_cast<size_t>(kBN) * rb; }
+__host__ __device__ constexpr size_t ctl_bytes() { return (sizeof(Ctl) + 15) & ~static_cast<size_t>(15); }
 
 size_t smem_bytes(int rb) {
   return 1024 /* alignment slack */ + 2 * tile_bytes_a(rb) + kStages * tile_bytes_b(rb) +
-         ((sizeof(Ctl) + 15) & ~static_cast<size_t>(15)) + kStashBytes;
+         ctl_bytes() + kStashBytes;
 }
 
 // Bounded wait on an mbarrier phase. Returns false (and raises the abort flag
@@ -102,20 +115,25 @@ __device__ bool warp_wait_bounded(uint32_t bar, uint32_t parity, Ctl* ctl, int* 
   return __all_sync(0xffffffffu, ok);
 }
 
+// Position of the next unit: pair b, query tile m, database tile n.
 struct Pos {
   int b;
   int64_t m, n;
 };
 
-__device__ __forceinline__ void advance(Pos& p, const Ctl* ctl, int batch) {
-  if (++p.n == ctl->nt) {
-    p.n = 0;
-    if (++p.m == ctl->mt[p.b]) {
-      p.m = 0;
-      do {
-        ++p.b;
-      } while (p.b < batch && ctl->mt[p.b] == 0);
-    }
+// Units left in the current segment (same pair and query tile).
+__device__ __forceinline__ int64_t seg_len(const Pos& p, int64_t u, int64_t u1, int64_t nt) {
+  return min(u1 - u, nt - p.n);
+}
+
+// Move to the first unit of the next segment.
+__device__ __forceinline__ void next_segment(Pos& p, const Ctl* ctl, int batch) {
+  p.n = 0;
+  if (++p.m == ctl->mt[p.b]) {
+    p.m = 0;
+    do {
+      ++p.b;
+    } while (p.b < batch && ctl->mt[p.b] == 0);
   }
 }
 
@@ -125,12 +143,12 @@ __device__ __forceinline__ void advance(Pos& p, const Ctl* ctl, int batch) {
 template <int RB>
 __device__ __forceinline__ void gather_a(uint8_t* tile, const NNArgs& a, int b, int64_t m,
                                          int cnt, int lane) {
-  constexpr int kChunks = RB / 16;
+  constexpr int kC = RB / 16;
 #pragma unroll
   for (int i = 0; i < kBM / 32; ++i) {
     const int r = lane + 32 * i;
     const int64_t k = m * kBM + r;
-    uint4 v[kChunks];
+    uint4 v[kC];
     const int64_t row = k < cnt ? nn_query_row(a, b, k) : -1;
     // Rows outside the query source (never produced by a healthy pipeline)
     // read as zeros instead of faulting.
@@ -138,14 +156,14 @@ __device__ __forceinline__ void gather_a(uint8_t* tile, const NNArgs& a, int b, 
       const uint4* src = reinterpret_cast<const uint4*>(
           a.q_rows + (static_cast<int64_t>(b) * a.q_rows_per_pair + row) * RB);
 #pragma unroll
-      for (int c = 0; c < kChunks; ++c) v[c] = __ldg(src + c);
+      for (int c = 0; c < kC; ++c) v[c] = __ldg(src + c);
     } else {
 #pragma unroll
-      for (int c = 0; c < kChunks; ++c) v[c] = make_uint4(0, 0, 0, 0);
+      for (int c = 0; c < kC; ++c) v[c] = make_uint4(0, 0, 0, 0);
     }
     const int swz = RB == 32 ? ((r >> 2) & 1) : ((r >> 1) & 3);
 #pragma unroll
-    for (int c = 0; c < kChunks; ++c)
+    for (int c = 0; c < kC; ++c)
       *reinterpret_cast<uint4*>(tile + r * RB + 16 * (c ^ swz)) = v[c];
   }
 }
@@ -180,13 +198,10 @@ struct Epi<FASTNN_BF16> {
 };
 
 // Fold 32 consecutive columns (global index col0 + j) into (best, bidx).
-// The chunk maximum is taken first; only when it beats the running best
-// strictly is the chunk rescanned for the first column holding it, so the
-// lowest index among equal scores survives. `valid` < 32 masks a ragged
-// database tail.
+// Used for the ragged last database tile: `valid` < 32 masks the tail.
 template <int DT>
-__device__ __forceinline__ void fold32(const uint32_t (&r)[32], uint32_t col0, int valid,
-                                       typename Epi<DT>::S& best, uint32_t& bidx) {
+__device__ __forceinline__ void fold32_masked(const uint32_t (&r)[32], uint32_t col0, int valid,
+                                              typename Epi<DT>::S& best, uint32_t& bidx) {
   using E = Epi<DT>;
   using S = typename E::S;
   S v[32];
@@ -205,25 +220,23 @@ __device__ __forceinline__ void fold32(const uint32_t (&r)[32], uint32_t col0, i
   }
 }
 
-// ---- fast epilogue for full 256-column tiles ------------------------------
-// Each thread owns one query row and 128 columns of the tile. The maximum of
-// those columns is formed with a reduction tree; only when it beats the
-// running best strictly (a new record for this row) is the first column
-// holding it searched for: the 16-column group (8 registers) holding it is
-// found from the tree's group maxima, staged to this thread's 32-byte slot in
-// shared memory, and scanned there, so the search needs no dynamic register
-// indexing. The lowest index among equal scores survives.
+// ---- fast epilogue for full tiles ------------------------------------------
+// Each thread owns one query row and kEpiCols columns of the tile. Their
+// maximum is formed with a reduction tree; only when it beats the running best
+// strictly (a new record for this row) is the first column holding it
+// searched for: the 8-register group holding it is found from the tree's
+// group maxima, staged to this thread's 32-byte slot in shared memory, and
+// scanned there, so the search needs no dynamic register indexing. The lowest
+// index among equal scores survives.
 
 __device__ __forceinline__ uint32_t vmax3_s16x2(uint32_t a, uint32_t b, uint32_t c) {
   return ptx::vmax_s16x2(ptx::vmax_s16x2(a, b), c);
 }
 
-// Tree maximum of 8 packed registers starting at r[o].
-template <int N>
-__device__ __forceinline__ uint32_t tree8_s16x2(const uint32_t (&r)[N], int o) {
-  const uint32_t x = vmax3_s16x2(r[o], r[o + 1], r[o + 2]);
-  const uint32_t y = vmax3_s16x2(r[o + 3], r[o + 4], r[o + 5]);
-  const uint32_t z = ptx::vmax_s16x2(r[o + 6], r[o + 7]);
+__device__ __forceinline__ uint32_t tree8_s16x2(const uint32_t* r) {
+  const uint32_t x = vmax3_s16x2(r[0], r[1], r[2]);
+  const uint32_t y = vmax3_s16x2(r[3], r[4], r[5]);
+  const uint32_t z = ptx::vmax_s16x2(r[6], r[7]);
   return vmax3_s16x2(x, y, z);
 }
 
@@ -236,29 +249,33 @@ __device__ __forceinline__ void stash8(uint4* slot, const uint32_t* r) {
 }
 
 // int8 scores that fit in 16 bits: r[c][i] holds columns 32c + 2i (low half)
-// and 32c + 2i + 1 (high half) of this thread's 64-column block.
-__device__ __forceinline__ void fold64_pack16(const uint32_t (&r0)[16], const uint32_t (&r1)[16],
-                                              uint32_t colbase, int& best, uint32_t& bidx,
-                                              uint4* slot) {
-  uint32_t g[4];
-  g[0] = tree8_s16x2(r0, 0);
-  g[1] = tree8_s16x2(r0, 8);
-  g[2] = tree8_s16x2(r1, 0);
-  g[3] = tree8_s16x2(r1, 8);
-  const uint32_t u = ptx::vmax_s16x2(ptx::vmax_s16x2(g[0], g[1]), ptx::vmax_s16x2(g[2], g[3]));
+// and 32c + 2i + 1 (high half) of this thread's block.
+template <int NC>
+__device__ __forceinline__ void fold_pack16(const uint32_t (&r)[NC][16], uint32_t colbase,
+                                            int& best, uint32_t& bidx, uint4* slot) {
+  constexpr int G = 2 * NC;  // groups of 8 registers = 16 columns
+  uint32_t g[G];
+#pragma unroll
+  for (int i = 0; i < G; ++i) g[i] = tree8_s16x2(&r[i / 2][(i % 2) * 8]);
+  uint32_t u;
+  if constexpr (G == 2) {
+    u = ptx::vmax_s16x2(g[0], g[1]);
+  } else if constexpr (G == 4) {
+    u = ptx::vmax_s16x2(ptx::vmax_s16x2(g[0], g[1]), ptx::vmax_s16x2(g[2], g[3]));
+  } else {
+    u = vmax3_s16x2(vmax3_s16x2(g[0], g[1], g[2]), vmax3_s16x2(g[3], g[4], g[5]),
+                    ptx::vmax_s16x2(g[6], g[7]));
+  }
   const int m = max(lo16(u), hi16(u));
   if (m > best) {
     best = m;
-    int gi = 3;
+    int gi = G - 1;
 #pragma unroll
-    for (int i = 3; i >= 0; --i)
+    for (int i = G - 1; i >= 0; --i)
       if (lo16(g[i]) == m || hi16(g[i]) == m) gi = i;
-    switch (gi) {
-      case 0: stash8(slot, r0); break;
-      case 1: stash8(slot, r0 + 8); break;
-      case 2: stash8(slot, r1); break;
-      default: stash8(slot, r1 + 8); break;
-    }
+#pragma unroll
+    for (int i = 0; i < G; ++i)
+      if (i == gi) stash8(slot, &r[i / 2][(i % 2) * 8]);
     const uint4 a = slot[0], b = slot[1];
     const uint32_t x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
     int w = 15;
@@ -271,37 +288,34 @@ __device__ __forceinline__ void fold64_pack16(const uint32_t (&r0)[16], const ui
   }
 }
 
-// 32-bit scores (int32, or fp32 for bf16 descriptors): 64 columns in r.
-template <int DT>
-__device__ __forceinline__ void fold64_wide(const uint32_t (&r)[64], uint32_t colbase,
-                                            typename Epi<DT>::S& best, uint32_t& bidx,
-                                            uint4* slot) {
+// 32-bit scores (int32, or fp32 for bf16 descriptors): r[c][i] = column 32c + i.
+template <int DT, int NC>
+__device__ __forceinline__ void fold_wide(const uint32_t (&r)[NC][32], uint32_t colbase,
+                                          typename Epi<DT>::S& best, uint32_t& bidx,
+                                          uint4* slot) {
   using E = Epi<DT>;
   using S = typename E::S;
-  S g[8];
+  constexpr int G = 4 * NC;  // groups of 8 registers = 8 columns
+  S g[G];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const S a0 = E::mx3(E::as_score(r[8 * i]), E::as_score(r[8 * i + 1]), E::as_score(r[8 * i + 2]));
-    const S a1 = E::mx3(E::as_score(r[8 * i + 3]), E::as_score(r[8 * i + 4]), E::as_score(r[8 * i + 5]));
-    g[i] = E::mx3(a0, a1, E::mx(E::as_score(r[8 * i + 6]), E::as_score(r[8 * i + 7])));
+  for (int i = 0; i < G; ++i) {
+    const uint32_t* q = &r[i / 4][(i % 4) * 8];
+    const S a0 = E::mx3(E::as_score(q[0]), E::as_score(q[1]), E::as_score(q[2]));
+    const S a1 = E::mx3(E::as_score(q[3]), E::as_score(q[4]), E::as_score(q[5]));
+    g[i] = E::mx3(a0, a1, E::mx(E::as_score(q[6]), E::as_score(q[7])));
   }
-  const S m = E::mx3(E::mx3(g[0], g[1], g[2]), E::mx3(g[3], g[4], g[5]), E::mx(g[6], g[7]));
+  S m = g[0];
+#pragma unroll
+  for (int i = 1; i < G; ++i) m = E::mx(m, g[i]);
   if (m > best) {
     best = m;
-    int gi = 7;
+    int gi = G - 1;
 #pragma unroll
-    for (int i = 7; i >= 0; --i)
+    for (int i = G - 1; i >= 0; --i)
       if (g[i] == m) gi = i;
-    switch (gi) {
-      case 0: stash8(slot, r); break;
-      case 1: stash8(slot, r + 8); break;
-      case 2: stash8(slot, r + 16); break;
-      case 3: stash8(slot, r + 24); break;
-      case 4: stash8(slot, r + 32); break;
-      case 5: stash8(slot, r + 40); break;
-      case 6: stash8(slot, r + 48); break;
-      default: stash8(slot, r + 56); break;
-    }
+#pragma unroll
+    for (int i = 0; i < G; ++i)
+      if (i == gi) stash8(slot, &r[i / 4][(i % 4) * 8]);
     const uint4 a = slot[0], b = slot[1];
     const uint32_t x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
     int w = 7;
@@ -320,11 +334,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* tileA = smem;                              // 2 x kBM x RB
-  uint8_t* tileB = tileA + 2 * tile_bytes_a(RB);      // kStages x kBN x RB
+  uint8_t* tileA = smem;                          // 2 x kBM x RB
+  uint8_t* tileB = tileA + 2 * tile_bytes_a(RB);  // kStages x kBN x RB
   Ctl* ctl = reinterpret_cast<Ctl*>(tileB + kStages * tile_bytes_b(RB));
-  uint4* stash = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(ctl) +
-                                          ((sizeof(Ctl) + 15) & ~static_cast<size_t>(15)));
+  uint4* stash = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(ctl) + ctl_bytes());
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -365,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ctl->n0 = nt > 0 ? rem % nt : 0;
     for (int i = 0; i < kNumBars; ++i) {
       uint32_t count = 1;
-      if (i >= kBarAFull && i < kBarAFull + 2) count = 32;        // producer lanes
+      if (i >= kBarAFull && i < kBarAFull + 2) count = 32;  // producer lanes
       if (i >= kBarAccEmpty && i < kBarAccEmpty + kAcc) count = kEpiWarps;
       ptx::mbar_init(ptx::smem_u32(&ctl->bars[i]), count);
     }
@@ -396,33 +409,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     int64_t last_issue[kStages];
 #pragma unroll
     for (int s = 0; s < kStages; ++s) last_issue[s] = -1;
-    for (int64_t u = u0; u < u1; ++u) {
-      if (u == u0 || p.n == 0) {
-        const int as = static_cast<int>(seg & 1);
-        if (!warp_wait_bounded(bar(kBarAEmpty + as), static_cast<uint32_t>(((seg >> 1) & 1) ^ 1),
-                               ctl, a.status))
+    bool ok = true;
+    for (int64_t u = u0; ok && u < u1; ++seg) {
+      const int64_t len = seg_len(p, u, u1, nt);
+      const int as = static_cast<int>(seg & 1);
+      if (!warp_wait_bounded(bar(kBarAEmpty + as), static_cast<uint32_t>(((seg >> 1) & 1) ^ 1),
+                             ctl, a.status))
+        break;
+      gather_a<RB>(tileA + as * tile_bytes_a(RB), a, p.b, p.m, ctl->cnt[p.b], lane);
+      ptx::fence_proxy_async_smem();
+      ptx::mbar_arrive(bar(kBarAFull + as));
+      const int64_t row0 = static_cast<int64_t>(p.b) * a.ndb + p.n * kBN;
+      for (int64_t j = 0; j < len; ++j, ++it) {
+        const int s = static_cast<int>(it % kStages);
+        const uint32_t ph = static_cast<uint32_t>((it / kStages) & 1);
+        bool lok = true;
+        if (lane == 0) {
+          lok = wait_bounded(bar(kBarBEmpty + s), ph ^ 1, ctl, a.status);
+          if (lok) {
+            ptx::mbar_arrive_expect_tx(bar(kBarBFull + s), static_cast<uint32_t>(tile_bytes_b(RB)));
+            ptx::tma_load_2d(ptx::smem_u32(tileB + s * tile_bytes_b(RB)), &tmap_db, 0,
+                             static_cast<int32_t>(row0 + j * kBN), bar(kBarBFull + s));
+            last_issue[s] = it;
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, lok ? 1 : 0, 0)) {
+          ok = false;
           break;
-        gather_a<RB>(tileA + as * tile_bytes_a(RB), a, p.b, p.m, ctl->cnt[p.b], lane);
-        ptx::fence_proxy_async_smem();
-        ptx::mbar_arrive(bar(kBarAFull + as));
-        ++seg;
-      }
-      const int s = static_cast<int>(it % kStages);
-      const uint32_t ph = static_cast<uint32_t>((it / kStages) & 1);
-      bool ok = true;
-      if (lane == 0) {
-        ok = wait_bounded(bar(kBarBEmpty + s), ph ^ 1, ctl, a.status);
-        if (ok) {
-          ptx::mbar_arrive_expect_tx(bar(kBarBFull + s), static_cast<uint32_t>(tile_bytes_b(RB)));
-          ptx::tma_load_2d(ptx::smem_u32(tileB + s * tile_bytes_b(RB)), &tmap_db, 0,
-                           static_cast<int32_t>(static_cast<int64_t>(p.b) * a.ndb + p.n * kBN),
-                           bar(kBarBFull + s));
-          last_issue[s] = it;
         }
       }
-      if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
-      ++it;
-      advance(p, ctl, batch);
+      u += len;
+      next_segment(p, ctl, batch);
     }
     // Drain: every TMA load this warp issued must land before smem is freed.
     if (lane == 0) {
@@ -440,44 +457,44 @@ __global__ void __launch_bounds__(kThreads, 1)
               : ((1u << 4) | (1u << 7) | (1u << 10) | ((kBN >> 3) << 17) | ((kBM >> 4) << 24));
       Pos p = start;
       int64_t it = 0, seg = 0;
-      int as = 0;
-      for (int64_t u = u0; u < u1; ++u) {
-        if (u == u0 || p.n == 0) {
-          as = static_cast<int>(seg & 1);
-          if (!wait_bounded(bar(kBarAFull + as), static_cast<uint32_t>((seg >> 1) & 1), ctl,
-                            a.status))
-            break;
-          ptx::tc_fence_after();
-          ++seg;
-        }
-        const int acc = static_cast<int>(it & 1);
-        if (!wait_bounded(bar(kBarAccEmpty + acc), static_cast<uint32_t>(((it >> 1) & 1) ^ 1), ctl,
+      bool ok = true;
+      for (int64_t u = u0; ok && u < u1; ++seg) {
+        const int64_t len = seg_len(p, u, u1, nt);
+        const int as = static_cast<int>(seg & 1);
+        if (!wait_bounded(bar(kBarAFull + as), static_cast<uint32_t>((seg >> 1) & 1), ctl,
                           a.status))
           break;
         ptx::tc_fence_after();
-        const int s = static_cast<int>(it % kStages);
-        if (!wait_bounded(bar(kBarBFull + s), static_cast<uint32_t>((it / kStages) & 1), ctl,
-                          a.status))
-          break;
-        ptx::tc_fence_after();
-        const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * kBN);
         const uint64_t adesc =
             ptx::smem_desc_kmajor(ptx::smem_u32(tileA + as * tile_bytes_a(RB)), RB);
-        const uint64_t bdesc =
-            ptx::smem_desc_kmajor(ptx::smem_u32(tileB + s * tile_bytes_b(RB)), RB);
-        if constexpr (DT == FASTNN_I8) {
-          ptx::mma_i8(d_tmem, adesc, bdesc, kIdesc, 0u);
-        } else {
-          // K = 32 bf16 = two K = 16 steps; the second starts 32 bytes in.
-          ptx::mma_bf16(d_tmem, adesc, bdesc, kIdesc, 0u);
-          ptx::mma_bf16(d_tmem, adesc + 2, bdesc + 2, kIdesc, 1u);
+        for (int64_t j = 0; j < len; ++j, ++it) {
+          const int acc = static_cast<int>(it % kAcc);
+          const int s = static_cast<int>(it % kStages);
+          if (!wait_bounded(bar(kBarAccEmpty + acc),
+                            static_cast<uint32_t>(((it / kAcc) & 1) ^ 1), ctl, a.status) ||
+              !wait_bounded(bar(kBarBFull + s), static_cast<uint32_t>((it / kStages) & 1), ctl,
+                            a.status)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * kBN);
+          const uint64_t bdesc =
+              ptx::smem_desc_kmajor(ptx::smem_u32(tileB + s * tile_bytes_b(RB)), RB);
+          if constexpr (DT == FASTNN_I8) {
+            ptx::mma_i8(d_tmem, adesc, bdesc, kIdesc, 0u);
+          } else {
+            // K = 32 bf16 = two K = 16 steps; the second starts 32 bytes in.
+            ptx::mma_bf16(d_tmem, adesc, bdesc, kIdesc, 0u);
+            ptx::mma_bf16(d_tmem, adesc + 2, bdesc + 2, kIdesc, 1u);
+          }
+          ptx::mma_commit(bar(kBarBEmpty + s));
+          ptx::mma_commit(bar(kBarAccFull + acc));
         }
-        ptx::mma_commit(bar(kBarBEmpty + s));
-        ptx::mma_commit(bar(kBarAccFull + acc));
-        const bool seg_end = (u + 1 == u1) || (p.n == nt - 1);
-        if (seg_end) ptx::mma_commit(bar(kBarAEmpty + as));
-        ++it;
-        advance(p, ctl, batch);
+        if (!ok) break;
+        ptx::mma_commit(bar(kBarAEmpty + as));
+        u += len;
+        next_segment(p, ctl, batch);
       }
       // Every MMA issued above completes before TMEM is released.
       ptx::mma_commit(bar(kBarDone));
@@ -486,67 +503,71 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ---------------------------------------------------------------- epilogue
     const int lg = warp & 3;  // TMEM lane quarter this warp may access
-    const int h = warp >> 2;  // column block (of kEpiCols) of the 256-wide tile
+    const int h = warp >> 2;  // column block (of kEpiCols) of the tile
+    const bool pack16 = ctl->pack16 != 0;
+    const int tail = static_cast<int>(a.ndb - (nt - 1) * kBN);  // valid columns, last tile
+    uint4* slot = stash + 2 * threadIdx.x;
     Pos p = start;
     int64_t it = 0;
-    typename E::S best = E::lowest();
-    uint32_t bidx = 0xFFFFFFFFu;
-    const int tail = static_cast<int>(a.ndb - (nt - 1) * kBN);  // valid columns, last tile
-    const bool pack16 = ctl->pack16 != 0;
-    uint4* slot = stash + 2 * threadIdx.x;
-    for (int64_t u = u0; u < u1; ++u) {
-      const int acc = static_cast<int>(it & 1);
-      if (!warp_wait_bounded(bar(kBarAccFull + acc), static_cast<uint32_t>((it >> 1) & 1), ctl,
-                             a.status))
-        break;
-      ptx::tc_fence_after();
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(lg * 32) << 16) +
-                             static_cast<uint32_t>(acc * kBN + h * kEpiCols);
-      const uint32_t colbase = static_cast<uint32_t>(p.n * kBN + h * kEpiCols);
-      if (p.n == nt - 1 && tail < kBN) {
-        // Ragged last tile of the database: column-masked fold.
-        const int valid_blk = tail - h * kEpiCols;
-#pragma unroll 1
-        for (int c = 0; c < kEpiCols / 32; ++c) {
-          uint32_t r[32];
-          ptx::tmem_ld32(taddr + c * 32, r);
-          ptx::tmem_ld_wait();
-          const int valid = min(32, max(0, valid_blk - c * 32));
-          fold32<DT>(r, colbase + c * 32, valid, best, bidx);
+    bool ok = true;
+    for (int64_t u = u0; ok && u < u1;) {
+      const int64_t len = seg_len(p, u, u1, nt);
+      typename E::S best = E::lowest();
+      uint32_t bidx = 0xFFFFFFFFu;
+      for (int64_t j = 0; j < len; ++j, ++it) {
+        const int acc = static_cast<int>(it % kAcc);
+        if (!warp_wait_bounded(bar(kBarAccFull + acc), static_cast<uint32_t>((it / kAcc) & 1),
+                               ctl, a.status)) {
+          ok = false;
+          break;
         }
-        ptx::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(bar(kBarAccEmpty + acc));
-      } else if (DT == FASTNN_I8 && pack16) {
-        uint32_t r0[16], r1[16];
-        ptx::tmem_ld16_pack(taddr, r0);
-        ptx::tmem_ld16_pack(taddr + 32, r1);
-        ptx::tmem_ld_wait();
-        // The accumulator is free for the next MMA as soon as it is in registers.
-        ptx::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(bar(kBarAccEmpty + acc));
-        if constexpr (DT == FASTNN_I8) fold64_pack16(r0, r1, colbase, best, bidx, slot);
-      } else {
-        uint32_t r0[64];
-        ptx::tmem_ld64(taddr, r0);
-        ptx::tmem_ld_wait();
-        ptx::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(bar(kBarAccEmpty + acc));
-        fold64_wide<DT>(r0, colbase, best, bidx, slot);
+        ptx::tc_fence_after();
+        const int64_t n = p.n + j;
+        const uint32_t taddr = tmem + (static_cast<uint32_t>(lg * 32) << 16) +
+                               static_cast<uint32_t>(acc * kBN + h * kEpiCols);
+        const uint32_t colbase = static_cast<uint32_t>(n * kBN + h * kEpiCols);
+        if (n == nt - 1 && tail < kBN) {
+          // Ragged last tile of the database: column-masked fold.
+          const int valid_blk = tail - h * kEpiCols;
+#pragma unroll 1
+          for (int c = 0; c < kChunks; ++c) {
+            uint32_t r[32];
+            ptx::tmem_ld32(taddr + c * 32, r);
+            ptx::tmem_ld_wait();
+            const int valid = min(32, max(0, valid_blk - c * 32));
+            fold32_masked<DT>(r, colbase + c * 32, valid, best, bidx);
+          }
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(bar(kBarAccEmpty + acc));
+        } else if (DT == FASTNN_I8 && pack16) {
+          uint32_t r[kChunks][16];
+#pragma unroll
+          for (int c = 0; c < kChunks; ++c) ptx::tmem_ld16_pack(taddr + c * 32, r[c]);
+          ptx::tmem_ld_wait();
+          // The accumulator is free for the next MMA once it is in registers.
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(bar(kBarAccEmpty + acc));
+          if constexpr (DT == FASTNN_I8) fold_pack16<kChunks>(r, colbase, best, bidx, slot);
+        } else {
+          uint32_t r[kChunks][32];
+#pragma unroll
+          for (int c = 0; c < kChunks; ++c) ptx::tmem_ld32(taddr + c * 32, r[c]);
+          ptx::tmem_ld_wait();
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(bar(kBarAccEmpty + acc));
+          fold_wide<DT, kChunks>(r, colbase, best, bidx, slot);
+        }
       }
-      const bool seg_end = (u + 1 == u1) || (p.n == nt - 1);
-      if (seg_end) {
-        const int64_t k = p.m * kBM + lg * 32 + lane;
-        if (k < ctl->cnt[p.b] && bidx != 0xFFFFFFFFu)
-          atomicMax(reinterpret_cast<unsigned long long*>(&a.out_key[p.b * a.q_cap + k]),
-                    static_cast<unsigned long long>(make_key(E::ord(best), bidx)));
-        best = E::lowest();
-        bidx = 0xFFFFFFFFu;
-      }
-      ++it;
-      advance(p, ctl, batch);
+      if (!ok) break;
+      const int64_t k = p.m * kBM + lg * 32 + lane;
+      if (k < ctl->cnt[p.b] && bidx != 0xFFFFFFFFu)
+        atomicMax(reinterpret_cast<unsigned long long*>(&a.out_key[p.b * a.q_cap + k]),
+                  static_cast<unsigned long long>(make_key(E::ord(best), bidx)));
+      u += len;
+      next_segment(p, ctl, batch);
     }
   }
 
