@@ -7,17 +7,18 @@
 // primitive of both the dense reciprocal set and the fast scheme).
 //
 // Design (one persistent CTA per SM, warp-specialised):
-//   epilogue warps (kEpiWarps): tcgen05.ld score tiles from TMEM and fold
-//       them into a running (max score, lowest index) per query row; warp w
-//       reads TMEM lanes 32 (w mod 4) .. +31 and a block of kEpiCols columns.
-//       The score matrix never leaves the SM.
+//   epilogue warps (two groups of 8): group g owns TMEM accumulator g, so
+//       one group loads a score tile while the other folds the previous one
+//       into a running (max score, lowest index) per query row. Warp w of a
+//       group reads TMEM lanes 32 (w mod 4) .. +31 and one half (128
+//       columns) of the tile. The score matrix never leaves the SM.
 //   producer warp: gathers the 128 query rows of a tile into shared memory
 //       (swizzled, K-major) and streams kBN-row database tiles with TMA
 //       (cp.async.bulk.tensor, no multicast) into a kStages-deep ring.
 //   MMA warp (one thread): tcgen05.mma kind::i8 (int8 -> int32, K = 32) or
-//       kind::f16 (bf16 -> fp32, 2 x K = 16) into a ring of kAcc TMEM
-//       accumulators of kBN columns; tcgen05.commit frees the database stage
-//       and hands the accumulator to the epilogue.
+//       kind::f16 (bf16 -> fp32, 2 x K = 16) into the two 256-column TMEM
+//       accumulators in turn; tcgen05.commit frees the database stage and
+//       hands the accumulator to its epilogue group.
 // Work: units (pair, 128-query tile, kBN-row database tile) in row-major
 // order, split into contiguous ranges over the CTAs. A run of units that
 // share a query tile is a segment; at its end the CTA merges each row's
@@ -32,34 +33,24 @@
 #include "nn_tc.cuh"
 #include "ptx.cuh"
 
-#ifndef FASTNN_BN
-#define FASTNN_BN 128
-#endif
-#ifndef FASTNN_EPI_WARPS
-#define FASTNN_EPI_WARPS 16
-#endif
-
 namespace fastnn {
 
 namespace {
 
 constexpr int kBM = 128;
-constexpr int kBN = FASTNN_BN;                  // database rows per unit = accumulator columns
-constexpr int kAcc = 512 / kBN;                 // TMEM accumulator ring (512 columns)
-constexpr int kStages = 49152 / (kBN * 32);     // database ring: 48 KB (int8) / 96 KB (bf16)
-constexpr int kEpiWarps = FASTNN_EPI_WARPS;
+constexpr int kBN = 256;                        // database rows per unit = accumulator columns
+constexpr int kAcc = 2;                         // TMEM accumulators (2 x 256 = 512 columns)
+constexpr int kStages = 6;                      // database ring: 48 KB (int8) / 96 KB (bf16)
+constexpr int kGroupWarps = 8;                  // epilogue warps per accumulator
+constexpr int kEpiWarps = kAcc * kGroupWarps;
 constexpr int kProducerWarp = kEpiWarps;
 constexpr int kMmaWarp = kEpiWarps + 1;
 constexpr int kThreads = 32 * (kEpiWarps + 2);
-constexpr int kEpiCols = kBN / (kEpiWarps / 4);  // columns of a tile per epilogue thread
-constexpr int kChunks = kEpiCols / 32;           // 32-column TMEM loads per unit and thread
+constexpr int kEpiCols = kBN / 2;               // columns of a tile per epilogue thread
+constexpr int kChunks = kEpiCols / 32;          // 32-column TMEM loads per unit and thread
 constexpr int kMaxBatch = 1024;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr int kStashBytes = kEpiWarps * 32 * 32;  // 32 B per epilogue thread
-
-static_assert(kBN == 128 || kBN == 256, "tile width");
-static_assert(kEpiWarps == 8 || kEpiWarps == 16, "epilogue warps");
-static_assert(kChunks >= 1 && kChunks <= 4, "columns per epilogue thread");
 
 // Barrier slots inside the barrier block.
 constexpr int kBarBFull = 0;
@@ -94,19 +85,38 @@ size_t smem_bytes(int rb) {
 // Bounded wait on an mbarrier phase. Returns false (and raises the abort flag
 // and the device status) if the phase did not complete within kTimeoutNs, or
 // if another role already aborted.
-__device__ bool wait_bounded(uint32_t bar, uint32_t parity, Ctl* ctl, int* status) {
-  if (ptx::mbar_try_wait(bar, parity)) return true;
+__device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, Ctl* ctl, int* status) {
   const uint64_t t0 = ptx::globaltimer_ns();
-  while (true) {
+  for (uint32_t n = 1;; ++n) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
-    if (*reinterpret_cast<volatile int*>(&ctl->abort_flag)) return false;
-    if (ptx::globaltimer_ns() - t0 > kTimeoutNs) {
-      *reinterpret_cast<volatile int*>(&ctl->abort_flag) = 1;
-      atomicOr(status, kStatusTimeout);
-      return false;
+    if ((n & 255) == 0) {
+      if (*reinterpret_cast<volatile int*>(&ctl->abort_flag)) return false;
+      if (ptx::globaltimer_ns() - t0 > kTimeoutNs) {
+        *reinterpret_cast<volatile int*>(&ctl->abort_flag) = 1;
+        atomicOr(status, kStatusTimeout);
+        return false;
+      }
     }
   }
 }
+
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, Ctl* ctl, int* status) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  return wait_slow(bar, parity, ctl, status);
+}
+
+// Index and phase bit of a ring of mbarrier-guarded slots.
+struct Ring {
+  int idx = 0;
+  uint32_t phase = 0;
+  template <int N>
+  __device__ __forceinline__ void next() {
+    if (++idx == N) {
+      idx = 0;
+      phase ^= 1u;
+    }
+  }
+};
 
 // Warp-uniform bounded wait: every lane polls, the warp proceeds only if all
 // lanes saw the phase complete.
@@ -327,7 +337,7 @@ __device__ __forceinline__ void fold_wide(const uint32_t (&r)[NC][32], uint32_t 
 }
 
 template <int DT>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __maxnreg__(112)
     nn_tc_kernel(const __grid_constant__ CUtensorMap tmap_db, NNArgs a) {
   constexpr int RB = row_bytes(DT);
   using E = Epi<DT>;
@@ -379,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < kNumBars; ++i) {
       uint32_t count = 1;
       if (i >= kBarAFull && i < kBarAFull + 2) count = 32;  // producer lanes
-      if (i >= kBarAccEmpty && i < kBarAccEmpty + kAcc) count = kEpiWarps;
+      if (i >= kBarAccEmpty && i < kBarAccEmpty + kAcc) count = kGroupWarps;
       ptx::mbar_init(ptx::smem_u32(&ctl->bars[i]), count);
     }
     ptx::fence_mbar_init();
@@ -405,10 +415,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kProducerWarp) {
     // ---------------------------------------------------------------- producer
     Pos p = start;
-    int64_t it = 0, seg = 0;
-    int64_t last_issue[kStages];
+    Ring st;            // database stage ring
+    int64_t seg = 0;
+    int last_phase[kStages];  // phase bit of the last load issued into each stage, or -1
 #pragma unroll
-    for (int s = 0; s < kStages; ++s) last_issue[s] = -1;
+    for (int s = 0; s < kStages; ++s) last_phase[s] = -1;
     bool ok = true;
     for (int64_t u = u0; ok && u < u1; ++seg) {
       const int64_t len = seg_len(p, u, u1, nt);
@@ -419,34 +430,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       gather_a<RB>(tileA + as * tile_bytes_a(RB), a, p.b, p.m, ctl->cnt[p.b], lane);
       ptx::fence_proxy_async_smem();
       ptx::mbar_arrive(bar(kBarAFull + as));
-      const int64_t row0 = static_cast<int64_t>(p.b) * a.ndb + p.n * kBN;
-      for (int64_t j = 0; j < len; ++j, ++it) {
-        const int s = static_cast<int>(it % kStages);
-        const uint32_t ph = static_cast<uint32_t>((it / kStages) & 1);
-        bool lok = true;
-        if (lane == 0) {
-          lok = wait_bounded(bar(kBarBEmpty + s), ph ^ 1, ctl, a.status);
-          if (lok) {
-            ptx::mbar_arrive_expect_tx(bar(kBarBFull + s), static_cast<uint32_t>(tile_bytes_b(RB)));
-            ptx::tma_load_2d(ptx::smem_u32(tileB + s * tile_bytes_b(RB)), &tmap_db, 0,
-                             static_cast<int32_t>(row0 + j * kBN), bar(kBarBFull + s));
-            last_issue[s] = it;
+      if (lane == 0) {
+        int32_t row = static_cast<int32_t>(static_cast<int64_t>(p.b) * a.ndb + p.n * kBN);
+        for (int64_t j = 0; j < len; ++j, row += kBN) {
+          if (!wait_bounded(bar(kBarBEmpty + st.idx), st.phase ^ 1u, ctl, a.status)) {
+            ok = false;
+            break;
           }
-        }
-        if (!__shfl_sync(0xffffffffu, lok ? 1 : 0, 0)) {
-          ok = false;
-          break;
+          ptx::mbar_arrive_expect_tx(bar(kBarBFull + st.idx), static_cast<uint32_t>(tile_bytes_b(RB)));
+          ptx::tma_load_2d(ptx::smem_u32(tileB + st.idx * tile_bytes_b(RB)), &tmap_db, 0, row,
+                           bar(kBarBFull + st.idx));
+          last_phase[st.idx] = static_cast<int>(st.phase);
+          st.next<kStages>();
         }
       }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       u += len;
       next_segment(p, ctl, batch);
     }
     // Drain: every TMA load this warp issued must land before smem is freed.
     if (lane == 0) {
       for (int s = 0; s < kStages; ++s)
-        if (last_issue[s] >= 0)
-          wait_bounded(bar(kBarBFull + s), static_cast<uint32_t>((last_issue[s] / kStages) & 1),
-                       ctl, a.status);
+        if (last_phase[s] >= 0)
+          wait_bounded(bar(kBarBFull + s), static_cast<uint32_t>(last_phase[s]), ctl, a.status);
     }
   } else if (warp == kMmaWarp) {
     // --------------------------------------------------------------- MMA issue
@@ -456,7 +462,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               ? ((2u << 4) | (1u << 7) | (1u << 10) | ((kBN >> 3) << 17) | ((kBM >> 4) << 24))
               : ((1u << 4) | (1u << 7) | (1u << 10) | ((kBN >> 3) << 17) | ((kBM >> 4) << 24));
       Pos p = start;
-      int64_t it = 0, seg = 0;
+      Ring st, ac;  // database stage ring, accumulator ring
+      int64_t seg = 0;
       bool ok = true;
       for (int64_t u = u0; ok && u < u1; ++seg) {
         const int64_t len = seg_len(p, u, u1, nt);
@@ -467,20 +474,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tc_fence_after();
         const uint64_t adesc =
             ptx::smem_desc_kmajor(ptx::smem_u32(tileA + as * tile_bytes_a(RB)), RB);
-        for (int64_t j = 0; j < len; ++j, ++it) {
-          const int acc = static_cast<int>(it % kAcc);
-          const int s = static_cast<int>(it % kStages);
-          if (!wait_bounded(bar(kBarAccEmpty + acc),
-                            static_cast<uint32_t>(((it / kAcc) & 1) ^ 1), ctl, a.status) ||
-              !wait_bounded(bar(kBarBFull + s), static_cast<uint32_t>((it / kStages) & 1), ctl,
-                            a.status)) {
+        const uint64_t bdesc0 = ptx::smem_desc_kmajor(ptx::smem_u32(tileB), RB);
+        for (int64_t j = 0; j < len; ++j) {
+          if (!wait_bounded(bar(kBarAccEmpty + ac.idx), ac.phase ^ 1u, ctl, a.status) ||
+              !wait_bounded(bar(kBarBFull + st.idx), st.phase, ctl, a.status)) {
             ok = false;
             break;
           }
           ptx::tc_fence_after();
-          const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * kBN);
-          const uint64_t bdesc =
-              ptx::smem_desc_kmajor(ptx::smem_u32(tileB + s * tile_bytes_b(RB)), RB);
+          const uint32_t d_tmem = tmem + static_cast<uint32_t>(ac.idx * kBN);
+          const uint64_t bdesc = bdesc0 + static_cast<uint64_t>((st.idx * tile_bytes_b(RB)) >> 4);
           if constexpr (DT == FASTNN_I8) {
             ptx::mma_i8(d_tmem, adesc, bdesc, kIdesc, 0u);
           } else {
@@ -488,8 +491,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mma_bf16(d_tmem, adesc, bdesc, kIdesc, 0u);
             ptx::mma_bf16(d_tmem, adesc + 2, bdesc + 2, kIdesc, 1u);
           }
-          ptx::mma_commit(bar(kBarBEmpty + s));
-          ptx::mma_commit(bar(kBarAccFull + acc));
+          ptx::mma_commit(bar(kBarBEmpty + st.idx));
+          ptx::mma_commit(bar(kBarAccFull + ac.idx));
+          st.next<kStages>();
+          ac.next<kAcc>();
         }
         if (!ok) break;
         ptx::mma_commit(bar(kBarAEmpty + as));
@@ -502,29 +507,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------------------------------------------------------- epilogue
-    const int lg = warp & 3;  // TMEM lane quarter this warp may access
-    const int h = warp >> 2;  // column block (of kEpiCols) of the tile
+    // Group g folds the units whose running index is congruent to g mod 2,
+    // i.e. the ones the MMA wrote into accumulator g.
+    const int grp = warp / kGroupWarps;
+    const int gw = warp % kGroupWarps;
+    const int lg = gw & 3;   // TMEM lane quarter (warp id mod 4)
+    const int h = gw >> 2;   // column half of the tile
     const bool pack16 = ctl->pack16 != 0;
     const int tail = static_cast<int>(a.ndb - (nt - 1) * kBN);  // valid columns, last tile
+    const uint32_t acc_bar = bar(kBarAccFull + grp);
+    const uint32_t rel_bar = bar(kBarAccEmpty + grp);
+    const uint32_t taddr = tmem + (static_cast<uint32_t>(lg * 32) << 16) +
+                           static_cast<uint32_t>(grp * kBN + h * kEpiCols);
     uint4* slot = stash + 2 * threadIdx.x;
     Pos p = start;
-    int64_t it = 0;
+    int64_t it = 0;        // running unit index at the start of the segment
+    uint32_t phase = 0;    // phase bit of this group's accumulator barrier
     bool ok = true;
     for (int64_t u = u0; ok && u < u1;) {
       const int64_t len = seg_len(p, u, u1, nt);
       typename E::S best = E::lowest();
       uint32_t bidx = 0xFFFFFFFFu;
-      for (int64_t j = 0; j < len; ++j, ++it) {
-        const int acc = static_cast<int>(it % kAcc);
-        if (!warp_wait_bounded(bar(kBarAccFull + acc), static_cast<uint32_t>((it / kAcc) & 1),
-                               ctl, a.status)) {
+      for (int64_t j = ((grp - it) & 1); j < len; j += kAcc) {
+        if (!warp_wait_bounded(acc_bar, phase, ctl, a.status)) {
           ok = false;
           break;
         }
+        phase ^= 1u;
         ptx::tc_fence_after();
         const int64_t n = p.n + j;
-        const uint32_t taddr = tmem + (static_cast<uint32_t>(lg * 32) << 16) +
-                               static_cast<uint32_t>(acc * kBN + h * kEpiCols);
         const uint32_t colbase = static_cast<uint32_t>(n * kBN + h * kEpiCols);
         if (n == nt - 1 && tail < kBN) {
           // Ragged last tile of the database: column-masked fold.
@@ -539,7 +550,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           ptx::tc_fence_before();
           __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(bar(kBarAccEmpty + acc));
+          if (lane == 0) ptx::mbar_arrive(rel_bar);
         } else if (DT == FASTNN_I8 && pack16) {
           uint32_t r[kChunks][16];
 #pragma unroll
@@ -548,17 +559,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           // The accumulator is free for the next MMA once it is in registers.
           ptx::tc_fence_before();
           __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(bar(kBarAccEmpty + acc));
+          if (lane == 0) ptx::mbar_arrive(rel_bar);
           if constexpr (DT == FASTNN_I8) fold_pack16<kChunks>(r, colbase, best, bidx, slot);
         } else {
-          uint32_t r[kChunks][32];
-#pragma unroll
-          for (int c = 0; c < kChunks; ++c) ptx::tmem_ld32(taddr + c * 32, r[c]);
+          // 32-bit scores: two 64-column halves, the accumulator is released
+          // after the second load.
+          uint32_t r[2][32];
+          ptx::tmem_ld32(taddr, r[0]);
+          ptx::tmem_ld32(taddr + 32, r[1]);
+          ptx::tmem_ld_wait();
+          fold_wide<DT, 2>(r, colbase, best, bidx, slot);
+          ptx::tmem_ld32(taddr + 64, r[0]);
+          ptx::tmem_ld32(taddr + 96, r[1]);
           ptx::tmem_ld_wait();
           ptx::tc_fence_before();
           __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(bar(kBarAccEmpty + acc));
-          fold_wide<DT, kChunks>(r, colbase, best, bidx, slot);
+          if (lane == 0) ptx::mbar_arrive(rel_bar);
+          fold_wide<DT, 2>(r, colbase + 64, best, bidx, slot);
         }
       }
       if (!ok) break;
@@ -567,6 +584,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         atomicMax(reinterpret_cast<unsigned long long*>(&a.out_key[p.b * a.q_cap + k]),
                   static_cast<unsigned long long>(make_key(E::ord(best), bidx)));
       u += len;
+      it += len;
       next_segment(p, ctl, batch);
     }
   }
