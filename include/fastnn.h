@@ -149,6 +149,10 @@ int fastnn_device_status(const void *workspace, fastnn_stream_t stream);
 int fastnn_kernel_timer_enable(int capacity);
 int fastnn_kernel_timer_read(int *launches, double *total_ms);
 
+/* Text of the last CUDA runtime error this library saw on the calling host
+ * thread (the cause behind a FASTNN_ERR_CUDA return); a static string. */
+const char *fastnn_last_cuda_error(void);
+
 /* Human-readable name of a fastnn_status value (static string). */
 const char *fastnn_status_str(int status);
 

@@ -22,7 +22,10 @@ _lib = None
 class FastNNError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
-        super().__init__(f"{what}: {fastnn_status_str(status)} ({status})")
+        msg = f"{what}: {fastnn_status_str(status)} ({status})"
+        if status == -4:
+            msg += ": " + library().fastnn_last_cuda_error().decode()
+        super().__init__(msg)
 
 
 def library_path() -> str:
@@ -54,6 +57,8 @@ def library():
     lib.fastnn_kernel_timer_enable.restype = I
     lib.fastnn_kernel_timer_read.argtypes = [ctypes.POINTER(I), ctypes.POINTER(ctypes.c_double)]
     lib.fastnn_kernel_timer_read.restype = I
+    lib.fastnn_last_cuda_error.argtypes = []
+    lib.fastnn_last_cuda_error.restype = ctypes.c_char_p
     lib.fastnn_status_str.argtypes = [I]
     lib.fastnn_status_str.restype = ctypes.c_char_p
     _lib = lib

@@ -9,6 +9,13 @@
 
 using namespace fastnn;
 
+namespace fastnn {
+namespace {
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+}
+void note_cuda_error(cudaError_t e) { g_last_cuda_error = e; }
+}  // namespace fastnn
+
 namespace {
 
 constexpr size_t kAlign = 256;
@@ -327,6 +334,10 @@ int fastnn_kernel_timer_enable(int capacity) { return kernel_timer_enable(capaci
 
 int fastnn_kernel_timer_read(int* launches, double* total_ms) {
   return kernel_timer_read(launches, total_ms);
+}
+
+const char* fastnn_last_cuda_error(void) {
+  return cudaGetErrorString(fastnn::g_last_cuda_error);
 }
 
 const char* fastnn_status_str(int status) {

@@ -84,8 +84,17 @@ __device__ __forceinline__ int64_t nn_query_row(const NNArgs& a, int b, int64_t 
 
 }  // namespace fastnn
 
+namespace fastnn {
+// Records the most recent CUDA runtime error seen by the library (read with
+// fastnn_last_cuda_error()).
+void note_cuda_error(cudaError_t e);
+}  // namespace fastnn
+
 #define FASTNN_CUDA_TRY(expr)                              \
   do {                                                     \
     cudaError_t e_ = (expr);                               \
-    if (e_ != cudaSuccess) return FASTNN_ERR_CUDA;         \
+    if (e_ != cudaSuccess) {                               \
+      ::fastnn::note_cuda_error(e_);                       \
+      return FASTNN_ERR_CUDA;                              \
+    }                                                      \
   } while (0)
