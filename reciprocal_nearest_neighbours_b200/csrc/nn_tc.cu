@@ -337,7 +337,7 @@ __device__ __forceinline__ void fold_wide(const uint32_t (&r)[NC][32], uint32_t 
 }
 
 template <int DT>
-__global__ void __maxnreg__(104)
+__global__ void __launch_bounds__(kThreads, 1)
     nn_tc_kernel(const __grid_constant__ CUtensorMap tmap_db, NNArgs a) {
   constexpr int RB = row_bytes(DT);
   using E = Epi<DT>;
