@@ -50,6 +50,7 @@ constexpr int kEpiCols = kBN / 2;               // columns of a tile per epilogu
 constexpr int kChunks = kEpiCols / 32;          // 32-column TMEM loads per unit and thread
 constexpr int kMaxBatch = 1024;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
+constexpr int kStashBytes = kEpiWarps * 32 * 32;  // 32 B per epilogue thread
 
 // Barrier slots inside the barrier block.
 constexpr int kBarBFull = 0;
@@ -78,7 +79,7 @@ __host__ __device__ constexpr size_t ctl_bytes() { return (sizeof(Ctl) + 15) & ~
 
 size_t smem_bytes(int rb) {
   return 1024 /* alignment slack */ + 2 * tile_bytes_a(rb) + kStages * tile_bytes_b(rb) +
-         ctl_bytes();
+         ctl_bytes() + kStashBytes;
 }
 
 // Bounded wait on an mbarrier phase. Returns false (and raises the abort flag
@@ -230,14 +231,13 @@ __device__ __forceinline__ void fold32_masked(const uint32_t (&r)[32], uint32_t 
 }
 
 // ---- fast epilogue for full tiles ------------------------------------------
-// Each thread owns one query row and a block of columns of the tile. Their
-// maximum is formed with a reduction tree over registers that die as the tree
-// consumes them. Only when it beats the running best strictly (a new record
-// for this row) is the first column holding it searched for: the 32-column
-// chunk holding it is read again from TMEM (the accumulator is released only
-// after this check) and scanned. The lowest index among equal scores
-// survives because columns are visited in ascending order and a record needs
-// a strictly greater score.
+// Each thread owns one query row and kEpiCols columns of the tile. Their
+// maximum is formed with a reduction tree; only when it beats the running best
+// strictly (a new record for this row) is the first column holding it
+// searched for: the 8-register group holding it is found from the tree's
+// group maxima, staged to this thread's 32-byte slot in shared memory, and
+// scanned there, so the search needs no dynamic register indexing. The lowest
+// index among equal scores survives.
 
 __device__ __forceinline__ uint32_t vmax3_s16x2(uint32_t a, uint32_t b, uint32_t c) {
   return ptx::vmax_s16x2(ptx::vmax_s16x2(a, b), c);
@@ -253,109 +253,86 @@ __device__ __forceinline__ uint32_t tree8_s16x2(const uint32_t* r) {
 __device__ __forceinline__ int lo16(uint32_t x) { return static_cast<int>(static_cast<int16_t>(x & 0xFFFFu)); }
 __device__ __forceinline__ int hi16(uint32_t x) { return static_cast<int>(x) >> 16; }
 
-// int8 scores that fit in 16 bits, 128 columns at TMEM address `taddr`
-// (global column colbase + c): packed loads put columns 2i / 2i + 1 of a
-// 32-column chunk into the low / high half of register i.
-__device__ __forceinline__ void fold128_pack16(uint32_t taddr, uint32_t colbase, int& best,
-                                               uint32_t& bidx) {
-  uint32_t g[8];  // maxima of 16-column groups
-  {
-    uint32_t r[4][16];
+__device__ __forceinline__ void stash8(uint4* slot, const uint32_t* r) {
+  slot[0] = make_uint4(r[0], r[1], r[2], r[3]);
+  slot[1] = make_uint4(r[4], r[5], r[6], r[7]);
+}
+
+// int8 scores that fit in 16 bits: r[c][i] holds columns 32c + 2i (low half)
+// and 32c + 2i + 1 (high half) of this thread's block.
+template <int NC>
+__device__ __forceinline__ void fold_pack16(const uint32_t (&r)[NC][16], uint32_t colbase,
+                                            int& best, uint32_t& bidx, uint4* slot) {
+  constexpr int G = 2 * NC;  // groups of 8 registers = 16 columns
+  uint32_t g[G];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) ptx::tmem_ld16_pack(taddr + c * 32, r[c]);
-    ptx::tmem_ld_wait();
-#pragma unroll
-    for (int i = 0; i < 8; ++i) g[i] = tree8_s16x2(&r[i / 2][(i % 2) * 8]);
+  for (int i = 0; i < G; ++i) g[i] = tree8_s16x2(&r[i / 2][(i % 2) * 8]);
+  uint32_t u;
+  if constexpr (G == 2) {
+    u = ptx::vmax_s16x2(g[0], g[1]);
+  } else if constexpr (G == 4) {
+    u = ptx::vmax_s16x2(ptx::vmax_s16x2(g[0], g[1]), ptx::vmax_s16x2(g[2], g[3]));
+  } else {
+    u = vmax3_s16x2(vmax3_s16x2(g[0], g[1], g[2]), vmax3_s16x2(g[3], g[4], g[5]),
+                    ptx::vmax_s16x2(g[6], g[7]));
   }
-  const uint32_t u = vmax3_s16x2(vmax3_s16x2(g[0], g[1], g[2]), vmax3_s16x2(g[3], g[4], g[5]),
-                                 ptx::vmax_s16x2(g[6], g[7]));
   const int m = max(lo16(u), hi16(u));
-  const bool rec = m > best;
-  if (__any_sync(0xffffffffu, rec)) {
-    int gi = 7;
+  if (m > best) {
+    best = m;
+    int gi = G - 1;
 #pragma unroll
-    for (int i = 7; i >= 0; --i)
+    for (int i = G - 1; i >= 0; --i)
       if (lo16(g[i]) == m || hi16(g[i]) == m) gi = i;
-    int w = 0;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const bool mine = rec && (gi >> 1) == c;
-      if (__any_sync(0xffffffffu, mine)) {
-        uint32_t x[16];
-        ptx::tmem_ld16_pack(taddr + c * 32, x);
-        ptx::tmem_ld_wait();
-        if (mine) {
-          const bool up = gi & 1;
-          int ww = 15;
+    for (int i = 0; i < G; ++i)
+      if (i == gi) stash8(slot, &r[i / 2][(i % 2) * 8]);
+    const uint4 a = slot[0], b = slot[1];
+    const uint32_t x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    int w = 15;
 #pragma unroll
-          for (int j = 7; j >= 0; --j) {
-            const uint32_t v = up ? x[8 + j] : x[j];
-            if (hi16(v) == m) ww = 2 * j + 1;
-            if (lo16(v) == m) ww = 2 * j;
-          }
-          w = ww;
-        }
-      }
+    for (int j = 7; j >= 0; --j) {
+      if (hi16(x[j]) == m) w = 2 * j + 1;
+      if (lo16(x[j]) == m) w = 2 * j;
     }
-    if (rec) {
-      best = m;
-      bidx = colbase + 16 * gi + w;
-    }
+    bidx = colbase + 16 * gi + w;
   }
 }
 
-// 32-bit scores (int32, or fp32 for bf16 descriptors), 64 columns at TMEM
-// address `taddr` (global column colbase + c).
-template <int DT>
-__device__ __forceinline__ void fold64_wide(uint32_t taddr, uint32_t colbase,
-                                            typename Epi<DT>::S& best, uint32_t& bidx) {
+// 32-bit scores (int32, or fp32 for bf16 descriptors): r[c][i] = column 32c + i.
+template <int DT, int NC>
+__device__ __forceinline__ void fold_wide(const uint32_t (&r)[NC][32], uint32_t colbase,
+                                          typename Epi<DT>::S& best, uint32_t& bidx,
+                                          uint4* slot) {
   using E = Epi<DT>;
   using S = typename E::S;
-  S g[8];  // maxima of 8-column groups
-  {
-    uint32_t r[2][32];
-    ptx::tmem_ld32(taddr, r[0]);
-    ptx::tmem_ld32(taddr + 32, r[1]);
-    ptx::tmem_ld_wait();
+  constexpr int G = 4 * NC;  // groups of 8 registers = 8 columns
+  S g[G];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint32_t* q = &r[i / 4][(i % 4) * 8];
-      const S a0 = E::mx3(E::as_score(q[0]), E::as_score(q[1]), E::as_score(q[2]));
-      const S a1 = E::mx3(E::as_score(q[3]), E::as_score(q[4]), E::as_score(q[5]));
-      g[i] = E::mx3(a0, a1, E::mx(E::as_score(q[6]), E::as_score(q[7])));
-    }
+  for (int i = 0; i < G; ++i) {
+    const uint32_t* q = &r[i / 4][(i % 4) * 8];
+    const S a0 = E::mx3(E::as_score(q[0]), E::as_score(q[1]), E::as_score(q[2]));
+    const S a1 = E::mx3(E::as_score(q[3]), E::as_score(q[4]), E::as_score(q[5]));
+    g[i] = E::mx3(a0, a1, E::mx(E::as_score(q[6]), E::as_score(q[7])));
   }
-  const S m = E::mx3(E::mx3(g[0], g[1], g[2]), E::mx3(g[3], g[4], g[5]), E::mx(g[6], g[7]));
-  const bool rec = m > best;
-  if (__any_sync(0xffffffffu, rec)) {
-    int gi = 7;
+  S m = g[0];
 #pragma unroll
-    for (int i = 7; i >= 0; --i)
+  for (int i = 1; i < G; ++i) m = E::mx(m, g[i]);
+  if (m > best) {
+    best = m;
+    int gi = G - 1;
+#pragma unroll
+    for (int i = G - 1; i >= 0; --i)
       if (g[i] == m) gi = i;
-    int w = 0;
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      const bool mine = rec && (gi >> 2) == c;
-      if (__any_sync(0xffffffffu, mine)) {
-        uint32_t x[32];
-        ptx::tmem_ld32(taddr + c * 32, x);
-        ptx::tmem_ld_wait();
-        if (mine) {
-          const int q = gi & 3;
-          int ww = 7;
+    for (int i = 0; i < G; ++i)
+      if (i == gi) stash8(slot, &r[i / 4][(i % 4) * 8]);
+    const uint4 a = slot[0], b = slot[1];
+    const uint32_t x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    int w = 7;
 #pragma unroll
-          for (int j = 7; j >= 0; --j) {
-            const uint32_t v = q == 0 ? x[j] : q == 1 ? x[8 + j] : q == 2 ? x[16 + j] : x[24 + j];
-            if (E::as_score(v) == m) ww = j;
-          }
-          w = ww;
-        }
-      }
-    }
-    if (rec) {
-      best = m;
-      bidx = colbase + 8 * gi + w;
-    }
+    for (int j = 7; j >= 0; --j)
+      if (E::as_score(x[j]) == m) w = j;
+    bidx = colbase + 8 * gi + w;
   }
 }
 
@@ -370,6 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* tileA = smem;                          // 2 x kBM x RB
   uint8_t* tileB = tileA + 2 * tile_bytes_a(RB);  // kStages x kBN x RB
   Ctl* ctl = reinterpret_cast<Ctl*>(tileB + kStages * tile_bytes_b(RB));
+  uint4* stash = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(ctl) + ctl_bytes());
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -541,26 +519,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t rel_bar = bar(kBarAccEmpty + grp);
     const uint32_t taddr = tmem + (static_cast<uint32_t>(lg * 32) << 16) +
                            static_cast<uint32_t>(grp * kBN + h * kEpiCols);
+    uint4* slot = stash + 2 * threadIdx.x;
     Pos p = start;
-    int par = 0;           // parity of the running unit index at the segment start
+    int64_t it = 0;        // running unit index at the start of the segment
     uint32_t phase = 0;    // phase bit of this group's accumulator barrier
     bool ok = true;
-    const int last_n = static_cast<int>(nt - 1);
     for (int64_t u = u0; ok && u < u1;) {
-      const int len = static_cast<int>(seg_len(p, u, u1, nt));
-      const int n0 = static_cast<int>(p.n);
+      const int64_t len = seg_len(p, u, u1, nt);
       typename E::S best = E::lowest();
       uint32_t bidx = 0xFFFFFFFFu;
-      for (int j = (grp - par) & 1; j < len; j += kAcc) {
+      for (int64_t j = ((grp - it) & 1); j < len; j += kAcc) {
         if (!warp_wait_bounded(acc_bar, phase, ctl, a.status)) {
           ok = false;
           break;
         }
         phase ^= 1u;
         ptx::tc_fence_after();
-        const int n = n0 + j;
-        const uint32_t colbase = static_cast<uint32_t>(n) * kBN + h * kEpiCols;
-        if (n == last_n && tail < kBN) {
+        const int64_t n = p.n + j;
+        const uint32_t colbase = static_cast<uint32_t>(n * kBN + h * kEpiCols);
+        if (n == nt - 1 && tail < kBN) {
           // Ragged last tile of the database: column-masked fold.
           const int valid_blk = tail - h * kEpiCols;
 #pragma unroll 1
@@ -574,22 +551,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           ptx::tc_fence_before();
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(rel_bar);
-        } else {
-          if constexpr (DT == FASTNN_I8) {
-            if (pack16) {
-              fold128_pack16(taddr, colbase, best, bidx);
-            } else {
-              fold64_wide<DT>(taddr, colbase, best, bidx);
-              fold64_wide<DT>(taddr + 64, colbase + 64, best, bidx);
-            }
-          } else {
-            fold64_wide<DT>(taddr, colbase, best, bidx);
-            fold64_wide<DT>(taddr + 64, colbase + 64, best, bidx);
-          }
-          // The accumulator goes back to the MMA once every read of it is done.
+        } else if (DT == FASTNN_I8 && pack16) {
+          uint32_t r[kChunks][16];
+#pragma unroll
+          for (int c = 0; c < kChunks; ++c) ptx::tmem_ld16_pack(taddr + c * 32, r[c]);
+          ptx::tmem_ld_wait();
+          // The accumulator is free for the next MMA once it is in registers.
           ptx::tc_fence_before();
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(rel_bar);
+          if constexpr (DT == FASTNN_I8) fold_pack16<kChunks>(r, colbase, best, bidx, slot);
+        } else {
+          // 32-bit scores: two 64-column halves, the accumulator is released
+          // after the second load.
+          uint32_t r[2][32];
+          ptx::tmem_ld32(taddr, r[0]);
+          ptx::tmem_ld32(taddr + 32, r[1]);
+          ptx::tmem_ld_wait();
+          fold_wide<DT, 2>(r, colbase, best, bidx, slot);
+          ptx::tmem_ld32(taddr + 64, r[0]);
+          ptx::tmem_ld32(taddr + 96, r[1]);
+          ptx::tmem_ld_wait();
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(rel_bar);
+          fold_wide<DT, 2>(r, colbase + 64, best, bidx, slot);
         }
       }
       if (!ok) break;
@@ -598,7 +584,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         atomicMax(reinterpret_cast<unsigned long long*>(&a.out_key[p.b * a.q_cap + k]),
                   static_cast<unsigned long long>(make_key(E::ord(best), bidx)));
       u += len;
-      par ^= len & 1;
+      it += len;
       next_segment(p, ctl, batch);
     }
   }
