@@ -53,23 +53,14 @@ constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr int kStashBytes = kEpiWarps * 32 * 32;  // 32 B per epilogue thread
 
 // Barrier slots inside the barrier block.
-//   BFull[s]   database tile s landed (TMA transaction count)
-//   Tile[s]    the MMA that read stage s finished: stage s may be refilled and
-//              its accumulator (unit index mod 2) may be read. Units cycle
-//              through the stages, and kStages is a multiple of kAcc, so the
-//              k-th unit lands in stage k mod kStages and accumulator k mod 2;
-//              one tcgen05.commit per unit serves both waiters.
-//   AFull/AEmpty  query tile gathered / no longer read (two buffers)
-//   AccEmpty[g]   epilogue group g has read accumulator g
-//   Done       every MMA issued so far has completed (teardown)
 constexpr int kBarBFull = 0;
-constexpr int kBarTile = kBarBFull + kStages;
-constexpr int kBarAFull = kBarTile + kStages;
+constexpr int kBarBEmpty = kBarBFull + kStages;
+constexpr int kBarAFull = kBarBEmpty + kStages;
 constexpr int kBarAEmpty = kBarAFull + 2;
-constexpr int kBarAccEmpty = kBarAEmpty + 2;
+constexpr int kBarAccFull = kBarAEmpty + 2;
+constexpr int kBarAccEmpty = kBarAccFull + kAcc;
 constexpr int kBarDone = kBarAccEmpty + kAcc;
 constexpr int kNumBars = kBarDone + 1;
-static_assert(kStages % kAcc == 0, "stage ring must be a multiple of the accumulator ring");
 
 struct Ctl {
   uint64_t bars[kNumBars];
@@ -442,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         int32_t row = static_cast<int32_t>(static_cast<int64_t>(p.b) * a.ndb + p.n * kBN);
         for (int64_t j = 0; j < len; ++j, row += kBN) {
-          if (!wait_bounded(bar(kBarTile + st.idx), st.phase ^ 1u, ctl, a.status)) {
+          if (!wait_bounded(bar(kBarBEmpty + st.idx), st.phase ^ 1u, ctl, a.status)) {
             ok = false;
             break;
           }
@@ -500,7 +491,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mma_bf16(d_tmem, adesc, bdesc, kIdesc, 0u);
             ptx::mma_bf16(d_tmem, adesc + 2, bdesc + 2, kIdesc, 1u);
           }
-          ptx::mma_commit(bar(kBarTile + st.idx));
+          ptx::mma_commit(bar(kBarBEmpty + st.idx));
+          ptx::mma_commit(bar(kBarAccFull + ac.idx));
           st.next<kStages>();
           ac.next<kAcc>();
         }
@@ -523,29 +515,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int h = gw >> 2;   // column half of the tile
     const bool pack16 = ctl->pack16 != 0;
     const int tail = static_cast<int>(a.ndb - (nt - 1) * kBN);  // valid columns, last tile
+    const uint32_t acc_bar = bar(kBarAccFull + grp);
     const uint32_t rel_bar = bar(kBarAccEmpty + grp);
-    int ts = grp;          // stage (= tile barrier) of this group's next unit
     const uint32_t taddr = tmem + (static_cast<uint32_t>(lg * 32) << 16) +
                            static_cast<uint32_t>(grp * kBN + h * kEpiCols);
     uint4* slot = stash + 2 * threadIdx.x;
     Pos p = start;
     int64_t it = 0;        // running unit index at the start of the segment
-    uint32_t phase = 0;    // phase bit of that tile barrier
+    uint32_t phase = 0;    // phase bit of this group's accumulator barrier
     bool ok = true;
     for (int64_t u = u0; ok && u < u1;) {
       const int64_t len = seg_len(p, u, u1, nt);
       typename E::S best = E::lowest();
       uint32_t bidx = 0xFFFFFFFFu;
       for (int64_t j = ((grp - it) & 1); j < len; j += kAcc) {
-        if (!warp_wait_bounded(bar(kBarTile + ts), phase, ctl, a.status)) {
+        if (!warp_wait_bounded(acc_bar, phase, ctl, a.status)) {
           ok = false;
           break;
         }
-        ts += kAcc;
-        if (ts >= kStages) {
-          ts -= kStages;
-          phase ^= 1u;
-        }
+        phase ^= 1u;
         ptx::tc_fence_after();
         const int64_t n = p.n + j;
         const uint32_t colbase = static_cast<uint32_t>(n * kBN + h * kEpiCols);
