@@ -22,7 +22,8 @@ constexpr size_t kAlign = 256;
 constexpr int kPadRows = 256;  // zero rows after each repacked database (one TMA box)
 constexpr int kMaxIter = 255;
 // Status block at the head of every workspace: [0] device status word,
-// [1] / [2] max |element| of the first / second int8 map.
+// [1] / [2] max |element| of the first / second int8 map, [4] / [5] grid-
+// barrier arrival counter and abort word of the persistent matching kernel.
 constexpr size_t kStatusBytes = 64 * sizeof(int);
 constexpr int64_t kMaxSeeds = (int64_t{1} << 24) - 1;
 
@@ -200,73 +201,58 @@ int fastnn_reciprocal(const void* desc1, int H1, int W1, const void* desc2, int 
   Carver c{static_cast<uint8_t*>(workspace)};
   RecLayout L = carve_rec(c, N1, N2, dtype, batch, S);
 
+  // Status block: status word, per-map max |element|, grid-barrier words.
   FASTNN_CUDA_TRY(cudaMemsetAsync(L.status, 0, kStatusBytes, st));
-  FASTNN_CUDA_TRY(cudaMemsetAsync(L.fwd, 0, static_cast<size_t>(batch) * S * 8, st));
-  FASTNN_CUDA_TRY(cudaMemsetAsync(L.bwd, 0, static_cast<size_t>(batch) * S * 8, st));
-  FASTNN_CUDA_TRY(cudaMemsetAsync(L.claim, 0xFF, static_cast<size_t>(batch) * N1 * 4, st));
-  FASTNN_CUDA_TRY(cudaMemsetAsync(out_count, 0, static_cast<size_t>(batch) * 4, st));
-  if (out_iters) FASTNN_CUDA_TRY(cudaMemsetAsync(out_iters, 0, static_cast<size_t>(batch) * 4, st));
-  if (out_frontier)
-    FASTNN_CUDA_TRY(cudaMemsetAsync(out_frontier, 0, static_cast<size_t>(batch) * max_iter * 4, st));
   FASTNN_TRY(launch_repack(desc1, batch * N1, d, dtype, L.d1rep, kPadRows, L.status + 1, st));
   FASTNN_TRY(launch_repack(desc2, batch * N2, d, dtype, L.d2rep, kPadRows, L.status + 2, st));
-  FASTNN_TRY(launch_seed(L.F[0], S, L.claim, N1, L.cnt[0], H1, W1, subsample,
-                         static_cast<int>(S), batch, st));
 
-  for (int t = 1; t <= max_iter; ++t) {
-    const int cur = (t - 1) & 1, nxt = t & 1;
-    NNArgs fwd{};
-    fwd.q_rows = L.d1rep;
-    fwd.q_rows_per_pair = N1;
-    fwd.q_index = L.F[cur];
-    fwd.q_cap = S;
-    fwd.q_count = L.cnt[cur];
-    fwd.db_rows = L.d2rep;
-    fwd.ndb = N2;
-    fwd.out_key = L.fwd;
-    fwd.batch = batch;
-    fwd.status = L.status;
-    fwd.d = d;
-    fwd.q_absmax = L.status + 1;
-    fwd.db_absmax = L.status + 2;
-    FASTNN_TRY(launch_nn_tc(fwd, dtype, batch * N2 + kPadRows, st));
-
-    NNArgs bwd{};
-    bwd.q_rows = L.d2rep;
-    bwd.q_rows_per_pair = N2;
-    bwd.q_key = L.fwd;
-    bwd.q_cap = S;
-    bwd.q_count = L.cnt[cur];
-    bwd.db_rows = L.d1rep;
-    bwd.ndb = N1;
-    bwd.out_key = L.bwd;
-    bwd.batch = batch;
-    bwd.status = L.status;
-    bwd.d = d;
-    bwd.q_absmax = L.status + 2;
-    bwd.db_absmax = L.status + 1;
-    FASTNN_TRY(launch_nn_tc(bwd, dtype, batch * N1 + kPadRows, st));
-
-    CompactArgs ca{};
-    ca.F_cur = L.F[cur];
-    ca.F_next = L.F[nxt];
-    ca.S_cap = S;
-    ca.cnt_cur = L.cnt[cur];
-    ca.cnt_next = L.cnt[nxt];
-    ca.fwd_key = L.fwd;
-    ca.bwd_key = L.bwd;
-    ca.claim = L.claim;
-    ca.N1 = N1;
-    ca.out_pairs = out_pairs;
-    ca.out_score = out_score;
-    ca.cap = capacity;
-    ca.out_count = out_count;
-    ca.out_iters = out_iters;
-    ca.out_frontier = out_frontier;
-    ca.max_iter = max_iter;
-    FASTNN_TRY(launch_check_compact(ca, dtype, t, t == max_iter, batch, st));
-  }
-  return FASTNN_OK;
+  RecArgs r{};
+  r.fwd.q_rows = L.d1rep;
+  r.fwd.q_rows_per_pair = N1;
+  r.fwd.q_cap = S;
+  r.fwd.db_rows = L.d2rep;
+  r.fwd.ndb = N2;
+  r.fwd.out_key = L.fwd;
+  r.fwd.batch = batch;
+  r.fwd.status = L.status;
+  r.fwd.d = d;
+  r.fwd.q_absmax = L.status + 1;
+  r.fwd.db_absmax = L.status + 2;
+  r.bwd = r.fwd;
+  r.bwd.q_rows = L.d2rep;
+  r.bwd.q_rows_per_pair = N2;
+  r.bwd.q_key = L.fwd;
+  r.bwd.db_rows = L.d1rep;
+  r.bwd.ndb = N1;
+  r.bwd.out_key = L.bwd;
+  r.bwd.q_absmax = L.status + 2;
+  r.bwd.db_absmax = L.status + 1;
+  r.cmp.S_cap = S;
+  r.cmp.fwd_key = L.fwd;
+  r.cmp.bwd_key = L.bwd;
+  r.cmp.claim = L.claim;
+  r.cmp.N1 = N1;
+  r.cmp.out_pairs = out_pairs;
+  r.cmp.out_score = out_score;
+  r.cmp.cap = capacity;
+  r.cmp.out_count = out_count;
+  r.cmp.out_iters = out_iters;
+  r.cmp.out_frontier = out_frontier;
+  r.cmp.max_iter = max_iter;
+  r.F[0] = L.F[0];
+  r.F[1] = L.F[1];
+  r.cnt[0] = L.cnt[0];
+  r.cnt[1] = L.cnt[1];
+  r.N1 = N1;
+  r.S = S;
+  r.W1 = W1;
+  r.sub = subsample;
+  r.max_iter = max_iter;
+  r.batch = batch;
+  r.grid_count = reinterpret_cast<uint32_t*>(L.status + 4);
+  r.grid_abort = L.status + 5;
+  r.status = L.status;
+  return launch_reciprocal(r, dtype, batch * N1 + kPadRows, batch * N2 + kPadRows, st);
 }
 
 int fastnn_mutual_dense(const void* desc1, int64_t n1, const void* desc2, int64_t n2, int d,

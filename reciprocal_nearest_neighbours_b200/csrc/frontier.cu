@@ -1,11 +1,12 @@
 // Memory-bound kernels around the nearest-neighbour passes:
 //   repack          descriptor rows [rows][d] -> zero-padded [rows][32 elems]
-//   seed_grid       sparse seed grid of image 1 -> round-1 frontier
-//   check_compact   reciprocal test of one round + next-frontier compaction
 //   mutual_*        dense mutual-pair test and ordered emission
 //   decode_nn       packed keys -> (index, score)
+// (The fast scheme's seeds and per-round check/compaction run inside the
+// persistent matching kernel, see frontier_dev.cuh and nn_tc.cu.)
 #include "common.cuh"
 #include "frontier.cuh"
+#include "frontier_dev.cuh"
 
 namespace fastnn {
 
@@ -60,132 +61,6 @@ __global__ void repack_kernel(const uint8_t* __restrict__ src, int64_t rows, int
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     if ((threadIdx.x & 31) == 0 && amax > 0) atomicMax(absmax, amax);
-  }
-}
-
-// ------------------------------------------------------------- seed grid ---
-// Seeds of pair b: pixels (x, y) with x = sub * (k mod gx), y = sub * (k div gx).
-// Each seed claims its pixel with stamp 0 (round 0, slot k).
-__global__ void seed_kernel(int32_t* __restrict__ F0, int64_t S_cap, uint32_t* __restrict__ claim,
-                            int64_t N1, int32_t* __restrict__ cnt0, int H1, int W1, int sub,
-                            int S) {
-  const int b = blockIdx.y;
-  const int gx = (W1 + sub - 1) / sub;
-  for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < S; k += gridDim.x * blockDim.x) {
-    const int y = (k / gx) * sub;
-    const int x = (k % gx) * sub;
-    const int u = y * W1 + x;
-    F0[b * S_cap + k] = u;
-    claim[b * N1 + u] = static_cast<uint32_t>(k);
-  }
-  if (blockIdx.x == 0 && threadIdx.x == 0) cnt0[b] = S;
-}
-
-// Block-wide exclusive scan of two 0/1 flags (warp ballots + one smem pass).
-// Returns the exclusive prefix of each flag and writes the block totals.
-struct Scan2 {
-  int ex0, ex1, tot0, tot1;
-};
-
-__device__ __forceinline__ Scan2 block_scan2(bool f0, bool f1, int* sm /* 2 * 32 ints */) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  const unsigned b0 = __ballot_sync(0xffffffffu, f0);
-  const unsigned b1 = __ballot_sync(0xffffffffu, f1);
-  const unsigned lt = (1u << lane) - 1u;
-  if (lane == 0) {
-    sm[warp] = __popc(b0);
-    sm[32 + warp] = __popc(b1);
-  }
-  __syncthreads();
-  int off0 = 0, off1 = 0, t0 = 0, t1 = 0;
-  for (int w = 0; w < nw; ++w) {
-    const int c0 = sm[w], c1 = sm[32 + w];
-    if (w < warp) {
-      off0 += c0;
-      off1 += c1;
-    }
-    t0 += c0;
-    t1 += c1;
-  }
-  __syncthreads();
-  return Scan2{off0 + __popc(b0 & lt), off1 + __popc(b1 & lt), t0, t1};
-}
-
-// --------------------------------------------------------- check+compact ---
-// One CTA per pair. Round t (1-based) of the fast scheme: slot k holds seed
-// u = F[k], its forward match v and the backward match u'. u' == u keeps
-// (u, v); otherwise u' is pushed to the next frontier if no frontier of this
-// call has held it yet: phase 1 claims u' with atomicMin on a (round, slot)
-// stamp, phase 2 lets only the claiming slot push, so duplicates within the
-// round and pixels seen in earlier rounds are dropped, deterministically.
-// Kept pairs and pushes are compacted in slot order. The round's key slots
-// are reset to 0 for the next round's atomicMax merges.
-template <int DT>
-__global__ void __launch_bounds__(1024) check_compact_kernel(CompactArgs c, int t, int last_round) {
-  __shared__ int sm[64];
-  __shared__ int base_out;
-  const int b = blockIdx.x;
-  const int cnt = c.cnt_cur[b];
-  if (cnt == 0) {
-    if (threadIdx.x == 0) c.cnt_next[b] = 0;
-    return;
-  }
-  const int32_t* F = c.F_cur + b * c.S_cap;
-  uint64_t* fwd = c.fwd_key + b * c.S_cap;
-  uint64_t* bwd = c.bwd_key + b * c.S_cap;
-  uint32_t* claim = c.claim + b * c.N1;
-  const uint32_t stamp_hi = static_cast<uint32_t>(t) << 24;
-
-  if (!last_round) {
-    for (int k = threadIdx.x; k < cnt; k += blockDim.x) {
-      const uint32_t u2 = key_index(bwd[k]);
-      if (u2 != static_cast<uint32_t>(F[k]) && u2 < static_cast<uint32_t>(c.N1))
-        atomicMin(&claim[u2], stamp_hi | static_cast<uint32_t>(k));
-    }
-  }
-  if (threadIdx.x == 0) base_out = c.out_count[b];
-  __syncthreads();
-  int out0 = base_out, next0 = 0;
-  for (int s = 0; s < cnt; s += blockDim.x) {
-    const int k = s + threadIdx.x;
-    bool conv = false, push = false;
-    uint32_t u = 0, v = 0, u2 = 0;
-    uint64_t fk = 0;
-    if (k < cnt) {
-      u = static_cast<uint32_t>(F[k]);
-      fk = fwd[k];
-      v = key_index(fk);
-      u2 = key_index(bwd[k]);
-      conv = (u2 == u);
-      push = !conv && !last_round && u2 < static_cast<uint32_t>(c.N1) &&
-             claim[u2] == (stamp_hi | static_cast<uint32_t>(k));
-      fwd[k] = 0;
-      bwd[k] = 0;
-    }
-    const Scan2 sc = block_scan2(conv, push, sm);
-    if (conv) {
-      const int64_t pos = out0 + sc.ex0;
-      if (pos < c.cap) {
-        int32_t* op = c.out_pairs + (b * c.cap + pos) * 2;
-        op[0] = static_cast<int32_t>(u);
-        op[1] = static_cast<int32_t>(v);
-        if (c.out_score) {
-          if (DT == FASTNN_I8)
-            static_cast<int32_t*>(c.out_score)[b * c.cap + pos] = unord_i32(key_score_bits(fk));
-          else
-            static_cast<float*>(c.out_score)[b * c.cap + pos] = unord_f32(key_score_bits(fk));
-        }
-      }
-    }
-    if (push) c.F_next[b * c.S_cap + next0 + sc.ex1] = static_cast<int32_t>(u2);
-    out0 += sc.tot0;
-    next0 += sc.tot1;
-  }
-  if (threadIdx.x == 0) {
-    c.out_count[b] = out0;
-    c.cnt_next[b] = next0;
-    if (c.out_iters) c.out_iters[b] = t;
-    if (c.out_frontier) c.out_frontier[b * c.max_iter + (t - 1)] = cnt;
   }
 }
 
@@ -312,24 +187,6 @@ int launch_repack(const void* src, int64_t rows, int d, int dtype, void* dst, in
     repack_kernel<2><<<grid_for(total, 256), 256, 0, st>>>(static_cast<const uint8_t*>(src), rows,
                                                             d, static_cast<uint8_t*>(dst), pad_rows,
                                                             nullptr);
-  FASTNN_CUDA_TRY(cudaGetLastError());
-  return FASTNN_OK;
-}
-
-int launch_seed(int32_t* F0, int64_t S_cap, uint32_t* claim, int64_t N1, int32_t* cnt0, int H1,
-                int W1, int sub, int S, int batch, cudaStream_t st) {
-  dim3 grid(grid_for(S, 256, 64), batch);
-  seed_kernel<<<grid, 256, 0, st>>>(F0, S_cap, claim, N1, cnt0, H1, W1, sub, S);
-  FASTNN_CUDA_TRY(cudaGetLastError());
-  return FASTNN_OK;
-}
-
-int launch_check_compact(const CompactArgs& c, int dtype, int t, bool last_round, int batch,
-                         cudaStream_t st) {
-  if (dtype == FASTNN_I8)
-    check_compact_kernel<FASTNN_I8><<<batch, 1024, 0, st>>>(c, t, last_round ? 1 : 0);
-  else
-    check_compact_kernel<FASTNN_BF16><<<batch, 1024, 0, st>>>(c, t, last_round ? 1 : 0);
   FASTNN_CUDA_TRY(cudaGetLastError());
   return FASTNN_OK;
 }

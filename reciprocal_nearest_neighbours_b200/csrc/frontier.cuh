@@ -27,10 +27,6 @@ struct CompactArgs {
 
 int launch_repack(const void* src, int64_t rows, int d, int dtype, void* dst, int64_t pad_rows,
                   int* absmax, cudaStream_t st);
-int launch_seed(int32_t* F0, int64_t S_cap, uint32_t* claim, int64_t N1, int32_t* cnt0, int H1,
-                int W1, int sub, int S, int batch, cudaStream_t st);
-int launch_check_compact(const CompactArgs& c, int dtype, int t, bool last_round, int batch,
-                         cudaStream_t st);
 int mutual_blocks(int64_t n1);
 int launch_mutual(const uint64_t* k12, const uint64_t* k21, int64_t n1, int64_t n2,
                   int32_t* block_scratch, int dtype, int32_t* out_pairs, void* out_score,

@@ -30,6 +30,7 @@
 #include <cuda.h>
 
 #include "common.cuh"
+#include "frontier_dev.cuh"
 #include "nn_tc.cuh"
 #include "ptx.cuh"
 
@@ -67,6 +68,9 @@ struct Ctl {
   uint32_t tmem_base;
   int abort_flag;
   int pack16;
+  int grid_ok;
+  int more;
+  int scan[66];  // block-scan scratch of the per-pair compaction
   int b0;
   int64_t m0, n0, u0, u1, nt;
   int mt[kMaxBatch];
@@ -336,56 +340,47 @@ __device__ __forceinline__ void fold_wide(const uint32_t (&r)[NC][32], uint32_t 
   }
 }
 
-template <int DT>
-__global__ void __launch_bounds__(kThreads, 1)
-    nn_tc_kernel(const __grid_constant__ CUtensorMap tmap_db, NNArgs a) {
-  constexpr int RB = row_bytes(DT);
-  using E = Epi<DT>;
+// ---- pipeline set-up, phases and teardown --------------------------------
+// A "phase" is one nearest-neighbour pass over a work list. The standalone
+// kernel runs one phase; the persistent fast-matching kernel runs two per
+// round. Barrier phases, ring positions and the TMEM allocation carry over
+// from phase to phase, so a phase costs no set-up.
+
+struct SmemLayout {
+  uint8_t* tileA;  // 2 x kBM x RB query tiles
+  uint8_t* tileB;  // kStages x kBN x RB database tiles
+  Ctl* ctl;
+  uint4* stash;    // 32 B per epilogue thread
+};
+
+template <int RB>
+__device__ __forceinline__ SmemLayout smem_layout() {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* tileA = smem;                          // 2 x kBM x RB
-  uint8_t* tileB = tileA + 2 * tile_bytes_a(RB);  // kStages x kBN x RB
-  Ctl* ctl = reinterpret_cast<Ctl*>(tileB + kStages * tile_bytes_b(RB));
-  uint4* stash = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(ctl) + ctl_bytes());
+  SmemLayout L;
+  L.tileA = base;
+  L.tileB = base + 2 * tile_bytes_a(RB);
+  L.ctl = reinterpret_cast<Ctl*>(L.tileB + kStages * tile_bytes_b(RB));
+  L.stash = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(L.ctl) + ctl_bytes());
+  return L;
+}
 
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int batch = a.batch;
+// Per-thread pipeline state that persists across phases (each role uses its
+// own fields).
+struct PipeState {
+  Ring st;                  // producer, MMA: database stage ring
+  Ring ac;                  // MMA: accumulator ring
+  int64_t seg = 0;          // producer, MMA: segments started (query-tile buffer)
+  int last_phase[kStages];  // producer lane 0: phase bit of the last load per stage
+  uint32_t ephase = 0;      // epilogue: phase bit of its accumulator barrier
+  int epar = 0;             // epilogue: parity of the running unit index
+};
 
-  // ---- work range of this CTA (thread 0), barrier init --------------------
+// Barrier init and TMEM allocation; ends with a CTA barrier.
+__device__ __forceinline__ void pipe_setup(Ctl* ctl) {
   if (threadIdx.x == 0) {
-    const int64_t nt = (a.ndb + kBN - 1) / kBN;
-    int64_t total = 0;
-    for (int b = 0; b < batch; ++b) {
-      const int64_t c = nn_count(a, b);
-      ctl->cnt[b] = static_cast<int>(c);
-      ctl->mt[b] = static_cast<int>((c + kBM - 1) / kBM);
-      total += static_cast<int64_t>(ctl->mt[b]) * nt;
-    }
-    const int64_t G = gridDim.x;
-    const int64_t u0 = total * blockIdx.x / G;
-    const int64_t u1 = total * (blockIdx.x + 1) / G;
-    ctl->nt = nt;
-    ctl->u0 = u0;
-    ctl->u1 = u1;
     ctl->abort_flag = 0;
-    // int8 scores fit in 16 bits when d * max|q| * max|db| < 2^15; the repack
-    // pass measured both maxima.
-    ctl->pack16 = (DT == FASTNN_I8 && a.q_absmax && a.db_absmax &&
-                   static_cast<int64_t>(*a.q_absmax) * (*a.db_absmax) * a.d <= 32767)
-                      ? 1
-                      : 0;
-    int64_t acc = 0;
-    int b = 0;
-    while (b < batch && acc + static_cast<int64_t>(ctl->mt[b]) * nt <= u0) {
-      acc += static_cast<int64_t>(ctl->mt[b]) * nt;
-      ++b;
-    }
-    ctl->b0 = b;
-    const int64_t rem = u0 - acc;
-    ctl->m0 = nt > 0 ? rem / nt : 0;
-    ctl->n0 = nt > 0 ? rem % nt : 0;
     for (int i = 0; i < kNumBars; ++i) {
       uint32_t count = 1;
       if (i >= kBarAFull && i < kBarAFull + 2) count = 32;  // producer lanes
@@ -394,205 +389,392 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     ptx::fence_mbar_init();
   }
-  __syncthreads();
-  const int64_t u0 = ctl->u0, u1 = ctl->u1;
-  if (u0 >= u1) return;  // uniform over the CTA: nothing was allocated yet
-
-  if (warp == 0) {
+  if ((threadIdx.x >> 5) == 0) {
     ptx::tmem_alloc(ptx::smem_u32(&ctl->tmem_base), 512);
     ptx::tmem_relinquish();
   }
-  if (warp == kProducerWarp && lane == 0) ptx::prefetch_tmap(&tmap_db);
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
-  const uint32_t tmem = ctl->tmem_base;
+}
 
+// Work list of this CTA for one phase (thread 0).
+template <int DT>
+__device__ void plan_phase(const NNArgs& a, Ctl* ctl) {
+  const int batch = a.batch;
+  const int64_t nt = (a.ndb + kBN - 1) / kBN;
+  int64_t total = 0;
+  for (int b = 0; b < batch; ++b) {
+    const int64_t c = nn_count(a, b);
+    ctl->cnt[b] = static_cast<int>(c);
+    ctl->mt[b] = static_cast<int>((c + kBM - 1) / kBM);
+    total += static_cast<int64_t>(ctl->mt[b]) * nt;
+  }
+  const int64_t G = gridDim.x;
+  const int64_t u0 = total * blockIdx.x / G;
+  const int64_t u1 = total * (blockIdx.x + 1) / G;
+  ctl->nt = nt;
+  ctl->u0 = u0;
+  ctl->u1 = u1;
+  // int8 scores fit in 16 bits when d * max|q| * max|db| < 2^15; the repack
+  // pass measured both maxima.
+  ctl->pack16 = (DT == FASTNN_I8 && a.q_absmax && a.db_absmax &&
+                 static_cast<int64_t>(__ldcg(a.q_absmax)) * __ldcg(a.db_absmax) * a.d <= 32767)
+                    ? 1
+                    : 0;
+  int64_t acc = 0;
+  int b = 0;
+  while (b < batch && acc + static_cast<int64_t>(ctl->mt[b]) * nt <= u0) {
+    acc += static_cast<int64_t>(ctl->mt[b]) * nt;
+    ++b;
+  }
+  ctl->b0 = b;
+  const int64_t rem = u0 - acc;
+  ctl->m0 = nt > 0 ? rem / nt : 0;
+  ctl->n0 = nt > 0 ? rem % nt : 0;
+}
+
+// One nearest-neighbour phase: plan (thread 0), then each role runs its loop
+// over this CTA's units. Ends with a CTA barrier, after which every MMA of the
+// phase has completed and every result has been merged into a.out_key.
+template <int DT>
+__device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const SmemLayout& L,
+                          uint32_t tmem, PipeState& ps) {
+  constexpr int RB = row_bytes(DT);
+  using E = Epi<DT>;
+  Ctl* ctl = L.ctl;
+  uint8_t* tileA = L.tileA;
+  uint8_t* tileB = L.tileB;
+  if (threadIdx.x == 0) plan_phase<DT>(a, ctl);
+  __syncthreads();
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int batch = a.batch;
+  const int64_t u0 = ctl->u0, u1 = ctl->u1;
   auto bar = [&](int i) { return ptx::smem_u32(&ctl->bars[i]); };
   const Pos start{ctl->b0, ctl->m0, ctl->n0};
   const int64_t nt = ctl->nt;
 
-  if (warp == kProducerWarp) {
-    // ---------------------------------------------------------------- producer
-    Pos p = start;
-    Ring st;            // database stage ring
-    int64_t seg = 0;
-    int last_phase[kStages];  // phase bit of the last load issued into each stage, or -1
-#pragma unroll
-    for (int s = 0; s < kStages; ++s) last_phase[s] = -1;
-    bool ok = true;
-    for (int64_t u = u0; ok && u < u1; ++seg) {
-      const int64_t len = seg_len(p, u, u1, nt);
-      const int as = static_cast<int>(seg & 1);
-      if (!warp_wait_bounded(bar(kBarAEmpty + as), static_cast<uint32_t>(((seg >> 1) & 1) ^ 1),
-                             ctl, a.status))
-        break;
-      gather_a<RB>(tileA + as * tile_bytes_a(RB), a, p.b, p.m, ctl->cnt[p.b], lane);
-      ptx::fence_proxy_async_smem();
-      ptx::mbar_arrive(bar(kBarAFull + as));
-      if (lane == 0) {
-        int32_t row = static_cast<int32_t>(static_cast<int64_t>(p.b) * a.ndb + p.n * kBN);
-        for (int64_t j = 0; j < len; ++j, row += kBN) {
-          if (!wait_bounded(bar(kBarBEmpty + st.idx), st.phase ^ 1u, ctl, a.status)) {
-            ok = false;
-            break;
-          }
-          ptx::mbar_arrive_expect_tx(bar(kBarBFull + st.idx), static_cast<uint32_t>(tile_bytes_b(RB)));
-          ptx::tma_load_2d(ptx::smem_u32(tileB + st.idx * tile_bytes_b(RB)), &tmap_db, 0, row,
-                           bar(kBarBFull + st.idx));
-          last_phase[st.idx] = static_cast<int>(st.phase);
-          st.next<kStages>();
-        }
-      }
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-      u += len;
-      next_segment(p, ctl, batch);
-    }
-    // Drain: every TMA load this warp issued must land before smem is freed.
-    if (lane == 0) {
-      for (int s = 0; s < kStages; ++s)
-        if (last_phase[s] >= 0)
-          wait_bounded(bar(kBarBFull + s), static_cast<uint32_t>(last_phase[s]), ctl, a.status);
-    }
-  } else if (warp == kMmaWarp) {
-    // --------------------------------------------------------------- MMA issue
-    if (lane == 0) {
-      constexpr uint32_t kIdesc =
-          DT == FASTNN_I8
-              ? ((2u << 4) | (1u << 7) | (1u << 10) | ((kBN >> 3) << 17) | ((kBM >> 4) << 24))
-              : ((1u << 4) | (1u << 7) | (1u << 10) | ((kBN >> 3) << 17) | ((kBM >> 4) << 24));
+  if (u0 < u1 && !ctl->abort_flag) {
+    if (warp == kProducerWarp) {
+      // -------------------------------------------------------------- producer
       Pos p = start;
-      Ring st, ac;  // database stage ring, accumulator ring
-      int64_t seg = 0;
       bool ok = true;
-      for (int64_t u = u0; ok && u < u1; ++seg) {
+      for (int64_t u = u0; ok && u < u1; ++ps.seg) {
         const int64_t len = seg_len(p, u, u1, nt);
-        const int as = static_cast<int>(seg & 1);
-        if (!wait_bounded(bar(kBarAFull + as), static_cast<uint32_t>((seg >> 1) & 1), ctl,
-                          a.status))
+        const int as = static_cast<int>(ps.seg & 1);
+        if (!warp_wait_bounded(bar(kBarAEmpty + as),
+                               static_cast<uint32_t>(((ps.seg >> 1) & 1) ^ 1), ctl, a.status))
           break;
-        ptx::tc_fence_after();
-        const uint64_t adesc =
-            ptx::smem_desc_kmajor(ptx::smem_u32(tileA + as * tile_bytes_a(RB)), RB);
-        const uint64_t bdesc0 = ptx::smem_desc_kmajor(ptx::smem_u32(tileB), RB);
-        for (int64_t j = 0; j < len; ++j) {
-          if (!wait_bounded(bar(kBarAccEmpty + ac.idx), ac.phase ^ 1u, ctl, a.status) ||
-              !wait_bounded(bar(kBarBFull + st.idx), st.phase, ctl, a.status)) {
-            ok = false;
-            break;
+        gather_a<RB>(tileA + as * tile_bytes_a(RB), a, p.b, p.m, ctl->cnt[p.b], lane);
+        ptx::fence_proxy_async_smem();
+        ptx::mbar_arrive(bar(kBarAFull + as));
+        if (lane == 0) {
+          int32_t row = static_cast<int32_t>(static_cast<int64_t>(p.b) * a.ndb + p.n * kBN);
+          for (int64_t j = 0; j < len; ++j, row += kBN) {
+            if (!wait_bounded(bar(kBarBEmpty + ps.st.idx), ps.st.phase ^ 1u, ctl, a.status)) {
+              ok = false;
+              break;
+            }
+            ptx::mbar_arrive_expect_tx(bar(kBarBFull + ps.st.idx),
+                                       static_cast<uint32_t>(tile_bytes_b(RB)));
+            ptx::tma_load_2d(ptx::smem_u32(tileB + ps.st.idx * tile_bytes_b(RB)), tmap_db, 0, row,
+                             bar(kBarBFull + ps.st.idx));
+            ps.last_phase[ps.st.idx] = static_cast<int>(ps.st.phase);
+            ps.st.next<kStages>();
           }
-          ptx::tc_fence_after();
-          const uint32_t d_tmem = tmem + static_cast<uint32_t>(ac.idx * kBN);
-          const uint64_t bdesc = bdesc0 + static_cast<uint64_t>((st.idx * tile_bytes_b(RB)) >> 4);
-          if constexpr (DT == FASTNN_I8) {
-            ptx::mma_i8(d_tmem, adesc, bdesc, kIdesc, 0u);
-          } else {
-            // K = 32 bf16 = two K = 16 steps; the second starts 32 bytes in.
-            ptx::mma_bf16(d_tmem, adesc, bdesc, kIdesc, 0u);
-            ptx::mma_bf16(d_tmem, adesc + 2, bdesc + 2, kIdesc, 1u);
-          }
-          ptx::mma_commit(bar(kBarBEmpty + st.idx));
-          ptx::mma_commit(bar(kBarAccFull + ac.idx));
-          st.next<kStages>();
-          ac.next<kAcc>();
         }
-        if (!ok) break;
-        ptx::mma_commit(bar(kBarAEmpty + as));
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         u += len;
         next_segment(p, ctl, batch);
       }
-      // Every MMA issued above completes before TMEM is released.
-      ptx::mma_commit(bar(kBarDone));
-      wait_bounded(bar(kBarDone), 0, ctl, a.status);
-    }
-  } else {
-    // ---------------------------------------------------------------- epilogue
-    // Group g folds the units whose running index is congruent to g mod 2,
-    // i.e. the ones the MMA wrote into accumulator g.
-    const int grp = warp / kGroupWarps;
-    const int gw = warp % kGroupWarps;
-    const int lg = gw & 3;   // TMEM lane quarter (warp id mod 4)
-    const int h = gw >> 2;   // column half of the tile
-    const bool pack16 = ctl->pack16 != 0;
-    const int tail = static_cast<int>(a.ndb - (nt - 1) * kBN);  // valid columns, last tile
-    const uint32_t acc_bar = bar(kBarAccFull + grp);
-    const uint32_t rel_bar = bar(kBarAccEmpty + grp);
-    const uint32_t taddr = tmem + (static_cast<uint32_t>(lg * 32) << 16) +
-                           static_cast<uint32_t>(grp * kBN + h * kEpiCols);
-    uint4* slot = stash + 2 * threadIdx.x;
-    Pos p = start;
-    int64_t it = 0;        // running unit index at the start of the segment
-    uint32_t phase = 0;    // phase bit of this group's accumulator barrier
-    bool ok = true;
-    for (int64_t u = u0; ok && u < u1;) {
-      const int64_t len = seg_len(p, u, u1, nt);
-      typename E::S best = E::lowest();
-      uint32_t bidx = 0xFFFFFFFFu;
-      for (int64_t j = ((grp - it) & 1); j < len; j += kAcc) {
-        if (!warp_wait_bounded(acc_bar, phase, ctl, a.status)) {
-          ok = false;
-          break;
-        }
-        phase ^= 1u;
-        ptx::tc_fence_after();
-        const int64_t n = p.n + j;
-        const uint32_t colbase = static_cast<uint32_t>(n * kBN + h * kEpiCols);
-        if (n == nt - 1 && tail < kBN) {
-          // Ragged last tile of the database: column-masked fold.
-          const int valid_blk = tail - h * kEpiCols;
-#pragma unroll 1
-          for (int c = 0; c < kChunks; ++c) {
-            uint32_t r[32];
-            ptx::tmem_ld32(taddr + c * 32, r);
-            ptx::tmem_ld_wait();
-            const int valid = min(32, max(0, valid_blk - c * 32));
-            fold32_masked<DT>(r, colbase + c * 32, valid, best, bidx);
+      // Ring positions are per lane; lane 0 advanced the shared ring.
+      ps.st.idx = __shfl_sync(0xffffffffu, ps.st.idx, 0);
+      ps.st.phase = __shfl_sync(0xffffffffu, ps.st.phase, 0);
+    } else if (warp == kMmaWarp) {
+      // ------------------------------------------------------------- MMA issue
+      if (lane == 0) {
+        constexpr uint32_t kIdesc =
+            DT == FASTNN_I8
+                ? ((2u << 4) | (1u << 7) | (1u << 10) | ((kBN >> 3) << 17) | ((kBM >> 4) << 24))
+                : ((1u << 4) | (1u << 7) | (1u << 10) | ((kBN >> 3) << 17) | ((kBM >> 4) << 24));
+        Pos p = start;
+        bool ok = true;
+        for (int64_t u = u0; ok && u < u1; ++ps.seg) {
+          const int64_t len = seg_len(p, u, u1, nt);
+          const int as = static_cast<int>(ps.seg & 1);
+          if (!wait_bounded(bar(kBarAFull + as), static_cast<uint32_t>((ps.seg >> 1) & 1), ctl,
+                            a.status))
+            break;
+          ptx::tc_fence_after();
+          const uint64_t adesc =
+              ptx::smem_desc_kmajor(ptx::smem_u32(tileA + as * tile_bytes_a(RB)), RB);
+          const uint64_t bdesc0 = ptx::smem_desc_kmajor(ptx::smem_u32(tileB), RB);
+          for (int64_t j = 0; j < len; ++j) {
+            if (!wait_bounded(bar(kBarAccEmpty + ps.ac.idx), ps.ac.phase ^ 1u, ctl, a.status) ||
+                !wait_bounded(bar(kBarBFull + ps.st.idx), ps.st.phase, ctl, a.status)) {
+              ok = false;
+              break;
+            }
+            ptx::tc_fence_after();
+            const uint32_t d_tmem = tmem + static_cast<uint32_t>(ps.ac.idx * kBN);
+            const uint64_t bdesc =
+                bdesc0 + static_cast<uint64_t>((ps.st.idx * tile_bytes_b(RB)) >> 4);
+            if constexpr (DT == FASTNN_I8) {
+              ptx::mma_i8(d_tmem, adesc, bdesc, kIdesc, 0u);
+            } else {
+              // K = 32 bf16 = two K = 16 steps; the second starts 32 bytes in.
+              ptx::mma_bf16(d_tmem, adesc, bdesc, kIdesc, 0u);
+              ptx::mma_bf16(d_tmem, adesc + 2, bdesc + 2, kIdesc, 1u);
+            }
+            ptx::mma_commit(bar(kBarBEmpty + ps.st.idx));
+            ptx::mma_commit(bar(kBarAccFull + ps.ac.idx));
+            ps.st.next<kStages>();
+            ps.ac.next<kAcc>();
           }
-          ptx::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(rel_bar);
-        } else if (DT == FASTNN_I8 && pack16) {
-          uint32_t r[kChunks][16];
-#pragma unroll
-          for (int c = 0; c < kChunks; ++c) ptx::tmem_ld16_pack(taddr + c * 32, r[c]);
-          ptx::tmem_ld_wait();
-          // The accumulator is free for the next MMA once it is in registers.
-          ptx::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(rel_bar);
-          if constexpr (DT == FASTNN_I8) fold_pack16<kChunks>(r, colbase, best, bidx, slot);
-        } else {
-          // 32-bit scores: two 64-column halves, the accumulator is released
-          // after the second load.
-          uint32_t r[2][32];
-          ptx::tmem_ld32(taddr, r[0]);
-          ptx::tmem_ld32(taddr + 32, r[1]);
-          ptx::tmem_ld_wait();
-          fold_wide<DT, 2>(r, colbase, best, bidx, slot);
-          ptx::tmem_ld32(taddr + 64, r[0]);
-          ptx::tmem_ld32(taddr + 96, r[1]);
-          ptx::tmem_ld_wait();
-          ptx::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(rel_bar);
-          fold_wide<DT, 2>(r, colbase + 64, best, bidx, slot);
+          if (!ok) break;
+          ptx::mma_commit(bar(kBarAEmpty + as));
+          u += len;
+          next_segment(p, ctl, batch);
         }
       }
-      if (!ok) break;
-      const int64_t k = p.m * kBM + lg * 32 + lane;
-      if (k < ctl->cnt[p.b] && bidx != 0xFFFFFFFFu)
-        atomicMax(reinterpret_cast<unsigned long long*>(&a.out_key[p.b * a.q_cap + k]),
-                  static_cast<unsigned long long>(make_key(E::ord(best), bidx)));
-      u += len;
-      it += len;
-      next_segment(p, ctl, batch);
+    } else {
+      // -------------------------------------------------------------- epilogue
+      // Group g folds the units whose running index is congruent to g mod 2,
+      // i.e. the ones the MMA wrote into accumulator g.
+      const int grp = warp / kGroupWarps;
+      const int gw = warp % kGroupWarps;
+      const int lg = gw & 3;  // TMEM lane quarter (warp id mod 4)
+      const int h = gw >> 2;  // column half of the tile
+      const bool pack16 = ctl->pack16 != 0;
+      const int tail = static_cast<int>(a.ndb - (nt - 1) * kBN);  // valid columns, last tile
+      const uint32_t acc_bar = bar(kBarAccFull + grp);
+      const uint32_t rel_bar = bar(kBarAccEmpty + grp);
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(lg * 32) << 16) +
+                             static_cast<uint32_t>(grp * kBN + h * kEpiCols);
+      uint4* slot = L.stash + 2 * threadIdx.x;
+      Pos p = start;
+      bool ok = true;
+      for (int64_t u = u0; ok && u < u1;) {
+        const int64_t len = seg_len(p, u, u1, nt);
+        typename E::S best = E::lowest();
+        uint32_t bidx = 0xFFFFFFFFu;
+        for (int64_t j = ((grp - ps.epar) & 1); j < len; j += kAcc) {
+          if (!warp_wait_bounded(acc_bar, ps.ephase, ctl, a.status)) {
+            ok = false;
+            break;
+          }
+          ps.ephase ^= 1u;
+          ptx::tc_fence_after();
+          const int64_t n = p.n + j;
+          const uint32_t colbase = static_cast<uint32_t>(n * kBN + h * kEpiCols);
+          if (n == nt - 1 && tail < kBN) {
+            // Ragged last tile of the database: column-masked fold.
+            const int valid_blk = tail - h * kEpiCols;
+#pragma unroll 1
+            for (int c = 0; c < kChunks; ++c) {
+              uint32_t r[32];
+              ptx::tmem_ld32(taddr + c * 32, r);
+              ptx::tmem_ld_wait();
+              const int valid = min(32, max(0, valid_blk - c * 32));
+              fold32_masked<DT>(r, colbase + c * 32, valid, best, bidx);
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(rel_bar);
+          } else if (DT == FASTNN_I8 && pack16) {
+            uint32_t r[kChunks][16];
+#pragma unroll
+            for (int c = 0; c < kChunks; ++c) ptx::tmem_ld16_pack(taddr + c * 32, r[c]);
+            ptx::tmem_ld_wait();
+            // The accumulator is free for the next MMA once it is in registers.
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(rel_bar);
+            if constexpr (DT == FASTNN_I8) fold_pack16<kChunks>(r, colbase, best, bidx, slot);
+          } else {
+            // 32-bit scores: two 64-column halves, the accumulator is released
+            // after the second load.
+            uint32_t r[2][32];
+            ptx::tmem_ld32(taddr, r[0]);
+            ptx::tmem_ld32(taddr + 32, r[1]);
+            ptx::tmem_ld_wait();
+            fold_wide<DT, 2>(r, colbase, best, bidx, slot);
+            ptx::tmem_ld32(taddr + 64, r[0]);
+            ptx::tmem_ld32(taddr + 96, r[1]);
+            ptx::tmem_ld_wait();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(rel_bar);
+            fold_wide<DT, 2>(r, colbase + 64, best, bidx, slot);
+          }
+        }
+        if (!ok) break;
+        const int64_t k = p.m * kBM + lg * 32 + lane;
+        if (k < ctl->cnt[p.b] && bidx != 0xFFFFFFFFu)
+          atomicMax(reinterpret_cast<unsigned long long*>(&a.out_key[p.b * a.q_cap + k]),
+                    static_cast<unsigned long long>(make_key(E::ord(best), bidx)));
+        u += len;
+        ps.epar ^= static_cast<int>(len & 1);
+        next_segment(p, ctl, batch);
+      }
     }
   }
+  __syncthreads();
+}
 
+// Drain (every issued MMA and TMA load completes) and release TMEM.
+__device__ __forceinline__ void pipe_teardown(Ctl* ctl, uint32_t tmem, PipeState& ps,
+                                              int* status) {
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  auto bar = [&](int i) { return ptx::smem_u32(&ctl->bars[i]); };
+  if (warp == kMmaWarp && lane == 0) {
+    ptx::mma_commit(bar(kBarDone));
+    wait_bounded(bar(kBarDone), 0, ctl, status);
+  }
+  if (warp == kProducerWarp && lane == 0) {
+    for (int s = 0; s < kStages; ++s)
+      if (ps.last_phase[s] >= 0)
+        wait_bounded(bar(kBarBFull + s), static_cast<uint32_t>(ps.last_phase[s]), ctl, status);
+  }
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
   if (warp == 0) ptx::tmem_dealloc(tmem, 512);
+}
+
+template <int DT>
+__global__ void __launch_bounds__(kThreads, 1)
+    nn_tc_kernel(const __grid_constant__ CUtensorMap tmap_db, NNArgs a) {
+  constexpr int RB = row_bytes(DT);
+  const SmemLayout L = smem_layout<RB>();
+  if ((threadIdx.x >> 5) == kProducerWarp && (threadIdx.x & 31) == 0) ptx::prefetch_tmap(&tmap_db);
+  pipe_setup(L.ctl);
+  const uint32_t tmem = L.ctl->tmem_base;
+  PipeState ps;
+#pragma unroll
+  for (int s = 0; s < kStages; ++s) ps.last_phase[s] = -1;
+  run_phase<DT>(&tmap_db, a, L, tmem, ps);
+  pipe_teardown(L.ctl, tmem, ps, a.status);
+}
+
+// ---- persistent fast reciprocal matching ----------------------------------
+
+// Grid-wide barrier over co-resident CTAs (cooperative launch): a monotonic
+// arrival counter; every CTA waits (bounded) until it reaches the next
+// multiple of the grid size. A CTA that aborted, or a wait that ran out, sets
+// the shared abort word so that every CTA leaves the round loop. Returns the
+// CTA-uniform verdict.
+__device__ bool grid_sync(const RecArgs& r, uint32_t& target, Ctl* ctl) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    target += gridDim.x;
+    bool ok = !ctl->abort_flag;
+    if (!ok) atomicExch(r.grid_abort, 1);
+    __threadfence();
+    atomicAdd(r.grid_count, 1u);
+    const uint64_t t0 = ptx::globaltimer_ns();
+    for (uint32_t n = 1;; ++n) {
+      if (*reinterpret_cast<volatile uint32_t*>(r.grid_count) >= target) break;
+      if ((n & 63) == 0) {
+        if (*reinterpret_cast<volatile int*>(r.grid_abort)) {
+          ok = false;
+          break;
+        }
+        if (ptx::globaltimer_ns() - t0 > kTimeoutNs) {
+          atomicOr(r.status, kStatusTimeout);
+          atomicExch(r.grid_abort, 1);
+          ok = false;
+          break;
+        }
+      }
+    }
+    __threadfence();
+    if (*reinterpret_cast<volatile int*>(r.grid_abort)) ok = false;
+    ctl->grid_ok = ok ? 1 : 0;
+  }
+  __syncthreads();
+  return ctl->grid_ok != 0;
+}
+
+// MASt3R fast reciprocal matching of `batch` pairs in one launch: clear the
+// per-call state, seed the grid, then per round a forward pass (image 1 -> 2),
+// a backward pass (matches -> image 1) and the per-pair check/compaction,
+// separated by grid barriers; stops when every pair's frontier is empty or
+// after max_iter rounds.
+template <int DT>
+__global__ void __launch_bounds__(kThreads, 1)
+    reciprocal_kernel(const __grid_constant__ CUtensorMap tmap_d2,
+                      const __grid_constant__ CUtensorMap tmap_d1, RecArgs r) {
+  constexpr int RB = row_bytes(DT);
+  const SmemLayout L = smem_layout<RB>();
+  Ctl* ctl = L.ctl;
+  if ((threadIdx.x >> 5) == kProducerWarp && (threadIdx.x & 31) == 0) {
+    ptx::prefetch_tmap(&tmap_d1);
+    ptx::prefetch_tmap(&tmap_d2);
+  }
+  pipe_setup(ctl);
+  const uint32_t tmem = ctl->tmem_base;
+  PipeState ps;
+#pragma unroll
+  for (int s = 0; s < kStages; ++s) ps.last_phase[s] = -1;
+  uint32_t target = 0;
+  const int batch = r.batch;
+  const int64_t S = r.S;
+  const int64_t gtid = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  const int64_t gsize = static_cast<int64_t>(gridDim.x) * blockDim.x;
+
+  // Clear per-call state: keys, first-visit claims, outputs.
+  for (int64_t i = gtid; i < batch * S; i += gsize) {
+    r.cmp.fwd_key[i] = 0;
+    r.cmp.bwd_key[i] = 0;
+  }
+  for (int64_t i = gtid; i < batch * r.N1; i += gsize) r.cmp.claim[i] = 0xFFFFFFFFu;
+  for (int64_t i = gtid; i < batch; i += gsize) {
+    r.cmp.out_count[i] = 0;
+    if (r.cmp.out_iters) r.cmp.out_iters[i] = 0;
+  }
+  if (r.cmp.out_frontier)
+    for (int64_t i = gtid; i < batch * r.max_iter; i += gsize) r.cmp.out_frontier[i] = 0;
+  bool ok = grid_sync(r, target, ctl);
+  if (ok) {
+    // Seeds: the round-1 frontier of every pair.
+    for (int64_t i = gtid; i < batch * S; i += gsize)
+      seed_one(r.F[0], S, r.cmp.claim, r.N1, r.W1, r.sub, static_cast<int>(i / S),
+               static_cast<int>(i % S));
+    for (int64_t i = gtid; i < batch; i += gsize) r.cnt[0][i] = static_cast<int>(S);
+    ok = grid_sync(r, target, ctl);
+  }
+  for (int t = 1; ok && t <= r.max_iter; ++t) {
+    const int cur = (t - 1) & 1, nxt = t & 1;
+    NNArgs f = r.fwd;
+    f.q_index = r.F[cur];
+    f.q_count = r.cnt[cur];
+    run_phase<DT>(&tmap_d2, f, L, tmem, ps);
+    if (!grid_sync(r, target, ctl)) break;
+    NNArgs bw = r.bwd;
+    bw.q_count = r.cnt[cur];
+    run_phase<DT>(&tmap_d1, bw, L, tmem, ps);
+    if (!grid_sync(r, target, ctl)) break;
+    CompactArgs c = r.cmp;
+    c.F_cur = r.F[cur];
+    c.F_next = r.F[nxt];
+    c.cnt_cur = r.cnt[cur];
+    c.cnt_next = r.cnt[nxt];
+    for (int b = blockIdx.x; b < batch; b += gridDim.x)
+      compact_pair<DT>(c, b, t, t == r.max_iter, ctl->scan);
+    if (!grid_sync(r, target, ctl)) break;
+    // Every CTA reads the same counts after the barrier: a uniform exit.
+    if (threadIdx.x == 0) {
+      int any = 0;
+      for (int b = 0; b < batch; ++b) any |= __ldcg(r.cnt[nxt] + b);
+      ctl->more = any != 0 ? 1 : 0;
+    }
+    __syncthreads();
+    if (!ctl->more) break;
+  }
+  pipe_teardown(ctl, tmem, ps, r.status);
 }
 
 using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -661,28 +843,53 @@ int kernel_timer_read(int* launches, double* total_ms) {
 int nn_tc_min_rows() { return kBN; }
 int nn_tc_max_batch() { return kMaxBatch; }
 
-int launch_nn_tc(const NNArgs& a, int dtype, int64_t db_total_rows, cudaStream_t stream) {
-  const int rb = row_bytes(dtype);
-  if (db_total_rows < kBN || a.batch < 1 || a.batch > kMaxBatch) return FASTNN_ERR_INVALID;
+namespace {
+
+int make_tmap(CUtensorMap* tm, const uint8_t* rows, int64_t total_rows, int rb) {
   EncodeFn encode = get_encode();
   if (!encode) return FASTNN_ERR_CUDA;
-  CUtensorMap tm;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(rb), static_cast<cuuint64_t>(db_total_rows)};
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(rb), static_cast<cuuint64_t>(total_rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(rb)};
   const cuuint32_t box[2] = {static_cast<cuuint32_t>(rb), static_cast<cuuint32_t>(kBN)};
   const cuuint32_t estr[2] = {1, 1};
-  CUresult r = encode(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a.db_rows), dims,
-                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                      rb == 32 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B,
-                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return FASTNN_ERR_INVALID;
+  const CUresult r = encode(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(rows), dims,
+                            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            rb == 32 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FASTNN_OK : FASTNN_ERR_INVALID;
+}
 
-  int dev = 0, sms = 0;
+int sm_count(int* sms) {
+  int dev = 0;
   FASTNN_CUDA_TRY(cudaGetDevice(&dev));
-  FASTNN_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-  const size_t smem = smem_bytes(rb);
+  FASTNN_CUDA_TRY(cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev));
+  return FASTNN_OK;
+}
+
+int timer_begin(cudaStream_t stream) {
   const int slot = (g_timer.ev && g_timer.used < g_timer.cap) ? g_timer.used++ : -1;
-  if (slot >= 0) FASTNN_CUDA_TRY(cudaEventRecord(g_timer.ev[2 * slot], stream));
+  if (slot >= 0 && cudaEventRecord(g_timer.ev[2 * slot], stream) != cudaSuccess) return -2;
+  return slot;
+}
+
+int timer_end(int slot, cudaStream_t stream) {
+  if (slot >= 0) FASTNN_CUDA_TRY(cudaEventRecord(g_timer.ev[2 * slot + 1], stream));
+  return FASTNN_OK;
+}
+
+}  // namespace
+
+int launch_nn_tc(const NNArgs& a, int dtype, int64_t db_total_rows, cudaStream_t stream) {
+  const int rb = row_bytes(dtype);
+  if (db_total_rows < kBN || a.batch < 1 || a.batch > kMaxBatch) return FASTNN_ERR_INVALID;
+  CUtensorMap tm;
+  int rc = make_tmap(&tm, a.db_rows, db_total_rows, rb);
+  if (rc != FASTNN_OK) return rc;
+  int sms = 0;
+  if ((rc = sm_count(&sms)) != FASTNN_OK) return rc;
+  const size_t smem = smem_bytes(rb);
+  const int slot = timer_begin(stream);
+  if (slot == -2) return FASTNN_ERR_CUDA;
   if (dtype == FASTNN_I8) {
     FASTNN_CUDA_TRY(cudaFuncSetAttribute(nn_tc_kernel<FASTNN_I8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -695,8 +902,34 @@ int launch_nn_tc(const NNArgs& a, int dtype, int64_t db_total_rows, cudaStream_t
     nn_tc_kernel<FASTNN_BF16><<<sms, kThreads, smem, stream>>>(tm, a);
   }
   FASTNN_CUDA_TRY(cudaGetLastError());
-  if (slot >= 0) FASTNN_CUDA_TRY(cudaEventRecord(g_timer.ev[2 * slot + 1], stream));
-  return FASTNN_OK;
+  return timer_end(slot, stream);
+}
+
+int launch_reciprocal(const RecArgs& r, int dtype, int64_t d1_rows, int64_t d2_rows,
+                      cudaStream_t stream) {
+  const int rb = row_bytes(dtype);
+  if (d1_rows < kBN || d2_rows < kBN || r.batch < 1 || r.batch > kMaxBatch)
+    return FASTNN_ERR_INVALID;
+  CUtensorMap tm2, tm1;
+  int rc = make_tmap(&tm2, r.fwd.db_rows, d2_rows, rb);
+  if (rc != FASTNN_OK) return rc;
+  if ((rc = make_tmap(&tm1, r.bwd.db_rows, d1_rows, rb)) != FASTNN_OK) return rc;
+  int sms = 0;
+  if ((rc = sm_count(&sms)) != FASTNN_OK) return rc;
+  const size_t smem = smem_bytes(rb);
+  const void* fn = dtype == FASTNN_I8 ? reinterpret_cast<const void*>(reciprocal_kernel<FASTNN_I8>)
+                                      : reinterpret_cast<const void*>(reciprocal_kernel<FASTNN_BF16>);
+  FASTNN_CUDA_TRY(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem)));
+  int per_sm = 0;
+  FASTNN_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, smem));
+  if (per_sm < 1) return FASTNN_ERR_UNSUPPORTED;
+  RecArgs args = r;
+  void* params[] = {&tm2, &tm1, &args};
+  const int slot = timer_begin(stream);
+  if (slot == -2) return FASTNN_ERR_CUDA;
+  FASTNN_CUDA_TRY(cudaLaunchCooperativeKernel(fn, dim3(sms), dim3(kThreads), params, smem, stream));
+  return timer_end(slot, stream);
 }
 
 }  // namespace fastnn
