@@ -128,6 +128,36 @@ int fastnn_mutual_dense(const void *desc1, int64_t n1, const void *desc2,
                         fastnn_stream_t stream);
 
 /*
+ * fastnn_reciprocal_noalloc -- fastnn_reciprocal for callers that cannot
+ * allocate device memory (a plugin inside an application that owns every
+ * allocation, a real-time loop that must not take cudaMalloc's implicit
+ * synchronisation, a fixed pre-reserved memory budget). The pages describe no
+ * such entry point: it is a property of this library, with no counterpart in
+ * the method.
+ *   Arguments and results are those of fastnn_reciprocal without the
+ *   workspace: the scratch is a static device array of
+ *   FASTNN_NOALLOC_SCRATCH_BYTES (32 MiB) that every GPU loading this library
+ *   holds until the process exits. Calls whose workspace would exceed it
+ *   (fastnn_workspace_size) return FASTNN_ERR_CAPACITY and enqueue nothing;
+ *   one 512x384 pair with int8 or bf16 descriptors fits.
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture. The call allocates nothing.
+ *   All calls share the one array and it keeps the last call's contents (the
+ *   call clears what must start at zero). Calls that overlap on the GPU (on
+ *   different streams, or from several host threads without ordering) race on
+ *   it; read results with fastnn_device_status only from the last call.
+ */
+#define FASTNN_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+int fastnn_reciprocal_noalloc(const void *desc1, int H1, int W1, const void *desc2,
+                              int H2, int W2, int d, int dtype, int subsample,
+                              int max_iter, int batch, int32_t *out_pairs,
+                              void *out_score, int64_t capacity,
+                              int32_t *out_count, int32_t *out_iters,
+                              int32_t *out_frontier, fastnn_stream_t stream);
+
+/*
  * fastnn_device_status -- synchronise `stream` and read the device status
  * word of the last call that used `workspace`: FASTNN_OK, or
  * FASTNN_ERR_TIMEOUT when a kernel's bounded wait ran out (its outputs are

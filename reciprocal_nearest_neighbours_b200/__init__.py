@@ -23,6 +23,7 @@ from ._lib import (  # noqa: F401
     fastnn_mutual_dense,
     fastnn_nn,
     fastnn_reciprocal,
+    fastnn_reciprocal_noalloc,
     fastnn_status_str,
     fastnn_workspace_size,
     library,

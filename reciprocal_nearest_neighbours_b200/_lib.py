@@ -49,6 +49,8 @@ def library():
     lib.fastnn_nn.restype = I
     lib.fastnn_reciprocal.argtypes = [P, I, I, P, I, I, I, I, I, I, I, P, P, I64, P, P, P, P, SZ, P]
     lib.fastnn_reciprocal.restype = I
+    lib.fastnn_reciprocal_noalloc.argtypes = [P, I, I, P, I, I, I, I, I, I, I, P, P, I64, P, P, P, P]
+    lib.fastnn_reciprocal_noalloc.restype = I
     lib.fastnn_mutual_dense.argtypes = [P, I64, P, I64, I, I, P, P, I64, P, P, SZ, P]
     lib.fastnn_mutual_dense.restype = I
     lib.fastnn_device_status.argtypes = [P, P]
@@ -182,6 +184,31 @@ def fastnn_reciprocal(desc1: torch.Tensor, desc2: torch.Tensor, subsample: int, 
                                      _ptr(ws), nbytes,
                                      _stream(stream))
     _check(rc, "fastnn_reciprocal")
+    return out_pairs, out_score, out_count, out_iters
+
+
+def fastnn_reciprocal_noalloc(desc1: torch.Tensor, desc2: torch.Tensor, subsample: int,
+                              max_iter: int, out_pairs: torch.Tensor, out_score: torch.Tensor,
+                              out_count: torch.Tensor, out_iters=None, out_frontier=None,
+                              stream=None):
+    """fastnn_reciprocal without a workspace, for callers that cannot allocate.
+
+    The library's fixed device scratch array stands in for the workspace (see
+    include/fastnn.h); the caller passes every output buffer. Calls on one
+    device share that array, so they must not overlap on the GPU.
+    """
+    _need_cuda(desc1, desc2, out_pairs, out_score, out_count)
+    code = _dtype_code(desc1)
+    if desc1.dim() == 3:
+        desc1, desc2 = desc1.unsqueeze(0), desc2.unsqueeze(0)
+    B, H1, W1, d = desc1.shape
+    _, H2, W2, _ = desc2.shape
+    cap = out_pairs.shape[-2]
+    rc = library().fastnn_reciprocal_noalloc(
+        _ptr(desc1), H1, W1, _ptr(desc2), H2, W2, d, code, subsample, max_iter, B,
+        _ptr(out_pairs), _ptr(out_score), cap, _ptr(out_count), _ptr(out_iters),
+        _ptr(out_frontier), _stream(stream))
+    _check(rc, "fastnn_reciprocal_noalloc")
     return out_pairs, out_score, out_count, out_iters
 
 
