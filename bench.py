@@ -242,6 +242,35 @@ class ClockSampler:
                 "samples": len(mine), "power_w_max": max(power) if power else None}
 
 
+# DRAM traffic per launch of the dominant kernel, from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum; profiles/*.md), keyed by
+# workload and by a hash of the kernel sources it was taken on. A changed
+# kernel reports null until it is captured again.
+TRAFFIC = {
+    "pair_512x384_d24_i8": (12.70e6, "feee733055579d59"),
+}
+KERNEL_SOURCES = ["reciprocal_nearest_neighbours_b200/csrc/nn_tc.cu",
+                  "reciprocal_nearest_neighbours_b200/csrc/frontier_dev.cuh",
+                  "reciprocal_nearest_neighbours_b200/csrc/common.cuh",
+                  "reciprocal_nearest_neighbours_b200/csrc/ptx.cuh"]
+
+
+def kernel_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(name):
+    rec = TRAFFIC.get(name)
+    if rec is None or rec[1] != kernel_source_hash():
+        return None
+    return rec[0]
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -415,7 +444,8 @@ def run_ours(args, rank, world, local):
                 "bound": "tensor", "kernel": kname,
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": (achieved / peak) if achieved else None,
-                "traffic": None,
+                "traffic": traffic_for(w.name),
+                "traffic_unit": "bytes per launch (ncu dram read + write)",
                 "peak_source": (f"{src}: bf16_tflops {bf16_peak}" +
                                 (" x 2 (int8 = 2 x bf16, nominal ratio)" if i8 else "")),
                 "ops": f"2 x useful MACs (d = {d}) per step: {macs_per_step:.4g} MAC",
