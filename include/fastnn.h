@@ -55,7 +55,12 @@ typedef enum {
 
 typedef enum { FASTNN_I8 = 0, FASTNN_BF16 = 1 } fastnn_dtype;
 
-typedef enum { FASTNN_OP_NN = 0, FASTNN_OP_RECIPROCAL = 1, FASTNN_OP_MUTUAL_DENSE = 2 } fastnn_op;
+typedef enum {
+    FASTNN_OP_NN = 0,
+    FASTNN_OP_RECIPROCAL = 1,
+    FASTNN_OP_MUTUAL_DENSE = 2,
+    FASTNN_OP_MUTUAL_FROM_NN = 3
+} fastnn_op;
 
 /*
  * Workspace bytes one call needs.
@@ -63,6 +68,8 @@ typedef enum { FASTNN_OP_NN = 0, FASTNN_OP_RECIPROCAL = 1, FASTNN_OP_MUTUAL_DENS
  *   FASTNN_OP_RECIPROCAL:   n1 = H1*W1, n2 = H2*W2, max_queries = number of
  *                           grid seeds per pair, batch = pairs
  *   FASTNN_OP_MUTUAL_DENSE: n1, n2 = pixel counts (batch, max_queries unused)
+ *   FASTNN_OP_MUTUAL_FROM_NN: n1 = local image-1 rows, n2 = image-2 rows
+ *                           (d must still be 1..32; unused)
  * Returns 0 for arguments no call would accept.
  */
 size_t fastnn_workspace_size(int op, int64_t n1, int64_t n2, int d, int dtype,
@@ -126,6 +133,25 @@ int fastnn_mutual_dense(const void *desc1, int64_t n1, const void *desc2,
                         void *out_score, int64_t capacity, int32_t *out_count,
                         void *workspace, size_t workspace_bytes,
                         fastnn_stream_t stream);
+
+/*
+ * fastnn_mutual_from_nn -- the mutual test of the reciprocal set ("MASt3R
+ * dissection", section 1 and section 3) applied to nearest-neighbour indices
+ * that were computed elsewhere, for a row shard of image 1: local row i (global
+ * row i0 + i) with partner j = nn12[i] is kept iff nn21[j] == i0 + i. This is
+ * the last step of the dense mutual set when image 1's rows are split across
+ * GPUs and nn21 (all n2 image-2 rows, global image-1 indices) was gathered.
+ *   nn12: [n1] int32 in [0, n2); score12: [n1] int32/float or NULL;
+ *   nn21: [n2] int32 in [0, n1_total). Output (i0 + i, j) in ascending i into
+ *   out_pairs [capacity][2], scores into out_score (or NULL), *out_count =
+ *   pairs. capacity >= min(n1, n2). n1 == 0 writes *out_count = 0.
+ */
+int fastnn_mutual_from_nn(const int32_t *nn12, const void *score12, int64_t n1,
+                          int64_t i0, const int32_t *nn21, int64_t n2,
+                          int64_t n1_total, int dtype, int32_t *out_pairs,
+                          void *out_score, int64_t capacity, int32_t *out_count,
+                          void *workspace, size_t workspace_bytes,
+                          fastnn_stream_t stream);
 
 /*
  * fastnn_reciprocal_noalloc -- fastnn_reciprocal for callers that cannot

@@ -14,6 +14,7 @@ from ._lib import (  # noqa: F401
     FASTNN_BF16,
     FASTNN_I8,
     FASTNN_OP_MUTUAL_DENSE,
+    FASTNN_OP_MUTUAL_FROM_NN,
     FASTNN_OP_NN,
     FASTNN_OP_RECIPROCAL,
     FastNNError,
@@ -21,6 +22,7 @@ from ._lib import (  # noqa: F401
     fastnn_kernel_timer_enable,
     fastnn_kernel_timer_read,
     fastnn_mutual_dense,
+    fastnn_mutual_from_nn,
     fastnn_nn,
     fastnn_reciprocal,
     fastnn_reciprocal_noalloc,

@@ -15,6 +15,7 @@ FASTNN_BF16 = 1
 FASTNN_OP_NN = 0
 FASTNN_OP_RECIPROCAL = 1
 FASTNN_OP_MUTUAL_DENSE = 2
+FASTNN_OP_MUTUAL_FROM_NN = 3
 
 _lib = None
 
@@ -53,6 +54,8 @@ def library():
     lib.fastnn_reciprocal_noalloc.restype = I
     lib.fastnn_mutual_dense.argtypes = [P, I64, P, I64, I, I, P, P, I64, P, P, SZ, P]
     lib.fastnn_mutual_dense.restype = I
+    lib.fastnn_mutual_from_nn.argtypes = [P, P, I64, I64, P, I64, I64, I, P, P, I64, P, P, SZ, P]
+    lib.fastnn_mutual_from_nn.restype = I
     lib.fastnn_device_status.argtypes = [P, P]
     lib.fastnn_device_status.restype = I
     lib.fastnn_kernel_timer_enable.argtypes = [I]
@@ -240,6 +243,37 @@ def fastnn_mutual_dense(desc1: torch.Tensor, desc2: torch.Tensor, capacity: int 
                                        _ptr(out_score), cap, _ptr(out_count), _ptr(ws), nbytes,
                                        _stream(stream))
     _check(rc, "fastnn_mutual_dense")
+    return out_pairs, out_score, out_count
+
+
+def fastnn_mutual_from_nn(nn12: torch.Tensor, score12, i0: int, nn21: torch.Tensor,
+                          n1_total: int, capacity: int | None = None, out_pairs=None,
+                          out_score=None, out_count=None, workspace=None, stream=None):
+    """Mutual pairs of a row shard of image 1 from nearest-neighbour indices.
+
+    ``nn12`` [n1] int32 (partners of global rows i0 .. i0 + n1 - 1),
+    ``score12`` [n1] int32 or float32 (or None), ``nn21`` [n2] int32 (global
+    image-1 partner of every image-2 row). Returns ``(pairs [cap,2],
+    score [cap], count [1])`` with pairs[:count] in ascending image-1 index.
+    """
+    _need_cuda(nn12, nn21)
+    n1, n2 = nn12.numel(), nn21.numel()
+    dev = nn12.device
+    sdt = score12.dtype if score12 is not None else torch.int32
+    code = FASTNN_BF16 if sdt == torch.float32 else FASTNN_I8
+    cap = max(1, min(n1, n2)) if capacity is None else int(capacity)
+    if out_pairs is None:
+        out_pairs = torch.empty((cap, 2), dtype=torch.int32, device=dev)
+    if out_score is None:
+        out_score = torch.empty(cap, dtype=sdt, device=dev)
+    if out_count is None:
+        out_count = torch.empty(1, dtype=torch.int32, device=dev)
+    nbytes = fastnn_workspace_size(FASTNN_OP_MUTUAL_FROM_NN, max(n1, 1), n2, 1, code)
+    ws = _workspace(nbytes, dev, workspace)
+    rc = library().fastnn_mutual_from_nn(_ptr(nn12), _ptr(score12), n1, int(i0), _ptr(nn21), n2,
+                                         int(n1_total), code, _ptr(out_pairs), _ptr(out_score),
+                                         cap, _ptr(out_count), _ptr(ws), nbytes, _stream(stream))
+    _check(rc, "fastnn_mutual_from_nn")
     return out_pairs, out_score, out_count
 
 

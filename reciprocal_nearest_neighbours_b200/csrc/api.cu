@@ -137,6 +137,9 @@ size_t fastnn_workspace_size(int op, int64_t n1, int64_t n2, int d, int dtype, i
       if (n1 < 1) return 0;
       carve_mut(c, n1, n2, dtype);
       break;
+    case FASTNN_OP_MUTUAL_FROM_NN:
+      c.take<int32_t>(static_cast<size_t>(mutual_blocks(n1 > 0 ? n1 : 1)));
+      break;
     default:
       return 0;
   }
@@ -303,8 +306,44 @@ int fastnn_mutual_dense(const void* desc1, int64_t n1, const void* desc2, int64_
   r.q_absmax = L.status + 2;
   r.db_absmax = L.status + 1;
   FASTNN_TRY(launch_nn_tc(r, dtype, n1 + kPadRows, st));
-  return launch_mutual(L.k12, L.k21, n1, n2, L.blocks, dtype, out_pairs, out_score, capacity,
-                       out_count, st);
+  MutualSrc m{};
+  m.k12 = L.k12;
+  m.k21 = L.k21;
+  m.n1 = n1;
+  m.n2 = n2;
+  return launch_mutual(m, L.blocks, dtype, out_pairs, out_score, capacity, out_count, st);
+}
+
+int fastnn_mutual_from_nn(const int32_t* nn12, const void* score12, int64_t n1, int64_t i0,
+                          const int32_t* nn21, int64_t n2, int64_t n1_total, int dtype,
+                          int32_t* out_pairs, void* out_score, int64_t capacity,
+                          int32_t* out_count, void* workspace, size_t workspace_bytes,
+                          fastnn_stream_t stream) {
+  if (!dtype_ok(dtype)) return FASTNN_ERR_UNSUPPORTED;
+  if (n1 < 0 || n2 < 1 || i0 < 0 || n1_total < i0 + n1 || n1_total > INT32_MAX ||
+      n2 > INT32_MAX)
+    return FASTNN_ERR_INVALID;
+  if (!out_count) return FASTNN_ERR_INVALID;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (n1 == 0) {
+    FASTNN_CUDA_TRY(cudaMemsetAsync(out_count, 0, sizeof(int32_t), st));
+    return FASTNN_OK;
+  }
+  if (!nn12 || !nn21 || !out_pairs || !workspace || !aligned(workspace, kAlign))
+    return FASTNN_ERR_INVALID;
+  if (capacity < (n1 < n2 ? n1 : n2)) return FASTNN_ERR_CAPACITY;
+  if (workspace_bytes < fastnn_workspace_size(FASTNN_OP_MUTUAL_FROM_NN, n1, n2, 1, dtype, 1, 0))
+    return FASTNN_ERR_CAPACITY;
+  Carver c{static_cast<uint8_t*>(workspace)};
+  int32_t* blocks = c.take<int32_t>(static_cast<size_t>(mutual_blocks(n1)));
+  MutualSrc m{};
+  m.nn12 = nn12;
+  m.nn21 = nn21;
+  m.score12 = score12;
+  m.n1 = n1;
+  m.n2 = n2;
+  m.i0 = i0;
+  return launch_mutual(m, blocks, dtype, out_pairs, out_score, capacity, out_count, st);
 }
 
 int fastnn_device_status(const void* workspace, fastnn_stream_t stream) {

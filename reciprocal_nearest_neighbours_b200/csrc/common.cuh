@@ -72,14 +72,22 @@ struct NNArgs {
   const int* db_absmax;    // int8: max |element| of the database map (or nullptr)
 };
 
+// The parts of a pass's query description that change from round to round
+// (the rest of NNArgs stays in kernel-parameter space).
+struct PhaseQ {
+  const int32_t* q_index;
+  const int32_t* q_count;
+};
+
 // Counts, frontier indices and keys may have been written by other CTAs of
 // the same (persistent) kernel: read them through L2 (ld.global.cg).
-__device__ __forceinline__ int64_t nn_count(const NNArgs& a, int b) {
-  return a.q_count ? static_cast<int64_t>(__ldcg(a.q_count + b)) : a.nq_static;
+__device__ __forceinline__ int64_t nn_count(const NNArgs& a, const PhaseQ& q, int b) {
+  return q.q_count ? static_cast<int64_t>(__ldcg(q.q_count + b)) : a.nq_static;
 }
 
-__device__ __forceinline__ int64_t nn_query_row(const NNArgs& a, int b, int64_t k) {
-  if (a.q_index) return __ldcg(a.q_index + b * a.q_cap + k);
+__device__ __forceinline__ int64_t nn_query_row(const NNArgs& a, const PhaseQ& q, int b,
+                                                int64_t k) {
+  if (q.q_index) return __ldcg(q.q_index + b * a.q_cap + k);
   if (a.q_key) return key_index(__ldcg(a.q_key + b * a.q_cap + k));
   return k;
 }

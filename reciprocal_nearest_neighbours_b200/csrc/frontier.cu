@@ -65,24 +65,25 @@ __global__ void repack_kernel(const uint8_t* __restrict__ src, int64_t rows, int
 }
 
 // ---------------------------------------------------------- dense mutual ---
-// flag(i) = NN21(NN12(i)) == i. Three passes keep the output in ascending i
-// without inter-CTA waiting: per-block counts, one scan block, ordered emit.
-__device__ __forceinline__ bool mutual_flag(const uint64_t* k12, const uint64_t* k21, int64_t n1,
-                                            int64_t n2, int64_t i, uint32_t& j) {
-  if (i >= n1) return false;
-  j = key_index(k12[i]);
-  if (j >= static_cast<uint64_t>(n2)) return false;
-  return key_index(k21[j]) == static_cast<uint32_t>(i);
+// flag(i) = NN21(NN12(i)) == i0 + i for local image-1 row i. The NN results
+// come either as packed keys (single-GPU dense path) or as index arrays plus
+// scores (a row shard of image 1 checked against the full NN21 gathered from
+// every rank). Three passes keep the output in ascending i without inter-CTA
+// waiting: per-block counts, one scan block, ordered emit.
+__device__ __forceinline__ bool mutual_flag(const MutualSrc& m, int64_t i, uint32_t& j) {
+  if (i >= m.n1) return false;
+  j = m.k12 ? key_index(m.k12[i]) : static_cast<uint32_t>(m.nn12[i]);
+  if (j >= static_cast<uint64_t>(m.n2)) return false;
+  const uint32_t back = m.k21 ? key_index(m.k21[j]) : static_cast<uint32_t>(m.nn21[j]);
+  return back == static_cast<uint32_t>(m.i0 + i);
 }
 
-__global__ void __launch_bounds__(1024) mutual_count_kernel(const uint64_t* __restrict__ k12,
-                                                            const uint64_t* __restrict__ k21,
-                                                            int64_t n1, int64_t n2,
+__global__ void __launch_bounds__(1024) mutual_count_kernel(MutualSrc m,
                                                             int32_t* __restrict__ block_cnt) {
   __shared__ int sm[64];
   const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   uint32_t j;
-  const bool f = mutual_flag(k12, k21, n1, n2, i, j);
+  const bool f = mutual_flag(m, i, j);
   const Scan2 sc = block_scan2(f, false, sm);
   if (threadIdx.x == 0) block_cnt[blockIdx.x] = sc.tot0;
 }
@@ -122,9 +123,7 @@ __global__ void __launch_bounds__(1024) mutual_scan_kernel(int32_t* __restrict__
 }
 
 template <int DT>
-__global__ void __launch_bounds__(1024) mutual_emit_kernel(const uint64_t* __restrict__ k12,
-                                                           const uint64_t* __restrict__ k21,
-                                                           int64_t n1, int64_t n2,
+__global__ void __launch_bounds__(1024) mutual_emit_kernel(MutualSrc m,
                                                            const int32_t* __restrict__ block_off,
                                                            int32_t* __restrict__ out_pairs,
                                                            void* __restrict__ out_score,
@@ -132,19 +131,26 @@ __global__ void __launch_bounds__(1024) mutual_emit_kernel(const uint64_t* __res
   __shared__ int sm[64];
   const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   uint32_t j = 0;
-  const bool f = mutual_flag(k12, k21, n1, n2, i, j);
+  const bool f = mutual_flag(m, i, j);
   const Scan2 sc = block_scan2(f, false, sm);
   if (f) {
     const int64_t pos = block_off[blockIdx.x] + sc.ex0;
     if (pos < cap) {
-      out_pairs[pos * 2] = static_cast<int32_t>(i);
+      out_pairs[pos * 2] = static_cast<int32_t>(m.i0 + i);
       out_pairs[pos * 2 + 1] = static_cast<int32_t>(j);
       if (out_score) {
-        const uint32_t h = key_score_bits(k12[i]);
-        if (DT == FASTNN_I8)
-          static_cast<int32_t*>(out_score)[pos] = unord_i32(h);
-        else
-          static_cast<float*>(out_score)[pos] = unord_f32(h);
+        if (m.k12) {
+          const uint32_t h = key_score_bits(m.k12[i]);
+          if (DT == FASTNN_I8)
+            static_cast<int32_t*>(out_score)[pos] = unord_i32(h);
+          else
+            static_cast<float*>(out_score)[pos] = unord_f32(h);
+        } else if (m.score12) {
+          if (DT == FASTNN_I8)
+            static_cast<int32_t*>(out_score)[pos] = static_cast<const int32_t*>(m.score12)[i];
+          else
+            static_cast<float*>(out_score)[pos] = static_cast<const float*>(m.score12)[i];
+        }
       }
     }
   }
@@ -193,18 +199,16 @@ int launch_repack(const void* src, int64_t rows, int d, int dtype, void* dst, in
 
 int mutual_blocks(int64_t n1) { return static_cast<int>((n1 + 1023) / 1024); }
 
-int launch_mutual(const uint64_t* k12, const uint64_t* k21, int64_t n1, int64_t n2,
-                  int32_t* block_scratch, int dtype, int32_t* out_pairs, void* out_score,
-                  int64_t cap, int32_t* out_count, cudaStream_t st) {
-  const int nb = mutual_blocks(n1);
-  mutual_count_kernel<<<nb, 1024, 0, st>>>(k12, k21, n1, n2, block_scratch);
+int launch_mutual(const MutualSrc& m, int32_t* block_scratch, int dtype, int32_t* out_pairs,
+                  void* out_score, int64_t cap, int32_t* out_count, cudaStream_t st) {
+  const int nb = mutual_blocks(m.n1);
+  mutual_count_kernel<<<nb, 1024, 0, st>>>(m, block_scratch);
   mutual_scan_kernel<<<1, 1024, 0, st>>>(block_scratch, nb, out_count);
   if (dtype == FASTNN_I8)
-    mutual_emit_kernel<FASTNN_I8><<<nb, 1024, 0, st>>>(k12, k21, n1, n2, block_scratch, out_pairs,
-                                                       out_score, cap);
+    mutual_emit_kernel<FASTNN_I8><<<nb, 1024, 0, st>>>(m, block_scratch, out_pairs, out_score, cap);
   else
-    mutual_emit_kernel<FASTNN_BF16><<<nb, 1024, 0, st>>>(k12, k21, n1, n2, block_scratch,
-                                                         out_pairs, out_score, cap);
+    mutual_emit_kernel<FASTNN_BF16><<<nb, 1024, 0, st>>>(m, block_scratch, out_pairs, out_score,
+                                                         cap);
   FASTNN_CUDA_TRY(cudaGetLastError());
   return FASTNN_OK;
 }

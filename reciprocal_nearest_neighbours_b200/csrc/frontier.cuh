@@ -27,10 +27,23 @@ struct CompactArgs {
 
 int launch_repack(const void* src, int64_t rows, int d, int dtype, void* dst, int64_t pad_rows,
                   int* absmax, cudaStream_t st);
+// Nearest-neighbour results for the mutual test: packed keys (k12/k21) or
+// index arrays (nn12/nn21, with scores score12). Local image-1 row i is
+// global row i0 + i; nn21 / k21 index global image-1 rows.
+struct MutualSrc {
+  const uint64_t* k12;
+  const uint64_t* k21;
+  const int32_t* nn12;
+  const int32_t* nn21;
+  const void* score12;
+  int64_t n1;  // local image-1 rows
+  int64_t n2;  // image-2 rows
+  int64_t i0;  // global index of local row 0
+};
+
 int mutual_blocks(int64_t n1);
-int launch_mutual(const uint64_t* k12, const uint64_t* k21, int64_t n1, int64_t n2,
-                  int32_t* block_scratch, int dtype, int32_t* out_pairs, void* out_score,
-                  int64_t cap, int32_t* out_count, cudaStream_t st);
+int launch_mutual(const MutualSrc& m, int32_t* block_scratch, int dtype, int32_t* out_pairs,
+                  void* out_score, int64_t cap, int32_t* out_count, cudaStream_t st);
 int launch_decode(const uint64_t* key, int64_t n, int dtype, int32_t* out_idx, void* out_score,
                   cudaStream_t st);
 

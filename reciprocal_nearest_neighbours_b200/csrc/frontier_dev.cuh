@@ -53,6 +53,14 @@ __device__ __forceinline__ void seed_one(int32_t* F0, int64_t S_cap, uint32_t* c
   claim[b * N1 + u] = static_cast<uint32_t>(k);
 }
 
+// The round's frontier buffers (the rest of CompactArgs is fixed per call).
+struct FrontierBufs {
+  const int32_t* F_cur;
+  int32_t* F_next;
+  const int32_t* cnt_cur;
+  int32_t* cnt_next;
+};
+
 // Round t (1-based) of the fast scheme for pair b, run by one whole CTA.
 // Slot k holds pixel u = F[k] of image 1, its forward match v = NN(D1[u], D2)
 // and the backward match u' = NN(D2[v], D1). u' == u keeps (u, v); otherwise
@@ -63,13 +71,14 @@ __device__ __forceinline__ void seed_one(int32_t* F0, int64_t S_cap, uint32_t* c
 // compacted in slot order. The round's key slots are reset to 0 for the next
 // round's atomicMax merges. `sm` holds 66 ints.
 template <int DT>
-__device__ void compact_pair(const CompactArgs& c, int b, int t, bool last_round, int* sm) {
-  const int cnt = __ldcg(c.cnt_cur + b);
+__device__ void compact_pair(const CompactArgs& c, const FrontierBufs& fb, int b, int t,
+                             bool last_round, int* sm) {
+  const int cnt = __ldcg(fb.cnt_cur + b);
   if (cnt == 0) {
-    if (threadIdx.x == 0) c.cnt_next[b] = 0;
+    if (threadIdx.x == 0) fb.cnt_next[b] = 0;
     return;
   }
-  const int32_t* F = c.F_cur + b * c.S_cap;
+  const int32_t* F = fb.F_cur + b * c.S_cap;
   uint64_t* fwd = c.fwd_key + b * c.S_cap;
   uint64_t* bwd = c.bwd_key + b * c.S_cap;
   uint32_t* claim = c.claim + b * c.N1;
@@ -116,13 +125,13 @@ __device__ void compact_pair(const CompactArgs& c, int b, int t, bool last_round
         }
       }
     }
-    if (push) c.F_next[b * c.S_cap + next0 + sc.ex1] = static_cast<int32_t>(u2);
+    if (push) fb.F_next[b * c.S_cap + next0 + sc.ex1] = static_cast<int32_t>(u2);
     out0 += sc.tot0;
     next0 += sc.tot1;
   }
   if (threadIdx.x == 0) {
     c.out_count[b] = out0;
-    c.cnt_next[b] = next0;
+    fb.cnt_next[b] = next0;
     if (c.out_iters) c.out_iters[b] = t;
     if (c.out_frontier) c.out_frontier[b * c.max_iter + (t - 1)] = cnt;
   }

@@ -65,6 +65,12 @@ constexpr int kNumBars = kBarDone + 1;
 
 struct Ctl {
   uint64_t bars[kNumBars];
+  // Producer and MMA ring positions, kept here between phases so that only
+  // the one or two threads that use them hold them in registers.
+  int64_t p_seg, m_seg;
+  int p_st_idx, m_st_idx, m_ac_idx;
+  uint32_t p_st_phase, m_st_phase, m_ac_phase;
+  int p_last_phase[kStages];
   uint32_t tmem_base;
   int abort_flag;
   int pack16;
@@ -155,15 +161,15 @@ __device__ __forceinline__ void next_segment(Pos& p, const Ctl* ctl, int batch) 
 // with the 32B (rb = 32) or 64B (rb = 64) swizzle the MMA descriptor names:
 // the 16-byte chunk c of row r lands at r * rb + 16 * (c ^ swz(r)).
 template <int RB>
-__device__ __forceinline__ void gather_a(uint8_t* tile, const NNArgs& a, int b, int64_t m,
-                                         int cnt, int lane) {
+__device__ __forceinline__ void gather_a(uint8_t* tile, const NNArgs& a, const PhaseQ& q, int b,
+                                         int64_t m, int cnt, int lane) {
   constexpr int kC = RB / 16;
 #pragma unroll
   for (int i = 0; i < kBM / 32; ++i) {
     const int r = lane + 32 * i;
     const int64_t k = m * kBM + r;
     uint4 v[kC];
-    const int64_t row = k < cnt ? nn_query_row(a, b, k) : -1;
+    const int64_t row = k < cnt ? nn_query_row(a, q, b, k) : -1;
     // Rows outside the query source (never produced by a healthy pipeline)
     // read as zeros instead of faulting.
     if (row >= 0 && row < a.q_rows_per_pair) {
@@ -366,21 +372,21 @@ __device__ __forceinline__ SmemLayout smem_layout() {
   return L;
 }
 
-// Per-thread pipeline state that persists across phases (each role uses its
-// own fields).
+// Epilogue state that persists across phases (per thread). The producer's and
+// the MMA thread's ring positions live in Ctl.
 struct PipeState {
-  Ring st;                  // producer, MMA: database stage ring
-  Ring ac;                  // MMA: accumulator ring
-  int64_t seg = 0;          // producer, MMA: segments started (query-tile buffer)
-  int last_phase[kStages];  // producer lane 0: phase bit of the last load per stage
-  uint32_t ephase = 0;      // epilogue: phase bit of its accumulator barrier
-  int epar = 0;             // epilogue: parity of the running unit index
+  uint32_t ephase = 0;  // phase bit of this group's accumulator barrier
+  int epar = 0;         // parity of the running unit index
 };
 
 // Barrier init and TMEM allocation; ends with a CTA barrier.
 __device__ __forceinline__ void pipe_setup(Ctl* ctl) {
   if (threadIdx.x == 0) {
     ctl->abort_flag = 0;
+    ctl->p_seg = ctl->m_seg = 0;
+    ctl->p_st_idx = ctl->m_st_idx = ctl->m_ac_idx = 0;
+    ctl->p_st_phase = ctl->m_st_phase = ctl->m_ac_phase = 0;
+    for (int s = 0; s < kStages; ++s) ctl->p_last_phase[s] = -1;
     for (int i = 0; i < kNumBars; ++i) {
       uint32_t count = 1;
       if (i >= kBarAFull && i < kBarAFull + 2) count = 32;  // producer lanes
@@ -400,12 +406,12 @@ __device__ __forceinline__ void pipe_setup(Ctl* ctl) {
 
 // Work list of this CTA for one phase (thread 0).
 template <int DT>
-__device__ void plan_phase(const NNArgs& a, Ctl* ctl) {
+__device__ void plan_phase(const NNArgs& a, const PhaseQ& q, Ctl* ctl) {
   const int batch = a.batch;
   const int64_t nt = (a.ndb + kBN - 1) / kBN;
   int64_t total = 0;
   for (int b = 0; b < batch; ++b) {
-    const int64_t c = nn_count(a, b);
+    const int64_t c = nn_count(a, q, b);
     ctl->cnt[b] = static_cast<int>(c);
     ctl->mt[b] = static_cast<int>((c + kBM - 1) / kBM);
     total += static_cast<int64_t>(ctl->mt[b]) * nt;
@@ -438,14 +444,14 @@ __device__ void plan_phase(const NNArgs& a, Ctl* ctl) {
 // over this CTA's units. Ends with a CTA barrier, after which every MMA of the
 // phase has completed and every result has been merged into a.out_key.
 template <int DT>
-__device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const SmemLayout& L,
-                          uint32_t tmem, PipeState& ps) {
+__device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const PhaseQ q,
+                          const SmemLayout& L, uint32_t tmem, PipeState& ps) {
   constexpr int RB = row_bytes(DT);
   using E = Epi<DT>;
   Ctl* ctl = L.ctl;
   uint8_t* tileA = L.tileA;
   uint8_t* tileB = L.tileB;
-  if (threadIdx.x == 0) plan_phase<DT>(a, ctl);
+  if (threadIdx.x == 0) plan_phase<DT>(a, q, ctl);
   __syncthreads();
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -460,37 +466,43 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Sme
       // -------------------------------------------------------------- producer
       Pos p = start;
       bool ok = true;
-      for (int64_t u = u0; ok && u < u1; ++ps.seg) {
-        const int64_t len = seg_len(p, u, u1, nt);
-        const int as = static_cast<int>(ps.seg & 1);
-        if (!warp_wait_bounded(bar(kBarAEmpty + as),
-                               static_cast<uint32_t>(((ps.seg >> 1) & 1) ^ 1), ctl, a.status))
+      int64_t seg = ctl->p_seg;
+      Ring st;
+      st.idx = ctl->p_st_idx;
+      st.phase = ctl->p_st_phase;
+      for (int64_t u = u0; ok && u < u1; ++seg) {
+        const int len = static_cast<int>(seg_len(p, u, u1, nt));
+        const int as = static_cast<int>(seg & 1);
+        if (!warp_wait_bounded(bar(kBarAEmpty + as), static_cast<uint32_t>(((seg >> 1) & 1) ^ 1),
+                               ctl, a.status))
           break;
-        gather_a<RB>(tileA + as * tile_bytes_a(RB), a, p.b, p.m, ctl->cnt[p.b], lane);
+        gather_a<RB>(tileA + as * tile_bytes_a(RB), a, q, p.b, p.m, ctl->cnt[p.b], lane);
         ptx::fence_proxy_async_smem();
         ptx::mbar_arrive(bar(kBarAFull + as));
         if (lane == 0) {
           int32_t row = static_cast<int32_t>(static_cast<int64_t>(p.b) * a.ndb + p.n * kBN);
-          for (int64_t j = 0; j < len; ++j, row += kBN) {
-            if (!wait_bounded(bar(kBarBEmpty + ps.st.idx), ps.st.phase ^ 1u, ctl, a.status)) {
+          for (int j = 0; j < len; ++j, row += kBN) {
+            if (!wait_bounded(bar(kBarBEmpty + st.idx), st.phase ^ 1u, ctl, a.status)) {
               ok = false;
               break;
             }
-            ptx::mbar_arrive_expect_tx(bar(kBarBFull + ps.st.idx),
+            ptx::mbar_arrive_expect_tx(bar(kBarBFull + st.idx),
                                        static_cast<uint32_t>(tile_bytes_b(RB)));
-            ptx::tma_load_2d(ptx::smem_u32(tileB + ps.st.idx * tile_bytes_b(RB)), tmap_db, 0, row,
-                             bar(kBarBFull + ps.st.idx));
-            ps.last_phase[ps.st.idx] = static_cast<int>(ps.st.phase);
-            ps.st.next<kStages>();
+            ptx::tma_load_2d(ptx::smem_u32(tileB + st.idx * tile_bytes_b(RB)), tmap_db, 0, row,
+                             bar(kBarBFull + st.idx));
+            ctl->p_last_phase[st.idx] = static_cast<int>(st.phase);
+            st.next<kStages>();
           }
         }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         u += len;
         next_segment(p, ctl, batch);
       }
-      // Ring positions are per lane; lane 0 advanced the shared ring.
-      ps.st.idx = __shfl_sync(0xffffffffu, ps.st.idx, 0);
-      ps.st.phase = __shfl_sync(0xffffffffu, ps.st.phase, 0);
+      if (lane == 0) {
+        ctl->p_seg = seg;
+        ctl->p_st_idx = st.idx;
+        ctl->p_st_phase = st.phase;
+      }
     } else if (warp == kMmaWarp) {
       // ------------------------------------------------------------- MMA issue
       if (lane == 0) {
@@ -500,26 +512,32 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Sme
                 : ((1u << 4) | (1u << 7) | (1u << 10) | ((kBN >> 3) << 17) | ((kBM >> 4) << 24));
         Pos p = start;
         bool ok = true;
-        for (int64_t u = u0; ok && u < u1; ++ps.seg) {
-          const int64_t len = seg_len(p, u, u1, nt);
-          const int as = static_cast<int>(ps.seg & 1);
-          if (!wait_bounded(bar(kBarAFull + as), static_cast<uint32_t>((ps.seg >> 1) & 1), ctl,
+        int64_t seg = ctl->m_seg;
+        Ring st, ac;
+        st.idx = ctl->m_st_idx;
+        st.phase = ctl->m_st_phase;
+        ac.idx = ctl->m_ac_idx;
+        ac.phase = ctl->m_ac_phase;
+        for (int64_t u = u0; ok && u < u1; ++seg) {
+          const int len = static_cast<int>(seg_len(p, u, u1, nt));
+          const int as = static_cast<int>(seg & 1);
+          if (!wait_bounded(bar(kBarAFull + as), static_cast<uint32_t>((seg >> 1) & 1), ctl,
                             a.status))
             break;
           ptx::tc_fence_after();
           const uint64_t adesc =
               ptx::smem_desc_kmajor(ptx::smem_u32(tileA + as * tile_bytes_a(RB)), RB);
           const uint64_t bdesc0 = ptx::smem_desc_kmajor(ptx::smem_u32(tileB), RB);
-          for (int64_t j = 0; j < len; ++j) {
-            if (!wait_bounded(bar(kBarAccEmpty + ps.ac.idx), ps.ac.phase ^ 1u, ctl, a.status) ||
-                !wait_bounded(bar(kBarBFull + ps.st.idx), ps.st.phase, ctl, a.status)) {
+          for (int j = 0; j < len; ++j) {
+            if (!wait_bounded(bar(kBarAccEmpty + ac.idx), ac.phase ^ 1u, ctl, a.status) ||
+                !wait_bounded(bar(kBarBFull + st.idx), st.phase, ctl, a.status)) {
               ok = false;
               break;
             }
             ptx::tc_fence_after();
-            const uint32_t d_tmem = tmem + static_cast<uint32_t>(ps.ac.idx * kBN);
+            const uint32_t d_tmem = tmem + static_cast<uint32_t>(ac.idx * kBN);
             const uint64_t bdesc =
-                bdesc0 + static_cast<uint64_t>((ps.st.idx * tile_bytes_b(RB)) >> 4);
+                bdesc0 + static_cast<uint64_t>((st.idx * tile_bytes_b(RB)) >> 4);
             if constexpr (DT == FASTNN_I8) {
               ptx::mma_i8(d_tmem, adesc, bdesc, kIdesc, 0u);
             } else {
@@ -527,16 +545,21 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Sme
               ptx::mma_bf16(d_tmem, adesc, bdesc, kIdesc, 0u);
               ptx::mma_bf16(d_tmem, adesc + 2, bdesc + 2, kIdesc, 1u);
             }
-            ptx::mma_commit(bar(kBarBEmpty + ps.st.idx));
-            ptx::mma_commit(bar(kBarAccFull + ps.ac.idx));
-            ps.st.next<kStages>();
-            ps.ac.next<kAcc>();
+            ptx::mma_commit(bar(kBarBEmpty + st.idx));
+            ptx::mma_commit(bar(kBarAccFull + ac.idx));
+            st.next<kStages>();
+            ac.next<kAcc>();
           }
           if (!ok) break;
           ptx::mma_commit(bar(kBarAEmpty + as));
           u += len;
           next_segment(p, ctl, batch);
         }
+        ctl->m_seg = seg;
+        ctl->m_st_idx = st.idx;
+        ctl->m_st_phase = st.phase;
+        ctl->m_ac_idx = ac.idx;
+        ctl->m_ac_phase = ac.phase;
       }
     } else {
       // -------------------------------------------------------------- epilogue
@@ -555,20 +578,22 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Sme
       uint4* slot = L.stash + 2 * threadIdx.x;
       Pos p = start;
       bool ok = true;
+      const int last_n = static_cast<int>(nt - 1);
       for (int64_t u = u0; ok && u < u1;) {
-        const int64_t len = seg_len(p, u, u1, nt);
+        const int len = static_cast<int>(seg_len(p, u, u1, nt));
+        const int n0 = static_cast<int>(p.n);
         typename E::S best = E::lowest();
         uint32_t bidx = 0xFFFFFFFFu;
-        for (int64_t j = ((grp - ps.epar) & 1); j < len; j += kAcc) {
+        for (int j = (grp - ps.epar) & 1; j < len; j += kAcc) {
           if (!warp_wait_bounded(acc_bar, ps.ephase, ctl, a.status)) {
             ok = false;
             break;
           }
           ps.ephase ^= 1u;
           ptx::tc_fence_after();
-          const int64_t n = p.n + j;
-          const uint32_t colbase = static_cast<uint32_t>(n * kBN + h * kEpiCols);
-          if (n == nt - 1 && tail < kBN) {
+          const int n = n0 + j;
+          const uint32_t colbase = static_cast<uint32_t>(n) * kBN + h * kEpiCols;
+          if (n == last_n && tail < kBN) {
             // Ragged last tile of the database: column-masked fold.
             const int valid_blk = tail - h * kEpiCols;
 #pragma unroll 1
@@ -615,7 +640,7 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Sme
           atomicMax(reinterpret_cast<unsigned long long*>(&a.out_key[p.b * a.q_cap + k]),
                     static_cast<unsigned long long>(make_key(E::ord(best), bidx)));
         u += len;
-        ps.epar ^= static_cast<int>(len & 1);
+        ps.epar ^= len & 1;
         next_segment(p, ctl, batch);
       }
     }
@@ -624,8 +649,7 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Sme
 }
 
 // Drain (every issued MMA and TMA load completes) and release TMEM.
-__device__ __forceinline__ void pipe_teardown(Ctl* ctl, uint32_t tmem, PipeState& ps,
-                                              int* status) {
+__device__ __forceinline__ void pipe_teardown(Ctl* ctl, uint32_t tmem, int* status) {
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   auto bar = [&](int i) { return ptx::smem_u32(&ctl->bars[i]); };
@@ -635,8 +659,8 @@ __device__ __forceinline__ void pipe_teardown(Ctl* ctl, uint32_t tmem, PipeState
   }
   if (warp == kProducerWarp && lane == 0) {
     for (int s = 0; s < kStages; ++s)
-      if (ps.last_phase[s] >= 0)
-        wait_bounded(bar(kBarBFull + s), static_cast<uint32_t>(ps.last_phase[s]), ctl, status);
+      if (ctl->p_last_phase[s] >= 0)
+        wait_bounded(bar(kBarBFull + s), static_cast<uint32_t>(ctl->p_last_phase[s]), ctl, status);
   }
   ptx::tc_fence_before();
   __syncthreads();
@@ -646,17 +670,15 @@ __device__ __forceinline__ void pipe_teardown(Ctl* ctl, uint32_t tmem, PipeState
 
 template <int DT>
 __global__ void __launch_bounds__(kThreads, 1)
-    nn_tc_kernel(const __grid_constant__ CUtensorMap tmap_db, NNArgs a) {
+    nn_tc_kernel(const __grid_constant__ CUtensorMap tmap_db, const __grid_constant__ NNArgs a) {
   constexpr int RB = row_bytes(DT);
   const SmemLayout L = smem_layout<RB>();
   if ((threadIdx.x >> 5) == kProducerWarp && (threadIdx.x & 31) == 0) ptx::prefetch_tmap(&tmap_db);
   pipe_setup(L.ctl);
   const uint32_t tmem = L.ctl->tmem_base;
   PipeState ps;
-#pragma unroll
-  for (int s = 0; s < kStages; ++s) ps.last_phase[s] = -1;
-  run_phase<DT>(&tmap_db, a, L, tmem, ps);
-  pipe_teardown(L.ctl, tmem, ps, a.status);
+  run_phase<DT>(&tmap_db, a, PhaseQ{a.q_index, a.q_count}, L, tmem, ps);
+  pipe_teardown(L.ctl, tmem, a.status);
 }
 
 // ---- persistent fast reciprocal matching ----------------------------------
@@ -706,7 +728,8 @@ __device__ bool grid_sync(const RecArgs& r, uint32_t& target, Ctl* ctl) {
 template <int DT>
 __global__ void __launch_bounds__(kThreads, 1)
     reciprocal_kernel(const __grid_constant__ CUtensorMap tmap_d2,
-                      const __grid_constant__ CUtensorMap tmap_d1, RecArgs r) {
+                      const __grid_constant__ CUtensorMap tmap_d1,
+                      const __grid_constant__ RecArgs r) {
   constexpr int RB = row_bytes(DT);
   const SmemLayout L = smem_layout<RB>();
   Ctl* ctl = L.ctl;
@@ -717,8 +740,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   pipe_setup(ctl);
   const uint32_t tmem = ctl->tmem_base;
   PipeState ps;
-#pragma unroll
-  for (int s = 0; s < kStages; ++s) ps.last_phase[s] = -1;
   uint32_t target = 0;
   const int batch = r.batch;
   const int64_t S = r.S;
@@ -748,22 +769,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   for (int t = 1; ok && t <= r.max_iter; ++t) {
     const int cur = (t - 1) & 1, nxt = t & 1;
-    NNArgs f = r.fwd;
-    f.q_index = r.F[cur];
-    f.q_count = r.cnt[cur];
-    run_phase<DT>(&tmap_d2, f, L, tmem, ps);
+    run_phase<DT>(&tmap_d2, r.fwd, PhaseQ{r.F[cur], r.cnt[cur]}, L, tmem, ps);
     if (!grid_sync(r, target, ctl)) break;
-    NNArgs bw = r.bwd;
-    bw.q_count = r.cnt[cur];
-    run_phase<DT>(&tmap_d1, bw, L, tmem, ps);
+    run_phase<DT>(&tmap_d1, r.bwd, PhaseQ{nullptr, r.cnt[cur]}, L, tmem, ps);
     if (!grid_sync(r, target, ctl)) break;
-    CompactArgs c = r.cmp;
-    c.F_cur = r.F[cur];
-    c.F_next = r.F[nxt];
-    c.cnt_cur = r.cnt[cur];
-    c.cnt_next = r.cnt[nxt];
+    const FrontierBufs fb{r.F[cur], r.F[nxt], r.cnt[cur], r.cnt[nxt]};
     for (int b = blockIdx.x; b < batch; b += gridDim.x)
-      compact_pair<DT>(c, b, t, t == r.max_iter, ctl->scan);
+      compact_pair<DT>(r.cmp, fb, b, t, t == r.max_iter, ctl->scan);
     if (!grid_sync(r, target, ctl)) break;
     // Every CTA reads the same counts after the barrier: a uniform exit.
     if (threadIdx.x == 0) {
@@ -774,7 +786,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (!ctl->more) break;
   }
-  pipe_teardown(ctl, tmem, ps, r.status);
+  pipe_teardown(ctl, tmem, r.status);
 }
 
 using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,

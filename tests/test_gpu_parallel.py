@@ -1,0 +1,76 @@
+"""The sharded dense path's GPU steps (one process, one GPU)."""
+
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from reciprocal_nearest_neighbours_b200 import (fastnn_mutual_dense, fastnn_mutual_from_nn,
+                                                fastnn_nn, parallel)
+from tests._dev import require_cuda, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _cuda():
+    require_cuda()
+
+
+def test_mutual_from_nn_matches_definition_with_row_offset():
+    rng = np.random.default_rng(0)
+    n1_total, n2, i0, n1 = 5000, 3000, 1234, 1700
+    nn12 = rng.integers(0, n2, size=n1).astype(np.int32)
+    nn21 = rng.integers(0, n1_total, size=n2).astype(np.int32)
+    # plant mutual pairs
+    for i in rng.choice(n1, size=300, replace=False):
+        nn21[nn12[i]] = i0 + i
+    score = rng.integers(-1000, 1000, size=n1).astype(np.int32)
+    pairs, sc, cnt = fastnn_mutual_from_nn(torch.from_numpy(nn12).cuda(),
+                                           torch.from_numpy(score).cuda(), i0,
+                                           torch.from_numpy(nn21).cuda(), n1_total)
+    n = int(cnt[0])
+    i = np.arange(n1)
+    keep = nn21[nn12] == i0 + i
+    exp = np.stack([i0 + i[keep], nn12[keep]], axis=1)
+    assert np.array_equal(pairs[:n].cpu().numpy(), exp)
+    assert np.array_equal(sc[:n].cpu().numpy(), score[keep])
+    # an empty shard reports zero pairs
+    _, _, c0 = fastnn_mutual_from_nn(torch.zeros(0, dtype=torch.int32, device="cuda"), None, 0,
+                                     torch.from_numpy(nn21).cuda(), n1_total)
+    assert int(c0[0]) == 0
+
+
+def test_sharded_path_single_rank_equals_dense_kernel():
+    w = synth.make_workload("tiny_64x48_d24_i8")
+    p = w.pairs[0]
+    d1 = to_dev(p.desc1.reshape(-1, 24))
+    d2 = to_dev(p.desc2.reshape(-1, 24))
+    pairs, scores = parallel.sharded_mutual_dense(d1, d2)
+    ref_p, ref_s, ref_c = fastnn_mutual_dense(d1, d2)
+    n = int(ref_c[0])
+    assert torch.equal(pairs, ref_p[:n]) and torch.equal(scores, ref_s[:n])
+    dm = oracle.dense_mutual(p.desc1.reshape(-1, 24), p.desc2.reshape(-1, 24), "i8")
+    assert np.array_equal(pairs.cpu().numpy().astype(np.int64), dm.pairs)
+
+
+def test_sharded_path_rank_blocks_compose_on_one_gpu():
+    """Emulate two ranks' row blocks on one GPU (no collective needed) and check
+    that the concatenated per-rank outputs form the dense set."""
+    m = synth.warped_pair_int8(99, H=48, W=64, d=24)
+    D1 = to_dev(m.desc1.reshape(-1, 24))
+    D2 = to_dev(m.desc2.reshape(-1, 24))
+    n1, n2 = D1.shape[0], D2.shape[0]
+    idx21 = torch.cat([fastnn_nn(D2[lo:hi].contiguous(), D1)[0]
+                       for lo, hi in (parallel.shard_bounds(n2, r, 2) for r in range(2))])
+    out = []
+    for r in range(2):
+        lo, hi = parallel.shard_bounds(n1, r, 2)
+        i12, s12 = fastnn_nn(D1[lo:hi].contiguous(), D2)
+        pr, sc, c = fastnn_mutual_from_nn(i12, s12, lo, idx21, n1)
+        out.append(pr[: int(c[0])])
+    ref_p, _, ref_c = fastnn_mutual_dense(D1, D2)
+    assert torch.equal(torch.cat(out), ref_p[: int(ref_c[0])])
