@@ -45,8 +45,8 @@ constexpr int kStages = 6;                      // database ring: 48 KB (int8) /
 constexpr int kGroupWarps = 8;                  // epilogue warps per accumulator
 constexpr int kEpiWarps = kAcc * kGroupWarps;
 constexpr int kProducerWarp = kEpiWarps;
-constexpr int kMmaWarp = kEpiWarps + 1;
-constexpr int kThreads = 32 * (kEpiWarps + 2);
+constexpr int kMmaWarp0 = kEpiWarps + 1;        // MMA issuers: warp kMmaWarp0 + g feeds accumulator g
+constexpr int kThreads = 32 * (kEpiWarps + 1 + kAcc);
 constexpr int kEpiCols = kBN / 2;               // columns of a tile per epilogue thread
 constexpr int kChunks = kEpiCols / 32;          // 32-column TMEM loads per unit and thread
 constexpr int kMaxBatch = 1024;
@@ -62,14 +62,18 @@ constexpr int kBarAccFull = kBarAEmpty + 2;
 constexpr int kBarAccEmpty = kBarAccFull + kAcc;
 constexpr int kBarDone = kBarAccEmpty + kAcc;
 constexpr int kNumBars = kBarDone + 1;
+static_assert(kStages % kAcc == 0 && (kAcc & (kAcc - 1)) == 0, "issuer g owns stages g, g + kAcc, ...");
 
 struct Ctl {
   uint64_t bars[kNumBars];
   // Producer and MMA ring positions, kept here between phases so that only
   // the one or two threads that use them hold them in registers.
-  int64_t p_seg, m_seg;
-  int p_st_idx, m_st_idx, m_ac_idx;
-  uint32_t p_st_phase, m_st_phase, m_ac_phase;
+  int64_t p_seg;
+  int p_st_idx;
+  uint32_t p_st_phase;
+  int64_t m_seg[kAcc];
+  int m_st_idx[kAcc], m_par[kAcc];
+  uint32_t m_st_phase[kAcc], m_ac_phase[kAcc];
   int p_last_phase[kStages];
   uint32_t tmem_base;
   int abort_flag;
@@ -383,13 +387,22 @@ struct PipeState {
 __device__ __forceinline__ void pipe_setup(Ctl* ctl) {
   if (threadIdx.x == 0) {
     ctl->abort_flag = 0;
-    ctl->p_seg = ctl->m_seg = 0;
-    ctl->p_st_idx = ctl->m_st_idx = ctl->m_ac_idx = 0;
-    ctl->p_st_phase = ctl->m_st_phase = ctl->m_ac_phase = 0;
+    ctl->p_seg = 0;
+    ctl->p_st_idx = 0;
+    ctl->p_st_phase = 0;
+    for (int g = 0; g < kAcc; ++g) {
+      ctl->m_seg[g] = 0;
+      ctl->m_st_idx[g] = g;  // issuer g handles units g, g + kAcc, ... -> stages g, g + kAcc, ...
+      ctl->m_st_phase[g] = 0;
+      ctl->m_ac_phase[g] = 0;
+      ctl->m_par[g] = 0;
+    }
     for (int s = 0; s < kStages; ++s) ctl->p_last_phase[s] = -1;
     for (int i = 0; i < kNumBars; ++i) {
       uint32_t count = 1;
-      if (i >= kBarAFull && i < kBarAFull + 2) count = 32;  // producer lanes
+      if (i >= kBarAFull && i < kBarAFull + 2) count = 32;    // producer lanes
+      if (i >= kBarAEmpty && i < kBarAEmpty + 2) count = kAcc;  // one commit per MMA issuer
+      if (i == kBarDone) count = kAcc;
       if (i >= kBarAccEmpty && i < kBarAccEmpty + kAcc) count = kGroupWarps;
       ptx::mbar_init(ptx::smem_u32(&ctl->bars[i]), count);
     }
@@ -503,21 +516,26 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Pha
         ctl->p_st_idx = st.idx;
         ctl->p_st_phase = st.phase;
       }
-    } else if (warp == kMmaWarp) {
+    } else if (warp >= kMmaWarp0) {
       // ------------------------------------------------------------- MMA issue
+      // Issuer g (one thread) handles the units whose running index is
+      // congruent to g mod kAcc: accumulator g, stages g, g + kAcc, ... The
+      // issuers sit in different warps, so their per-unit waits and commits
+      // overlap.
       if (lane == 0) {
         constexpr uint32_t kIdesc =
             DT == FASTNN_I8
                 ? ((2u << 4) | (1u << 7) | (1u << 10) | ((kBN >> 3) << 17) | ((kBM >> 4) << 24))
                 : ((1u << 4) | (1u << 7) | (1u << 10) | ((kBN >> 3) << 17) | ((kBM >> 4) << 24));
+        const int g = warp - kMmaWarp0;
         Pos p = start;
         bool ok = true;
-        int64_t seg = ctl->m_seg;
-        Ring st, ac;
-        st.idx = ctl->m_st_idx;
-        st.phase = ctl->m_st_phase;
-        ac.idx = ctl->m_ac_idx;
-        ac.phase = ctl->m_ac_phase;
+        int64_t seg = ctl->m_seg[g];
+        int st_idx = ctl->m_st_idx[g];
+        uint32_t st_phase = ctl->m_st_phase[g];
+        uint32_t ac_phase = ctl->m_ac_phase[g];
+        int par = ctl->m_par[g];
+        const uint32_t d_tmem = tmem + static_cast<uint32_t>(g * kBN);
         for (int64_t u = u0; ok && u < u1; ++seg) {
           const int len = static_cast<int>(seg_len(p, u, u1, nt));
           const int as = static_cast<int>(seg & 1);
@@ -528,16 +546,15 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Pha
           const uint64_t adesc =
               ptx::smem_desc_kmajor(ptx::smem_u32(tileA + as * tile_bytes_a(RB)), RB);
           const uint64_t bdesc0 = ptx::smem_desc_kmajor(ptx::smem_u32(tileB), RB);
-          for (int j = 0; j < len; ++j) {
-            if (!wait_bounded(bar(kBarAccEmpty + ac.idx), ac.phase ^ 1u, ctl, a.status) ||
-                !wait_bounded(bar(kBarBFull + st.idx), st.phase, ctl, a.status)) {
+          for (int j = (g - par) & (kAcc - 1); j < len; j += kAcc) {
+            if (!wait_bounded(bar(kBarAccEmpty + g), ac_phase ^ 1u, ctl, a.status) ||
+                !wait_bounded(bar(kBarBFull + st_idx), st_phase, ctl, a.status)) {
               ok = false;
               break;
             }
             ptx::tc_fence_after();
-            const uint32_t d_tmem = tmem + static_cast<uint32_t>(ac.idx * kBN);
             const uint64_t bdesc =
-                bdesc0 + static_cast<uint64_t>((st.idx * tile_bytes_b(RB)) >> 4);
+                bdesc0 + static_cast<uint64_t>((st_idx * tile_bytes_b(RB)) >> 4);
             if constexpr (DT == FASTNN_I8) {
               ptx::mma_i8(d_tmem, adesc, bdesc, kIdesc, 0u);
             } else {
@@ -545,21 +562,27 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Pha
               ptx::mma_bf16(d_tmem, adesc, bdesc, kIdesc, 0u);
               ptx::mma_bf16(d_tmem, adesc + 2, bdesc + 2, kIdesc, 1u);
             }
-            ptx::mma_commit(bar(kBarBEmpty + st.idx));
-            ptx::mma_commit(bar(kBarAccFull + ac.idx));
-            st.next<kStages>();
-            ac.next<kAcc>();
+            ptx::mma_commit(bar(kBarBEmpty + st_idx));
+            ptx::mma_commit(bar(kBarAccFull + g));
+            ac_phase ^= 1u;
+            st_idx += kAcc;
+            if (st_idx >= kStages) {
+              st_idx -= kStages;
+              st_phase ^= 1u;
+            }
           }
           if (!ok) break;
+          // The query tile may be refilled once both issuers' MMAs on it completed.
           ptx::mma_commit(bar(kBarAEmpty + as));
           u += len;
+          par ^= len & 1;
           next_segment(p, ctl, batch);
         }
-        ctl->m_seg = seg;
-        ctl->m_st_idx = st.idx;
-        ctl->m_st_phase = st.phase;
-        ctl->m_ac_idx = ac.idx;
-        ctl->m_ac_phase = ac.phase;
+        ctl->m_seg[g] = seg;
+        ctl->m_st_idx[g] = st_idx;
+        ctl->m_st_phase[g] = st_phase;
+        ctl->m_ac_phase[g] = ac_phase;
+        ctl->m_par[g] = par;
       }
     } else {
       // -------------------------------------------------------------- epilogue
@@ -653,7 +676,7 @@ __device__ __forceinline__ void pipe_teardown(Ctl* ctl, uint32_t tmem, int* stat
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   auto bar = [&](int i) { return ptx::smem_u32(&ctl->bars[i]); };
-  if (warp == kMmaWarp && lane == 0) {
+  if (warp >= kMmaWarp0 && lane == 0) {
     ptx::mma_commit(bar(kBarDone));
     wait_bounded(bar(kBarDone), 0, ctl, status);
   }
