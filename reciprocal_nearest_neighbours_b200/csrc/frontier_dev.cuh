@@ -73,10 +73,6 @@ struct FrontierBufs {
 template <int DT>
 __device__ void compact_pair(const CompactArgs& c, const FrontierBufs& fb, int b, int t,
                              bool last_round, int* sm) {
-  // Each thread handles up to kPer slots per batch, all of whose loads are
-  // issued together, so a round costs a few L2 round trips instead of a few
-  // per block-sized chunk.
-  constexpr int kPer = 8;
   const int cnt = __ldcg(fb.cnt_cur + b);
   if (cnt == 0) {
     if (threadIdx.x == 0) fb.cnt_next[b] = 0;
@@ -87,80 +83,51 @@ __device__ void compact_pair(const CompactArgs& c, const FrontierBufs& fb, int b
   uint64_t* bwd = c.bwd_key + b * c.S_cap;
   uint32_t* claim = c.claim + b * c.N1;
   const uint32_t stamp_hi = static_cast<uint32_t>(t) << 24;
-  const int step = blockDim.x * kPer;
 
-  // Phase 1: claim every pushed pixel with the smallest (round, slot) stamp.
   if (!last_round) {
-    for (int base = 0; base < cnt; base += step) {
-      uint32_t u[kPer], u2[kPer];
-#pragma unroll
-      for (int i = 0; i < kPer; ++i) {
-        const int k = base + threadIdx.x + i * blockDim.x;
-        u[i] = k < cnt ? static_cast<uint32_t>(__ldcg(F + k)) : 0u;
-        u2[i] = k < cnt ? key_index(__ldcg(bwd + k)) : 0u;
-      }
-#pragma unroll
-      for (int i = 0; i < kPer; ++i) {
-        const int k = base + threadIdx.x + i * blockDim.x;
-        if (k < cnt && u2[i] != u[i] && u2[i] < static_cast<uint32_t>(c.N1))
-          atomicMin(&claim[u2[i]], stamp_hi | static_cast<uint32_t>(k));
-      }
+    for (int k = threadIdx.x; k < cnt; k += blockDim.x) {
+      const uint32_t u2 = key_index(__ldcg(bwd + k));
+      if (u2 != static_cast<uint32_t>(__ldcg(F + k)) && u2 < static_cast<uint32_t>(c.N1))
+        atomicMin(&claim[u2], stamp_hi | static_cast<uint32_t>(k));
     }
   }
   if (threadIdx.x == 0) sm[64] = __ldcg(c.out_count + b);
   __syncthreads();
-
-  // Phase 2: kept pairs and pushes, compacted in slot order.
   int out0 = sm[64], next0 = 0;
-  for (int base = 0; base < cnt; base += step) {
-    uint32_t u[kPer], u2[kPer], cl[kPer];
-    uint64_t fk[kPer];
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      const int k = base + threadIdx.x + i * blockDim.x;
-      const bool in = k < cnt;
-      u[i] = in ? static_cast<uint32_t>(__ldcg(F + k)) : 0u;
-      fk[i] = in ? __ldcg(fwd + k) : 0ull;
-      u2[i] = in ? key_index(__ldcg(bwd + k)) : 0u;
+  for (int s = 0; s < cnt; s += blockDim.x) {
+    const int k = s + threadIdx.x;
+    bool conv = false, push = false;
+    uint32_t u = 0, v = 0, u2 = 0;
+    uint64_t fk = 0;
+    if (k < cnt) {
+      u = static_cast<uint32_t>(__ldcg(F + k));
+      fk = __ldcg(fwd + k);
+      v = key_index(fk);
+      u2 = key_index(__ldcg(bwd + k));
+      conv = (u2 == u);
+      push = !conv && !last_round && u2 < static_cast<uint32_t>(c.N1) &&
+             __ldcg(claim + u2) == (stamp_hi | static_cast<uint32_t>(k));
+      fwd[k] = 0;
+      bwd[k] = 0;
     }
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      const int k = base + threadIdx.x + i * blockDim.x;
-      cl[i] = (k < cnt && !last_round && u2[i] != u[i] && u2[i] < static_cast<uint32_t>(c.N1))
-                  ? __ldcg(claim + u2[i])
-                  : 0xFFFFFFFFu;
-    }
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      const int k = base + threadIdx.x + i * blockDim.x;
-      if (base + i * blockDim.x >= cnt) break;  // uniform over the block
-      const bool in = k < cnt;
-      const bool conv = in && u2[i] == u[i];
-      const bool push = in && !conv && cl[i] == (stamp_hi | static_cast<uint32_t>(k));
-      if (in) {
-        fwd[k] = 0;
-        bwd[k] = 0;
-      }
-      const Scan2 sc = block_scan2(conv, push, sm);
-      if (conv) {
-        const int64_t pos = out0 + sc.ex0;
-        if (pos < c.cap) {
-          int32_t* op = c.out_pairs + (b * c.cap + pos) * 2;
-          op[0] = static_cast<int32_t>(u[i]);
-          op[1] = static_cast<int32_t>(key_index(fk[i]));
-          if (c.out_score) {
-            if (DT == FASTNN_I8)
-              static_cast<int32_t*>(c.out_score)[b * c.cap + pos] =
-                  unord_i32(key_score_bits(fk[i]));
-            else
-              static_cast<float*>(c.out_score)[b * c.cap + pos] = unord_f32(key_score_bits(fk[i]));
-          }
+    const Scan2 sc = block_scan2(conv, push, sm);
+    if (conv) {
+      const int64_t pos = out0 + sc.ex0;
+      if (pos < c.cap) {
+        int32_t* op = c.out_pairs + (b * c.cap + pos) * 2;
+        op[0] = static_cast<int32_t>(u);
+        op[1] = static_cast<int32_t>(v);
+        if (c.out_score) {
+          if (DT == FASTNN_I8)
+            static_cast<int32_t*>(c.out_score)[b * c.cap + pos] = unord_i32(key_score_bits(fk));
+          else
+            static_cast<float*>(c.out_score)[b * c.cap + pos] = unord_f32(key_score_bits(fk));
         }
       }
-      if (push) fb.F_next[b * c.S_cap + next0 + sc.ex1] = static_cast<int32_t>(u2[i]);
-      out0 += sc.tot0;
-      next0 += sc.tot1;
     }
+    if (push) fb.F_next[b * c.S_cap + next0 + sc.ex1] = static_cast<int32_t>(u2);
+    out0 += sc.tot0;
+    next0 += sc.tot1;
   }
   if (threadIdx.x == 0) {
     c.out_count[b] = out0;
