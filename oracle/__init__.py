@@ -54,7 +54,7 @@ def build(force: bool = False) -> str:
     """Compile ``oracle.c`` into ``liboracle.so`` next to it (gcc -O2, OpenMP)."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
         cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared",
-               "-std=c11", "-Wall", "-o", _LIB, _SRC]
+               "-std=c11", "-Wall", "-o", _LIB, _SRC, "-lm"]
         # Portable x86-64 code: the built library travels to other hosts.
         subprocess.run(cmd, check=True, capture_output=True, text=True)
     return _LIB
@@ -71,6 +71,10 @@ def _load():
         lib.oracle_nn_i8.restype = ctypes.c_int
         lib.oracle_nn_bf16.argtypes = [P, I64, P, I64, ctypes.c_int, P, P, P, ctypes.c_int]
         lib.oracle_nn_bf16.restype = ctypes.c_int
+        lib.oracle_nn_f16.argtypes = [P, I64, P, I64, ctypes.c_int, P, P, P, ctypes.c_int]
+        lib.oracle_nn_f16.restype = ctypes.c_int
+        lib.oracle_half_to_double.argtypes = [ctypes.c_uint16]
+        lib.oracle_half_to_double.restype = ctypes.c_double
         _lib = lib
     return _lib
 
@@ -94,7 +98,7 @@ def nn(q: np.ndarray, db: np.ndarray, dtype: str, nthreads: int | None = None) -
     """Nearest neighbour of every row of ``q`` among the rows of ``db``.
 
     ``q`` is [nq, d], ``db`` is [ndb, d]; int8 arrays for ``dtype == "i8"``,
-    uint16 bfloat16 bit patterns for ``dtype == "bf16"``.
+    uint16 bit patterns of bfloat16 (``"bf16"``) or IEEE half (``"f16"``).
     """
     lib = _load()
     nthreads = default_threads() if nthreads is None else nthreads
@@ -110,12 +114,12 @@ def nn(q: np.ndarray, db: np.ndarray, dtype: str, nthreads: int | None = None) -
         rc = lib.oracle_nn_i8(_ptr(q), nq, _ptr(db), ndb, d, _ptr(idx), _ptr(score), nthreads)
         assert rc == 0
         return NNResult(idx, score)
-    if dtype == "bf16":
+    if dtype in ("bf16", "f16"):
         assert q.dtype == np.uint16 and db.dtype == np.uint16
         score = np.empty(nq, dtype=np.float64)
         second = np.empty(nq, dtype=np.float64)
-        rc = lib.oracle_nn_bf16(_ptr(q), nq, _ptr(db), ndb, d, _ptr(idx), _ptr(score),
-                                _ptr(second), nthreads)
+        fn = lib.oracle_nn_bf16 if dtype == "bf16" else lib.oracle_nn_f16
+        rc = fn(_ptr(q), nq, _ptr(db), ndb, d, _ptr(idx), _ptr(score), _ptr(second), nthreads)
         assert rc == 0
         return NNResult(idx, score, second)
     raise ValueError(dtype)
@@ -125,6 +129,10 @@ def score_of(D1: np.ndarray, i: np.ndarray, D2: np.ndarray, j: np.ndarray, dtype
     """Exact scores <D1[i], D2[j]> for paired index arrays (int64 or float64)."""
     if dtype == "i8":
         return (D1[i].astype(np.int64) * D2[j].astype(np.int64)).sum(axis=1)
+    if dtype == "f16":
+        a = D1[i].view(np.float16).astype(np.float64)
+        b = D2[j].view(np.float16).astype(np.float64)
+        return (a * b).sum(axis=1)
     a = (D1[i].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
     b = (D2[j].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
     return (a * b).sum(axis=1)
@@ -216,5 +224,5 @@ def fast_reciprocal(D1: np.ndarray, H1: int, W1: int, D2: np.ndarray, H2: int, W
         chain_gap = nxt_gap
     us = sorted(kept)
     pairs = np.array([[u, kept[u][0]] for u in us], dtype=np.int64).reshape(-1, 2)
-    sc = np.array([kept[u][1] for u in us], dtype=np.float64 if dtype == "bf16" else np.int64)
+    sc = np.array([kept[u][1] for u in us], dtype=np.int64 if dtype == "i8" else np.float64)
     return FastResult(pairs, sc, sizes, first, kept_gap if track_gaps else {})

@@ -14,11 +14,12 @@
  * wins (the tie rule this build fixes; the pages are silent on ties).
  *
  * Precision: int8 descriptors are multiplied and summed exactly in int64.
- * bfloat16 descriptors are widened exactly to double; each product of two
- * 8-bit significands is exact in double and the sum of d <= 64 such terms
- * carries an error far below any score gap the tests look at.
+ * bfloat16 and IEEE half descriptors are widened exactly to double; each
+ * product of two 8- or 11-bit significands is exact in double and the sum of
+ * d <= 64 such terms carries an error far below any score gap the tests look
+ * at.
  *
- * The bf16 scan also returns the runner-up score (the best score over every
+ * The float scans also return the runner-up score (the best score over every
  * k other than the chosen one; equal to the best when the best is tied),
  * which the float tolerance rule needs.
  *
@@ -26,6 +27,7 @@
  * per-query scan is the plain sequential loop above either way.
  */
 #include <stdint.h>
+#include <math.h>
 #include <string.h>
 
 static double bf16_to_double(uint16_t b)
@@ -35,6 +37,24 @@ static double bf16_to_double(uint16_t b)
     memcpy(&f, &u, sizeof f);
     return (double)f;
 }
+
+/* IEEE 754 binary16 to double, exactly: sign, 5-bit exponent (bias 15),
+ * 10-bit fraction; exponent 0 holds subnormals (fraction * 2^-24). Inputs
+ * are finite. */
+static double f16_to_double(uint16_t h)
+{
+    const int sign = (h >> 15) & 1;
+    const int e = (h >> 10) & 0x1F;
+    const int f = h & 0x3FF;
+    double v;
+    if (e == 0)
+        v = ldexp((double)f, -24);
+    else
+        v = ldexp((double)(f | 0x400), e - 25);
+    return sign ? -v : v;
+}
+
+typedef double (*to_double_fn)(uint16_t);
 
 int oracle_nn_i8(const int8_t *q, int64_t nq, const int8_t *db, int64_t ndb,
                  int d, int32_t *out_idx, int64_t *out_score, int nthreads)
@@ -63,9 +83,10 @@ int oracle_nn_i8(const int8_t *q, int64_t nq, const int8_t *db, int64_t ndb,
     return 0;
 }
 
-int oracle_nn_bf16(const uint16_t *q, int64_t nq, const uint16_t *db,
-                   int64_t ndb, int d, int32_t *out_idx, double *out_score,
-                   double *out_second, int nthreads)
+/* 16-bit float descriptors; `cvt` widens bfloat16 or IEEE half exactly. */
+static int nn_f16_like(const uint16_t *q, int64_t nq, const uint16_t *db,
+                       int64_t ndb, int d, int32_t *out_idx, double *out_score,
+                       double *out_second, int nthreads, to_double_fn cvt)
 {
     if (nq < 0 || ndb <= 0 || d <= 0 || d > 64)
         return -1;
@@ -74,7 +95,7 @@ int oracle_nn_bf16(const uint16_t *q, int64_t nq, const uint16_t *db,
     for (int64_t i = 0; i < nq; ++i) {
         double qi[64];
         for (int c = 0; c < d; ++c)
-            qi[c] = bf16_to_double(q[i * (int64_t)d + c]);
+            qi[c] = cvt(q[i * (int64_t)d + c]);
         double best = 0.0, second = 0.0;
         int32_t best_k = -1;
         int have_second = 0;
@@ -82,7 +103,7 @@ int oracle_nn_bf16(const uint16_t *q, int64_t nq, const uint16_t *db,
             const uint16_t *dk = db + k * (int64_t)d;
             double s = 0.0;
             for (int c = 0; c < d; ++c)
-                s += qi[c] * bf16_to_double(dk[c]);
+                s += qi[c] * cvt(dk[c]);
             if (best_k < 0) {
                 best = s;
                 best_k = (int32_t)k;
@@ -102,3 +123,22 @@ int oracle_nn_bf16(const uint16_t *q, int64_t nq, const uint16_t *db,
     }
     return 0;
 }
+
+int oracle_nn_bf16(const uint16_t *q, int64_t nq, const uint16_t *db,
+                   int64_t ndb, int d, int32_t *out_idx, double *out_score,
+                   double *out_second, int nthreads)
+{
+    return nn_f16_like(q, nq, db, ndb, d, out_idx, out_score, out_second,
+                       nthreads, bf16_to_double);
+}
+
+int oracle_nn_f16(const uint16_t *q, int64_t nq, const uint16_t *db,
+                  int64_t ndb, int d, int32_t *out_idx, double *out_score,
+                  double *out_second, int nthreads)
+{
+    return nn_f16_like(q, nq, db, ndb, d, out_idx, out_score, out_second,
+                       nthreads, f16_to_double);
+}
+
+/* Exposed for the oracle's own tests (exhaustive check of the conversion). */
+double oracle_half_to_double(uint16_t h) { return f16_to_double(h); }

@@ -38,6 +38,7 @@ __all__ = [
     "planted_sign_pair",
     "random_int8_pair",
     "f64_to_bf16_bits",
+    "f64_to_f16_bits",
     "bf16_bits_to_f64",
 ]
 
@@ -116,6 +117,11 @@ def f64_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     u = f32.view(np.uint32).astype(np.uint64)
     bias = ((u >> 16) & 1) + 0x7FFF
     return ((u + bias) >> 16).astype(np.uint16)
+
+
+def f64_to_f16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float64 values to IEEE half (round-to-nearest-even); raw uint16 bits."""
+    return np.asarray(x, dtype=np.float64).astype(np.float16).view(np.uint16)
 
 
 def bf16_bits_to_f64(b: np.ndarray) -> np.ndarray:
@@ -220,7 +226,8 @@ def _unit_rows(x: np.ndarray) -> np.ndarray:
 
 
 def warped_pair_bf16(seed: int, H: int = 384, W: int = 512, d: int = 24,
-                     sigma: float = 0.05, outlier_frac: float = 0.3) -> PairMaps:
+                     sigma: float = 0.05, outlier_frac: float = 0.3,
+                     storage: str = "bf16") -> PairMaps:
     """Unit-norm float descriptors stored as bfloat16.
 
     map1 ~ N(0, 1)^d per pixel, L2-normalised in float64. map2 = the warped
@@ -240,8 +247,8 @@ def warped_pair_bf16(seed: int, H: int = 384, W: int = 512, d: int = 24,
     m2[out] = rng.standard_normal((int(out.sum()), d))
     m2 = _unit_rows(m2)
     gt = np.where(out, -1, src)
-    return PairMaps(f64_to_bf16_bits(m1).reshape(H, W, d),
-                    f64_to_bf16_bits(m2).reshape(H, W, d), gt, "bf16")
+    cvt = f64_to_bf16_bits if storage == "bf16" else f64_to_f16_bits
+    return PairMaps(cvt(m1).reshape(H, W, d), cvt(m2).reshape(H, W, d), gt, storage)
 
 
 def planted_sign_pair(seed: int, H: int, W: int, d: int, c: int = 8,

@@ -308,3 +308,39 @@ def test_bf16_fast_gap_tracking_on_tiny_pair():
     r = oracle.fast_reciprocal(p.desc1, 24, 32, p.desc2, 24, 32, "bf16", 4, 10, track_gaps=True)
     assert set(r.min_gap) == set(r.pairs[:, 0].tolist())
     assert all(g >= 0 for g in r.min_gap.values())
+
+
+# ---------------------------------------------------------------------------
+# IEEE half descriptors
+# ---------------------------------------------------------------------------
+
+def test_half_widening_is_exact_on_every_finite_pattern():
+    lib = oracle._load()
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    ref = bits.view(np.float16).astype(np.float64)
+    finite = np.isfinite(ref)
+    got = np.array([lib.oracle_half_to_double(int(b)) for b in bits[finite]])
+    assert np.array_equal(got, ref[finite])
+
+
+def test_nn_f16_matches_float64_argmax_and_runner_up():
+    p = synth.warped_pair_bf16(synth.BASE_SEED + 4, H=48, W=64, storage="f16")
+    D1 = p.desc1.reshape(-1, p.d)
+    D2 = p.desc2.reshape(-1, p.d)
+    r = oracle.nn(D1[:400], D2, "f16")
+    S = D1[:400].view(np.float16).astype(np.float64) @ D2.view(np.float16).astype(np.float64).T
+    srt = np.sort(S, axis=1)
+    assert np.allclose(r.score, srt[:, -1], atol=1e-12, rtol=0)
+    assert np.allclose(r.second, srt[:, -2], atol=1e-12, rtol=0)
+    sure = srt[:, -1] - srt[:, -2] > 1e-9
+    assert np.array_equal(r.idx[sure], np.argmax(S, axis=1)[sure])
+    assert np.array_equal(oracle.score_of(D1, np.arange(400), D2, r.idx, "f16"), r.score)
+
+
+def test_nn_long_descriptors_d64_by_definition():
+    rng = np.random.default_rng(64)
+    q = rng.integers(-2, 3, size=(30, 64)).astype(np.int8)
+    db = rng.integers(-2, 3, size=(50, 64)).astype(np.int8)
+    r = oracle.nn(q, db, "i8", nthreads=1)
+    for i in range(30):
+        assert (r.idx[i], r.score[i]) == _brute.nn_by_definition(q[i], db)
