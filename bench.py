@@ -81,19 +81,19 @@ def load_workload(name, rank):
     seed = synth.CONFIGS[name]["seed"] + 7919 * rank
     if name.startswith("batch16"):
         w.pairs = [synth.warped_pair_int8(seed + 1000 * b, H=288, W=512, d=32) for b in range(16)]
-    elif name.endswith("bf16"):
-        w.pairs = [synth.warped_pair_bf16(seed)]
+    elif name.endswith("bf16") or name.endswith("f16"):
+        w.pairs = [synth.warped_pair_bf16(seed, storage=w.pairs[0].dtype)]
     elif name.startswith("tiny"):
         w.pairs = [synth.tiny_permuted_pair(seed)]
     else:
-        w.pairs = [synth.warped_pair_int8(seed)]
+        w.pairs = [synth.warped_pair_int8(seed, d=w.pairs[0].d)]
     return w
 
 
 def config_dict(w, extra=None):
     p = w.pairs[0]
     c = {"workload": w.name, "image": f"{p.W1}x{p.H1}", "d": p.d,
-         "descriptor": "bf16 unit-norm" if p.dtype == "bf16" else "int8",
+         "descriptor": {"bf16": "bf16 unit-norm", "f16": "IEEE half unit-norm"}.get(p.dtype, "int8"),
          "pairs_per_rank_per_step": w.batch,
          "parallelism": "pair-parallel replicas, no collective",
          "l2": "flushed between timed steps (256 MiB write)"}
@@ -109,9 +109,10 @@ def config_dict(w, extra=None):
     return c
 
 
-def to_pinned(arr, torch):
+def to_pinned(arr, torch, storage="i8"):
     if arr.dtype == np.uint16:
-        return torch.from_numpy(arr.view(np.int16)).view(torch.bfloat16).pin_memory()
+        half = torch.float16 if storage == "f16" else torch.bfloat16
+        return torch.from_numpy(arr.view(np.int16)).view(half).pin_memory()
     return torch.from_numpy(arr).pin_memory()
 
 
@@ -302,15 +303,15 @@ def run_ours(args, rank, world, local):
     H2, W2, _ = p0.desc2.shape
     N1, N2 = H1 * W1, H2 * W2
     i8 = p0.dtype == "i8"
-    code = fnn.FASTNN_I8 if i8 else fnn.FASTNN_BF16
+    code = {"i8": fnn.FASTNN_I8, "bf16": fnn.FASTNN_BF16, "f16": fnn.FASTNN_F16}[p0.dtype]
     sdt = torch.int32 if i8 else torch.float32
     esize = 1 if i8 else 2
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     if w.dense:
-        h1 = to_pinned(np.ascontiguousarray(p0.desc1.reshape(-1, d)), torch)
-        h2 = to_pinned(np.ascontiguousarray(p0.desc2.reshape(-1, d)), torch)
+        h1 = to_pinned(np.ascontiguousarray(p0.desc1.reshape(-1, d)), torch, p0.dtype)
+        h2 = to_pinned(np.ascontiguousarray(p0.desc2.reshape(-1, d)), torch, p0.dtype)
         cap = min(N1, N2)
         out_pairs = torch.empty((cap, 2), dtype=torch.int32, device=dev)
         out_score = torch.empty(cap, dtype=sdt, device=dev)
@@ -320,7 +321,7 @@ def run_ours(args, rank, world, local):
         hp_score = torch.empty(cap, dtype=sdt).pin_memory()
     else:
         d1n, d2n = w.stacked()
-        h1, h2 = to_pinned(d1n, torch), to_pinned(d2n, torch)
+        h1, h2 = to_pinned(d1n, torch, p0.dtype), to_pinned(d2n, torch, p0.dtype)
         S = fnn.seed_count(H1, W1, w.subsample)
         out_pairs = torch.empty((B, S, 2), dtype=torch.int32, device=dev)
         out_score = torch.empty((B, S), dtype=sdt, device=dev)
@@ -437,7 +438,8 @@ def run_ours(args, rank, world, local):
             "metric": metric_for(w.name), "value": value, "unit": UNIT, "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": total_ms / K,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "int8" if i8 else "bf16", "data": "synthetic", "config": config_dict(w),
+            "dtype": {"i8": "int8", "bf16": "bf16", "f16": "f16"}[p0.dtype], "data": "synthetic",
+            "config": config_dict(w),
             "pairs_per_s": pairs_per_s,
             "matches_per_step_rank0": matches,
             "roofline": {

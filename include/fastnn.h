@@ -19,9 +19,9 @@
  *   - Descriptor maps are row-major [rows][d] (an image is [H][W][d], pixel
  *     index p = y * W + x); batches are [batch][rows][d].
  *   - dtype FASTNN_I8: int8 descriptors, int32 scores (exact).
- *     dtype FASTNN_BF16: bfloat16 descriptors (raw 16-bit patterns), float32
- *     scores (fp32 accumulation of exact bf16 products).
- *     1 <= d <= 32 for both.
+ *     dtype FASTNN_BF16 / FASTNN_F16: bfloat16 / IEEE half descriptors (raw
+ *     16-bit patterns), float32 scores (fp32 accumulation of exact products).
+ *     1 <= d <= 64 for all three (d <= 32 runs one 32-element K step).
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the
  *     legacy default stream). The host blocks only in fastnn_device_status().
  *   - Return value: FASTNN_OK, or a negative fastnn_status describing an
@@ -47,13 +47,13 @@ typedef struct CUstream_st *fastnn_stream_t; /* same type as cudaStream_t */
 typedef enum {
     FASTNN_OK = 0,
     FASTNN_ERR_INVALID = -1,     /* bad pointer, size, alignment or argument */
-    FASTNN_ERR_UNSUPPORTED = -2, /* d or dtype outside what the kernels take */
+    FASTNN_ERR_UNSUPPORTED = -2, /* d (1..64) or dtype outside what the kernels take */
     FASTNN_ERR_CAPACITY = -3,    /* output capacity or workspace too small */
     FASTNN_ERR_CUDA = -4,        /* a CUDA runtime call or launch failed */
     FASTNN_ERR_TIMEOUT = -5      /* a device-side bounded wait ran out */
 } fastnn_status;
 
-typedef enum { FASTNN_I8 = 0, FASTNN_BF16 = 1 } fastnn_dtype;
+typedef enum { FASTNN_I8 = 0, FASTNN_BF16 = 1, FASTNN_F16 = 2 } fastnn_dtype;
 
 typedef enum {
     FASTNN_OP_NN = 0,

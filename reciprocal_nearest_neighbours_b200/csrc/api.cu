@@ -41,7 +41,8 @@ struct Carver {
   }
 };
 
-bool dtype_ok(int dtype) { return dtype == FASTNN_I8 || dtype == FASTNN_BF16; }
+bool dtype_ok(int dtype) { return dtype == FASTNN_I8 || dtype == FASTNN_BF16 || dtype == FASTNN_F16; }
+bool d_ok(int d) { return d >= 1 && d <= 64; }
 
 struct NNLayout {
   int* status;
@@ -49,9 +50,9 @@ struct NNLayout {
   uint8_t* dbrep;
   uint64_t* keys;
 };
-NNLayout carve_nn(Carver& c, int64_t nq, int64_t ndb, int dtype) {
+NNLayout carve_nn(Carver& c, int64_t nq, int64_t ndb, int d, int dtype) {
   NNLayout L;
-  const int rb = row_bytes(dtype);
+  const int rb = row_bytes(dtype, d);
   L.status = c.take<int>(64);
   L.qrep = c.take<uint8_t>(static_cast<size_t>(nq) * rb);
   L.dbrep = c.take<uint8_t>(static_cast<size_t>(ndb + kPadRows) * rb);
@@ -69,9 +70,9 @@ struct RecLayout {
   uint32_t* claim;
   int32_t* cnt[2];
 };
-RecLayout carve_rec(Carver& c, int64_t N1, int64_t N2, int dtype, int batch, int64_t S) {
+RecLayout carve_rec(Carver& c, int64_t N1, int64_t N2, int d, int dtype, int batch, int64_t S) {
   RecLayout L;
-  const int rb = row_bytes(dtype);
+  const int rb = row_bytes(dtype, d);
   L.status = c.take<int>(64);
   L.d1rep = c.take<uint8_t>(static_cast<size_t>(batch * N1 + kPadRows) * rb);
   L.d2rep = c.take<uint8_t>(static_cast<size_t>(batch * N2 + kPadRows) * rb);
@@ -93,9 +94,9 @@ struct MutLayout {
   uint64_t* k21;
   int32_t* blocks;
 };
-MutLayout carve_mut(Carver& c, int64_t n1, int64_t n2, int dtype) {
+MutLayout carve_mut(Carver& c, int64_t n1, int64_t n2, int d, int dtype) {
   MutLayout L;
-  const int rb = row_bytes(dtype);
+  const int rb = row_bytes(dtype, d);
   L.status = c.take<int>(64);
   L.d1rep = c.take<uint8_t>(static_cast<size_t>(n1 + kPadRows) * rb);
   L.d2rep = c.take<uint8_t>(static_cast<size_t>(n2 + kPadRows) * rb);
@@ -123,19 +124,19 @@ extern "C" {
 
 size_t fastnn_workspace_size(int op, int64_t n1, int64_t n2, int d, int dtype, int batch,
                              int64_t max_queries) {
-  if (!dtype_ok(dtype) || d < 1 || d > 32 || n1 < 0 || n2 < 1) return 0;
+  if (!dtype_ok(dtype) || !d_ok(d) || n1 < 0 || n2 < 1) return 0;
   Carver c{nullptr};
   switch (op) {
     case FASTNN_OP_NN:
-      carve_nn(c, n1, n2, dtype);
+      carve_nn(c, n1, n2, d, dtype);
       break;
     case FASTNN_OP_RECIPROCAL:
       if (batch < 1 || max_queries < 1 || n1 < 1) return 0;
-      carve_rec(c, n1, n2, dtype, batch, max_queries);
+      carve_rec(c, n1, n2, d, dtype, batch, max_queries);
       break;
     case FASTNN_OP_MUTUAL_DENSE:
       if (n1 < 1) return 0;
-      carve_mut(c, n1, n2, dtype);
+      carve_mut(c, n1, n2, d, dtype);
       break;
     case FASTNN_OP_MUTUAL_FROM_NN:
       c.take<int32_t>(static_cast<size_t>(mutual_blocks(n1 > 0 ? n1 : 1)));
@@ -149,7 +150,7 @@ size_t fastnn_workspace_size(int op, int64_t n1, int64_t n2, int d, int dtype, i
 int fastnn_nn(const void* q, int64_t nq, const void* db, int64_t ndb, int d, int dtype,
               int32_t* out_idx, void* out_score, void* workspace, size_t workspace_bytes,
               fastnn_stream_t stream) {
-  if (!dtype_ok(dtype) || d < 1 || d > 32) return FASTNN_ERR_UNSUPPORTED;
+  if (!dtype_ok(dtype) || !d_ok(d)) return FASTNN_ERR_UNSUPPORTED;
   if (nq < 0 || ndb < 1 || nq > INT32_MAX || ndb > INT32_MAX - kPadRows) return FASTNN_ERR_INVALID;
   if (nq == 0) return FASTNN_OK;
   if (!q || !db || !out_idx || !workspace || !aligned(workspace, kAlign)) return FASTNN_ERR_INVALID;
@@ -157,7 +158,7 @@ int fastnn_nn(const void* q, int64_t nq, const void* db, int64_t ndb, int d, int
     return FASTNN_ERR_CAPACITY;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   Carver c{static_cast<uint8_t*>(workspace)};
-  NNLayout L = carve_nn(c, nq, ndb, dtype);
+  NNLayout L = carve_nn(c, nq, ndb, d, dtype);
   FASTNN_CUDA_TRY(cudaMemsetAsync(L.status, 0, kStatusBytes, st));
   FASTNN_CUDA_TRY(cudaMemsetAsync(L.keys, 0, static_cast<size_t>(nq) * sizeof(uint64_t), st));
   FASTNN_TRY(launch_repack(q, nq, d, dtype, L.qrep, 0, L.status + 1, st));
@@ -184,7 +185,7 @@ int fastnn_reciprocal(const void* desc1, int H1, int W1, const void* desc2, int 
                       void* out_score, int64_t capacity, int32_t* out_count, int32_t* out_iters,
                       int32_t* out_frontier, void* workspace, size_t workspace_bytes,
                       fastnn_stream_t stream) {
-  if (!dtype_ok(dtype) || d < 1 || d > 32) return FASTNN_ERR_UNSUPPORTED;
+  if (!dtype_ok(dtype) || !d_ok(d)) return FASTNN_ERR_UNSUPPORTED;
   if (H1 < 1 || W1 < 1 || H2 < 1 || W2 < 1 || subsample < 1 || max_iter < 1 ||
       max_iter > kMaxIter || batch < 1 || batch > nn_tc_max_batch())
     return FASTNN_ERR_INVALID;
@@ -202,7 +203,7 @@ int fastnn_reciprocal(const void* desc1, int H1, int W1, const void* desc2, int 
     return FASTNN_ERR_CAPACITY;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   Carver c{static_cast<uint8_t*>(workspace)};
-  RecLayout L = carve_rec(c, N1, N2, dtype, batch, S);
+  RecLayout L = carve_rec(c, N1, N2, d, dtype, batch, S);
 
   // Status block: status word, per-map max |element|, grid-barrier words.
   FASTNN_CUDA_TRY(cudaMemsetAsync(L.status, 0, kStatusBytes, st));
@@ -262,7 +263,7 @@ int fastnn_mutual_dense(const void* desc1, int64_t n1, const void* desc2, int64_
                         int dtype, int32_t* out_pairs, void* out_score, int64_t capacity,
                         int32_t* out_count, void* workspace, size_t workspace_bytes,
                         fastnn_stream_t stream) {
-  if (!dtype_ok(dtype) || d < 1 || d > 32) return FASTNN_ERR_UNSUPPORTED;
+  if (!dtype_ok(dtype) || !d_ok(d)) return FASTNN_ERR_UNSUPPORTED;
   if (n1 < 1 || n2 < 1 || n1 > INT32_MAX - kPadRows || n2 > INT32_MAX - kPadRows)
     return FASTNN_ERR_INVALID;
   if (!desc1 || !desc2 || !out_pairs || !out_count || !workspace || !aligned(workspace, kAlign))
@@ -272,7 +273,7 @@ int fastnn_mutual_dense(const void* desc1, int64_t n1, const void* desc2, int64_
     return FASTNN_ERR_CAPACITY;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   Carver c{static_cast<uint8_t*>(workspace)};
-  MutLayout L = carve_mut(c, n1, n2, dtype);
+  MutLayout L = carve_mut(c, n1, n2, d, dtype);
   FASTNN_CUDA_TRY(cudaMemsetAsync(L.status, 0, kStatusBytes, st));
   FASTNN_CUDA_TRY(cudaMemsetAsync(L.k12, 0, static_cast<size_t>(n1) * 8, st));
   FASTNN_CUDA_TRY(cudaMemsetAsync(L.k21, 0, static_cast<size_t>(n2) * 8, st));

@@ -44,8 +44,12 @@ __host__ __device__ __forceinline__ uint32_t key_score_bits(uint64_t key) {
   return static_cast<uint32_t>(key >> 32);
 }
 
-// Bytes of one repacked descriptor row: d <= 32 elements zero-padded to 32.
-__host__ __device__ constexpr int row_bytes(int dtype) { return dtype == FASTNN_I8 ? 32 : 64; }
+// Bytes of one repacked descriptor row: d elements zero-padded to K = 32
+// (d <= 32) or K = 64 (d <= 64) elements of 1 (int8) or 2 (bf16, half) bytes.
+__host__ __device__ constexpr int elem_bytes(int dtype) { return dtype == FASTNN_I8 ? 1 : 2; }
+__host__ __device__ constexpr int row_bytes(int dtype, int d) {
+  return elem_bytes(dtype) * (d <= 32 ? 32 : 64);
+}
 
 // Where the query rows of one nearest-neighbour pass come from.
 //   row id of slot k of pair b:

@@ -13,16 +13,16 @@ namespace fastnn {
 namespace {
 
 // ---------------------------------------------------------------- repack ---
-// One thread per output row. Source rows of d elements (esize bytes each) are
-// copied into 32-element rows (32 B int8 / 64 B bf16) with zero padding, so
-// every row is 16-byte aligned for TMA and the MMA's K extent is exactly 32.
+// One thread per output row. Source rows of d elements (ESIZE bytes each) are
+// copied into RB-byte rows (K = 32 or 64 elements) with zero padding, so every
+// row is 16-byte aligned for TMA and the MMA's K extent is a whole number of
+// 32-byte steps.
 // For int8 maps, `absmax` (if given) receives max |element| over the map
 // (atomicMax), which tells the nearest-neighbour kernel whether every score
 // fits in 16 bits.
-template <int ESIZE>
+template <int ESIZE, int RB>
 __global__ void repack_kernel(const uint8_t* __restrict__ src, int64_t rows, int d,
                               uint8_t* __restrict__ dst, int64_t pad_rows, int* absmax) {
-  constexpr int RB = 32 * ESIZE;
   constexpr int NW = RB / 4;
   const int nbytes = d * ESIZE;
   const bool words = (nbytes % 4) == 0 && (reinterpret_cast<uintptr_t>(src) % 4) == 0;
@@ -186,13 +186,25 @@ int launch_repack(const void* src, int64_t rows, int d, int dtype, void* dst, in
                   int* absmax, cudaStream_t st) {
   const int64_t total = rows + pad_rows;
   if (total <= 0) return FASTNN_OK;
-  if (dtype == FASTNN_I8)
-    repack_kernel<1><<<grid_for(total, 256), 256, 0, st>>>(static_cast<const uint8_t*>(src), rows,
-                                                            d, static_cast<uint8_t*>(dst), pad_rows, absmax);
-  else
-    repack_kernel<2><<<grid_for(total, 256), 256, 0, st>>>(static_cast<const uint8_t*>(src), rows,
-                                                            d, static_cast<uint8_t*>(dst), pad_rows,
-                                                            nullptr);
+  const uint8_t* s8 = static_cast<const uint8_t*>(src);
+  uint8_t* d8 = static_cast<uint8_t*>(dst);
+  const int g = grid_for(total, 256);
+  switch (row_bytes(dtype, d)) {
+    case 32:
+      repack_kernel<1, 32><<<g, 256, 0, st>>>(s8, rows, d, d8, pad_rows, absmax);
+      break;
+    case 64:
+      if (dtype == FASTNN_I8)
+        repack_kernel<1, 64><<<g, 256, 0, st>>>(s8, rows, d, d8, pad_rows, absmax);
+      else
+        repack_kernel<2, 64><<<g, 256, 0, st>>>(s8, rows, d, d8, pad_rows, nullptr);
+      break;
+    case 128:
+      repack_kernel<2, 128><<<g, 256, 0, st>>>(s8, rows, d, d8, pad_rows, nullptr);
+      break;
+    default:
+      return FASTNN_ERR_UNSUPPORTED;
+  }
   FASTNN_CUDA_TRY(cudaGetLastError());
   return FASTNN_OK;
 }

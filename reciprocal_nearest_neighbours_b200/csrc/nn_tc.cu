@@ -14,7 +14,7 @@
 //       columns) of the tile. The score matrix never leaves the SM.
 //   producer warp: gathers the 128 query rows of a tile into shared memory
 //       (swizzled, K-major) and streams kBN-row database tiles with TMA
-//       (cp.async.bulk.tensor, no multicast) into a kStages-deep ring.
+//       (cp.async.bulk.tensor, no multicast) into a 4- or 6-deep ring.
 //   MMA warp (one thread): tcgen05.mma kind::i8 (int8 -> int32, K = 32) or
 //       kind::f16 (bf16 -> fp32, 2 x K = 16) into the two 256-column TMEM
 //       accumulators in turn; tcgen05.commit frees the database stage and
@@ -41,7 +41,11 @@ namespace {
 constexpr int kBM = 128;
 constexpr int kBN = 256;                        // database rows per unit = accumulator columns
 constexpr int kAcc = 2;                         // TMEM accumulators (2 x 256 = 512 columns)
-constexpr int kStages = 6;                      // database ring: 48 KB (int8) / 96 KB (bf16)
+constexpr int kMaxStages = 6;                   // database ring slots laid out in Ctl
+
+// Database ring depth for RB-byte rows: 6 x 256-row tiles (48 KB / 96 KB) for
+// 32- and 64-byte rows, 4 (128 KB) for 128-byte rows.
+__host__ __device__ constexpr int stages_for(int rb) { return rb == 128 ? 4 : 6; }
 constexpr int kGroupWarps = 8;                  // epilogue warps per accumulator
 constexpr int kEpiWarps = kAcc * kGroupWarps;
 constexpr int kProducerWarp = kEpiWarps;
@@ -55,14 +59,15 @@ constexpr int kStashBytes = kEpiWarps * 32 * 32;  // 32 B per epilogue thread
 
 // Barrier slots inside the barrier block.
 constexpr int kBarBFull = 0;
-constexpr int kBarBEmpty = kBarBFull + kStages;
-constexpr int kBarAFull = kBarBEmpty + kStages;
+constexpr int kBarBEmpty = kBarBFull + kMaxStages;
+constexpr int kBarAFull = kBarBEmpty + kMaxStages;
 constexpr int kBarAEmpty = kBarAFull + 2;
 constexpr int kBarAccFull = kBarAEmpty + 2;
 constexpr int kBarAccEmpty = kBarAccFull + kAcc;
 constexpr int kBarDone = kBarAccEmpty + kAcc;
 constexpr int kNumBars = kBarDone + 1;
-static_assert(kStages % kAcc == 0 && (kAcc & (kAcc - 1)) == 0, "issuer g owns stages g, g + kAcc, ...");
+static_assert(stages_for(32) % kAcc == 0 && stages_for(128) % kAcc == 0 && (kAcc & (kAcc - 1)) == 0,
+              "issuer g owns stages g, g + kAcc, ...");
 
 struct Ctl {
   uint64_t bars[kNumBars];
@@ -74,7 +79,7 @@ struct Ctl {
   int64_t m_seg[kAcc];
   int m_st_idx[kAcc], m_par[kAcc];
   uint32_t m_st_phase[kAcc], m_ac_phase[kAcc];
-  int p_last_phase[kStages];
+  int p_last_phase[kMaxStages];
   uint32_t tmem_base;
   int abort_flag;
   int pack16;
@@ -92,7 +97,7 @@ __host__ __device__ constexpr size_t tile_bytes_b(int rb) { return static_cast<s
 __host__ __device__ constexpr size_t ctl_bytes() { return (sizeof(Ctl) + 15) & ~static_cast<size_t>(15); }
 
 size_t smem_bytes(int rb) {
-  return 1024 /* alignment slack */ + 2 * tile_bytes_a(rb) + kStages * tile_bytes_b(rb) +
+  return 1024 /* alignment slack */ + 2 * tile_bytes_a(rb) + stages_for(rb) * tile_bytes_b(rb) +
          ctl_bytes() + kStashBytes;
 }
 
@@ -162,8 +167,8 @@ __device__ __forceinline__ void next_segment(Pos& p, const Ctl* ctl, int batch) 
 }
 
 // Query-tile gather: 32 lanes copy 128 rows of `rb` bytes into a K-major tile
-// with the 32B (rb = 32) or 64B (rb = 64) swizzle the MMA descriptor names:
-// the 16-byte chunk c of row r lands at r * rb + 16 * (c ^ swz(r)).
+// with the 32B / 64B / 128B swizzle (rb = 32 / 64 / 128) the MMA descriptor
+// names: the 16-byte chunk c of row r lands at r * rb + 16 * (c ^ swz(r)).
 template <int RB>
 __device__ __forceinline__ void gather_a(uint8_t* tile, const NNArgs& a, const PhaseQ& q, int b,
                                          int64_t m, int cnt, int lane) {
@@ -185,7 +190,7 @@ __device__ __forceinline__ void gather_a(uint8_t* tile, const NNArgs& a, const P
 #pragma unroll
       for (int c = 0; c < kC; ++c) v[c] = make_uint4(0, 0, 0, 0);
     }
-    const int swz = RB == 32 ? ((r >> 2) & 1) : ((r >> 1) & 3);
+    const int swz = RB == 32 ? ((r >> 2) & 1) : RB == 64 ? ((r >> 1) & 3) : (r & 7);
 #pragma unroll
     for (int c = 0; c < kC; ++c)
       *reinterpret_cast<uint4*>(tile + r * RB + 16 * (c ^ swz)) = v[c];
@@ -206,7 +211,7 @@ struct Epi<FASTNN_I8> {
   static __device__ __forceinline__ uint32_t ord(S s) { return ord_i32(s); }
 };
 
-// bf16 descriptors: fp32 scores.
+// bf16 and half descriptors: fp32 scores.
 template <>
 struct Epi<FASTNN_BF16> {
   using S = float;
@@ -220,6 +225,9 @@ struct Epi<FASTNN_BF16> {
   }
   static __device__ __forceinline__ uint32_t ord(S s) { return ord_f32(s); }
 };
+
+template <>
+struct Epi<FASTNN_F16> : Epi<FASTNN_BF16> {};
 
 // Fold 32 consecutive columns (global index col0 + j) into (best, bidx).
 // Used for the ragged last database tile: `valid` < 32 masks the tail.
@@ -358,7 +366,7 @@ __device__ __forceinline__ void fold_wide(const uint32_t (&r)[NC][32], uint32_t 
 
 struct SmemLayout {
   uint8_t* tileA;  // 2 x kBM x RB query tiles
-  uint8_t* tileB;  // kStages x kBN x RB database tiles
+  uint8_t* tileB;  // stages_for(RB) x kBN x RB database tiles
   Ctl* ctl;
   uint4* stash;    // 32 B per epilogue thread
 };
@@ -371,7 +379,7 @@ __device__ __forceinline__ SmemLayout smem_layout() {
   SmemLayout L;
   L.tileA = base;
   L.tileB = base + 2 * tile_bytes_a(RB);
-  L.ctl = reinterpret_cast<Ctl*>(L.tileB + kStages * tile_bytes_b(RB));
+  L.ctl = reinterpret_cast<Ctl*>(L.tileB + stages_for(RB) * tile_bytes_b(RB));
   L.stash = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(L.ctl) + ctl_bytes());
   return L;
 }
@@ -397,7 +405,7 @@ __device__ __forceinline__ void pipe_setup(Ctl* ctl) {
       ctl->m_ac_phase[g] = 0;
       ctl->m_par[g] = 0;
     }
-    for (int s = 0; s < kStages; ++s) ctl->p_last_phase[s] = -1;
+    for (int s = 0; s < kMaxStages; ++s) ctl->p_last_phase[s] = -1;
     for (int i = 0; i < kNumBars; ++i) {
       uint32_t count = 1;
       if (i >= kBarAFull && i < kBarAFull + 2) count = 32;    // producer lanes
@@ -456,10 +464,11 @@ __device__ void plan_phase(const NNArgs& a, const PhaseQ& q, Ctl* ctl) {
 // One nearest-neighbour phase: plan (thread 0), then each role runs its loop
 // over this CTA's units. Ends with a CTA barrier, after which every MMA of the
 // phase has completed and every result has been merged into a.out_key.
-template <int DT>
+template <int DT, int RB>
 __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const PhaseQ q,
                           const SmemLayout& L, uint32_t tmem, PipeState& ps) {
-  constexpr int RB = row_bytes(DT);
+  constexpr int NS = stages_for(RB);  // database ring depth
+  constexpr int KS = RB / 32;         // MMAs per tile: 32 bytes of K each
   using E = Epi<DT>;
   Ctl* ctl = L.ctl;
   uint8_t* tileA = L.tileA;
@@ -504,7 +513,7 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Pha
             ptx::tma_load_2d(ptx::smem_u32(tileB + st.idx * tile_bytes_b(RB)), tmap_db, 0, row,
                              bar(kBarBFull + st.idx));
             ctl->p_last_phase[st.idx] = static_cast<int>(st.phase);
-            st.next<kStages>();
+            st.next<NS>();
           }
         }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -523,10 +532,11 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Pha
       // issuers sit in different warps, so their per-unit waits and commits
       // overlap.
       if (lane == 0) {
-        constexpr uint32_t kIdesc =
-            DT == FASTNN_I8
-                ? ((2u << 4) | (1u << 7) | (1u << 10) | ((kBN >> 3) << 17) | ((kBM >> 4) << 24))
-                : ((1u << 4) | (1u << 7) | (1u << 10) | ((kBN >> 3) << 17) | ((kBM >> 4) << 24));
+        // Instruction descriptor: accumulator format (S32 / F32), A and B formats
+        // (S8 / BF16 / F16), both K-major, N >> 3, M >> 4.
+        constexpr uint32_t kFmt = DT == FASTNN_I8 ? 1u : DT == FASTNN_BF16 ? 1u : 0u;
+        constexpr uint32_t kIdesc = ((DT == FASTNN_I8 ? 2u : 1u) << 4) | (kFmt << 7) |
+                                    (kFmt << 10) | ((kBN >> 3) << 17) | ((kBM >> 4) << 24);
         const int g = warp - kMmaWarp0;
         Pos p = start;
         bool ok = true;
@@ -555,19 +565,21 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Pha
             ptx::tc_fence_after();
             const uint64_t bdesc =
                 bdesc0 + static_cast<uint64_t>((st_idx * tile_bytes_b(RB)) >> 4);
-            if constexpr (DT == FASTNN_I8) {
-              ptx::mma_i8(d_tmem, adesc, bdesc, kIdesc, 0u);
-            } else {
-              // K = 32 bf16 = two K = 16 steps; the second starts 32 bytes in.
-              ptx::mma_bf16(d_tmem, adesc, bdesc, kIdesc, 0u);
-              ptx::mma_bf16(d_tmem, adesc + 2, bdesc + 2, kIdesc, 1u);
+            // K steps of 32 bytes (32 int8 or 16 16-bit elements); step s
+            // starts 32 * s bytes into the swizzled rows.
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+              if constexpr (DT == FASTNN_I8)
+                ptx::mma_i8(d_tmem, adesc + 2 * ks, bdesc + 2 * ks, kIdesc, ks > 0 ? 1u : 0u);
+              else
+                ptx::mma_bf16(d_tmem, adesc + 2 * ks, bdesc + 2 * ks, kIdesc, ks > 0 ? 1u : 0u);
             }
             ptx::mma_commit(bar(kBarBEmpty + st_idx));
             ptx::mma_commit(bar(kBarAccFull + g));
             ac_phase ^= 1u;
             st_idx += kAcc;
-            if (st_idx >= kStages) {
-              st_idx -= kStages;
+            if (st_idx >= NS) {
+              st_idx -= NS;
               st_phase ^= 1u;
             }
           }
@@ -681,7 +693,7 @@ __device__ __forceinline__ void pipe_teardown(Ctl* ctl, uint32_t tmem, int* stat
     wait_bounded(bar(kBarDone), 0, ctl, status);
   }
   if (warp == kProducerWarp && lane == 0) {
-    for (int s = 0; s < kStages; ++s)
+    for (int s = 0; s < kMaxStages; ++s)
       if (ctl->p_last_phase[s] >= 0)
         wait_bounded(bar(kBarBFull + s), static_cast<uint32_t>(ctl->p_last_phase[s]), ctl, status);
   }
@@ -691,16 +703,15 @@ __device__ __forceinline__ void pipe_teardown(Ctl* ctl, uint32_t tmem, int* stat
   if (warp == 0) ptx::tmem_dealloc(tmem, 512);
 }
 
-template <int DT>
+template <int DT, int RB>
 __global__ void __launch_bounds__(kThreads, 1)
     nn_tc_kernel(const __grid_constant__ CUtensorMap tmap_db, const __grid_constant__ NNArgs a) {
-  constexpr int RB = row_bytes(DT);
   const SmemLayout L = smem_layout<RB>();
   if ((threadIdx.x >> 5) == kProducerWarp && (threadIdx.x & 31) == 0) ptx::prefetch_tmap(&tmap_db);
   pipe_setup(L.ctl);
   const uint32_t tmem = L.ctl->tmem_base;
   PipeState ps;
-  run_phase<DT>(&tmap_db, a, PhaseQ{a.q_index, a.q_count}, L, tmem, ps);
+  run_phase<DT, RB>(&tmap_db, a, PhaseQ{a.q_index, a.q_count}, L, tmem, ps);
   pipe_teardown(L.ctl, tmem, a.status);
 }
 
@@ -748,12 +759,11 @@ __device__ bool grid_sync(const RecArgs& r, uint32_t& target, Ctl* ctl) {
 // a backward pass (matches -> image 1) and the per-pair check/compaction,
 // separated by grid barriers; stops when every pair's frontier is empty or
 // after max_iter rounds.
-template <int DT>
+template <int DT, int RB>
 __global__ void __launch_bounds__(kThreads, 1)
     reciprocal_kernel(const __grid_constant__ CUtensorMap tmap_d2,
                       const __grid_constant__ CUtensorMap tmap_d1,
                       const __grid_constant__ RecArgs r) {
-  constexpr int RB = row_bytes(DT);
   const SmemLayout L = smem_layout<RB>();
   Ctl* ctl = L.ctl;
   if ((threadIdx.x >> 5) == kProducerWarp && (threadIdx.x & 31) == 0) {
@@ -792,9 +802,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   for (int t = 1; ok && t <= r.max_iter; ++t) {
     const int cur = (t - 1) & 1, nxt = t & 1;
-    run_phase<DT>(&tmap_d2, r.fwd, PhaseQ{r.F[cur], r.cnt[cur]}, L, tmem, ps);
+    run_phase<DT, RB>(&tmap_d2, r.fwd, PhaseQ{r.F[cur], r.cnt[cur]}, L, tmem, ps);
     if (!grid_sync(r, target, ctl)) break;
-    run_phase<DT>(&tmap_d1, r.bwd, PhaseQ{nullptr, r.cnt[cur]}, L, tmem, ps);
+    run_phase<DT, RB>(&tmap_d1, r.bwd, PhaseQ{nullptr, r.cnt[cur]}, L, tmem, ps);
     if (!grid_sync(r, target, ctl)) break;
     const FrontierBufs fb{r.F[cur], r.F[nxt], r.cnt[cur], r.cnt[nxt]};
     for (int b = blockIdx.x; b < batch; b += gridDim.x)
@@ -889,7 +899,9 @@ int make_tmap(CUtensorMap* tm, const uint8_t* rows, int64_t total_rows, int rb) 
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = encode(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(rows), dims,
                             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                            rb == 32 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B,
+                            rb == 32   ? CU_TENSOR_MAP_SWIZZLE_32B
+                            : rb == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                       : CU_TENSOR_MAP_SWIZZLE_128B,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? FASTNN_OK : FASTNN_ERR_INVALID;
 }
@@ -914,37 +926,59 @@ int timer_end(int slot, cudaStream_t stream) {
 
 }  // namespace
 
+namespace {
+
+// Kernel instance for (dtype, row bytes), or nullptr for an unsupported pair.
+const void* nn_kernel_for(int dtype, int rb) {
+  if (dtype == FASTNN_I8 && rb == 32) return reinterpret_cast<const void*>(nn_tc_kernel<FASTNN_I8, 32>);
+  if (dtype == FASTNN_I8 && rb == 64) return reinterpret_cast<const void*>(nn_tc_kernel<FASTNN_I8, 64>);
+  if (dtype == FASTNN_BF16 && rb == 64) return reinterpret_cast<const void*>(nn_tc_kernel<FASTNN_BF16, 64>);
+  if (dtype == FASTNN_BF16 && rb == 128) return reinterpret_cast<const void*>(nn_tc_kernel<FASTNN_BF16, 128>);
+  if (dtype == FASTNN_F16 && rb == 64) return reinterpret_cast<const void*>(nn_tc_kernel<FASTNN_F16, 64>);
+  if (dtype == FASTNN_F16 && rb == 128) return reinterpret_cast<const void*>(nn_tc_kernel<FASTNN_F16, 128>);
+  return nullptr;
+}
+
+const void* rec_kernel_for(int dtype, int rb) {
+  if (dtype == FASTNN_I8 && rb == 32) return reinterpret_cast<const void*>(reciprocal_kernel<FASTNN_I8, 32>);
+  if (dtype == FASTNN_I8 && rb == 64) return reinterpret_cast<const void*>(reciprocal_kernel<FASTNN_I8, 64>);
+  if (dtype == FASTNN_BF16 && rb == 64) return reinterpret_cast<const void*>(reciprocal_kernel<FASTNN_BF16, 64>);
+  if (dtype == FASTNN_BF16 && rb == 128) return reinterpret_cast<const void*>(reciprocal_kernel<FASTNN_BF16, 128>);
+  if (dtype == FASTNN_F16 && rb == 64) return reinterpret_cast<const void*>(reciprocal_kernel<FASTNN_F16, 64>);
+  if (dtype == FASTNN_F16 && rb == 128) return reinterpret_cast<const void*>(reciprocal_kernel<FASTNN_F16, 128>);
+  return nullptr;
+}
+
+}  // namespace
+
 int launch_nn_tc(const NNArgs& a, int dtype, int64_t db_total_rows, cudaStream_t stream) {
-  const int rb = row_bytes(dtype);
+  const int rb = row_bytes(dtype, a.d);
   if (db_total_rows < kBN || a.batch < 1 || a.batch > kMaxBatch) return FASTNN_ERR_INVALID;
+  const void* fn = nn_kernel_for(dtype, rb);
+  if (!fn) return FASTNN_ERR_UNSUPPORTED;
   CUtensorMap tm;
   int rc = make_tmap(&tm, a.db_rows, db_total_rows, rb);
   if (rc != FASTNN_OK) return rc;
   int sms = 0;
   if ((rc = sm_count(&sms)) != FASTNN_OK) return rc;
   const size_t smem = smem_bytes(rb);
+  FASTNN_CUDA_TRY(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem)));
+  NNArgs args = a;
+  void* params[] = {&tm, &args};
   const int slot = timer_begin(stream);
   if (slot == -2) return FASTNN_ERR_CUDA;
-  if (dtype == FASTNN_I8) {
-    FASTNN_CUDA_TRY(cudaFuncSetAttribute(nn_tc_kernel<FASTNN_I8>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem)));
-    nn_tc_kernel<FASTNN_I8><<<sms, kThreads, smem, stream>>>(tm, a);
-  } else {
-    FASTNN_CUDA_TRY(cudaFuncSetAttribute(nn_tc_kernel<FASTNN_BF16>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem)));
-    nn_tc_kernel<FASTNN_BF16><<<sms, kThreads, smem, stream>>>(tm, a);
-  }
-  FASTNN_CUDA_TRY(cudaGetLastError());
+  FASTNN_CUDA_TRY(cudaLaunchKernel(fn, dim3(sms), dim3(kThreads), params, smem, stream));
   return timer_end(slot, stream);
 }
 
 int launch_reciprocal(const RecArgs& r, int dtype, int64_t d1_rows, int64_t d2_rows,
                       cudaStream_t stream) {
-  const int rb = row_bytes(dtype);
+  const int rb = row_bytes(dtype, r.fwd.d);
   if (d1_rows < kBN || d2_rows < kBN || r.batch < 1 || r.batch > kMaxBatch)
     return FASTNN_ERR_INVALID;
+  const void* fn = rec_kernel_for(dtype, rb);
+  if (!fn) return FASTNN_ERR_UNSUPPORTED;
   CUtensorMap tm2, tm1;
   int rc = make_tmap(&tm2, r.fwd.db_rows, d2_rows, rb);
   if (rc != FASTNN_OK) return rc;
@@ -952,8 +986,6 @@ int launch_reciprocal(const RecArgs& r, int dtype, int64_t d1_rows, int64_t d2_r
   int sms = 0;
   if ((rc = sm_count(&sms)) != FASTNN_OK) return rc;
   const size_t smem = smem_bytes(rb);
-  const void* fn = dtype == FASTNN_I8 ? reinterpret_cast<const void*>(reciprocal_kernel<FASTNN_I8>)
-                                      : reinterpret_cast<const void*>(reciprocal_kernel<FASTNN_BF16>);
   FASTNN_CUDA_TRY(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem)));
   int per_sm = 0;

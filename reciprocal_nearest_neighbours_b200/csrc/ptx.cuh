@@ -103,7 +103,8 @@ __device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t
       : "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, bf16 x bf16 -> fp32.
+// D[tmem] (+)= A[smem] * B[smem]^T, 16-bit floats (bf16 or half, as the
+// instruction descriptor says) -> fp32.
 __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                          uint32_t idesc, uint32_t accumulate) {
   asm volatile(
@@ -167,13 +168,14 @@ __device__ __forceinline__ void tmem_ld_wait() {
 }
 
 // Shared-memory matrix descriptor for a K-major operand tile whose rows are
-// `row_bytes` (32 or 64) long and stored with the matching 32B / 64B swizzle
-// (8-row groups, consecutive rows): start address, leading offset 16 B
-// (unused for a K extent inside one swizzle atom), stride offset = 8 rows,
-// descriptor version 1, swizzle mode in bits 61..63 (6 = 32B, 4 = 64B).
+// `row_bytes` (32, 64 or 128) long and stored with the matching 32B / 64B /
+// 128B swizzle (8-row groups, consecutive rows): start address, leading
+// offset 16 B (unused for a K extent inside one swizzle atom), stride offset
+// = 8 rows, descriptor version 1, swizzle mode in bits 61..63 (6 = 32B,
+// 4 = 64B, 2 = 128B).
 __device__ __forceinline__ uint64_t smem_desc_kmajor(uint32_t saddr, int row_bytes) {
   const uint64_t sbo = static_cast<uint64_t>(8 * row_bytes) >> 4;
-  const uint64_t mode = row_bytes == 32 ? 6ull : 4ull;
+  const uint64_t mode = row_bytes == 32 ? 6ull : row_bytes == 64 ? 4ull : 2ull;
   return (static_cast<uint64_t>((saddr >> 4) & 0x3FFF)) | (1ull << 16) | (sbo << 32) |
          (1ull << 46) | (mode << 61);
 }

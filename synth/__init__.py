@@ -314,6 +314,14 @@ CONFIGS = {
         seed=BASE_SEED + 4,
         note="one 512x384 pair, d=24, unit-norm bf16; map2 warped map1 plus "
              "N(0,0.05) noise, renormalised, 30% outliers; 8-px grid, max_iter=10"),
+    "pair_512x384_d24_f16": dict(
+        seed=BASE_SEED + 4,
+        note="the bf16 512x384 pair above (same seed, same float maps) stored as "
+             "IEEE half; 8-px grid, max_iter=10"),
+    "pair_512x384_d64_i8": dict(
+        seed=BASE_SEED + 6,
+        note="one 512x384 pair, d=64, int8 uniform in [-16,16], warped as the d=24 "
+             "pair; 8-px grid (3,072 seeds), max_iter=10"),
     "batch16_512x288_d32_i8": dict(
         seed=BASE_SEED + 5,
         note="16 independent 512x288 pairs, d=32, int8 uniform in [-16,16], warped "
@@ -340,6 +348,12 @@ def make_workload(name: str, batch: int | None = None) -> Workload:
                         dense=True, note=cfg["note"])
     if name == "pair_512x384_d24_bf16":
         return Workload(name, [warped_pair_bf16(seed)], subsample=8, max_iter=10,
+                        note=cfg["note"])
+    if name == "pair_512x384_d24_f16":
+        return Workload(name, [warped_pair_bf16(seed, storage="f16")], subsample=8,
+                        max_iter=10, note=cfg["note"])
+    if name == "pair_512x384_d64_i8":
+        return Workload(name, [warped_pair_int8(seed, d=64)], subsample=8, max_iter=10,
                         note=cfg["note"])
     if name == "batch16_512x288_d32_i8":
         nb = 16 if batch is None else batch

@@ -16,13 +16,15 @@ def require_cuda():
         pytest.skip("needs a CUDA device")
 
 
-def to_dev(a: np.ndarray) -> torch.Tensor:
-    """int8 arrays stay int8; uint16 arrays are bfloat16 bit patterns."""
+def to_dev(a: np.ndarray, half: str = "bf16") -> torch.Tensor:
+    """int8 arrays stay int8; uint16 arrays are the bit patterns of bfloat16
+    (``half="bf16"``) or IEEE half (``half="f16"``) descriptors."""
     a = np.ascontiguousarray(a)
     if a.dtype == np.int8:
         return torch.from_numpy(a).cuda()
     if a.dtype == np.uint16:
-        return torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
+        t = torch.from_numpy(a.view(np.int16)).cuda()
+        return t.view(torch.bfloat16 if half == "bf16" else torch.float16)
     raise TypeError(a.dtype)
 
 
@@ -42,7 +44,7 @@ def check_nn_exact(idx_g, score_g, ref: oracle.NNResult):
     assert np.array_equal(score_g.astype(np.int64), ref.score)
 
 
-def check_nn_bf16(idx_g, score_g, q, db, ref: oracle.NNResult, tol=BF16_TOL):
+def check_nn_bf16(idx_g, score_g, q, db, ref: oracle.NNResult, tol=BF16_TOL, dtype="bf16"):
     """Tolerance rule for float descriptors.
 
     The GPU score must be within tol of the exact score of the pair it chose,
@@ -51,7 +53,7 @@ def check_nn_bf16(idx_g, score_g, q, db, ref: oracle.NNResult, tol=BF16_TOL):
     """
     idx_g = idx_g.cpu().numpy().astype(np.int64)
     score_g = score_g.cpu().numpy().astype(np.float64)
-    exact_chosen = oracle.score_of(q, np.arange(len(idx_g)), db, idx_g, "bf16")
+    exact_chosen = oracle.score_of(q, np.arange(len(idx_g)), db, idx_g, dtype)
     assert np.all(np.abs(score_g - exact_chosen) <= tol)
     assert np.all(ref.score - exact_chosen <= tol)
     diff = idx_g != ref.idx

@@ -63,8 +63,14 @@ def test_workspace_sizes(lib):
     assert a >= 2 * (196608 + 256) * 32 + 196608 * 4
     assert ws(fnn.FASTNN_OP_NN, 10, 1000, 24, fnn.FASTNN_I8) > 1000 * 32
     assert ws(fnn.FASTNN_OP_MUTUAL_DENSE, 3072, 3072, 24, fnn.FASTNN_I8) > 2 * 3072 * 40
+    # half descriptors take the bf16 layout; 32 < d <= 64 doubles the repacked rows
+    assert ws(fnn.FASTNN_OP_RECIPROCAL, 196608, 196608, 24, fnn.FASTNN_F16, 1, 3072) == b
+    e = ws(fnn.FASTNN_OP_RECIPROCAL, 196608, 196608, 64, fnn.FASTNN_I8, 1, 3072)
+    assert e == b and e - a >= 2 * 196608 * 32
+    assert ws(fnn.FASTNN_OP_NN, 10, 1000, 48, fnn.FASTNN_BF16) > 1000 * 128
     # unsupported arguments size to 0
-    assert ws(fnn.FASTNN_OP_NN, 10, 10, 33, fnn.FASTNN_I8) == 0
+    assert ws(fnn.FASTNN_OP_NN, 10, 10, 65, fnn.FASTNN_I8) == 0
+    assert ws(fnn.FASTNN_OP_NN, 10, 10, 65, fnn.FASTNN_F16) == 0
     assert ws(fnn.FASTNN_OP_NN, 10, 10, 0, fnn.FASTNN_I8) == 0
     assert ws(fnn.FASTNN_OP_NN, 10, 10, 24, 7) == 0
     assert ws(7, 10, 10, 24, fnn.FASTNN_I8) == 0
@@ -78,7 +84,8 @@ def test_argument_errors_are_reported_on_the_host(lib):
     big = 1 << 30
     I8 = fnn.FASTNN_I8
     # unsupported d / dtype
-    assert lib.fastnn_nn(fake, 4, fake, 4, 33, I8, fake, None, fake, big, None) == -2
+    assert lib.fastnn_nn(fake, 4, fake, 4, 65, I8, fake, None, fake, big, None) == -2
+    assert lib.fastnn_nn(fake, 4, fake, 4, 0, fnn.FASTNN_F16, fake, None, fake, big, None) == -2
     assert lib.fastnn_nn(fake, 4, fake, 4, 24, 5, fake, None, fake, big, None) == -2
     # empty query set is a no-op, even with null pointers
     assert lib.fastnn_nn(None, 0, None, 4, 24, I8, None, None, None, 0, None) == 0

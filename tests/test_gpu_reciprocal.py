@@ -29,9 +29,9 @@ def _cuda():
     require_cuda()
 
 
-def run_gpu(m1, m2, sub, max_iter, capacity=None):
-    d1 = to_dev(m1)
-    d2 = to_dev(m2)
+def run_gpu(m1, m2, sub, max_iter, capacity=None, half="bf16"):
+    d1 = to_dev(m1, half)
+    d2 = to_dev(m2, half)
     pairs, score, count, iters = fastnn_reciprocal(d1, d2, sub, max_iter, capacity=capacity)
     torch.cuda.synchronize()
     return pairs, score, count, iters
@@ -185,7 +185,7 @@ def test_batch16_512x288_full_size():
             assert all(int(u) in kept for u, x in zip(probe, u2) if u == x)
 
 
-def check_fast_bf16(m1, m2, sub, max_iter, gpu=None, tol=BF16_TOL):
+def check_fast_bf16(m1, m2, sub, max_iter, gpu=None, tol=BF16_TOL, dtype="bf16"):
     """Certificate rule for float descriptors.
 
     Each GPU pair (u, v) is approximately reciprocal: the exact best score of
@@ -195,16 +195,17 @@ def check_fast_bf16(m1, m2, sub, max_iter, gpu=None, tol=BF16_TOL):
     """
     H1, W1, d = m1.shape
     H2, W2, _ = m2.shape
-    pairs, score, count, iters = gpu if gpu is not None else run_gpu(m1, m2, sub, max_iter)
+    pairs, score, count, iters = (gpu if gpu is not None
+                                  else run_gpu(m1, m2, sub, max_iter, half=dtype))
     p, s = gpu_pairs(pairs, score, count)
     D1 = m1.reshape(-1, d)
     D2 = m2.reshape(-1, d)
-    exact = oracle.score_of(D1, p[:, 0], D2, p[:, 1], "bf16")
+    exact = oracle.score_of(D1, p[:, 0], D2, p[:, 1], dtype)
     assert np.all(np.abs(s - exact) <= tol)
-    r12 = oracle.nn(D1[p[:, 0]], D2, "bf16")
-    r21 = oracle.nn(D2[p[:, 1]], D1, "bf16")
+    r12 = oracle.nn(D1[p[:, 0]], D2, dtype)
+    r21 = oracle.nn(D2[p[:, 1]], D1, dtype)
     assert np.all(r12.score - exact <= tol) and np.all(r21.score - exact <= tol)
-    ref = oracle.fast_reciprocal(m1, H1, W1, m2, H2, W2, "bf16", sub, max_iter, track_gaps=True)
+    ref = oracle.fast_reciprocal(m1, H1, W1, m2, H2, W2, dtype, sub, max_iter, track_gaps=True)
     got = set(map(tuple, p.tolist()))
     exp = set(map(tuple, ref.pairs.tolist()))
     for u, v in exp - got:
