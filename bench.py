@@ -248,7 +248,7 @@ class ClockSampler:
 # workload and by a hash of the kernel sources it was taken on. A changed
 # kernel reports null until it is captured again.
 TRAFFIC = {
-    "pair_512x384_d24_i8": (12.70e6, "feee733055579d59"),
+    "pair_512x384_d24_i8": (12.69e6, "b4246b055f54aa62"),
 }
 KERNEL_SOURCES = ["reciprocal_nearest_neighbours_b200/csrc/nn_tc.cu",
                   "reciprocal_nearest_neighbours_b200/csrc/frontier_dev.cuh",
