@@ -11,7 +11,10 @@ What the oracle computes, step by step, in the pages' order:
 * ``nn`` -- the nearest neighbour of each query descriptor in a database by
   dot product, argmax_k <q, DB_k>, lowest index on ties ("MASt3R dissection",
   section 3 Napkin Formula, the inference-time reciprocal matching set). The
-  scan itself is the plain C loop in ``oracle.c``.
+  scan itself is the plain C loop in ``oracle.c``. For pointmaps
+  (``dtype="l2"``) it is the nearest 3D point, argmin_k |q - DB_k|^2, lowest
+  index on ties ("DUSt3R / MASt3R explained": pixels match when their
+  predicted 3D points are nearest neighbours in the shared frame).
 * ``dense_mutual`` -- the reciprocal (mutual nearest-neighbour) set
   M = {(i, j) : NN(D1[i], D2) = j and NN(D2[j], D1) = i}
   ("MASt3R dissection", section 1 architecture diagram and section 3; "DUSt3R
@@ -73,6 +76,8 @@ def _load():
         lib.oracle_nn_bf16.restype = ctypes.c_int
         lib.oracle_nn_f16.argtypes = [P, I64, P, I64, ctypes.c_int, P, P, P, ctypes.c_int]
         lib.oracle_nn_f16.restype = ctypes.c_int
+        lib.oracle_nn_l2.argtypes = [P, I64, P, I64, ctypes.c_int, P, P, P, ctypes.c_int]
+        lib.oracle_nn_l2.restype = ctypes.c_int
         lib.oracle_half_to_double.argtypes = [ctypes.c_uint16]
         lib.oracle_half_to_double.restype = ctypes.c_double
         _lib = lib
@@ -90,15 +95,17 @@ def _ptr(a: np.ndarray) -> int:
 @dataclass
 class NNResult:
     idx: np.ndarray  # int32 [nq]
-    score: np.ndarray  # int64 (int8 descriptors) or float64 (bf16) [nq]
-    second: np.ndarray | None = None  # float64 runner-up score (bf16 only)
+    score: np.ndarray  # int64 (int8), float64 (bf16, f16), float64 squared distance (l2) [nq]
+    second: np.ndarray | None = None  # float64 runner-up (float types; for l2 the 2nd smallest)
 
 
 def nn(q: np.ndarray, db: np.ndarray, dtype: str, nthreads: int | None = None) -> NNResult:
     """Nearest neighbour of every row of ``q`` among the rows of ``db``.
 
     ``q`` is [nq, d], ``db`` is [ndb, d]; int8 arrays for ``dtype == "i8"``,
-    uint16 bit patterns of bfloat16 (``"bf16"``) or IEEE half (``"f16"``).
+    uint16 bit patterns of bfloat16 (``"bf16"``) or IEEE half (``"f16"``),
+    float32 points with d <= 3 for ``"l2"`` (nearest by Euclidean distance;
+    ``score`` is then the squared distance, lower is better).
     """
     lib = _load()
     nthreads = default_threads() if nthreads is None else nthreads
@@ -122,11 +129,32 @@ def nn(q: np.ndarray, db: np.ndarray, dtype: str, nthreads: int | None = None) -
         rc = fn(_ptr(q), nq, _ptr(db), ndb, d, _ptr(idx), _ptr(score), _ptr(second), nthreads)
         assert rc == 0
         return NNResult(idx, score, second)
+    if dtype == "l2":
+        assert q.dtype == np.float32 and db.dtype == np.float32 and d <= 3
+        d2 = np.empty(nq, dtype=np.float64)
+        second = np.empty(nq, dtype=np.float64)
+        rc = lib.oracle_nn_l2(_ptr(q), nq, _ptr(db), ndb, d, _ptr(idx), _ptr(d2), _ptr(second),
+                              nthreads)
+        assert rc == 0
+        return NNResult(idx, d2, second)
     raise ValueError(dtype)
 
 
+def margin(r: NNResult, dtype: str) -> np.ndarray:
+    """How far each query's winner is ahead of its runner-up (>= 0; 0 on a tie).
+
+    Scores are maximised for the descriptor types and squared distances are
+    minimised for ``"l2"``.
+    """
+    return r.second - r.score if dtype == "l2" else r.score - r.second
+
+
 def score_of(D1: np.ndarray, i: np.ndarray, D2: np.ndarray, j: np.ndarray, dtype: str) -> np.ndarray:
-    """Exact scores <D1[i], D2[j]> for paired index arrays (int64 or float64)."""
+    """Exact scores <D1[i], D2[j]> for paired index arrays (int64 or float64);
+    for ``"l2"`` the squared distances |D1[i] - D2[j]|^2 in float64."""
+    if dtype == "l2":
+        diff = D1[i].astype(np.float64) - D2[j].astype(np.float64)
+        return (diff * diff).sum(axis=1)
     if dtype == "i8":
         return (D1[i].astype(np.int64) * D2[j].astype(np.int64)).sum(axis=1)
     if dtype == "f16":
@@ -184,10 +212,11 @@ def fast_reciprocal(D1: np.ndarray, H1: int, W1: int, D2: np.ndarray, H2: int, W
     taken as a set. Walks still open after ``max_iter`` rounds are dropped.
 
     ``first_seen[t-1]`` counts the members of F_t that appear in no earlier
-    frontier. With ``track_gaps`` (bf16), ``min_gap[u]`` for a kept pixel u
-    is, over all walks that end at u, the largest value of the smallest top-2
-    score gap met on that walk (forward and backward steps, u's own included):
-    when it is below a tolerance, every walk to u passes a near-tie.
+    frontier. With ``track_gaps`` (float types), ``min_gap[u]`` for a kept
+    pixel u is, over all walks that end at u, the largest value of the
+    smallest top-2 margin (``margin``) met on that walk (forward and backward
+    steps, u's own included): when it is below a tolerance, every walk to u
+    passes a near-tie. For ``"l2"`` the scores kept are squared distances.
     """
     D1 = D1.reshape(H1 * W1, -1)
     D2 = D2.reshape(H2 * W2, -1)
@@ -207,14 +236,15 @@ def fast_reciprocal(D1: np.ndarray, H1: int, W1: int, D2: np.ndarray, H2: int, W
         seen.update(F)
         fwd = nn(D1[np.array(F)], D2, dtype, nthreads)
         bwd = nn(D2[fwd.idx], D1, dtype, nthreads)
+        if track_gaps:
+            fm, bm = margin(fwd, dtype), margin(bwd, dtype)
         nxt_gap = {}
         for k, u in enumerate(F):
             v = int(fwd.idx[k])
             u2 = int(bwd.idx[k])
             g = np.inf
             if track_gaps:
-                g = min(chain_gap[u], fwd.score[k] - fwd.second[k],
-                        bwd.score[k] - bwd.second[k])
+                g = min(chain_gap[u], fm[k], bm[k])
             if u2 == u:
                 kept[u] = (v, fwd.score[k])
                 kept_gap[u] = max(kept_gap.get(u, -np.inf), g)

@@ -23,6 +23,15 @@
  * k other than the chosen one; equal to the best when the best is tied),
  * which the float tolerance rule needs.
  *
+ * Pointmaps ("DUSt3R / MASt3R explained", the paragraph on recovering the
+ * cameras: two pixels match when their predicted 3D points are nearest
+ * neighbours in the shared frame): oracle_nn_l2 returns, for every query
+ * point a, argmin_k |a - DB_k|^2 over float32 points of d <= 3 coordinates,
+ * again by a linear scan that replaces the running best only on a STRICTLY
+ * smaller distance (lowest index on ties). Each coordinate difference of two
+ * float32 values is exact in double for the magnitudes pointmaps hold, and
+ * the squared distance is summed in double.
+ *
  * Queries are independent, so the outer loop may run on several threads; the
  * per-query scan is the plain sequential loop above either way.
  */
@@ -138,6 +147,46 @@ int oracle_nn_f16(const uint16_t *q, int64_t nq, const uint16_t *db,
 {
     return nn_f16_like(q, nq, db, ndb, d, out_idx, out_score, out_second,
                        nthreads, f16_to_double);
+}
+
+int oracle_nn_l2(const float *q, int64_t nq, const float *db, int64_t ndb,
+                 int d, int32_t *out_idx, double *out_d2, double *out_second,
+                 int nthreads)
+{
+    if (nq < 0 || ndb <= 0 || d <= 0 || d > 3)
+        return -1;
+    (void)nthreads;
+#pragma omp parallel for schedule(dynamic, 16) num_threads(nthreads > 0 ? nthreads : 1)
+    for (int64_t i = 0; i < nq; ++i) {
+        const float *qi = q + i * (int64_t)d;
+        double best = 0.0, second = 0.0;
+        int32_t best_k = -1;
+        int have_second = 0;
+        for (int64_t k = 0; k < ndb; ++k) {
+            const float *dk = db + k * (int64_t)d;
+            double s = 0.0;
+            for (int c = 0; c < d; ++c) {
+                const double diff = (double)qi[c] - (double)dk[c];
+                s += diff * diff;
+            }
+            if (best_k < 0) {
+                best = s;
+                best_k = (int32_t)k;
+            } else if (s < best) {
+                second = best;
+                have_second = 1;
+                best = s;
+                best_k = (int32_t)k;
+            } else if (!have_second || s < second) {
+                second = s;
+                have_second = 1;
+            }
+        }
+        out_idx[i] = best_k;
+        out_d2[i] = best;
+        out_second[i] = have_second ? second : 1.0e300;
+    }
+    return 0;
 }
 
 /* Exposed for the oracle's own tests (exhaustive check of the conversion). */

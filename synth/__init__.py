@@ -17,8 +17,13 @@ of Simple Fast Space-Efficient Statistically Good Algorithms for Random Number
 Generation", 2014), seeded with the integers listed in ``CONFIGS``.
 
 Layout of every map: row-major ``[H, W, d]`` (pixel index p = y * W + x),
-``int8`` for integer descriptors, ``uint16`` bit patterns of bfloat16 for float
-descriptors.
+``int8`` for integer descriptors, ``uint16`` bit patterns of bfloat16 or IEEE
+half for float descriptors, ``float32`` for pointmaps (d = 3).
+
+Pointmaps stand in for DUSt3R's per-pixel 3D points: both views' points in the
+first camera's frame ("DUSt3R / MASt3R explained", the pointmap and
+coordinate-frame paragraphs), so matched pixels of the two views carry nearly
+the same point.
 """
 
 from __future__ import annotations
@@ -35,6 +40,7 @@ __all__ = [
     "tiny_permuted_pair",
     "warped_pair_int8",
     "warped_pair_bf16",
+    "pointmap_pair",
     "planted_sign_pair",
     "random_int8_pair",
     "f64_to_bf16_bits",
@@ -57,7 +63,7 @@ class PairMaps:
     desc1: np.ndarray  # [H1, W1, d]
     desc2: np.ndarray  # [H2, W2, d]
     gt_src: np.ndarray  # [H2 * W2] int64
-    dtype: str  # "i8" or "bf16"
+    dtype: str  # "i8", "bf16", "f16" or "l2" (float32 pointmaps)
 
     @property
     def H1(self) -> int:
@@ -251,6 +257,44 @@ def warped_pair_bf16(seed: int, H: int = 384, W: int = 512, d: int = 24,
     return PairMaps(cvt(m1).reshape(H, W, d), cvt(m2).reshape(H, W, d), gt, storage)
 
 
+def pointmap_pair(seed: int, H: int = 384, W: int = 512, noise: float = 0.002,
+                  outlier_frac: float = 0.3) -> PairMaps:
+    """Two float32 pointmaps of one smooth surface in the first camera's frame.
+
+    View 1: pinhole rays (focal 0.9 W px, principal point at the centre) hit a
+    depth surface z(x, y) = 3 + 0.6 y / H + a seeded sum of four low-frequency
+    sinusoids of amplitude up to 0.15 (metres). View 2: the warp generator of
+    the descriptor pairs picks each pixel's source pixel in view 1 and the
+    point is that view-1 point plus N(0, noise * z) per coordinate (regression
+    blur); a seeded outlier_frac of the pixels, plus those whose source fell
+    outside view 1, get fresh points uniform in the bounding box of view 1.
+    """
+    rng = np.random.Generator(np.random.PCG64(seed))
+    n = H * W
+    ys, xs = np.meshgrid(np.arange(H, dtype=np.float64), np.arange(W, dtype=np.float64),
+                         indexing="ij")
+    f = 0.9 * W
+    z = 3.0 + 0.6 * ys / H
+    for _ in range(4):
+        kx, ky = rng.uniform(0.5, 3.0, size=2)
+        ph = rng.uniform(0, 2 * np.pi)
+        z = z + rng.uniform(0.03, 0.15) * np.sin(2 * np.pi * (kx * xs / W + ky * ys / H) + ph)
+    p1 = np.stack([(xs - (W - 1) / 2.0) / f * z, (ys - (H - 1) / 2.0) / f * z, z],
+                  axis=-1).reshape(n, 3)
+    src = _warp_sources(rng, H, W)
+    p2 = p1[np.maximum(src, 0)]
+    p2 = p2 + noise * p2[:, 2:3] * rng.standard_normal((n, 3))
+    k = int(round(outlier_frac * n))
+    out = np.zeros(n, dtype=bool)
+    out[rng.choice(n, size=k, replace=False)] = True
+    out |= src < 0
+    lo, hi = p1.min(axis=0), p1.max(axis=0)
+    p2[out] = rng.uniform(lo, hi, size=(int(out.sum()), 3))
+    gt = np.where(out, -1, src)
+    return PairMaps(p1.astype(np.float32).reshape(H, W, 3),
+                    p2.astype(np.float32).reshape(H, W, 3), gt, "l2")
+
+
 def planted_sign_pair(seed: int, H: int, W: int, d: int, c: int = 8,
                       redraw_frac: float = 0.2) -> PairMaps:
     """Sign-vector maps with a planted permutation.
@@ -322,6 +366,13 @@ CONFIGS = {
         seed=BASE_SEED + 6,
         note="one 512x384 pair, d=64, int8 uniform in [-16,16], warped as the d=24 "
              "pair; 8-px grid (3,072 seeds), max_iter=10"),
+    "pair_512x384_pts3_f32": dict(
+        seed=BASE_SEED + 7,
+        note="one 512x384 pair of float32 pointmaps (d=3, metres, camera-1 frame): "
+             "a smooth random depth surface at 3-3.6 m seen by view 1; view 2 the "
+             "warp generator's sources with N(0, 0.002 z) noise and 30% outliers "
+             "uniform in the scene's bounding box; nearest 3D point by Euclidean "
+             "distance; 8-px grid (3,072 seeds), max_iter=10"),
     "batch16_512x288_d32_i8": dict(
         seed=BASE_SEED + 5,
         note="16 independent 512x288 pairs, d=32, int8 uniform in [-16,16], warped "
@@ -355,6 +406,8 @@ def make_workload(name: str, batch: int | None = None) -> Workload:
     if name == "pair_512x384_d64_i8":
         return Workload(name, [warped_pair_int8(seed, d=64)], subsample=8, max_iter=10,
                         note=cfg["note"])
+    if name == "pair_512x384_pts3_f32":
+        return Workload(name, [pointmap_pair(seed)], subsample=8, max_iter=10, note=cfg["note"])
     if name == "batch16_512x288_d32_i8":
         nb = 16 if batch is None else batch
         pairs = [warped_pair_int8(seed + 1000 * b, H=288, W=512, d=32)

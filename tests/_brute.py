@@ -9,6 +9,9 @@ running scan, so that a slip in one is caught by the other:
   and ties-or-beats every k > j in row i, and i does the same in column j.
 * ``walks``: follows every seed's walk u -> NN21(NN12(u)) on its own, without
   frontiers or sets, and reads the fast scheme's result off the walks.
+* ``nn_l2_by_definition``: for pointmaps, the lowest index among the points at
+  the minimal squared Euclidean distance (the minimal set first, then its
+  minimum index).
 """
 
 from __future__ import annotations
@@ -39,13 +42,19 @@ def mutual_by_quantifiers(D1, D2):
     return out
 
 
-def walk_step(u, D1, D2):
-    v, s = nn_by_definition(D1[u], D2)
-    u2, _ = nn_by_definition(D2[v], D1)
+def nn_l2_by_definition(q, db):
+    dist = [sum((float(a) - float(b)) ** 2 for a, b in zip(q, row)) for row in db]
+    m = min(dist)
+    return min(k for k, s in enumerate(dist) if s == m), m
+
+
+def walk_step(u, D1, D2, nn=nn_by_definition):
+    v, s = nn(D1[u], D2)
+    u2, _ = nn(D2[v], D1)
     return v, s, u2
 
 
-def walks(seeds, D1, D2, max_iter):
+def walks(seeds, D1, D2, max_iter, nn=nn_by_definition):
     """Per-seed walks. Returns (kept set of (u, v, s), list of walks).
 
     A seed's walk visits u_0 = seed, u_1, ... with u_{t+1} = NN21(NN12(u_t));
@@ -59,7 +68,7 @@ def walks(seeds, D1, D2, max_iter):
         nodes, scores = [u], []
         fixed = None
         for t in range(max_iter):
-            v, s, u2 = walk_step(u, D1, D2)
+            v, s, u2 = walk_step(u, D1, D2, nn)
             scores.append(s)
             if u2 == u:
                 fixed = (u, v, s)
