@@ -41,6 +41,8 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 METRIC = "reciprocal matches/sec and pairs/sec at 512×384 d=24; tensor-pipe % of peak"
+# FP32 fused multiply-add peak of one B200: 148 SMs x 128 lanes x 2 flop x 1.965 GHz.
+FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 UNIT = "matches/s"
 DEFAULT_WORKLOAD = "pair_512x384_d24_i8"
 L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
@@ -68,8 +70,10 @@ def dist_env():
 def metric_for(name):
     if name == DEFAULT_WORKLOAD:
         return METRIC
-    if name.startswith("dense"):
+    if name == "dense_512x384_d24_i8":
         return "dense mutual nearest-neighbour pairs/sec at 512×384 d=24 (all 196,608 pixels)"
+    if name.startswith("dense"):
+        return f"dense mutual nearest-neighbour pairs/sec, workload {name}"
     return f"reciprocal matches/sec, workload {name}"
 
 
@@ -81,6 +85,8 @@ def load_workload(name, rank):
     seed = synth.CONFIGS[name]["seed"] + 7919 * rank
     if name.startswith("batch16"):
         w.pairs = [synth.warped_pair_int8(seed + 1000 * b, H=288, W=512, d=32) for b in range(16)]
+    elif name.endswith("pts3_f32"):
+        w.pairs = [synth.pointmap_pair(seed)]
     elif name.endswith("bf16") or name.endswith("f16"):
         w.pairs = [synth.warped_pair_bf16(seed, storage=w.pairs[0].dtype)]
     elif name.startswith("tiny"):
@@ -93,7 +99,8 @@ def load_workload(name, rank):
 def config_dict(w, extra=None):
     p = w.pairs[0]
     c = {"workload": w.name, "image": f"{p.W1}x{p.H1}", "d": p.d,
-         "descriptor": {"bf16": "bf16 unit-norm", "f16": "IEEE half unit-norm"}.get(p.dtype, "int8"),
+         "descriptor": {"bf16": "bf16 unit-norm", "f16": "IEEE half unit-norm",
+                        "l2": "float32 3D pointmap, Euclidean distance"}.get(p.dtype, "int8"),
          "pairs_per_rank_per_step": w.batch,
          "parallelism": "pair-parallel replicas, no collective",
          "l2": "flushed between timed steps (256 MiB write)"}
@@ -303,9 +310,11 @@ def run_ours(args, rank, world, local):
     H2, W2, _ = p0.desc2.shape
     N1, N2 = H1 * W1, H2 * W2
     i8 = p0.dtype == "i8"
-    code = {"i8": fnn.FASTNN_I8, "bf16": fnn.FASTNN_BF16, "f16": fnn.FASTNN_F16}[p0.dtype]
+    code = {"i8": fnn.FASTNN_I8, "bf16": fnn.FASTNN_BF16, "f16": fnn.FASTNN_F16,
+            "l2": fnn.FASTNN_F32_L2}[p0.dtype]
     sdt = torch.int32 if i8 else torch.float32
-    esize = 1 if i8 else 2
+    l2 = p0.dtype == "l2"
+    esize = 1 if i8 else 4 if l2 else 2
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
@@ -362,9 +371,10 @@ def run_ours(args, rank, world, local):
     assert fnn.fastnn_device_status(ws) == 0
     matches = int(out_count.cpu().sum())
     if w.dense:
-        macs_per_step = 2 * N1 * N2 * d
+        pairs_per_step = 2 * N1 * N2
     else:
-        macs_per_step = int(out_front.cpu().sum()) * (N1 + N2) * d
+        pairs_per_step = int(out_front.cpu().sum()) * (N1 + N2)
+    macs_per_step = pairs_per_step * d
 
     # ---- device-timed region ------------------------------------------------
     uuid = None
@@ -427,30 +437,51 @@ def run_ours(args, rank, world, local):
         pairs_per_s = world * B * K / (total_ms / 1e3)
         peaks, src = measured_peaks()
         bf16_peak = float(peaks["bf16_tflops"])
-        peak = 2.0 * bf16_peak if i8 else bf16_peak  # dense int8 = 2 x bf16 (nominal ratio)
-        achieved = 2.0 * macs_per_step * K / (nn_ms / 1e3) / 1e12 if nn_ms > 0 else None
+        if l2:
+            # Pointmaps: 3 fused multiply-adds per (query, point) pair on the
+            # FP32 pipe; peak = 148 SMs x 128 FMA lanes x 2 flop x 1.965 GHz.
+            peak = FP32_FMA_TFLOPS
+            achieved = 6.0 * pairs_per_step * K / (nn_ms / 1e3) / 1e12 if nn_ms > 0 else None
+        else:
+            peak = 2.0 * bf16_peak if i8 else bf16_peak  # dense int8 = 2 x bf16 (nominal ratio)
+            achieved = 2.0 * macs_per_step * K / (nn_ms / 1e3) / 1e12 if nn_ms > 0 else None
         bytes_in = (N1 + N2) * d * esize * B
         bytes_out = int(hp_count.numel() * 4 + hp_pairs.numel() * 4 + hp_score.numel() * 4)
-        kname = ("nn_tc_kernel (tcgen05 argmax-GEMM, one launch per direction)" if w.dense else
-                 "reciprocal_kernel (persistent: seeds, tcgen05 forward and backward passes, "
-                 "per-pair compaction)")
+        if l2:
+            kname = ("nn_l2_kernel (FP32 FFMA2 nearest point, one launch per direction)"
+                     if w.dense else
+                     "reciprocal_l2_kernel (persistent: seeds, FP32 FFMA2 forward and backward "
+                     "passes, per-pair compaction)")
+        else:
+            kname = ("nn_tc_kernel (tcgen05 argmax-GEMM, one launch per direction)" if w.dense else
+                     "reciprocal_kernel (persistent: seeds, tcgen05 forward and backward passes, "
+                     "per-pair compaction)")
+        if l2:
+            peak_source = ("derived: FP32 FMA pipe, 148 SMs x 128 lanes x 2 flop x 1.965 GHz "
+                           "(clocks.max.sm)")
+            ops = (f"3 FMA = 6 flop per (query, point) pair: {pairs_per_step:.4g} pairs "
+                   f"per step")
+        else:
+            peak_source = (f"{src}: bf16_tflops {bf16_peak}" +
+                           (" x 2 (int8 = 2 x bf16, nominal ratio)" if i8 else ""))
+            ops = f"2 x useful MACs (d = {d}) per step: {macs_per_step:.4g} MAC"
         line = {
             "metric": metric_for(w.name), "value": value, "unit": UNIT, "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": total_ms / K,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": {"i8": "int8", "bf16": "bf16", "f16": "f16"}[p0.dtype], "data": "synthetic",
+            "dtype": {"i8": "int8", "bf16": "bf16", "f16": "f16", "l2": "f32"}[p0.dtype],
+            "data": "synthetic",
             "config": config_dict(w),
             "pairs_per_s": pairs_per_s,
             "matches_per_step_rank0": matches,
             "roofline": {
-                "bound": "tensor", "kernel": kname,
+                "bound": "alu" if l2 else "tensor", "kernel": kname,
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": (achieved / peak) if achieved else None,
                 "traffic": traffic_for(w.name),
                 "traffic_unit": "bytes per launch (ncu dram read + write)",
-                "peak_source": (f"{src}: bf16_tflops {bf16_peak}" +
-                                (" x 2 (int8 = 2 x bf16, nominal ratio)" if i8 else "")),
-                "ops": f"2 x useful MACs (d = {d}) per step: {macs_per_step:.4g} MAC",
+                "peak_source": peak_source,
+                "ops": ops,
                 "kernel_ms_per_step": nn_ms / K, "kernel_launches": nn_launches,
                 "kernel_share_of_step": nn_ms / total_ms if total_ms else None,
             },

@@ -10,6 +10,11 @@
  *   A reciprocal match is a pair (i, j) with NN(D1[i], D2) = j and
  *   NN(D2[j], D1) = i ("MASt3R dissection", section 1 architecture diagram
  *   and section 3).
+ *   Pointmaps (dtype FASTNN_F32_L2): rows are 3D points and the nearest
+ *   neighbour is the nearest point, argmin_k |q - db_k|^2, lowest k on ties
+ *   ("DUSt3R / MASt3R explained", the paragraph on recovering the cameras:
+ *   pixels match when their predicted 3D points are nearest neighbours in
+ *   the shared frame). The same reciprocal and fast schemes apply.
  *
  * Conventions shared by every entry point
  *   - Every data pointer is a DEVICE pointer owned by the caller. The library
@@ -22,6 +27,13 @@
  *     dtype FASTNN_BF16 / FASTNN_F16: bfloat16 / IEEE half descriptors (raw
  *     16-bit patterns), float32 scores (fp32 accumulation of exact products).
  *     1 <= d <= 64 for all three (d <= 32 runs one 32-element K step).
+ *     dtype FASTNN_F32_L2: float32 points, 1 <= d <= 3 (DUSt3R pointmaps
+ *     have d = 3); scores are float32 SQUARED DISTANCES (lower is nearer),
+ *     computed from the coordinate differences of the reported pair. Inputs
+ *     must be finite. Selection is computed in fp32 as the maximum of
+ *     2<q, p> - |p|^2, which orders points like -|q - p|^2; two points whose
+ *     exact squared distances differ by less than about 2^-20 (|q| + max|p|)^2
+ *     may be ordered either way.
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the
  *     legacy default stream). The host blocks only in fastnn_device_status().
  *   - Return value: FASTNN_OK, or a negative fastnn_status describing an
@@ -47,13 +59,18 @@ typedef struct CUstream_st *fastnn_stream_t; /* same type as cudaStream_t */
 typedef enum {
     FASTNN_OK = 0,
     FASTNN_ERR_INVALID = -1,     /* bad pointer, size, alignment or argument */
-    FASTNN_ERR_UNSUPPORTED = -2, /* d (1..64) or dtype outside what the kernels take */
+    FASTNN_ERR_UNSUPPORTED = -2, /* d (1..64; 1..3 for pointmaps) or dtype not taken */
     FASTNN_ERR_CAPACITY = -3,    /* output capacity or workspace too small */
     FASTNN_ERR_CUDA = -4,        /* a CUDA runtime call or launch failed */
     FASTNN_ERR_TIMEOUT = -5      /* a device-side bounded wait ran out */
 } fastnn_status;
 
-typedef enum { FASTNN_I8 = 0, FASTNN_BF16 = 1, FASTNN_F16 = 2 } fastnn_dtype;
+typedef enum {
+    FASTNN_I8 = 0,     /* int8 descriptors, dot product, int32 scores */
+    FASTNN_BF16 = 1,   /* bfloat16 descriptors, dot product, float32 scores */
+    FASTNN_F16 = 2,    /* IEEE half descriptors, dot product, float32 scores */
+    FASTNN_F32_L2 = 3  /* float32 3D points, Euclidean distance, float32 squared distances */
+} fastnn_dtype;
 
 typedef enum {
     FASTNN_OP_NN = 0,
@@ -78,8 +95,9 @@ size_t fastnn_workspace_size(int op, int64_t n1, int64_t n2, int d, int dtype,
 /*
  * fastnn_nn -- nearest neighbour of every query row in a database.
  *   For i < nq: out_idx[i] = argmax_k <q[i], db[k]> (lowest k on ties),
- *   out_score[i] = that score (int32 for FASTNN_I8, float for FASTNN_BF16;
- *   out_score may be NULL). This is the primitive of both matching schemes
+ *   out_score[i] = that score (int32 for FASTNN_I8, float for the float
+ *   types; out_score may be NULL). For FASTNN_F32_L2, out_idx[i] is the
+ *   nearest point and out_score[i] its squared distance. This is the primitive of both matching schemes
  *   ("MASt3R dissection", section 3, argmax of dot products).
  *   q: [nq][d], db: [ndb][d]; nq >= 0, ndb >= 1; nq == 0 is a no-op.
  */

@@ -13,6 +13,7 @@ from __future__ import annotations
 from ._lib import (  # noqa: F401
     FASTNN_BF16,
     FASTNN_F16,
+    FASTNN_F32_L2,
     FASTNN_I8,
     FASTNN_OP_MUTUAL_DENSE,
     FASTNN_OP_MUTUAL_FROM_NN,

@@ -13,6 +13,7 @@ _LIB_PATH = os.path.join(HERE, "libfastnn.so")
 FASTNN_I8 = 0
 FASTNN_BF16 = 1
 FASTNN_F16 = 2
+FASTNN_F32_L2 = 3
 FASTNN_OP_NN = 0
 FASTNN_OP_RECIPROCAL = 1
 FASTNN_OP_MUTUAL_DENSE = 2
@@ -87,7 +88,10 @@ def _dtype_code(t: torch.Tensor) -> int:
         return FASTNN_BF16
     if t.dtype == torch.float16:
         return FASTNN_F16
-    raise TypeError(f"descriptors must be int8, bfloat16 or float16, got {t.dtype}")
+    if t.dtype == torch.float32:
+        return FASTNN_F32_L2
+    raise TypeError(f"descriptors must be int8, bfloat16 or float16 (dot product) or float32 "
+                    f"3D points (Euclidean distance), got {t.dtype}")
 
 
 def _score_dtype(code: int):
@@ -133,7 +137,9 @@ def fastnn_nn(q: torch.Tensor, db: torch.Tensor, out_idx=None, out_score=None,
     """Nearest neighbour of each row of ``q`` [nq, d] among rows of ``db`` [ndb, d].
 
     Returns ``(idx int32 [nq], score [nq])`` (int32 scores for int8
-    descriptors, float32 for bfloat16 and float16).
+    descriptors, float32 for bfloat16 and float16). float32 inputs are 3D
+    points (d <= 3): the nearest point by Euclidean distance, with its
+    squared distance as the score.
     """
     _need_cuda(q, db)
     code = _dtype_code(q)

@@ -12,8 +12,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libfastnn.so")
-SOURCES = ["api.cu", "nn_tc.cu", "frontier.cu", "noalloc.cu"]
-HEADERS = ["common.cuh", "ptx.cuh", "nn_tc.cuh", "frontier.cuh", "frontier_dev.cuh"]
+SOURCES = ["api.cu", "nn_tc.cu", "l2_nn.cu", "frontier.cu", "noalloc.cu"]
+HEADERS = ["common.cuh", "ptx.cuh", "nn_tc.cuh", "l2_nn.cuh", "frontier.cuh", "frontier_dev.cuh"]
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 
 

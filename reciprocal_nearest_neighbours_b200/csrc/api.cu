@@ -5,6 +5,7 @@
 
 #include "common.cuh"
 #include "frontier.cuh"
+#include "l2_nn.cuh"
 #include "nn_tc.cuh"
 
 using namespace fastnn;
@@ -41,8 +42,11 @@ struct Carver {
   }
 };
 
-bool dtype_ok(int dtype) { return dtype == FASTNN_I8 || dtype == FASTNN_BF16 || dtype == FASTNN_F16; }
-bool d_ok(int d) { return d >= 1 && d <= 64; }
+bool dtype_ok(int dtype) {
+  return dtype == FASTNN_I8 || dtype == FASTNN_BF16 || dtype == FASTNN_F16 ||
+         dtype == FASTNN_F32_L2;
+}
+bool d_ok(int d, int dtype) { return d >= 1 && d <= (dtype == FASTNN_F32_L2 ? 3 : 64); }
 
 struct NNLayout {
   int* status;
@@ -124,7 +128,7 @@ extern "C" {
 
 size_t fastnn_workspace_size(int op, int64_t n1, int64_t n2, int d, int dtype, int batch,
                              int64_t max_queries) {
-  if (!dtype_ok(dtype) || !d_ok(d) || n1 < 0 || n2 < 1) return 0;
+  if (!dtype_ok(dtype) || !d_ok(d, dtype) || n1 < 0 || n2 < 1) return 0;
   Carver c{nullptr};
   switch (op) {
     case FASTNN_OP_NN:
@@ -150,7 +154,7 @@ size_t fastnn_workspace_size(int op, int64_t n1, int64_t n2, int d, int dtype, i
 int fastnn_nn(const void* q, int64_t nq, const void* db, int64_t ndb, int d, int dtype,
               int32_t* out_idx, void* out_score, void* workspace, size_t workspace_bytes,
               fastnn_stream_t stream) {
-  if (!dtype_ok(dtype) || !d_ok(d)) return FASTNN_ERR_UNSUPPORTED;
+  if (!dtype_ok(dtype) || !d_ok(d, dtype)) return FASTNN_ERR_UNSUPPORTED;
   if (nq < 0 || ndb < 1 || nq > INT32_MAX || ndb > INT32_MAX - kPadRows) return FASTNN_ERR_INVALID;
   if (nq == 0) return FASTNN_OK;
   if (!q || !db || !out_idx || !workspace || !aligned(workspace, kAlign)) return FASTNN_ERR_INVALID;
@@ -176,6 +180,12 @@ int fastnn_nn(const void* q, int64_t nq, const void* db, int64_t ndb, int d, int
   a.d = d;
   a.q_absmax = L.status + 1;
   a.db_absmax = L.status + 2;
+  if (dtype == FASTNN_F32_L2) {
+    FASTNN_TRY(launch_nn_l2(a, st));
+    return launch_decode(L.keys, nq, dtype, out_idx, out_score, st,
+                         reinterpret_cast<const float4*>(L.qrep),
+                         reinterpret_cast<const float4*>(L.dbrep), ndb);
+  }
   FASTNN_TRY(launch_nn_tc(a, dtype, ndb + kPadRows, st));
   return launch_decode(L.keys, nq, dtype, out_idx, out_score, st);
 }
@@ -185,7 +195,7 @@ int fastnn_reciprocal(const void* desc1, int H1, int W1, const void* desc2, int 
                       void* out_score, int64_t capacity, int32_t* out_count, int32_t* out_iters,
                       int32_t* out_frontier, void* workspace, size_t workspace_bytes,
                       fastnn_stream_t stream) {
-  if (!dtype_ok(dtype) || !d_ok(d)) return FASTNN_ERR_UNSUPPORTED;
+  if (!dtype_ok(dtype) || !d_ok(d, dtype)) return FASTNN_ERR_UNSUPPORTED;
   if (H1 < 1 || W1 < 1 || H2 < 1 || W2 < 1 || subsample < 1 || max_iter < 1 ||
       max_iter > kMaxIter || batch < 1 || batch > nn_tc_max_batch())
     return FASTNN_ERR_INVALID;
@@ -236,6 +246,9 @@ int fastnn_reciprocal(const void* desc1, int H1, int W1, const void* desc2, int 
   r.cmp.bwd_key = L.bwd;
   r.cmp.claim = L.claim;
   r.cmp.N1 = N1;
+  r.cmp.N2 = N2;
+  r.cmp.pts1 = reinterpret_cast<const float4*>(L.d1rep);
+  r.cmp.pts2 = reinterpret_cast<const float4*>(L.d2rep);
   r.cmp.out_pairs = out_pairs;
   r.cmp.out_score = out_score;
   r.cmp.cap = capacity;
@@ -256,6 +269,7 @@ int fastnn_reciprocal(const void* desc1, int H1, int W1, const void* desc2, int 
   r.grid_count = reinterpret_cast<uint32_t*>(L.status + 4);
   r.grid_abort = L.status + 5;
   r.status = L.status;
+  if (dtype == FASTNN_F32_L2) return launch_reciprocal_l2(r, st);
   return launch_reciprocal(r, dtype, batch * N1 + kPadRows, batch * N2 + kPadRows, st);
 }
 
@@ -263,7 +277,7 @@ int fastnn_mutual_dense(const void* desc1, int64_t n1, const void* desc2, int64_
                         int dtype, int32_t* out_pairs, void* out_score, int64_t capacity,
                         int32_t* out_count, void* workspace, size_t workspace_bytes,
                         fastnn_stream_t stream) {
-  if (!dtype_ok(dtype) || !d_ok(d)) return FASTNN_ERR_UNSUPPORTED;
+  if (!dtype_ok(dtype) || !d_ok(d, dtype)) return FASTNN_ERR_UNSUPPORTED;
   if (n1 < 1 || n2 < 1 || n1 > INT32_MAX - kPadRows || n2 > INT32_MAX - kPadRows)
     return FASTNN_ERR_INVALID;
   if (!desc1 || !desc2 || !out_pairs || !out_count || !workspace || !aligned(workspace, kAlign))
@@ -292,7 +306,10 @@ int fastnn_mutual_dense(const void* desc1, int64_t n1, const void* desc2, int64_
   a.d = d;
   a.q_absmax = L.status + 1;
   a.db_absmax = L.status + 2;
-  FASTNN_TRY(launch_nn_tc(a, dtype, n2 + kPadRows, st));
+  if (dtype == FASTNN_F32_L2)
+    FASTNN_TRY(launch_nn_l2(a, st));
+  else
+    FASTNN_TRY(launch_nn_tc(a, dtype, n2 + kPadRows, st));
   NNArgs r{};
   r.q_rows = L.d2rep;
   r.q_rows_per_pair = n2;
@@ -306,10 +323,15 @@ int fastnn_mutual_dense(const void* desc1, int64_t n1, const void* desc2, int64_
   r.d = d;
   r.q_absmax = L.status + 2;
   r.db_absmax = L.status + 1;
-  FASTNN_TRY(launch_nn_tc(r, dtype, n1 + kPadRows, st));
+  if (dtype == FASTNN_F32_L2)
+    FASTNN_TRY(launch_nn_l2(r, st));
+  else
+    FASTNN_TRY(launch_nn_tc(r, dtype, n1 + kPadRows, st));
   MutualSrc m{};
   m.k12 = L.k12;
   m.k21 = L.k21;
+  m.pts1 = reinterpret_cast<const float4*>(L.d1rep);
+  m.pts2 = reinterpret_cast<const float4*>(L.d2rep);
   m.n1 = n1;
   m.n2 = n2;
   return launch_mutual(m, L.blocks, dtype, out_pairs, out_score, capacity, out_count, st);

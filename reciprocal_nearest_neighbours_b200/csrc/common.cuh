@@ -18,6 +18,9 @@
 namespace fastnn {
 
 constexpr int kStatusTimeout = 1;  // bit set in the device status word
+// Every bounded wait in the kernels (mbarrier phases, grid barriers) gives up
+// after this long, sets kStatusTimeout and unwinds.
+constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 __host__ __device__ __forceinline__ uint32_t ord_i32(int32_t s) {
   return static_cast<uint32_t>(s) ^ 0x80000000u;
@@ -46,9 +49,19 @@ __host__ __device__ __forceinline__ uint32_t key_score_bits(uint64_t key) {
 
 // Bytes of one repacked descriptor row: d elements zero-padded to K = 32
 // (d <= 32) or K = 64 (d <= 64) elements of 1 (int8) or 2 (bf16, half) bytes.
-__host__ __device__ constexpr int elem_bytes(int dtype) { return dtype == FASTNN_I8 ? 1 : 2; }
+// Pointmap rows (FASTNN_F32_L2, d <= 3) become one float4 (x, y, z, -|p|^2).
+__host__ __device__ constexpr int elem_bytes(int dtype) {
+  return dtype == FASTNN_I8 ? 1 : dtype == FASTNN_F32_L2 ? 4 : 2;
+}
 __host__ __device__ constexpr int row_bytes(int dtype, int d) {
-  return elem_bytes(dtype) * (d <= 32 ? 32 : 64);
+  return dtype == FASTNN_F32_L2 ? 16 : elem_bytes(dtype) * (d <= 32 ? 32 : 64);
+}
+
+// Squared Euclidean distance of two repacked pointmap rows, in fp32 from the
+// coordinate differences (the .w components hold -|p|^2 and are ignored).
+__device__ __forceinline__ float sq_dist3(float4 a, float4 b) {
+  const float dx = a.x - b.x, dy = a.y - b.y, dz = a.z - b.z;
+  return __fmaf_rn(dz, dz, __fmaf_rn(dy, dy, dx * dx));
 }
 
 // Where the query rows of one nearest-neighbour pass come from.
@@ -71,7 +84,7 @@ struct NNArgs {
   uint64_t* out_key;       // [batch][q_cap], merged with atomicMax
   int batch;
   int* status;
-  int d;                   // descriptor length (<= 32)
+  int d;                   // descriptor length (<= 64; <= 3 for pointmaps)
   const int* q_absmax;     // int8: max |element| of the query map (or nullptr)
   const int* db_absmax;    // int8: max |element| of the database map (or nullptr)
 };

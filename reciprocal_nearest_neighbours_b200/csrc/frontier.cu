@@ -143,6 +143,8 @@ __global__ void __launch_bounds__(1024) mutual_emit_kernel(MutualSrc m,
           const uint32_t h = key_score_bits(m.k12[i]);
           if (DT == FASTNN_I8)
             static_cast<int32_t*>(out_score)[pos] = unord_i32(h);
+          else if (DT == FASTNN_F32_L2)
+            static_cast<float*>(out_score)[pos] = sq_dist3(m.pts1[i], m.pts2[j]);
           else
             static_cast<float*>(out_score)[pos] = unord_f32(h);
         } else if (m.score12) {
@@ -159,7 +161,9 @@ __global__ void __launch_bounds__(1024) mutual_emit_kernel(MutualSrc m,
 // ------------------------------------------------------------ decode nn ---
 template <int DT>
 __global__ void decode_kernel(const uint64_t* __restrict__ key, int64_t n,
-                              int32_t* __restrict__ out_idx, void* __restrict__ out_score) {
+                              int32_t* __restrict__ out_idx, void* __restrict__ out_score,
+                              const float4* __restrict__ q_pts,
+                              const float4* __restrict__ db_pts, int64_t ndb) {
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const uint64_t k = key[i];
@@ -167,9 +171,31 @@ __global__ void decode_kernel(const uint64_t* __restrict__ key, int64_t n,
     if (out_score) {
       if (DT == FASTNN_I8)
         static_cast<int32_t*>(out_score)[i] = unord_i32(key_score_bits(k));
+      else if (DT == FASTNN_F32_L2)
+        static_cast<float*>(out_score)[i] =
+            key_index(k) < ndb ? sq_dist3(q_pts[i], db_pts[key_index(k)]) : INFINITY;
       else
         static_cast<float*>(out_score)[i] = unord_f32(key_score_bits(k));
     }
+  }
+}
+
+// Pointmap rows: float32 [rows][d] (d <= 3) -> float4 (x, y, z, -|p|^2),
+// missing coordinates zero; pad_rows zero rows follow. The norm is computed
+// in fp32 as fma(z, z, fma(y, y, x * x)).
+__global__ void repack_l2_kernel(const float* __restrict__ src, int64_t rows, int d,
+                                 float4* __restrict__ dst, int64_t pad_rows) {
+  for (int64_t row = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+       row < rows + pad_rows; row += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (row < rows) {
+      const float* s = src + row * d;
+      p.x = __ldg(s);
+      if (d > 1) p.y = __ldg(s + 1);
+      if (d > 2) p.z = __ldg(s + 2);
+      p.w = -__fmaf_rn(p.z, p.z, __fmaf_rn(p.y, p.y, p.x * p.x));
+    }
+    dst[row] = p;
   }
 }
 
@@ -189,6 +215,12 @@ int launch_repack(const void* src, int64_t rows, int d, int dtype, void* dst, in
   const uint8_t* s8 = static_cast<const uint8_t*>(src);
   uint8_t* d8 = static_cast<uint8_t*>(dst);
   const int g = grid_for(total, 256);
+  if (dtype == FASTNN_F32_L2) {
+    repack_l2_kernel<<<g, 256, 0, st>>>(static_cast<const float*>(src), rows, d,
+                                        static_cast<float4*>(dst), pad_rows);
+    FASTNN_CUDA_TRY(cudaGetLastError());
+    return FASTNN_OK;
+  }
   switch (row_bytes(dtype, d)) {
     case 32:
       repack_kernel<1, 32><<<g, 256, 0, st>>>(s8, rows, d, d8, pad_rows, absmax);
@@ -218,6 +250,9 @@ int launch_mutual(const MutualSrc& m, int32_t* block_scratch, int dtype, int32_t
   mutual_scan_kernel<<<1, 1024, 0, st>>>(block_scratch, nb, out_count);
   if (dtype == FASTNN_I8)
     mutual_emit_kernel<FASTNN_I8><<<nb, 1024, 0, st>>>(m, block_scratch, out_pairs, out_score, cap);
+  else if (dtype == FASTNN_F32_L2)
+    mutual_emit_kernel<FASTNN_F32_L2><<<nb, 1024, 0, st>>>(m, block_scratch, out_pairs, out_score,
+                                                           cap);
   else
     mutual_emit_kernel<FASTNN_BF16><<<nb, 1024, 0, st>>>(m, block_scratch, out_pairs, out_score,
                                                          cap);
@@ -226,12 +261,16 @@ int launch_mutual(const MutualSrc& m, int32_t* block_scratch, int dtype, int32_t
 }
 
 int launch_decode(const uint64_t* key, int64_t n, int dtype, int32_t* out_idx, void* out_score,
-                  cudaStream_t st) {
+                  cudaStream_t st, const float4* q_pts, const float4* db_pts, int64_t ndb) {
   if (n <= 0) return FASTNN_OK;
+  const int g = grid_for(n, 256);
   if (dtype == FASTNN_I8)
-    decode_kernel<FASTNN_I8><<<grid_for(n, 256), 256, 0, st>>>(key, n, out_idx, out_score);
+    decode_kernel<FASTNN_I8><<<g, 256, 0, st>>>(key, n, out_idx, out_score, nullptr, nullptr, 0);
+  else if (dtype == FASTNN_F32_L2)
+    decode_kernel<FASTNN_F32_L2><<<g, 256, 0, st>>>(key, n, out_idx, out_score, q_pts, db_pts,
+                                                    ndb);
   else
-    decode_kernel<FASTNN_BF16><<<grid_for(n, 256), 256, 0, st>>>(key, n, out_idx, out_score);
+    decode_kernel<FASTNN_BF16><<<g, 256, 0, st>>>(key, n, out_idx, out_score, nullptr, nullptr, 0);
   FASTNN_CUDA_TRY(cudaGetLastError());
   return FASTNN_OK;
 }

@@ -16,6 +16,9 @@ struct CompactArgs {
   uint64_t* bwd_key;      // [batch][S_cap] NN21 of those matches (reset to 0 here)
   uint32_t* claim;        // [batch][N1] first-visit stamps (round << 24 | slot)
   int64_t N1;
+  int64_t N2;
+  const float4* pts1;     // pointmaps: repacked rows [batch][N1] (score = |p1 - p2|^2)
+  const float4* pts2;     // pointmaps: repacked rows [batch][N2]
   int32_t* out_pairs;     // [batch][cap][2]
   void* out_score;        // [batch][cap] or nullptr
   int64_t cap;
@@ -23,6 +26,21 @@ struct CompactArgs {
   int32_t* out_iters;     // [batch] or nullptr
   int32_t* out_frontier;  // [batch][max_iter] or nullptr
   int max_iter;
+};
+
+// Everything a persistent fast-matching kernel needs (device pointers).
+struct RecArgs {
+  NNArgs fwd;        // forward pass template: queries = image-1 rows, database = image 2
+  NNArgs bwd;        // backward pass template: queries = image-2 rows of the forward keys
+  CompactArgs cmp;   // per-round check/compaction template
+  int32_t* F[2];     // frontier ping-pong [batch][S]
+  int32_t* cnt[2];   // frontier sizes ping-pong [batch]
+  int64_t N1;        // pixels of image 1
+  int64_t S;         // seeds per pair
+  int W1, sub, max_iter, batch;
+  uint32_t* grid_count;  // grid-barrier arrival counter (zero before the launch)
+  int* grid_abort;       // set when any CTA gives up (zero before the launch)
+  int* status;
 };
 
 int launch_repack(const void* src, int64_t rows, int d, int dtype, void* dst, int64_t pad_rows,
@@ -36,6 +54,8 @@ struct MutualSrc {
   const int32_t* nn12;
   const int32_t* nn21;
   const void* score12;
+  const float4* pts1;  // pointmaps with keys: repacked rows of image 1 (local rows) and 2
+  const float4* pts2;
   int64_t n1;  // local image-1 rows
   int64_t n2;  // image-2 rows
   int64_t i0;  // global index of local row 0
@@ -44,7 +64,11 @@ struct MutualSrc {
 int mutual_blocks(int64_t n1);
 int launch_mutual(const MutualSrc& m, int32_t* block_scratch, int dtype, int32_t* out_pairs,
                   void* out_score, int64_t cap, int32_t* out_count, cudaStream_t st);
+// Keys -> (index, score). For pointmaps the score is the squared distance
+// of query row i (q_pts) and its nearest row (db_pts, ndb rows), both
+// repacked; a key without a candidate (index >= ndb) gets +inf.
 int launch_decode(const uint64_t* key, int64_t n, int dtype, int32_t* out_idx, void* out_score,
-                  cudaStream_t st);
+                  cudaStream_t st, const float4* q_pts = nullptr, const float4* db_pts = nullptr,
+                  int64_t ndb = 0);
 
 }  // namespace fastnn

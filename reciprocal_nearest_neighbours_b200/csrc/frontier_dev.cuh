@@ -6,8 +6,49 @@
 
 #include "common.cuh"
 #include "frontier.cuh"
+#include "ptx.cuh"
 
 namespace fastnn {
+
+// Grid-wide barrier over the co-resident CTAs of a cooperative launch: a
+// monotonic arrival counter (zero before the launch); each CTA waits, bounded
+// by kTimeoutNs, until the counter reaches its next multiple of the grid
+// size. A CTA that arrives with cta_ok == false, or a wait that runs out,
+// raises the shared abort word so that every CTA leaves. `flag` is a shared
+// int that carries thread 0's verdict to the CTA. Returns the CTA-uniform
+// verdict.
+__device__ __forceinline__ bool grid_barrier(uint32_t* count, int* abort_word, int* status,
+                                             uint32_t& target, bool cta_ok, int* flag) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    target += gridDim.x;
+    bool ok = cta_ok;
+    if (!ok) atomicExch(abort_word, 1);
+    __threadfence();
+    atomicAdd(count, 1u);
+    const uint64_t t0 = ptx::globaltimer_ns();
+    for (uint32_t n = 1;; ++n) {
+      if (*reinterpret_cast<volatile uint32_t*>(count) >= target) break;
+      if ((n & 63) == 0) {
+        if (*reinterpret_cast<volatile int*>(abort_word)) {
+          ok = false;
+          break;
+        }
+        if (ptx::globaltimer_ns() - t0 > kTimeoutNs) {
+          atomicOr(status, kStatusTimeout);
+          atomicExch(abort_word, 1);
+          ok = false;
+          break;
+        }
+      }
+    }
+    __threadfence();
+    if (*reinterpret_cast<volatile int*>(abort_word)) ok = false;
+    *flag = ok ? 1 : 0;
+  }
+  __syncthreads();
+  return *reinterpret_cast<volatile int*>(flag) != 0;
+}
 
 // Block-wide exclusive scan of two 0/1 flags (warp ballots + one smem pass).
 // Returns the exclusive prefix of each flag and the block totals. `sm` holds
@@ -104,7 +145,8 @@ __device__ void compact_pair(const CompactArgs& c, const FrontierBufs& fb, int b
       fk = __ldcg(fwd + k);
       v = key_index(fk);
       u2 = key_index(__ldcg(bwd + k));
-      conv = (u2 == u);
+      // A forward pass that found no candidate leaves v = 0xFFFFFFFF.
+      conv = (u2 == u) && v < static_cast<uint32_t>(c.N2);
       push = !conv && !last_round && u2 < static_cast<uint32_t>(c.N1) &&
              __ldcg(claim + u2) == (stamp_hi | static_cast<uint32_t>(k));
       fwd[k] = 0;
@@ -120,6 +162,9 @@ __device__ void compact_pair(const CompactArgs& c, const FrontierBufs& fb, int b
         if (c.out_score) {
           if (DT == FASTNN_I8)
             static_cast<int32_t*>(c.out_score)[b * c.cap + pos] = unord_i32(key_score_bits(fk));
+          else if (DT == FASTNN_F32_L2)
+            static_cast<float*>(c.out_score)[b * c.cap + pos] =
+                sq_dist3(c.pts1[b * c.N1 + u], c.pts2[b * c.N2 + v]);
           else
             static_cast<float*>(c.out_score)[b * c.cap + pos] = unord_f32(key_score_bits(fk));
         }
@@ -136,6 +181,68 @@ __device__ void compact_pair(const CompactArgs& c, const FrontierBufs& fb, int b
     if (c.out_frontier) c.out_frontier[b * c.max_iter + (t - 1)] = cnt;
   }
   __syncthreads();
+}
+
+// The fast scheme's round loop, shared by the persistent matching kernels:
+// clear the per-call state, seed the grid, then per round a forward pass
+// (image 1 -> 2), a backward pass (matches -> image 1) and the per-pair
+// check/compaction, separated by grid barriers; stops when every pair's
+// frontier is empty or after max_iter rounds. `nn(dir, q)` runs one
+// nearest-neighbour pass over the whole grid (dir 0: r.fwd, 1: r.bwd) and
+// ends with a CTA barrier. `cta_abort` is the CTA's own abort flag (shared
+// memory); `flag`, `more` and `scan` (66 ints) are shared scratch.
+template <int DT, class NNPass>
+__device__ void fast_rounds(const RecArgs& r, NNPass&& nn, volatile int* cta_abort, int* flag,
+                            int* more, int* scan) {
+  uint32_t target = 0;
+  const int batch = r.batch;
+  const int64_t S = r.S;
+  const int64_t gtid = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  const int64_t gsize = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  auto sync = [&]() {
+    return grid_barrier(r.grid_count, r.grid_abort, r.status, target, !*cta_abort, flag);
+  };
+
+  // Clear per-call state: keys, first-visit claims, outputs.
+  for (int64_t i = gtid; i < batch * S; i += gsize) {
+    r.cmp.fwd_key[i] = 0;
+    r.cmp.bwd_key[i] = 0;
+  }
+  for (int64_t i = gtid; i < batch * r.N1; i += gsize) r.cmp.claim[i] = 0xFFFFFFFFu;
+  for (int64_t i = gtid; i < batch; i += gsize) {
+    r.cmp.out_count[i] = 0;
+    if (r.cmp.out_iters) r.cmp.out_iters[i] = 0;
+  }
+  if (r.cmp.out_frontier)
+    for (int64_t i = gtid; i < batch * r.max_iter; i += gsize) r.cmp.out_frontier[i] = 0;
+  bool ok = sync();
+  if (ok) {
+    // Seeds: the round-1 frontier of every pair.
+    for (int64_t i = gtid; i < batch * S; i += gsize)
+      seed_one(r.F[0], S, r.cmp.claim, r.N1, r.W1, r.sub, static_cast<int>(i / S),
+               static_cast<int>(i % S));
+    for (int64_t i = gtid; i < batch; i += gsize) r.cnt[0][i] = static_cast<int>(S);
+    ok = sync();
+  }
+  for (int t = 1; ok && t <= r.max_iter; ++t) {
+    const int cur = (t - 1) & 1, nxt = t & 1;
+    nn(0, PhaseQ{r.F[cur], r.cnt[cur]});
+    if (!sync()) break;
+    nn(1, PhaseQ{nullptr, r.cnt[cur]});
+    if (!sync()) break;
+    const FrontierBufs fb{r.F[cur], r.F[nxt], r.cnt[cur], r.cnt[nxt]};
+    for (int b = blockIdx.x; b < batch; b += gridDim.x)
+      compact_pair<DT>(r.cmp, fb, b, t, t == r.max_iter, scan);
+    if (!sync()) break;
+    // Every CTA reads the same counts after the barrier: a uniform exit.
+    if (threadIdx.x == 0) {
+      int any = 0;
+      for (int b = 0; b < batch; ++b) any |= __ldcg(r.cnt[nxt] + b);
+      *more = any != 0 ? 1 : 0;
+    }
+    __syncthreads();
+    if (!*reinterpret_cast<volatile int*>(more)) break;
+  }
 }
 
 }  // namespace fastnn

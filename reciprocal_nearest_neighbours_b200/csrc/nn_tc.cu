@@ -54,7 +54,6 @@ constexpr int kThreads = 32 * (kEpiWarps + 1 + kAcc);
 constexpr int kEpiCols = kBN / 2;               // columns of a tile per epilogue thread
 constexpr int kChunks = kEpiCols / 32;          // 32-column TMEM loads per unit and thread
 constexpr int kMaxBatch = 1024;
-constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr int kStashBytes = kEpiWarps * 32 * 32;  // 32 B per epilogue thread
 
 // Barrier slots inside the barrier block.
@@ -717,48 +716,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---- persistent fast reciprocal matching ----------------------------------
 
-// Grid-wide barrier over co-resident CTAs (cooperative launch): a monotonic
-// arrival counter; every CTA waits (bounded) until it reaches the next
-// multiple of the grid size. A CTA that aborted, or a wait that ran out, sets
-// the shared abort word so that every CTA leaves the round loop. Returns the
-// CTA-uniform verdict.
-__device__ bool grid_sync(const RecArgs& r, uint32_t& target, Ctl* ctl) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    target += gridDim.x;
-    bool ok = !ctl->abort_flag;
-    if (!ok) atomicExch(r.grid_abort, 1);
-    __threadfence();
-    atomicAdd(r.grid_count, 1u);
-    const uint64_t t0 = ptx::globaltimer_ns();
-    for (uint32_t n = 1;; ++n) {
-      if (*reinterpret_cast<volatile uint32_t*>(r.grid_count) >= target) break;
-      if ((n & 63) == 0) {
-        if (*reinterpret_cast<volatile int*>(r.grid_abort)) {
-          ok = false;
-          break;
-        }
-        if (ptx::globaltimer_ns() - t0 > kTimeoutNs) {
-          atomicOr(r.status, kStatusTimeout);
-          atomicExch(r.grid_abort, 1);
-          ok = false;
-          break;
-        }
-      }
-    }
-    __threadfence();
-    if (*reinterpret_cast<volatile int*>(r.grid_abort)) ok = false;
-    ctl->grid_ok = ok ? 1 : 0;
-  }
-  __syncthreads();
-  return ctl->grid_ok != 0;
-}
-
-// MASt3R fast reciprocal matching of `batch` pairs in one launch: clear the
-// per-call state, seed the grid, then per round a forward pass (image 1 -> 2),
-// a backward pass (matches -> image 1) and the per-pair check/compaction,
-// separated by grid barriers; stops when every pair's frontier is empty or
-// after max_iter rounds.
+// MASt3R fast reciprocal matching of `batch` pairs in one launch (the round
+// loop is fast_rounds); its nearest-neighbour passes run the tensor-core
+// pipeline above, whose barrier phases, ring positions and TMEM allocation
+// carry over from pass to pass.
 template <int DT, int RB>
 __global__ void __launch_bounds__(kThreads, 1)
     reciprocal_kernel(const __grid_constant__ CUtensorMap tmap_d2,
@@ -773,52 +734,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   pipe_setup(ctl);
   const uint32_t tmem = ctl->tmem_base;
   PipeState ps;
-  uint32_t target = 0;
-  const int batch = r.batch;
-  const int64_t S = r.S;
-  const int64_t gtid = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
-  const int64_t gsize = static_cast<int64_t>(gridDim.x) * blockDim.x;
-
-  // Clear per-call state: keys, first-visit claims, outputs.
-  for (int64_t i = gtid; i < batch * S; i += gsize) {
-    r.cmp.fwd_key[i] = 0;
-    r.cmp.bwd_key[i] = 0;
-  }
-  for (int64_t i = gtid; i < batch * r.N1; i += gsize) r.cmp.claim[i] = 0xFFFFFFFFu;
-  for (int64_t i = gtid; i < batch; i += gsize) {
-    r.cmp.out_count[i] = 0;
-    if (r.cmp.out_iters) r.cmp.out_iters[i] = 0;
-  }
-  if (r.cmp.out_frontier)
-    for (int64_t i = gtid; i < batch * r.max_iter; i += gsize) r.cmp.out_frontier[i] = 0;
-  bool ok = grid_sync(r, target, ctl);
-  if (ok) {
-    // Seeds: the round-1 frontier of every pair.
-    for (int64_t i = gtid; i < batch * S; i += gsize)
-      seed_one(r.F[0], S, r.cmp.claim, r.N1, r.W1, r.sub, static_cast<int>(i / S),
-               static_cast<int>(i % S));
-    for (int64_t i = gtid; i < batch; i += gsize) r.cnt[0][i] = static_cast<int>(S);
-    ok = grid_sync(r, target, ctl);
-  }
-  for (int t = 1; ok && t <= r.max_iter; ++t) {
-    const int cur = (t - 1) & 1, nxt = t & 1;
-    run_phase<DT, RB>(&tmap_d2, r.fwd, PhaseQ{r.F[cur], r.cnt[cur]}, L, tmem, ps);
-    if (!grid_sync(r, target, ctl)) break;
-    run_phase<DT, RB>(&tmap_d1, r.bwd, PhaseQ{nullptr, r.cnt[cur]}, L, tmem, ps);
-    if (!grid_sync(r, target, ctl)) break;
-    const FrontierBufs fb{r.F[cur], r.F[nxt], r.cnt[cur], r.cnt[nxt]};
-    for (int b = blockIdx.x; b < batch; b += gridDim.x)
-      compact_pair<DT>(r.cmp, fb, b, t, t == r.max_iter, ctl->scan);
-    if (!grid_sync(r, target, ctl)) break;
-    // Every CTA reads the same counts after the barrier: a uniform exit.
-    if (threadIdx.x == 0) {
-      int any = 0;
-      for (int b = 0; b < batch; ++b) any |= __ldcg(r.cnt[nxt] + b);
-      ctl->more = any != 0 ? 1 : 0;
-    }
-    __syncthreads();
-    if (!ctl->more) break;
-  }
+  auto pass = [&](int dir, const PhaseQ& q) {
+    if (dir == 0)
+      run_phase<DT, RB>(&tmap_d2, r.fwd, q, L, tmem, ps);
+    else
+      run_phase<DT, RB>(&tmap_d1, r.bwd, q, L, tmem, ps);
+  };
+  fast_rounds<DT>(r, pass, &ctl->abort_flag, &ctl->grid_ok, &ctl->more, ctl->scan);
   pipe_teardown(ctl, tmem, r.status);
 }
 
@@ -925,6 +847,10 @@ int timer_end(int slot, cudaStream_t stream) {
 }
 
 }  // namespace
+
+int kernel_timer_begin(cudaStream_t stream) { return timer_begin(stream); }
+int kernel_timer_end(int slot, cudaStream_t stream) { return timer_end(slot, stream); }
+int device_sm_count(int* sms) { return sm_count(sms); }
 
 namespace {
 

@@ -373,6 +373,10 @@ CONFIGS = {
              "warp generator's sources with N(0, 0.002 z) noise and 30% outliers "
              "uniform in the scene's bounding box; nearest 3D point by Euclidean "
              "distance; 8-px grid (3,072 seeds), max_iter=10"),
+    "dense_512x384_pts3_f32": dict(
+        seed=BASE_SEED + 7,
+        note="dense mutual nearest 3D points over all 196,608 pixels of the 512x384 "
+             "pointmap pair above (same seed, same maps)"),
     "batch16_512x288_d32_i8": dict(
         seed=BASE_SEED + 5,
         note="16 independent 512x288 pairs, d=32, int8 uniform in [-16,16], warped "
@@ -408,6 +412,9 @@ def make_workload(name: str, batch: int | None = None) -> Workload:
                         note=cfg["note"])
     if name == "pair_512x384_pts3_f32":
         return Workload(name, [pointmap_pair(seed)], subsample=8, max_iter=10, note=cfg["note"])
+    if name == "dense_512x384_pts3_f32":
+        return Workload(name, [pointmap_pair(seed)], subsample=8, max_iter=10, dense=True,
+                        note=cfg["note"])
     if name == "batch16_512x288_d32_i8":
         nb = 16 if batch is None else batch
         pairs = [warped_pair_int8(seed + 1000 * b, H=288, W=512, d=32)

@@ -68,6 +68,11 @@ def test_workspace_sizes(lib):
     e = ws(fnn.FASTNN_OP_RECIPROCAL, 196608, 196608, 64, fnn.FASTNN_I8, 1, 3072)
     assert e == b and e - a >= 2 * 196608 * 32
     assert ws(fnn.FASTNN_OP_NN, 10, 1000, 48, fnn.FASTNN_BF16) > 1000 * 128
+    # pointmaps: one 16-byte row per point, d <= 3
+    assert ws(fnn.FASTNN_OP_NN, 10, 1000, 3, fnn.FASTNN_F32_L2) > 1000 * 16
+    assert ws(fnn.FASTNN_OP_RECIPROCAL, 196608, 196608, 3, fnn.FASTNN_F32_L2, 1, 3072) > \
+        2 * 196608 * 16
+    assert ws(fnn.FASTNN_OP_NN, 10, 10, 4, fnn.FASTNN_F32_L2) == 0
     # unsupported arguments size to 0
     assert ws(fnn.FASTNN_OP_NN, 10, 10, 65, fnn.FASTNN_I8) == 0
     assert ws(fnn.FASTNN_OP_NN, 10, 10, 65, fnn.FASTNN_F16) == 0
@@ -86,6 +91,7 @@ def test_argument_errors_are_reported_on_the_host(lib):
     # unsupported d / dtype
     assert lib.fastnn_nn(fake, 4, fake, 4, 65, I8, fake, None, fake, big, None) == -2
     assert lib.fastnn_nn(fake, 4, fake, 4, 0, fnn.FASTNN_F16, fake, None, fake, big, None) == -2
+    assert lib.fastnn_nn(fake, 4, fake, 4, 4, fnn.FASTNN_F32_L2, fake, None, fake, big, None) == -2
     assert lib.fastnn_nn(fake, 4, fake, 4, 24, 5, fake, None, fake, big, None) == -2
     # empty query set is a no-op, even with null pointers
     assert lib.fastnn_nn(None, 0, None, 4, 24, I8, None, None, None, 0, None) == 0

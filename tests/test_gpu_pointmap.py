@@ -1,0 +1,259 @@
+"""GPU parity of the pointmap path (nearest 3D point; FASTNN_F32_L2).
+
+Tolerance, from the kernel's fp32 arithmetic. The kernel ranks database
+points p for a query a by s = 2<a, p> - |p|^2, formed as three fused
+multiply-adds on top of -|p|^2 (itself one multiply and two fused
+multiply-adds). Each rounding is at most u = 2^-24 of a partial sum bounded
+by (|a| + |p|)^2, so |s~ - s| <= 6 u (|a| + |p|)^2, and two candidates can
+swap only when their exact squared distances differ by less than
+12 u (|a| + R)^2, R = max |p| over the database; the tests use 16 u. The
+reported score is the squared distance recomputed from the coordinate
+differences (relative error below 8 u).
+
+Integer-valued points make every one of those operations exact in fp32, so
+there the GPU must agree with the oracle bit for bit, ties included.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from reciprocal_nearest_neighbours_b200 import fastnn_mutual_dense, fastnn_nn, fastnn_reciprocal
+from tests._dev import gpu_pairs, require_cuda
+from tests.test_gpu_reciprocal import as_set, expected_rounds
+from tests.test_oracle_l2 import load_pointmap_golden
+
+pytestmark = pytest.mark.gpu
+
+U = 2.0 ** -24
+
+
+@pytest.fixture(autouse=True)
+def _cuda():
+    require_cuda()
+
+
+def dev(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
+
+
+def tol_for(q: np.ndarray, db: np.ndarray) -> np.ndarray:
+    R = np.sqrt((db.astype(np.float64) ** 2).sum(1)).max()
+    return 16 * U * (np.sqrt((q.astype(np.float64) ** 2).sum(1)) + R) ** 2
+
+
+def check_nn_l2(idx_g, score_g, q, db):
+    """Tolerance rule: the chosen point is within tol of the nearest, the
+    reported squared distance is that of the chosen point, and the index
+    differs from the oracle's only where its top-2 margin is below tol."""
+    ref = oracle.nn(q, db, "l2")
+    idx = idx_g.cpu().numpy().astype(np.int64)
+    sc = score_g.cpu().numpy().astype(np.float64)
+    assert np.all((idx >= 0) & (idx < len(db)))
+    tol = tol_for(q, db)
+    exact = oracle.score_of(q, np.arange(len(q)), db, idx, "l2")
+    assert np.all(exact - ref.score <= tol)
+    assert np.all(np.abs(sc - exact) <= 8 * U * exact + 1e-30)
+    diff = idx != ref.idx
+    assert np.all(oracle.margin(ref, "l2")[diff] < tol[diff])
+    return int(diff.sum())
+
+
+NN_CASES = [
+    # nq, ndb, d
+    (1, 1, 3), (5, 3, 3), (300, 1000, 3), (129, 1023, 3), (128, 1024, 3), (200, 1025, 3),
+    (1000, 5000, 3), (333, 4099, 2), (700, 2048, 1), (4000, 300, 3),
+]
+
+
+@pytest.mark.parametrize("nq,ndb,d", NN_CASES)
+def test_nn_l2_random_points_within_tolerance(nq, ndb, d):
+    rng = np.random.default_rng(nq * 7 + ndb + d)
+    q = rng.uniform(-3, 3, size=(nq, d)).astype(np.float32)
+    db = rng.uniform(-3, 3, size=(ndb, d)).astype(np.float32)
+    idx, score = fastnn_nn(dev(q), dev(db))
+    torch.cuda.synchronize()
+    assert check_nn_l2(idx, score, q, db) <= max(1, nq // 100)
+
+
+@pytest.mark.parametrize("nq,ndb,d,amp", [(300, 1000, 3, 2), (700, 2049, 3, 8), (129, 300, 1, 3),
+                                          (1000, 1024, 2, 1), (257, 5000, 3, 5)])
+def test_nn_l2_integer_points_bit_exact(nq, ndb, d, amp):
+    """Small integer coordinates: every fp32 step is exact, ties are massive,
+    and the lowest index must win exactly as in the oracle."""
+    rng = np.random.default_rng(nq + ndb * 3 + amp)
+    q = rng.integers(-amp, amp + 1, size=(nq, d)).astype(np.float32)
+    db = rng.integers(-amp, amp + 1, size=(ndb, d)).astype(np.float32)
+    idx, score = fastnn_nn(dev(q), dev(db))
+    ref = oracle.nn(q, db, "l2")
+    assert np.array_equal(idx.cpu().numpy(), ref.idx)
+    assert np.array_equal(score.cpu().numpy().astype(np.float64), ref.score)
+
+
+def test_nn_l2_identical_database_points_pick_index_zero():
+    q = np.full((300, 3), 0.5, dtype=np.float32)
+    db = np.ones((3000, 3), dtype=np.float32)
+    idx, score = fastnn_nn(dev(q), dev(db))
+    assert torch.all(idx == 0) and torch.all(score == 0.75)
+
+
+def test_nn_l2_full_size_pointmap_sampled_queries():
+    p = synth.make_workload("pair_512x384_pts3_f32").pairs[0]
+    D1, D2 = p.desc1.reshape(-1, 3), p.desc2.reshape(-1, 3)
+    rng = np.random.default_rng(3)
+    qi = np.sort(rng.choice(D1.shape[0], size=512, replace=False))
+    idx, score = fastnn_nn(dev(D1[qi]), dev(D2))
+    assert check_nn_l2(idx, score, D1[qi], D2) <= 10
+
+
+# ---------------------------------------------------------------- fast matching
+
+def run_fast(m1, m2, sub, max_iter):
+    pairs, score, count, iters = fastnn_reciprocal(dev(m1), dev(m2), sub, max_iter)
+    torch.cuda.synchronize()
+    return pairs, score, count, iters
+
+
+def check_fast_exact(m1, m2, sub, max_iter, b=0, gpu=None):
+    H1, W1, _ = m1.shape
+    H2, W2, _ = m2.shape
+    pairs, score, count, iters = gpu if gpu is not None else run_fast(m1, m2, sub, max_iter)
+    p, s = gpu_pairs(pairs, score, count, b)
+    ref = oracle.fast_reciprocal(m1, H1, W1, m2, H2, W2, "l2", sub, max_iter)
+    got = {(int(u), int(v), float(x)) for (u, v), x in zip(p.tolist(), s.tolist())}
+    exp = {(int(u), int(v), float(x)) for (u, v), x in zip(ref.pairs.tolist(), ref.score.tolist())}
+    assert len(got) == len(p)
+    assert got == exp, (sorted(got - exp)[:5], sorted(exp - got)[:5])
+    assert int(iters[b]) == expected_rounds(ref)
+    return p
+
+
+def test_golden_pointmap_fixture():
+    fx = load_pointmap_golden()
+    _, _, m1 = fx["image1"]
+    _, _, m2 = fx["image2"]
+    for case in fx["fast"]:
+        pairs, score, count, iters = run_fast(m1, m2, case["sub"], case["max_iter"])
+        p, s = gpu_pairs(pairs, score, count)
+        assert {(u, v, x) for (u, v), x in zip(p.tolist(), s.tolist())} == set(case["pairs"])
+        rounds = next((i for i, f in enumerate(case["first"]) if f == 0), len(case["first"]))
+        assert int(iters[0]) == rounds
+    D1, D2 = m1.reshape(-1, 3), m2.reshape(-1, 3)
+    pairs, score, count = fastnn_mutual_dense(dev(D1), dev(D2))
+    p, s = gpu_pairs(pairs, score, count)
+    assert [(u, v, x) for (u, v), x in zip(p.tolist(), s.tolist())] == fx["dense"]
+
+
+@pytest.mark.parametrize("seed", range(16))
+def test_fast_l2_integer_maps_exact(seed):
+    rng = np.random.default_rng(500 + seed)
+    H1, W1, H2, W2 = (int(x) for x in rng.integers(1, 48, size=4))
+    d = int(rng.integers(1, 4))
+    amp = int(rng.choice([1, 2, 4]))
+    m1 = rng.integers(-amp, amp + 1, size=(H1, W1, d)).astype(np.float32)
+    m2 = rng.integers(-amp, amp + 1, size=(H2, W2, d)).astype(np.float32)
+    check_fast_exact(m1, m2, int(rng.integers(1, 5)), int(rng.choice([1, 2, 10, 255])))
+
+
+def test_fast_l2_noise_free_permutation():
+    rng = np.random.default_rng(17)
+    H, W = 96, 128
+    p1 = rng.uniform(-2, 2, size=(H * W, 3)).astype(np.float32)
+    perm = rng.permutation(H * W)
+    p2 = np.empty_like(p1)
+    p2[perm] = p1
+    pairs, score, count, iters = run_fast(p1.reshape(H, W, 3), p2.reshape(H, W, 3), 4, 10)
+    p, s = gpu_pairs(pairs, score, count)
+    seeds = oracle.grid_seeds(H, W, 4)
+    assert sorted(p[:, 0].tolist()) == sorted(seeds.tolist())
+    assert np.array_equal(p[:, 1], perm[p[:, 0]]) and np.all(s == 0.0)
+    assert int(iters[0]) == 1
+
+
+def check_fast_l2_certificate(m1, m2, sub, max_iter, gpu=None):
+    """Each GPU pair is reciprocal up to the tolerance, its score is its
+    squared distance, and each oracle pair the GPU lacks sits at the end of
+    walks that all pass a near-tie."""
+    H1, W1, _ = m1.shape
+    H2, W2, _ = m2.shape
+    pairs, score, count, iters = gpu if gpu is not None else run_fast(m1, m2, sub, max_iter)
+    p, s = gpu_pairs(pairs, score, count)
+    D1, D2 = m1.reshape(-1, 3), m2.reshape(-1, 3)
+    tol = 16 * U * (2 * max(np.sqrt((D1.astype(np.float64) ** 2).sum(1)).max(),
+                            np.sqrt((D2.astype(np.float64) ** 2).sum(1)).max())) ** 2
+    exact = oracle.score_of(D1, p[:, 0], D2, p[:, 1], "l2")
+    assert np.all(np.abs(s - exact) <= 8 * U * exact + 1e-30)
+    r12 = oracle.nn(D1[p[:, 0]], D2, "l2")
+    r21 = oracle.nn(D2[p[:, 1]], D1, "l2")
+    assert np.all(exact - r12.score <= tol) and np.all(exact - r21.score <= tol)
+    ref = oracle.fast_reciprocal(m1, H1, W1, m2, H2, W2, "l2", sub, max_iter, track_gaps=True)
+    got = set(map(tuple, p.tolist()))
+    exp = set(map(tuple, ref.pairs.tolist()))
+    for u, v in exp - got:
+        assert ref.min_gap[u] < tol, (u, v, ref.min_gap[u], tol)
+    return len(got ^ exp), len(exp)
+
+
+def test_fast_l2_small_pointmaps_certificate():
+    for seed in range(4):
+        m = synth.pointmap_pair(600 + seed, H=48, W=64)
+        check_fast_l2_certificate(m.desc1, m.desc2, 4, 10)
+
+
+def test_fast_l2_pair_512x384_full_size():
+    w = synth.make_workload("pair_512x384_pts3_f32")
+    p = w.pairs[0]
+    symdiff, n = check_fast_l2_certificate(p.desc1, p.desc2, w.subsample, w.max_iter)
+    assert n > 1000 and symdiff <= 0.05 * n
+
+
+def test_fast_l2_batch_pairs_independent():
+    maps = [synth.pointmap_pair(700 + b, H=72, W=128) for b in range(3)]
+    d1 = np.stack([m.desc1 for m in maps])
+    d2 = np.stack([m.desc2 for m in maps])
+    g = run_fast(d1, d2, 4, 10)
+    for b in range(3):
+        gb = run_fast(maps[b].desc1, maps[b].desc2, 4, 10)
+        n = int(g[2][b])
+        assert n == int(gb[2][0]) and n > 100
+        assert torch.equal(g[0][b, :n], gb[0][0, :n])
+        assert torch.equal(g[1][b, :n], gb[1][0, :n])
+
+
+# ---------------------------------------------------------------- dense mutual
+
+@pytest.mark.parametrize("n1,n2,d,amp", [(1000, 777, 3, 3), (1, 1, 3, 1), (2049, 3000, 2, 6),
+                                         (513, 129, 1, 4)])
+def test_dense_l2_integer_points_exact(n1, n2, d, amp):
+    rng = np.random.default_rng(n1 * 5 + n2 + d)
+    D1 = rng.integers(-amp, amp + 1, size=(n1, d)).astype(np.float32)
+    D2 = rng.integers(-amp, amp + 1, size=(n2, d)).astype(np.float32)
+    pairs, score, count = fastnn_mutual_dense(dev(D1), dev(D2))
+    p, s = gpu_pairs(pairs, score, count)
+    ref = oracle.dense_mutual(D1, D2, "l2")
+    assert np.array_equal(p, ref.pairs)
+    assert np.array_equal(s.astype(np.float64), ref.score)
+
+
+def test_dense_l2_pointmaps_within_tolerance():
+    m = synth.pointmap_pair(800, H=48, W=64)
+    D1, D2 = m.desc1.reshape(-1, 3), m.desc2.reshape(-1, 3)
+    pairs, score, count = fastnn_mutual_dense(dev(D1), dev(D2))
+    p, s = gpu_pairs(pairs, score, count)
+    exact = oracle.score_of(D1, p[:, 0], D2, p[:, 1], "l2")
+    assert np.all(np.abs(s - exact) <= 8 * U * exact + 1e-30)
+    ref = oracle.dense_mutual(D1, D2, "l2")
+    tol1 = tol_for(D1, D2)
+    tol2 = tol_for(D2, D1)
+    got = set(map(tuple, p.tolist()))
+    exp = set(map(tuple, ref.pairs.tolist()))
+    m12 = oracle.margin(ref.nn12, "l2")
+    m21 = oracle.margin(ref.nn21, "l2")
+    for i, j in got ^ exp:
+        jj = ref.nn12.idx[i]
+        assert min(m12[i] - tol1[i], m21[jj] - tol2[jj], m21[j] - tol2[j]) < 0
+    assert len(got ^ exp) <= 0.02 * len(exp)
