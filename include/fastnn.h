@@ -28,12 +28,13 @@
  *     16-bit patterns), float32 scores (fp32 accumulation of exact products).
  *     1 <= d <= 64 for all three (d <= 32 runs one 32-element K step).
  *     dtype FASTNN_F32_L2: float32 points, 1 <= d <= 3 (DUSt3R pointmaps
- *     have d = 3); scores are float32 SQUARED DISTANCES (lower is nearer),
- *     computed from the coordinate differences of the reported pair. Inputs
- *     must be finite. Selection is computed in fp32 as the maximum of
- *     2<q, p> - |p|^2, which orders points like -|q - p|^2; two points whose
- *     exact squared distances differ by less than about 2^-20 (|q| + max|p|)^2
- *     may be ordered either way.
+ *     have d = 3); scores are float32 SQUARED DISTANCES (lower is nearer).
+ *     Inputs must be finite. The squared distance of a point is computed in
+ *     fp64 from the coordinate differences, (dx^2 + dy^2) + dz^2 with one
+ *     rounding per operation, and rounded to fp32; the nearest point is the
+ *     lowest index among those whose fp32 value is the smallest. (The
+ *     kernels scan with fp32 scores 2<q, p> - |p|^2 and re-rank every point
+ *     their rounding error could place first.)
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the
  *     legacy default stream). The host blocks only in fastnn_device_status().
  *   - Return value: FASTNN_OK, or a negative fastnn_status describing an

@@ -182,9 +182,7 @@ int fastnn_nn(const void* q, int64_t nq, const void* db, int64_t ndb, int d, int
   a.db_absmax = L.status + 2;
   if (dtype == FASTNN_F32_L2) {
     FASTNN_TRY(launch_nn_l2(a, st));
-    return launch_decode(L.keys, nq, dtype, out_idx, out_score, st,
-                         reinterpret_cast<const float4*>(L.qrep),
-                         reinterpret_cast<const float4*>(L.dbrep), ndb);
+    return launch_decode(L.keys, nq, dtype, out_idx, out_score, st);
   }
   FASTNN_TRY(launch_nn_tc(a, dtype, ndb + kPadRows, st));
   return launch_decode(L.keys, nq, dtype, out_idx, out_score, st);
@@ -247,8 +245,6 @@ int fastnn_reciprocal(const void* desc1, int H1, int W1, const void* desc2, int 
   r.cmp.claim = L.claim;
   r.cmp.N1 = N1;
   r.cmp.N2 = N2;
-  r.cmp.pts1 = reinterpret_cast<const float4*>(L.d1rep);
-  r.cmp.pts2 = reinterpret_cast<const float4*>(L.d2rep);
   r.cmp.out_pairs = out_pairs;
   r.cmp.out_score = out_score;
   r.cmp.cap = capacity;
@@ -330,8 +326,7 @@ int fastnn_mutual_dense(const void* desc1, int64_t n1, const void* desc2, int64_
   MutualSrc m{};
   m.k12 = L.k12;
   m.k21 = L.k21;
-  m.pts1 = reinterpret_cast<const float4*>(L.d1rep);
-  m.pts2 = reinterpret_cast<const float4*>(L.d2rep);
+
   m.n1 = n1;
   m.n2 = n2;
   return launch_mutual(m, L.blocks, dtype, out_pairs, out_score, capacity, out_count, st);

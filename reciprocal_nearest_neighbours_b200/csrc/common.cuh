@@ -6,7 +6,8 @@
 // so the maximum key over a set of candidates is the highest score with the
 // LOWEST index among equal scores, and partial results from any number of
 // CTAs merge with one 64-bit atomicMax in any order, deterministically.
-// key == 0 means "no candidate yet".
+// key == 0 means "no candidate yet". Pointmap keys carry the score
+// -(squared distance), so the maximum is the nearest point.
 #pragma once
 
 #include <cstdint>
@@ -57,12 +58,6 @@ __host__ __device__ constexpr int row_bytes(int dtype, int d) {
   return dtype == FASTNN_F32_L2 ? 16 : elem_bytes(dtype) * (d <= 32 ? 32 : 64);
 }
 
-// Squared Euclidean distance of two repacked pointmap rows, in fp32 from the
-// coordinate differences (the .w components hold -|p|^2 and are ignored).
-__device__ __forceinline__ float sq_dist3(float4 a, float4 b) {
-  const float dx = a.x - b.x, dy = a.y - b.y, dz = a.z - b.z;
-  return __fmaf_rn(dz, dz, __fmaf_rn(dy, dy, dx * dx));
-}
 
 // Where the query rows of one nearest-neighbour pass come from.
 //   row id of slot k of pair b:

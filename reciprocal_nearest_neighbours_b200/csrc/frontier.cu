@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(1024) mutual_emit_kernel(MutualSrc m,
           if (DT == FASTNN_I8)
             static_cast<int32_t*>(out_score)[pos] = unord_i32(h);
           else if (DT == FASTNN_F32_L2)
-            static_cast<float*>(out_score)[pos] = sq_dist3(m.pts1[i], m.pts2[j]);
+            static_cast<float*>(out_score)[pos] = -unord_f32(h);
           else
             static_cast<float*>(out_score)[pos] = unord_f32(h);
         } else if (m.score12) {
@@ -161,9 +161,7 @@ __global__ void __launch_bounds__(1024) mutual_emit_kernel(MutualSrc m,
 // ------------------------------------------------------------ decode nn ---
 template <int DT>
 __global__ void decode_kernel(const uint64_t* __restrict__ key, int64_t n,
-                              int32_t* __restrict__ out_idx, void* __restrict__ out_score,
-                              const float4* __restrict__ q_pts,
-                              const float4* __restrict__ db_pts, int64_t ndb) {
+                              int32_t* __restrict__ out_idx, void* __restrict__ out_score) {
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const uint64_t k = key[i];
@@ -172,8 +170,7 @@ __global__ void decode_kernel(const uint64_t* __restrict__ key, int64_t n,
       if (DT == FASTNN_I8)
         static_cast<int32_t*>(out_score)[i] = unord_i32(key_score_bits(k));
       else if (DT == FASTNN_F32_L2)
-        static_cast<float*>(out_score)[i] =
-            key_index(k) < ndb ? sq_dist3(q_pts[i], db_pts[key_index(k)]) : INFINITY;
+        static_cast<float*>(out_score)[i] = k ? -unord_f32(key_score_bits(k)) : INFINITY;
       else
         static_cast<float*>(out_score)[i] = unord_f32(key_score_bits(k));
     }
@@ -182,9 +179,11 @@ __global__ void decode_kernel(const uint64_t* __restrict__ key, int64_t n,
 
 // Pointmap rows: float32 [rows][d] (d <= 3) -> float4 (x, y, z, -|p|^2),
 // missing coordinates zero; pad_rows zero rows follow. The norm is computed
-// in fp32 as fma(z, z, fma(y, y, x * x)).
+// in fp32 as fma(z, z, fma(y, y, x * x)); its maximum over the map goes to
+// *max_p2 (fp32 bits; non-negative floats order like their bits).
 __global__ void repack_l2_kernel(const float* __restrict__ src, int64_t rows, int d,
-                                 float4* __restrict__ dst, int64_t pad_rows) {
+                                 float4* __restrict__ dst, int64_t pad_rows, int* max_p2) {
+  float mx = 0.f;
   for (int64_t row = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
        row < rows + pad_rows; row += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -193,9 +192,16 @@ __global__ void repack_l2_kernel(const float* __restrict__ src, int64_t rows, in
       p.x = __ldg(s);
       if (d > 1) p.y = __ldg(s + 1);
       if (d > 2) p.z = __ldg(s + 2);
-      p.w = -__fmaf_rn(p.z, p.z, __fmaf_rn(p.y, p.y, p.x * p.x));
+      const float n2 = __fmaf_rn(p.z, p.z, __fmaf_rn(p.y, p.y, p.x * p.x));
+      p.w = -n2;
+      mx = fmaxf(mx, n2);
     }
     dst[row] = p;
+  }
+  if (max_p2) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if ((threadIdx.x & 31) == 0 && mx > 0.f) atomicMax(max_p2, __float_as_int(mx));
   }
 }
 
@@ -217,7 +223,7 @@ int launch_repack(const void* src, int64_t rows, int d, int dtype, void* dst, in
   const int g = grid_for(total, 256);
   if (dtype == FASTNN_F32_L2) {
     repack_l2_kernel<<<g, 256, 0, st>>>(static_cast<const float*>(src), rows, d,
-                                        static_cast<float4*>(dst), pad_rows);
+                                        static_cast<float4*>(dst), pad_rows, absmax);
     FASTNN_CUDA_TRY(cudaGetLastError());
     return FASTNN_OK;
   }
@@ -261,16 +267,15 @@ int launch_mutual(const MutualSrc& m, int32_t* block_scratch, int dtype, int32_t
 }
 
 int launch_decode(const uint64_t* key, int64_t n, int dtype, int32_t* out_idx, void* out_score,
-                  cudaStream_t st, const float4* q_pts, const float4* db_pts, int64_t ndb) {
+                  cudaStream_t st) {
   if (n <= 0) return FASTNN_OK;
   const int g = grid_for(n, 256);
   if (dtype == FASTNN_I8)
-    decode_kernel<FASTNN_I8><<<g, 256, 0, st>>>(key, n, out_idx, out_score, nullptr, nullptr, 0);
+    decode_kernel<FASTNN_I8><<<g, 256, 0, st>>>(key, n, out_idx, out_score);
   else if (dtype == FASTNN_F32_L2)
-    decode_kernel<FASTNN_F32_L2><<<g, 256, 0, st>>>(key, n, out_idx, out_score, q_pts, db_pts,
-                                                    ndb);
+    decode_kernel<FASTNN_F32_L2><<<g, 256, 0, st>>>(key, n, out_idx, out_score);
   else
-    decode_kernel<FASTNN_BF16><<<g, 256, 0, st>>>(key, n, out_idx, out_score, nullptr, nullptr, 0);
+    decode_kernel<FASTNN_BF16><<<g, 256, 0, st>>>(key, n, out_idx, out_score);
   FASTNN_CUDA_TRY(cudaGetLastError());
   return FASTNN_OK;
 }

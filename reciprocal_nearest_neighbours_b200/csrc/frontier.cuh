@@ -17,8 +17,6 @@ struct CompactArgs {
   uint32_t* claim;        // [batch][N1] first-visit stamps (round << 24 | slot)
   int64_t N1;
   int64_t N2;
-  const float4* pts1;     // pointmaps: repacked rows [batch][N1] (score = |p1 - p2|^2)
-  const float4* pts2;     // pointmaps: repacked rows [batch][N2]
   int32_t* out_pairs;     // [batch][cap][2]
   void* out_score;        // [batch][cap] or nullptr
   int64_t cap;
@@ -43,6 +41,9 @@ struct RecArgs {
   int* status;
 };
 
+// Repack `rows` rows (plus pad_rows zero rows) into the kernels' layout.
+// absmax (optional) receives, by atomicMax, the largest |element| (int8) or
+// the fp32 bits of the largest |p|^2 (pointmaps).
 int launch_repack(const void* src, int64_t rows, int d, int dtype, void* dst, int64_t pad_rows,
                   int* absmax, cudaStream_t st);
 // Nearest-neighbour results for the mutual test: packed keys (k12/k21) or
@@ -54,8 +55,6 @@ struct MutualSrc {
   const int32_t* nn12;
   const int32_t* nn21;
   const void* score12;
-  const float4* pts1;  // pointmaps with keys: repacked rows of image 1 (local rows) and 2
-  const float4* pts2;
   int64_t n1;  // local image-1 rows
   int64_t n2;  // image-2 rows
   int64_t i0;  // global index of local row 0
@@ -64,11 +63,9 @@ struct MutualSrc {
 int mutual_blocks(int64_t n1);
 int launch_mutual(const MutualSrc& m, int32_t* block_scratch, int dtype, int32_t* out_pairs,
                   void* out_score, int64_t cap, int32_t* out_count, cudaStream_t st);
-// Keys -> (index, score). For pointmaps the score is the squared distance
-// of query row i (q_pts) and its nearest row (db_pts, ndb rows), both
-// repacked; a key without a candidate (index >= ndb) gets +inf.
+// Keys -> (index, score); pointmap scores are the squared distances the keys
+// carry (negated).
 int launch_decode(const uint64_t* key, int64_t n, int dtype, int32_t* out_idx, void* out_score,
-                  cudaStream_t st, const float4* q_pts = nullptr, const float4* db_pts = nullptr,
-                  int64_t ndb = 0);
+                  cudaStream_t st);
 
 }  // namespace fastnn

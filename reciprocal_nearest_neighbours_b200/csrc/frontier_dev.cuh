@@ -163,8 +163,7 @@ __device__ void compact_pair(const CompactArgs& c, const FrontierBufs& fb, int b
           if (DT == FASTNN_I8)
             static_cast<int32_t*>(c.out_score)[b * c.cap + pos] = unord_i32(key_score_bits(fk));
           else if (DT == FASTNN_F32_L2)
-            static_cast<float*>(c.out_score)[b * c.cap + pos] =
-                sq_dist3(c.pts1[b * c.N1 + u], c.pts2[b * c.N2 + v]);
+            static_cast<float*>(c.out_score)[b * c.cap + pos] = -unord_f32(key_score_bits(fk));
           else
             static_cast<float*>(c.out_score)[b * c.cap + pos] = unord_f32(key_score_bits(fk));
         }

@@ -11,19 +11,34 @@
 // fused multiply-adds, issued as FFMA2 on a pair of database rows, and a
 // three-input max folds both scores of the pair into the running maximum.
 //
+// Exact ranking. The fp32 score s~ is within E = 8 u (|a| + R)^2 of s
+// (u = 2^-24, R = the largest |p| of the database, measured by the repack
+// kernel; the rounding analysis of the six operations gives 6 u plus
+// second-order terms). A point whose s~ is more than 2E below the largest s~
+// seen cannot be the nearest, so only the points inside that window are
+// ranked again, by their squared distance computed in fp64 from the
+// coordinate differences -- (dx^2 + dy^2) + dz^2, each operation rounded
+// once, the order of a plain loop over the coordinates -- and rounded to
+// fp32. The result is the lowest index among the points whose fp64 squared
+// distance rounds to the same fp32 value as the smallest one, and the score
+// reported is that fp32 value.
+//
 // Work: units (pair b, 128-query tile m, 1024-row database chunk n), split
 // into contiguous ranges over persistent CTAs of 16 warps. Each chunk comes
 // into shared memory with one bulk copy on the TMA engine (double-buffered,
 // completion on an mbarrier, every wait bounded). Each warp holds 8 queries
 // in registers and its lanes stride over the chunk (lane l scores rows
-// 64 s + l and 64 s + 32 + l). Per chunk a lane keeps only the maximum score
-// of each query; when a warp vote finds a lane above the warp's best so far,
-// the warp reduces the maximum, and all 32 lanes re-score the 32 rows of the
-// lane holding it (same FMA order, so bit-identical scores) to find its
-// first, i.e. lowest-index, row with that score. Consecutive chunks of one
-// (pair, tile) form a segment; at its end lane q of each warp merges query
-// q's (score, index) into the 64-bit key with atomicMax: the highest score
-// (nearest point) with the lowest index, whatever the order of the merges.
+// 64 s + l and 64 s + 32 + l). Per chunk a lane keeps only the maximum s~ of
+// each query; a warp vote asks whether any lane reached the query's window.
+// Only then does the warp reduce the maximum and walk the lanes inside the
+// window: all 32 lanes re-score the 32 rows of one such lane (same FMA order,
+// so bit-identical s~), rank the rows inside the window by fp64 distance and
+// fold the best (fp32 distance, index) key into the query's winner. The
+// warp's per-query state (largest s~, window width, winner) lives in shared
+// memory. Consecutive chunks of one (pair, tile) form a segment; at its end
+// lane q of each warp merges query q's winner into the 64-bit key with
+// atomicMax on (ordered -distance, inverted index): the nearest point with
+// the lowest index, whatever the order of the merges.
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -44,8 +59,16 @@ constexpr int kSteps = kDC / 64;    // 64-row steps per chunk: two rows per lane
 constexpr int kMaxBatchL2 = 1024;
 constexpr unsigned kFull = 0xffffffffu;
 
+// Per-warp, per-query state of the exact ranking (warp-uniform values).
+struct WarpState {
+  float smax[kQW];                // largest fp32 score s~ seen in the segment
+  float win2[kQW];                // window width 2E
+  unsigned long long key[kQW];    // (fp32 distance bits << 32) | index, minimum so far
+};
+
 struct __align__(16) L2Smem {
   float4 buf[2][kDC];
+  WarpState ws[kWarps];
   unsigned long long bar[2];
   uint32_t bar_phase[2];
   int pending[2];  // a bulk copy into buffer i is in flight (thread 0's view)
@@ -157,8 +180,11 @@ struct Queries {
   float2 x[kQW], y[kQW], z[kQW];  // (2 q, 2 q) per coordinate, both halves equal
 };
 
+// Loads the warp's 8 queries and resets its ranking state. max_p2 = largest
+// |p|^2 (fp32) over the database.
 __device__ __forceinline__ void load_queries(const NNArgs& a, const PhaseQ& q, int b, int64_t k0,
-                                             int cnt, int lane, Queries& Q) {
+                                             int cnt, int lane, float max_p2, WarpState& W,
+                                             Queries& Q) {
   float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
   const int64_t k = k0 + lane;
   if (lane < kQW && k < cnt) {
@@ -166,6 +192,16 @@ __device__ __forceinline__ void load_queries(const NNArgs& a, const PhaseQ& q, i
     if (row >= 0 && row < a.q_rows_per_pair)
       v = __ldg(reinterpret_cast<const float4*>(a.q_rows) + b * a.q_rows_per_pair + row);
   }
+  if (lane < kQW) {
+    // 2E = 16 u (|a| + R)^2; the norms come from fp32 sums (relative error
+    // below 3 u), inflated by 2^-20 to stay an upper bound.
+    const float ra = sqrtf(fmaxf(-v.w, 0.f)) * (1.f + 0x1p-20f);
+    const float rp = sqrtf(max_p2) * (1.f + 0x1p-20f);
+    W.win2[lane] = 0x1p-20f * (ra + rp) * (ra + rp) * (1.f + 0x1p-20f);
+    W.smax[lane] = -INFINITY;
+    W.key[lane] = ~0ull;
+  }
+  __syncwarp();
 #pragma unroll
   for (int i = 0; i < kQW; ++i) {
     const float x = 2.f * __shfl_sync(kFull, v.x, i);
@@ -191,10 +227,18 @@ __device__ __forceinline__ void score_pair(const float4 p0, const float4 p1, con
   }
 }
 
+// fp64 squared distance of query (ax, ay, az) and point p in the order of a
+// plain loop over the coordinates, one rounding per operation.
+__device__ __forceinline__ double dist2_f64(float ax, float ay, float az, const float4 p) {
+  const double dx = __dsub_rn(static_cast<double>(ax), static_cast<double>(p.x));
+  const double dy = __dsub_rn(static_cast<double>(ay), static_cast<double>(p.y));
+  const double dz = __dsub_rn(static_cast<double>(az), static_cast<double>(p.z));
+  return __dadd_rn(__dadd_rn(__dmul_rn(dx, dx), __dmul_rn(dy, dy)), __dmul_rn(dz, dz));
+}
+
 // One chunk (rows valid rows at database index base) for one warp.
 __device__ __forceinline__ void l2_chunk(const float4* __restrict__ buf, int rows, uint32_t base,
-                                         const Queries& Q, float (&best)[kQW],
-                                         uint32_t (&bidx)[kQW], int lane) {
+                                         const Queries& Q, WarpState& W, int lane) {
   float mx[kQW];
 #pragma unroll
   for (int i = 0; i < kQW; ++i) mx[i] = -INFINITY;
@@ -210,35 +254,48 @@ __device__ __forceinline__ void l2_chunk(const float4* __restrict__ buf, int row
       score_pair(j0 < rows ? buf[j0] : never, j1 < rows ? buf[j1] : never, Q, mx);
     }
   }
+  // Row t of lane L in increasing order: 64 (t >> 1) + 32 (t & 1) + L.
+  const int jt = 64 * (lane >> 1) + 32 * (lane & 1);
 #pragma unroll
   for (int i = 0; i < kQW; ++i) {
-    if (!__any_sync(kFull, mx[i] > best[i])) continue;
+    const float win2 = W.win2[i];
+    if (!__any_sync(kFull, mx[i] > -INFINITY && mx[i] >= W.smax[i] - win2)) continue;
     float M = mx[i];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
-    // Lanes holding the maximum; lane t re-scores the t-th row of each
-    // (rows of lane L in increasing order: 64 (t >> 1) + 32 (t & 1) + L).
-    unsigned cand = __ballot_sync(kFull, mx[i] == M);
-    uint32_t J = 0xFFFFFFFFu;
-    const int jt = 64 * (lane >> 1) + 32 * (lane & 1);
+    const float smax = fmaxf(W.smax[i], M);
+    const float thr = smax - win2;
+    const float ax = 0.5f * Q.x[i].x, ay = 0.5f * Q.y[i].x, az = 0.5f * Q.z[i].x;
+    unsigned long long best = W.key[i];
+    unsigned cand = __ballot_sync(kFull, mx[i] >= thr);
     while (cand) {
       const int L = __ffs(cand) - 1;
       cand &= cand - 1;
-      float sc = -INFINITY;
-      if (jt + L < rows) {
-        const float4 p = buf[jt + L];
-        sc = __fmaf_rn(Q.z[i].x, p.z, __fmaf_rn(Q.y[i].x, p.y, __fmaf_rn(Q.x[i].x, p.x, p.w)));
+      unsigned long long key = ~0ull;
+      const int j = jt + L;
+      if (j < rows) {
+        const float4 p = buf[j];
+        const float sc =
+            __fmaf_rn(Q.z[i].x, p.z, __fmaf_rn(Q.y[i].x, p.y, __fmaf_rn(Q.x[i].x, p.x, p.w)));
+        if (sc >= thr) {
+          const float d2 = __double2float_rn(dist2_f64(ax, ay, az, p));
+          key = (static_cast<unsigned long long>(__float_as_uint(d2)) << 32) |
+                static_cast<unsigned long long>(base + static_cast<uint32_t>(j));
+        }
       }
-      const unsigned hit = __ballot_sync(kFull, sc == M);
-      if (hit) {
-        const int t = __ffs(hit) - 1;
-        J = min(J, static_cast<uint32_t>(64 * (t >> 1) + 32 * (t & 1) + L));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const unsigned long long other = __shfl_xor_sync(kFull, key, o);
+        key = other < key ? other : key;
       }
+      best = key < best ? key : best;
     }
-    if (J != 0xFFFFFFFFu) {
-      best[i] = M;
-      bidx[i] = base + J;
+    __syncwarp();
+    if (lane == 0) {
+      W.smax[i] = smax;
+      W.key[i] = best;
     }
+    __syncwarp();
   }
 }
 
@@ -258,8 +315,8 @@ __device__ void l2_phase(const NNArgs& a, const PhaseQ q, L2Smem& s) {
   int64_t m = s.m0, n = s.n0;
   if (threadIdx.x == 0) l2_issue(a, s, 0, b, n);
   Queries Q;
-  float best[kQW];
-  uint32_t bidx[kQW];
+  WarpState& W = s.ws[warp];
+  const float max_p2 = a.db_absmax ? __int_as_float(__ldcg(a.db_absmax)) : INFINITY;
   bool seg_start = true, ok = true;
   for (int64_t u = u0; u < u1; ++u) {
     const int i = static_cast<int>((u - u0) & 1);
@@ -278,26 +335,21 @@ __device__ void l2_phase(const NNArgs& a, const PhaseQ q, L2Smem& s) {
     if (threadIdx.x == 0 && u + 1 < u1) l2_issue(a, s, i ^ 1, nb, nn);
     const int64_t k0 = m * kQT + warp * kQW;
     const bool active = k0 < s.cnt[b];  // warp-uniform
-    if (seg_start) {
-      load_queries(a, q, b, k0, s.cnt[b], lane, Q);
-#pragma unroll
-      for (int j = 0; j < kQW; ++j) {
-        best[j] = -INFINITY;
-        bidx[j] = 0xFFFFFFFFu;
-      }
-    }
+    if (seg_start) load_queries(a, q, b, k0, s.cnt[b], lane, max_p2, W, Q);
     ok = l2_wait(s, i, ph[i], a.status) && ok;
     ph[i] ^= 1u;
     if (threadIdx.x == 0 && ok) s.pending[i] = 0;
     const int rows = static_cast<int>(min(static_cast<int64_t>(kDC), a.ndb - n * kDC));
-    if (active && ok) l2_chunk(s.buf[i], rows, static_cast<uint32_t>(n * kDC), Q, best, bidx, lane);
+    if (active && ok) l2_chunk(s.buf[i], rows, static_cast<uint32_t>(n * kDC), Q, W, lane);
     const bool seg_end = (nn == 0) || (u + 1 == u1);
-    if (seg_end && active && ok) {
-#pragma unroll
-      for (int j = 0; j < kQW; ++j)
-        if (lane == j && k0 + j < s.cnt[b] && bidx[j] != 0xFFFFFFFFu)
-          atomicMax(reinterpret_cast<unsigned long long*>(&a.out_key[b * a.q_cap + k0 + j]),
-                    static_cast<unsigned long long>(make_key(ord_f32(best[j]), bidx[j])));
+    if (seg_end && active && ok && lane < kQW && k0 + lane < s.cnt[b]) {
+      const unsigned long long w = W.key[lane];
+      if (w != ~0ull) {
+        const float d2 = __uint_as_float(static_cast<uint32_t>(w >> 32));
+        atomicMax(reinterpret_cast<unsigned long long*>(&a.out_key[b * a.q_cap + k0 + lane]),
+                  static_cast<unsigned long long>(
+                      make_key(ord_f32(-d2), static_cast<uint32_t>(w & 0xFFFFFFFFu))));
+      }
     }
     seg_start = seg_end;
     b = nb;

@@ -1,17 +1,18 @@
 """GPU parity of the pointmap path (nearest 3D point; FASTNN_F32_L2).
 
-Tolerance, from the kernel's fp32 arithmetic. The kernel ranks database
-points p for a query a by s = 2<a, p> - |p|^2, formed as three fused
-multiply-adds on top of -|p|^2 (itself one multiply and two fused
-multiply-adds). Each rounding is at most u = 2^-24 of a partial sum bounded
-by (|a| + |p|)^2, so |s~ - s| <= 6 u (|a| + |p|)^2, and two candidates can
-swap only when their exact squared distances differ by less than
-12 u (|a| + R)^2, R = max |p| over the database; the tests use 16 u. The
-reported score is the squared distance recomputed from the coordinate
-differences (relative error below 8 u).
+What the GPU returns, by construction: the nearest point by the fp64
+squared distance (dx^2 + dy^2) + dz^2 (the oracle's own expression and
+order) rounded to fp32, the lowest index among points whose fp32 values tie;
+the score is that fp32 value. (The fp32 scan only preselects; every point its
+rounding error could place first is re-ranked this way.) So against the
+oracle, which ranks by the fp64 value itself:
 
-Integer-valued points make every one of those operations exact in fp32, so
-there the GPU must agree with the oracle bit for bit, ties included.
+* scores equal float32(oracle squared distance) bit for bit;
+* an index differs only when two fp64 distances round to the same fp32
+  value, and then the GPU's index is the lower one.
+
+Integer-valued points make all arithmetic exact, so there every result must
+match the oracle exactly, ties included.
 """
 
 from __future__ import annotations
@@ -24,12 +25,13 @@ import oracle
 import synth
 from reciprocal_nearest_neighbours_b200 import fastnn_mutual_dense, fastnn_nn, fastnn_reciprocal
 from tests._dev import gpu_pairs, require_cuda
-from tests.test_gpu_reciprocal import as_set, expected_rounds
+from tests.test_gpu_reciprocal import expected_rounds
 from tests.test_oracle_l2 import load_pointmap_golden
 
 pytestmark = pytest.mark.gpu
 
-U = 2.0 ** -24
+# An oracle walk whose top-2 margin is this small may pass an fp32 collision.
+COLLISION_GAP = 1e-9
 
 
 @pytest.fixture(autouse=True)
@@ -41,25 +43,22 @@ def dev(a: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
 
 
-def tol_for(q: np.ndarray, db: np.ndarray) -> np.ndarray:
-    R = np.sqrt((db.astype(np.float64) ** 2).sum(1)).max()
-    return 16 * U * (np.sqrt((q.astype(np.float64) ** 2).sum(1)) + R) ** 2
+def f32(x):
+    return np.asarray(x, dtype=np.float64).astype(np.float32)
 
 
 def check_nn_l2(idx_g, score_g, q, db):
-    """Tolerance rule: the chosen point is within tol of the nearest, the
-    reported squared distance is that of the chosen point, and the index
-    differs from the oracle's only where its top-2 margin is below tol."""
+    """Scores are float32 of the fp64 distance of the chosen point; the chosen
+    point ties the oracle's in fp32 and is never a higher index."""
     ref = oracle.nn(q, db, "l2")
     idx = idx_g.cpu().numpy().astype(np.int64)
-    sc = score_g.cpu().numpy().astype(np.float64)
+    sc = score_g.cpu().numpy()
     assert np.all((idx >= 0) & (idx < len(db)))
-    tol = tol_for(q, db)
     exact = oracle.score_of(q, np.arange(len(q)), db, idx, "l2")
-    assert np.all(exact - ref.score <= tol)
-    assert np.all(np.abs(sc - exact) <= 8 * U * exact + 1e-30)
+    assert np.array_equal(sc, f32(exact))
+    assert np.array_equal(f32(exact), f32(ref.score))
     diff = idx != ref.idx
-    assert np.all(oracle.margin(ref, "l2")[diff] < tol[diff])
+    assert np.all(idx[diff] < ref.idx[diff])
     return int(diff.sum())
 
 
@@ -77,7 +76,7 @@ def test_nn_l2_random_points_within_tolerance(nq, ndb, d):
     db = rng.uniform(-3, 3, size=(ndb, d)).astype(np.float32)
     idx, score = fastnn_nn(dev(q), dev(db))
     torch.cuda.synchronize()
-    assert check_nn_l2(idx, score, q, db) <= max(1, nq // 100)
+    check_nn_l2(idx, score, q, db)
 
 
 @pytest.mark.parametrize("nq,ndb,d,amp", [(300, 1000, 3, 2), (700, 2049, 3, 8), (129, 300, 1, 3),
@@ -107,7 +106,7 @@ def test_nn_l2_full_size_pointmap_sampled_queries():
     rng = np.random.default_rng(3)
     qi = np.sort(rng.choice(D1.shape[0], size=512, replace=False))
     idx, score = fastnn_nn(dev(D1[qi]), dev(D2))
-    assert check_nn_l2(idx, score, D1[qi], D2) <= 10
+    assert check_nn_l2(idx, score, D1[qi], D2) == 0
 
 
 # ---------------------------------------------------------------- fast matching
@@ -175,26 +174,28 @@ def test_fast_l2_noise_free_permutation():
 
 
 def check_fast_l2_certificate(m1, m2, sub, max_iter, gpu=None):
-    """Each GPU pair is reciprocal up to the tolerance, its score is its
-    squared distance, and each oracle pair the GPU lacks sits at the end of
-    walks that all pass a near-tie."""
+    """Kept pairs and their scores equal the oracle's, except pairs reached
+    only through walks that pass an fp32 collision (oracle margin below
+    COLLISION_GAP); the GPU round count matches unless such a walk exists."""
     H1, W1, _ = m1.shape
     H2, W2, _ = m2.shape
     pairs, score, count, iters = gpu if gpu is not None else run_fast(m1, m2, sub, max_iter)
     p, s = gpu_pairs(pairs, score, count)
     D1, D2 = m1.reshape(-1, 3), m2.reshape(-1, 3)
-    tol = 16 * U * (2 * max(np.sqrt((D1.astype(np.float64) ** 2).sum(1)).max(),
-                            np.sqrt((D2.astype(np.float64) ** 2).sum(1)).max())) ** 2
-    exact = oracle.score_of(D1, p[:, 0], D2, p[:, 1], "l2")
-    assert np.all(np.abs(s - exact) <= 8 * U * exact + 1e-30)
-    r12 = oracle.nn(D1[p[:, 0]], D2, "l2")
-    r21 = oracle.nn(D2[p[:, 1]], D1, "l2")
-    assert np.all(exact - r12.score <= tol) and np.all(exact - r21.score <= tol)
+    assert np.array_equal(s, f32(oracle.score_of(D1, p[:, 0], D2, p[:, 1], "l2")))
     ref = oracle.fast_reciprocal(m1, H1, W1, m2, H2, W2, "l2", sub, max_iter, track_gaps=True)
     got = set(map(tuple, p.tolist()))
     exp = set(map(tuple, ref.pairs.tolist()))
     for u, v in exp - got:
-        assert ref.min_gap[u] < tol, (u, v, ref.min_gap[u], tol)
+        assert ref.min_gap[u] < COLLISION_GAP, (u, v, ref.min_gap[u])
+    for u, v in got - exp:
+        # a walk that left the oracle's path at a collision still ends at a
+        # pair of mutually nearest points (in fp32)
+        d2 = f32(oracle.score_of(D1, np.array([u]), D2, np.array([v]), "l2"))[0]
+        assert d2 == f32(oracle.nn(D1[[u]], D2, "l2").score)[0], (u, v)
+        assert d2 == f32(oracle.nn(D2[[v]], D1, "l2").score)[0], (u, v)
+    if got == exp:
+        assert int(iters[0]) == expected_rounds(ref)
     return len(got ^ exp), len(exp)
 
 
@@ -208,7 +209,7 @@ def test_fast_l2_pair_512x384_full_size():
     w = synth.make_workload("pair_512x384_pts3_f32")
     p = w.pairs[0]
     symdiff, n = check_fast_l2_certificate(p.desc1, p.desc2, w.subsample, w.max_iter)
-    assert n > 1000 and symdiff <= 0.05 * n
+    assert n > 1000 and symdiff == 0
 
 
 def test_fast_l2_batch_pairs_independent():
@@ -239,21 +240,39 @@ def test_dense_l2_integer_points_exact(n1, n2, d, amp):
     assert np.array_equal(s.astype(np.float64), ref.score)
 
 
-def test_dense_l2_pointmaps_within_tolerance():
+def test_dense_l2_pointmaps_match_oracle():
     m = synth.pointmap_pair(800, H=48, W=64)
     D1, D2 = m.desc1.reshape(-1, 3), m.desc2.reshape(-1, 3)
     pairs, score, count = fastnn_mutual_dense(dev(D1), dev(D2))
     p, s = gpu_pairs(pairs, score, count)
-    exact = oracle.score_of(D1, p[:, 0], D2, p[:, 1], "l2")
-    assert np.all(np.abs(s - exact) <= 8 * U * exact + 1e-30)
+    assert np.array_equal(s, f32(oracle.score_of(D1, p[:, 0], D2, p[:, 1], "l2")))
     ref = oracle.dense_mutual(D1, D2, "l2")
-    tol1 = tol_for(D1, D2)
-    tol2 = tol_for(D2, D1)
     got = set(map(tuple, p.tolist()))
     exp = set(map(tuple, ref.pairs.tolist()))
     m12 = oracle.margin(ref.nn12, "l2")
     m21 = oracle.margin(ref.nn21, "l2")
     for i, j in got ^ exp:
         jj = ref.nn12.idx[i]
-        assert min(m12[i] - tol1[i], m21[jj] - tol2[jj], m21[j] - tol2[j]) < 0
-    assert len(got ^ exp) <= 0.02 * len(exp)
+        assert min(m12[i], m21[jj], m21[j]) < COLLISION_GAP
+    assert got == exp
+
+
+def test_dense_l2_full_size_sampled():
+    """All 196,608 x 196,608 distances of the full pointmap pair: output
+    structure, scores, and the oracle's verdict on sampled pixels."""
+    m = synth.make_workload("dense_512x384_pts3_f32").pairs[0]
+    D1, D2 = m.desc1.reshape(-1, 3), m.desc2.reshape(-1, 3)
+    pairs, score, count = fastnn_mutual_dense(dev(D1), dev(D2))
+    p, s = gpu_pairs(pairs, score, count)
+    assert len(p) > 10000
+    assert np.all(np.diff(p[:, 0]) > 0) and len(np.unique(p[:, 1])) == len(p)
+    assert np.array_equal(s, f32(oracle.score_of(D1, p[:, 0], D2, p[:, 1], "l2")))
+    rng = np.random.default_rng(6)
+    sel = p[rng.choice(len(p), size=300, replace=False)]
+    assert np.array_equal(oracle.nn(D1[sel[:, 0]], D2, "l2").idx, sel[:, 1])
+    assert np.array_equal(oracle.nn(D2[sel[:, 1]], D1, "l2").idx, sel[:, 0])
+    probe = np.sort(rng.choice(D1.shape[0], size=300, replace=False))
+    v = oracle.nn(D1[probe], D2, "l2").idx
+    back = oracle.nn(D2[v], D1, "l2").idx
+    kept = set(p[:, 0].tolist())
+    assert all((int(u) in kept) == (int(b) == int(u)) for u, b in zip(probe, back))
