@@ -8,8 +8,10 @@
 //     s(a, p) = 2<a, p> - |p|^2 = |a|^2 - |a - p|^2,
 // so argmax_p s is the nearest point. A repacked row holds (x, y, z, -|p|^2)
 // (the norm computed once per point by the repack kernel); one score is three
-// fused multiply-adds, issued as FFMA2 on a pair of database rows, and a
-// three-input max folds both scores of the pair into the running maximum.
+// fused multiply-adds, and a three-input max folds the scores of two rows
+// into the running maximum. (Packed FFMA2 on pairs of rows measured no
+// faster on B200: the packing moves cost more than they save, and with a
+// pre-paired layout the gain was 3%.)
 //
 // Exact ranking. The fp32 score s~ is within E = 8 u (|a| + R)^2 of s
 // (u = 2^-24, R = the largest |p| of the database, measured by the repack
@@ -24,21 +26,27 @@
 // reported is that fp32 value.
 //
 // Work: units (pair b, 128-query tile m, 1024-row database chunk n), split
-// into contiguous ranges over persistent CTAs of 16 warps. Each chunk comes
-// into shared memory with one bulk copy on the TMA engine (double-buffered,
-// completion on an mbarrier, every wait bounded). Each warp holds 8 queries
-// in registers and its lanes stride over the chunk (lane l scores rows
-// 64 s + l and 64 s + 32 + l). Per chunk a lane keeps only the maximum s~ of
-// each query; a warp vote asks whether any lane reached the query's window.
-// Only then does the warp reduce the maximum and walk the lanes inside the
-// window: all 32 lanes re-score the 32 rows of one such lane (same FMA order,
-// so bit-identical s~), rank the rows inside the window by fp64 distance and
-// fold the best (fp32 distance, index) key into the query's winner. The
-// warp's per-query state (largest s~, window width, winner) lives in shared
-// memory. Consecutive chunks of one (pair, tile) form a segment; at its end
-// lane q of each warp merges query q's winner into the 64-bit key with
-// atomicMax on (ordered -distance, inverted index): the nearest point with
-// the lowest index, whatever the order of the merges.
+// into contiguous ranges over persistent CTAs of 16 warps. Chunks come into a
+// 4-deep ring of shared-memory buffers by bulk copies on the TMA engine,
+// completing on one mbarrier per buffer (every wait bounded). There is no
+// CTA-wide barrier per chunk: each warp counts itself out of a buffer when it
+// is done with it, and the last warp out issues the copy of the unit four
+// ahead into it, so warps drift up to three chunks apart and uneven work
+// evens out. Each warp holds 8 queries in registers and its lanes stride over
+// the chunk (lane l scores rows 64 s + l and 64 s + 32 + l). Per chunk a lane
+// keeps only the maximum s~ of each query; a warp vote asks whether any lane
+// reached the query's window. Only then does the warp reduce the maximum and
+// walk the lanes inside the window: all 32 lanes re-score the 32 rows of one
+// such lane (same FMA order, so bit-identical s~), rank the rows inside the
+// window by fp64 distance and fold the best (fp32 distance, index) key into
+// the query's winner. Consecutive units of one (pair, tile) form a segment,
+// visiting the database chunks in a scrambled order (the ranking does not
+// depend on the order, and spatially ordered rows would otherwise open the
+// re-ranking at nearly every chunk); at its end lane q of each warp merges
+// query q's winner into the 64-bit key with atomicMax on (ordered -distance,
+// inverted index): the nearest point with the lowest index, whatever the
+// order of the merges.
+#include <cfloat>
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -56,38 +64,50 @@ constexpr int kQW = 8;              // queries per warp, held by every lane
 constexpr int kQT = kWarps * kQW;   // queries per tile
 constexpr int kDC = 1024;           // database rows per chunk (16 KB)
 constexpr int kSteps = kDC / 64;    // 64-row steps per chunk: two rows per lane per step
+constexpr int kNS = 4;              // chunk ring depth
 constexpr int kMaxBatchL2 = 1024;
 constexpr unsigned kFull = 0xffffffffu;
 
-// Per-warp, per-query state of the exact ranking (warp-uniform values).
+// Per-warp, per-query state of the exact ranking that only a vote that fires
+// touches (warp-uniform values).
 struct WarpState {
-  float smax[kQW];                // largest fp32 score s~ seen in the segment
-  float win2[kQW];                // window width 2E
-  unsigned long long key[kQW];    // (fp32 distance bits << 32) | index, minimum so far
+  unsigned long long key[kQW];  // winner: (fp32 distance bits << 32) | index
+  float smax[kQW];              // largest fp32 score s~ seen in the segment
+  float win2[kQW];              // window width 2E
 };
 
 struct __align__(16) L2Smem {
-  float4 buf[2][kDC];
+  float4 buf[kNS][kDC];
   WarpState ws[kWarps];
-  unsigned long long bar[2];
-  uint32_t bar_phase[2];
-  int pending[2];  // a bulk copy into buffer i is in flight (thread 0's view)
+  unsigned long long bar[kNS];
+  uint32_t bar_phase[kNS];  // consumers' next parity per buffer, carried across passes
+  uint32_t issued[kNS];     // copies issued into each buffer (teardown waits for the last)
+  int empty_cnt[kNS];       // warps done with the buffer's current chunk
   int abort_flag;
   int grid_ok;
   int more;
   int b0;
   long long nt, u0, u1, m0, n0;
+  long long perm;  // chunk n of a segment is database chunk (n * perm) mod nt; perm < nt
   int scan[66];
   int cnt[kMaxBatchL2];
   int mt[kMaxBatchL2];
 };
 
+constexpr size_t kSmemBytes = sizeof(L2Smem);
+
+__device__ __forceinline__ L2Smem& l2_smem() {
+  extern __shared__ __align__(16) unsigned char l2_dyn[];
+  return *reinterpret_cast<L2Smem*>(l2_dyn);
+}
+
 __device__ __forceinline__ void l2_setup(L2Smem& s) {
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kNS; ++i) {
       ptx::mbar_init(ptx::smem_u32(&s.bar[i]), 1);
       s.bar_phase[i] = 0;
-      s.pending[i] = 0;
+      s.issued[i] = 0;
+      s.empty_cnt[i] = 0;
     }
     s.abort_flag = 0;
     ptx::fence_mbar_init();
@@ -118,27 +138,63 @@ __device__ __forceinline__ bool l2_wait(L2Smem& s, int i, uint32_t parity, int* 
   return l2_wait_slow(s, i, parity, status);
 }
 
-// Thread 0: wait (bounded) for copies still in flight so that none lands
-// after the CTA has moved on; called before exit.
+// Thread 0: wait (bounded) for the last copy issued into every buffer, so
+// that none lands after the CTA has exited; called before exit.
 __device__ void l2_teardown(L2Smem& s, int* status) {
   __syncthreads();
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i)
-      if (s.pending[i]) {
+    for (int i = 0; i < kNS; ++i)
+      if (s.issued[i]) {
         const uint32_t bar = ptx::smem_u32(&s.bar[i]);
+        const uint32_t parity = (s.issued[i] - 1u) & 1u;
         const uint64_t t0 = ptx::globaltimer_ns();
-        while (!ptx::mbar_try_wait(bar, s.bar_phase[i]))
+        while (!ptx::mbar_try_wait(bar, parity))
           if (ptx::globaltimer_ns() - t0 > kTimeoutNs) {
             atomicOr(status, kStatusTimeout);
             break;
           }
-        s.pending[i] = 0;
       }
   }
   __syncthreads();
 }
 
-// Thread 0: this CTA's contiguous range of units for one pass.
+// Position of a unit: pair b, query tile m, position n in the segment and
+// the database chunk c it visits.
+struct Walk {
+  int b;
+  int64_t m, n, c;
+};
+
+__device__ __forceinline__ void walk_next(Walk& w, const L2Smem& s, int batch) {
+  ++w.n;
+  w.c += s.perm;
+  if (w.c >= s.nt) w.c -= s.nt;
+  if (w.n == s.nt) {
+    w.n = 0;
+    w.c = 0;
+    if (++w.m == s.mt[w.b]) {
+      w.m = 0;
+      do {
+        ++w.b;
+      } while (w.b < batch && s.mt[w.b] == 0);
+    }
+  }
+}
+
+// Issue the copy of database chunk w.c of pair w.b into buffer i.
+__device__ __forceinline__ void l2_issue(const NNArgs& a, L2Smem& s, int i, const Walk& w) {
+  const int64_t r0 = w.c * kDC;
+  const int64_t rows = min(static_cast<int64_t>(kDC), a.ndb - r0);
+  const uint32_t bytes = static_cast<uint32_t>(rows) * 16u;
+  const uint32_t bar = ptx::smem_u32(&s.bar[i]);
+  ptx::fence_proxy_async_smem();
+  ptx::mbar_arrive_expect_tx(bar, bytes);
+  ptx::bulk_load(ptx::smem_u32(&s.buf[i][0]), a.db_rows + (w.b * a.ndb + r0) * 16, bytes, bar);
+  s.issued[i] += 1u;
+}
+
+// Thread 0: this CTA's contiguous range of units for one pass, and the
+// copies of its first kNS units.
 __device__ void l2_plan(const NNArgs& a, const PhaseQ& q, L2Smem& s) {
   const int64_t nt = (a.ndb + kDC - 1) / kDC;
   int64_t total = 0;
@@ -151,6 +207,15 @@ __device__ void l2_plan(const NNArgs& a, const PhaseQ& q, L2Smem& s) {
   const int64_t G = gridDim.x;
   const int64_t u0 = total * blockIdx.x / G;
   s.nt = nt;
+  // A multiplier coprime with nt scatters the chunks of every segment over
+  // the database: rows of a pointmap are spatially ordered, and in storage
+  // order nearly every chunk would bring a point nearer than all before it,
+  // each time opening the exact re-ranking.
+  long long perm = 1;
+  const long long primes[6] = {97, 89, 83, 79, 73, 71};
+  for (int t = 0; t < 6 && perm == 1; ++t)
+    if (nt % primes[t] != 0) perm = primes[t] % nt == 0 ? 1 : primes[t];
+  s.perm = perm % nt;
   s.u0 = u0;
   s.u1 = total * (blockIdx.x + 1) / G;
   int64_t acc = 0;
@@ -162,29 +227,30 @@ __device__ void l2_plan(const NNArgs& a, const PhaseQ& q, L2Smem& s) {
   s.b0 = b;
   s.m0 = nt > 0 ? (u0 - acc) / nt : 0;
   s.n0 = nt > 0 ? (u0 - acc) % nt : 0;
-}
-
-// Thread 0: bring chunk n of pair b's database into buffer i.
-__device__ __forceinline__ void l2_issue(const NNArgs& a, L2Smem& s, int i, int b, int64_t n) {
-  const int64_t r0 = n * kDC;
-  const int64_t rows = min(static_cast<int64_t>(kDC), a.ndb - r0);
-  const uint32_t bytes = static_cast<uint32_t>(rows) * 16u;
-  const uint32_t bar = ptx::smem_u32(&s.bar[i]);
-  ptx::fence_proxy_async_smem();
-  ptx::mbar_arrive_expect_tx(bar, bytes);
-  ptx::bulk_load(ptx::smem_u32(&s.buf[i][0]), a.db_rows + (b * a.ndb + r0) * 16, bytes, bar);
-  s.pending[i] = 1;
+  if (!s.abort_flag) {
+    Walk w{b, s.m0, s.n0, (s.n0 * s.perm) % nt};
+    for (int64_t u = u0; u < s.u1 && u < u0 + kNS; ++u) {
+      l2_issue(a, s, static_cast<int>(u - u0), w);
+      walk_next(w, s, a.batch);
+    }
+  }
 }
 
 struct Queries {
-  float2 x[kQW], y[kQW], z[kQW];  // (2 q, 2 q) per coordinate, both halves equal
+  float x[kQW], y[kQW], z[kQW];  // 2 q per coordinate
+};
+
+// Per-query lower edge of the re-ranking window, smax - 2E, or -FLT_MAX
+// before any score (warp-uniform values, read every chunk).
+struct Window {
+  float thr[kQW];
 };
 
 // Loads the warp's 8 queries and resets its ranking state. max_p2 = largest
 // |p|^2 (fp32) over the database.
 __device__ __forceinline__ void load_queries(const NNArgs& a, const PhaseQ& q, int b, int64_t k0,
                                              int cnt, int lane, float max_p2, WarpState& W,
-                                             Queries& Q) {
+                                             Queries& Q, Window& Wn) {
   float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
   const int64_t k = k0 + lane;
   if (lane < kQW && k < cnt) {
@@ -201,30 +267,26 @@ __device__ __forceinline__ void load_queries(const NNArgs& a, const PhaseQ& q, i
     W.smax[lane] = -INFINITY;
     W.key[lane] = ~0ull;
   }
-  __syncwarp();
 #pragma unroll
   for (int i = 0; i < kQW; ++i) {
-    const float x = 2.f * __shfl_sync(kFull, v.x, i);
-    const float y = 2.f * __shfl_sync(kFull, v.y, i);
-    const float z = 2.f * __shfl_sync(kFull, v.z, i);
-    Q.x[i] = make_float2(x, x);
-    Q.y[i] = make_float2(y, y);
-    Q.z[i] = make_float2(z, z);
+    Q.x[i] = 2.f * __shfl_sync(kFull, v.x, i);
+    Q.y[i] = 2.f * __shfl_sync(kFull, v.y, i);
+    Q.z[i] = 2.f * __shfl_sync(kFull, v.z, i);
+    Wn.thr[i] = -FLT_MAX;
   }
+  __syncwarp();
+}
+
+// Score of point p for query i (2q scaled): 2<q, p> - |p|^2.
+__device__ __forceinline__ float l2_score(const Queries& Q, int i, const float4 p) {
+  return __fmaf_rn(Q.z[i], p.z, __fmaf_rn(Q.y[i], p.y, __fmaf_rn(Q.x[i], p.x, p.w)));
 }
 
 // Scores of two rows against the 8 queries, folded into mx.
 __device__ __forceinline__ void score_pair(const float4 p0, const float4 p1, const Queries& Q,
                                            float (&mx)[kQW]) {
-  const float2 X = make_float2(p0.x, p1.x), Y = make_float2(p0.y, p1.y);
-  const float2 Z = make_float2(p0.z, p1.z), N = make_float2(p0.w, p1.w);
 #pragma unroll
-  for (int i = 0; i < kQW; ++i) {
-    float2 t = __ffma2_rn(Q.x[i], X, N);
-    t = __ffma2_rn(Q.y[i], Y, t);
-    t = __ffma2_rn(Q.z[i], Z, t);
-    mx[i] = ptx::fmax3(mx[i], t.x, t.y);
-  }
+  for (int i = 0; i < kQW; ++i) mx[i] = ptx::fmax3(mx[i], l2_score(Q, i, p0), l2_score(Q, i, p1));
 }
 
 // fp64 squared distance of query (ax, ay, az) and point p in the order of a
@@ -238,12 +300,12 @@ __device__ __forceinline__ double dist2_f64(float ax, float ay, float az, const 
 
 // One chunk (rows valid rows at database index base) for one warp.
 __device__ __forceinline__ void l2_chunk(const float4* __restrict__ buf, int rows, uint32_t base,
-                                         const Queries& Q, WarpState& W, int lane) {
+                                         const Queries& Q, Window& Wn, WarpState& W, int lane) {
   float mx[kQW];
 #pragma unroll
   for (int i = 0; i < kQW; ++i) mx[i] = -INFINITY;
   if (rows == kDC) {
-#pragma unroll 2
+#pragma unroll 4
     for (int st = 0; st < kSteps; ++st)
       score_pair(buf[64 * st + lane], buf[64 * st + 32 + lane], Q, mx);
   } else {
@@ -258,42 +320,41 @@ __device__ __forceinline__ void l2_chunk(const float4* __restrict__ buf, int row
   const int jt = 64 * (lane >> 1) + 32 * (lane & 1);
 #pragma unroll
   for (int i = 0; i < kQW; ++i) {
-    const float win2 = W.win2[i];
-    if (!__any_sync(kFull, mx[i] > -INFINITY && mx[i] >= W.smax[i] - win2)) continue;
+    if (!__any_sync(kFull, mx[i] >= Wn.thr[i])) continue;
     float M = mx[i];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
     const float smax = fmaxf(W.smax[i], M);
-    const float thr = smax - win2;
-    const float ax = 0.5f * Q.x[i].x, ay = 0.5f * Q.y[i].x, az = 0.5f * Q.z[i].x;
+    const float thr = smax - W.win2[i];
+    Wn.thr[i] = thr;
+    const float ax = 0.5f * Q.x[i], ay = 0.5f * Q.y[i], az = 0.5f * Q.z[i];
     unsigned long long best = W.key[i];
     unsigned cand = __ballot_sync(kFull, mx[i] >= thr);
     while (cand) {
       const int L = __ffs(cand) - 1;
       cand &= cand - 1;
-      unsigned long long key = ~0ull;
+      // (distance bits, index) of this lane's row, or (~0, ~0) outside the
+      // window; the warp minimum in two 32-bit reductions (distance, then
+      // index among the lanes at that distance). Non-negative floats order
+      // like their bits.
+      uint32_t dbits = 0xFFFFFFFFu, jidx = 0xFFFFFFFFu;
       const int j = jt + L;
       if (j < rows) {
         const float4 p = buf[j];
-        const float sc =
-            __fmaf_rn(Q.z[i].x, p.z, __fmaf_rn(Q.y[i].x, p.y, __fmaf_rn(Q.x[i].x, p.x, p.w)));
-        if (sc >= thr) {
-          const float d2 = __double2float_rn(dist2_f64(ax, ay, az, p));
-          key = (static_cast<unsigned long long>(__float_as_uint(d2)) << 32) |
-                static_cast<unsigned long long>(base + static_cast<uint32_t>(j));
+        if (l2_score(Q, i, p) >= thr) {
+          dbits = __float_as_uint(__double2float_rn(dist2_f64(ax, ay, az, p)));
+          jidx = base + static_cast<uint32_t>(j);
         }
       }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const unsigned long long other = __shfl_xor_sync(kFull, key, o);
-        key = other < key ? other : key;
-      }
-      best = key < best ? key : best;
+      const uint32_t dmin = __reduce_min_sync(kFull, dbits);
+      const uint32_t jmin = __reduce_min_sync(kFull, dbits == dmin ? jidx : 0xFFFFFFFFu);
+      const unsigned long long k = (static_cast<unsigned long long>(dmin) << 32) | jmin;
+      best = k < best ? k : best;
     }
     __syncwarp();
     if (lane == 0) {
-      W.smax[i] = smax;
       W.key[i] = best;
+      W.smax[i] = smax;
     }
     __syncwarp();
   }
@@ -304,70 +365,74 @@ __device__ __forceinline__ void l2_chunk(const float4* __restrict__ buf, int row
 __device__ void l2_phase(const NNArgs& a, const PhaseQ q, L2Smem& s) {
   if (threadIdx.x == 0) l2_plan(a, q, s);
   __syncthreads();
-  const int64_t u0 = s.u0, u1 = s.u1, nt = s.nt;
+  const int64_t u0 = s.u0, u1 = s.u1;
   if (u0 >= u1 || *reinterpret_cast<volatile int*>(&s.abort_flag)) {
     __syncthreads();
     return;
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint32_t ph[2] = {s.bar_phase[0], s.bar_phase[1]};
-  int b = s.b0;
-  int64_t m = s.m0, n = s.n0;
-  if (threadIdx.x == 0) l2_issue(a, s, 0, b, n);
-  Queries Q;
+  uint32_t ph[kNS];
+#pragma unroll
+  for (int i = 0; i < kNS; ++i) ph[i] = s.bar_phase[i];
+  Walk w{s.b0, s.m0, s.n0, (s.n0 * s.perm) % s.nt};
+  Walk ahead = w;  // the unit kNS ahead: the one a released buffer receives
+  for (int k = 0; k < kNS; ++k) walk_next(ahead, s, a.batch);
   WarpState& W = s.ws[warp];
   const float max_p2 = a.db_absmax ? __int_as_float(__ldcg(a.db_absmax)) : INFINITY;
+  Queries Q;
+  Window Wn;
   bool seg_start = true, ok = true;
+  int i = 0;
   for (int64_t u = u0; u < u1; ++u) {
-    const int i = static_cast<int>((u - u0) & 1);
-    // Position of the next unit.
-    int nb = b;
-    int64_t nm = m, nn = n + 1;
-    if (nn == nt) {
-      nn = 0;
-      if (++nm == s.mt[nb]) {
-        nm = 0;
-        do {
-          ++nb;
-        } while (nb < a.batch && s.mt[nb] == 0);
-      }
-    }
-    if (threadIdx.x == 0 && u + 1 < u1) l2_issue(a, s, i ^ 1, nb, nn);
-    const int64_t k0 = m * kQT + warp * kQW;
-    const bool active = k0 < s.cnt[b];  // warp-uniform
-    if (seg_start) load_queries(a, q, b, k0, s.cnt[b], lane, max_p2, W, Q);
-    ok = l2_wait(s, i, ph[i], a.status) && ok;
+    const int64_t k0 = w.m * kQT + warp * kQW;
+    const int cnt = s.cnt[w.b];
+    const bool active = k0 < cnt;  // warp-uniform
+    if (seg_start) load_queries(a, q, w.b, k0, cnt, lane, max_p2, W, Q, Wn);
+    ok = __all_sync(kFull, l2_wait(s, i, ph[i], a.status));
     ph[i] ^= 1u;
-    if (threadIdx.x == 0 && ok) s.pending[i] = 0;
-    const int rows = static_cast<int>(min(static_cast<int64_t>(kDC), a.ndb - n * kDC));
-    if (active && ok) l2_chunk(s.buf[i], rows, static_cast<uint32_t>(n * kDC), Q, W, lane);
-    const bool seg_end = (nn == 0) || (u + 1 == u1);
-    if (seg_end && active && ok && lane < kQW && k0 + lane < s.cnt[b]) {
-      const unsigned long long w = W.key[lane];
-      if (w != ~0ull) {
-        const float d2 = __uint_as_float(static_cast<uint32_t>(w >> 32));
-        atomicMax(reinterpret_cast<unsigned long long*>(&a.out_key[b * a.q_cap + k0 + lane]),
+    if (ok && active) {
+      const int rows = static_cast<int>(min(static_cast<int64_t>(kDC), a.ndb - w.c * kDC));
+      l2_chunk(s.buf[i], rows, static_cast<uint32_t>(w.c * kDC), Q, Wn, W, lane);
+    }
+    Walk nx = w;
+    walk_next(nx, s, a.batch);
+    const bool seg_end = (nx.n == 0) || (u + 1 == u1);
+    if (seg_end && active && ok && lane < kQW && k0 + lane < cnt) {
+      const unsigned long long kw = W.key[lane];
+      if (kw != ~0ull) {
+        const float d2 = __uint_as_float(static_cast<uint32_t>(kw >> 32));
+        atomicMax(reinterpret_cast<unsigned long long*>(&a.out_key[w.b * a.q_cap + k0 + lane]),
                   static_cast<unsigned long long>(
-                      make_key(ord_f32(-d2), static_cast<uint32_t>(w & 0xFFFFFFFFu))));
+                      make_key(ord_f32(-d2), static_cast<uint32_t>(kw & 0xFFFFFFFFu))));
       }
     }
+    if (!ok) {
+      *reinterpret_cast<volatile int*>(&s.abort_flag) = 1;
+      break;
+    }
+    // Count this warp out of buffer i; the last one refills it.
+    __syncwarp();
+    if (lane == 0 && atomicAdd(&s.empty_cnt[i], 1) == kWarps - 1) {
+      atomicExch(&s.empty_cnt[i], 0);
+      if (u + kNS < u1 && !*reinterpret_cast<volatile int*>(&s.abort_flag))
+        l2_issue(a, s, i, ahead);
+    }
+    __syncwarp();
+    walk_next(ahead, s, a.batch);
     seg_start = seg_end;
-    b = nb;
-    m = nm;
-    n = nn;
-    // Buffer i is free for the copy issued at the top of the next iteration.
-    if (!__syncthreads_and(ok)) break;
+    w = nx;
+    i = i + 1 == kNS ? 0 : i + 1;
   }
+  __syncthreads();
   if (threadIdx.x == 0) {
-    s.bar_phase[0] = ph[0];
-    s.bar_phase[1] = ph[1];
-    if (!ok) s.abort_flag = 1;
+#pragma unroll
+    for (int k = 0; k < kNS; ++k) s.bar_phase[k] = ph[k];
   }
   __syncthreads();
 }
 
 __global__ void __launch_bounds__(kThreads, 1) nn_l2_kernel(const __grid_constant__ NNArgs a) {
-  __shared__ L2Smem s;
+  L2Smem& s = l2_smem();
   l2_setup(s);
   l2_phase(a, PhaseQ{a.q_index, a.q_count}, s);
   l2_teardown(s, a.status);
@@ -377,7 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1) nn_l2_kernel(const __grid_constan
 // passes above.
 __global__ void __launch_bounds__(kThreads, 1)
     reciprocal_l2_kernel(const __grid_constant__ RecArgs r) {
-  __shared__ L2Smem s;
+  L2Smem& s = l2_smem();
   l2_setup(s);
   auto pass = [&](int dir, const PhaseQ& q) { l2_phase(dir == 0 ? r.fwd : r.bwd, q, s); };
   fast_rounds<FASTNN_F32_L2>(r, pass, &s.abort_flag, &s.grid_ok, &s.more, s.scan);
@@ -392,9 +457,11 @@ int launch_nn_l2(const NNArgs& a, cudaStream_t stream) {
   if (a.batch < 1 || a.batch > kMaxBatchL2 || a.ndb < 1) return FASTNN_ERR_INVALID;
   int sms = 0, rc = device_sm_count(&sms);
   if (rc != FASTNN_OK) return rc;
+  FASTNN_CUDA_TRY(cudaFuncSetAttribute(nn_l2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kSmemBytes)));
   const int slot = kernel_timer_begin(stream);
   if (slot == -2) return FASTNN_ERR_CUDA;
-  nn_l2_kernel<<<sms, kThreads, 0, stream>>>(a);
+  nn_l2_kernel<<<sms, kThreads, kSmemBytes, stream>>>(a);
   FASTNN_CUDA_TRY(cudaGetLastError());
   return kernel_timer_end(slot, stream);
 }
@@ -405,14 +472,18 @@ int launch_reciprocal_l2(const RecArgs& r, cudaStream_t stream) {
   int sms = 0, rc = device_sm_count(&sms);
   if (rc != FASTNN_OK) return rc;
   const void* fn = reinterpret_cast<const void*>(reciprocal_l2_kernel);
+  FASTNN_CUDA_TRY(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kSmemBytes)));
   int per_sm = 0;
-  FASTNN_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, 0));
+  FASTNN_CUDA_TRY(
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, kSmemBytes));
   if (per_sm < 1) return FASTNN_ERR_UNSUPPORTED;
   RecArgs args = r;
   void* params[] = {&args};
   const int slot = kernel_timer_begin(stream);
   if (slot == -2) return FASTNN_ERR_CUDA;
-  FASTNN_CUDA_TRY(cudaLaunchCooperativeKernel(fn, dim3(sms), dim3(kThreads), params, 0, stream));
+  FASTNN_CUDA_TRY(
+      cudaLaunchCooperativeKernel(fn, dim3(sms), dim3(kThreads), params, kSmemBytes, stream));
   return kernel_timer_end(slot, stream);
 }
 
