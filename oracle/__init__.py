@@ -26,6 +26,16 @@ What the oracle computes, step by step, in the pages' order:
   to image 1; pixels that return to themselves are kept; the others continue
   from where they landed, for at most ``max_iter`` rounds.
 
+* ``confident`` / ``nn_masked`` / ``dense_mutual_masked`` /
+  ``fast_reciprocal_masked`` -- the same matching restricted to confident
+  pixels: the network predicts a per-pixel confidence alongside its outputs
+  ("DUSt3R / MASt3R explained", the pointmap paragraph), and the remedy for
+  pixels whose geometry is not trustworthy is to mask them or reject their
+  low-confidence matches ("MASt3R dissection", section 5, hidden
+  assumptions). A pixel takes part iff its confidence is at least the
+  threshold: it is then a candidate in its image's database and, if on the
+  grid, a seed; other pixels are neither.
+
 Readings taken where the pages are silent (each listed in the design notes):
 dot-product similarity for unnormalised integer descriptors; lowest index on
 ties; grid origin (0, 0) with step ``subsample`` in x and y; convergence means
@@ -256,3 +266,83 @@ def fast_reciprocal(D1: np.ndarray, H1: int, W1: int, D2: np.ndarray, H2: int, W
     pairs = np.array([[u, kept[u][0]] for u in us], dtype=np.int64).reshape(-1, 2)
     sc = np.array([kept[u][1] for u in us], dtype=np.int64 if dtype == "i8" else np.float64)
     return FastResult(pairs, sc, sizes, first, kept_gap if track_gaps else {})
+
+
+# ---------------------------------------------------------------------------
+# confidence masks
+# ---------------------------------------------------------------------------
+
+def confident(conf: np.ndarray | None, n: int, threshold: float) -> np.ndarray:
+    """Boolean [n]: pixel takes part iff conf >= threshold (all, without a map)."""
+    if conf is None:
+        return np.ones(n, dtype=bool)
+    return np.asarray(conf, dtype=np.float32).reshape(-1) >= np.float32(threshold)
+
+
+def nn_masked(q: np.ndarray, db: np.ndarray, keep_db: np.ndarray, dtype: str,
+              nthreads: int | None = None) -> NNResult:
+    """NN of every query among the database rows with keep_db set: the lowest
+    kept index with the best score. The scan runs over the kept rows in
+    increasing index order, so it is the plain scan of the definition with the
+    excluded rows skipped. idx = -1 when no row is kept."""
+    sub = np.nonzero(keep_db)[0]
+    if sub.size == 0:
+        nq = q.shape[0]
+        z = np.zeros(nq, dtype=np.int64 if dtype == "i8" else np.float64)
+        return NNResult(np.full(nq, -1, dtype=np.int64), z, z.copy())
+    r = nn(q, db[sub], dtype, nthreads)
+    return NNResult(sub[r.idx], r.score, r.second)
+
+
+def dense_mutual_masked(D1: np.ndarray, keep1: np.ndarray, D2: np.ndarray, keep2: np.ndarray,
+                        dtype: str, nthreads: int | None = None) -> DenseResult:
+    """Mutual nearest-neighbour pairs among the kept pixels of both maps
+    (pixel indices of the full maps, ascending i)."""
+    i_all = np.nonzero(keep1)[0]
+    r12 = nn_masked(D1[i_all], D2, keep2, dtype, nthreads)
+    if i_all.size == 0 or r12.idx[0] < 0:
+        return DenseResult(np.zeros((0, 2), dtype=np.int64), r12.score[:0], r12, None)
+    j_all = np.nonzero(keep2)[0]
+    r21 = nn_masked(D2[j_all], D1, keep1, dtype, nthreads)
+    back = dict(zip(j_all.tolist(), r21.idx.tolist()))
+    keep = np.array([back[int(j)] == int(i) for i, j in zip(i_all, r12.idx)], dtype=bool)
+    pairs = np.stack([i_all[keep], r12.idx[keep].astype(np.int64)], axis=1)
+    return DenseResult(pairs, r12.score[keep], r12, r21)
+
+
+def fast_reciprocal_masked(D1: np.ndarray, H1: int, W1: int, keep1: np.ndarray,
+                           D2: np.ndarray, H2: int, W2: int, keep2: np.ndarray,
+                           dtype: str, subsample: int, max_iter: int,
+                           nthreads: int | None = None) -> FastResult:
+    """The fast scheme among confident pixels: the seeds are the kept grid
+    pixels (grid order); every nearest-neighbour step searches the kept
+    pixels of the other image only; everything else is ``fast_reciprocal``.
+    A walk whose step finds no kept pixel ends."""
+    D1 = D1.reshape(H1 * W1, -1)
+    D2 = D2.reshape(H2 * W2, -1)
+    F = [int(u) for u in grid_seeds(H1, W1, subsample) if keep1[u]]
+    kept = {}
+    sizes, first = [], []
+    seen: set = set()
+    for _ in range(max_iter):
+        if not F:
+            break
+        sizes.append(len(F))
+        first.append(sum(1 for u in F if u not in seen))
+        seen.update(F)
+        fwd = nn_masked(D1[np.array(F)], D2, keep2, dtype, nthreads)
+        if fwd.idx[0] < 0:
+            break
+        bwd = nn_masked(D2[fwd.idx], D1, keep1, dtype, nthreads)
+        nxt = set()
+        for k, u in enumerate(F):
+            v, u2 = int(fwd.idx[k]), int(bwd.idx[k])
+            if u2 == u:
+                kept[u] = (v, fwd.score[k])
+            else:
+                nxt.add(u2)
+        F = sorted(nxt)
+    us = sorted(kept)
+    pairs = np.array([[u, kept[u][0]] for u in us], dtype=np.int64).reshape(-1, 2)
+    sc = np.array([kept[u][1] for u in us], dtype=np.int64 if dtype == "i8" else np.float64)
+    return FastResult(pairs, sc, sizes, first, {})

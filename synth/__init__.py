@@ -41,6 +41,7 @@ __all__ = [
     "warped_pair_int8",
     "warped_pair_bf16",
     "pointmap_pair",
+    "confidence_maps",
     "planted_sign_pair",
     "random_int8_pair",
     "f64_to_bf16_bits",
@@ -295,6 +296,35 @@ def pointmap_pair(seed: int, H: int = 384, W: int = 512, noise: float = 0.002,
                     p2.astype(np.float32).reshape(H, W, 3), gt, "l2")
 
 
+def confidence_maps(seed: int, H: int, W: int, gt_src: np.ndarray | None = None,
+                    sky_frac: float = 0.12) -> tuple[np.ndarray, np.ndarray]:
+    """Per-pixel confidences for the two views of a pair, float32 [H, W], >= 1.
+
+    Shaped like the confidences DUSt3R predicts beside its pointmaps (1 plus
+    an exponential): conf = 1 + exp(0.8 + 0.6 f) with f a seeded smooth
+    field (four low-frequency sinusoids), a low-confidence band over the top
+    sky_frac of the rows (conf in [1, 1.3]), and, in view 2, confidence in
+    [1, 1.5] on 80% of the generator's outlier pixels (gt_src == -1).
+    """
+    rng = np.random.Generator(np.random.PCG64(seed))
+    ys, xs = np.meshgrid(np.arange(H, dtype=np.float64), np.arange(W, dtype=np.float64),
+                         indexing="ij")
+    out = []
+    for view in range(2):
+        f = np.zeros((H, W))
+        for _ in range(4):
+            kx, ky = rng.uniform(0.5, 4.0, size=2)
+            f += np.sin(2 * np.pi * (kx * xs / W + ky * ys / H) + rng.uniform(0, 2 * np.pi))
+        conf = 1.0 + np.exp(0.8 + 0.6 * f / 2.0)
+        sky = ys < sky_frac * H
+        conf[sky] = rng.uniform(1.0, 1.3, size=int(sky.sum()))
+        if view == 1 and gt_src is not None:
+            o = (gt_src.reshape(H, W) < 0) & (rng.uniform(size=(H, W)) < 0.8)
+            conf[o] = rng.uniform(1.0, 1.5, size=int(o.sum()))
+        out.append(conf.astype(np.float32))
+    return out[0], out[1]
+
+
 def planted_sign_pair(seed: int, H: int, W: int, d: int, c: int = 8,
                       redraw_frac: float = 0.2) -> PairMaps:
     """Sign-vector maps with a planted permutation.
@@ -377,6 +407,12 @@ CONFIGS = {
         seed=BASE_SEED + 7,
         note="dense mutual nearest 3D points over all 196,608 pixels of the 512x384 "
              "pointmap pair above (same seed, same maps)"),
+    "pair_512x384_d24_i8_conf": dict(
+        seed=BASE_SEED + 2,
+        note="the int8 512x384 pair (same seed, same maps) with per-pixel "
+             "confidences (confidence_maps, seed + 50): a pixel takes part iff its "
+             "confidence >= 2.0 (about 80% of view 1 and 60% of view 2 do); "
+             "8-px grid, max_iter=10"),
     "batch16_512x288_d32_i8": dict(
         seed=BASE_SEED + 5,
         note="16 independent 512x288 pairs, d=32, int8 uniform in [-16,16], warped "
@@ -415,6 +451,11 @@ def make_workload(name: str, batch: int | None = None) -> Workload:
     if name == "dense_512x384_pts3_f32":
         return Workload(name, [pointmap_pair(seed)], subsample=8, max_iter=10, dense=True,
                         note=cfg["note"])
+    if name == "pair_512x384_d24_i8_conf":
+        p = warped_pair_int8(seed)
+        c1, c2 = confidence_maps(seed + 50, p.H1, p.W1, p.gt_src)
+        return Workload(name, [p], subsample=8, max_iter=10, note=cfg["note"],
+                        extra={"conf1": [c1], "conf2": [c2], "threshold": 2.0})
     if name == "batch16_512x288_d32_i8":
         nb = 16 if batch is None else batch
         pairs = [warped_pair_int8(seed + 1000 * b, H=288, W=512, d=32)
