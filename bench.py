@@ -111,6 +111,10 @@ def config_dict(w, extra=None):
                   "subsample": w.subsample, "max_iter": w.max_iter,
                   "seeds_per_pair": (p.H1 + w.subsample - 1) // w.subsample
                   * ((p.W1 + w.subsample - 1) // w.subsample)})
+    if "conf1" in w.extra:
+        c.update({"method": "confidence-masked fast reciprocal matching "
+                            "(fastnn_reciprocal_masked)",
+                  "conf_threshold": w.extra["threshold"]})
     if extra:
         c.update(extra)
     return c
@@ -150,6 +154,18 @@ def oracle_sample(w, n_seeds, dense_rows=None):
         dt = time.perf_counter() - t0
         return found, dt, threads, (f"mutual pairs among the first {dense_rows} image-1 pixels "
                                     f"(nearest neighbours over all {D2.shape[0]} pixels each way)")
+    if "conf1" in w.extra:
+        thr = w.extra["threshold"]
+        k1 = oracle.confident(w.extra["conf1"][0], p.H1 * p.W1, thr)
+        k2 = oracle.confident(w.extra["conf2"][0], p.H2 * p.W2, thr)
+        t0 = time.perf_counter()
+        r = oracle.fast_reciprocal_masked(p.desc1, p.H1, p.W1, k1, p.desc2, p.H2, p.W2, k2,
+                                          p.dtype, w.subsample, w.max_iter, nthreads=threads,
+                                          max_seeds=n_seeds)
+        dt = time.perf_counter() - t0
+        return len(r.pairs), dt, threads, (f"confidence-masked fast reciprocal matching of pair 0 "
+                                           f"from its first {n_seeds} kept grid seeds, "
+                                           f"max_iter {w.max_iter}")
     seeds = oracle.grid_seeds(p.H1, p.W1, w.subsample)[:n_seeds]
     t0 = time.perf_counter()
     r = oracle.fast_reciprocal(p.desc1, p.H1, p.W1, p.desc2, p.H2, p.W2, p.dtype, w.subsample,
@@ -314,6 +330,7 @@ def run_ours(args, rank, world, local):
             "l2": fnn.FASTNN_F32_L2}[p0.dtype]
     sdt = torch.int32 if i8 else torch.float32
     l2 = p0.dtype == "l2"
+    masked = "conf1" in w.extra
     esize = 1 if i8 else 4 if l2 else 2
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -337,13 +354,19 @@ def run_ours(args, rank, world, local):
         out_count = torch.empty(B, dtype=torch.int32, device=dev)
         out_iters = torch.empty(B, dtype=torch.int32, device=dev)
         out_front = torch.empty((B, w.max_iter), dtype=torch.int32, device=dev)
-        nbytes = fnn.fastnn_workspace_size(fnn.FASTNN_OP_RECIPROCAL, N1, N2, d, code, B, S)
+        op = fnn.FASTNN_OP_RECIPROCAL_MASKED if masked else fnn.FASTNN_OP_RECIPROCAL
+        nbytes = fnn.fastnn_workspace_size(op, N1, N2, d, code, B, S)
         hp_pairs = torch.empty((B, S, 2), dtype=torch.int32).pin_memory()
         hp_score = torch.empty((B, S), dtype=sdt).pin_memory()
     hp_count = torch.empty(out_count.shape, dtype=torch.int32).pin_memory()
     d1 = h1.to(dev)
     d2 = h2.to(dev)
     ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    hc1 = hc2 = c1 = c2 = None
+    if masked:
+        hc1 = torch.from_numpy(np.ascontiguousarray(np.stack(w.extra["conf1"]))).pin_memory()
+        hc2 = torch.from_numpy(np.ascontiguousarray(np.stack(w.extra["conf2"]))).pin_memory()
+        c1, c2 = hc1.to(dev), hc2.to(dev)
 
     if w.dense:
         def call():
@@ -351,6 +374,16 @@ def run_ours(args, rank, world, local):
                                     out_count=out_count, workspace=ws, stream=stream)
         launches_per_step = 2 + 2 + 3  # 2 repack, 2 tensor-core passes, count/scan/emit
         kernels_per_step = 2
+    elif masked:
+        def call():
+            fnn.fastnn_reciprocal_masked(d1, d2, w.subsample, w.max_iter, conf1=c1, conf2=c2,
+                                         threshold=w.extra["threshold"], out_pairs=out_pairs,
+                                         out_score=out_score, out_count=out_count,
+                                         out_iters=out_iters, out_frontier=out_front,
+                                         workspace=ws, stream=stream)
+        # 2 x (count, scan, emit) mask compaction, seeds, 1 persistent matching kernel
+        launches_per_step = 8
+        kernels_per_step = 1
     else:
         def call():
             fnn.fastnn_reciprocal(d1, d2, w.subsample, w.max_iter, out_pairs=out_pairs,
@@ -413,6 +446,9 @@ def run_ours(args, rank, world, local):
         evs2[i][0].record(stream)
         d1.copy_(h1, non_blocking=True)
         d2.copy_(h2, non_blocking=True)
+        if masked:
+            c1.copy_(hc1, non_blocking=True)
+            c2.copy_(hc2, non_blocking=True)
         call()
         hp_count.copy_(out_count, non_blocking=True)
         hp_pairs.copy_(out_pairs, non_blocking=True)
@@ -445,7 +481,7 @@ def run_ours(args, rank, world, local):
         else:
             peak = 2.0 * bf16_peak if i8 else bf16_peak  # dense int8 = 2 x bf16 (nominal ratio)
             achieved = 2.0 * macs_per_step * K / (nn_ms / 1e3) / 1e12 if nn_ms > 0 else None
-        bytes_in = (N1 + N2) * d * esize * B
+        bytes_in = (N1 + N2) * d * esize * B + ((N1 + N2) * 4 * B if masked else 0)
         bytes_out = int(hp_count.numel() * 4 + hp_pairs.numel() * 4 + hp_score.numel() * 4)
         if l2:
             kname = ("nn_l2_kernel (FP32 FFMA2 nearest point, one launch per direction)"

@@ -77,7 +77,9 @@ typedef enum {
     FASTNN_OP_NN = 0,
     FASTNN_OP_RECIPROCAL = 1,
     FASTNN_OP_MUTUAL_DENSE = 2,
-    FASTNN_OP_MUTUAL_FROM_NN = 3
+    FASTNN_OP_MUTUAL_FROM_NN = 3,
+    FASTNN_OP_RECIPROCAL_MASKED = 4,
+    FASTNN_OP_MUTUAL_DENSE_MASKED = 5
 } fastnn_op;
 
 /*
@@ -87,7 +89,9 @@ typedef enum {
  *                           grid seeds per pair, batch = pairs
  *   FASTNN_OP_MUTUAL_DENSE: n1, n2 = pixel counts (batch, max_queries unused)
  *   FASTNN_OP_MUTUAL_FROM_NN: n1 = local image-1 rows, n2 = image-2 rows
- *                           (d must still be 1..32; unused)
+ *                           (d must still be valid for dtype; unused)
+ *   FASTNN_OP_RECIPROCAL_MASKED, FASTNN_OP_MUTUAL_DENSE_MASKED: as the
+ *                           unmasked ops
  * Returns 0 for arguments no call would accept.
  */
 size_t fastnn_workspace_size(int op, int64_t n1, int64_t n2, int d, int dtype,
@@ -171,6 +175,42 @@ int fastnn_mutual_from_nn(const int32_t *nn12, const void *score12, int64_t n1,
                           void *out_score, int64_t capacity, int32_t *out_count,
                           void *workspace, size_t workspace_bytes,
                           fastnn_stream_t stream);
+
+/*
+ * Confidence-masked matching. The network predicts a confidence beside every
+ * per-pixel output ("DUSt3R / MASt3R explained", the pointmap paragraph), and
+ * the remedy for pixels whose geometry cannot be trusted is to mask them or
+ * reject their low-confidence matches ("MASt3R dissection", section 5).
+ * Here a pixel takes part iff conf >= conf_threshold: it is a candidate in
+ * its image's database and, if on the seed grid, a seed; other pixels are
+ * neither. Without a confidence map (NULL) every pixel of that image takes
+ * part. Reported indices are pixel indices of the full maps; everything else
+ * (tie rule, order of the output, scores, capacities, errors) is that of the
+ * unmasked call. The kept pixels are compacted on the device, in pixel order,
+ * before matching; confidences must not be NaN for pixels meant to be kept.
+ *   conf1: [batch][H1][W1] float32 or NULL; conf2: [batch][H2][W2] or NULL.
+ *   Workspace: FASTNN_OP_RECIPROCAL_MASKED (or _MUTUAL_DENSE_MASKED) sizes.
+ *   capacity >= S (fast) / min(n1, n2) (dense) as for the unmasked calls;
+ *   out_frontier counts kept seeds in round 1. A pair whose image 2 keeps no
+ *   pixel runs one round and keeps nothing.
+ */
+int fastnn_reciprocal_masked(const void *desc1, const float *conf1, int H1,
+                             int W1, const void *desc2, const float *conf2,
+                             int H2, int W2, int d, int dtype,
+                             float conf_threshold, int subsample, int max_iter,
+                             int batch, int32_t *out_pairs, void *out_score,
+                             int64_t capacity, int32_t *out_count,
+                             int32_t *out_iters, int32_t *out_frontier,
+                             void *workspace, size_t workspace_bytes,
+                             fastnn_stream_t stream);
+
+int fastnn_mutual_dense_masked(const void *desc1, const float *conf1, int64_t n1,
+                               const void *desc2, const float *conf2,
+                               int64_t n2, int d, int dtype,
+                               float conf_threshold, int32_t *out_pairs,
+                               void *out_score, int64_t capacity,
+                               int32_t *out_count, void *workspace,
+                               size_t workspace_bytes, fastnn_stream_t stream);
 
 /*
  * fastnn_reciprocal_noalloc -- fastnn_reciprocal for callers that cannot

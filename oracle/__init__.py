@@ -313,14 +313,16 @@ def dense_mutual_masked(D1: np.ndarray, keep1: np.ndarray, D2: np.ndarray, keep2
 def fast_reciprocal_masked(D1: np.ndarray, H1: int, W1: int, keep1: np.ndarray,
                            D2: np.ndarray, H2: int, W2: int, keep2: np.ndarray,
                            dtype: str, subsample: int, max_iter: int,
-                           nthreads: int | None = None) -> FastResult:
+                           nthreads: int | None = None,
+                           max_seeds: int | None = None) -> FastResult:
     """The fast scheme among confident pixels: the seeds are the kept grid
     pixels (grid order); every nearest-neighbour step searches the kept
     pixels of the other image only; everything else is ``fast_reciprocal``.
-    A walk whose step finds no kept pixel ends."""
+    A walk whose step finds no kept pixel ends. ``max_seeds`` keeps only the
+    first kept seeds (a bounded sample for timing)."""
     D1 = D1.reshape(H1 * W1, -1)
     D2 = D2.reshape(H2 * W2, -1)
-    F = [int(u) for u in grid_seeds(H1, W1, subsample) if keep1[u]]
+    F = [int(u) for u in grid_seeds(H1, W1, subsample) if keep1[u]][:max_seeds]
     kept = {}
     sizes, first = [], []
     seen: set = set()

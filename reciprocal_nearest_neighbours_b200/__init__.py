@@ -16,17 +16,21 @@ from ._lib import (  # noqa: F401
     FASTNN_F32_L2,
     FASTNN_I8,
     FASTNN_OP_MUTUAL_DENSE,
+    FASTNN_OP_MUTUAL_DENSE_MASKED,
     FASTNN_OP_MUTUAL_FROM_NN,
     FASTNN_OP_NN,
     FASTNN_OP_RECIPROCAL,
+    FASTNN_OP_RECIPROCAL_MASKED,
     FastNNError,
     fastnn_device_status,
     fastnn_kernel_timer_enable,
     fastnn_kernel_timer_read,
     fastnn_mutual_dense,
+    fastnn_mutual_dense_masked,
     fastnn_mutual_from_nn,
     fastnn_nn,
     fastnn_reciprocal,
+    fastnn_reciprocal_masked,
     fastnn_reciprocal_noalloc,
     fastnn_status_str,
     fastnn_workspace_size,

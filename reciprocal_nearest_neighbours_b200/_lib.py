@@ -18,6 +18,8 @@ FASTNN_OP_NN = 0
 FASTNN_OP_RECIPROCAL = 1
 FASTNN_OP_MUTUAL_DENSE = 2
 FASTNN_OP_MUTUAL_FROM_NN = 3
+FASTNN_OP_RECIPROCAL_MASKED = 4
+FASTNN_OP_MUTUAL_DENSE_MASKED = 5
 
 _lib = None
 
@@ -56,6 +58,13 @@ def library():
     lib.fastnn_reciprocal_noalloc.restype = I
     lib.fastnn_mutual_dense.argtypes = [P, I64, P, I64, I, I, P, P, I64, P, P, SZ, P]
     lib.fastnn_mutual_dense.restype = I
+    F = ctypes.c_float
+    lib.fastnn_reciprocal_masked.argtypes = [P, P, I, I, P, P, I, I, I, I, F, I, I, I, P, P, I64,
+                                             P, P, P, P, SZ, P]
+    lib.fastnn_reciprocal_masked.restype = I
+    lib.fastnn_mutual_dense_masked.argtypes = [P, P, I64, P, P, I64, I, I, F, P, P, I64, P, P, SZ,
+                                               P]
+    lib.fastnn_mutual_dense_masked.restype = I
     lib.fastnn_mutual_from_nn.argtypes = [P, P, I64, I64, P, I64, I64, I, P, P, I64, P, P, SZ, P]
     lib.fastnn_mutual_from_nn.restype = I
     lib.fastnn_device_status.argtypes = [P, P]
@@ -303,3 +312,88 @@ def fastnn_kernel_timer_read():
     _check(library().fastnn_kernel_timer_read(ctypes.byref(n), ctypes.byref(ms)),
            "fastnn_kernel_timer_read")
     return int(n.value), float(ms.value)
+
+
+def _conf(conf, n_expected, dev):
+    if conf is None:
+        return None
+    if not (conf.is_cuda and conf.is_contiguous() and conf.dtype == torch.float32):
+        raise ValueError("confidence maps must be contiguous float32 CUDA tensors")
+    if conf.numel() != n_expected:
+        raise ValueError("confidence map size does not match the descriptor map")
+    return conf
+
+
+def fastnn_reciprocal_masked(desc1: torch.Tensor, desc2: torch.Tensor, subsample: int,
+                             max_iter: int, conf1: torch.Tensor | None = None,
+                             conf2: torch.Tensor | None = None, threshold: float = 0.0,
+                             capacity: int | None = None, out_pairs=None, out_score=None,
+                             out_count=None, out_iters=None, out_frontier=None, workspace=None,
+                             stream=None):
+    """Fast reciprocal matching among confident pixels (conf >= threshold).
+
+    ``conf1`` [B,H1,W1] / ``conf2`` [B,H2,W2] float32, or None (every pixel of
+    that image takes part). Everything else as ``fastnn_reciprocal``; the
+    pairs are pixel indices of the full maps.
+    """
+    _need_cuda(desc1, desc2)
+    code = _dtype_code(desc1)
+    assert desc2.dtype == desc1.dtype
+    if desc1.dim() == 3:
+        desc1, desc2 = desc1.unsqueeze(0), desc2.unsqueeze(0)
+    B, H1, W1, d = desc1.shape
+    B2, H2, W2, d2 = desc2.shape
+    assert B2 == B and d2 == d
+    conf1 = _conf(conf1, B * H1 * W1, desc1.device)
+    conf2 = _conf(conf2, B * H2 * W2, desc1.device)
+    S = seed_count(H1, W1, subsample)
+    cap = S if capacity is None else int(capacity)
+    dev = desc1.device
+    if out_pairs is None:
+        out_pairs = torch.empty((B, cap, 2), dtype=torch.int32, device=dev)
+    if out_score is None:
+        out_score = torch.empty((B, cap), dtype=_score_dtype(code), device=dev)
+    if out_count is None:
+        out_count = torch.empty(B, dtype=torch.int32, device=dev)
+    if out_iters is None:
+        out_iters = torch.empty(B, dtype=torch.int32, device=dev)
+    nbytes = fastnn_workspace_size(FASTNN_OP_RECIPROCAL_MASKED, H1 * W1, H2 * W2, d, code, B, S)
+    ws = _workspace(nbytes, dev, workspace)
+    rc = library().fastnn_reciprocal_masked(
+        _ptr(desc1), _ptr(conf1), H1, W1, _ptr(desc2), _ptr(conf2), H2, W2, d, code,
+        float(threshold), subsample, max_iter, B, _ptr(out_pairs), _ptr(out_score), cap,
+        _ptr(out_count), _ptr(out_iters), _ptr(out_frontier), _ptr(ws), nbytes, _stream(stream))
+    _check(rc, "fastnn_reciprocal_masked")
+    return out_pairs, out_score, out_count, out_iters
+
+
+def fastnn_mutual_dense_masked(desc1: torch.Tensor, desc2: torch.Tensor,
+                               conf1: torch.Tensor | None = None,
+                               conf2: torch.Tensor | None = None, threshold: float = 0.0,
+                               capacity: int | None = None, out_pairs=None, out_score=None,
+                               out_count=None, workspace=None, stream=None):
+    """Every mutual nearest-neighbour pair among the confident pixels of two maps."""
+    _need_cuda(desc1, desc2)
+    code = _dtype_code(desc1)
+    desc1 = desc1.reshape(-1, desc1.shape[-1])
+    desc2 = desc2.reshape(-1, desc2.shape[-1])
+    n1, d = desc1.shape
+    n2 = desc2.shape[0]
+    conf1 = _conf(conf1, n1, desc1.device)
+    conf2 = _conf(conf2, n2, desc1.device)
+    cap = min(n1, n2) if capacity is None else int(capacity)
+    dev = desc1.device
+    if out_pairs is None:
+        out_pairs = torch.empty((cap, 2), dtype=torch.int32, device=dev)
+    if out_score is None:
+        out_score = torch.empty(cap, dtype=_score_dtype(code), device=dev)
+    if out_count is None:
+        out_count = torch.empty(1, dtype=torch.int32, device=dev)
+    nbytes = fastnn_workspace_size(FASTNN_OP_MUTUAL_DENSE_MASKED, n1, n2, d, code)
+    ws = _workspace(nbytes, dev, workspace)
+    rc = library().fastnn_mutual_dense_masked(
+        _ptr(desc1), _ptr(conf1), n1, _ptr(desc2), _ptr(conf2), n2, d, code, float(threshold),
+        _ptr(out_pairs), _ptr(out_score), cap, _ptr(out_count), _ptr(ws), nbytes,
+        _stream(stream))
+    _check(rc, "fastnn_mutual_dense_masked")
+    return out_pairs, out_score, out_count

@@ -110,6 +110,29 @@ MutLayout carve_mut(Carver& c, int64_t n1, int64_t n2, int d, int dtype) {
   return L;
 }
 
+// Compaction state of the confidence-masked calls.
+struct MaskLayout {
+  int32_t* c2p1;     // [batch][N1] pixel of compacted image-1 slot
+  int32_t* p2c1;     // [batch][N1] slot of image-1 pixel (-1: dropped); fast scheme only
+  int32_t* c2p2;     // [batch][N2]
+  int32_t* cnt1;     // [batch] kept pixels of image 1
+  int32_t* cnt2;     // [batch]
+  int32_t* seedcnt;  // [batch] kept seeds
+  int32_t* blocks;   // per-block scan scratch, reused by both maps
+};
+MaskLayout carve_mask(Carver& c, int64_t N1, int64_t N2, int batch, bool seeds) {
+  MaskLayout L;
+  L.c2p1 = c.take<int32_t>(static_cast<size_t>(batch) * N1);
+  L.p2c1 = seeds ? c.take<int32_t>(static_cast<size_t>(batch) * N1) : nullptr;
+  L.c2p2 = c.take<int32_t>(static_cast<size_t>(batch) * N2);
+  L.cnt1 = c.take<int32_t>(static_cast<size_t>(batch));
+  L.cnt2 = c.take<int32_t>(static_cast<size_t>(batch));
+  L.seedcnt = c.take<int32_t>(static_cast<size_t>(batch));
+  const int bpp = mask_blocks(N1) > mask_blocks(N2) ? mask_blocks(N1) : mask_blocks(N2);
+  L.blocks = c.take<int32_t>(static_cast<size_t>(batch) * bpp);
+  return L;
+}
+
 int64_t seed_count(int H, int W, int sub) {
   return static_cast<int64_t>((H + sub - 1) / sub) * ((W + sub - 1) / sub);
 }
@@ -144,6 +167,16 @@ size_t fastnn_workspace_size(int op, int64_t n1, int64_t n2, int d, int dtype, i
       break;
     case FASTNN_OP_MUTUAL_FROM_NN:
       c.take<int32_t>(static_cast<size_t>(mutual_blocks(n1 > 0 ? n1 : 1)));
+      break;
+    case FASTNN_OP_RECIPROCAL_MASKED:
+      if (batch < 1 || max_queries < 1 || n1 < 1) return 0;
+      carve_rec(c, n1, n2, d, dtype, batch, max_queries);
+      carve_mask(c, n1, n2, batch, true);
+      break;
+    case FASTNN_OP_MUTUAL_DENSE_MASKED:
+      if (n1 < 1) return 0;
+      carve_mut(c, n1, n2, d, dtype);
+      carve_mask(c, n1, n2, 1, false);
       break;
     default:
       return 0;
@@ -188,11 +221,17 @@ int fastnn_nn(const void* q, int64_t nq, const void* db, int64_t ndb, int d, int
   return launch_decode(L.keys, nq, dtype, out_idx, out_score, st);
 }
 
-int fastnn_reciprocal(const void* desc1, int H1, int W1, const void* desc2, int H2, int W2, int d,
-                      int dtype, int subsample, int max_iter, int batch, int32_t* out_pairs,
-                      void* out_score, int64_t capacity, int32_t* out_count, int32_t* out_iters,
-                      int32_t* out_frontier, void* workspace, size_t workspace_bytes,
-                      fastnn_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// The fast scheme, unmasked or (masked == true) among confident pixels.
+int reciprocal_impl(const void* desc1, const float* conf1, int H1, int W1, const void* desc2,
+                    const float* conf2, int H2, int W2, int d, int dtype, bool masked,
+                    float threshold, int subsample, int max_iter, int batch, int32_t* out_pairs,
+                    void* out_score, int64_t capacity, int32_t* out_count, int32_t* out_iters,
+                    int32_t* out_frontier, void* workspace, size_t workspace_bytes,
+                    fastnn_stream_t stream) {
   if (!dtype_ok(dtype) || !d_ok(d, dtype)) return FASTNN_ERR_UNSUPPORTED;
   if (H1 < 1 || W1 < 1 || H2 < 1 || W2 < 1 || subsample < 1 || max_iter < 1 ||
       max_iter > kMaxIter || batch < 1 || batch > nn_tc_max_batch())
@@ -206,8 +245,8 @@ int fastnn_reciprocal(const void* desc1, int H1, int W1, const void* desc2, int 
   if (!desc1 || !desc2 || !out_pairs || !out_count || !workspace || !aligned(workspace, kAlign))
     return FASTNN_ERR_INVALID;
   if (capacity < S) return FASTNN_ERR_CAPACITY;
-  if (workspace_bytes <
-      fastnn_workspace_size(FASTNN_OP_RECIPROCAL, N1, N2, d, dtype, batch, S))
+  const int op = masked ? FASTNN_OP_RECIPROCAL_MASKED : FASTNN_OP_RECIPROCAL;
+  if (workspace_bytes < fastnn_workspace_size(op, N1, N2, d, dtype, batch, S))
     return FASTNN_ERR_CAPACITY;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   Carver c{static_cast<uint8_t*>(workspace)};
@@ -215,8 +254,21 @@ int fastnn_reciprocal(const void* desc1, int H1, int W1, const void* desc2, int 
 
   // Status block: status word, per-map max |element|, grid-barrier words.
   FASTNN_CUDA_TRY(cudaMemsetAsync(L.status, 0, kStatusBytes, st));
-  FASTNN_TRY(launch_repack(desc1, batch * N1, d, dtype, L.d1rep, kPadRows, L.status + 1, st));
-  FASTNN_TRY(launch_repack(desc2, batch * N2, d, dtype, L.d2rep, kPadRows, L.status + 2, st));
+  MaskLayout M{};
+  if (masked) {
+    // Kept pixels of each map, compacted in pixel order; kept grid seeds.
+    M = carve_mask(c, N1, N2, batch, true);
+    MaskArgs m1{static_cast<const uint8_t*>(desc1), conf1, threshold, N1, batch, d,
+                L.d1rep, M.c2p1, M.p2c1, M.cnt1, L.status + 1, M.blocks, 0};
+    FASTNN_TRY(launch_mask_compact(m1, dtype, st));
+    MaskArgs m2{static_cast<const uint8_t*>(desc2), conf2, threshold, N2, batch, d,
+                L.d2rep, M.c2p2, nullptr, M.cnt2, L.status + 2, M.blocks, 0};
+    FASTNN_TRY(launch_mask_compact(m2, dtype, st));
+    FASTNN_TRY(launch_masked_seeds(M.p2c1, batch, N1, W1, subsample, S, L.F[0], M.seedcnt, st));
+  } else {
+    FASTNN_TRY(launch_repack(desc1, batch * N1, d, dtype, L.d1rep, kPadRows, L.status + 1, st));
+    FASTNN_TRY(launch_repack(desc2, batch * N2, d, dtype, L.d2rep, kPadRows, L.status + 2, st));
+  }
 
   RecArgs r{};
   r.fwd.q_rows = L.d1rep;
@@ -239,6 +291,13 @@ int fastnn_reciprocal(const void* desc1, int H1, int W1, const void* desc2, int 
   r.bwd.out_key = L.bwd;
   r.bwd.q_absmax = L.status + 2;
   r.bwd.db_absmax = L.status + 1;
+  if (masked) {
+    r.fwd.ndb_dev = M.cnt2;
+    r.bwd.ndb_dev = M.cnt1;
+    r.seed_cnt = M.seedcnt;
+    r.cmp.map1 = M.c2p1;
+    r.cmp.map2 = M.c2p2;
+  }
   r.cmp.S_cap = S;
   r.cmp.fwd_key = L.fwd;
   r.cmp.bwd_key = L.bwd;
@@ -269,17 +328,50 @@ int fastnn_reciprocal(const void* desc1, int H1, int W1, const void* desc2, int 
   return launch_reciprocal(r, dtype, batch * N1 + kPadRows, batch * N2 + kPadRows, st);
 }
 
-int fastnn_mutual_dense(const void* desc1, int64_t n1, const void* desc2, int64_t n2, int d,
-                        int dtype, int32_t* out_pairs, void* out_score, int64_t capacity,
-                        int32_t* out_count, void* workspace, size_t workspace_bytes,
-                        fastnn_stream_t stream) {
+}  // namespace
+
+extern "C" {
+
+int fastnn_reciprocal(const void* desc1, int H1, int W1, const void* desc2, int H2, int W2, int d,
+                      int dtype, int subsample, int max_iter, int batch, int32_t* out_pairs,
+                      void* out_score, int64_t capacity, int32_t* out_count, int32_t* out_iters,
+                      int32_t* out_frontier, void* workspace, size_t workspace_bytes,
+                      fastnn_stream_t stream) {
+  return reciprocal_impl(desc1, nullptr, H1, W1, desc2, nullptr, H2, W2, d, dtype, false, 0.f,
+                         subsample, max_iter, batch, out_pairs, out_score, capacity, out_count,
+                         out_iters, out_frontier, workspace, workspace_bytes, stream);
+}
+
+int fastnn_reciprocal_masked(const void* desc1, const float* conf1, int H1, int W1,
+                             const void* desc2, const float* conf2, int H2, int W2, int d,
+                             int dtype, float conf_threshold, int subsample, int max_iter,
+                             int batch, int32_t* out_pairs, void* out_score, int64_t capacity,
+                             int32_t* out_count, int32_t* out_iters, int32_t* out_frontier,
+                             void* workspace, size_t workspace_bytes, fastnn_stream_t stream) {
+  if (conf_threshold != conf_threshold) return FASTNN_ERR_INVALID;  // NaN threshold
+  return reciprocal_impl(desc1, conf1, H1, W1, desc2, conf2, H2, W2, d, dtype, true,
+                         conf_threshold, subsample, max_iter, batch, out_pairs, out_score,
+                         capacity, out_count, out_iters, out_frontier, workspace,
+                         workspace_bytes, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+int mutual_dense_impl(const void* desc1, const float* conf1, int64_t n1, const void* desc2,
+                      const float* conf2, int64_t n2, int d, int dtype, bool masked,
+                      float threshold, int32_t* out_pairs, void* out_score, int64_t capacity,
+                      int32_t* out_count, void* workspace, size_t workspace_bytes,
+                      fastnn_stream_t stream) {
   if (!dtype_ok(dtype) || !d_ok(d, dtype)) return FASTNN_ERR_UNSUPPORTED;
   if (n1 < 1 || n2 < 1 || n1 > INT32_MAX - kPadRows || n2 > INT32_MAX - kPadRows)
     return FASTNN_ERR_INVALID;
   if (!desc1 || !desc2 || !out_pairs || !out_count || !workspace || !aligned(workspace, kAlign))
     return FASTNN_ERR_INVALID;
   if (capacity < (n1 < n2 ? n1 : n2)) return FASTNN_ERR_CAPACITY;
-  if (workspace_bytes < fastnn_workspace_size(FASTNN_OP_MUTUAL_DENSE, n1, n2, d, dtype, 1, 0))
+  const int op = masked ? FASTNN_OP_MUTUAL_DENSE_MASKED : FASTNN_OP_MUTUAL_DENSE;
+  if (workspace_bytes < fastnn_workspace_size(op, n1, n2, d, dtype, 1, 0))
     return FASTNN_ERR_CAPACITY;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   Carver c{static_cast<uint8_t*>(workspace)};
@@ -287,8 +379,19 @@ int fastnn_mutual_dense(const void* desc1, int64_t n1, const void* desc2, int64_
   FASTNN_CUDA_TRY(cudaMemsetAsync(L.status, 0, kStatusBytes, st));
   FASTNN_CUDA_TRY(cudaMemsetAsync(L.k12, 0, static_cast<size_t>(n1) * 8, st));
   FASTNN_CUDA_TRY(cudaMemsetAsync(L.k21, 0, static_cast<size_t>(n2) * 8, st));
-  FASTNN_TRY(launch_repack(desc1, n1, d, dtype, L.d1rep, kPadRows, L.status + 1, st));
-  FASTNN_TRY(launch_repack(desc2, n2, d, dtype, L.d2rep, kPadRows, L.status + 2, st));
+  MaskLayout M{};
+  if (masked) {
+    M = carve_mask(c, n1, n2, 1, false);
+    MaskArgs m1{static_cast<const uint8_t*>(desc1), conf1, threshold, n1, 1, d,
+                L.d1rep, M.c2p1, nullptr, M.cnt1, L.status + 1, M.blocks, 0};
+    FASTNN_TRY(launch_mask_compact(m1, dtype, st));
+    MaskArgs m2{static_cast<const uint8_t*>(desc2), conf2, threshold, n2, 1, d,
+                L.d2rep, M.c2p2, nullptr, M.cnt2, L.status + 2, M.blocks, 0};
+    FASTNN_TRY(launch_mask_compact(m2, dtype, st));
+  } else {
+    FASTNN_TRY(launch_repack(desc1, n1, d, dtype, L.d1rep, kPadRows, L.status + 1, st));
+    FASTNN_TRY(launch_repack(desc2, n2, d, dtype, L.d2rep, kPadRows, L.status + 2, st));
+  }
   NNArgs a{};
   a.q_rows = L.d1rep;
   a.q_rows_per_pair = n1;
@@ -302,6 +405,10 @@ int fastnn_mutual_dense(const void* desc1, int64_t n1, const void* desc2, int64_
   a.d = d;
   a.q_absmax = L.status + 1;
   a.db_absmax = L.status + 2;
+  if (masked) {
+    a.q_count = M.cnt1;
+    a.ndb_dev = M.cnt2;
+  }
   if (dtype == FASTNN_F32_L2)
     FASTNN_TRY(launch_nn_l2(a, st));
   else
@@ -319,6 +426,10 @@ int fastnn_mutual_dense(const void* desc1, int64_t n1, const void* desc2, int64_
   r.d = d;
   r.q_absmax = L.status + 2;
   r.db_absmax = L.status + 1;
+  if (masked) {
+    r.q_count = M.cnt2;
+    r.ndb_dev = M.cnt1;
+  }
   if (dtype == FASTNN_F32_L2)
     FASTNN_TRY(launch_nn_l2(r, st));
   else
@@ -329,7 +440,33 @@ int fastnn_mutual_dense(const void* desc1, int64_t n1, const void* desc2, int64_
 
   m.n1 = n1;
   m.n2 = n2;
+  m.map1 = M.c2p1;
+  m.map2 = M.c2p2;
   return launch_mutual(m, L.blocks, dtype, out_pairs, out_score, capacity, out_count, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int fastnn_mutual_dense(const void* desc1, int64_t n1, const void* desc2, int64_t n2, int d,
+                        int dtype, int32_t* out_pairs, void* out_score, int64_t capacity,
+                        int32_t* out_count, void* workspace, size_t workspace_bytes,
+                        fastnn_stream_t stream) {
+  return mutual_dense_impl(desc1, nullptr, n1, desc2, nullptr, n2, d, dtype, false, 0.f,
+                           out_pairs, out_score, capacity, out_count, workspace,
+                           workspace_bytes, stream);
+}
+
+int fastnn_mutual_dense_masked(const void* desc1, const float* conf1, int64_t n1,
+                               const void* desc2, const float* conf2, int64_t n2, int d,
+                               int dtype, float conf_threshold, int32_t* out_pairs,
+                               void* out_score, int64_t capacity, int32_t* out_count,
+                               void* workspace, size_t workspace_bytes, fastnn_stream_t stream) {
+  if (conf_threshold != conf_threshold) return FASTNN_ERR_INVALID;  // NaN threshold
+  return mutual_dense_impl(desc1, conf1, n1, desc2, conf2, n2, d, dtype, true, conf_threshold,
+                           out_pairs, out_score, capacity, out_count, workspace,
+                           workspace_bytes, stream);
 }
 
 int fastnn_mutual_from_nn(const int32_t* nn12, const void* score12, int64_t n1, int64_t i0,

@@ -75,7 +75,9 @@ struct NNArgs {
   const int32_t* q_count;
   int64_t nq_static;
   const uint8_t* db_rows;  // repacked database rows [batch][ndb][row_bytes]
-  int64_t ndb;
+  int64_t ndb;             // database rows per pair, and the stride between pairs
+  const int32_t* ndb_dev;  // optional [batch]: pair b searches only its first ndb_dev[b]
+                           // (<= ndb) rows (device counts of masked, compacted maps)
   uint64_t* out_key;       // [batch][q_cap], merged with atomicMax
   int batch;
   int* status;

@@ -88,9 +88,14 @@ __global__ void __launch_bounds__(1024) mutual_count_kernel(MutualSrc m,
   if (threadIdx.x == 0) block_cnt[blockIdx.x] = sc.tot0;
 }
 
+// Exclusive scan, in place, of the nblocks counts of segment blockIdx.x
+// (block_cnt + blockIdx.x * nblocks); the segment's total goes to
+// out_count[blockIdx.x].
 __global__ void __launch_bounds__(1024) mutual_scan_kernel(int32_t* __restrict__ block_cnt,
                                                            int nblocks,
                                                            int32_t* __restrict__ out_count) {
+  block_cnt += static_cast<int64_t>(blockIdx.x) * nblocks;
+  out_count += blockIdx.x;
   __shared__ int sm[64];
   __shared__ int carry;
   if (threadIdx.x == 0) carry = 0;
@@ -136,8 +141,8 @@ __global__ void __launch_bounds__(1024) mutual_emit_kernel(MutualSrc m,
   if (f) {
     const int64_t pos = block_off[blockIdx.x] + sc.ex0;
     if (pos < cap) {
-      out_pairs[pos * 2] = static_cast<int32_t>(m.i0 + i);
-      out_pairs[pos * 2 + 1] = static_cast<int32_t>(j);
+      out_pairs[pos * 2] = m.map1 ? m.map1[i] : static_cast<int32_t>(m.i0 + i);
+      out_pairs[pos * 2 + 1] = m.map2 ? m.map2[j] : static_cast<int32_t>(j);
       if (out_score) {
         if (m.k12) {
           const uint32_t h = key_score_bits(m.k12[i]);
@@ -212,7 +217,144 @@ int grid_for(int64_t n, int threads, int max_blocks = 148 * 16) {
   return static_cast<int>(g);
 }
 
+// ------------------------------------------------------- confidence masks ---
+// A pixel takes part iff its confidence is at least the threshold (no map:
+// every pixel). Each map is compacted, in pixel order, to its kept rows:
+// per-block counts, a per-pair scan of the counts, then an ordered scatter
+// that repacks each kept row into slot (pair b, position) and records the
+// slot's pixel (c2p) and the pixel's slot (p2c, -1 when dropped). Order is
+// kept, so the lowest compacted index among equal scores is the lowest pixel.
+__device__ __forceinline__ bool mask_kept(const MaskArgs& m, int64_t g) {
+  return !m.conf || __ldg(m.conf + g) >= m.threshold;
+}
+
+__global__ void __launch_bounds__(1024) mask_count_kernel(MaskArgs m) {
+  __shared__ int sm[64];
+  const int b = blockIdx.x / m.bpp, blk = blockIdx.x % m.bpp;
+  const int64_t p = static_cast<int64_t>(blk) * 1024 + threadIdx.x;
+  const bool f = p < m.N && mask_kept(m, b * m.N + p);
+  const Scan2 sc = block_scan2(f, false, sm);
+  if (threadIdx.x == 0) m.blocks[blockIdx.x] = sc.tot0;
+}
+
+// Descriptor row (ESIZE-byte elements) into an RB-byte slot; returns max
+// |element| for int8 rows, 0 otherwise.
+template <int ESIZE, int RB>
+__device__ __forceinline__ int repack_row(const uint8_t* __restrict__ s, int d,
+                                          uint8_t* __restrict__ o) {
+  constexpr int NW = RB / 4;
+  uint32_t w[NW];
+#pragma unroll
+  for (int i = 0; i < NW; ++i) w[i] = 0;
+  const int nbytes = d * ESIZE;
+#pragma unroll
+  for (int i = 0; i < RB; ++i)
+    if (i < nbytes) w[i / 4] |= static_cast<uint32_t>(__ldg(s + i)) << (8 * (i % 4));
+  int amax = 0;
+  if (ESIZE == 1) {
+#pragma unroll
+    for (int i = 0; i < NW; ++i)
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        amax = max(amax, abs(static_cast<int>(static_cast<int8_t>(w[i] >> (8 * k)))));
+  }
+  uint4* o4 = reinterpret_cast<uint4*>(o);
+#pragma unroll
+  for (int i = 0; i < RB / 16; ++i) o4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+  return amax;
+}
+
+// Pointmap row into a float4 (x, y, z, -|p|^2); returns the fp32 bits of |p|^2.
+__device__ __forceinline__ int repack_point(const float* __restrict__ s, int d, float4* o) {
+  float4 p = make_float4(__ldg(s), d > 1 ? __ldg(s + 1) : 0.f, d > 2 ? __ldg(s + 2) : 0.f, 0.f);
+  const float n2 = __fmaf_rn(p.z, p.z, __fmaf_rn(p.y, p.y, p.x * p.x));
+  p.w = -n2;
+  *o = p;
+  return __float_as_int(n2);
+}
+
+// KIND 0: descriptor rows (ESIZE, RB); KIND 1: pointmap rows.
+template <int KIND, int ESIZE, int RB>
+__global__ void __launch_bounds__(1024) mask_emit_kernel(MaskArgs m) {
+  __shared__ int sm[64];
+  const int b = blockIdx.x / m.bpp, blk = blockIdx.x % m.bpp;
+  const int64_t p = static_cast<int64_t>(blk) * 1024 + threadIdx.x;
+  const int64_t g = b * m.N + p;
+  const bool f = p < m.N && mask_kept(m, g);
+  const Scan2 sc = block_scan2(f, false, sm);
+  int mag = 0;
+  if (p < m.N) {
+    const int64_t slot = b * m.N + m.blocks[blockIdx.x] + sc.ex0;
+    if (m.p2c) m.p2c[g] = f ? static_cast<int32_t>(slot - b * m.N) : -1;
+    if (f) {
+      m.c2p[slot] = static_cast<int32_t>(p);
+      if (KIND == 1)
+        mag = repack_point(reinterpret_cast<const float*>(m.src) + g * m.d, m.d,
+                           reinterpret_cast<float4*>(m.dst) + slot);
+      else
+        mag = repack_row<ESIZE, RB>(m.src + g * m.d * ESIZE, m.d, m.dst + slot * RB);
+    }
+  }
+  if (m.absmax) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mag = max(mag, __shfl_xor_sync(0xffffffffu, mag, o));
+    if ((threadIdx.x & 31) == 0 && mag > 0) atomicMax(m.absmax, mag);
+  }
+}
+
+// Seeds of the masked fast scheme: the kept grid pixels of each pair in grid
+// order, as compacted indices (p2c), and their count. One CTA per pair.
+__global__ void __launch_bounds__(1024) masked_seeds_kernel(const int32_t* __restrict__ p2c,
+                                                            int64_t N1, int W1, int sub,
+                                                            int64_t S, int32_t* __restrict__ F0,
+                                                            int32_t* __restrict__ seed_cnt) {
+  __shared__ int sm[64];
+  const int b = blockIdx.x;
+  const int gx = (W1 + sub - 1) / sub;
+  int base = 0;
+  for (int64_t s0 = 0; s0 < S; s0 += blockDim.x) {
+    const int64_t k = s0 + threadIdx.x;
+    int32_t pos = -1;
+    if (k < S) {
+      const int64_t u = (k / gx) * sub * static_cast<int64_t>(W1) + (k % gx) * sub;
+      pos = __ldg(p2c + b * N1 + u);
+    }
+    const Scan2 sc = block_scan2(pos >= 0, false, sm);
+    if (pos >= 0) F0[b * S + base + sc.ex0] = pos;
+    base += sc.tot0;
+  }
+  if (threadIdx.x == 0) seed_cnt[b] = base;
+}
+
 }  // namespace
+
+int mask_blocks(int64_t N) { return static_cast<int>((N + 1023) / 1024); }
+
+int launch_mask_compact(const MaskArgs& m0, int dtype, cudaStream_t st) {
+  MaskArgs m = m0;
+  m.bpp = mask_blocks(m.N);
+  const int nb = m.batch * m.bpp;
+  if (nb <= 0) return FASTNN_OK;
+  mask_count_kernel<<<nb, 1024, 0, st>>>(m);
+  mutual_scan_kernel<<<m.batch, 1024, 0, st>>>(m.blocks, m.bpp, m.count);
+  switch (dtype == FASTNN_F32_L2 ? 0 : row_bytes(dtype, m.d) * (dtype == FASTNN_I8 ? 1 : -1)) {
+    case 0: mask_emit_kernel<1, 4, 16><<<nb, 1024, 0, st>>>(m); break;
+    case 32: mask_emit_kernel<0, 1, 32><<<nb, 1024, 0, st>>>(m); break;
+    case 64: mask_emit_kernel<0, 1, 64><<<nb, 1024, 0, st>>>(m); break;
+    case -64: mask_emit_kernel<0, 2, 64><<<nb, 1024, 0, st>>>(m); break;
+    case -128: mask_emit_kernel<0, 2, 128><<<nb, 1024, 0, st>>>(m); break;
+    default: return FASTNN_ERR_UNSUPPORTED;
+  }
+  FASTNN_CUDA_TRY(cudaGetLastError());
+  return FASTNN_OK;
+}
+
+int launch_masked_seeds(const int32_t* p2c, int batch, int64_t N1, int W1, int sub, int64_t S,
+                        int32_t* F0, int32_t* seed_cnt, cudaStream_t st) {
+  masked_seeds_kernel<<<batch, 1024, 0, st>>>(p2c, N1, W1, sub, S, F0, seed_cnt);
+  FASTNN_CUDA_TRY(cudaGetLastError());
+  return FASTNN_OK;
+}
 
 int launch_repack(const void* src, int64_t rows, int d, int dtype, void* dst, int64_t pad_rows,
                   int* absmax, cudaStream_t st) {

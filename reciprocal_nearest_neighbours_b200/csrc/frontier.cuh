@@ -17,6 +17,8 @@ struct CompactArgs {
   uint32_t* claim;        // [batch][N1] first-visit stamps (round << 24 | slot)
   int64_t N1;
   int64_t N2;
+  const int32_t* map1;    // optional [batch][N1]: pixel of compacted image-1 index (masks)
+  const int32_t* map2;    // optional [batch][N2]: pixel of compacted image-2 index
   int32_t* out_pairs;     // [batch][cap][2]
   void* out_score;        // [batch][cap] or nullptr
   int64_t cap;
@@ -39,7 +41,32 @@ struct RecArgs {
   uint32_t* grid_count;  // grid-barrier arrival counter (zero before the launch)
   int* grid_abort;       // set when any CTA gives up (zero before the launch)
   int* status;
+  const int32_t* seed_cnt;  // optional [batch]: F[0] already holds this many seeds per pair
 };
+
+// Confidence-mask compaction of one map (all pairs of a batch).
+struct MaskArgs {
+  const uint8_t* src;   // [batch][N][d] rows of the map (dtype's element size)
+  const float* conf;    // [batch][N] confidences, or nullptr (every pixel kept)
+  float threshold;      // kept iff conf >= threshold
+  int64_t N;            // pixels per pair
+  int batch;
+  int d;
+  uint8_t* dst;         // [batch][N] repacked rows; the first count[b] of pair b are kept
+  int32_t* c2p;         // [batch][N]: pixel of compacted slot
+  int32_t* p2c;         // [batch][N]: slot of pixel, -1 when dropped (or nullptr)
+  int32_t* count;       // [batch] kept pixels
+  int* absmax;          // int8: max |element|; pointmaps: bits of max |p|^2 (or nullptr)
+  int32_t* blocks;      // [batch][mask_blocks(N)] scratch
+  int bpp;              // set by the launcher
+};
+
+int mask_blocks(int64_t N);
+int launch_mask_compact(const MaskArgs& m, int dtype, cudaStream_t st);
+// Kept grid seeds per pair (compacted indices, grid order) into F0, counts
+// into seed_cnt.
+int launch_masked_seeds(const int32_t* p2c, int batch, int64_t N1, int W1, int sub, int64_t S,
+                        int32_t* F0, int32_t* seed_cnt, cudaStream_t st);
 
 // Repack `rows` rows (plus pad_rows zero rows) into the kernels' layout.
 // absmax (optional) receives, by atomicMax, the largest |element| (int8) or
@@ -55,6 +82,8 @@ struct MutualSrc {
   const int32_t* nn12;
   const int32_t* nn21;
   const void* score12;
+  const int32_t* map1;  // optional: pixel of compacted image-1 row i (masked maps)
+  const int32_t* map2;  // optional: pixel of compacted image-2 row j
   int64_t n1;  // local image-1 rows
   int64_t n2;  // image-2 rows
   int64_t i0;  // global index of local row 0

@@ -145,9 +145,11 @@ __device__ void compact_pair(const CompactArgs& c, const FrontierBufs& fb, int b
       fk = __ldcg(fwd + k);
       v = key_index(fk);
       u2 = key_index(__ldcg(bwd + k));
-      // A forward pass that found no candidate leaves v = 0xFFFFFFFF.
+      // A forward pass that found no candidate leaves v = 0xFFFFFFFF: the
+      // walk ends there.
       conv = (u2 == u) && v < static_cast<uint32_t>(c.N2);
-      push = !conv && !last_round && u2 < static_cast<uint32_t>(c.N1) &&
+      push = !conv && !last_round && v < static_cast<uint32_t>(c.N2) &&
+             u2 < static_cast<uint32_t>(c.N1) &&
              __ldcg(claim + u2) == (stamp_hi | static_cast<uint32_t>(k));
       fwd[k] = 0;
       bwd[k] = 0;
@@ -157,8 +159,8 @@ __device__ void compact_pair(const CompactArgs& c, const FrontierBufs& fb, int b
       const int64_t pos = out0 + sc.ex0;
       if (pos < c.cap) {
         int32_t* op = c.out_pairs + (b * c.cap + pos) * 2;
-        op[0] = static_cast<int32_t>(u);
-        op[1] = static_cast<int32_t>(v);
+        op[0] = c.map1 ? c.map1[b * c.N1 + u] : static_cast<int32_t>(u);
+        op[1] = c.map2 ? c.map2[b * c.N2 + v] : static_cast<int32_t>(v);
         if (c.out_score) {
           if (DT == FASTNN_I8)
             static_cast<int32_t*>(c.out_score)[b * c.cap + pos] = unord_i32(key_score_bits(fk));
@@ -216,11 +218,22 @@ __device__ void fast_rounds(const RecArgs& r, NNPass&& nn, volatile int* cta_abo
     for (int64_t i = gtid; i < batch * r.max_iter; i += gsize) r.cmp.out_frontier[i] = 0;
   bool ok = sync();
   if (ok) {
-    // Seeds: the round-1 frontier of every pair.
-    for (int64_t i = gtid; i < batch * S; i += gsize)
-      seed_one(r.F[0], S, r.cmp.claim, r.N1, r.W1, r.sub, static_cast<int>(i / S),
-               static_cast<int>(i % S));
-    for (int64_t i = gtid; i < batch; i += gsize) r.cnt[0][i] = static_cast<int>(S);
+    // Seeds: the round-1 frontier of every pair (the grid, or the kept grid
+    // pixels already written to F[0] when seed_cnt is given); each claims
+    // its pixel with stamp (round 0, slot k).
+    if (r.seed_cnt) {
+      for (int64_t i = gtid; i < batch * S; i += gsize) {
+        const int b = static_cast<int>(i / S), k = static_cast<int>(i % S);
+        if (k < __ldcg(r.seed_cnt + b))
+          r.cmp.claim[b * r.N1 + __ldcg(r.F[0] + i)] = static_cast<uint32_t>(k);
+      }
+      for (int64_t i = gtid; i < batch; i += gsize) r.cnt[0][i] = __ldcg(r.seed_cnt + i);
+    } else {
+      for (int64_t i = gtid; i < batch * S; i += gsize)
+        seed_one(r.F[0], S, r.cmp.claim, r.N1, r.W1, r.sub, static_cast<int>(i / S),
+                 static_cast<int>(i % S));
+      for (int64_t i = gtid; i < batch; i += gsize) r.cnt[0][i] = static_cast<int>(S);
+    }
     ok = sync();
   }
   for (int t = 1; ok && t <= r.max_iter; ++t) {

@@ -87,11 +87,13 @@ struct __align__(16) L2Smem {
   int grid_ok;
   int more;
   int b0;
-  long long nt, u0, u1, m0, n0;
-  long long perm;  // chunk n of a segment is database chunk (n * perm) mod nt; perm < nt
+  long long u0, u1, m0, n0;
   int scan[66];
-  int cnt[kMaxBatchL2];
-  int mt[kMaxBatchL2];
+  int cnt[kMaxBatchL2];   // queries per pair
+  int mt[kMaxBatchL2];    // query tiles per pair (0 when the pair has no database row)
+  int nt[kMaxBatchL2];    // database chunks per pair
+  int rows[kMaxBatchL2];  // database rows per pair
+  int step[kMaxBatchL2];  // chunk n of a segment is chunk (n * step) mod nt; step < nt
 };
 
 constexpr size_t kSmemBytes = sizeof(L2Smem);
@@ -166,10 +168,11 @@ struct Walk {
 };
 
 __device__ __forceinline__ void walk_next(Walk& w, const L2Smem& s, int batch) {
+  const int nt = s.nt[w.b];
   ++w.n;
-  w.c += s.perm;
-  if (w.c >= s.nt) w.c -= s.nt;
-  if (w.n == s.nt) {
+  w.c += s.step[w.b];
+  if (w.c >= nt) w.c -= nt;
+  if (w.n == nt) {
     w.n = 0;
     w.c = 0;
     if (++w.m == s.mt[w.b]) {
@@ -184,7 +187,7 @@ __device__ __forceinline__ void walk_next(Walk& w, const L2Smem& s, int batch) {
 // Issue the copy of database chunk w.c of pair w.b into buffer i.
 __device__ __forceinline__ void l2_issue(const NNArgs& a, L2Smem& s, int i, const Walk& w) {
   const int64_t r0 = w.c * kDC;
-  const int64_t rows = min(static_cast<int64_t>(kDC), a.ndb - r0);
+  const int64_t rows = min(static_cast<int64_t>(kDC), s.rows[w.b] - r0);
   const uint32_t bytes = static_cast<uint32_t>(rows) * 16u;
   const uint32_t bar = ptx::smem_u32(&s.bar[i]);
   ptx::fence_proxy_async_smem();
@@ -193,42 +196,57 @@ __device__ __forceinline__ void l2_issue(const NNArgs& a, L2Smem& s, int i, cons
   s.issued[i] += 1u;
 }
 
+__device__ __forceinline__ int gcd_i(int x, int y) {
+  while (y) {
+    const int t = x % y;
+    x = y;
+    y = t;
+  }
+  return x;
+}
+
 // Thread 0: this CTA's contiguous range of units for one pass, and the
 // copies of its first kNS units.
 __device__ void l2_plan(const NNArgs& a, const PhaseQ& q, L2Smem& s) {
-  const int64_t nt = (a.ndb + kDC - 1) / kDC;
   int64_t total = 0;
   for (int b = 0; b < a.batch; ++b) {
     const int64_t c = nn_count(a, q, b);
+    const int64_t rows = a.ndb_dev ? min(static_cast<int64_t>(__ldcg(a.ndb_dev + b)), a.ndb)
+                                   : a.ndb;
+    const int nt = static_cast<int>(rows > 0 ? (rows + kDC - 1) / kDC : 0);
     s.cnt[b] = static_cast<int>(c);
-    s.mt[b] = static_cast<int>((c + kQT - 1) / kQT);
+    s.rows[b] = static_cast<int>(rows);
+    s.nt[b] = nt;
+    s.mt[b] = nt > 0 ? static_cast<int>((c + kQT - 1) / kQT) : 0;
+    // A stride coprime with nt near 0.618 nt scatters the chunks of every
+    // segment over the database: rows of a pointmap are spatially ordered,
+    // and in storage order nearly every chunk would bring a point nearer
+    // than all before it, each time opening the exact re-ranking.
+    int st = nt > 1 ? static_cast<int>(0.618 * nt) : 0;
+    if (nt > 1) {
+      if (st < 1) st = 1;
+      while (gcd_i(st, nt) != 1) ++st;
+      st %= nt;
+    }
+    s.step[b] = st;
     total += static_cast<int64_t>(s.mt[b]) * nt;
   }
   const int64_t G = gridDim.x;
   const int64_t u0 = total * blockIdx.x / G;
-  s.nt = nt;
-  // A multiplier coprime with nt scatters the chunks of every segment over
-  // the database: rows of a pointmap are spatially ordered, and in storage
-  // order nearly every chunk would bring a point nearer than all before it,
-  // each time opening the exact re-ranking.
-  long long perm = 1;
-  const long long primes[6] = {97, 89, 83, 79, 73, 71};
-  for (int t = 0; t < 6 && perm == 1; ++t)
-    if (nt % primes[t] != 0) perm = primes[t] % nt == 0 ? 1 : primes[t];
-  s.perm = perm % nt;
   s.u0 = u0;
   s.u1 = total * (blockIdx.x + 1) / G;
   int64_t acc = 0;
   int b = 0;
-  while (b < a.batch && acc + static_cast<int64_t>(s.mt[b]) * nt <= u0) {
-    acc += static_cast<int64_t>(s.mt[b]) * nt;
+  while (b < a.batch && acc + static_cast<int64_t>(s.mt[b]) * s.nt[b] <= u0) {
+    acc += static_cast<int64_t>(s.mt[b]) * s.nt[b];
     ++b;
   }
+  const int64_t nt = b < a.batch ? s.nt[b] : 0;
   s.b0 = b;
   s.m0 = nt > 0 ? (u0 - acc) / nt : 0;
   s.n0 = nt > 0 ? (u0 - acc) % nt : 0;
-  if (!s.abort_flag) {
-    Walk w{b, s.m0, s.n0, (s.n0 * s.perm) % nt};
+  if (!s.abort_flag && u0 < s.u1) {
+    Walk w{b, s.m0, s.n0, (s.n0 * s.step[b]) % nt};
     for (int64_t u = u0; u < s.u1 && u < u0 + kNS; ++u) {
       l2_issue(a, s, static_cast<int>(u - u0), w);
       walk_next(w, s, a.batch);
@@ -374,7 +392,7 @@ __device__ void l2_phase(const NNArgs& a, const PhaseQ q, L2Smem& s) {
   uint32_t ph[kNS];
 #pragma unroll
   for (int i = 0; i < kNS; ++i) ph[i] = s.bar_phase[i];
-  Walk w{s.b0, s.m0, s.n0, (s.n0 * s.perm) % s.nt};
+  Walk w{s.b0, s.m0, s.n0, (s.n0 * s.step[s.b0]) % s.nt[s.b0]};
   Walk ahead = w;  // the unit kNS ahead: the one a released buffer receives
   for (int k = 0; k < kNS; ++k) walk_next(ahead, s, a.batch);
   WarpState& W = s.ws[warp];
@@ -391,7 +409,7 @@ __device__ void l2_phase(const NNArgs& a, const PhaseQ q, L2Smem& s) {
     ok = __all_sync(kFull, l2_wait(s, i, ph[i], a.status));
     ph[i] ^= 1u;
     if (ok && active) {
-      const int rows = static_cast<int>(min(static_cast<int64_t>(kDC), a.ndb - w.c * kDC));
+      const int rows = static_cast<int>(min(static_cast<int64_t>(kDC), s.rows[w.b] - w.c * kDC));
       l2_chunk(s.buf[i], rows, static_cast<uint32_t>(w.c * kDC), Q, Wn, W, lane);
     }
     Walk nx = w;

@@ -86,9 +86,11 @@ struct Ctl {
   int more;
   int scan[66];  // block-scan scratch of the per-pair compaction
   int b0;
-  int64_t m0, n0, u0, u1, nt;
-  int mt[kMaxBatch];
-  int cnt[kMaxBatch];
+  int64_t m0, n0, u0, u1;
+  int mt[kMaxBatch];      // query tiles per pair (0 when the pair has no database row)
+  int cnt[kMaxBatch];     // queries per pair
+  int nt[kMaxBatch];      // database tiles per pair
+  int rows[kMaxBatch];    // database rows per pair
 };
 
 __host__ __device__ constexpr size_t tile_bytes_a(int rb) { return static_cast<size_t>(kBM) * rb; }
@@ -150,8 +152,8 @@ struct Pos {
 };
 
 // Units left in the current segment (same pair and query tile).
-__device__ __forceinline__ int64_t seg_len(const Pos& p, int64_t u, int64_t u1, int64_t nt) {
-  return min(u1 - u, nt - p.n);
+__device__ __forceinline__ int64_t seg_len(const Pos& p, int64_t u, int64_t u1, const Ctl* ctl) {
+  return min(u1 - u, static_cast<int64_t>(ctl->nt[p.b]) - p.n);
 }
 
 // Move to the first unit of the next segment.
@@ -428,18 +430,21 @@ __device__ __forceinline__ void pipe_setup(Ctl* ctl) {
 template <int DT>
 __device__ void plan_phase(const NNArgs& a, const PhaseQ& q, Ctl* ctl) {
   const int batch = a.batch;
-  const int64_t nt = (a.ndb + kBN - 1) / kBN;
   int64_t total = 0;
   for (int b = 0; b < batch; ++b) {
     const int64_t c = nn_count(a, q, b);
+    const int64_t rows = a.ndb_dev ? min(static_cast<int64_t>(__ldcg(a.ndb_dev + b)), a.ndb)
+                                   : a.ndb;
+    const int64_t nt = rows > 0 ? (rows + kBN - 1) / kBN : 0;
     ctl->cnt[b] = static_cast<int>(c);
-    ctl->mt[b] = static_cast<int>((c + kBM - 1) / kBM);
+    ctl->rows[b] = static_cast<int>(rows);
+    ctl->nt[b] = static_cast<int>(nt);
+    ctl->mt[b] = nt > 0 ? static_cast<int>((c + kBM - 1) / kBM) : 0;
     total += static_cast<int64_t>(ctl->mt[b]) * nt;
   }
   const int64_t G = gridDim.x;
   const int64_t u0 = total * blockIdx.x / G;
   const int64_t u1 = total * (blockIdx.x + 1) / G;
-  ctl->nt = nt;
   ctl->u0 = u0;
   ctl->u1 = u1;
   // int8 scores fit in 16 bits when d * max|q| * max|db| < 2^15; the repack
@@ -450,12 +455,13 @@ __device__ void plan_phase(const NNArgs& a, const PhaseQ& q, Ctl* ctl) {
                     : 0;
   int64_t acc = 0;
   int b = 0;
-  while (b < batch && acc + static_cast<int64_t>(ctl->mt[b]) * nt <= u0) {
-    acc += static_cast<int64_t>(ctl->mt[b]) * nt;
+  while (b < batch && acc + static_cast<int64_t>(ctl->mt[b]) * ctl->nt[b] <= u0) {
+    acc += static_cast<int64_t>(ctl->mt[b]) * ctl->nt[b];
     ++b;
   }
   ctl->b0 = b;
   const int64_t rem = u0 - acc;
+  const int64_t nt = b < batch ? ctl->nt[b] : 0;
   ctl->m0 = nt > 0 ? rem / nt : 0;
   ctl->n0 = nt > 0 ? rem % nt : 0;
 }
@@ -480,7 +486,6 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Pha
   const int64_t u0 = ctl->u0, u1 = ctl->u1;
   auto bar = [&](int i) { return ptx::smem_u32(&ctl->bars[i]); };
   const Pos start{ctl->b0, ctl->m0, ctl->n0};
-  const int64_t nt = ctl->nt;
 
   if (u0 < u1 && !ctl->abort_flag) {
     if (warp == kProducerWarp) {
@@ -492,7 +497,7 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Pha
       st.idx = ctl->p_st_idx;
       st.phase = ctl->p_st_phase;
       for (int64_t u = u0; ok && u < u1; ++seg) {
-        const int len = static_cast<int>(seg_len(p, u, u1, nt));
+        const int len = static_cast<int>(seg_len(p, u, u1, ctl));
         const int as = static_cast<int>(seg & 1);
         if (!warp_wait_bounded(bar(kBarAEmpty + as), static_cast<uint32_t>(((seg >> 1) & 1) ^ 1),
                                ctl, a.status))
@@ -546,7 +551,7 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Pha
         int par = ctl->m_par[g];
         const uint32_t d_tmem = tmem + static_cast<uint32_t>(g * kBN);
         for (int64_t u = u0; ok && u < u1; ++seg) {
-          const int len = static_cast<int>(seg_len(p, u, u1, nt));
+          const int len = static_cast<int>(seg_len(p, u, u1, ctl));
           const int as = static_cast<int>(seg & 1);
           if (!wait_bounded(bar(kBarAFull + as), static_cast<uint32_t>((seg >> 1) & 1), ctl,
                             a.status))
@@ -604,7 +609,6 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Pha
       const int lg = gw & 3;  // TMEM lane quarter (warp id mod 4)
       const int h = gw >> 2;  // column half of the tile
       const bool pack16 = ctl->pack16 != 0;
-      const int tail = static_cast<int>(a.ndb - (nt - 1) * kBN);  // valid columns, last tile
       const uint32_t acc_bar = bar(kBarAccFull + grp);
       const uint32_t rel_bar = bar(kBarAccEmpty + grp);
       const uint32_t taddr = tmem + (static_cast<uint32_t>(lg * 32) << 16) +
@@ -612,10 +616,11 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Pha
       uint4* slot = L.stash + 2 * threadIdx.x;
       Pos p = start;
       bool ok = true;
-      const int last_n = static_cast<int>(nt - 1);
       for (int64_t u = u0; ok && u < u1;) {
-        const int len = static_cast<int>(seg_len(p, u, u1, nt));
+        const int len = static_cast<int>(seg_len(p, u, u1, ctl));
         const int n0 = static_cast<int>(p.n);
+        const int last_n = ctl->nt[p.b] - 1;
+        const int tail = ctl->rows[p.b] - last_n * kBN;  // valid columns of the last tile
         typename E::S best = E::lowest();
         uint32_t bidx = 0xFFFFFFFFu;
         for (int j = (grp - ps.epar) & 1; j < len; j += kAcc) {

@@ -73,6 +73,11 @@ def test_workspace_sizes(lib):
     assert ws(fnn.FASTNN_OP_RECIPROCAL, 196608, 196608, 3, fnn.FASTNN_F32_L2, 1, 3072) > \
         2 * 196608 * 16
     assert ws(fnn.FASTNN_OP_NN, 10, 10, 4, fnn.FASTNN_F32_L2) == 0
+    # masked ops: the unmasked workspace plus compaction state
+    am = ws(fnn.FASTNN_OP_RECIPROCAL_MASKED, 196608, 196608, 24, fnn.FASTNN_I8, 1, 3072)
+    assert am >= a + 3 * 196608 * 4
+    dm = ws(fnn.FASTNN_OP_MUTUAL_DENSE_MASKED, 3072, 3072, 24, fnn.FASTNN_I8)
+    assert dm > ws(fnn.FASTNN_OP_MUTUAL_DENSE, 3072, 3072, 24, fnn.FASTNN_I8) + 2 * 3072 * 4
     # unsupported arguments size to 0
     assert ws(fnn.FASTNN_OP_NN, 10, 10, 65, fnn.FASTNN_I8) == 0
     assert ws(fnn.FASTNN_OP_NN, 10, 10, 65, fnn.FASTNN_F16) == 0
@@ -116,6 +121,20 @@ def test_argument_errors_are_reported_on_the_host(lib):
                None, fake, big, None) == -1
     assert rec(fake, 48, 64, fake, 48, 64, 24, I8, 8, 10, 1, fake, None, S, fake, None,
                None, fake, 64, None) == -3
+    # masked calls: a NaN threshold, then the unmasked calls' own checks
+    nan = float("nan")
+    recm = lib.fastnn_reciprocal_masked
+    assert recm(fake, None, 48, 64, fake, None, 48, 64, 24, I8, nan, 8, 10, 1, fake, None, S,
+                fake, None, None, fake, big, None) == -1
+    assert recm(fake, None, 48, 64, fake, None, 48, 64, 24, I8, 1.0, 8, 10, 1, fake, None, S - 1,
+                fake, None, None, fake, big, None) == -3
+    assert recm(fake, None, 48, 64, fake, None, 48, 64, 65, I8, 1.0, 8, 10, 1, fake, None, S,
+                fake, None, None, fake, big, None) == -2
+    mutm = lib.fastnn_mutual_dense_masked
+    assert mutm(fake, None, 100, fake, None, 50, 24, I8, nan, fake, None, 50, fake, fake, big,
+                None) == -1
+    assert mutm(fake, None, 100, fake, None, 50, 24, I8, 0.5, fake, None, 49, fake, fake, big,
+                None) == -3
     # dense: capacity below min(n1, n2)
     mut = lib.fastnn_mutual_dense
     assert mut(fake, 100, fake, 50, 24, I8, fake, None, 49, fake, fake, big, None) == -3
