@@ -561,14 +561,17 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Pha
               ptx::smem_desc_kmajor(ptx::smem_u32(tileA + as * tile_bytes_a(RB)), RB);
           const uint64_t bdesc0 = ptx::smem_desc_kmajor(ptx::smem_u32(tileB), RB);
           for (int j = (g - par) & (kAcc - 1); j < len; j += kAcc) {
-            if (!wait_bounded(bar(kBarAccEmpty + g), ac_phase ^ 1u, ctl, a.status) ||
-                !wait_bounded(bar(kBarBFull + st_idx), st_phase, ctl, a.status)) {
+            // The database stage is loaded long before the accumulator frees
+            // up: check it first, so that only the MMA issue follows the
+            // accumulator's hand-back.
+            const uint64_t bdesc =
+                bdesc0 + static_cast<uint64_t>((st_idx * tile_bytes_b(RB)) >> 4);
+            if (!wait_bounded(bar(kBarBFull + st_idx), st_phase, ctl, a.status) ||
+                !wait_bounded(bar(kBarAccEmpty + g), ac_phase ^ 1u, ctl, a.status)) {
               ok = false;
               break;
             }
             ptx::tc_fence_after();
-            const uint64_t bdesc =
-                bdesc0 + static_cast<uint64_t>((st_idx * tile_bytes_b(RB)) >> 4);
             // K steps of 32 bytes (32 int8 or 16 16-bit elements); step s
             // starts 32 * s bytes into the swizzled rows.
 #pragma unroll
@@ -578,8 +581,8 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Pha
               else
                 ptx::mma_bf16(d_tmem, adesc + 2 * ks, bdesc + 2 * ks, kIdesc, ks > 0 ? 1u : 0u);
             }
-            ptx::mma_commit(bar(kBarBEmpty + st_idx));
             ptx::mma_commit(bar(kBarAccFull + g));
+            ptx::mma_commit(bar(kBarBEmpty + st_idx));
             ac_phase ^= 1u;
             st_idx += kAcc;
             if (st_idx >= NS) {
@@ -624,15 +627,16 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Pha
         typename E::S best = E::lowest();
         uint32_t bidx = 0xFFFFFFFFu;
         for (int j = (grp - ps.epar) & 1; j < len; j += kAcc) {
+          const int n = n0 + j;
+          const uint32_t colbase = static_cast<uint32_t>(n) * kBN + h * kEpiCols;
+          const bool ragged = n == last_n && tail < kBN;
           if (!warp_wait_bounded(acc_bar, ps.ephase, ctl, a.status)) {
             ok = false;
             break;
           }
           ps.ephase ^= 1u;
           ptx::tc_fence_after();
-          const int n = n0 + j;
-          const uint32_t colbase = static_cast<uint32_t>(n) * kBN + h * kEpiCols;
-          if (n == last_n && tail < kBN) {
+          if (ragged) {
             // Ragged last tile of the database: column-masked fold.
             const int valid_blk = tail - h * kEpiCols;
 #pragma unroll 1
