@@ -652,8 +652,8 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Pha
             if (lane == 0) ptx::mbar_arrive(rel_bar);
           } else if (DT == FASTNN_I8 && pack16) {
             uint32_t r[kChunks][16];
-#pragma unroll
-            for (int c = 0; c < kChunks; ++c) ptx::tmem_ld16_pack(taddr + c * 32, r[c]);
+            static_assert(kChunks * 16 == 64, "one packed 128-column load");
+            ptx::tmem_ld64_pack(taddr, reinterpret_cast<uint32_t(&)[64]>(r));
             ptx::tmem_ld_wait();
             // The accumulator is free for the next MMA once it is in registers.
             ptx::tc_fence_before();
@@ -664,12 +664,10 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Pha
             // 32-bit scores: two 64-column halves, the accumulator is released
             // after the second load.
             uint32_t r[2][32];
-            ptx::tmem_ld32(taddr, r[0]);
-            ptx::tmem_ld32(taddr + 32, r[1]);
+            ptx::tmem_ld64(taddr, reinterpret_cast<uint32_t(&)[64]>(r));
             ptx::tmem_ld_wait();
             fold_wide<DT, 2>(r, colbase, best, bidx, slot);
-            ptx::tmem_ld32(taddr + 64, r[0]);
-            ptx::tmem_ld32(taddr + 96, r[1]);
+            ptx::tmem_ld64(taddr + 64, reinterpret_cast<uint32_t(&)[64]>(r));
             ptx::tmem_ld_wait();
             ptx::tc_fence_before();
             __syncwarp();
