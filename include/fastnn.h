@@ -177,6 +177,19 @@ int fastnn_mutual_from_nn(const int32_t *nn12, const void *score12, int64_t n1,
                           fastnn_stream_t stream);
 
 /*
+ * fastnn_set_wait_timeout_ns -- limit of the kernels' bounded waits for the
+ * calls that follow (process-wide; 0 restores the default of 2 s). Every wait
+ * inside the kernels (a pipeline stage, an accumulator, a grid barrier) gives
+ * up after this long: the kernel then stops issuing work, drains what it has
+ * in flight (those waits always use the 2 s default), frees its tensor
+ * memory and returns, and fastnn_device_status() reports FASTNN_ERR_TIMEOUT;
+ * the outputs of that call are undefined, the context stays usable. Meant
+ * for supervision and for testing that failure path (a limit far below a
+ * call's duration makes its waits run out); the pages have no counterpart.
+ */
+void fastnn_set_wait_timeout_ns(uint64_t ns);
+
+/*
  * Confidence-masked matching. The network predicts a confidence beside every
  * per-pixel output ("DUSt3R / MASt3R explained", the pointmap paragraph), and
  * the remedy for pixels whose geometry cannot be trusted is to mask them or

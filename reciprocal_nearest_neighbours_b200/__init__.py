@@ -32,6 +32,7 @@ from ._lib import (  # noqa: F401
     fastnn_reciprocal,
     fastnn_reciprocal_masked,
     fastnn_reciprocal_noalloc,
+    fastnn_set_wait_timeout_ns,
     fastnn_status_str,
     fastnn_workspace_size,
     library,

@@ -75,6 +75,8 @@ def library():
     lib.fastnn_kernel_timer_read.restype = I
     lib.fastnn_last_cuda_error.argtypes = []
     lib.fastnn_last_cuda_error.restype = ctypes.c_char_p
+    lib.fastnn_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
+    lib.fastnn_set_wait_timeout_ns.restype = None
     lib.fastnn_status_str.argtypes = [I]
     lib.fastnn_status_str.restype = ctypes.c_char_p
     _lib = lib
@@ -397,3 +399,8 @@ def fastnn_mutual_dense_masked(desc1: torch.Tensor, desc2: torch.Tensor,
         _stream(stream))
     _check(rc, "fastnn_mutual_dense_masked")
     return out_pairs, out_score, out_count
+
+
+def fastnn_set_wait_timeout_ns(ns: int) -> None:
+    """Limit of the kernels' bounded waits for later calls (0: the 2 s default)."""
+    library().fastnn_set_wait_timeout_ns(int(ns))

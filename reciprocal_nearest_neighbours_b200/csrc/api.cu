@@ -1,6 +1,7 @@
 // C ABI entry points (declared in include/fastnn.h): argument checks,
 // workspace carving and the launch sequence of each operation. No memory is
 // allocated here; every launch goes on the caller's stream.
+#include <atomic>
 #include <cstring>
 
 #include "common.cuh"
@@ -18,6 +19,10 @@ void note_cuda_error(cudaError_t e) { g_last_cuda_error = e; }
 }  // namespace fastnn
 
 namespace {
+
+// Limit of the kernels' bounded pipeline waits for subsequent calls (0: the
+// kernels' default of two seconds); see fastnn_set_wait_timeout_ns.
+std::atomic<uint64_t> g_wait_ns{0};
 
 constexpr size_t kAlign = 256;
 constexpr int kPadRows = 256;  // zero rows after each repacked database (one TMA box)
@@ -213,6 +218,7 @@ int fastnn_nn(const void* q, int64_t nq, const void* db, int64_t ndb, int d, int
   a.d = d;
   a.q_absmax = L.status + 1;
   a.db_absmax = L.status + 2;
+  a.wait_ns = g_wait_ns.load();
   if (dtype == FASTNN_F32_L2) {
     FASTNN_TRY(launch_nn_l2(a, st));
     return launch_decode(L.keys, nq, dtype, out_idx, out_score, st);
@@ -282,6 +288,7 @@ int reciprocal_impl(const void* desc1, const float* conf1, int H1, int W1, const
   r.fwd.d = d;
   r.fwd.q_absmax = L.status + 1;
   r.fwd.db_absmax = L.status + 2;
+  r.fwd.wait_ns = g_wait_ns.load();
   r.bwd = r.fwd;
   r.bwd.q_rows = L.d2rep;
   r.bwd.q_rows_per_pair = N2;
@@ -405,6 +412,7 @@ int mutual_dense_impl(const void* desc1, const float* conf1, int64_t n1, const v
   a.d = d;
   a.q_absmax = L.status + 1;
   a.db_absmax = L.status + 2;
+  a.wait_ns = g_wait_ns.load();
   if (masked) {
     a.q_count = M.cnt1;
     a.ndb_dev = M.cnt2;
@@ -426,6 +434,7 @@ int mutual_dense_impl(const void* desc1, const float* conf1, int64_t n1, const v
   r.d = d;
   r.q_absmax = L.status + 2;
   r.db_absmax = L.status + 1;
+  r.wait_ns = g_wait_ns.load();
   if (masked) {
     r.q_count = M.cnt2;
     r.ndb_dev = M.cnt1;
@@ -511,6 +520,8 @@ int fastnn_device_status(const void* workspace, fastnn_stream_t stream) {
 }
 
 int fastnn_kernel_timer_enable(int capacity) { return kernel_timer_enable(capacity); }
+
+void fastnn_set_wait_timeout_ns(uint64_t ns) { g_wait_ns.store(ns); }
 
 int fastnn_kernel_timer_read(int* launches, double* total_ms) {
   return kernel_timer_read(launches, total_ms);

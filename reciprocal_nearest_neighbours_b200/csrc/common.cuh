@@ -20,8 +20,15 @@ namespace fastnn {
 
 constexpr int kStatusTimeout = 1;  // bit set in the device status word
 // Every bounded wait in the kernels (mbarrier phases, grid barriers) gives up
-// after this long, sets kStatusTimeout and unwinds.
+// after this long (or after NNArgs::wait_ns when set), sets kStatusTimeout
+// and unwinds. The waits that drain in-flight copies and MMAs before a kernel
+// exits always use kTimeoutNs.
 constexpr uint64_t kTimeoutNs = 2000000000ull;
+
+// A wait's limit: the configured one, or kTimeoutNs.
+__host__ __device__ __forceinline__ uint64_t wait_limit(uint64_t configured) {
+  return configured ? configured : kTimeoutNs;
+}
 
 __host__ __device__ __forceinline__ uint32_t ord_i32(int32_t s) {
   return static_cast<uint32_t>(s) ^ 0x80000000u;
@@ -84,6 +91,7 @@ struct NNArgs {
   int d;                   // descriptor length (<= 64; <= 3 for pointmaps)
   const int* q_absmax;     // int8: max |element| of the query map (or nullptr)
   const int* db_absmax;    // int8: max |element| of the database map (or nullptr)
+  uint64_t wait_ns;        // limit of the pipeline's bounded waits (0: kTimeoutNs)
 };
 
 // The parts of a pass's query description that change from round to round

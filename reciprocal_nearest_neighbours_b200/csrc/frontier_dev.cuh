@@ -12,13 +12,14 @@ namespace fastnn {
 
 // Grid-wide barrier over the co-resident CTAs of a cooperative launch: a
 // monotonic arrival counter (zero before the launch); each CTA waits, bounded
-// by kTimeoutNs, until the counter reaches its next multiple of the grid
+// by limit_ns, until the counter reaches its next multiple of the grid
 // size. A CTA that arrives with cta_ok == false, or a wait that runs out,
 // raises the shared abort word so that every CTA leaves. `flag` is a shared
 // int that carries thread 0's verdict to the CTA. Returns the CTA-uniform
 // verdict.
 __device__ __forceinline__ bool grid_barrier(uint32_t* count, int* abort_word, int* status,
-                                             uint32_t& target, bool cta_ok, int* flag) {
+                                             uint32_t& target, bool cta_ok, int* flag,
+                                             uint64_t limit_ns) {
   __syncthreads();
   if (threadIdx.x == 0) {
     target += gridDim.x;
@@ -29,12 +30,12 @@ __device__ __forceinline__ bool grid_barrier(uint32_t* count, int* abort_word, i
     const uint64_t t0 = ptx::globaltimer_ns();
     for (uint32_t n = 1;; ++n) {
       if (*reinterpret_cast<volatile uint32_t*>(count) >= target) break;
-      if ((n & 63) == 0) {
+      if ((n & 63) == 0 || n == 8) {
         if (*reinterpret_cast<volatile int*>(abort_word)) {
           ok = false;
           break;
         }
-        if (ptx::globaltimer_ns() - t0 > kTimeoutNs) {
+        if (ptx::globaltimer_ns() - t0 > limit_ns) {
           atomicOr(status, kStatusTimeout);
           atomicExch(abort_word, 1);
           ok = false;
@@ -201,7 +202,8 @@ __device__ void fast_rounds(const RecArgs& r, NNPass&& nn, volatile int* cta_abo
   const int64_t gtid = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   const int64_t gsize = static_cast<int64_t>(gridDim.x) * blockDim.x;
   auto sync = [&]() {
-    return grid_barrier(r.grid_count, r.grid_abort, r.status, target, !*cta_abort, flag);
+    return grid_barrier(r.grid_count, r.grid_abort, r.status, target, !*cta_abort, flag,
+                        wait_limit(r.fwd.wait_ns));
   };
 
   // Clear per-call state: keys, first-visit claims, outputs.

@@ -87,6 +87,7 @@ struct __align__(16) L2Smem {
   int grid_ok;
   int more;
   int b0;
+  unsigned long long wait_ns;  // limit of the pipeline's bounded waits
   long long u0, u1, m0, n0;
   int scan[66];
   int cnt[kMaxBatchL2];   // queries per pair
@@ -112,6 +113,7 @@ __device__ __forceinline__ void l2_setup(L2Smem& s) {
       s.empty_cnt[i] = 0;
     }
     s.abort_flag = 0;
+    s.wait_ns = kTimeoutNs;
     ptx::fence_mbar_init();
   }
   __syncthreads();
@@ -122,11 +124,12 @@ __device__ __forceinline__ void l2_setup(L2Smem& s) {
 __device__ __noinline__ bool l2_wait_slow(L2Smem& s, int i, uint32_t parity, int* status) {
   const uint32_t bar = ptx::smem_u32(&s.bar[i]);
   const uint64_t t0 = ptx::globaltimer_ns();
+  const uint64_t limit = s.wait_ns;
   for (uint32_t n = 1;; ++n) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
-    if ((n & 255) == 0) {
+    if ((n & 255) == 0 || n == 8) {
       if (*reinterpret_cast<volatile int*>(&s.abort_flag)) return false;
-      if (ptx::globaltimer_ns() - t0 > kTimeoutNs) {
+      if (ptx::globaltimer_ns() - t0 > limit) {
         *reinterpret_cast<volatile int*>(&s.abort_flag) = 1;
         atomicOr(status, kStatusTimeout);
         return false;
@@ -208,6 +211,7 @@ __device__ __forceinline__ int gcd_i(int x, int y) {
 // Thread 0: this CTA's contiguous range of units for one pass, and the
 // copies of its first kNS units.
 __device__ void l2_plan(const NNArgs& a, const PhaseQ& q, L2Smem& s) {
+  s.wait_ns = wait_limit(a.wait_ns);
   int64_t total = 0;
   for (int b = 0; b < a.batch; ++b) {
     const int64_t c = nn_count(a, q, b);

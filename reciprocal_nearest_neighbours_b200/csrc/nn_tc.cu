@@ -84,6 +84,7 @@ struct Ctl {
   int pack16;
   int grid_ok;
   int more;
+  uint64_t wait_ns;  // limit of the bounded waits in force (kTimeoutNs while draining)
   int scan[66];  // block-scan scratch of the per-pair compaction
   int b0;
   int64_t m0, n0, u0, u1;
@@ -107,11 +108,12 @@ size_t smem_bytes(int rb) {
 // if another role already aborted.
 __device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, Ctl* ctl, int* status) {
   const uint64_t t0 = ptx::globaltimer_ns();
+  const uint64_t limit = ctl->wait_ns;
   for (uint32_t n = 1;; ++n) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
-    if ((n & 255) == 0) {
+    if ((n & 255) == 0 || n == 8) {
       if (*reinterpret_cast<volatile int*>(&ctl->abort_flag)) return false;
-      if (ptx::globaltimer_ns() - t0 > kTimeoutNs) {
+      if (ptx::globaltimer_ns() - t0 > limit) {
         *reinterpret_cast<volatile int*>(&ctl->abort_flag) = 1;
         atomicOr(status, kStatusTimeout);
         return false;
@@ -396,6 +398,7 @@ struct PipeState {
 __device__ __forceinline__ void pipe_setup(Ctl* ctl) {
   if (threadIdx.x == 0) {
     ctl->abort_flag = 0;
+    ctl->wait_ns = kTimeoutNs;
     ctl->p_seg = 0;
     ctl->p_st_idx = 0;
     ctl->p_st_phase = 0;
@@ -430,6 +433,7 @@ __device__ __forceinline__ void pipe_setup(Ctl* ctl) {
 template <int DT>
 __device__ void plan_phase(const NNArgs& a, const PhaseQ& q, Ctl* ctl) {
   const int batch = a.batch;
+  ctl->wait_ns = wait_limit(a.wait_ns);
   int64_t total = 0;
   for (int b = 0; b < batch; ++b) {
     const int64_t c = nn_count(a, q, b);
@@ -694,6 +698,9 @@ __device__ __forceinline__ void pipe_teardown(Ctl* ctl, uint32_t tmem, int* stat
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   auto bar = [&](int i) { return ptx::smem_u32(&ctl->bars[i]); };
+  // Draining waits for work already issued: always the long limit.
+  if (threadIdx.x == 0) ctl->wait_ns = kTimeoutNs;
+  __syncthreads();
   if (warp >= kMmaWarp0 && lane == 0) {
     ptx::mma_commit(bar(kBarDone));
     wait_bounded(bar(kBarDone), 0, ctl, status);
