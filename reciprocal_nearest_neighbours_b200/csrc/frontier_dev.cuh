@@ -25,7 +25,9 @@ __device__ __forceinline__ bool grid_barrier(uint32_t* count, int* abort_word, i
     target += gridDim.x;
     bool ok = cta_ok;
     if (!ok) atomicExch(abort_word, 1);
-    __threadfence();
+    // Release: the CTA's writes (ordered before this thread by the barrier
+    // above) become visible to every CTA that observes the arrival.
+    ptx::fence_acq_rel_gpu();
     atomicAdd(count, 1u);
     const uint64_t t0 = ptx::globaltimer_ns();
     for (uint32_t n = 1;; ++n) {
@@ -43,7 +45,9 @@ __device__ __forceinline__ bool grid_barrier(uint32_t* count, int* abort_word, i
         }
       }
     }
-    __threadfence();
+    // Acquire: every other CTA's writes before its arrival are visible to
+    // this CTA after the barrier below.
+    ptx::fence_acq_rel_gpu();
     if (*reinterpret_cast<volatile int*>(abort_word)) ok = false;
     *flag = ok ? 1 : 0;
   }
