@@ -74,6 +74,7 @@ struct RecLayout {
   uint8_t* d1rep;
   uint8_t* d2rep;
   int32_t* F[2];
+  uint32_t* Bd[2];
   uint64_t* fwd;
   uint64_t* bwd;
   uint32_t* claim;
@@ -87,6 +88,8 @@ RecLayout carve_rec(Carver& c, int64_t N1, int64_t N2, int d, int dtype, int bat
   L.d2rep = c.take<uint8_t>(static_cast<size_t>(batch * N2 + kPadRows) * rb);
   L.F[0] = c.take<int32_t>(static_cast<size_t>(batch) * S);
   L.F[1] = c.take<int32_t>(static_cast<size_t>(batch) * S);
+  L.Bd[0] = c.take<uint32_t>(static_cast<size_t>(batch) * S);
+  L.Bd[1] = c.take<uint32_t>(static_cast<size_t>(batch) * S);
   L.fwd = c.take<uint64_t>(static_cast<size_t>(batch) * S);
   L.bwd = c.take<uint64_t>(static_cast<size_t>(batch) * S);
   L.claim = c.take<uint32_t>(static_cast<size_t>(batch) * N1);
@@ -320,6 +323,8 @@ int reciprocal_impl(const void* desc1, const float* conf1, int H1, int W1, const
   r.cmp.max_iter = max_iter;
   r.F[0] = L.F[0];
   r.F[1] = L.F[1];
+  r.Bd[0] = L.Bd[0];
+  r.Bd[1] = L.Bd[1];
   r.cnt[0] = L.cnt[0];
   r.cnt[1] = L.cnt[1];
   r.N1 = N1;

@@ -99,6 +99,11 @@ struct NNArgs {
 struct PhaseQ {
   const int32_t* q_index;
   const int32_t* q_count;
+  // Optional lower bound on each query's best score, as ordered score bits
+  // (0: none) at bound[(b * q_cap + k) * bstride]: a score the query is known
+  // to reach, so that only larger-or-equal scores need a record.
+  const uint32_t* bound;
+  int bstride;
 };
 
 // Counts, frontier indices and keys may have been written by other CTAs of

@@ -34,6 +34,7 @@ struct RecArgs {
   NNArgs bwd;        // backward pass template: queries = image-2 rows of the forward keys
   CompactArgs cmp;   // per-round check/compaction template
   int32_t* F[2];     // frontier ping-pong [batch][S]
+  uint32_t* Bd[2];   // score bounds of the frontier entries (ordered bits) [batch][S]
   int32_t* cnt[2];   // frontier sizes ping-pong [batch]
   int64_t N1;        // pixels of image 1
   int64_t S;         // seeds per pair

@@ -99,23 +99,56 @@ __device__ __forceinline__ void seed_one(int32_t* F0, int64_t S_cap, uint32_t* c
   claim[b * N1 + u] = static_cast<uint32_t>(k);
 }
 
+// Block-wide exclusive scan of two small per-thread counts (each block total
+// below 2^16), packed in one word: a warp shuffle scan, then one pass over
+// the warp totals. `sm` holds 32 ints; every thread of the block must call it.
+__device__ __forceinline__ Scan2 block_scan_counts(int c0, int c1, int* sm) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int x = c0 | (c1 << 16);
+  int inc = x;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  if (lane == 31) sm[warp] = inc;
+  __syncthreads();
+  int off = 0, tot = 0;
+  for (int w = 0; w < nw; ++w) {
+    const int cw = sm[w];
+    if (w < warp) off += cw;
+    tot += cw;
+  }
+  __syncthreads();
+  const int ex = off + inc - x;
+  return Scan2{ex & 0xFFFF, ex >> 16, tot & 0xFFFF, tot >> 16};
+}
+
 // The round's frontier buffers (the rest of CompactArgs is fixed per call).
 struct FrontierBufs {
   const int32_t* F_cur;
   int32_t* F_next;
   const int32_t* cnt_cur;
   int32_t* cnt_next;
+  uint32_t* B_next;  // score bound of each pushed pixel (see fast_rounds)
 };
+
+// Slots per thread and pass of the per-pair compaction: each thread loads
+// its run of kCE consecutive slots at once, so that one pass costs a few
+// dependent L2 round trips rather than a few per slot.
+constexpr int kCE = 4;
 
 // Round t (1-based) of the fast scheme for pair b, run by one whole CTA.
 // Slot k holds pixel u = F[k] of image 1, its forward match v = NN(D1[u], D2)
 // and the backward match u' = NN(D2[v], D1). u' == u keeps (u, v); otherwise
 // u' is pushed to the next frontier if no frontier of this call has held it
-// yet: phase 1 claims u' with atomicMin on a (round, slot) stamp, phase 2 lets
-// only the claiming slot push, so duplicates within the round and pixels seen
-// in earlier rounds are dropped, deterministically. Kept pairs and pushes are
-// compacted in slot order. The round's key slots are reset to 0 for the next
-// round's atomicMax merges. `sm` holds 66 ints.
+// yet: every slot claims its u' with atomicMin on a (round, slot) stamp and
+// only the claiming slot pushes, so duplicates within the round and pixels
+// seen in earlier rounds are dropped, deterministically. A pass checks a
+// slot's claim once the claims of that pass and of all earlier passes have
+// landed: a later slot's stamp is larger and cannot undercut it. Kept pairs
+// and pushes are compacted in slot order. The round's key slots are reset to
+// 0 for the next round's atomicMax merges. `sm` holds 66 ints.
 template <int DT>
 __device__ void compact_pair(const CompactArgs& c, const FrontierBufs& fb, int b, int t,
                              bool last_round, int* sm) {
@@ -129,54 +162,77 @@ __device__ void compact_pair(const CompactArgs& c, const FrontierBufs& fb, int b
   uint64_t* bwd = c.bwd_key + b * c.S_cap;
   uint32_t* claim = c.claim + b * c.N1;
   const uint32_t stamp_hi = static_cast<uint32_t>(t) << 24;
+  const uint32_t N1 = static_cast<uint32_t>(c.N1), N2 = static_cast<uint32_t>(c.N2);
 
-  if (!last_round) {
-    for (int k = threadIdx.x; k < cnt; k += blockDim.x) {
-      const uint32_t u2 = key_index(__ldcg(bwd + k));
-      if (u2 != static_cast<uint32_t>(__ldcg(F + k)) && u2 < static_cast<uint32_t>(c.N1))
-        atomicMin(&claim[u2], stamp_hi | static_cast<uint32_t>(k));
-    }
-  }
   if (threadIdx.x == 0) sm[64] = __ldcg(c.out_count + b);
   __syncthreads();
   int out0 = sm[64], next0 = 0;
-  for (int s = 0; s < cnt; s += blockDim.x) {
-    const int k = s + threadIdx.x;
-    bool conv = false, push = false;
-    uint32_t u = 0, v = 0, u2 = 0;
-    uint64_t fk = 0;
-    if (k < cnt) {
-      u = static_cast<uint32_t>(__ldcg(F + k));
-      fk = __ldcg(fwd + k);
-      v = key_index(fk);
-      u2 = key_index(__ldcg(bwd + k));
-      // A forward pass that found no candidate leaves v = 0xFFFFFFFF: the
-      // walk ends there.
-      conv = (u2 == u) && v < static_cast<uint32_t>(c.N2);
-      push = !conv && !last_round && v < static_cast<uint32_t>(c.N2) &&
-             u2 < static_cast<uint32_t>(c.N1) &&
-             __ldcg(claim + u2) == (stamp_hi | static_cast<uint32_t>(k));
-      fwd[k] = 0;
-      bwd[k] = 0;
+  const int per_pass = static_cast<int>(blockDim.x) * kCE;
+  for (int s = 0; s < cnt; s += per_pass) {
+    const int k0 = s + static_cast<int>(threadIdx.x) * kCE;
+    uint32_t u[kCE], u2[kCE], s2[kCE];
+    uint64_t fk[kCE];
+#pragma unroll
+    for (int j = 0; j < kCE; ++j) {
+      const bool in = k0 + j < cnt;
+      u[j] = in ? static_cast<uint32_t>(__ldcg(F + k0 + j)) : 0u;
+      fk[j] = in ? __ldcg(fwd + k0 + j) : 0ull;
+      const uint64_t bk = in ? __ldcg(bwd + k0 + j) : 0ull;
+      u2[j] = key_index(bk);
+      s2[j] = key_score_bits(bk);
     }
-    const Scan2 sc = block_scan2(conv, push, sm);
-    if (conv) {
-      const int64_t pos = out0 + sc.ex0;
-      if (pos < c.cap) {
-        int32_t* op = c.out_pairs + (b * c.cap + pos) * 2;
-        op[0] = c.map1 ? c.map1[b * c.N1 + u] : static_cast<int32_t>(u);
-        op[1] = c.map2 ? c.map2[b * c.N2 + v] : static_cast<int32_t>(v);
-        if (c.out_score) {
-          if (DT == FASTNN_I8)
-            static_cast<int32_t*>(c.out_score)[b * c.cap + pos] = unord_i32(key_score_bits(fk));
-          else if (DT == FASTNN_F32_L2)
-            static_cast<float*>(c.out_score)[b * c.cap + pos] = -unord_f32(key_score_bits(fk));
-          else
-            static_cast<float*>(c.out_score)[b * c.cap + pos] = unord_f32(key_score_bits(fk));
+    if (!last_round) {
+#pragma unroll
+      for (int j = 0; j < kCE; ++j)
+        if (k0 + j < cnt && u2[j] != u[j] && u2[j] < N1)
+          atomicMin(&claim[u2[j]], stamp_hi | static_cast<uint32_t>(k0 + j));
+      __syncthreads();
+    }
+    unsigned conv_m = 0, push_m = 0;
+#pragma unroll
+    for (int j = 0; j < kCE; ++j) {
+      const int k = k0 + j;
+      if (k < cnt) {
+        // A forward pass that found no candidate leaves v = 0xFFFFFFFF: the
+        // walk ends there.
+        const uint32_t v = key_index(fk[j]);
+        if (u2[j] == u[j] && v < N2) {
+          conv_m |= 1u << j;
+        } else if (!last_round && v < N2 && u2[j] < N1 &&
+                   __ldcg(claim + u2[j]) == (stamp_hi | static_cast<uint32_t>(k))) {
+          push_m |= 1u << j;
         }
+        fwd[k] = 0;
+        bwd[k] = 0;
       }
     }
-    if (push) fb.F_next[b * c.S_cap + next0 + sc.ex1] = static_cast<int32_t>(u2);
+    const Scan2 sc = block_scan_counts(__popc(conv_m), __popc(push_m), sm);
+    int pos = out0 + sc.ex0, nxt = next0 + sc.ex1;
+#pragma unroll
+    for (int j = 0; j < kCE; ++j) {
+      if ((conv_m >> j) & 1u) {
+        if (pos < c.cap) {
+          const uint32_t v = key_index(fk[j]);
+          int32_t* op = c.out_pairs + (b * c.cap + pos) * 2;
+          op[0] = c.map1 ? c.map1[b * c.N1 + u[j]] : static_cast<int32_t>(u[j]);
+          op[1] = c.map2 ? c.map2[b * c.N2 + v] : static_cast<int32_t>(v);
+          if (c.out_score) {
+            if (DT == FASTNN_I8)
+              static_cast<int32_t*>(c.out_score)[b * c.cap + pos] = unord_i32(key_score_bits(fk[j]));
+            else if (DT == FASTNN_F32_L2)
+              static_cast<float*>(c.out_score)[b * c.cap + pos] = -unord_f32(key_score_bits(fk[j]));
+            else
+              static_cast<float*>(c.out_score)[b * c.cap + pos] = unord_f32(key_score_bits(fk[j]));
+          }
+        }
+        ++pos;
+      }
+      if ((push_m >> j) & 1u) {
+        fb.F_next[b * c.S_cap + nxt] = static_cast<int32_t>(u2[j]);
+        fb.B_next[b * c.S_cap + nxt] = s2[j];
+        ++nxt;
+      }
+    }
     out0 += sc.tot0;
     next0 += sc.tot1;
   }
@@ -244,11 +300,15 @@ __device__ void fast_rounds(const RecArgs& r, NNPass&& nn, volatile int* cta_abo
   }
   for (int t = 1; ok && t <= r.max_iter; ++t) {
     const int cur = (t - 1) & 1, nxt = t & 1;
-    nn(0, PhaseQ{r.F[cur], r.cnt[cur]});
+    // Score bounds: a pushed pixel u' reaches at least its backward score
+    // <D2[v], D1[u']> in the forward pass, and a match v reaches at least its
+    // forward score <D1[u], D2[v]> in the backward pass (the same dot
+    // product). The seeds of round 1 have none.
+    nn(0, PhaseQ{r.F[cur], r.cnt[cur], t > 1 ? r.Bd[cur] : nullptr, 1});
     if (!sync()) break;
-    nn(1, PhaseQ{nullptr, r.cnt[cur]});
+    nn(1, PhaseQ{nullptr, r.cnt[cur], reinterpret_cast<const uint32_t*>(r.cmp.fwd_key) + 1, 2});
     if (!sync()) break;
-    const FrontierBufs fb{r.F[cur], r.F[nxt], r.cnt[cur], r.cnt[nxt]};
+    const FrontierBufs fb{r.F[cur], r.F[nxt], r.cnt[cur], r.cnt[nxt], r.Bd[nxt]};
     for (int b = blockIdx.x; b < batch; b += gridDim.x)
       compact_pair<DT>(r.cmp, fb, b, t, t == r.max_iter, scan);
     if (!sync()) break;

@@ -456,7 +456,7 @@ __device__ void l2_phase(const NNArgs& a, const PhaseQ q, L2Smem& s) {
 __global__ void __launch_bounds__(kThreads, 1) nn_l2_kernel(const __grid_constant__ NNArgs a) {
   L2Smem& s = l2_smem();
   l2_setup(s);
-  l2_phase(a, PhaseQ{a.q_index, a.q_count}, s);
+  l2_phase(a, PhaseQ{a.q_index, a.q_count, nullptr, 0}, s);
   l2_teardown(s, a.status);
 }
 

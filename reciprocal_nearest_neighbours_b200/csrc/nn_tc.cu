@@ -54,6 +54,10 @@ constexpr int kThreads = 32 * (kEpiWarps + 1 + kAcc);
 constexpr int kEpiCols = kBN / 2;               // columns of a tile per epilogue thread
 constexpr int kChunks = kEpiCols / 32;          // 32-column TMEM loads per unit and thread
 constexpr int kMaxBatch = 1024;
+// Work-split cost of starting a segment, in units (measured: a CTA whose
+// range holds two segments ran ~5 us, about 10 units, longer than one with
+// a single segment of the same length).
+constexpr int64_t kSegCost = 8;
 constexpr int kStashBytes = kEpiWarps * 32 * 32;  // 32 B per epilogue thread
 
 // Barrier slots inside the barrier block.
@@ -212,6 +216,8 @@ struct Epi<FASTNN_I8> {
   static __device__ __forceinline__ S mx(S x, S y) { return max(x, y); }
   static __device__ __forceinline__ S mx3(S x, S y, S z) { return max(max(x, y), z); }
   static __device__ __forceinline__ uint32_t ord(S s) { return ord_i32(s); }
+  // Running best that a score equal to the bound beats (scores are exact).
+  static __device__ __forceinline__ S below_bound(uint32_t bits) { return unord_i32(bits) - 1; }
 };
 
 // bf16 and half descriptors: fp32 scores.
@@ -227,6 +233,13 @@ struct Epi<FASTNN_BF16> {
     return r;
   }
   static __device__ __forceinline__ uint32_t ord(S s) { return ord_f32(s); }
+  // Running best that the bound's own dot product beats: the bound was
+  // accumulated with the operands' roles swapped, so it is lowered by a margin
+  // far above any difference in rounding between the two sums.
+  static __device__ __forceinline__ S below_bound(uint32_t bits) {
+    const float s = unord_f32(bits);
+    return s - (fabsf(s) + 1.0f) * 0x1p-12f;
+  }
 };
 
 template <>
@@ -434,7 +447,6 @@ template <int DT>
 __device__ void plan_phase(const NNArgs& a, const PhaseQ& q, Ctl* ctl) {
   const int batch = a.batch;
   ctl->wait_ns = wait_limit(a.wait_ns);
-  int64_t total = 0;
   for (int b = 0; b < batch; ++b) {
     const int64_t c = nn_count(a, q, b);
     const int64_t rows = a.ndb_dev ? min(static_cast<int64_t>(__ldcg(a.ndb_dev + b)), a.ndb)
@@ -444,30 +456,49 @@ __device__ void plan_phase(const NNArgs& a, const PhaseQ& q, Ctl* ctl) {
     ctl->rows[b] = static_cast<int>(rows);
     ctl->nt[b] = static_cast<int>(nt);
     ctl->mt[b] = nt > 0 ? static_cast<int>((c + kBM - 1) / kBM) : 0;
-    total += static_cast<int64_t>(ctl->mt[b]) * nt;
   }
+  // Contiguous ranges of equal cost, where a segment (one query tile of one
+  // pair: nt units on the same query tile) costs its units plus kSegCost for
+  // starting it (query gather, pipeline refill, result flush), so that a CTA
+  // whose range starts a new segment takes that many fewer units.
   const int64_t G = gridDim.x;
-  const int64_t u0 = total * blockIdx.x / G;
-  const int64_t u1 = total * (blockIdx.x + 1) / G;
-  ctl->u0 = u0;
-  ctl->u1 = u1;
+  int64_t cost = 0;
+  for (int b = 0; b < batch; ++b) cost += static_cast<int64_t>(ctl->mt[b]) * (ctl->nt[b] + kSegCost);
+  // Unit index at cost position C (monotone in C; 0 at 0, total at cost).
+  auto unit_at = [&](int64_t C, int& b_out, int64_t& m_out, int64_t& n_out) {
+    int64_t units = 0, acc = 0;
+    int b = 0;
+    while (b < batch) {
+      const int64_t segc = ctl->nt[b] + kSegCost;
+      const int64_t pc = static_cast<int64_t>(ctl->mt[b]) * segc;
+      if (acc + pc > C) break;
+      acc += pc;
+      units += static_cast<int64_t>(ctl->mt[b]) * ctl->nt[b];
+      ++b;
+    }
+    b_out = b;
+    m_out = n_out = 0;
+    if (b >= batch) return units;
+    const int64_t segc = ctl->nt[b] + kSegCost;
+    const int64_t j = (C - acc) / segc;
+    const int64_t off = max(static_cast<int64_t>(0), (C - acc) - j * segc - kSegCost);
+    m_out = j;
+    n_out = off;
+    return units + j * ctl->nt[b] + off;
+  };
+  int b, b_end;
+  int64_t m0, n0, m_end, n_end;
+  ctl->u0 = unit_at(cost * blockIdx.x / G, b, m0, n0);
+  ctl->u1 = unit_at(cost * (blockIdx.x + 1) / G, b_end, m_end, n_end);
   // int8 scores fit in 16 bits when d * max|q| * max|db| < 2^15; the repack
   // pass measured both maxima.
   ctl->pack16 = (DT == FASTNN_I8 && a.q_absmax && a.db_absmax &&
                  static_cast<int64_t>(__ldcg(a.q_absmax)) * __ldcg(a.db_absmax) * a.d <= 32767)
                     ? 1
                     : 0;
-  int64_t acc = 0;
-  int b = 0;
-  while (b < batch && acc + static_cast<int64_t>(ctl->mt[b]) * ctl->nt[b] <= u0) {
-    acc += static_cast<int64_t>(ctl->mt[b]) * ctl->nt[b];
-    ++b;
-  }
   ctl->b0 = b;
-  const int64_t rem = u0 - acc;
-  const int64_t nt = b < batch ? ctl->nt[b] : 0;
-  ctl->m0 = nt > 0 ? rem / nt : 0;
-  ctl->n0 = nt > 0 ? rem % nt : 0;
+  ctl->m0 = m0;
+  ctl->n0 = n0;
 }
 
 // One nearest-neighbour phase: plan (thread 0), then each role runs its loop
@@ -628,7 +659,16 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Pha
         const int n0 = static_cast<int>(p.n);
         const int last_n = ctl->nt[p.b] - 1;
         const int tail = ctl->rows[p.b] - last_n * kBN;  // valid columns of the last tile
+        // A row with a score bound starts just below it: only tiles that
+        // reach the bound can hold the row's maximum, and only they search
+        // for its column. A row whose tiles all stay below keeps no result
+        // here; another CTA's range holds the bound's own column.
+        const int64_t krow = p.m * kBM + lg * 32 + lane;
         typename E::S best = E::lowest();
+        if (q.bound && krow < ctl->cnt[p.b]) {
+          const uint32_t bits = __ldcg(q.bound + (p.b * a.q_cap + krow) * q.bstride);
+          if (bits != 0u) best = E::below_bound(bits);
+        }
         uint32_t bidx = 0xFFFFFFFFu;
         for (int j = (grp - ps.epar) & 1; j < len; j += kAcc) {
           const int n = n0 + j;
@@ -680,9 +720,8 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Pha
           }
         }
         if (!ok) break;
-        const int64_t k = p.m * kBM + lg * 32 + lane;
-        if (k < ctl->cnt[p.b] && bidx != 0xFFFFFFFFu)
-          atomicMax(reinterpret_cast<unsigned long long*>(&a.out_key[p.b * a.q_cap + k]),
+        if (krow < ctl->cnt[p.b] && bidx != 0xFFFFFFFFu)
+          atomicMax(reinterpret_cast<unsigned long long*>(&a.out_key[p.b * a.q_cap + krow]),
                     static_cast<unsigned long long>(make_key(E::ord(best), bidx)));
         u += len;
         ps.epar ^= len & 1;
@@ -724,7 +763,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   pipe_setup(L.ctl);
   const uint32_t tmem = L.ctl->tmem_base;
   PipeState ps;
-  run_phase<DT, RB>(&tmap_db, a, PhaseQ{a.q_index, a.q_count}, L, tmem, ps);
+  run_phase<DT, RB>(&tmap_db, a, PhaseQ{a.q_index, a.q_count, nullptr, 0}, L, tmem, ps);
   pipe_teardown(L.ctl, tmem, a.status);
 }
 

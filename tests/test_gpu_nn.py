@@ -110,3 +110,24 @@ def test_nn_bf16_full_size_database_sampled_queries():
     qi = np.sort(rng.choice(D1.shape[0], size=256, replace=False))
     idx, score = fastnn_nn(to_dev(D1[qi]), to_dev(D2))
     check_nn_bf16(idx, score, D1[qi], D2, oracle.nn(D1[qi], D2, "bf16"))
+
+
+@pytest.mark.parametrize("half", ["bf16", "f16"])
+def test_float_dot_products_do_not_depend_on_operand_roles(half):
+    """The score of a mutual pair is the same fp32 number whichever map holds
+    the queries. The fast scheme's passes start each query at the score it is
+    known to reach from the previous pass (computed with the roles swapped),
+    lowered by a safety margin; equality here means the margin is never used."""
+    p = synth.warped_pair_bf16(synth.BASE_SEED + 9, H=96, W=128)
+    D1 = p.desc1.reshape(-1, p.d)
+    D2 = p.desc2.reshape(-1, p.d)
+    if half == "f16":
+        D1 = synth.f64_to_f16_bits(synth.bf16_bits_to_f64(D1))
+        D2 = synth.f64_to_f16_bits(synth.bf16_bits_to_f64(D2))
+    i12, s12 = fastnn_nn(to_dev(D1, half), to_dev(D2, half))
+    i21, s21 = fastnn_nn(to_dev(D2, half), to_dev(D1, half))
+    i12, s12 = i12.cpu().numpy(), s12.cpu().numpy()
+    i21, s21 = i21.cpu().numpy(), s21.cpu().numpy()
+    mutual = np.nonzero(i21[i12] == np.arange(len(i12)))[0]
+    assert len(mutual) > 1000
+    assert np.array_equal(s12[mutual].view(np.uint32), s21[i12[mutual]].view(np.uint32))
