@@ -23,7 +23,10 @@
 // once, the order of a plain loop over the coordinates -- and rounded to
 // fp32. The result is the lowest index among the points whose fp64 squared
 // distance rounds to the same fp32 value as the smallest one, and the score
-// reported is that fp32 value.
+// reported is that fp32 value. In the fast scheme's passes a query usually
+// comes with the fp32 distance D of a point it is known to reach (its partner
+// in the previous pass); the window then starts at the floor that D implies
+// instead of opening at every chunk until a near point has been seen.
 //
 // Work: units (pair b, 128-query tile m, 1024-row database chunk n), split
 // into contiguous ranges over persistent CTAs of 16 warps. Chunks come into a
@@ -74,6 +77,7 @@ struct WarpState {
   unsigned long long key[kQW];  // winner: (fp32 distance bits << 32) | index
   float smax[kQW];              // largest fp32 score s~ seen in the segment
   float win2[kQW];              // window width 2E
+  float floor[kQW];             // lowest window edge the query's bound allows, or -FLT_MAX
 };
 
 struct __align__(16) L2Smem {
@@ -262,8 +266,8 @@ struct Queries {
   float x[kQW], y[kQW], z[kQW];  // 2 q per coordinate
 };
 
-// Per-query lower edge of the re-ranking window, smax - 2E, or -FLT_MAX
-// before any score (warp-uniform values, read every chunk).
+// Per-query lower edge of the re-ranking window, max(smax - 2E, floor), or
+// the floor before any score (warp-uniform values, read every chunk).
 struct Window {
   float thr[kQW];
 };
@@ -275,17 +279,31 @@ __device__ __forceinline__ void load_queries(const NNArgs& a, const PhaseQ& q, i
                                              Queries& Q, Window& Wn) {
   float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
   const int64_t k = k0 + lane;
+  uint32_t bound = 0u;
   if (lane < kQW && k < cnt) {
     const int64_t row = nn_query_row(a, q, b, k);
     if (row >= 0 && row < a.q_rows_per_pair)
       v = __ldg(reinterpret_cast<const float4*>(a.q_rows) + b * a.q_rows_per_pair + row);
+    if (q.bound) bound = __ldcg(q.bound + (b * a.q_cap + k) * q.bstride);
   }
+  float floor = -FLT_MAX;
   if (lane < kQW) {
     // 2E = 16 u (|a| + R)^2; the norms come from fp32 sums (relative error
     // below 3 u), inflated by 2^-20 to stay an upper bound.
     const float ra = sqrtf(fmaxf(-v.w, 0.f)) * (1.f + 0x1p-20f);
     const float rp = sqrtf(max_p2) * (1.f + 0x1p-20f);
-    W.win2[lane] = 0x1p-20f * (ra + rp) * (ra + rp) * (1.f + 0x1p-20f);
+    const float win2 = 0x1p-20f * (ra + rp) * (ra + rp) * (1.f + 0x1p-20f);
+    // A bound (ordered bits of -D, D the fp32 distance of a point this query
+    // is known to reach) means the answer r has |a - r|^2 <= D (1 + 2u), so
+    // s(r) >= |a|^2 - D (1 + 2u) and s~(r) >= that - E. The floor lowers
+    // both terms by 2^-20 (16 u, above the rounding of |a|^2, of D and of
+    // these operations) and subtracts 2E.
+    if (bound != 0u) {
+      const float D = -unord_f32(bound);
+      floor = (-v.w) * (1.f - 0x1p-20f) - D * (1.f + 0x1p-20f) - win2;
+    }
+    W.win2[lane] = win2;
+    W.floor[lane] = floor;
     W.smax[lane] = -INFINITY;
     W.key[lane] = ~0ull;
   }
@@ -294,7 +312,7 @@ __device__ __forceinline__ void load_queries(const NNArgs& a, const PhaseQ& q, i
     Q.x[i] = 2.f * __shfl_sync(kFull, v.x, i);
     Q.y[i] = 2.f * __shfl_sync(kFull, v.y, i);
     Q.z[i] = 2.f * __shfl_sync(kFull, v.z, i);
-    Wn.thr[i] = -FLT_MAX;
+    Wn.thr[i] = __shfl_sync(kFull, floor, i);
   }
   __syncwarp();
 }
@@ -347,7 +365,7 @@ __device__ __forceinline__ void l2_chunk(const float4* __restrict__ buf, int row
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
     const float smax = fmaxf(W.smax[i], M);
-    const float thr = smax - W.win2[i];
+    const float thr = fmaxf(smax - W.win2[i], W.floor[i]);
     Wn.thr[i] = thr;
     const float ax = 0.5f * Q.x[i], ay = 0.5f * Q.y[i], az = 0.5f * Q.z[i];
     unsigned long long best = W.key[i];

@@ -20,9 +20,12 @@
 //       accumulators in turn; tcgen05.commit frees the database stage and
 //       hands the accumulator to its epilogue group.
 // Work: units (pair, 128-query tile, kBN-row database tile) in row-major
-// order, split into contiguous ranges over the CTAs. A run of units that
-// share a query tile is a segment; at its end the CTA merges each row's
-// partial result with one 64-bit atomicMax, which is order independent.
+// order, split into contiguous ranges of equal cost over the CTAs. A run of
+// units that share a query tile is a segment; at its end the CTA merges each
+// row's partial result with one 64-bit atomicMax, which is order
+// independent. A query may come with a score it is known to reach (the fast
+// scheme's previous pass); its running best then starts just below that
+// score, so that only tiles reaching it search for the column.
 // Descriptors are zero-padded to 32 elements (32 B int8 rows, 64 B bf16 rows)
 // by the repack kernel, so the padding adds nothing to any score.
 // Every mbarrier wait is bounded; on expiry the kernel records
@@ -131,6 +134,19 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, Ctl*
   return wait_slow(bar, parity, ctl, status);
 }
 
+// Bounded wait that polls with the non-blocking test first: used where the
+// wait is on the critical path of the accumulator hand-off (the MMA issuer
+// waiting for an epilogue group to free its accumulator), since a thread
+// suspended in try_wait resumes later than a polling one notices the phase.
+// After kSpinPolls polls it continues as wait_bounded.
+constexpr int kSpinPolls = 2048;
+__device__ __forceinline__ bool spin_wait_bounded(uint32_t bar, uint32_t parity, Ctl* ctl,
+                                                  int* status) {
+  for (int n = 0; n < kSpinPolls; ++n)
+    if (ptx::mbar_test_wait(bar, parity)) return true;
+  return wait_slow(bar, parity, ctl, status);
+}
+
 // Index and phase bit of a ring of mbarrier-guarded slots.
 struct Ring {
   int idx = 0;
@@ -176,31 +192,47 @@ __device__ __forceinline__ void next_segment(Pos& p, const Ctl* ctl, int batch) 
 // Query-tile gather: 32 lanes copy 128 rows of `rb` bytes into a K-major tile
 // with the 32B / 64B / 128B swizzle (rb = 32 / 64 / 128) the MMA descriptor
 // names: the 16-byte chunk c of row r lands at r * rb + 16 * (c ^ swz(r)).
+// All row indices are loaded first, then the rows in batches of kRB: the
+// loads of a batch are in flight together instead of one dependent index
+// and row load per row.
 template <int RB>
 __device__ __forceinline__ void gather_a(uint8_t* tile, const NNArgs& a, const PhaseQ& q, int b,
                                          int64_t m, int cnt, int lane) {
   constexpr int kC = RB / 16;
+  constexpr int kR = kBM / 32;             // rows per lane
+  constexpr int kRB = RB == 32 ? kR : 2;   // rows per batch of loads
+  int64_t row[kR];
 #pragma unroll
-  for (int i = 0; i < kBM / 32; ++i) {
-    const int r = lane + 32 * i;
-    const int64_t k = m * kBM + r;
-    uint4 v[kC];
-    const int64_t row = k < cnt ? nn_query_row(a, q, b, k) : -1;
-    // Rows outside the query source (never produced by a healthy pipeline)
-    // read as zeros instead of faulting.
-    if (row >= 0 && row < a.q_rows_per_pair) {
-      const uint4* src = reinterpret_cast<const uint4*>(
-          a.q_rows + (static_cast<int64_t>(b) * a.q_rows_per_pair + row) * RB);
+  for (int i = 0; i < kR; ++i) {
+    const int64_t k = m * kBM + lane + 32 * i;
+    row[i] = k < cnt ? nn_query_row(a, q, b, k) : -1;
+  }
 #pragma unroll
-      for (int c = 0; c < kC; ++c) v[c] = __ldg(src + c);
-    } else {
+  for (int i0 = 0; i0 < kR; i0 += kRB) {
+    uint4 v[kRB][kC];
 #pragma unroll
-      for (int c = 0; c < kC; ++c) v[c] = make_uint4(0, 0, 0, 0);
+    for (int i = 0; i < kRB; ++i) {
+      // Rows outside the query source (never produced by a healthy
+      // pipeline) read as zeros instead of faulting.
+      const int64_t rw = row[i0 + i];
+      if (rw >= 0 && rw < a.q_rows_per_pair) {
+        const uint4* src = reinterpret_cast<const uint4*>(
+            a.q_rows + (static_cast<int64_t>(b) * a.q_rows_per_pair + rw) * RB);
+#pragma unroll
+        for (int c = 0; c < kC; ++c) v[i][c] = __ldg(src + c);
+      } else {
+#pragma unroll
+        for (int c = 0; c < kC; ++c) v[i][c] = make_uint4(0, 0, 0, 0);
+      }
     }
-    const int swz = RB == 32 ? ((r >> 2) & 1) : RB == 64 ? ((r >> 1) & 3) : (r & 7);
 #pragma unroll
-    for (int c = 0; c < kC; ++c)
-      *reinterpret_cast<uint4*>(tile + r * RB + 16 * (c ^ swz)) = v[c];
+    for (int i = 0; i < kRB; ++i) {
+      const int r = lane + 32 * (i0 + i);
+      const int swz = RB == 32 ? ((r >> 2) & 1) : RB == 64 ? ((r >> 1) & 3) : (r & 7);
+#pragma unroll
+      for (int c = 0; c < kC; ++c)
+        *reinterpret_cast<uint4*>(tile + r * RB + 16 * (c ^ swz)) = v[i][c];
+    }
   }
 }
 
@@ -446,6 +478,10 @@ __device__ __forceinline__ void pipe_setup(Ctl* ctl) {
 template <int DT>
 __device__ void plan_phase(const NNArgs& a, const PhaseQ& q, Ctl* ctl) {
   const int batch = a.batch;
+  // Loaded up front so that their latency overlaps the count loads.
+  const bool have_absmax = DT == FASTNN_I8 && a.q_absmax && a.db_absmax;
+  const int q_absmax = have_absmax ? __ldcg(a.q_absmax) : 0;
+  const int db_absmax = have_absmax ? __ldcg(a.db_absmax) : 0;
   ctl->wait_ns = wait_limit(a.wait_ns);
   for (int b = 0; b < batch; ++b) {
     const int64_t c = nn_count(a, q, b);
@@ -492,10 +528,8 @@ __device__ void plan_phase(const NNArgs& a, const PhaseQ& q, Ctl* ctl) {
   ctl->u1 = unit_at(cost * (blockIdx.x + 1) / G, b_end, m_end, n_end);
   // int8 scores fit in 16 bits when d * max|q| * max|db| < 2^15; the repack
   // pass measured both maxima.
-  ctl->pack16 = (DT == FASTNN_I8 && a.q_absmax && a.db_absmax &&
-                 static_cast<int64_t>(__ldcg(a.q_absmax)) * __ldcg(a.db_absmax) * a.d <= 32767)
-                    ? 1
-                    : 0;
+  ctl->pack16 =
+      (have_absmax && static_cast<int64_t>(q_absmax) * db_absmax * a.d <= 32767) ? 1 : 0;
   ctl->b0 = b;
   ctl->m0 = m0;
   ctl->n0 = n0;
@@ -537,6 +571,9 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Pha
         if (!warp_wait_bounded(bar(kBarAEmpty + as), static_cast<uint32_t>(((seg >> 1) & 1) ^ 1),
                                ctl, a.status))
           break;
+        // (Issuing the database loads of free stages before the gather was
+        // measured slower: at a pass start every CTA's burst of tile loads
+        // delays the gather's dependent loads.)
         gather_a<RB>(tileA + as * tile_bytes_a(RB), a, q, p.b, p.m, ctl->cnt[p.b], lane);
         ptx::fence_proxy_async_smem();
         ptx::mbar_arrive(bar(kBarAFull + as));
@@ -602,7 +639,7 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Pha
             const uint64_t bdesc =
                 bdesc0 + static_cast<uint64_t>((st_idx * tile_bytes_b(RB)) >> 4);
             if (!wait_bounded(bar(kBarBFull + st_idx), st_phase, ctl, a.status) ||
-                !wait_bounded(bar(kBarAccEmpty + g), ac_phase ^ 1u, ctl, a.status)) {
+                !spin_wait_bounded(bar(kBarAccEmpty + g), ac_phase ^ 1u, ctl, a.status)) {
               ok = false;
               break;
             }
