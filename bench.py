@@ -375,7 +375,9 @@ def run_ours(args, rank, world, local):
         def call():
             fnn.fastnn_mutual_dense(d1, d2, out_pairs=out_pairs, out_score=out_score,
                                     out_count=out_count, workspace=ws, stream=stream)
-        launches_per_step = 2 + 2 + 3  # 2 repack, 2 tensor-core passes, count/scan/emit
+        # 2 repack, forward pass, image list (mark/count/scan/emit), backward
+        # pass, mutual count/scan/emit
+        launches_per_step = 2 + 1 + 4 + 1 + 3
         kernels_per_step = 2
     elif masked:
         def call():
@@ -406,8 +408,13 @@ def run_ours(args, rank, world, local):
     torch.cuda.synchronize(dev)
     assert fnn.fastnn_device_status(ws) == 0
     matches = int(out_count.cpu().sum())
+    image = None
     if w.dense:
-        pairs_per_step = 2 * N1 * N2
+        # The backward pass runs on the image of NN12 only (the rows that can
+        # be in a mutual pair): count them for the useful-work figure.
+        idx12, _ = fnn.fastnn_nn(d1, d2)
+        image = int(torch.unique(idx12[(idx12 >= 0) & (idx12 < N2)]).numel())
+        pairs_per_step = N1 * N2 + image * N1
     else:
         pairs_per_step = int(out_front.cpu().sum()) * (N1 + N2)
     macs_per_step = pairs_per_step * d
@@ -487,12 +494,14 @@ def run_ours(args, rank, world, local):
         bytes_in = (N1 + N2) * d * esize * B + ((N1 + N2) * 4 * B if masked else 0)
         bytes_out = int(hp_count.numel() * 4 + hp_pairs.numel() * 4 + hp_score.numel() * 4)
         if l2:
-            kname = ("nn_l2_kernel (FP32 FFMA2 nearest point, one launch per direction)"
+            kname = ("nn_l2_kernel (FP32 FMA nearest point: forward pass over every image-1 "
+                     "point, backward pass over the image of the forward matches)"
                      if w.dense else
-                     "reciprocal_l2_kernel (persistent: seeds, FP32 FFMA2 forward and backward "
+                     "reciprocal_l2_kernel (persistent: seeds, FP32 FMA forward and backward "
                      "passes, per-pair compaction)")
         else:
-            kname = ("nn_tc_kernel (tcgen05 argmax-GEMM, one launch per direction)" if w.dense else
+            kname = ("nn_tc_kernel (tcgen05 argmax-GEMM: forward pass over every image-1 row, "
+                     "backward pass over the image of the forward matches)" if w.dense else
                      "reciprocal_kernel (persistent: seeds, tcgen05 forward and backward passes, "
                      "per-pair compaction)")
         if l2:
@@ -500,10 +509,14 @@ def run_ours(args, rank, world, local):
                            "(clocks.max.sm)")
             ops = (f"3 FMA = 6 flop per (query, point) pair: {pairs_per_step:.4g} pairs "
                    f"per step")
+            if image is not None:
+                ops += f" ({N1} x {N2} forward + {image} x {N1} backward)"
         else:
             peak_source = (f"{src}: bf16_tflops {bf16_peak}" +
                            (" x 2 (int8 = 2 x bf16, nominal ratio)" if i8 else ""))
             ops = f"2 x useful MACs (d = {d}) per step: {macs_per_step:.4g} MAC"
+            if image is not None:
+                ops += f" ({N1} x {N2} forward + {image} x {N1} backward)"
         line = {
             "metric": metric_for(w.name), "value": value, "unit": UNIT, "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": total_ms / K,

@@ -150,6 +150,8 @@ int fastnn_reciprocal(const void *desc1, int H1, int W1, const void *desc2,
  *   out_pairs [capacity][2] int32 and out_score [capacity] (or NULL);
  *   *out_count (device int32) = number of pairs. capacity must be
  *   >= min(n1, n2), else FASTNN_ERR_CAPACITY.
+ *   Work: NN12 for every row of desc1, then NN21 only for the rows of desc2
+ *   that are some row's NN12 (no other row can be in a mutual pair).
  */
 int fastnn_mutual_dense(const void *desc1, int64_t n1, const void *desc2,
                         int64_t n2, int d, int dtype, int32_t *out_pairs,

@@ -105,6 +105,10 @@ struct MutLayout {
   uint64_t* k12;
   uint64_t* k21;
   int32_t* blocks;
+  int32_t* pos21;    // [n2] slot of image-2 row j in the backward list, or -1
+  int32_t* list21;   // [n2] image-2 rows of the backward pass (the image of NN12)
+  int32_t* cnt21;    // [1] their number
+  int32_t* blocks2;  // image-list scan scratch
 };
 MutLayout carve_mut(Carver& c, int64_t n1, int64_t n2, int d, int dtype) {
   MutLayout L;
@@ -115,6 +119,10 @@ MutLayout carve_mut(Carver& c, int64_t n1, int64_t n2, int d, int dtype) {
   L.k12 = c.take<uint64_t>(static_cast<size_t>(n1));
   L.k21 = c.take<uint64_t>(static_cast<size_t>(n2));
   L.blocks = c.take<int32_t>(static_cast<size_t>(mutual_blocks(n1)));
+  L.pos21 = c.take<int32_t>(static_cast<size_t>(n2));
+  L.list21 = c.take<int32_t>(static_cast<size_t>(n2));
+  L.cnt21 = c.take<int32_t>(1);
+  L.blocks2 = c.take<int32_t>(static_cast<size_t>(mutual_blocks(n2)));
   return L;
 }
 
@@ -391,6 +399,7 @@ int mutual_dense_impl(const void* desc1, const float* conf1, int64_t n1, const v
   FASTNN_CUDA_TRY(cudaMemsetAsync(L.status, 0, kStatusBytes, st));
   FASTNN_CUDA_TRY(cudaMemsetAsync(L.k12, 0, static_cast<size_t>(n1) * 8, st));
   FASTNN_CUDA_TRY(cudaMemsetAsync(L.k21, 0, static_cast<size_t>(n2) * 8, st));
+  FASTNN_CUDA_TRY(cudaMemsetAsync(L.pos21, 0xFF, static_cast<size_t>(n2) * 4, st));
   MaskLayout M{};
   if (masked) {
     M = carve_mask(c, n1, n2, 1, false);
@@ -426,11 +435,17 @@ int mutual_dense_impl(const void* desc1, const float* conf1, int64_t n1, const v
     FASTNN_TRY(launch_nn_l2(a, st));
   else
     FASTNN_TRY(launch_nn_tc(a, dtype, n2 + kPadRows, st));
+  // A mutual pair (i, j) has j = NN12(i): the backward pass needs only the
+  // rows in the image of NN12, listed in ascending order; its keys are
+  // indexed by list slot.
+  FASTNN_TRY(launch_image_list(L.k12, n1, n2, L.pos21, L.list21, L.cnt21, L.blocks2, st));
   NNArgs r{};
   r.q_rows = L.d2rep;
   r.q_rows_per_pair = n2;
   r.q_cap = n2;
   r.nq_static = n2;
+  r.q_index = L.list21;
+  r.q_count = L.cnt21;
   r.db_rows = L.d1rep;
   r.ndb = n1;
   r.out_key = L.k21;
@@ -440,10 +455,7 @@ int mutual_dense_impl(const void* desc1, const float* conf1, int64_t n1, const v
   r.q_absmax = L.status + 2;
   r.db_absmax = L.status + 1;
   r.wait_ns = g_wait_ns.load();
-  if (masked) {
-    r.q_count = M.cnt2;
-    r.ndb_dev = M.cnt1;
-  }
+  if (masked) r.ndb_dev = M.cnt1;
   if (dtype == FASTNN_F32_L2)
     FASTNN_TRY(launch_nn_l2(r, st));
   else
@@ -456,6 +468,7 @@ int mutual_dense_impl(const void* desc1, const float* conf1, int64_t n1, const v
   m.n2 = n2;
   m.map1 = M.c2p1;
   m.map2 = M.c2p2;
+  m.pos21 = L.pos21;
   return launch_mutual(m, L.blocks, dtype, out_pairs, out_score, capacity, out_count, st);
 }
 

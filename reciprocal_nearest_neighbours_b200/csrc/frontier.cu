@@ -74,7 +74,8 @@ __device__ __forceinline__ bool mutual_flag(const MutualSrc& m, int64_t i, uint3
   if (i >= m.n1) return false;
   j = m.k12 ? key_index(m.k12[i]) : static_cast<uint32_t>(m.nn12[i]);
   if (j >= static_cast<uint64_t>(m.n2)) return false;
-  const uint32_t back = m.k21 ? key_index(m.k21[j]) : static_cast<uint32_t>(m.nn21[j]);
+  const uint32_t back = m.k21 ? key_index(m.k21[m.pos21 ? m.pos21[j] : j])
+                              : static_cast<uint32_t>(m.nn21[j]);
   return back == static_cast<uint32_t>(m.i0 + i);
 }
 
@@ -160,6 +161,41 @@ __global__ void __launch_bounds__(1024) mutual_emit_kernel(MutualSrc m,
         }
       }
     }
+  }
+}
+
+// ------------------------------------------------- image of the matching ---
+// Rows of image 2 that are some image-1 row's forward match: only they can
+// be in a mutual pair, so the backward pass runs on them alone.
+__global__ void image_mark_kernel(const uint64_t* __restrict__ k12, int64_t n1, int64_t n2,
+                                  int32_t* __restrict__ pos) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n1;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint32_t j = key_index(k12[i]);
+    if (j < static_cast<uint64_t>(n2)) pos[j] = 0;
+  }
+}
+
+__global__ void __launch_bounds__(1024) image_count_kernel(const int32_t* __restrict__ pos,
+                                                           int64_t n2,
+                                                           int32_t* __restrict__ block_cnt) {
+  __shared__ int sm[64];
+  const int64_t j = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  const Scan2 sc = block_scan2(j < n2 && pos[j] >= 0, false, sm);
+  if (threadIdx.x == 0) block_cnt[blockIdx.x] = sc.tot0;
+}
+
+__global__ void __launch_bounds__(1024) image_emit_kernel(int32_t* __restrict__ pos, int64_t n2,
+                                                          const int32_t* __restrict__ block_off,
+                                                          int32_t* __restrict__ list) {
+  __shared__ int sm[64];
+  const int64_t j = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  const bool f = j < n2 && pos[j] >= 0;
+  const Scan2 sc = block_scan2(f, false, sm);
+  if (f) {
+    const int32_t slot = block_off[blockIdx.x] + sc.ex0;
+    list[slot] = static_cast<int32_t>(j);
+    pos[j] = slot;
   }
 }
 
@@ -404,6 +440,17 @@ int launch_mutual(const MutualSrc& m, int32_t* block_scratch, int dtype, int32_t
   else
     mutual_emit_kernel<FASTNN_BF16><<<nb, 1024, 0, st>>>(m, block_scratch, out_pairs, out_score,
                                                          cap);
+  FASTNN_CUDA_TRY(cudaGetLastError());
+  return FASTNN_OK;
+}
+
+int launch_image_list(const uint64_t* k12, int64_t n1, int64_t n2, int32_t* pos, int32_t* list,
+                      int32_t* count, int32_t* block_scratch, cudaStream_t st) {
+  const int nb = mutual_blocks(n2);
+  image_mark_kernel<<<grid_for(n1, 256), 256, 0, st>>>(k12, n1, n2, pos);
+  image_count_kernel<<<nb, 1024, 0, st>>>(pos, n2, block_scratch);
+  mutual_scan_kernel<<<1, 1024, 0, st>>>(block_scratch, nb, count);
+  image_emit_kernel<<<nb, 1024, 0, st>>>(pos, n2, block_scratch, list);
   FASTNN_CUDA_TRY(cudaGetLastError());
   return FASTNN_OK;
 }

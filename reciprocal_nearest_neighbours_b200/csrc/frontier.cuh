@@ -85,12 +85,19 @@ struct MutualSrc {
   const void* score12;
   const int32_t* map1;  // optional: pixel of compacted image-1 row i (masked maps)
   const int32_t* map2;  // optional: pixel of compacted image-2 row j
+  const int32_t* pos21; // optional: slot of row j in k21 when the backward pass ran on a list
   int64_t n1;  // local image-1 rows
   int64_t n2;  // image-2 rows
   int64_t i0;  // global index of local row 0
 };
 
 int mutual_blocks(int64_t n1);
+// The image of NN12 (the rows j that are some row's forward match) as an
+// ascending list: on entry pos[j] < 0 for every j; on exit list[0..*count)
+// holds the matched rows and pos[j] their slot (-1 for the others).
+// block_scratch holds mutual_blocks(n2) ints.
+int launch_image_list(const uint64_t* k12, int64_t n1, int64_t n2, int32_t* pos, int32_t* list,
+                      int32_t* count, int32_t* block_scratch, cudaStream_t st);
 int launch_mutual(const MutualSrc& m, int32_t* block_scratch, int dtype, int32_t* out_pairs,
                   void* out_score, int64_t cap, int32_t* out_count, cudaStream_t st);
 // Keys -> (index, score); pointmap scores are the squared distances the keys
