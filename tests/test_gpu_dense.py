@@ -108,3 +108,29 @@ def test_dense_512x384_full_size_sampled():
     fp, fs, fc, _ = fastnn_reciprocal(to_dev(m.desc1), to_dev(m.desc2), 8, 10)
     fast, _ = gpu_pairs(fp, fs, fc)
     assert set(map(tuple, fast.tolist())) <= set(map(tuple, p.tolist()))
+
+
+def test_backward_pass_on_a_one_row_image():
+    """Every forward match is the same dominant row j*: the backward pass runs
+    on a one-row list, and the only mutual pair is (NN21(j*), j*)."""
+    rng = np.random.default_rng(77)
+    D1 = rng.integers(1, 9, size=(3000, 24)).astype(np.int8)
+    D2 = rng.integers(-8, 9, size=(2000, 24)).astype(np.int8)
+    D2[1234] = 127
+    p = check_dense_int8(D1, D2)
+    assert len(p) == 1 and int(p[0, 1]) == 1234
+
+
+def test_backward_pass_on_a_two_row_image_with_ties():
+    """Two equal dominant rows: every forward match is the lower one (lowest
+    index wins), so the image is that row alone; ties in the backward pass
+    keep the lowest image-1 index."""
+    rng = np.random.default_rng(78)
+    D1 = rng.integers(1, 3, size=(700, 8)).astype(np.int8)
+    D1[5] = 2
+    D1[9] = 2
+    D2 = rng.integers(-2, 3, size=(900, 8)).astype(np.int8)
+    D2[300] = 100
+    D2[600] = 100
+    p = check_dense_int8(D1, D2)
+    assert p.tolist() == [[5, 300]]

@@ -184,3 +184,17 @@ def test_masked_dense_bf16_within_tolerance():
     got = set(map(tuple, p.tolist()))
     exp = set(map(tuple, ref.pairs.tolist()))
     assert len(got ^ exp) <= 0.05 * max(1, len(exp))
+
+
+@pytest.mark.parametrize("keep1,keep2", [(False, True), (True, False), (False, False)])
+def test_masked_dense_with_an_empty_side(keep1, keep2):
+    """No kept pixel on one side: the forward pass has no query or no database
+    row, the image of NN12 is empty, and no pair comes out."""
+    rng = np.random.default_rng(79)
+    D1 = rng.integers(-4, 5, size=(1500, 24)).astype(np.int8)
+    D2 = rng.integers(-4, 5, size=(1300, 24)).astype(np.int8)
+    c1 = np.full(1500, 1.0 if keep1 else 0.0, np.float32)
+    c2 = np.full(1300, 1.0 if keep2 else 0.0, np.float32)
+    pairs, score, count = fastnn_mutual_dense_masked(dev(D1), dev(D2), conf1=dev(c1),
+                                                     conf2=dev(c2), threshold=0.5)
+    assert int(count[0]) == 0
