@@ -75,6 +75,8 @@ struct RecLayout {
   uint8_t* d2rep;
   int32_t* F[2];
   uint32_t* Bd[2];
+  float4* box1;  // pointmaps: chunk boxes of image 1 (database of the backward pass)
+  float4* box2;  // pointmaps: chunk boxes of image 2
   uint64_t* fwd;
   uint64_t* bwd;
   uint32_t* claim;
@@ -90,6 +92,11 @@ RecLayout carve_rec(Carver& c, int64_t N1, int64_t N2, int d, int dtype, int bat
   L.F[1] = c.take<int32_t>(static_cast<size_t>(batch) * S);
   L.Bd[0] = c.take<uint32_t>(static_cast<size_t>(batch) * S);
   L.Bd[1] = c.take<uint32_t>(static_cast<size_t>(batch) * S);
+  L.box1 = L.box2 = nullptr;
+  if (dtype == FASTNN_F32_L2) {
+    L.box1 = c.take<float4>(static_cast<size_t>(batch) * 2 * ((N1 + kL2Chunk - 1) / kL2Chunk));
+    L.box2 = c.take<float4>(static_cast<size_t>(batch) * 2 * ((N2 + kL2Chunk - 1) / kL2Chunk));
+  }
   L.fwd = c.take<uint64_t>(static_cast<size_t>(batch) * S);
   L.bwd = c.take<uint64_t>(static_cast<size_t>(batch) * S);
   L.claim = c.take<uint32_t>(static_cast<size_t>(batch) * N1);
@@ -105,10 +112,14 @@ struct MutLayout {
   uint64_t* k12;
   uint64_t* k21;
   int32_t* blocks;
-  int32_t* pos21;    // [n2] slot of image-2 row j in the backward list, or -1
+  int32_t* pos21;    // [n2] slot of image-2 row j in the backward list (matched rows only)
+  uint32_t* first21; // [n2] first image-1 row matched to j
   int32_t* list21;   // [n2] image-2 rows of the backward pass (the image of NN12)
   int32_t* cnt21;    // [1] their number
   int32_t* blocks2;  // image-list scan scratch
+  uint32_t* best21;  // [n2] best forward score bits among the rows matched to j
+  uint32_t* bnd21;   // [n2] the same, per list slot: the backward pass's score bounds
+  float4* box1;      // pointmaps: chunk boxes of image 1 (database of the backward pass)
 };
 MutLayout carve_mut(Carver& c, int64_t n1, int64_t n2, int d, int dtype) {
   MutLayout L;
@@ -122,7 +133,13 @@ MutLayout carve_mut(Carver& c, int64_t n1, int64_t n2, int d, int dtype) {
   L.pos21 = c.take<int32_t>(static_cast<size_t>(n2));
   L.list21 = c.take<int32_t>(static_cast<size_t>(n2));
   L.cnt21 = c.take<int32_t>(1);
-  L.blocks2 = c.take<int32_t>(static_cast<size_t>(mutual_blocks(n2)));
+  L.blocks2 = c.take<int32_t>(static_cast<size_t>(mutual_blocks(n1)));
+  L.first21 = c.take<uint32_t>(static_cast<size_t>(n2));
+  L.best21 = c.take<uint32_t>(static_cast<size_t>(n2));
+  L.bnd21 = c.take<uint32_t>(static_cast<size_t>(n2));
+  L.box1 = dtype == FASTNN_F32_L2
+               ? c.take<float4>(static_cast<size_t>(2 * ((n1 + kL2Chunk - 1) / kL2Chunk)))
+               : nullptr;
   return L;
 }
 
@@ -309,6 +326,8 @@ int reciprocal_impl(const void* desc1, const float* conf1, int H1, int W1, const
   r.bwd.out_key = L.bwd;
   r.bwd.q_absmax = L.status + 2;
   r.bwd.db_absmax = L.status + 1;
+  r.fwd.db_box = L.box2;
+  r.bwd.db_box = L.box1;
   if (masked) {
     r.fwd.ndb_dev = M.cnt2;
     r.bwd.ndb_dev = M.cnt1;
@@ -399,7 +418,8 @@ int mutual_dense_impl(const void* desc1, const float* conf1, int64_t n1, const v
   FASTNN_CUDA_TRY(cudaMemsetAsync(L.status, 0, kStatusBytes, st));
   FASTNN_CUDA_TRY(cudaMemsetAsync(L.k12, 0, static_cast<size_t>(n1) * 8, st));
   FASTNN_CUDA_TRY(cudaMemsetAsync(L.k21, 0, static_cast<size_t>(n2) * 8, st));
-  FASTNN_CUDA_TRY(cudaMemsetAsync(L.pos21, 0xFF, static_cast<size_t>(n2) * 4, st));
+  FASTNN_CUDA_TRY(cudaMemsetAsync(L.first21, 0xFF, static_cast<size_t>(n2) * 4, st));
+  FASTNN_CUDA_TRY(cudaMemsetAsync(L.best21, 0, static_cast<size_t>(n2) * 4, st));
   MaskLayout M{};
   if (masked) {
     M = carve_mask(c, n1, n2, 1, false);
@@ -436,9 +456,10 @@ int mutual_dense_impl(const void* desc1, const float* conf1, int64_t n1, const v
   else
     FASTNN_TRY(launch_nn_tc(a, dtype, n2 + kPadRows, st));
   // A mutual pair (i, j) has j = NN12(i): the backward pass needs only the
-  // rows in the image of NN12, listed in ascending order; its keys are
-  // indexed by list slot.
-  FASTNN_TRY(launch_image_list(L.k12, n1, n2, L.pos21, L.list21, L.cnt21, L.blocks2, st));
+  // rows in the image of NN12, listed in the order of the first image-1 row
+  // matched to each; its keys are indexed by list slot.
+  FASTNN_TRY(launch_image_list(L.k12, n1, n2, L.first21, L.best21, L.pos21, L.list21, L.bnd21,
+                               L.cnt21, L.blocks2, st));
   NNArgs r{};
   r.q_rows = L.d2rep;
   r.q_rows_per_pair = n2;
@@ -446,6 +467,12 @@ int mutual_dense_impl(const void* desc1, const float* conf1, int64_t n1, const v
   r.nq_static = n2;
   r.q_index = L.list21;
   r.q_count = L.cnt21;
+  r.q_bound = L.bnd21;
+  if (dtype == FASTNN_F32_L2) {
+    FASTNN_TRY(launch_chunk_boxes(reinterpret_cast<const float4*>(L.d1rep), n1, 1,
+                                  masked ? M.cnt1 : nullptr, L.box1, st));
+    r.db_box = L.box1;
+  }
   r.db_rows = L.d1rep;
   r.ndb = n1;
   r.out_key = L.k21;

@@ -73,6 +73,10 @@ __host__ __device__ constexpr int row_bytes(int dtype, int d) {
 //     otherwise          : k
 //   rows live in q_rows + (b * q_rows_per_pair + row) * row_bytes.
 //   Active slots of pair b: q_count ? q_count[b] : nq_static.
+// Database rows per chunk of the pointmap kernels (a chunk's points also
+// have a bounding box, for skipping chunks a query cannot be near).
+constexpr int kL2Chunk = 1024;
+
 struct NNArgs {
   const uint8_t* q_rows;
   int64_t q_rows_per_pair;
@@ -92,6 +96,10 @@ struct NNArgs {
   const int* q_absmax;     // int8: max |element| of the query map (or nullptr)
   const int* db_absmax;    // int8: max |element| of the database map (or nullptr)
   uint64_t wait_ns;        // limit of the pipeline's bounded waits (0: kTimeoutNs)
+  const uint32_t* q_bound; // optional [batch][q_cap]: ordered bits of a score each query is
+                           // known to reach (0: none), for the standalone passes
+  const float4* db_box;    // pointmaps, optional: [batch][ceil(ndb / kL2Chunk)][2] box (lo, hi)
+                           // of each database chunk's points
 };
 
 // The parts of a pass's query description that change from round to round

@@ -164,37 +164,109 @@ __global__ void __launch_bounds__(1024) mutual_emit_kernel(MutualSrc m,
   }
 }
 
-// ------------------------------------------------- image of the matching ---
-// Rows of image 2 that are some image-1 row's forward match: only they can
-// be in a mutual pair, so the backward pass runs on them alone.
-__global__ void image_mark_kernel(const uint64_t* __restrict__ k12, int64_t n1, int64_t n2,
-                                  int32_t* __restrict__ pos) {
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n1;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const uint32_t j = key_index(k12[i]);
-    if (j < static_cast<uint64_t>(n2)) pos[j] = 0;
+// ------------------------------------------------------- chunk boxes ---
+__global__ void __launch_bounds__(256) chunk_box_kernel(const float4* __restrict__ rows,
+                                                        int64_t N, int nchunk,
+                                                        const int32_t* __restrict__ count,
+                                                        float4* __restrict__ box) {
+  const int b = blockIdx.x / nchunk, c = blockIdx.x % nchunk;
+  const int64_t n = count ? min(static_cast<int64_t>(count[b]), N) : N;
+  const int64_t r0 = static_cast<int64_t>(c) * kL2Chunk;
+  const int64_t r1 = min(r0 + kL2Chunk, n);
+  float lo[3] = {INFINITY, INFINITY, INFINITY}, hi[3] = {-INFINITY, -INFINITY, -INFINITY};
+  for (int64_t r = r0 + threadIdx.x; r < r1; r += blockDim.x) {
+    const float4 p = __ldg(rows + b * N + r);
+    lo[0] = fminf(lo[0], p.x);
+    lo[1] = fminf(lo[1], p.y);
+    lo[2] = fminf(lo[2], p.z);
+    hi[0] = fmaxf(hi[0], p.x);
+    hi[1] = fmaxf(hi[1], p.y);
+    hi[2] = fmaxf(hi[2], p.z);
+  }
+  __shared__ float sm[6][8];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      lo[k] = fminf(lo[k], __shfl_xor_sync(0xffffffffu, lo[k], o));
+      hi[k] = fmaxf(hi[k], __shfl_xor_sync(0xffffffffu, hi[k], o));
+    }
+    if (lane == 0) {
+      sm[k][warp] = lo[k];
+      sm[3 + k][warp] = hi[k];
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float l[3], h[3];
+    for (int k = 0; k < 3; ++k) {
+      l[k] = sm[k][0];
+      h[k] = sm[3 + k][0];
+      for (int w = 1; w < static_cast<int>(blockDim.x >> 5); ++w) {
+        l[k] = fminf(l[k], sm[k][w]);
+        h[k] = fmaxf(h[k], sm[3 + k][w]);
+      }
+    }
+    box[2 * static_cast<int64_t>(blockIdx.x)] = make_float4(l[0], l[1], l[2], 0.f);
+    box[2 * static_cast<int64_t>(blockIdx.x) + 1] = make_float4(h[0], h[1], h[2], 0.f);
   }
 }
 
-__global__ void __launch_bounds__(1024) image_count_kernel(const int32_t* __restrict__ pos,
-                                                           int64_t n2,
+// ------------------------------------------------- image of the matching ---
+// Rows of image 2 that are some image-1 row's forward match: only they can
+// be in a mutual pair, so the backward pass runs on them alone.
+// The best forward score among the rows matched to j is a score NN21(j)
+// reaches (the same dot product, or distance, with the roles swapped).
+__global__ void image_mark_kernel(const uint64_t* __restrict__ k12, int64_t n1, int64_t n2,
+                                  uint32_t* __restrict__ first, uint32_t* __restrict__ best) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n1;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint64_t key = k12[i];
+    const uint32_t j = key_index(key);
+    if (j < static_cast<uint64_t>(n2)) {
+      atomicMin(first + j, static_cast<uint32_t>(i));
+      atomicMax(best + j, key_score_bits(key));
+    }
+  }
+}
+
+// Row i of image 1 introduces j = NN12(i) when it is the first row matched to j.
+__device__ __forceinline__ bool image_first(const uint64_t* k12, const uint32_t* first, int64_t n1,
+                                            int64_t n2, int64_t i, uint32_t& j) {
+  if (i >= n1) return false;
+  j = key_index(k12[i]);
+  return j < static_cast<uint64_t>(n2) && first[j] == static_cast<uint32_t>(i);
+}
+
+__global__ void __launch_bounds__(1024) image_count_kernel(const uint64_t* __restrict__ k12,
+                                                           const uint32_t* __restrict__ first,
+                                                           int64_t n1, int64_t n2,
                                                            int32_t* __restrict__ block_cnt) {
   __shared__ int sm[64];
-  const int64_t j = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
-  const Scan2 sc = block_scan2(j < n2 && pos[j] >= 0, false, sm);
+  const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  uint32_t j;
+  const Scan2 sc = block_scan2(image_first(k12, first, n1, n2, i, j), false, sm);
   if (threadIdx.x == 0) block_cnt[blockIdx.x] = sc.tot0;
 }
 
-__global__ void __launch_bounds__(1024) image_emit_kernel(int32_t* __restrict__ pos, int64_t n2,
+__global__ void __launch_bounds__(1024) image_emit_kernel(const uint64_t* __restrict__ k12,
+                                                          const uint32_t* __restrict__ first,
+                                                          const uint32_t* __restrict__ best,
+                                                          int64_t n1, int64_t n2,
                                                           const int32_t* __restrict__ block_off,
-                                                          int32_t* __restrict__ list) {
+                                                          int32_t* __restrict__ pos,
+                                                          int32_t* __restrict__ list,
+                                                          uint32_t* __restrict__ list_bound) {
   __shared__ int sm[64];
-  const int64_t j = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
-  const bool f = j < n2 && pos[j] >= 0;
+  const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  uint32_t j = 0;
+  const bool f = image_first(k12, first, n1, n2, i, j);
   const Scan2 sc = block_scan2(f, false, sm);
   if (f) {
     const int32_t slot = block_off[blockIdx.x] + sc.ex0;
     list[slot] = static_cast<int32_t>(j);
+    list_bound[slot] = best[j];
     pos[j] = slot;
   }
 }
@@ -444,13 +516,24 @@ int launch_mutual(const MutualSrc& m, int32_t* block_scratch, int dtype, int32_t
   return FASTNN_OK;
 }
 
-int launch_image_list(const uint64_t* k12, int64_t n1, int64_t n2, int32_t* pos, int32_t* list,
+int launch_chunk_boxes(const float4* rows, int64_t N, int batch, const int32_t* count,
+                       float4* box, cudaStream_t st) {
+  const int nchunk = static_cast<int>((N + kL2Chunk - 1) / kL2Chunk);
+  if (batch < 1 || nchunk < 1) return FASTNN_OK;
+  chunk_box_kernel<<<batch * nchunk, 256, 0, st>>>(rows, N, nchunk, count, box);
+  FASTNN_CUDA_TRY(cudaGetLastError());
+  return FASTNN_OK;
+}
+
+int launch_image_list(const uint64_t* k12, int64_t n1, int64_t n2, uint32_t* first,
+                      uint32_t* best, int32_t* pos, int32_t* list, uint32_t* list_bound,
                       int32_t* count, int32_t* block_scratch, cudaStream_t st) {
-  const int nb = mutual_blocks(n2);
-  image_mark_kernel<<<grid_for(n1, 256), 256, 0, st>>>(k12, n1, n2, pos);
-  image_count_kernel<<<nb, 1024, 0, st>>>(pos, n2, block_scratch);
+  const int nb = mutual_blocks(n1);
+  image_mark_kernel<<<grid_for(n1, 256), 256, 0, st>>>(k12, n1, n2, first, best);
+  image_count_kernel<<<nb, 1024, 0, st>>>(k12, first, n1, n2, block_scratch);
   mutual_scan_kernel<<<1, 1024, 0, st>>>(block_scratch, nb, count);
-  image_emit_kernel<<<nb, 1024, 0, st>>>(pos, n2, block_scratch, list);
+  image_emit_kernel<<<nb, 1024, 0, st>>>(k12, first, best, n1, n2, block_scratch, pos, list,
+                                         list_bound);
   FASTNN_CUDA_TRY(cudaGetLastError());
   return FASTNN_OK;
 }

@@ -92,11 +92,22 @@ struct MutualSrc {
 };
 
 int mutual_blocks(int64_t n1);
-// The image of NN12 (the rows j that are some row's forward match) as an
-// ascending list: on entry pos[j] < 0 for every j; on exit list[0..*count)
-// holds the matched rows and pos[j] their slot (-1 for the others).
-// block_scratch holds mutual_blocks(n2) ints.
-int launch_image_list(const uint64_t* k12, int64_t n1, int64_t n2, int32_t* pos, int32_t* list,
+// Bounding box (lo, hi; xyz) of every kL2Chunk-row chunk of each pair's
+// repacked pointmap rows [batch][N]: box[(b * nchunk + c) * 2 + {0, 1}],
+// nchunk = ceil(N / kL2Chunk). With `count`, pair b has count[b] rows;
+// chunks past them get an empty box (lo = +inf, hi = -inf).
+int launch_chunk_boxes(const float4* rows, int64_t N, int batch, const int32_t* count,
+                       float4* box, cudaStream_t st);
+// The image of NN12 (the rows j that are some row's forward match) as a
+// list in the order of the first image-1 row matched to each j (queries next
+// to each other in the list then lie near each other, whatever the order of
+// image 2): on entry first[j] = 0xFFFFFFFF and best[j] = 0 for every j; on
+// exit list[0..*count) holds the matched rows, pos[j] their slot (only for
+// matched j) and list_bound[slot] the best forward score bits among the rows
+// matched to j (a score NN21(j) reaches). block_scratch holds
+// mutual_blocks(n1) ints.
+int launch_image_list(const uint64_t* k12, int64_t n1, int64_t n2, uint32_t* first,
+                      uint32_t* best, int32_t* pos, int32_t* list, uint32_t* list_bound,
                       int32_t* count, int32_t* block_scratch, cudaStream_t st);
 int launch_mutual(const MutualSrc& m, int32_t* block_scratch, int dtype, int32_t* out_pairs,
                   void* out_score, int64_t cap, int32_t* out_count, cudaStream_t st);

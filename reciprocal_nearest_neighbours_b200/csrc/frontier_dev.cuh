@@ -253,9 +253,11 @@ __device__ void compact_pair(const CompactArgs& c, const FrontierBufs& fb, int b
 // nearest-neighbour pass over the whole grid (dir 0: r.fwd, 1: r.bwd) and
 // ends with a CTA barrier. `cta_abort` is the CTA's own abort flag (shared
 // memory); `flag`, `more` and `scan` (66 ints) are shared scratch.
-template <int DT, class NNPass>
-__device__ void fast_rounds(const RecArgs& r, NNPass&& nn, volatile int* cta_abort, int* flag,
-                            int* more, int* scan) {
+// `prologue()` runs in every CTA beside the clearing of the per-call state,
+// before the first grid barrier.
+template <int DT, class NNPass, class Prologue>
+__device__ void fast_rounds(const RecArgs& r, NNPass&& nn, Prologue&& prologue,
+                            volatile int* cta_abort, int* flag, int* more, int* scan) {
   uint32_t target = 0;
   const int batch = r.batch;
   const int64_t S = r.S;
@@ -278,6 +280,7 @@ __device__ void fast_rounds(const RecArgs& r, NNPass&& nn, volatile int* cta_abo
   }
   if (r.cmp.out_frontier)
     for (int64_t i = gtid; i < batch * r.max_iter; i += gsize) r.cmp.out_frontier[i] = 0;
+  prologue();
   bool ok = sync();
   if (ok) {
     // Seeds: the round-1 frontier of every pair (the grid, or the kept grid

@@ -65,7 +65,7 @@ constexpr int kWarps = 16;
 constexpr int kThreads = 32 * kWarps;
 constexpr int kQW = 8;              // queries per warp, held by every lane
 constexpr int kQT = kWarps * kQW;   // queries per tile
-constexpr int kDC = 1024;           // database rows per chunk (16 KB)
+constexpr int kDC = kL2Chunk;       // database rows per chunk (16 KB)
 constexpr int kSteps = kDC / 64;    // 64-row steps per chunk: two rows per lane per step
 constexpr int kNS = 4;              // chunk ring depth
 constexpr int kMaxBatchL2 = 1024;
@@ -78,6 +78,8 @@ struct WarpState {
   float smax[kQW];              // largest fp32 score s~ seen in the segment
   float win2[kQW];              // window width 2E
   float floor[kQW];             // lowest window edge the query's bound allows, or -FLT_MAX
+  float4 qlo, qhi;              // box of the warp's queries; qlo.w = largest bound distance
+                                // (+inf if a query has none)
 };
 
 struct __align__(16) L2Smem {
@@ -287,6 +289,27 @@ __device__ __forceinline__ void load_queries(const NNArgs& a, const PhaseQ& q, i
     if (q.bound) bound = __ldcg(q.bound + (b * a.q_cap + k) * q.bstride);
   }
   float floor = -FLT_MAX;
+  // Box of the warp's queries and the largest of their bound distances
+  // (+inf if one has none): a chunk whose box is farther from this box than
+  // that holds none of their answers.
+  const bool valid = lane < kQW && k < cnt;
+  float lx = valid ? v.x : INFINITY, ly = valid ? v.y : INFINITY, lz = valid ? v.z : INFINITY;
+  float hx = valid ? v.x : -INFINITY, hy = valid ? v.y : -INFINITY, hz = valid ? v.z : -INFINITY;
+  float bd = valid ? (bound != 0u ? -unord_f32(bound) : INFINITY) : -INFINITY;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lx = fminf(lx, __shfl_xor_sync(kFull, lx, o));
+    ly = fminf(ly, __shfl_xor_sync(kFull, ly, o));
+    lz = fminf(lz, __shfl_xor_sync(kFull, lz, o));
+    hx = fmaxf(hx, __shfl_xor_sync(kFull, hx, o));
+    hy = fmaxf(hy, __shfl_xor_sync(kFull, hy, o));
+    hz = fmaxf(hz, __shfl_xor_sync(kFull, hz, o));
+    bd = fmaxf(bd, __shfl_xor_sync(kFull, bd, o));
+  }
+  if (lane == 0) {
+    W.qlo = make_float4(lx, ly, lz, bd);
+    W.qhi = make_float4(hx, hy, hz, 0.f);
+  }
   if (lane < kQW) {
     // 2E = 16 u (|a| + R)^2; the norms come from fp32 sums (relative error
     // below 3 u), inflated by 2^-20 to stay an upper bound.
@@ -428,9 +451,28 @@ __device__ void l2_phase(const NNArgs& a, const PhaseQ q, L2Smem& s) {
     const int cnt = s.cnt[w.b];
     const bool active = k0 < cnt;  // warp-uniform
     if (seg_start) load_queries(a, q, w.b, k0, cnt, lane, max_p2, W, Q, Wn);
+    float4 blo = make_float4(0.f, 0.f, 0.f, 0.f), bhi = blo;
+    if (a.db_box && active) {
+      const float4* bx = a.db_box + 2 * (w.b * ((a.ndb + kDC - 1) / kDC) + w.c);
+      blo = __ldcg(bx);
+      bhi = __ldcg(bx + 1);
+    }
     ok = __all_sync(kFull, l2_wait(s, i, ph[i], a.status));
     ph[i] ^= 1u;
-    if (ok && active) {
+    // Skip the chunk when its box is farther from the queries' box than every
+    // bound: each of its points is then beyond every query's answer. The
+    // box distance loses at most a few ulps in fp32; the 2^-20 margins on
+    // both sides cover that and the rounding of the bounds themselves.
+    bool skip = false;
+    if (a.db_box && active) {
+      const float4 ql = W.qlo, qh = W.qhi;
+      const float dx = fmaxf(fmaxf(blo.x - qh.x, ql.x - bhi.x), 0.f);
+      const float dy = fmaxf(fmaxf(blo.y - qh.y, ql.y - bhi.y), 0.f);
+      const float dz = fmaxf(fmaxf(blo.z - qh.z, ql.z - bhi.z), 0.f);
+      const float d2 = __fmaf_rn(dz, dz, __fmaf_rn(dy, dy, dx * dx));
+      skip = d2 * (1.f - 0x1p-20f) > ql.w * (1.f + 0x1p-20f);
+    }
+    if (ok && active && !skip) {
       const int rows = static_cast<int>(min(static_cast<int64_t>(kDC), s.rows[w.b] - w.c * kDC));
       l2_chunk(s.buf[i], rows, static_cast<uint32_t>(w.c * kDC), Q, Wn, W, lane);
     }
@@ -474,18 +516,66 @@ __device__ void l2_phase(const NNArgs& a, const PhaseQ q, L2Smem& s) {
 __global__ void __launch_bounds__(kThreads, 1) nn_l2_kernel(const __grid_constant__ NNArgs a) {
   L2Smem& s = l2_smem();
   l2_setup(s);
-  l2_phase(a, PhaseQ{a.q_index, a.q_count, nullptr, 0}, s);
+  l2_phase(a, PhaseQ{a.q_index, a.q_count, a.q_bound, 1}, s);
   l2_teardown(s, a.status);
 }
 
 // Fast reciprocal matching of pointmaps: the shared round loop with the
 // passes above.
+// Box (lo, hi) of the points of every database chunk of both maps, one
+// chunk per warp (32 rows per lane), written into the passes' db_box arrays
+// (workspace) before the first grid barrier; the passes read them through L2.
+__device__ void l2_boxes(const RecArgs& r) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t nc1 = (r.bwd.ndb + kDC - 1) / kDC, nc2 = (r.fwd.ndb + kDC - 1) / kDC;
+  const int64_t total = r.batch * (nc1 + nc2);
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * kWarps + warp; t < total;
+       t += static_cast<int64_t>(gridDim.x) * kWarps) {
+    const bool img1 = t < r.batch * nc1;
+    const NNArgs& a = img1 ? r.bwd : r.fwd;  // the pass whose database this map is
+    const int64_t nc = img1 ? nc1 : nc2, tt = img1 ? t : t - r.batch * nc1;
+    const int b = static_cast<int>(tt / nc);
+    const int64_t c = tt % nc;
+    const int64_t n = a.ndb_dev ? min(static_cast<int64_t>(__ldg(a.ndb_dev + b)), a.ndb) : a.ndb;
+    const float4* rows = reinterpret_cast<const float4*>(a.db_rows) + b * a.ndb;
+    float v[6] = {INFINITY, INFINITY, INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 8
+    for (int h = 0; h < kDC / 32; ++h) {
+      const int64_t row = c * kDC + h * 32 + lane;
+      if (row < n) {
+        const float4 p = __ldg(rows + row);
+        v[0] = fminf(v[0], p.x);
+        v[1] = fminf(v[1], p.y);
+        v[2] = fminf(v[2], p.z);
+        v[3] = fmaxf(v[3], p.x);
+        v[4] = fmaxf(v[4], p.y);
+        v[5] = fmaxf(v[5], p.z);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+      for (int k = 0; k < 6; ++k) {
+        const float y = __shfl_xor_sync(kFull, v[k], o);
+        v[k] = k < 3 ? fminf(v[k], y) : fmaxf(v[k], y);
+      }
+    if (lane == 0) {
+      float4* box = const_cast<float4*>(a.db_box) + 2 * (b * nc + c);
+      box[0] = make_float4(v[0], v[1], v[2], 0.f);
+      box[1] = make_float4(v[3], v[4], v[5], 0.f);
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     reciprocal_l2_kernel(const __grid_constant__ RecArgs r) {
   L2Smem& s = l2_smem();
   l2_setup(s);
   auto pass = [&](int dir, const PhaseQ& q) { l2_phase(dir == 0 ? r.fwd : r.bwd, q, s); };
-  fast_rounds<FASTNN_F32_L2>(r, pass, &s.abort_flag, &s.grid_ok, &s.more, s.scan);
+  auto boxes = [&] {
+    if (r.fwd.db_box && r.bwd.db_box) l2_boxes(r);
+  };
+  fast_rounds<FASTNN_F32_L2>(r, pass, boxes, &s.abort_flag, &s.grid_ok, &s.more, s.scan);
   l2_teardown(s, r.status);
 }
 

@@ -800,7 +800,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   pipe_setup(L.ctl);
   const uint32_t tmem = L.ctl->tmem_base;
   PipeState ps;
-  run_phase<DT, RB>(&tmap_db, a, PhaseQ{a.q_index, a.q_count, nullptr, 0}, L, tmem, ps);
+  run_phase<DT, RB>(&tmap_db, a, PhaseQ{a.q_index, a.q_count, a.q_bound, 1}, L, tmem, ps);
   pipe_teardown(L.ctl, tmem, a.status);
 }
 
@@ -830,7 +830,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     else
       run_phase<DT, RB>(&tmap_d1, r.bwd, q, L, tmem, ps);
   };
-  fast_rounds<DT>(r, pass, &ctl->abort_flag, &ctl->grid_ok, &ctl->more, ctl->scan);
+  fast_rounds<DT>(r, pass, [] {}, &ctl->abort_flag, &ctl->grid_ok, &ctl->more, ctl->scan);
   pipe_teardown(ctl, tmem, r.status);
 }
 

@@ -23,7 +23,8 @@ import torch
 
 import oracle
 import synth
-from reciprocal_nearest_neighbours_b200 import fastnn_mutual_dense, fastnn_nn, fastnn_reciprocal
+from reciprocal_nearest_neighbours_b200 import (fastnn_mutual_dense, fastnn_nn, fastnn_reciprocal,
+                                                fastnn_reciprocal_masked)
 from tests._dev import gpu_pairs, require_cuda
 from tests.test_gpu_reciprocal import expected_rounds
 from tests.test_oracle_l2 import load_pointmap_golden
@@ -210,6 +211,28 @@ def test_fast_l2_pair_512x384_full_size():
     p = w.pairs[0]
     symdiff, n = check_fast_l2_certificate(p.desc1, p.desc2, w.subsample, w.max_iter)
     assert n > 1000 and symdiff == 0
+
+
+def test_fast_l2_outlier_free_surfaces_exact():
+    """Smooth surfaces without outliers in either view: both passes skip most
+    database chunks (their boxes are far from the queries' box by more than
+    every bound); the result must still equal the oracle's."""
+    for seed in range(3):
+        m = synth.pointmap_pair(650 + seed, H=96, W=256, outlier_frac=0.0)
+        symdiff, n = check_fast_l2_certificate(m.desc1, m.desc2, 4, 10)
+        assert n > 200 and symdiff == 0
+
+
+def test_fast_l2_outlier_free_surfaces_masked_exact():
+    m = synth.pointmap_pair(660, H=96, W=256, outlier_frac=0.0)
+    c1, c2 = synth.confidence_maps(661, 96, 256, m.gt_src)
+    k1, k2 = oracle.confident(c1, 96 * 256, 2.0), oracle.confident(c2, 96 * 256, 2.0)
+    pairs, score, count, iters = fastnn_reciprocal_masked(
+        dev(m.desc1), dev(m.desc2), 4, 10, conf1=dev(c1), conf2=dev(c2), threshold=2.0)
+    p, s = gpu_pairs(pairs, score, count)
+    ref = oracle.fast_reciprocal_masked(m.desc1, 96, 256, k1, m.desc2, 96, 256, k2, "l2", 4, 10)
+    assert set(map(tuple, p.tolist())) == set(map(tuple, ref.pairs.tolist()))
+    assert len(p) > 100
 
 
 def test_fast_l2_batch_pairs_independent():
