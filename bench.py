@@ -273,6 +273,8 @@ class ClockSampler:
 TRAFFIC = {
     "pair_512x384_d24_i8": (12.716e6, "172ee1fa511b4f34"),
     "pair_512x384_pts3_f32": (6.441e6, "172ee1fa511b4f34"),
+    # Dense: the two launches of one step (forward 14.21 MB + backward 13.59 MB).
+    "dense_512x384_d24_i8": (27.80e6, "172ee1fa511b4f34"),
 }
 KERNEL_SOURCES = ["reciprocal_nearest_neighbours_b200/csrc/nn_tc.cu",
                   "reciprocal_nearest_neighbours_b200/csrc/l2_nn.cu",
@@ -531,7 +533,8 @@ def run_ours(args, rank, world, local):
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": (achieved / peak) if achieved else None,
                 "traffic": traffic_for(w.name),
-                "traffic_unit": "bytes per launch (ncu dram read + write)",
+                "traffic_unit": ("bytes per step: forward + backward launch (ncu dram read + write)"
+                                 if w.dense else "bytes per launch (ncu dram read + write)"),
                 "peak_source": peak_source,
                 "ops": ops,
                 "kernel_ms_per_step": nn_ms / K, "kernel_launches": nn_launches,
