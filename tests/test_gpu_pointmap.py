@@ -223,6 +223,20 @@ def test_fast_l2_outlier_free_surfaces_exact():
         assert n > 200 and symdiff == 0
 
 
+@pytest.mark.parametrize("scale,offset", [(1e4, 1e5), (1e-4, 0.0), (3.0, -2e3)])
+def test_fast_l2_extreme_scales_exact(scale, offset):
+    """Coordinates far from unit scale or far from the origin: the window
+    floor and the chunk-skip test keep their margins relative to the
+    magnitudes involved, so the result still follows the oracle's."""
+    m = synth.pointmap_pair(670, H=64, W=192, outlier_frac=0.1)
+    m1 = (m.desc1.astype(np.float64) * scale + offset).astype(np.float32)
+    m2 = (m.desc2.astype(np.float64) * scale + offset).astype(np.float32)
+    # Any difference from the oracle must sit on an fp32 collision (checked
+    # inside); a margin too narrow would show up as a difference elsewhere.
+    _, n = check_fast_l2_certificate(m1, m2, 4, 10)
+    assert n > 100
+
+
 def test_fast_l2_outlier_free_surfaces_masked_exact():
     m = synth.pointmap_pair(660, H=96, W=256, outlier_frac=0.0)
     c1, c2 = synth.confidence_maps(661, 96, 256, m.gt_src)
