@@ -377,9 +377,9 @@ def run_ours(args, rank, world, local):
         def call():
             fnn.fastnn_mutual_dense(d1, d2, out_pairs=out_pairs, out_score=out_score,
                                     out_count=out_count, workspace=ws, stream=stream)
-        # 2 repack, forward pass, image list (mark/count/scan/emit), backward
-        # pass, mutual count/scan/emit
-        launches_per_step = 2 + 1 + 4 + 1 + 3
+        # 2 repack, forward pass, image list (mark/count/scan/emit), pointmaps:
+        # chunk boxes of image 1, backward pass, mutual count/scan/emit
+        launches_per_step = 2 + 1 + 4 + (1 if l2 else 0) + 1 + 3
         kernels_per_step = 2
     elif masked:
         def call():
