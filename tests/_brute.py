@@ -78,3 +78,46 @@ def walks(seeds, D1, D2, max_iter, nn=nn_by_definition):
             nodes.append(u)
         info.append((nodes, scores, fixed))
     return kept, info
+
+
+def nn_margin_by_definition(q, db, score):
+    """Nearest neighbour with its top-2 margin, from the full score list.
+
+    ``score(q, row)`` returns an exact score (higher is better). Returns
+    (index, best, margin): the lowest index among the maximal scores, that
+    score, and best minus the largest score over every OTHER row (0 on a tie,
+    ``inf`` for a one-row database).
+    """
+    scores = [score(q, row) for row in db]
+    m = max(scores)
+    k = min(i for i, s in enumerate(scores) if s == m)
+    others = [s for i, s in enumerate(scores) if i != k]
+    return k, m, (m - max(others)) if others else float("inf")
+
+
+def walk_gaps(seeds, D1, D2, max_iter, score, backward=True):
+    """The walk-gap record of the fast scheme, read off per-seed walks.
+
+    Each seed's walk u_0 = seed, u_{t+1} = NN21(NN12(u_t)) is followed on its
+    own for at most ``max_iter`` steps. The gap of a walk is the smallest
+    top-2 margin met on it, over the forward step (row u_t against image 2)
+    and the backward step (its match against image 1) of every step taken,
+    the last (fixed-point) step included (``backward=False`` counts the
+    forward steps only, to show which cases the backward margins decide).
+    For each pixel u at which some walk stops at a fixed point, the record
+    is the LARGEST gap over all walks that stop at u: it is small only when
+    every walk to u passes a near-tie. Returns {u: [gap of each walk that
+    stops at u]}; the record is the maximum of each list.
+    """
+    out = {}
+    for s0 in seeds:
+        u, g = s0, float("inf")
+        for _ in range(max_iter):
+            v, _, fm = nn_margin_by_definition(D1[u], D2, score)
+            u2, _, bm = nn_margin_by_definition(D2[v], D1, score)
+            g = min(g, fm, bm) if backward else min(g, fm)
+            if u2 == u:
+                out.setdefault(u, []).append(g)
+                break
+            u = u2
+    return out

@@ -311,6 +311,83 @@ def test_bf16_fast_gap_tracking_on_tiny_pair():
 
 
 # ---------------------------------------------------------------------------
+# the walk-gap record behind the float tolerance rule
+# ---------------------------------------------------------------------------
+
+def _dyadic_pair(rng, H1, W1, H2, W2, d):
+    """Integer maps k1, k2 (values in -9..9, read as k/8 by the float types):
+    a third of image 2's rows are copies of image-1 rows nudged by one step in
+    one coordinate, and some rows repeat, so near-ties and exact ties are
+    frequent and walks merge."""
+    k1 = rng.integers(-8, 9, size=(H1 * W1, d))
+    k2 = rng.integers(-8, 9, size=(H2 * W2, d))
+    for j in rng.choice(H2 * W2, size=max(1, (H2 * W2) // 3), replace=False):
+        k2[j] = k1[rng.integers(H1 * W1)]
+        k2[j, rng.integers(d)] += rng.choice([-1, 1])
+    if H1 * W1 > 2:
+        k1[rng.integers(H1 * W1)] = k1[rng.integers(H1 * W1)]
+    return k1, k2
+
+
+def _as_bf16(k):
+    """Bit patterns of the bfloat16 values k / 8 (exact for |k| <= 9)."""
+    return (np.asarray(k, dtype=np.float32) / np.float32(8)).view(np.uint32).__rshift__(16) \
+        .astype(np.uint16)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "l2"])
+def test_walk_gap_record_equals_per_seed_walks(dtype):
+    """min_gap[u] = max over the walks that stop at u of the smallest top-2
+    margin met on the walk, forward and backward steps included; computed by
+    following each seed's walk on its own with exact scores."""
+    rng = np.random.default_rng(2024 if dtype == "bf16" else 2025)
+    if dtype == "bf16":
+        # 64 <q, p> is an integer: exact in the brute force and in the oracle's doubles
+        score = _brute.dot
+        scale = 64.0
+    else:
+        # -64 |q - p|^2, exact likewise (float32 coordinates k / 8)
+        def score(a, b):
+            return -sum((int(x) - int(y)) ** 2 for x, y in zip(a, b))
+        scale = 64.0
+    merges = backward_decides = finite = 0
+    for _ in range(120):
+        H1, W1, H2, W2 = (int(x) for x in rng.integers(1, 6, size=4))
+        if H1 * W1 < 2 or H2 * W2 < 2:
+            continue
+        d = int(rng.integers(1, 4))
+        k1, k2 = _dyadic_pair(rng, H1, W1, H2, W2, d)
+        sub = int(rng.integers(1, 3))
+        max_iter = int(rng.choice([1, 2, 3, 10]))
+        if dtype == "bf16":
+            m1, m2 = _as_bf16(k1), _as_bf16(k2)
+        else:
+            m1 = (k1.astype(np.float32) / np.float32(8))
+            m2 = (k2.astype(np.float32) / np.float32(8))
+        r = oracle.fast_reciprocal(m1, H1, W1, m2, H2, W2, dtype, sub, max_iter,
+                                   nthreads=1, track_gaps=True)
+        seeds = oracle.grid_seeds(H1, W1, sub).tolist()
+        walks = _brute.walk_gaps(seeds, k1.tolist(), k2.tolist(), max_iter, score)
+        fwd_only = _brute.walk_gaps(seeds, k1.tolist(), k2.tolist(), max_iter, score,
+                                    backward=False)
+        assert set(r.min_gap) == set(walks) == set(r.pairs[:, 0].tolist())
+        for u, gaps in walks.items():
+            want = max(gaps)
+            got = r.min_gap[u] * scale
+            if want == float("inf"):
+                assert got > 1e290
+            else:
+                assert got == want, (u, got, want, gaps)
+                finite += want > 0
+            merges += len(set(gaps)) > 1
+            backward_decides += max(fwd_only[u]) != want
+    # the cases exercise every part of the record: positive finite gaps,
+    # walks to one pixel with different gaps (the maximum over walks), and
+    # walks whose smallest margin is a backward step's
+    assert finite > 20 and merges > 5 and backward_decides > 5, (finite, merges, backward_decides)
+
+
+# ---------------------------------------------------------------------------
 # IEEE half descriptors
 # ---------------------------------------------------------------------------
 
