@@ -246,7 +246,9 @@ int fastnn_mutual_dense_masked(const void *desc1, const float *conf1, int64_t n1
  *   All calls share the one array and it keeps the last call's contents (the
  *   call clears what must start at zero). Calls that overlap on the GPU (on
  *   different streams, or from several host threads without ordering) race on
- *   it; read results with fastnn_device_status only from the last call.
+ *   it. Argument errors are returned before anything is enqueued, with the
+ *   statuses fastnn_reciprocal gives; a device-side bounded wait that ran out
+ *   is read with fastnn_noalloc_device_status().
  */
 #define FASTNN_NOALLOC_SCRATCH_BYTES (32u << 20)
 
@@ -256,6 +258,18 @@ int fastnn_reciprocal_noalloc(const void *desc1, int H1, int W1, const void *des
                               void *out_score, int64_t capacity,
                               int32_t *out_count, int32_t *out_iters,
                               int32_t *out_frontier, fastnn_stream_t stream);
+
+/*
+ * fastnn_noalloc_device_status -- synchronise `stream` and read the device
+ * status word that the last fastnn_reciprocal_noalloc call on the CURRENT
+ * device left in the static scratch array: FASTNN_OK, or FASTNN_ERR_TIMEOUT
+ * when one of that call's bounded waits ran out (its outputs are then
+ * invalid). Blocks the host. If no allocation-free call has run on this
+ * device yet, the first use looks up the array's address (as the first
+ * allocation-free call does). Like the array itself, this has no counterpart
+ * in the pages.
+ */
+int fastnn_noalloc_device_status(fastnn_stream_t stream);
 
 /*
  * fastnn_device_status -- synchronise `stream` and read the device status

@@ -29,6 +29,7 @@ from ._lib import (  # noqa: F401
     fastnn_mutual_dense_masked,
     fastnn_mutual_from_nn,
     fastnn_nn,
+    fastnn_noalloc_device_status,
     fastnn_reciprocal,
     fastnn_reciprocal_masked,
     fastnn_reciprocal_noalloc,

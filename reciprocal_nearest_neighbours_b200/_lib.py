@@ -69,6 +69,8 @@ def library():
     lib.fastnn_mutual_from_nn.restype = I
     lib.fastnn_device_status.argtypes = [P, P]
     lib.fastnn_device_status.restype = I
+    lib.fastnn_noalloc_device_status.argtypes = [P]
+    lib.fastnn_noalloc_device_status.restype = I
     lib.fastnn_kernel_timer_enable.argtypes = [I]
     lib.fastnn_kernel_timer_enable.restype = I
     lib.fastnn_kernel_timer_read.argtypes = [ctypes.POINTER(I), ctypes.POINTER(ctypes.c_double)]
@@ -300,6 +302,12 @@ def fastnn_mutual_from_nn(nn12: torch.Tensor, score12, i0: int, nn21: torch.Tens
 def fastnn_device_status(workspace: torch.Tensor, stream=None) -> int:
     """Synchronise and return the device status of the last call on ``workspace``."""
     return int(library().fastnn_device_status(_ptr(workspace), _stream(stream)))
+
+
+def fastnn_noalloc_device_status(stream=None) -> int:
+    """Synchronise and return the device status of the last allocation-free
+    call on the current device (read from the library's static scratch)."""
+    return int(library().fastnn_noalloc_device_status(_stream(stream)))
 
 
 def fastnn_kernel_timer_enable(capacity: int) -> None:

@@ -57,10 +57,19 @@ extern "C" int fastnn_reciprocal_noalloc(const void* desc1, int H1, int W1, cons
                                          void* out_score, int64_t capacity, int32_t* out_count,
                                          int32_t* out_iters, int32_t* out_frontier,
                                          fastnn_stream_t stream) {
-  if (subsample < 1 || H1 < 1 || W1 < 1 || H2 < 1 || W2 < 1 || batch < 1)
+  // Every argument check runs before the scratch lookup (the first CUDA call),
+  // in fastnn_reciprocal's order, so that both entry points return the same
+  // status for the same bad arguments.
+  const bool dtype_ok = dtype == FASTNN_I8 || dtype == FASTNN_BF16 || dtype == FASTNN_F16 ||
+                        dtype == FASTNN_F32_L2;
+  if (!dtype_ok || d < 1 || d > (dtype == FASTNN_F32_L2 ? 3 : 64)) return FASTNN_ERR_UNSUPPORTED;
+  if (subsample < 1 || H1 < 1 || W1 < 1 || H2 < 1 || W2 < 1 || batch < 1 || max_iter < 1 ||
+      max_iter > 255)
     return FASTNN_ERR_INVALID;
+  if (!desc1 || !desc2 || !out_pairs || !out_count) return FASTNN_ERR_INVALID;
   const int64_t S = static_cast<int64_t>((H1 + subsample - 1) / subsample) *
                     ((W1 + subsample - 1) / subsample);
+  if (capacity < S) return FASTNN_ERR_CAPACITY;
   const size_t need =
       fastnn_workspace_size(FASTNN_OP_RECIPROCAL, static_cast<int64_t>(H1) * W1,
                             static_cast<int64_t>(H2) * W2, d, dtype, batch, S);
@@ -74,4 +83,12 @@ extern "C" int fastnn_reciprocal_noalloc(const void* desc1, int H1, int W1, cons
   return fastnn_reciprocal(desc1, H1, W1, desc2, H2, W2, d, dtype, subsample, max_iter, batch,
                            out_pairs, out_score, capacity, out_count, out_iters, out_frontier,
                            scratch, need, stream);
+}
+
+// The status word sits at the head of the scratch array, where
+// fastnn_reciprocal keeps it at the head of any workspace.
+extern "C" int fastnn_noalloc_device_status(fastnn_stream_t stream) {
+  void* scratch = scratch_for_current_device();
+  if (!scratch) return FASTNN_ERR_CUDA;
+  return fastnn_device_status(scratch, stream);
 }

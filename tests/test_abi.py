@@ -140,3 +140,43 @@ def test_argument_errors_are_reported_on_the_host(lib):
     assert mut(fake, 100, fake, 50, 24, I8, fake, None, 49, fake, fake, big, None) == -3
     assert mut(fake, 0, fake, 50, 24, I8, fake, None, 49, fake, fake, big, None) == -1
     assert mut(fake, 100, fake, 50, 24, I8, None, None, 50, fake, fake, big, None) == -1
+
+
+def test_noalloc_argument_errors_are_reported_on_the_host(lib):
+    """The allocation-free entry point rejects bad arguments, with
+    fastnn_reciprocal's statuses, before its first CUDA call (the scratch
+    lookup): every call here returns without touching a device."""
+    P = ctypes.c_void_p
+    fake = P(1 << 20)  # never dereferenced: validation rejects first
+    I8 = fnn.FASTNN_I8
+    na = lib.fastnn_reciprocal_noalloc
+    S = fnn.seed_count(48, 64, 8)
+    count = (ctypes.c_int32 * 16)(*([-7] * 16))
+    cnt = ctypes.cast(count, P)
+
+    def call(H1=48, W1=64, H2=48, W2=64, d=24, dt=I8, sub=8, it=10, batch=1, cap=S,
+             pairs=fake, d1=fake):
+        return na(d1, H1, W1, fake, H2, W2, d, dt, sub, it, batch, pairs, None, cap, cnt,
+                  None, None, None)
+    # bad sizes, rounds, batch and pointers: FASTNN_ERR_INVALID
+    assert call(sub=0) == -1
+    assert call(H1=0) == -1 and call(W2=0) == -1
+    assert call(batch=0) == -1
+    assert call(it=0) == -1 and call(it=256) == -1
+    assert call(pairs=None) == -1 and call(d1=None) == -1
+    # unsupported d or dtype: FASTNN_ERR_UNSUPPORTED, as fastnn_reciprocal says
+    assert call(d=65) == -2 and call(d=0) == -2 and call(dt=9) == -2
+    assert call(d=4, dt=fnn.FASTNN_F32_L2) == -2
+    rec = lib.fastnn_reciprocal
+    assert rec(fake, 48, 64, fake, 48, 64, 65, I8, 8, 10, 1, fake, None, S, fake, None, None,
+               fake, 1 << 30, None) == -2
+    # capacity below the seed count, and workloads beyond the scratch array
+    assert call(cap=S - 1) == -3
+    need = fnn.fastnn_workspace_size(fnn.FASTNN_OP_RECIPROCAL, 288 * 512, 288 * 512, 32, I8,
+                                     16, 9216)
+    assert need > (32 << 20)
+    assert call(H1=288, W1=512, H2=288, W2=512, d=32, sub=4, it=15, batch=16, cap=9216) == -3
+    # one 512x384 pair fits (int8 and bf16); nothing was written by any call above
+    assert fnn.fastnn_workspace_size(fnn.FASTNN_OP_RECIPROCAL, 196608, 196608, 24,
+                                     fnn.FASTNN_BF16, 1, 3072) <= (32 << 20)
+    assert list(count) == [-7] * 16

@@ -151,38 +151,18 @@ def test_batch_pairs_are_independent_and_exact():
         assert torch.equal(g[0][b, :n], gb[0][0, :n])
 
 
-def _mutual_checks(D1, D2, p, dtype, k=256, seed=0):
-    """Every sampled GPU pair is a mutual nearest-neighbour pair (oracle NN scans)."""
-    rng = np.random.default_rng(seed)
-    sel = p[rng.choice(len(p), size=min(k, len(p)), replace=False)]
-    r12 = oracle.nn(D1[sel[:, 0]], D2, dtype)
-    r21 = oracle.nn(D2[sel[:, 1]], D1, dtype)
-    assert np.array_equal(r12.idx, sel[:, 1]) and np.array_equal(r21.idx, sel[:, 0])
-
-
-def test_batch16_512x288_full_size():
-    """The 16-pair workload in one call: pair 0 exactly, the rest by sampled properties."""
+@pytest.mark.slow
+def test_batch16_512x288_full_size_exact():
+    """The 16-pair workload in one call, every pair compared with the oracle
+    in full (kept set, scores and round count)."""
     w = synth.make_workload("batch16_512x288_d32_i8")
     d1, d2 = w.stacked()
+    assert len(oracle.grid_seeds(288, 512, w.subsample)) == 9216
     g = run_gpu(d1, d2, w.subsample, w.max_iter)
-    check_fast_int8(w.pairs[0].desc1, w.pairs[0].desc2, w.subsample, w.max_iter, b=0, gpu=g)
-    seeds = oracle.grid_seeds(288, 512, w.subsample)
-    assert len(seeds) == 9216
-    rng = np.random.default_rng(9)
-    for b in range(1, 16):
-        p, s = gpu_pairs(g[0], g[1], g[2], b)
-        D1 = w.pairs[b].desc1.reshape(-1, 32)
-        D2 = w.pairs[b].desc2.reshape(-1, 32)
-        assert len(set(p[:, 0].tolist())) == len(p)
-        assert np.array_equal(s.astype(np.int64), oracle.score_of(D1, p[:, 0], D2, p[:, 1], "i8"))
-        if b % 5 == 0:
-            _mutual_checks(D1, D2, p, "i8", k=128, seed=b)
-            # seeds that are mutual at once must all be kept
-            probe = rng.choice(seeds, size=64, replace=False)
-            v = oracle.nn(D1[probe], D2, "i8").idx
-            u2 = oracle.nn(D2[v], D1, "i8").idx
-            kept = set(p[:, 0].tolist())
-            assert all(int(u) in kept for u, x in zip(probe, u2) if u == x)
+    for b in range(16):
+        gp, ref = check_fast_int8(w.pairs[b].desc1, w.pairs[b].desc2, w.subsample, w.max_iter,
+                                  b=b, gpu=g)
+        assert len(gp) > 1000
 
 
 def check_fast_bf16(m1, m2, sub, max_iter, gpu=None, tol=BF16_TOL, dtype="bf16"):
