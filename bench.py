@@ -9,17 +9,22 @@ Inputs are synthetic (``synth``: a smooth warp of map 1 with 30% outliers and
 +-2 noise). Printed value: reciprocal matches per second (unique pairs kept /
 device time of the call), whole job over all ranks.
 
-Other workloads (``--workload``): ``pair_512x384_d24_bf16`` (float
-descriptors), ``batch16_512x288_d32_i8`` (16 pairs per call) and
-``dense_512x384_d24_i8`` (``fastnn_mutual_dense`` over all 196,608 pixels;
-value = mutual pairs per second).
+After the headline, the dense 196,608-pixel mutual set
+(``dense_512x384_d24_i8``), the bf16 pair (``pair_512x384_d24_bf16``) and the
+16-pair batch (``batch16_512x288_d32_i8``) are measured the same way and
+nested in the same JSON line under ``workloads`` (``--also`` changes the
+list). Every workload reports the mean and the 10th / 50th / 90th percentile
+of the per-step device time, its dominant kernel's roofline and the SM clocks
+sampled during its timed region. ``--workload`` makes any other
+configuration the main one.
 
 Each rank processes its own independent pair(s) (pair-level data parallelism,
 no collective on the data path); rank r > 0 draws its inputs from the
-workload's seed + 7919 r.
+workload's seed + 7919 r. ``--gpus N`` outside a launcher starts the N ranks
+itself (torch.distributed.run, rendezvous on 127.0.0.1).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME]
+                    [--workload NAME] [--also NAME,NAME] [--also-steps K2]
 """
 
 from __future__ import annotations
@@ -46,18 +51,34 @@ FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 UNIT = "matches/s"
 DEFAULT_WORKLOAD = "pair_512x384_d24_i8"
 L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
+# Workloads nested in the headline's JSON line by default.
+NESTED_DEFAULT = ["dense_512x384_d24_i8", "pair_512x384_d24_bf16", "batch16_512x288_d32_i8"]
 
 
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.CONFIGS))
     ap.add_argument("--cpu-baseline", type=int, default=1,
                     help="time the CPU oracle on a bounded sample (rank 0, N=1)")
-    return ap.parse_args()
+    ap.add_argument("--also", default=None,
+                    help="comma-separated workloads measured after the main one and nested "
+                         "in its JSON line (default with the headline workload: the dense, "
+                         "bf16 and 16-pair workloads; '' for none)")
+    ap.add_argument("--also-steps", type=int, default=100)
+    ap.add_argument("--stream-steps", type=int, default=None,
+                    help="steps of the 64M-row memory-bound kernel suite nested in the line "
+                         "(default 10 with the headline workload, else 0)")
+    ap.add_argument("--selftest-launcher", action="store_true", help=argparse.SUPPRESS)
+    a = ap.parse_args()
+    if a.also is None:
+        a.also = ",".join(NESTED_DEFAULT) if a.workload == DEFAULT_WORKLOAD else ""
+    if a.stream_steps is None:
+        a.stream_steps = 10 if a.workload == DEFAULT_WORKLOAD else 0
+    return a
 
 
 def dist_env():
@@ -309,244 +330,484 @@ def measured_peaks():
 
 
 # ---------------------------------------------------------------------------
+# ranks
+# ---------------------------------------------------------------------------
+
+def free_port():
+    import socket
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def launch_ranks(args):
+    """``--gpus N`` with N > 1 outside a launcher: start N ranks of this script
+    (one process per GPU, local rendezvous on 127.0.0.1) and return their exit
+    status. Under torchrun (RANK set) the ranks already exist: returns None."""
+    if args.gpus <= 1 or "RANK" in os.environ:
+        return None
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={args.gpus}", "--master-addr", "127.0.0.1",
+           f"--master-port={free_port()}", os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.run(cmd).returncode
+
+
+class Ranks:
+    """Process-group plumbing shared by the measurement and its CPU self-test:
+    barrier, and max / sum reductions of host values over ranks."""
+
+    def __init__(self, world, backend, device):
+        import datetime
+        import torch
+        import torch.distributed as dist
+        self.torch, self.dist, self.world, self.device = torch, dist, world, device
+        if world > 1:
+            kw = {"device_id": device} if backend == "nccl" else {}
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
+
+    def barrier(self):
+        if self.world > 1:
+            self.dist.barrier()
+        if self.device is not None and self.device.type == "cuda":
+            self.torch.cuda.synchronize(self.device)
+
+    def _reduce(self, values, op):
+        t = self.torch.tensor(values, dtype=self.torch.float64, device=self.device)
+        if self.world > 1:
+            self.dist.all_reduce(t, op=op)
+        return t.tolist()
+
+    def max(self, values):
+        return self._reduce(values, self.dist.ReduceOp.MAX)
+
+    def sum(self, values):
+        return self._reduce(values, self.dist.ReduceOp.SUM)
+
+    def close(self):
+        if self.world > 1:
+            self.dist.barrier()
+            self.dist.destroy_process_group()
+
+
+def selftest_launcher(rank, world):
+    """The rank launch and reductions without a GPU (gloo): each rank reports
+    rank + 1 and its rank; rank 0 prints the sum and the maximum."""
+    r = Ranks(world, "gloo", None)
+    s = r.sum([float(rank + 1)])[0]
+    m = r.max([float(rank)])[0]
+    if rank == 0:
+        print(json.dumps({"selftest": "launcher", "n_gpus": world, "rank_sum": s,
+                          "rank_max": m}), flush=True)
+    r.close()
+    return 0
+
+
+def percentiles(ms):
+    a = sorted(ms)
+    pick = lambda q: a[min(len(a) - 1, int(q * len(a)))]  # noqa: E731
+    return {"p10": pick(0.10), "p50": pick(0.50), "p90": pick(0.90)}
+
+
+# ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
 
+class Runner:
+    """One workload on this rank's GPU: device inputs, outputs and workspace,
+    the library call of one step, and its host copies for the end-to-end leg."""
+
+    def __init__(self, name, rank, dev, stream):
+        import torch
+        import reciprocal_nearest_neighbours_b200 as fnn
+        self.torch, self.fnn, self.dev, self.stream = torch, fnn, dev, stream
+        w = self.w = load_workload(name, rank)
+        p0 = w.pairs[0]
+        self.B = w.batch
+        H1, W1, d = p0.desc1.shape
+        H2, W2, _ = p0.desc2.shape
+        self.N1, self.N2, self.d = H1 * W1, H2 * W2, d
+        self.i8 = p0.dtype == "i8"
+        self.l2 = p0.dtype == "l2"
+        code = {"i8": fnn.FASTNN_I8, "bf16": fnn.FASTNN_BF16, "f16": fnn.FASTNN_F16,
+                "l2": fnn.FASTNN_F32_L2}[p0.dtype]
+        sdt = torch.int32 if self.i8 else torch.float32
+        self.masked = masked = "conf1" in w.extra
+        self.esize = 1 if self.i8 else 4 if self.l2 else 2
+        N1, N2, B = self.N1, self.N2, self.B
+        if w.dense:
+            h1 = to_pinned(np.ascontiguousarray(p0.desc1.reshape(-1, d)), torch, p0.dtype)
+            h2 = to_pinned(np.ascontiguousarray(p0.desc2.reshape(-1, d)), torch, p0.dtype)
+            cap = min(N1, N2)
+            self.out_pairs = torch.empty((cap, 2), dtype=torch.int32, device=dev)
+            self.out_score = torch.empty(cap, dtype=sdt, device=dev)
+            self.out_count = torch.empty(1, dtype=torch.int32, device=dev)
+            nbytes = fnn.fastnn_workspace_size(fnn.FASTNN_OP_MUTUAL_DENSE, N1, N2, d, code)
+            self.hp_pairs = torch.empty((cap, 2), dtype=torch.int32).pin_memory()
+            self.hp_score = torch.empty(cap, dtype=sdt).pin_memory()
+        else:
+            d1n, d2n = w.stacked()
+            h1, h2 = to_pinned(d1n, torch, p0.dtype), to_pinned(d2n, torch, p0.dtype)
+            S = fnn.seed_count(H1, W1, w.subsample)
+            self.out_pairs = torch.empty((B, S, 2), dtype=torch.int32, device=dev)
+            self.out_score = torch.empty((B, S), dtype=sdt, device=dev)
+            self.out_count = torch.empty(B, dtype=torch.int32, device=dev)
+            self.out_iters = torch.empty(B, dtype=torch.int32, device=dev)
+            self.out_front = torch.empty((B, w.max_iter), dtype=torch.int32, device=dev)
+            op = fnn.FASTNN_OP_RECIPROCAL_MASKED if masked else fnn.FASTNN_OP_RECIPROCAL
+            nbytes = fnn.fastnn_workspace_size(op, N1, N2, d, code, B, S)
+            self.hp_pairs = torch.empty((B, S, 2), dtype=torch.int32).pin_memory()
+            self.hp_score = torch.empty((B, S), dtype=sdt).pin_memory()
+        self.hp_count = torch.empty(self.out_count.shape, dtype=torch.int32).pin_memory()
+        self.h1, self.h2 = h1, h2
+        self.d1, self.d2 = h1.to(dev), h2.to(dev)
+        self.ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        self.hc1 = self.hc2 = self.c1 = self.c2 = None
+        if masked:
+            self.hc1 = torch.from_numpy(np.ascontiguousarray(np.stack(w.extra["conf1"]))).pin_memory()
+            self.hc2 = torch.from_numpy(np.ascontiguousarray(np.stack(w.extra["conf2"]))).pin_memory()
+            self.c1, self.c2 = self.hc1.to(dev), self.hc2.to(dev)
+        if w.dense:
+            # 2 repack, forward pass, image list (mark/count/scan/emit), pointmaps:
+            # chunk boxes of image 1, backward pass, mutual count/scan/emit
+            self.launches_per_step = 2 + 1 + 4 + (1 if self.l2 else 0) + 1 + 3
+            self.kernels_per_step = 2
+        elif masked:
+            # 2 x (count, scan, emit) mask compaction, seeds, 1 persistent matching kernel
+            self.launches_per_step = 8
+            self.kernels_per_step = 1
+        else:
+            self.launches_per_step = 3  # 2 repack kernels + 1 persistent matching kernel
+            self.kernels_per_step = 1
+
+    def call(self):
+        fnn, w = self.fnn, self.w
+        if w.dense:
+            fnn.fastnn_mutual_dense(self.d1, self.d2, out_pairs=self.out_pairs,
+                                    out_score=self.out_score, out_count=self.out_count,
+                                    workspace=self.ws, stream=self.stream)
+        elif self.masked:
+            fnn.fastnn_reciprocal_masked(self.d1, self.d2, w.subsample, w.max_iter, conf1=self.c1,
+                                         conf2=self.c2, threshold=w.extra["threshold"],
+                                         out_pairs=self.out_pairs, out_score=self.out_score,
+                                         out_count=self.out_count, out_iters=self.out_iters,
+                                         out_frontier=self.out_front, workspace=self.ws,
+                                         stream=self.stream)
+        else:
+            fnn.fastnn_reciprocal(self.d1, self.d2, w.subsample, w.max_iter,
+                                  out_pairs=self.out_pairs, out_score=self.out_score,
+                                  out_count=self.out_count, out_iters=self.out_iters,
+                                  out_frontier=self.out_front, workspace=self.ws,
+                                  stream=self.stream)
+
+    def call_e2e(self):
+        """One step through the public API with host buffers: inputs copied in
+        from pinned memory, the call, every output copied back."""
+        self.d1.copy_(self.h1, non_blocking=True)
+        self.d2.copy_(self.h2, non_blocking=True)
+        if self.masked:
+            self.c1.copy_(self.hc1, non_blocking=True)
+            self.c2.copy_(self.hc2, non_blocking=True)
+        self.call()
+        self.hp_count.copy_(self.out_count, non_blocking=True)
+        self.hp_pairs.copy_(self.out_pairs, non_blocking=True)
+        self.hp_score.copy_(self.out_score, non_blocking=True)
+
+    def bytes_per_step(self):
+        bin_ = (self.N1 + self.N2) * self.d * self.esize * self.B + \
+            ((self.N1 + self.N2) * 4 * self.B if self.masked else 0)
+        bout = int(self.hp_count.numel() * 4 + self.hp_pairs.numel() * 4 +
+                   self.hp_score.numel() * 4)
+        return bin_, bout
+
+    def matches(self):
+        return int(self.out_count.cpu().sum())
+
+    def work_per_step(self):
+        """(score elements per step, row count of the dense backward pass or None)."""
+        if self.w.dense:
+            # The backward pass runs on the image of NN12 only (the rows that
+            # can be in a mutual pair): count them for the useful-work figure.
+            idx12, _ = self.fnn.fastnn_nn(self.d1, self.d2)
+            image = int(self.torch.unique(idx12[(idx12 >= 0) & (idx12 < self.N2)]).numel())
+            return self.N1 * self.N2 + image * self.N1, image
+        return int(self.out_front.cpu().sum()) * (self.N1 + self.N2), None
+
+
+def time_steps(run, K, flush, ranks, e2e=False):
+    """K steps, L2 flushed before each; CUDA events on the launching stream
+    around each step. Returns per-step ms (max over ranks) and this rank's
+    (timed kernel launches, kernel ms)."""
+    torch, fnn = run.torch, run.fnn
+    if not e2e:
+        fnn.fastnn_kernel_timer_enable(K * run.kernels_per_step + 8)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K)]
+    ranks.barrier()
+    for i in range(K):
+        flush.zero_()
+        evs[i][0].record(run.stream)
+        if e2e:
+            run.call_e2e()
+        else:
+            run.call()
+        evs[i][1].record(run.stream)
+    ranks.barrier()
+    ms = [s.elapsed_time(e) for s, e in evs]
+    nn = (0, 0.0)
+    if not e2e:
+        nn = fnn.fastnn_kernel_timer_read()
+        fnn.fastnn_kernel_timer_enable(0)
+    return ranks.max(ms), nn
+
+
+def roofline_for(run, work, image, K, nn_launches, nn_ms, total_ms):
+    d, w, l2 = run.d, run.w, run.l2
+    peaks, src = measured_peaks()
+    bf16_peak = float(peaks["bf16_tflops"])
+    if l2:
+        # Pointmaps: 3 fused multiply-adds per (query, point) pair on the FP32
+        # pipe; peak = 148 SMs x 128 FMA lanes x 2 flop x 1.965 GHz.
+        peak = FP32_FMA_TFLOPS
+        achieved = 6.0 * work * K / (nn_ms / 1e3) / 1e12 if nn_ms > 0 else None
+        kname = ("nn_l2_kernel (FP32 FMA nearest point: forward pass over every image-1 "
+                 "point, backward pass over the image of the forward matches)" if w.dense else
+                 "reciprocal_l2_kernel (persistent: seeds, FP32 FMA forward and backward "
+                 "passes, per-pair compaction)")
+        peak_source = ("derived: FP32 FMA pipe, 148 SMs x 128 lanes x 2 flop x 1.965 GHz "
+                       "(clocks.max.sm)")
+        ops = f"3 FMA = 6 flop per (query, point) pair: {work:.4g} pairs per step"
+    else:
+        peak = 2.0 * bf16_peak if run.i8 else bf16_peak  # dense int8 = 2 x bf16 (nominal ratio)
+        achieved = 2.0 * work * d * K / (nn_ms / 1e3) / 1e12 if nn_ms > 0 else None
+        kname = ("nn_tc_kernel (tcgen05 argmax-GEMM: forward pass over every image-1 row, "
+                 "backward pass over the image of the forward matches)" if w.dense else
+                 "reciprocal_kernel (persistent: seeds, tcgen05 forward and backward passes, "
+                 "per-pair compaction)")
+        peak_source = (f"{src}: bf16_tflops {bf16_peak}" +
+                       (" x 2 (int8 = 2 x bf16, nominal ratio)" if run.i8 else ""))
+        ops = f"2 x useful MACs (d = {d}) per step: {work * d:.4g} MAC"
+    if image is not None:
+        ops += f" ({run.N1} x {run.N2} forward + {image} x {run.N1} backward)"
+    return {
+        "bound": "alu" if l2 else "tensor", "kernel": kname,
+        "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+        "frac": (achieved / peak) if achieved else None,
+        "traffic": traffic_for(w.name),
+        "traffic_unit": ("bytes per step: forward + backward launch (ncu dram read + write)"
+                         if w.dense else "bytes per launch (ncu dram read + write)"),
+        "peak_source": peak_source, "ops": ops,
+        "kernel_ms_per_step": nn_ms / K, "kernel_launches": nn_launches,
+        "kernel_share_of_step": nn_ms / total_ms if total_ms else None,
+    }
+
+
+def measure(name, K, W, rank, ranks, dev, stream, flush, sample_clocks, e2e_steps=0):
+    """Warm up, time K steps (and optionally an end-to-end leg) of one workload.
+    Returns this workload's result dict (meaningful on rank 0)."""
+    import torch
+    run = Runner(name, rank, dev, stream)
+    fnn = run.fnn
+    for _ in range(max(W, 3)):
+        flush.zero_()
+        run.call()
+    torch.cuda.synchronize(dev)
+    assert fnn.fastnn_device_status(run.ws) == 0
+    matches = run.matches()
+    work, image = run.work_per_step()
+    sampler = None
+    if sample_clocks:
+        uuid = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        except Exception:  # noqa: BLE001
+            pass
+        sampler = ClockSampler(uuid)
+        time.sleep(0.5)
+    step_ms, (nn_launches, nn_ms) = time_steps(run, K, flush, ranks)
+    clocks = sampler.stop() if sampler else None
+    assert fnn.fastnn_device_status(run.ws) == 0
+    assert run.matches() == matches
+    e2e_ms = None
+    if e2e_steps:
+        e2e_ms, _ = time_steps(run, e2e_steps, flush, ranks, e2e=True)
+        assert int(run.hp_count.sum()) == matches
+    total_ms = sum(step_ms)
+    nn_ms = ranks.max([nn_ms])[0]
+    all_matches = ranks.sum([float(matches)])[0]
+    world = ranks.world
+    res = {
+        "metric": metric_for(name, run.w.dense), "value": all_matches * K / (total_ms / 1e3),
+        "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": total_ms / K,
+        "ms_per_step_percentiles": percentiles(step_ms),
+        "dtype": {"i8": "int8", "bf16": "bf16", "f16": "f16", "l2": "f32"}[run.w.pairs[0].dtype],
+        "config": config_dict(run.w),
+        "pairs_per_s": world * run.B * K / (total_ms / 1e3),
+        "matches_per_step_rank0": matches,
+        "roofline": roofline_for(run, work, image, K, nn_launches, nn_ms, total_ms),
+        "gpu_launches": run.launches_per_step * K,
+        "clocks": clocks,
+    }
+    if not run.w.dense:
+        res["frontier_per_round_pair0"] = run.out_front[0].cpu().tolist()
+    if e2e_ms is not None:
+        bin_, bout = run.bytes_per_step()
+        res["e2e"] = {"value": all_matches * e2e_steps / (sum(e2e_ms) / 1e3), "unit": UNIT,
+                      "h2d_bytes_per_step": bin_, "d2h_bytes_per_step": bout,
+                      "steps": e2e_steps, "ms_per_step_percentiles": percentiles(e2e_ms)}
+    res["_workload"] = run.w
+    return res
+
+
+# ---------------------------------------------------------------------------
+# the memory-bound kernels at a scale where HBM bandwidth bounds them
+# ---------------------------------------------------------------------------
+
+STREAM_ROWS = 64 << 20  # 67,108,864 rows: inputs far larger than L2
+
+
+def measure_stream(K, ranks, dev, stream, flush, sample_clocks):
+    """Achieved HBM bandwidth of the repack, dense mutual test/emit and
+    confidence-mask compaction kernels on a 64M-row int8 map (d = 24; a few
+    GB on the device). Each kind is timed with the library's launch timer
+    restricted to that kind, inside an ordinary call:
+      repack  -- fastnn_nn of the 64M-row map against a 256-row database
+                 (its query map's repack: N x 24 B read, N x 32 B written);
+      mutual  -- fastnn_mutual_from_nn on 64M-row index arrays of a smooth
+                 synthetic correspondence (count, scan and ordered emit:
+                 2 x 8 B read per row, 16 B per kept pair);
+      mask    -- fastnn_mutual_dense_masked of the 64M-row map (confidences
+                 uniform in [0, 1), threshold 0.5) against a 256-row map
+                 (map 1's compaction: 2 x 4 B of confidence per row, and per
+                 kept row 24 B read, 32 + 4 B written).
+    Inputs are drawn on the device from a seeded generator."""
+    import torch
+    import reciprocal_nearest_neighbours_b200 as fnn
+    N, d = STREAM_ROWS, 24
+    g = torch.Generator(device=dev)
+    g.manual_seed(synth.BASE_SEED + 60 + 7919 * ranks_rank(ranks))
+    peaks, src = measured_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    out = {"workload": f"stream_{N >> 20}M_d{d}_i8", "rows": N, "steps": K,
+           "peak": hbm, "peak_source": f"{src}: hbm_gbs", "kernels": []}
+
+    def timed(kind, call, nbytes_fn):
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize(dev)
+        prev = fnn.fastnn_kernel_timer_select(kind)
+        fnn.fastnn_kernel_timer_enable(4 * K + 8)
+        sampler = ClockSampler(None) if sample_clocks else None
+        ranks.barrier()
+        for _ in range(K):
+            flush.zero_()
+            call()
+        ranks.barrier()
+        clocks = sampler.stop() if sampler else None
+        n, ms = fnn.fastnn_kernel_timer_read()
+        fnn.fastnn_kernel_timer_enable(0)
+        fnn.fastnn_kernel_timer_select(prev)
+        ms = ranks.max([ms])[0]
+        nbytes = nbytes_fn()
+        gbs = nbytes * K / (ms / 1e3) / 1e9
+        return {"launch_brackets": n, "ms_per_step": ms / K, "bytes_per_step": nbytes,
+                "achieved_gbs": gbs, "frac": gbs / hbm, "clocks": clocks}
+
+    A = torch.randint(-16, 17, (N, d), dtype=torch.int8, device=dev, generator=g)
+    db = torch.randint(-16, 17, (256, d), dtype=torch.int8, device=dev, generator=g)
+    ws = torch.empty(fnn.fastnn_workspace_size(fnn.FASTNN_OP_NN, N, 256, d, fnn.FASTNN_I8),
+                     dtype=torch.uint8, device=dev)
+    idx = torch.empty(N, dtype=torch.int32, device=dev)
+    r = timed(fnn.FASTNN_TIME_REPACK, lambda: fnn.fastnn_nn(A, db, out_idx=idx, workspace=ws),
+              lambda: N * d + N * 32 + 256 * d + 512 * 32)
+    r["kind"] = "repack (repack_staged_kernel: 64M x 24 B rows into 32 B rows)"
+    out["kernels"].append(r)
+    del ws, idx
+
+    # A smooth correspondence: row i's partner is i + a small signed offset,
+    # and a partner points back to i for about 70% of rows.
+    off = torch.randint(-3, 4, (N,), dtype=torch.int32, device=dev, generator=g)
+    ar = torch.arange(N, dtype=torch.int32, device=dev)
+    nn12 = (ar + off).clamp_(0, N - 1)
+    nn21 = ar.clone()
+    nn21[nn12] = ar
+    miss = torch.rand(N, device=dev, generator=g) < 0.3
+    nn21[miss] = (nn21[miss] + 1).clamp_(max=N - 1)
+    score = torch.randint(0, 1000, (N,), dtype=torch.int32, device=dev, generator=g)
+    mws = torch.empty(fnn.fastnn_workspace_size(fnn.FASTNN_OP_MUTUAL_FROM_NN, N, N, 1,
+                                                fnn.FASTNN_I8), dtype=torch.uint8, device=dev)
+    pairs = torch.empty((N, 2), dtype=torch.int32, device=dev)
+    pscore = torch.empty(N, dtype=torch.int32, device=dev)
+    cnt = torch.empty(1, dtype=torch.int32, device=dev)
+    r = timed(fnn.FASTNN_TIME_MUTUAL,
+              lambda: fnn.fastnn_mutual_from_nn(nn12, score, 0, nn21, N, out_pairs=pairs,
+                                                out_score=pscore, out_count=cnt, workspace=mws),
+              lambda: 16 * N + 16 * int(cnt.item()))
+    r["kind"] = "mutual test and ordered emit (mutual_count, mutual_scan, mutual_emit)"
+    r["kept"] = int(cnt.item())
+    out["kernels"].append(r)
+    del off, ar, nn12, nn21, miss, score, mws, pairs, pscore
+
+    conf = torch.rand(N, device=dev, generator=g)
+    kept1 = int((conf >= 0.5).sum().item())
+    wsm = torch.empty(fnn.fastnn_workspace_size(fnn.FASTNN_OP_MUTUAL_DENSE_MASKED, N, 256, d,
+                                                fnn.FASTNN_I8), dtype=torch.uint8, device=dev)
+    mp = torch.empty((256, 2), dtype=torch.int32, device=dev)
+    ms_ = torch.empty(256, dtype=torch.int32, device=dev)
+    r = timed(fnn.FASTNN_TIME_MASK,
+              lambda: fnn.fastnn_mutual_dense_masked(A, db, conf1=conf, threshold=0.5,
+                                                     out_pairs=mp, out_score=ms_, out_count=cnt,
+                                                     workspace=wsm),
+              lambda: 8 * N + kept1 * (d + 36) + 8 * 256 + 256 * (d + 36))
+    r["kind"] = ("confidence-mask compaction (mask_count, scan, mask_emit) of the 64M-row map "
+                 "and of the 256-row map")
+    r["kept"] = kept1
+    out["kernels"].append(r)
+    return out
+
+
+def ranks_rank(ranks):
+    return ranks.dist.get_rank() if ranks.world > 1 else 0
+
+
 def run_ours(args, rank, world, local):
     import torch
-    import torch.distributed as dist
-    import reciprocal_nearest_neighbours_b200 as fnn
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
-
-    w = load_workload(args.workload, rank)
-    p0 = w.pairs[0]
-    B = w.batch
-    H1, W1, d = p0.desc1.shape
-    H2, W2, _ = p0.desc2.shape
-    N1, N2 = H1 * W1, H2 * W2
-    i8 = p0.dtype == "i8"
-    code = {"i8": fnn.FASTNN_I8, "bf16": fnn.FASTNN_BF16, "f16": fnn.FASTNN_F16,
-            "l2": fnn.FASTNN_F32_L2}[p0.dtype]
-    sdt = torch.int32 if i8 else torch.float32
-    l2 = p0.dtype == "l2"
-    masked = "conf1" in w.extra
-    esize = 1 if i8 else 4 if l2 else 2
+    ranks = Ranks(world, "nccl", dev)
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
-    if w.dense:
-        h1 = to_pinned(np.ascontiguousarray(p0.desc1.reshape(-1, d)), torch, p0.dtype)
-        h2 = to_pinned(np.ascontiguousarray(p0.desc2.reshape(-1, d)), torch, p0.dtype)
-        cap = min(N1, N2)
-        out_pairs = torch.empty((cap, 2), dtype=torch.int32, device=dev)
-        out_score = torch.empty(cap, dtype=sdt, device=dev)
-        out_count = torch.empty(1, dtype=torch.int32, device=dev)
-        nbytes = fnn.fastnn_workspace_size(fnn.FASTNN_OP_MUTUAL_DENSE, N1, N2, d, code)
-        hp_pairs = torch.empty((cap, 2), dtype=torch.int32).pin_memory()
-        hp_score = torch.empty(cap, dtype=sdt).pin_memory()
-    else:
-        d1n, d2n = w.stacked()
-        h1, h2 = to_pinned(d1n, torch, p0.dtype), to_pinned(d2n, torch, p0.dtype)
-        S = fnn.seed_count(H1, W1, w.subsample)
-        out_pairs = torch.empty((B, S, 2), dtype=torch.int32, device=dev)
-        out_score = torch.empty((B, S), dtype=sdt, device=dev)
-        out_count = torch.empty(B, dtype=torch.int32, device=dev)
-        out_iters = torch.empty(B, dtype=torch.int32, device=dev)
-        out_front = torch.empty((B, w.max_iter), dtype=torch.int32, device=dev)
-        op = fnn.FASTNN_OP_RECIPROCAL_MASKED if masked else fnn.FASTNN_OP_RECIPROCAL
-        nbytes = fnn.fastnn_workspace_size(op, N1, N2, d, code, B, S)
-        hp_pairs = torch.empty((B, S, 2), dtype=torch.int32).pin_memory()
-        hp_score = torch.empty((B, S), dtype=sdt).pin_memory()
-    hp_count = torch.empty(out_count.shape, dtype=torch.int32).pin_memory()
-    d1 = h1.to(dev)
-    d2 = h2.to(dev)
-    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
-    hc1 = hc2 = c1 = c2 = None
-    if masked:
-        hc1 = torch.from_numpy(np.ascontiguousarray(np.stack(w.extra["conf1"]))).pin_memory()
-        hc2 = torch.from_numpy(np.ascontiguousarray(np.stack(w.extra["conf2"]))).pin_memory()
-        c1, c2 = hc1.to(dev), hc2.to(dev)
-
-    if w.dense:
-        def call():
-            fnn.fastnn_mutual_dense(d1, d2, out_pairs=out_pairs, out_score=out_score,
-                                    out_count=out_count, workspace=ws, stream=stream)
-        # 2 repack, forward pass, image list (mark/count/scan/emit), pointmaps:
-        # chunk boxes of image 1, backward pass, mutual count/scan/emit
-        launches_per_step = 2 + 1 + 4 + (1 if l2 else 0) + 1 + 3
-        kernels_per_step = 2
-    elif masked:
-        def call():
-            fnn.fastnn_reciprocal_masked(d1, d2, w.subsample, w.max_iter, conf1=c1, conf2=c2,
-                                         threshold=w.extra["threshold"], out_pairs=out_pairs,
-                                         out_score=out_score, out_count=out_count,
-                                         out_iters=out_iters, out_frontier=out_front,
-                                         workspace=ws, stream=stream)
-        # 2 x (count, scan, emit) mask compaction, seeds, 1 persistent matching kernel
-        launches_per_step = 8
-        kernels_per_step = 1
-    else:
-        def call():
-            fnn.fastnn_reciprocal(d1, d2, w.subsample, w.max_iter, out_pairs=out_pairs,
-                                  out_score=out_score, out_count=out_count, out_iters=out_iters,
-                                  out_frontier=out_front, workspace=ws, stream=stream)
-        launches_per_step = 3  # 2 repack kernels + 1 persistent matching kernel (all rounds)
-        kernels_per_step = 1
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize(dev)
-
-    for _ in range(max(args.warmup, 3)):
-        flush.zero_()
-        call()
-    torch.cuda.synchronize(dev)
-    assert fnn.fastnn_device_status(ws) == 0
-    matches = int(out_count.cpu().sum())
-    image = None
-    if w.dense:
-        # The backward pass runs on the image of NN12 only (the rows that can
-        # be in a mutual pair): count them for the useful-work figure.
-        idx12, _ = fnn.fastnn_nn(d1, d2)
-        image = int(torch.unique(idx12[(idx12 >= 0) & (idx12 < N2)]).numel())
-        pairs_per_step = N1 * N2 + image * N1
-    else:
-        pairs_per_step = int(out_front.cpu().sum()) * (N1 + N2)
-    macs_per_step = pairs_per_step * d
-
-    # ---- device-timed region ------------------------------------------------
-    uuid = None
-    try:
-        uuid = str(torch.cuda.get_device_properties(dev).uuid)
-    except Exception:  # noqa: BLE001
-        pass
-    sampler = ClockSampler(uuid) if rank == 0 else None
-    if sampler:
-        time.sleep(0.5)
-    K = args.steps
-    fnn.fastnn_kernel_timer_enable(K * kernels_per_step + 8)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(K)]
-    barrier()
-    for i in range(K):
-        flush.zero_()
-        evs[i][0].record(stream)
-        call()
-        evs[i][1].record(stream)
-    barrier()
-    clocks = sampler.stop() if sampler else None
-    total_ms = sum(s.elapsed_time(e) for s, e in evs)
-    nn_launches, nn_ms = fnn.fastnn_kernel_timer_read()
-    fnn.fastnn_kernel_timer_enable(0)
-    assert fnn.fastnn_device_status(ws) == 0
-    assert int(out_count.cpu().sum()) == matches
-
-    # ---- end to end through the C ABI with host buffers --------------------
-    Ke = max(1, min(K, 1000))
-    evs2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in range(Ke)]
-    barrier()
-    for i in range(Ke):
-        flush.zero_()
-        evs2[i][0].record(stream)
-        d1.copy_(h1, non_blocking=True)
-        d2.copy_(h2, non_blocking=True)
-        if masked:
-            c1.copy_(hc1, non_blocking=True)
-            c2.copy_(hc2, non_blocking=True)
-        call()
-        hp_count.copy_(out_count, non_blocking=True)
-        hp_pairs.copy_(out_pairs, non_blocking=True)
-        hp_score.copy_(out_score, non_blocking=True)
-        evs2[i][1].record(stream)
-    barrier()
-    e2e_ms = sum(s.elapsed_time(e) for s, e in evs2)
-    assert int(hp_count.sum()) == matches
-
-    # ---- reduce over ranks ----------------------------------------------------
-    vals = torch.tensor([total_ms, e2e_ms, nn_ms], dtype=torch.float64, device=dev)
-    m = torch.tensor([matches], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-        dist.all_reduce(m, op=dist.ReduceOp.SUM)
-    total_ms, e2e_ms, _ = vals.tolist()
-    all_matches = float(m.item())
-
+    head = measure(args.workload, args.steps, args.warmup, rank, ranks, dev, stream, flush,
+                   sample_clocks=rank == 0, e2e_steps=max(1, min(args.steps, 1000)))
+    also = [x for x in (args.also.split(",") if args.also else []) if x and x != args.workload]
+    nested = []
+    for name in also:
+        r = measure(name, args.also_steps, args.warmup, rank, ranks, dev, stream, flush,
+                    sample_clocks=rank == 0)
+        r.pop("_workload")
+        nested.append({k: r[k] for k in ("metric", "value", "unit", "steps", "ms_per_step",
+                                         "ms_per_step_percentiles", "dtype", "config",
+                                         "pairs_per_s", "roofline", "clocks", "gpu_launches")})
+    streams = None
+    if args.stream_steps > 0:
+        streams = measure_stream(args.stream_steps, ranks, dev, stream, flush,
+                                 sample_clocks=rank == 0)
     if rank == 0:
-        value = all_matches * K / (total_ms / 1e3)
-        e2e_value = all_matches * Ke / (e2e_ms / 1e3)
-        pairs_per_s = world * B * K / (total_ms / 1e3)
-        peaks, src = measured_peaks()
-        bf16_peak = float(peaks["bf16_tflops"])
-        if l2:
-            # Pointmaps: 3 fused multiply-adds per (query, point) pair on the
-            # FP32 pipe; peak = 148 SMs x 128 FMA lanes x 2 flop x 1.965 GHz.
-            peak = FP32_FMA_TFLOPS
-            achieved = 6.0 * pairs_per_step * K / (nn_ms / 1e3) / 1e12 if nn_ms > 0 else None
-        else:
-            peak = 2.0 * bf16_peak if i8 else bf16_peak  # dense int8 = 2 x bf16 (nominal ratio)
-            achieved = 2.0 * macs_per_step * K / (nn_ms / 1e3) / 1e12 if nn_ms > 0 else None
-        bytes_in = (N1 + N2) * d * esize * B + ((N1 + N2) * 4 * B if masked else 0)
-        bytes_out = int(hp_count.numel() * 4 + hp_pairs.numel() * 4 + hp_score.numel() * 4)
-        if l2:
-            kname = ("nn_l2_kernel (FP32 FMA nearest point: forward pass over every image-1 "
-                     "point, backward pass over the image of the forward matches)"
-                     if w.dense else
-                     "reciprocal_l2_kernel (persistent: seeds, FP32 FMA forward and backward "
-                     "passes, per-pair compaction)")
-        else:
-            kname = ("nn_tc_kernel (tcgen05 argmax-GEMM: forward pass over every image-1 row, "
-                     "backward pass over the image of the forward matches)" if w.dense else
-                     "reciprocal_kernel (persistent: seeds, tcgen05 forward and backward passes, "
-                     "per-pair compaction)")
-        if l2:
-            peak_source = ("derived: FP32 FMA pipe, 148 SMs x 128 lanes x 2 flop x 1.965 GHz "
-                           "(clocks.max.sm)")
-            ops = (f"3 FMA = 6 flop per (query, point) pair: {pairs_per_step:.4g} pairs "
-                   f"per step")
-            if image is not None:
-                ops += f" ({N1} x {N2} forward + {image} x {N1} backward)"
-        else:
-            peak_source = (f"{src}: bf16_tflops {bf16_peak}" +
-                           (" x 2 (int8 = 2 x bf16, nominal ratio)" if i8 else ""))
-            ops = f"2 x useful MACs (d = {d}) per step: {macs_per_step:.4g} MAC"
-            if image is not None:
-                ops += f" ({N1} x {N2} forward + {image} x {N1} backward)"
+        w = head.pop("_workload")
         line = {
-            "metric": metric_for(w.name, w.dense), "value": value, "unit": UNIT, "n_gpus": world,
-            "steps": K, "warmup": args.warmup, "ms_per_step": total_ms / K,
+            "metric": head["metric"], "value": head["value"], "unit": UNIT, "n_gpus": world,
+            "steps": head["steps"], "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": {"i8": "int8", "bf16": "bf16", "f16": "f16", "l2": "f32"}[p0.dtype],
-            "data": "synthetic",
-            "config": config_dict(w),
-            "pairs_per_s": pairs_per_s,
-            "matches_per_step_rank0": matches,
-            "roofline": {
-                "bound": "alu" if l2 else "tensor", "kernel": kname,
-                "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": (achieved / peak) if achieved else None,
-                "traffic": traffic_for(w.name),
-                "traffic_unit": ("bytes per step: forward + backward launch (ncu dram read + write)"
-                                 if w.dense else "bytes per launch (ncu dram read + write)"),
-                "peak_source": peak_source,
-                "ops": ops,
-                "kernel_ms_per_step": nn_ms / K, "kernel_launches": nn_launches,
-                "kernel_share_of_step": nn_ms / total_ms if total_ms else None,
-            },
-            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": bytes_in,
-                    "d2h_bytes_per_step": bytes_out, "steps": Ke},
-            "gpu_launches": launches_per_step * K,
-            "clocks": clocks,
+            "dtype": head["dtype"], "data": "synthetic", "config": head["config"],
         }
-        if not w.dense:
-            line["frontier_per_round_pair0"] = out_front[0].cpu().tolist()
+        line.update({k: v for k, v in head.items() if k not in line})
+        line["gpu_launches"] = head["gpu_launches"] + sum(n["gpu_launches"] for n in nested)
+        line["gpu_launches_headline"] = head["gpu_launches"]
+        if nested:
+            line["workloads"] = nested
+        if streams:
+            line["stream_kernels"] = streams
         if args.cpu_baseline and world == 1:
             try:
                 cm, cdt, cthreads, cdesc = oracle_sample(w, 256, dense_rows=1024)
@@ -557,15 +818,18 @@ def run_ours(args, rank, world, local):
                 line["cpu_baseline"] = {"value": None, "unit": UNIT, "cores": None,
                                         "kind": "oracle", "sample": f"failed: {e}"}
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    ranks.close()
     return 0
 
 
 def main():
     args = parse_args()
+    rc = launch_ranks(args)
+    if rc is not None:
+        return rc
     rank, world, local = dist_env()
+    if args.selftest_launcher:
+        return selftest_launcher(rank, world)
     if args.impl == "reference":
         return run_reference(args, rank, world)
     return run_ours(args, rank, world, local)

@@ -282,7 +282,8 @@ int fastnn_device_status(const void *workspace, fastnn_stream_t stream);
 /*
  * Benchmark instrumentation (not needed for matching). After
  * fastnn_kernel_timer_enable(capacity > 0), each of the next `capacity`
- * launches of the tensor-core nearest-neighbour kernel is bracketed by two
+ * launches of the selected kinds (fastnn_kernel_timer_select below; by
+ * default the nearest-neighbour and matching kernels) is bracketed by two
  * CUDA events recorded on the launching stream (events are created here, once,
  * not per call). fastnn_kernel_timer_read() waits for the recorded events,
  * returns the number of timed launches and their summed device time in
@@ -292,6 +293,24 @@ int fastnn_device_status(const void *workspace, fastnn_stream_t stream);
  */
 int fastnn_kernel_timer_enable(int capacity);
 int fastnn_kernel_timer_read(int *launches, double *total_ms);
+
+/*
+ * fastnn_kernel_timer_select -- which launches the timer above brackets, as a
+ * bit mask (each bracket covers the kernels one call of that kind launches):
+ *   FASTNN_TIME_MATCHING (1, the default): the tensor-core and pointmap
+ *     nearest-neighbour kernels and the persistent matching kernels;
+ *   FASTNN_TIME_REPACK (2): the repack of each descriptor map;
+ *   FASTNN_TIME_MUTUAL (4): the dense mutual test and ordered emit (count,
+ *     scan, emit), and the list of image-2 rows the dense backward pass runs on;
+ *   FASTNN_TIME_MASK (8): the confidence-mask compaction of each map.
+ * kinds <= 0 leaves the selection as it is. Returns the previous selection.
+ * Benchmark instrumentation: process-wide, like the timer itself.
+ */
+#define FASTNN_TIME_MATCHING 1
+#define FASTNN_TIME_REPACK 2
+#define FASTNN_TIME_MUTUAL 4
+#define FASTNN_TIME_MASK 8
+int fastnn_kernel_timer_select(int kinds);
 
 /* Text of the last CUDA runtime error this library saw on the calling host
  * thread (the cause behind a FASTNN_ERR_CUDA return); a static string. */

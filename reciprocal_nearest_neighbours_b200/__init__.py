@@ -21,10 +21,15 @@ from ._lib import (  # noqa: F401
     FASTNN_OP_NN,
     FASTNN_OP_RECIPROCAL,
     FASTNN_OP_RECIPROCAL_MASKED,
+    FASTNN_TIME_MASK,
+    FASTNN_TIME_MATCHING,
+    FASTNN_TIME_MUTUAL,
+    FASTNN_TIME_REPACK,
     FastNNError,
     fastnn_device_status,
     fastnn_kernel_timer_enable,
     fastnn_kernel_timer_read,
+    fastnn_kernel_timer_select,
     fastnn_mutual_dense,
     fastnn_mutual_dense_masked,
     fastnn_mutual_from_nn,

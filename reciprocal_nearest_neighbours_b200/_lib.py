@@ -73,6 +73,8 @@ def library():
     lib.fastnn_noalloc_device_status.restype = I
     lib.fastnn_kernel_timer_enable.argtypes = [I]
     lib.fastnn_kernel_timer_enable.restype = I
+    lib.fastnn_kernel_timer_select.argtypes = [I]
+    lib.fastnn_kernel_timer_select.restype = I
     lib.fastnn_kernel_timer_read.argtypes = [ctypes.POINTER(I), ctypes.POINTER(ctypes.c_double)]
     lib.fastnn_kernel_timer_read.restype = I
     lib.fastnn_last_cuda_error.argtypes = []
@@ -313,6 +315,18 @@ def fastnn_noalloc_device_status(stream=None) -> int:
 def fastnn_kernel_timer_enable(capacity: int) -> None:
     """Time the next ``capacity`` nearest-neighbour kernel launches with CUDA events."""
     _check(library().fastnn_kernel_timer_enable(int(capacity)), "fastnn_kernel_timer_enable")
+
+
+FASTNN_TIME_MATCHING = 1
+FASTNN_TIME_REPACK = 2
+FASTNN_TIME_MUTUAL = 4
+FASTNN_TIME_MASK = 8
+
+
+def fastnn_kernel_timer_select(kinds: int) -> int:
+    """Choose which launch kinds the timer brackets (FASTNN_TIME_* bit mask);
+    returns the previous selection."""
+    return int(library().fastnn_kernel_timer_select(int(kinds)))
 
 
 def fastnn_kernel_timer_read():

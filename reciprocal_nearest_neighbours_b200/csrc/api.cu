@@ -566,6 +566,8 @@ int fastnn_device_status(const void* workspace, fastnn_stream_t stream) {
 
 int fastnn_kernel_timer_enable(int capacity) { return kernel_timer_enable(capacity); }
 
+int fastnn_kernel_timer_select(int kinds) { return kernel_timer_select(kinds); }
+
 void fastnn_set_wait_timeout_ns(uint64_t ns) { g_wait_ns.store(ns); }
 
 int fastnn_kernel_timer_read(int* launches, double* total_ms) {

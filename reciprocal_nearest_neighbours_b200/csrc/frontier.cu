@@ -7,6 +7,7 @@
 #include "common.cuh"
 #include "frontier.cuh"
 #include "frontier_dev.cuh"
+#include "nn_tc.cuh"
 
 namespace fastnn {
 
@@ -61,6 +62,76 @@ __global__ void repack_kernel(const uint8_t* __restrict__ src, int64_t rows, int
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = max(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     if ((threadIdx.x & 31) == 0 && amax > 0) atomicMax(absmax, amax);
+  }
+}
+
+// Staged repack for source rows of a whole number of 8-byte words (int8
+// d = 8, 16, 24, 32, ...; 16-bit d = 4, 8, 12, ...) from a 16-byte aligned
+// source: a block copies a run of kRepackRows rows with coalesced 16-byte
+// loads into shared memory (kRepackRows * nbytes is a multiple of 16, so every
+// run starts 16-byte aligned), then writes the run's padded rows with
+// coalesced 16-byte stores, each thread assembling its output chunk from two
+// 8-byte words of the staged rows. This is a pure stream: every input byte is
+// read once and every output byte written once.
+constexpr int kRepackRows = 256;
+constexpr int kRepackThreads = 256;
+
+template <int RB>
+__global__ void __launch_bounds__(kRepackThreads)
+    repack_staged_kernel(const uint8_t* __restrict__ src, int64_t rows, int nbytes,
+                         uint8_t* __restrict__ dst, int64_t pad_rows, int* absmax) {
+  constexpr int kOutChunks = kRepackRows * RB / 16;  // 16-byte output chunks of a run
+  __shared__ __align__(16) uint8_t stage[kRepackRows * RB];  // nbytes <= RB per row
+  const int64_t total = rows + pad_rows;
+  const int64_t runs = (total + kRepackRows - 1) / kRepackRows;
+  const int64_t in_bytes = rows * nbytes;
+  uint32_t amax = 0;  // per-byte maxima of |x| (int8 maps only)
+  for (int64_t run = blockIdx.x; run < runs; run += gridDim.x) {
+    const int64_t r0 = run * kRepackRows;
+    const int64_t b0 = r0 * nbytes;  // first source byte of the run (16-byte aligned)
+    const int run_bytes = static_cast<int>(
+        max(static_cast<int64_t>(0), min(static_cast<int64_t>(kRepackRows) * nbytes, in_bytes - b0)));
+    // Load: full 16-byte chunks, then the run's ragged tail (at most 15 bytes).
+    const int full = run_bytes / 16;
+    for (int c = threadIdx.x; c < full; c += kRepackThreads) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + b0) + c);
+      reinterpret_cast<uint4*>(stage)[c] = v;
+      if (absmax) {
+        amax = __vmaxu4(amax, __vabs4(v.x));
+        amax = __vmaxu4(amax, __vabs4(v.y));
+        amax = __vmaxu4(amax, __vabs4(v.z));
+        amax = __vmaxu4(amax, __vabs4(v.w));
+      }
+    }
+    if (static_cast<int>(threadIdx.x) < run_bytes - 16 * full) {
+      const int i = 16 * full + threadIdx.x;
+      const uint8_t x = __ldg(src + b0 + i);
+      stage[i] = x;
+      if (absmax) amax = __vmaxu4(amax, __vabs4(static_cast<uint32_t>(x) * 0x01010101u) & 0xFFu);
+    }
+    __syncthreads();
+    // Store: output chunk k covers bytes [16 (k mod RB/16), +16) of row k / (RB/16).
+    for (int k = threadIdx.x; k < kOutChunks; k += kRepackThreads) {
+      const int r = k / (RB / 16);
+      const int off = 16 * (k % (RB / 16));
+      const int64_t row = r0 + r;
+      if (row >= total) break;
+      uint2 lo = make_uint2(0, 0), hi = make_uint2(0, 0);
+      if (row < rows) {
+        const uint8_t* srow = stage + r * nbytes;  // 8-byte aligned: nbytes % 8 == 0
+        if (off < nbytes) lo = *reinterpret_cast<const uint2*>(srow + off);
+        if (off + 8 < nbytes) hi = *reinterpret_cast<const uint2*>(srow + off + 8);
+      }
+      reinterpret_cast<uint4*>(dst + row * RB)[off / 16] = make_uint4(lo.x, lo.y, hi.x, hi.y);
+    }
+    __syncthreads();
+  }
+  if (absmax) {
+    int m = static_cast<int>(max(max(amax & 0xFFu, (amax >> 8) & 0xFFu),
+                                 max((amax >> 16) & 0xFFu, amax >> 24)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31) == 0 && m > 0) atomicMax(absmax, m);
   }
 }
 
@@ -438,7 +509,7 @@ __global__ void __launch_bounds__(1024) masked_seeds_kernel(const int32_t* __res
 
 int mask_blocks(int64_t N) { return static_cast<int>((N + 1023) / 1024); }
 
-int launch_mask_compact(const MaskArgs& m0, int dtype, cudaStream_t st) {
+static int launch_mask_compact_impl(const MaskArgs& m0, int dtype, cudaStream_t st) {
   MaskArgs m = m0;
   m.bpp = mask_blocks(m.N);
   const int nb = m.batch * m.bpp;
@@ -457,6 +528,14 @@ int launch_mask_compact(const MaskArgs& m0, int dtype, cudaStream_t st) {
   return FASTNN_OK;
 }
 
+int launch_mask_compact(const MaskArgs& m0, int dtype, cudaStream_t st) {
+  const int slot = kernel_timer_begin(st, kTimeMask);
+  if (slot == -2) return FASTNN_ERR_CUDA;
+  const int rc = launch_mask_compact_impl(m0, dtype, st);
+  if (rc != FASTNN_OK) return rc;
+  return kernel_timer_end(slot, st);
+}
+
 int launch_masked_seeds(const int32_t* p2c, int batch, int64_t N1, int W1, int sub, int64_t S,
                         int32_t* F0, int32_t* seed_cnt, cudaStream_t st) {
   masked_seeds_kernel<<<batch, 1024, 0, st>>>(p2c, N1, W1, sub, S, F0, seed_cnt);
@@ -464,7 +543,7 @@ int launch_masked_seeds(const int32_t* p2c, int batch, int64_t N1, int W1, int s
   return FASTNN_OK;
 }
 
-int launch_repack(const void* src, int64_t rows, int d, int dtype, void* dst, int64_t pad_rows,
+static int launch_repack_impl(const void* src, int64_t rows, int d, int dtype, void* dst, int64_t pad_rows,
                   int* absmax, cudaStream_t st) {
   const int64_t total = rows + pad_rows;
   if (total <= 0) return FASTNN_OK;
@@ -474,6 +553,28 @@ int launch_repack(const void* src, int64_t rows, int d, int dtype, void* dst, in
   if (dtype == FASTNN_F32_L2) {
     repack_l2_kernel<<<g, 256, 0, st>>>(static_cast<const float*>(src), rows, d,
                                         static_cast<float4*>(dst), pad_rows, absmax);
+    FASTNN_CUDA_TRY(cudaGetLastError());
+    return FASTNN_OK;
+  }
+  const int nbytes = d * elem_bytes(dtype);
+  if (nbytes % 8 == 0 && reinterpret_cast<uintptr_t>(src) % 16 == 0) {
+    // Staged stream copy; the grid covers the runs up to 148 SMs x 8 blocks.
+    const int64_t runs = (total + kRepackRows - 1) / kRepackRows;
+    const int gs = static_cast<int>(min(runs, static_cast<int64_t>(148 * 8)));
+    int* am = dtype == FASTNN_I8 ? absmax : nullptr;
+    switch (row_bytes(dtype, d)) {
+      case 32:
+        repack_staged_kernel<32><<<gs, kRepackThreads, 0, st>>>(s8, rows, nbytes, d8, pad_rows, am);
+        break;
+      case 64:
+        repack_staged_kernel<64><<<gs, kRepackThreads, 0, st>>>(s8, rows, nbytes, d8, pad_rows, am);
+        break;
+      case 128:
+        repack_staged_kernel<128><<<gs, kRepackThreads, 0, st>>>(s8, rows, nbytes, d8, pad_rows, am);
+        break;
+      default:
+        return FASTNN_ERR_UNSUPPORTED;
+    }
     FASTNN_CUDA_TRY(cudaGetLastError());
     return FASTNN_OK;
   }
@@ -497,9 +598,18 @@ int launch_repack(const void* src, int64_t rows, int d, int dtype, void* dst, in
   return FASTNN_OK;
 }
 
+int launch_repack(const void* src, int64_t rows, int d, int dtype, void* dst, int64_t pad_rows,
+                  int* absmax, cudaStream_t st) {
+  const int slot = kernel_timer_begin(st, kTimeRepack);
+  if (slot == -2) return FASTNN_ERR_CUDA;
+  const int rc = launch_repack_impl(src, rows, d, dtype, dst, pad_rows, absmax, st);
+  if (rc != FASTNN_OK) return rc;
+  return kernel_timer_end(slot, st);
+}
+
 int mutual_blocks(int64_t n1) { return static_cast<int>((n1 + 1023) / 1024); }
 
-int launch_mutual(const MutualSrc& m, int32_t* block_scratch, int dtype, int32_t* out_pairs,
+static int launch_mutual_impl(const MutualSrc& m, int32_t* block_scratch, int dtype, int32_t* out_pairs,
                   void* out_score, int64_t cap, int32_t* out_count, cudaStream_t st) {
   const int nb = mutual_blocks(m.n1);
   mutual_count_kernel<<<nb, 1024, 0, st>>>(m, block_scratch);
@@ -516,6 +626,16 @@ int launch_mutual(const MutualSrc& m, int32_t* block_scratch, int dtype, int32_t
   return FASTNN_OK;
 }
 
+int launch_mutual(const MutualSrc& m, int32_t* block_scratch, int dtype, int32_t* out_pairs,
+                  void* out_score, int64_t cap, int32_t* out_count, cudaStream_t st) {
+  const int slot = kernel_timer_begin(st, kTimeMutual);
+  if (slot == -2) return FASTNN_ERR_CUDA;
+  const int rc =
+      launch_mutual_impl(m, block_scratch, dtype, out_pairs, out_score, cap, out_count, st);
+  if (rc != FASTNN_OK) return rc;
+  return kernel_timer_end(slot, st);
+}
+
 int launch_chunk_boxes(const float4* rows, int64_t N, int batch, const int32_t* count,
                        float4* box, cudaStream_t st) {
   const int nchunk = static_cast<int>((N + kL2Chunk - 1) / kL2Chunk);
@@ -525,7 +645,7 @@ int launch_chunk_boxes(const float4* rows, int64_t N, int batch, const int32_t* 
   return FASTNN_OK;
 }
 
-int launch_image_list(const uint64_t* k12, int64_t n1, int64_t n2, uint32_t* first,
+static int launch_image_list_impl(const uint64_t* k12, int64_t n1, int64_t n2, uint32_t* first,
                       uint32_t* best, int32_t* pos, int32_t* list, uint32_t* list_bound,
                       int32_t* count, int32_t* block_scratch, cudaStream_t st) {
   const int nb = mutual_blocks(n1);
@@ -536,6 +656,17 @@ int launch_image_list(const uint64_t* k12, int64_t n1, int64_t n2, uint32_t* fir
                                          list_bound);
   FASTNN_CUDA_TRY(cudaGetLastError());
   return FASTNN_OK;
+}
+
+int launch_image_list(const uint64_t* k12, int64_t n1, int64_t n2, uint32_t* first,
+                      uint32_t* best, int32_t* pos, int32_t* list, uint32_t* list_bound,
+                      int32_t* count, int32_t* block_scratch, cudaStream_t st) {
+  const int slot = kernel_timer_begin(st, kTimeMutual);
+  if (slot == -2) return FASTNN_ERR_CUDA;
+  const int rc = launch_image_list_impl(k12, n1, n2, first, best, pos, list, list_bound, count,
+                                        block_scratch, st);
+  if (rc != FASTNN_OK) return rc;
+  return kernel_timer_end(slot, st);
 }
 
 int launch_decode(const uint64_t* key, int64_t n, int dtype, int32_t* out_idx, void* out_score,

@@ -589,7 +589,7 @@ int launch_nn_l2(const NNArgs& a, cudaStream_t stream) {
   if (rc != FASTNN_OK) return rc;
   FASTNN_CUDA_TRY(cudaFuncSetAttribute(nn_l2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSmemBytes)));
-  const int slot = kernel_timer_begin(stream);
+  const int slot = kernel_timer_begin(stream, kTimeMatching);
   if (slot == -2) return FASTNN_ERR_CUDA;
   nn_l2_kernel<<<sms, kThreads, kSmemBytes, stream>>>(a);
   FASTNN_CUDA_TRY(cudaGetLastError());
@@ -610,7 +610,7 @@ int launch_reciprocal_l2(const RecArgs& r, cudaStream_t stream) {
   if (per_sm < 1) return FASTNN_ERR_UNSUPPORTED;
   RecArgs args = r;
   void* params[] = {&args};
-  const int slot = kernel_timer_begin(stream);
+  const int slot = kernel_timer_begin(stream, kTimeMatching);
   if (slot == -2) return FASTNN_ERR_CUDA;
   FASTNN_CUDA_TRY(
       cudaLaunchCooperativeKernel(fn, dim3(sms), dim3(kThreads), params, kSmemBytes, stream));

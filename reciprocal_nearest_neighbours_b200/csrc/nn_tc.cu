@@ -735,24 +735,28 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Pha
             uint32_t r[kChunks][16];
             static_assert(kChunks * 16 == 64, "one packed 128-column load");
             ptx::tmem_ld64_pack(taddr, reinterpret_cast<uint32_t(&)[64]>(r));
-            ptx::tmem_ld_wait();
-            // The accumulator is free for the next MMA once it is in registers.
+            ptx::tmem_ld_wait_regs(reinterpret_cast<uint32_t(&)[64]>(r));
+            // The accumulator is free for the next MMA once it is in registers:
+            // release it before any of the fold (the pin keeps the fold's
+            // register-only work from being scheduled ahead of the arrive).
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(rel_bar);
+            ptx::pin_regs(reinterpret_cast<uint32_t(&)[64]>(r));
             if constexpr (DT == FASTNN_I8) fold_pack16<kChunks>(r, colbase, best, bidx, slot);
           } else {
             // 32-bit scores: two 64-column halves, the accumulator is released
             // after the second load.
             uint32_t r[2][32];
             ptx::tmem_ld64(taddr, reinterpret_cast<uint32_t(&)[64]>(r));
-            ptx::tmem_ld_wait();
+            ptx::tmem_ld_wait_regs(reinterpret_cast<uint32_t(&)[64]>(r));
             fold_wide<DT, 2>(r, colbase, best, bidx, slot);
             ptx::tmem_ld64(taddr + 64, reinterpret_cast<uint32_t(&)[64]>(r));
-            ptx::tmem_ld_wait();
+            ptx::tmem_ld_wait_regs(reinterpret_cast<uint32_t(&)[64]>(r));
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(rel_bar);
+            ptx::pin_regs(reinterpret_cast<uint32_t(&)[64]>(r));
             fold_wide<DT, 2>(r, colbase + 64, best, bidx, slot);
           }
         }
@@ -859,17 +863,20 @@ struct KernelTimer {
   cudaEvent_t* ev = nullptr;  // 2 * cap events
   int cap = 0;
   int used = 0;
+  int kinds = kTimeMatching;  // which launch kinds are bracketed
 };
 KernelTimer g_timer;
 
 }  // namespace
 
 int kernel_timer_enable(int capacity) {
+  const int kinds = g_timer.kinds;
   if (g_timer.ev) {
     for (int i = 0; i < 2 * g_timer.cap; ++i) cudaEventDestroy(g_timer.ev[i]);
     delete[] g_timer.ev;
     g_timer = KernelTimer{};
   }
+  g_timer.kinds = kinds;
   if (capacity <= 0) return FASTNN_OK;
   g_timer.ev = new cudaEvent_t[2 * capacity];
   for (int i = 0; i < 2 * capacity; ++i)
@@ -877,10 +884,17 @@ int kernel_timer_enable(int capacity) {
       for (int j = 0; j < i; ++j) cudaEventDestroy(g_timer.ev[j]);
       delete[] g_timer.ev;
       g_timer = KernelTimer{};
+      g_timer.kinds = kinds;
       return FASTNN_ERR_CUDA;
     }
   g_timer.cap = capacity;
   return FASTNN_OK;
+}
+
+int kernel_timer_select(int kinds) {
+  const int old = g_timer.kinds;
+  if (kinds > 0) g_timer.kinds = kinds;
+  return old;
 }
 
 int kernel_timer_read(int* launches, double* total_ms) {
@@ -925,7 +939,8 @@ int sm_count(int* sms) {
   return FASTNN_OK;
 }
 
-int timer_begin(cudaStream_t stream) {
+int timer_begin(cudaStream_t stream, int kind) {
+  if (!(g_timer.kinds & kind)) return -1;
   const int slot = (g_timer.ev && g_timer.used < g_timer.cap) ? g_timer.used++ : -1;
   if (slot >= 0 && cudaEventRecord(g_timer.ev[2 * slot], stream) != cudaSuccess) return -2;
   return slot;
@@ -938,7 +953,7 @@ int timer_end(int slot, cudaStream_t stream) {
 
 }  // namespace
 
-int kernel_timer_begin(cudaStream_t stream) { return timer_begin(stream); }
+int kernel_timer_begin(cudaStream_t stream, int kind) { return timer_begin(stream, kind); }
 int kernel_timer_end(int slot, cudaStream_t stream) { return timer_end(slot, stream); }
 int device_sm_count(int* sms) { return sm_count(sms); }
 
@@ -982,7 +997,7 @@ int launch_nn_tc(const NNArgs& a, int dtype, int64_t db_total_rows, cudaStream_t
                                        static_cast<int>(smem)));
   NNArgs args = a;
   void* params[] = {&tm, &args};
-  const int slot = timer_begin(stream);
+  const int slot = timer_begin(stream, kTimeMatching);
   if (slot == -2) return FASTNN_ERR_CUDA;
   FASTNN_CUDA_TRY(cudaLaunchKernel(fn, dim3(sms), dim3(kThreads), params, smem, stream));
   return timer_end(slot, stream);
@@ -1009,7 +1024,7 @@ int launch_reciprocal(const RecArgs& r, int dtype, int64_t d1_rows, int64_t d2_r
   if (per_sm < 1) return FASTNN_ERR_UNSUPPORTED;
   RecArgs args = r;
   void* params[] = {&tm2, &tm1, &args};
-  const int slot = timer_begin(stream);
+  const int slot = timer_begin(stream, kTimeMatching);
   if (slot == -2) return FASTNN_ERR_CUDA;
   FASTNN_CUDA_TRY(cudaLaunchCooperativeKernel(fn, dim3(sms), dim3(kThreads), params, smem, stream));
   return timer_end(slot, stream);

@@ -15,12 +15,18 @@ int nn_tc_max_batch();
 // Launch on `stream`. a.db_rows holds `db_total_rows` repacked rows (all
 // pairs back to back plus zero padding), 16-byte aligned. Returns a
 // fastnn_status.
-// Benchmark instrumentation behind fastnn_kernel_timer_enable/_read. A
-// launcher brackets its kernel with kernel_timer_begin (returns a slot, -1
-// when the timer is off or full, -2 on a CUDA error) and kernel_timer_end.
+// Benchmark instrumentation behind fastnn_kernel_timer_enable/_select/_read.
+// A launcher brackets its kernel(s) of one kind with kernel_timer_begin
+// (returns a slot; -1 when the timer is off, full or not selecting that
+// kind; -2 on a CUDA error) and kernel_timer_end.
+constexpr int kTimeMatching = 1;  // nearest-neighbour and persistent matching kernels
+constexpr int kTimeRepack = 2;    // repack of a descriptor map
+constexpr int kTimeMutual = 4;    // mutual test and ordered emit (and the dense image list)
+constexpr int kTimeMask = 8;      // confidence-mask compaction of a map
 int kernel_timer_enable(int capacity);
+int kernel_timer_select(int kinds);
 int kernel_timer_read(int* launches, double* total_ms);
-int kernel_timer_begin(cudaStream_t stream);
+int kernel_timer_begin(cudaStream_t stream, int kind);
 int kernel_timer_end(int slot, cudaStream_t stream);
 // Multiprocessors of the current device.
 int device_sm_count(int* sms);

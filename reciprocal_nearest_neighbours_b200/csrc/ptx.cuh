@@ -218,6 +218,25 @@ __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// Re-defines registers in an empty statement: no computation on their values
+// can be scheduled before this point (e.g. before an mbarrier arrive that must
+// be issued as early as possible).
+template <int N>
+__device__ __forceinline__ void pin_regs(uint32_t (&r)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
+
+// tcgen05.wait::ld for registers an earlier tcgen05.ld filled: the empty
+// statements after the wait re-define them, so no use of their values can be
+// scheduled before the wait (the load is asynchronous until it).
+template <int N>
+__device__ __forceinline__ void tmem_ld_wait_regs(uint32_t (&r)[N]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
+
 // Shared-memory matrix descriptor for a K-major operand tile whose rows are
 // `row_bytes` (32, 64 or 128) long and stored with the matching 32B / 64B /
 // 128B swizzle (8-row groups, consecutive rows): start address, leading

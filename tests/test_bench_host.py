@@ -43,3 +43,32 @@ def test_reference_arm_prints_one_json_line():
     assert j["metric"].startswith("dense mutual")
     assert j["cpu_baseline"]["kind"] == "oracle" and j["cpu_baseline"]["value"] == j["value"]
     assert j["e2e"]["h2d_bytes_per_step"] == 0 and j["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_gpus_n_starts_n_ranks_that_reduce_over_gloo():
+    """``bench.py --gpus 2`` outside a launcher starts two ranks itself (local
+    rendezvous); their sum and max reductions reach rank 0, which alone
+    prints, with n_gpus equal to the rank count."""
+    out = subprocess.run([sys.executable, "bench.py", "--gpus", "2", "--selftest-launcher"],
+                         cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [json.loads(x) for x in out.stdout.splitlines() if x.startswith("{")]
+    assert lines == [{"selftest": "launcher", "n_gpus": 2, "rank_sum": 3.0, "rank_max": 1.0}]
+
+
+def test_headline_nests_the_other_configurations_by_default():
+    old = sys.argv
+    try:
+        sys.argv = ["bench.py"]
+        a = bench.parse_args()
+        assert a.workload == bench.DEFAULT_WORKLOAD and a.gpus == 1
+        assert a.also.split(",") == bench.NESTED_DEFAULT
+        sys.argv = ["bench.py", "--workload", "pair_512x384_d24_bf16"]
+        assert bench.parse_args().also == ""
+        sys.argv = ["bench.py", "--also", ""]
+        assert bench.parse_args().also == ""
+    finally:
+        sys.argv = old
+    assert set(bench.NESTED_DEFAULT) <= set(synth.CONFIGS)
+    p = bench.percentiles([float(x) for x in range(1, 101)])
+    assert (p["p10"], p["p50"], p["p90"]) == (11.0, 51.0, 91.0)
