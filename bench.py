@@ -677,8 +677,9 @@ def measure_stream(K, ranks, dev, stream, flush, sample_clocks):
                  2 x 8 B read per row, 16 B per kept pair);
       mask    -- fastnn_mutual_dense_masked of the 64M-row map (confidences
                  uniform in [0, 1), threshold 0.5) against a 256-row map
-                 (map 1's compaction: 2 x 4 B of confidence per row, and per
-                 kept row 24 B read, 32 + 4 B written).
+                 (map 1's compaction: 2 x 4 B of confidence and the 24 B row
+                 read per pixel, 32 B repacked row + 4 B pixel index written
+                 per kept pixel).
     Inputs are drawn on the device from a seeded generator."""
     import torch
     import reciprocal_nearest_neighbours_b200 as fnn
@@ -757,7 +758,7 @@ def measure_stream(K, ranks, dev, stream, flush, sample_clocks):
               lambda: fnn.fastnn_mutual_dense_masked(A, db, conf1=conf, threshold=0.5,
                                                      out_pairs=mp, out_score=ms_, out_count=cnt,
                                                      workspace=wsm),
-              lambda: 8 * N + kept1 * (d + 36) + 8 * 256 + 256 * (d + 36))
+              lambda: 8 * N + N * d + kept1 * 36 + 256 * (8 + d + 36))
     r["kind"] = ("confidence-mask compaction (mask_count, scan, mask_emit) of the 64M-row map "
                  "and of the 256-row map")
     r["kept"] = kept1

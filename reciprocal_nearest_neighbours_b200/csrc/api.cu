@@ -133,7 +133,7 @@ MutLayout carve_mut(Carver& c, int64_t n1, int64_t n2, int d, int dtype) {
   L.pos21 = c.take<int32_t>(static_cast<size_t>(n2));
   L.list21 = c.take<int32_t>(static_cast<size_t>(n2));
   L.cnt21 = c.take<int32_t>(1);
-  L.blocks2 = c.take<int32_t>(static_cast<size_t>(mutual_blocks(n1)));
+  L.blocks2 = c.take<int32_t>(static_cast<size_t>(image_blocks(n1)));
   L.first21 = c.take<uint32_t>(static_cast<size_t>(n2));
   L.best21 = c.take<uint32_t>(static_cast<size_t>(n2));
   L.bnd21 = c.take<uint32_t>(static_cast<size_t>(n2));

@@ -141,62 +141,117 @@ __global__ void __launch_bounds__(kRepackThreads)
 // scores (a row shard of image 1 checked against the full NN21 gathered from
 // every rank). Three passes keep the output in ascending i without inter-CTA
 // waiting: per-block counts, one scan block, ordered emit.
-__device__ __forceinline__ bool mutual_flag(const MutualSrc& m, int64_t i, uint32_t& j) {
-  if (i >= m.n1) return false;
-  j = m.k12 ? key_index(m.k12[i]) : static_cast<uint32_t>(m.nn12[i]);
-  if (j >= static_cast<uint64_t>(m.n2)) return false;
-  const uint32_t back = m.k21 ? key_index(m.k21[m.pos21 ? m.pos21[j] : j])
-                              : static_cast<uint32_t>(m.nn21[j]);
-  return back == static_cast<uint32_t>(m.i0 + i);
+// A block of 1024 threads covers kMutBlockRows rows; thread t takes the four
+// consecutive rows 4t .. 4t + 3, read with 16-byte loads where aligned.
+constexpr int kMutRowsPerThread = 4;
+constexpr int kMutBlockRows = 1024 * kMutRowsPerThread;
+
+// Flags (and partners) of rows i .. i + 3 (local indices). The partners'
+// back-matches are loaded together, after all four partners are known.
+__device__ __forceinline__ void mutual_flags4(const MutualSrc& m, int64_t i, bool (&f)[4],
+                                              uint32_t (&j)[4]) {
+  const bool full = i + 3 < m.n1;
+  if (m.k12) {
+    uint64_t k[4] = {0, 0, 0, 0};
+    if (full && (reinterpret_cast<uintptr_t>(m.k12 + i) & 15) == 0) {
+      const ulonglong2 a = *reinterpret_cast<const ulonglong2*>(m.k12 + i);
+      const ulonglong2 b = *reinterpret_cast<const ulonglong2*>(m.k12 + i + 2);
+      k[0] = a.x; k[1] = a.y; k[2] = b.x; k[3] = b.y;
+    } else {
+#pragma unroll
+      for (int r = 0; r < 4; ++r) k[r] = i + r < m.n1 ? m.k12[i + r] : 0;
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) j[r] = key_index(k[r]);
+  } else {
+    if (full && (reinterpret_cast<uintptr_t>(m.nn12 + i) & 15) == 0) {
+      const int4 a = *reinterpret_cast<const int4*>(m.nn12 + i);
+      j[0] = a.x; j[1] = a.y; j[2] = a.z; j[3] = a.w;
+    } else {
+#pragma unroll
+      for (int r = 0; r < 4; ++r) j[r] = i + r < m.n1 ? static_cast<uint32_t>(m.nn12[i + r]) : 0xFFFFFFFFu;
+    }
+  }
+  uint32_t back[4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const bool ok = i + r < m.n1 && j[r] < static_cast<uint64_t>(m.n2);
+    back[r] = !ok ? 0xFFFFFFFFu
+              : m.k21 ? key_index(m.k21[m.pos21 ? m.pos21[j[r]] : j[r]])
+                      : static_cast<uint32_t>(m.nn21[j[r]]);
+    f[r] = ok && back[r] == static_cast<uint32_t>(m.i0 + i + r);
+  }
 }
 
 __global__ void __launch_bounds__(1024) mutual_count_kernel(MutualSrc m,
                                                             int32_t* __restrict__ block_cnt) {
-  __shared__ int sm[64];
-  const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
-  uint32_t j;
-  const bool f = mutual_flag(m, i, j);
-  const Scan2 sc = block_scan2(f, false, sm);
-  if (threadIdx.x == 0) block_cnt[blockIdx.x] = sc.tot0;
+  __shared__ int sm[32];
+  const int64_t i = blockIdx.x * static_cast<int64_t>(kMutBlockRows) + 4 * threadIdx.x;
+  bool f[4];
+  uint32_t j[4];
+  mutual_flags4(m, i, f, j);
+  int c = (f[0] ? 1 : 0) + (f[1] ? 1 : 0) + (f[2] ? 1 : 0) + (f[3] ? 1 : 0);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+  if ((threadIdx.x & 31) == 0) sm[threadIdx.x >> 5] = c;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int t = 0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) t += sm[w];
+    block_cnt[blockIdx.x] = t;
+  }
+}
+
+// Block-wide exclusive scan of one small count per thread; `sm` holds 32 ints.
+__device__ __forceinline__ int block_exclusive_scan(int c, int* sm) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sm[warp] = x;
+  __syncthreads();
+  int off = 0;
+  for (int w = 0; w < warp; ++w) off += sm[w];
+  return off + x - c;
 }
 
 // Exclusive scan, in place, of the nblocks counts of segment blockIdx.x
 // (block_cnt + blockIdx.x * nblocks); the segment's total goes to
-// out_count[blockIdx.x].
+// out_count[blockIdx.x]. Each thread scans a contiguous run of the counts;
+// one block-wide scan of the runs' totals joins them (a single pass, however
+// many counts).
 __global__ void __launch_bounds__(1024) mutual_scan_kernel(int32_t* __restrict__ block_cnt,
                                                            int nblocks,
                                                            int32_t* __restrict__ out_count) {
   block_cnt += static_cast<int64_t>(blockIdx.x) * nblocks;
   out_count += blockIdx.x;
-  __shared__ int sm[64];
-  __shared__ int carry;
-  if (threadIdx.x == 0) carry = 0;
-  __syncthreads();
-  for (int s = 0; s < nblocks; s += blockDim.x) {
-    const int k = s + threadIdx.x;
-    const int v = k < nblocks ? block_cnt[k] : 0;
-    // exclusive scan of counts via per-thread value: warp shuffles + smem
-    int x = v;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __shared__ int sm[32];
+  const int per = (nblocks + static_cast<int>(blockDim.x) - 1) / static_cast<int>(blockDim.x);
+  const int k0 = min(static_cast<int>(threadIdx.x) * per, nblocks);
+  const int k1 = min(k0 + per, nblocks);
+  int sum = 0;
+  for (int k = k0; k < k1; ++k) sum += block_cnt[k];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = sum;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
-    }
-    if (lane == 31) sm[warp] = x;
-    __syncthreads();
-    int woff = 0, tot = 0;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
-      if (w < warp) woff += sm[w];
-      tot += sm[w];
-    }
-    const int c0 = carry;
-    if (k < nblocks) block_cnt[k] = c0 + woff + x - v;
-    __syncthreads();
-    if (threadIdx.x == 0) carry = c0 + tot;
-    __syncthreads();
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
   }
-  if (threadIdx.x == 0) *out_count = carry;
+  if (lane == 31) sm[warp] = x;
+  __syncthreads();
+  int woff = 0;
+  for (int w = 0; w < warp; ++w) woff += sm[w];
+  int run = woff + x - sum;  // exclusive prefix of this thread's run
+  for (int k = k0; k < k1; ++k) {
+    const int v = block_cnt[k];
+    block_cnt[k] = run;
+    run += v;
+  }
+  if (threadIdx.x == blockDim.x - 1) *out_count = run;
 }
 
 template <int DT>
@@ -205,19 +260,29 @@ __global__ void __launch_bounds__(1024) mutual_emit_kernel(MutualSrc m,
                                                            int32_t* __restrict__ out_pairs,
                                                            void* __restrict__ out_score,
                                                            int64_t cap) {
-  __shared__ int sm[64];
-  const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
-  uint32_t j = 0;
-  const bool f = mutual_flag(m, i, j);
-  const Scan2 sc = block_scan2(f, false, sm);
-  if (f) {
-    const int64_t pos = block_off[blockIdx.x] + sc.ex0;
+  __shared__ int sm[32];
+  const int64_t i = blockIdx.x * static_cast<int64_t>(kMutBlockRows) + 4 * threadIdx.x;
+  bool f[4];
+  uint32_t j[4];
+  mutual_flags4(m, i, f, j);
+  const int c = (f[0] ? 1 : 0) + (f[1] ? 1 : 0) + (f[2] ? 1 : 0) + (f[3] ? 1 : 0);
+  int64_t pos = block_off[blockIdx.x] + block_exclusive_scan(c, sm);
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    if (!f[r]) continue;
     if (pos < cap) {
-      out_pairs[pos * 2] = m.map1 ? m.map1[i] : static_cast<int32_t>(m.i0 + i);
-      out_pairs[pos * 2 + 1] = m.map2 ? m.map2[j] : static_cast<int32_t>(j);
+      const int64_t ir = i + r;
+      const int32_t a = m.map1 ? m.map1[ir] : static_cast<int32_t>(m.i0 + ir);
+      const int32_t bj = m.map2 ? m.map2[j[r]] : static_cast<int32_t>(j[r]);
+      if ((reinterpret_cast<uintptr_t>(out_pairs) & 7) == 0) {
+        *reinterpret_cast<int2*>(out_pairs + pos * 2) = make_int2(a, bj);
+      } else {
+        out_pairs[pos * 2] = a;
+        out_pairs[pos * 2 + 1] = bj;
+      }
       if (out_score) {
         if (m.k12) {
-          const uint32_t h = key_score_bits(m.k12[i]);
+          const uint32_t h = key_score_bits(m.k12[ir]);
           if (DT == FASTNN_I8)
             static_cast<int32_t*>(out_score)[pos] = unord_i32(h);
           else if (DT == FASTNN_F32_L2)
@@ -226,12 +291,13 @@ __global__ void __launch_bounds__(1024) mutual_emit_kernel(MutualSrc m,
             static_cast<float*>(out_score)[pos] = unord_f32(h);
         } else if (m.score12) {
           if (DT == FASTNN_I8)
-            static_cast<int32_t*>(out_score)[pos] = static_cast<const int32_t*>(m.score12)[i];
+            static_cast<int32_t*>(out_score)[pos] = static_cast<const int32_t*>(m.score12)[ir];
           else
-            static_cast<float*>(out_score)[pos] = static_cast<const float*>(m.score12)[i];
+            static_cast<float*>(out_score)[pos] = static_cast<const float*>(m.score12)[ir];
         }
       }
     }
+    ++pos;
   }
 }
 
@@ -481,6 +547,80 @@ __global__ void __launch_bounds__(1024) mask_emit_kernel(MaskArgs m) {
   }
 }
 
+// Staged form of the ordered scatter, for descriptor rows of a whole number
+// of 8-byte words in a 16-byte aligned map whose pairs start 16-byte aligned.
+// Block blk of pair b covers the same 1024 pixels as mask_count_kernel's: it
+// loads their rows with coalesced 16-byte loads into shared memory
+// (1024 * nbytes bytes of dynamic shared memory), then places and writes the
+// kept rows in four rounds of 256 pixels.
+constexpr int kMaskEmitThreads = 256;
+
+template <int RB, bool I8>
+__global__ void __launch_bounds__(kMaskEmitThreads) mask_emit_staged_kernel(MaskArgs m,
+                                                                            int nbytes) {
+  extern __shared__ __align__(16) uint8_t stage[];
+  __shared__ int sm[64];
+  const int b = blockIdx.x / m.bpp, blk = blockIdx.x % m.bpp;
+  const int tid = static_cast<int>(threadIdx.x);
+  const int64_t p0 = static_cast<int64_t>(blk) * 1024;
+  const int rows = static_cast<int>(min(static_cast<int64_t>(1024), m.N - p0));
+  const uint8_t* src = m.src + (b * m.N + p0) * nbytes;
+  const int bytes = rows * nbytes;  // a multiple of 8
+  for (int c = tid; c < bytes / 16; c += kMaskEmitThreads)
+    reinterpret_cast<uint4*>(stage)[c] = __ldg(reinterpret_cast<const uint4*>(src) + c);
+  if (tid == 0 && (bytes & 15))
+    *reinterpret_cast<uint2*>(stage + bytes - 8) =
+        __ldg(reinterpret_cast<const uint2*>(src + bytes - 8));
+  // Four rounds of 256 pixels; in round r thread t takes pixel p0 + 256 r + t,
+  // so a round's kept rows go to consecutive slots from consecutive threads.
+  // The first scan's barriers also publish the staged rows.
+  int64_t base = b * m.N + m.blocks[blockIdx.x];
+  uint32_t amax = 0;  // per-byte maxima of |x| (int8)
+#pragma unroll 1
+  for (int r = 0; r < 1024 / kMaskEmitThreads; ++r) {
+    const int lr = r * kMaskEmitThreads + tid;  // row within the block
+    const int64_t p = p0 + lr;
+    const int64_t g = b * m.N + p;
+    const bool f = lr < rows && mask_kept(m, g);
+    const Scan2 sc = block_scan2(f, false, sm);
+    const int64_t slot = base + sc.ex0;
+    base += sc.tot0;
+    if (lr < rows && m.p2c) m.p2c[g] = f ? static_cast<int32_t>(slot - b * m.N) : -1;
+    if (!f) continue;
+    m.c2p[slot] = static_cast<int32_t>(p);
+    const uint8_t* srow = stage + lr * nbytes;  // 8-byte aligned
+    uint4* o = reinterpret_cast<uint4*>(m.dst + slot * RB);
+#pragma unroll
+    for (int c = 0; c < RB / 16; ++c) {
+      uint2 lo = make_uint2(0, 0), hi = make_uint2(0, 0);
+      if (16 * c < nbytes) lo = *reinterpret_cast<const uint2*>(srow + 16 * c);
+      if (16 * c + 8 < nbytes) hi = *reinterpret_cast<const uint2*>(srow + 16 * c + 8);
+      o[c] = make_uint4(lo.x, lo.y, hi.x, hi.y);
+      if (I8)
+        amax = __vmaxu4(__vmaxu4(amax, __vabs4(lo.x)),
+                        __vmaxu4(__vmaxu4(__vabs4(lo.y), __vabs4(hi.x)), __vabs4(hi.y)));
+    }
+  }
+  if (I8 && m.absmax) {
+    int mag = static_cast<int>(max(max(amax & 0xFFu, (amax >> 8) & 0xFFu),
+                                   max((amax >> 16) & 0xFFu, amax >> 24)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mag = max(mag, __shfl_xor_sync(0xffffffffu, mag, o));
+    if ((threadIdx.x & 31) == 0 && mag > 0) atomicMax(m.absmax, mag);
+  }
+}
+
+// Launch of the staged scatter for rows of RB repacked bytes.
+template <int RB, bool I8>
+int launch_mask_emit_staged(const MaskArgs& m, int nb, int nbytes, cudaStream_t st) {
+  const int smem = 1024 * nbytes;
+  // Above 48 KB of shared memory in all (static included) a kernel must opt in.
+  FASTNN_CUDA_TRY(cudaFuncSetAttribute(mask_emit_staged_kernel<RB, I8>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  mask_emit_staged_kernel<RB, I8><<<nb, kMaskEmitThreads, smem, st>>>(m, nbytes);
+  return FASTNN_OK;
+}
+
 // Seeds of the masked fast scheme: the kept grid pixels of each pair in grid
 // order, as compacted indices (p2c), and their count. One CTA per pair.
 __global__ void __launch_bounds__(1024) masked_seeds_kernel(const int32_t* __restrict__ p2c,
@@ -516,6 +656,30 @@ static int launch_mask_compact_impl(const MaskArgs& m0, int dtype, cudaStream_t 
   if (nb <= 0) return FASTNN_OK;
   mask_count_kernel<<<nb, 1024, 0, st>>>(m);
   mutual_scan_kernel<<<m.batch, 1024, 0, st>>>(m.blocks, m.bpp, m.count);
+  const int nbytes = m.d * elem_bytes(dtype);
+  if (dtype != FASTNN_F32_L2 && nbytes % 8 == 0 && reinterpret_cast<uintptr_t>(m.src) % 16 == 0 &&
+      (m.batch == 1 || (m.N * nbytes) % 16 == 0)) {
+    const bool i8 = dtype == FASTNN_I8;
+    int rc = FASTNN_OK;
+    switch (row_bytes(dtype, m.d)) {
+      case 32:
+        rc = i8 ? launch_mask_emit_staged<32, true>(m, nb, nbytes, st)
+                : launch_mask_emit_staged<32, false>(m, nb, nbytes, st);
+        break;
+      case 64:
+        rc = i8 ? launch_mask_emit_staged<64, true>(m, nb, nbytes, st)
+                : launch_mask_emit_staged<64, false>(m, nb, nbytes, st);
+        break;
+      case 128:
+        rc = launch_mask_emit_staged<128, false>(m, nb, nbytes, st);
+        break;
+      default:
+        return FASTNN_ERR_UNSUPPORTED;
+    }
+    if (rc != FASTNN_OK) return rc;
+    FASTNN_CUDA_TRY(cudaGetLastError());
+    return FASTNN_OK;
+  }
   switch (dtype == FASTNN_F32_L2 ? 0 : row_bytes(dtype, m.d) * (dtype == FASTNN_I8 ? 1 : -1)) {
     case 0: mask_emit_kernel<1, 4, 16><<<nb, 1024, 0, st>>>(m); break;
     case 32: mask_emit_kernel<0, 1, 32><<<nb, 1024, 0, st>>>(m); break;
@@ -543,8 +707,8 @@ int launch_masked_seeds(const int32_t* p2c, int batch, int64_t N1, int W1, int s
   return FASTNN_OK;
 }
 
-static int launch_repack_impl(const void* src, int64_t rows, int d, int dtype, void* dst, int64_t pad_rows,
-                  int* absmax, cudaStream_t st) {
+static int launch_repack_impl(const void* src, int64_t rows, int d, int dtype, void* dst,
+                              int64_t pad_rows, int* absmax, cudaStream_t st) {
   const int64_t total = rows + pad_rows;
   if (total <= 0) return FASTNN_OK;
   const uint8_t* s8 = static_cast<const uint8_t*>(src);
@@ -607,10 +771,14 @@ int launch_repack(const void* src, int64_t rows, int d, int dtype, void* dst, in
   return kernel_timer_end(slot, st);
 }
 
-int mutual_blocks(int64_t n1) { return static_cast<int>((n1 + 1023) / 1024); }
+int mutual_blocks(int64_t n1) {
+  return static_cast<int>((n1 + kMutBlockRows - 1) / kMutBlockRows);
+}
+int image_blocks(int64_t n1) { return static_cast<int>((n1 + 1023) / 1024); }
 
-static int launch_mutual_impl(const MutualSrc& m, int32_t* block_scratch, int dtype, int32_t* out_pairs,
-                  void* out_score, int64_t cap, int32_t* out_count, cudaStream_t st) {
+static int launch_mutual_impl(const MutualSrc& m, int32_t* block_scratch, int dtype,
+                              int32_t* out_pairs, void* out_score, int64_t cap,
+                              int32_t* out_count, cudaStream_t st) {
   const int nb = mutual_blocks(m.n1);
   mutual_count_kernel<<<nb, 1024, 0, st>>>(m, block_scratch);
   mutual_scan_kernel<<<1, 1024, 0, st>>>(block_scratch, nb, out_count);
@@ -645,10 +813,11 @@ int launch_chunk_boxes(const float4* rows, int64_t N, int batch, const int32_t* 
   return FASTNN_OK;
 }
 
-static int launch_image_list_impl(const uint64_t* k12, int64_t n1, int64_t n2, uint32_t* first,
-                      uint32_t* best, int32_t* pos, int32_t* list, uint32_t* list_bound,
-                      int32_t* count, int32_t* block_scratch, cudaStream_t st) {
-  const int nb = mutual_blocks(n1);
+static int launch_image_list_impl(const uint64_t* k12, int64_t n1, int64_t n2,
+                                  uint32_t* first, uint32_t* best, int32_t* pos, int32_t* list,
+                                  uint32_t* list_bound, int32_t* count, int32_t* block_scratch,
+                                  cudaStream_t st) {
+  const int nb = image_blocks(n1);
   image_mark_kernel<<<grid_for(n1, 256), 256, 0, st>>>(k12, n1, n2, first, best);
   image_count_kernel<<<nb, 1024, 0, st>>>(k12, first, n1, n2, block_scratch);
   mutual_scan_kernel<<<1, 1024, 0, st>>>(block_scratch, nb, count);

@@ -91,7 +91,9 @@ struct MutualSrc {
   int64_t i0;  // global index of local row 0
 };
 
+// Scan scratch (ints) of the mutual test over n1 rows, and of the image list.
 int mutual_blocks(int64_t n1);
+int image_blocks(int64_t n1);
 // Bounding box (lo, hi; xyz) of every kL2Chunk-row chunk of each pair's
 // repacked pointmap rows [batch][N]: box[(b * nchunk + c) * 2 + {0, 1}],
 // nchunk = ceil(N / kL2Chunk). With `count`, pair b has count[b] rows;
@@ -105,7 +107,7 @@ int launch_chunk_boxes(const float4* rows, int64_t N, int batch, const int32_t* 
 // exit list[0..*count) holds the matched rows, pos[j] their slot (only for
 // matched j) and list_bound[slot] the best forward score bits among the rows
 // matched to j (a score NN21(j) reaches). block_scratch holds
-// mutual_blocks(n1) ints.
+// image_blocks(n1) ints.
 int launch_image_list(const uint64_t* k12, int64_t n1, int64_t n2, uint32_t* first,
                       uint32_t* best, int32_t* pos, int32_t* list, uint32_t* list_bound,
                       int32_t* count, int32_t* block_scratch, cudaStream_t st);

@@ -281,7 +281,8 @@ struct Epi<FASTNN_F16> : Epi<FASTNN_BF16> {};
 // Used for the ragged last database tile: `valid` < 32 masks the tail.
 template <int DT>
 __device__ __forceinline__ void fold32_masked(const uint32_t (&r)[32], uint32_t col0, int valid,
-                                              typename Epi<DT>::S& best, uint32_t& bidx) {
+                                              typename Epi<DT>::S& best, uint32_t& bidx,
+                                              bool& exact) {
   using E = Epi<DT>;
   using S = typename E::S;
   S v[32];
@@ -297,6 +298,7 @@ __device__ __forceinline__ void fold32_masked(const uint32_t (&r)[32], uint32_t 
       if (v[j] == m) first = j;
     best = m;
     bidx = col0 + first;
+    exact = true;
   }
 }
 
@@ -329,10 +331,18 @@ __device__ __forceinline__ void stash8(uint4* slot, const uint32_t* r) {
 }
 
 // int8 scores that fit in 16 bits: r[c][i] holds columns 32c + 2i (low half)
-// and 32c + 2i + 1 (high half) of this thread's block.
-template <int NC>
+// and 32c + 2i + 1 (high half) of this thread's block. On a strict new
+// record the first 16-column group holding it is found from the tree's group
+// maxima. DEFER == false: that group is staged to this thread's 32-byte slot
+// in shared memory and scanned for the first column. DEFER == true: only the
+// group is noted (bidx = its first column, exact = false) and resolve_group
+// finds the column once, at the end of the segment -- cheaper when segments
+// are long (the standalone pass), dearer when a CTA's range holds many short
+// ones (the fast scheme's passes).
+template <int NC, bool DEFER>
 __device__ __forceinline__ void fold_pack16(const uint32_t (&r)[NC][16], uint32_t colbase,
-                                            int& best, uint32_t& bidx, uint4* slot) {
+                                            int& best, uint32_t& bidx, bool& exact,
+                                            uint4* slot) {
   constexpr int G = 2 * NC;  // groups of 8 registers = 16 columns
   uint32_t g[G];
 #pragma unroll
@@ -353,26 +363,71 @@ __device__ __forceinline__ void fold_pack16(const uint32_t (&r)[NC][16], uint32_
 #pragma unroll
     for (int i = G - 1; i >= 0; --i)
       if (lo16(g[i]) == m || hi16(g[i]) == m) gi = i;
+    if constexpr (DEFER) {
+      bidx = colbase + 16 * gi;
+      exact = false;
+    } else {
 #pragma unroll
-    for (int i = 0; i < G; ++i)
-      if (i == gi) stash8(slot, &r[i / 2][(i % 2) * 8]);
-    const uint4 a = slot[0], b = slot[1];
-    const uint32_t x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-    int w = 15;
+      for (int i = 0; i < G; ++i)
+        if (i == gi) stash8(slot, &r[i / 2][(i % 2) * 8]);
+      const uint4 a = slot[0], b = slot[1];
+      const uint32_t x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+      int w = 15;
 #pragma unroll
-    for (int j = 7; j >= 0; --j) {
-      if (hi16(x[j]) == m) w = 2 * j + 1;
-      if (lo16(x[j]) == m) w = 2 * j;
+      for (int j = 7; j >= 0; --j) {
+        if (hi16(x[j]) == m) w = 2 * j + 1;
+        if (lo16(x[j]) == m) w = 2 * j;
+      }
+      bidx = colbase + 16 * gi + w;
+      exact = true;
     }
-    bidx = colbase + 16 * gi + w;
   }
+}
+
+// The lowest column among the 16 from bidx whose int8 dot product with the
+// query equals best (one exists: the tile's tree found best in this group).
+// Rows are read from the repacked maps (L2): RB bytes of zero-padded int8; a
+// query row outside the source is the zero vector, as the query gather
+// treats it. Loads go in batches of four rows.
+template <int RB>
+__device__ __noinline__ uint32_t resolve_group(const uint8_t* __restrict__ qrow,
+                                               const uint8_t* __restrict__ db, uint32_t bidx,
+                                               int best) {
+  constexpr int NV = RB / 16;  // 16-byte words per row
+  int4 qv[NV];
+#pragma unroll
+  for (int i = 0; i < NV; ++i)
+    qv[i] = qrow ? __ldg(reinterpret_cast<const int4*>(qrow) + i) : make_int4(0, 0, 0, 0);
+  uint32_t found = 0xFFFFFFFFu;
+#pragma unroll 1
+  for (int c0 = 0; c0 < 16 && found == 0xFFFFFFFFu; c0 += 4) {
+    int4 rv[4][NV];
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+#pragma unroll
+      for (int i = 0; i < NV; ++i)
+        rv[c][i] = __ldg(reinterpret_cast<const int4*>(db + static_cast<int64_t>(bidx + c0 + c) * RB) + i);
+#pragma unroll
+    for (int c = 3; c >= 0; --c) {
+      int s = 0;
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        s = __dp4a(qv[i].x, rv[c][i].x, s);
+        s = __dp4a(qv[i].y, rv[c][i].y, s);
+        s = __dp4a(qv[i].z, rv[c][i].z, s);
+        s = __dp4a(qv[i].w, rv[c][i].w, s);
+      }
+      if (s == best) found = bidx + c0 + c;
+    }
+  }
+  return found != 0xFFFFFFFFu ? found : bidx;
 }
 
 // 32-bit scores (int32, or fp32 for bf16 descriptors): r[c][i] = column 32c + i.
 template <int DT, int NC>
 __device__ __forceinline__ void fold_wide(const uint32_t (&r)[NC][32], uint32_t colbase,
                                           typename Epi<DT>::S& best, uint32_t& bidx,
-                                          uint4* slot) {
+                                          bool& exact, uint4* slot) {
   using E = Epi<DT>;
   using S = typename E::S;
   constexpr int G = 4 * NC;  // groups of 8 registers = 8 columns
@@ -403,6 +458,7 @@ __device__ __forceinline__ void fold_wide(const uint32_t (&r)[NC][32], uint32_t 
     for (int j = 7; j >= 0; --j)
       if (E::as_score(x[j]) == m) w = j;
     bidx = colbase + 8 * gi + w;
+    exact = true;
   }
 }
 
@@ -538,7 +594,7 @@ __device__ void plan_phase(const NNArgs& a, const PhaseQ& q, Ctl* ctl) {
 // One nearest-neighbour phase: plan (thread 0), then each role runs its loop
 // over this CTA's units. Ends with a CTA barrier, after which every MMA of the
 // phase has completed and every result has been merged into a.out_key.
-template <int DT, int RB>
+template <int DT, int RB, bool DEFER>
 __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const PhaseQ q,
                           const SmemLayout& L, uint32_t tmem, PipeState& ps) {
   constexpr int NS = stages_for(RB);  // database ring depth
@@ -707,6 +763,7 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Pha
           if (bits != 0u) best = E::below_bound(bits);
         }
         uint32_t bidx = 0xFFFFFFFFu;
+        bool exact = true;  // false: bidx is a 16-column group still to resolve
         for (int j = (grp - ps.epar) & 1; j < len; j += kAcc) {
           const int n = n0 + j;
           const uint32_t colbase = static_cast<uint32_t>(n) * kBN + h * kEpiCols;
@@ -726,7 +783,7 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Pha
               ptx::tmem_ld32(taddr + c * 32, r);
               ptx::tmem_ld_wait();
               const int valid = min(32, max(0, valid_blk - c * 32));
-              fold32_masked<DT>(r, colbase + c * 32, valid, best, bidx);
+              fold32_masked<DT>(r, colbase + c * 32, valid, best, bidx, exact);
             }
             ptx::tc_fence_before();
             __syncwarp();
@@ -743,27 +800,39 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Pha
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(rel_bar);
             ptx::pin_regs(reinterpret_cast<uint32_t(&)[64]>(r));
-            if constexpr (DT == FASTNN_I8) fold_pack16<kChunks>(r, colbase, best, bidx, slot);
+            if constexpr (DT == FASTNN_I8)
+              fold_pack16<kChunks, DEFER>(r, colbase, best, bidx, exact, slot);
           } else {
             // 32-bit scores: two 64-column halves, the accumulator is released
             // after the second load.
             uint32_t r[2][32];
             ptx::tmem_ld64(taddr, reinterpret_cast<uint32_t(&)[64]>(r));
             ptx::tmem_ld_wait_regs(reinterpret_cast<uint32_t(&)[64]>(r));
-            fold_wide<DT, 2>(r, colbase, best, bidx, slot);
+            fold_wide<DT, 2>(r, colbase, best, bidx, exact, slot);
             ptx::tmem_ld64(taddr + 64, reinterpret_cast<uint32_t(&)[64]>(r));
             ptx::tmem_ld_wait_regs(reinterpret_cast<uint32_t(&)[64]>(r));
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(rel_bar);
             ptx::pin_regs(reinterpret_cast<uint32_t(&)[64]>(r));
-            fold_wide<DT, 2>(r, colbase + 64, best, bidx, slot);
+            fold_wide<DT, 2>(r, colbase + 64, best, bidx, exact, slot);
           }
         }
         if (!ok) break;
-        if (krow < ctl->cnt[p.b] && bidx != 0xFFFFFFFFu)
+        if (krow < ctl->cnt[p.b] && bidx != 0xFFFFFFFFu) {
+          if constexpr (DT == FASTNN_I8 && DEFER) {
+            if (!exact) {
+              const int64_t qr = nn_query_row(a, q, p.b, krow);
+              const uint8_t* qrow = (qr >= 0 && qr < a.q_rows_per_pair)
+                                        ? a.q_rows + (p.b * a.q_rows_per_pair + qr) * RB
+                                        : nullptr;
+              bidx = resolve_group<RB>(qrow, a.db_rows + static_cast<int64_t>(p.b) * a.ndb * RB,
+                                       bidx, best);
+            }
+          }
           atomicMax(reinterpret_cast<unsigned long long*>(&a.out_key[p.b * a.q_cap + krow]),
                     static_cast<unsigned long long>(make_key(E::ord(best), bidx)));
+        }
         u += len;
         ps.epar ^= len & 1;
         next_segment(p, ctl, batch);
@@ -804,7 +873,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   pipe_setup(L.ctl);
   const uint32_t tmem = L.ctl->tmem_base;
   PipeState ps;
-  run_phase<DT, RB>(&tmap_db, a, PhaseQ{a.q_index, a.q_count, a.q_bound, 1}, L, tmem, ps);
+  run_phase<DT, RB, true>(&tmap_db, a, PhaseQ{a.q_index, a.q_count, a.q_bound, 1}, L, tmem, ps);
   pipe_teardown(L.ctl, tmem, a.status);
 }
 
@@ -830,9 +899,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   PipeState ps;
   auto pass = [&](int dir, const PhaseQ& q) {
     if (dir == 0)
-      run_phase<DT, RB>(&tmap_d2, r.fwd, q, L, tmem, ps);
+      run_phase<DT, RB, false>(&tmap_d2, r.fwd, q, L, tmem, ps);
     else
-      run_phase<DT, RB>(&tmap_d1, r.bwd, q, L, tmem, ps);
+      run_phase<DT, RB, false>(&tmap_d1, r.bwd, q, L, tmem, ps);
   };
   fast_rounds<DT>(r, pass, [] {}, &ctl->abort_flag, &ctl->grid_ok, &ctl->more, ctl->scan);
   pipe_teardown(ctl, tmem, r.status);
