@@ -86,19 +86,6 @@ __device__ __forceinline__ Scan2 block_scan2(bool f0, bool f1, int* sm) {
   return Scan2{off0 + __popc(b0 & lt), off1 + __popc(b1 & lt), t0, t1};
 }
 
-// Seeds of pair b: pixels (x, y) with x = sub * (k mod gx), y = sub * (k div gx)
-// for k < S, written to the round-1 frontier; each seed claims its pixel with
-// stamp 0 (round 0, slot k).
-__device__ __forceinline__ void seed_one(int32_t* F0, int64_t S_cap, uint32_t* claim, int64_t N1,
-                                         int W1, int sub, int b, int k) {
-  const int gx = (W1 + sub - 1) / sub;
-  const int y = (k / gx) * sub;
-  const int x = (k % gx) * sub;
-  const int u = y * W1 + x;
-  F0[b * S_cap + k] = u;
-  claim[b * N1 + u] = static_cast<uint32_t>(k);
-}
-
 // Block-wide exclusive scan of two small per-thread counts (each block total
 // below 2^16), packed in one word: a warp shuffle scan, then one pass over
 // the warp totals. `sm` holds 32 ints; every thread of the block must call it.
@@ -273,7 +260,26 @@ __device__ void fast_rounds(const RecArgs& r, NNPass&& nn, Prologue&& prologue,
     r.cmp.fwd_key[i] = 0;
     r.cmp.bwd_key[i] = 0;
   }
-  for (int64_t i = gtid; i < batch * r.N1; i += gsize) r.cmp.claim[i] = 0xFFFFFFFFu;
+  if (r.seed_cnt) {
+    for (int64_t i = gtid; i < batch * r.N1; i += gsize) r.cmp.claim[i] = 0xFFFFFFFFu;
+  } else {
+    // Unmasked: the grid seeds are known, so the clearing pass writes each
+    // seed pixel's stamp (round 0, slot k) directly, with the round-1
+    // frontier, and seeding needs no pass (nor barrier) of its own.
+    const int gx = (r.W1 + r.sub - 1) / r.sub;
+    for (int64_t i = gtid; i < batch * r.N1; i += gsize) {
+      const int u = static_cast<int>(i % r.N1);
+      const int y = u / r.W1, x = u % r.W1;
+      r.cmp.claim[i] = (x % r.sub == 0 && y % r.sub == 0)
+                           ? static_cast<uint32_t>((y / r.sub) * gx + x / r.sub)
+                           : 0xFFFFFFFFu;
+    }
+    for (int64_t i = gtid; i < batch * S; i += gsize) {
+      const int k = static_cast<int>(i % S);
+      r.F[0][i] = (k / gx) * r.sub * r.W1 + (k % gx) * r.sub;
+    }
+    for (int64_t i = gtid; i < batch; i += gsize) r.cnt[0][i] = static_cast<int>(S);
+  }
   for (int64_t i = gtid; i < batch; i += gsize) {
     r.cmp.out_count[i] = 0;
     if (r.cmp.out_iters) r.cmp.out_iters[i] = 0;
@@ -282,23 +288,15 @@ __device__ void fast_rounds(const RecArgs& r, NNPass&& nn, Prologue&& prologue,
     for (int64_t i = gtid; i < batch * r.max_iter; i += gsize) r.cmp.out_frontier[i] = 0;
   prologue();
   bool ok = sync();
-  if (ok) {
-    // Seeds: the round-1 frontier of every pair (the grid, or the kept grid
-    // pixels already written to F[0] when seed_cnt is given); each claims
-    // its pixel with stamp (round 0, slot k).
-    if (r.seed_cnt) {
-      for (int64_t i = gtid; i < batch * S; i += gsize) {
-        const int b = static_cast<int>(i / S), k = static_cast<int>(i % S);
-        if (k < __ldcg(r.seed_cnt + b))
-          r.cmp.claim[b * r.N1 + __ldcg(r.F[0] + i)] = static_cast<uint32_t>(k);
-      }
-      for (int64_t i = gtid; i < batch; i += gsize) r.cnt[0][i] = __ldcg(r.seed_cnt + i);
-    } else {
-      for (int64_t i = gtid; i < batch * S; i += gsize)
-        seed_one(r.F[0], S, r.cmp.claim, r.N1, r.W1, r.sub, static_cast<int>(i / S),
-                 static_cast<int>(i % S));
-      for (int64_t i = gtid; i < batch; i += gsize) r.cnt[0][i] = static_cast<int>(S);
+  if (ok && r.seed_cnt) {
+    // Masked: the kept grid pixels are already in F[0]; each claims its pixel
+    // with stamp (round 0, slot k) once the claims are cleared.
+    for (int64_t i = gtid; i < batch * S; i += gsize) {
+      const int b = static_cast<int>(i / S), k = static_cast<int>(i % S);
+      if (k < __ldcg(r.seed_cnt + b))
+        r.cmp.claim[b * r.N1 + __ldcg(r.F[0] + i)] = static_cast<uint32_t>(k);
     }
+    for (int64_t i = gtid; i < batch; i += gsize) r.cnt[0][i] = __ldcg(r.seed_cnt + i);
     ok = sync();
   }
   for (int t = 1; ok && t <= r.max_iter; ++t) {
