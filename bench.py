@@ -67,7 +67,7 @@ def parse_args():
     ap.add_argument("--also", default=None,
                     help="comma-separated workloads measured after the main one and nested "
                          "in its JSON line (default with the headline workload: the dense, "
-                         "bf16 and 16-pair workloads; '' for none)")
+                         "bf16 and 16-pair workloads; 'none' for none)")
     ap.add_argument("--also-steps", type=int, default=100)
     ap.add_argument("--stream-steps", type=int, default=None,
                     help="steps of the 64M-row memory-bound kernel suite nested in the line "
@@ -476,7 +476,11 @@ class Runner:
             self.launches_per_step = 8
             self.kernels_per_step = 1
         else:
-            self.launches_per_step = 3  # 2 repack kernels + 1 persistent matching kernel
+            # The persistent matching kernel repacks both maps itself when their
+            # rows are whole 8-byte words (int8 d = 8, 16, 24, 32, ...; 16-bit
+            # d = 4, 8, ...); otherwise two repack kernels run before it.
+            in_kernel = not self.l2 and (d * self.esize) % 8 == 0
+            self.launches_per_step = 1 if in_kernel else 3
             self.kernels_per_step = 1
 
     def call(self):
@@ -781,7 +785,8 @@ def run_ours(args, rank, world, local):
 
     head = measure(args.workload, args.steps, args.warmup, rank, ranks, dev, stream, flush,
                    sample_clocks=rank == 0, e2e_steps=max(1, min(args.steps, 1000)))
-    also = [x for x in (args.also.split(",") if args.also else []) if x and x != args.workload]
+    also = [x for x in (args.also.split(",") if args.also and args.also != "none" else [])
+            if x and x != args.workload]
     nested = []
     for name in also:
         r = measure(name, args.also_steps, args.warmup, rank, ranks, dev, stream, flush,

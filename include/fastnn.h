@@ -79,7 +79,8 @@ typedef enum {
     FASTNN_OP_MUTUAL_DENSE = 2,
     FASTNN_OP_MUTUAL_FROM_NN = 3,
     FASTNN_OP_RECIPROCAL_MASKED = 4,
-    FASTNN_OP_MUTUAL_DENSE_MASKED = 5
+    FASTNN_OP_MUTUAL_DENSE_MASKED = 5,
+    FASTNN_OP_IMAGE_ROWS = 6
 } fastnn_op;
 
 /*
@@ -92,6 +93,8 @@ typedef enum {
  *                           (d must still be valid for dtype; unused)
  *   FASTNN_OP_RECIPROCAL_MASKED, FASTNN_OP_MUTUAL_DENSE_MASKED: as the
  *                           unmasked ops
+ *   FASTNN_OP_IMAGE_ROWS:   n1 = entries of nn12, n2 = image-2 rows (d must
+ *                           still be valid for dtype; unused)
  * Returns 0 for arguments no call would accept.
  */
 size_t fastnn_workspace_size(int op, int64_t n1, int64_t n2, int d, int dtype,
@@ -167,7 +170,9 @@ int fastnn_mutual_dense(const void *desc1, int64_t n1, const void *desc2,
  * the last step of the dense mutual set when image 1's rows are split across
  * GPUs and nn21 (all n2 image-2 rows, global image-1 indices) was gathered.
  *   nn12: [n1] int32 in [0, n2); score12: [n1] int32/float or NULL;
- *   nn21: [n2] int32 in [0, n1_total). Output (i0 + i, j) in ascending i into
+ *   nn21: [n2] int32 in [0, n1_total), or -1 for a row with no partner (a row
+ *   outside the image of NN12, see fastnn_image_rows). Output (i0 + i, j) in
+ *   ascending i into
  *   out_pairs [capacity][2], scores into out_score (or NULL), *out_count =
  *   pairs. capacity >= min(n1, n2). n1 == 0 writes *out_count = 0.
  */
@@ -177,6 +182,22 @@ int fastnn_mutual_from_nn(const int32_t *nn12, const void *score12, int64_t n1,
                           void *out_score, int64_t capacity, int32_t *out_count,
                           void *workspace, size_t workspace_bytes,
                           fastnn_stream_t stream);
+
+/*
+ * fastnn_image_rows -- the image-2 rows that can be in a mutual pair: a pair
+ * (i, j) of the reciprocal set ("MASt3R dissection", section 1 and section 3)
+ * has j = NN12(i), so only the rows some image-1 row matches need their own
+ * nearest neighbour in image 1. Writes the distinct values of nn12 that lie
+ * in [0, n2), in ascending order, to out_rows[0 .. *out_count) (device int32);
+ * out_rows must hold min(n1, n2) entries. When image 1's rows are split
+ * across GPUs, the gathered NN12 of all of them gives every rank the same
+ * list, whose rows are then split for the backward pass.
+ *   nn12: [n1] int32 (may be NULL when n1 == 0; values outside [0, n2) are
+ *   ignored). Workspace: FASTNN_OP_IMAGE_ROWS.
+ */
+int fastnn_image_rows(const int32_t *nn12, int64_t n1, int64_t n2,
+                      int32_t *out_rows, int32_t *out_count, void *workspace,
+                      size_t workspace_bytes, fastnn_stream_t stream);
 
 /*
  * fastnn_set_wait_timeout_ns -- limit of the kernels' bounded waits for the

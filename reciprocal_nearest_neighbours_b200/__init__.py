@@ -16,6 +16,7 @@ from ._lib import (  # noqa: F401
     FASTNN_F32_L2,
     FASTNN_I8,
     FASTNN_OP_MUTUAL_DENSE,
+    FASTNN_OP_IMAGE_ROWS,
     FASTNN_OP_MUTUAL_DENSE_MASKED,
     FASTNN_OP_MUTUAL_FROM_NN,
     FASTNN_OP_NN,
@@ -27,6 +28,7 @@ from ._lib import (  # noqa: F401
     FASTNN_TIME_REPACK,
     FastNNError,
     fastnn_device_status,
+    fastnn_image_rows,
     fastnn_kernel_timer_enable,
     fastnn_kernel_timer_read,
     fastnn_kernel_timer_select,

@@ -20,6 +20,7 @@ FASTNN_OP_MUTUAL_DENSE = 2
 FASTNN_OP_MUTUAL_FROM_NN = 3
 FASTNN_OP_RECIPROCAL_MASKED = 4
 FASTNN_OP_MUTUAL_DENSE_MASKED = 5
+FASTNN_OP_IMAGE_ROWS = 6
 
 _lib = None
 
@@ -67,6 +68,8 @@ def library():
     lib.fastnn_mutual_dense_masked.restype = I
     lib.fastnn_mutual_from_nn.argtypes = [P, P, I64, I64, P, I64, I64, I, P, P, I64, P, P, SZ, P]
     lib.fastnn_mutual_from_nn.restype = I
+    lib.fastnn_image_rows.argtypes = [P, I64, I64, P, P, P, SZ, P]
+    lib.fastnn_image_rows.restype = I
     lib.fastnn_device_status.argtypes = [P, P]
     lib.fastnn_device_status.restype = I
     lib.fastnn_noalloc_device_status.argtypes = [P]
@@ -299,6 +302,27 @@ def fastnn_mutual_from_nn(nn12: torch.Tensor, score12, i0: int, nn21: torch.Tens
                                          cap, _ptr(out_count), _ptr(ws), nbytes, _stream(stream))
     _check(rc, "fastnn_mutual_from_nn")
     return out_pairs, out_score, out_count
+
+
+def fastnn_image_rows(nn12: torch.Tensor, n2: int, out_rows=None, out_count=None,
+                      workspace=None, stream=None):
+    """Ascending distinct values of ``nn12`` [n1] int32 that lie in [0, n2):
+    the image-2 rows some image-1 row matches. Returns ``(rows [cap], count
+    [1])`` with rows[:count] valid (cap = min(n1, n2))."""
+    _need_cuda(nn12)
+    n1 = nn12.numel()
+    dev = nn12.device
+    cap = max(1, min(n1, int(n2)))
+    if out_rows is None:
+        out_rows = torch.empty(cap, dtype=torch.int32, device=dev)
+    if out_count is None:
+        out_count = torch.empty(1, dtype=torch.int32, device=dev)
+    nbytes = fastnn_workspace_size(FASTNN_OP_IMAGE_ROWS, n1, int(n2), 1, FASTNN_I8)
+    ws = _workspace(nbytes, dev, workspace)
+    rc = library().fastnn_image_rows(_ptr(nn12) if n1 else None, n1, int(n2), _ptr(out_rows),
+                                     _ptr(out_count), _ptr(ws), nbytes, _stream(stream))
+    _check(rc, "fastnn_image_rows")
+    return out_rows, out_count
 
 
 def fastnn_device_status(workspace: torch.Tensor, stream=None) -> int:

@@ -201,6 +201,10 @@ size_t fastnn_workspace_size(int op, int64_t n1, int64_t n2, int d, int dtype, i
     case FASTNN_OP_MUTUAL_FROM_NN:
       c.take<int32_t>(static_cast<size_t>(mutual_blocks(n1 > 0 ? n1 : 1)));
       break;
+    case FASTNN_OP_IMAGE_ROWS:
+      c.take<uint8_t>(static_cast<size_t>(n2));
+      c.take<int32_t>(static_cast<size_t>(mutual_blocks(n2)));
+      break;
     case FASTNN_OP_RECIPROCAL_MASKED:
       if (batch < 1 || max_queries < 1 || n1 < 1) return 0;
       carve_rec(c, n1, n2, d, dtype, batch, max_queries);
@@ -299,12 +303,25 @@ int reciprocal_impl(const void* desc1, const float* conf1, int H1, int W1, const
                 L.d2rep, M.c2p2, nullptr, M.cnt2, L.status + 2, M.blocks, 0};
     FASTNN_TRY(launch_mask_compact(m2, dtype, st));
     FASTNN_TRY(launch_masked_seeds(M.p2c1, batch, N1, W1, subsample, S, L.F[0], M.seedcnt, st));
-  } else {
+  }
+  // The tensor-core kernel repacks both maps itself (in its clearing pass)
+  // when their rows are whole 8-byte words at 8-byte aligned addresses;
+  // otherwise the repack kernels run first.
+  const int nbytes = d * (dtype == FASTNN_I8 ? 1 : dtype == FASTNN_F32_L2 ? 4 : 2);
+  const bool repack_in_kernel = !masked && dtype != FASTNN_F32_L2 && nbytes % 8 == 0 &&
+                                aligned(desc1, 8) && aligned(desc2, 8);
+  if (!masked && !repack_in_kernel) {
     FASTNN_TRY(launch_repack(desc1, batch * N1, d, dtype, L.d1rep, kPadRows, L.status + 1, st));
     FASTNN_TRY(launch_repack(desc2, batch * N2, d, dtype, L.d2rep, kPadRows, L.status + 2, st));
   }
 
   RecArgs r{};
+  if (repack_in_kernel) {
+    r.src1 = static_cast<const uint8_t*>(desc1);
+    r.src2 = static_cast<const uint8_t*>(desc2);
+    r.src_nbytes = nbytes;
+  }
+  r.N2 = N2;
   r.fwd.q_rows = L.d1rep;
   r.fwd.q_rows_per_pair = N1;
   r.fwd.q_cap = S;
@@ -553,6 +570,22 @@ int fastnn_mutual_from_nn(const int32_t* nn12, const void* score12, int64_t n1, 
   m.n2 = n2;
   m.i0 = i0;
   return launch_mutual(m, blocks, dtype, out_pairs, out_score, capacity, out_count, st);
+}
+
+int fastnn_image_rows(const int32_t* nn12, int64_t n1, int64_t n2, int32_t* out_rows,
+                      int32_t* out_count, void* workspace, size_t workspace_bytes,
+                      fastnn_stream_t stream) {
+  if (n1 < 0 || n2 < 1 || n2 > INT32_MAX) return FASTNN_ERR_INVALID;
+  if ((n1 > 0 && !nn12) || !out_rows || !out_count || !workspace || !aligned(workspace, kAlign))
+    return FASTNN_ERR_INVALID;
+  if (workspace_bytes <
+      fastnn_workspace_size(FASTNN_OP_IMAGE_ROWS, n1, n2, 1, FASTNN_I8, 1, 0))
+    return FASTNN_ERR_CAPACITY;
+  Carver c{static_cast<uint8_t*>(workspace)};
+  uint8_t* flag = c.take<uint8_t>(static_cast<size_t>(n2));
+  int32_t* blocks = c.take<int32_t>(static_cast<size_t>(mutual_blocks(n2)));
+  return launch_image_rows(nn12, n1, n2, flag, blocks, out_rows, out_count,
+                           reinterpret_cast<cudaStream_t>(stream));
 }
 
 int fastnn_device_status(const void* workspace, fastnn_stream_t stream) {

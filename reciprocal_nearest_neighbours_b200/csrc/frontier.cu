@@ -233,6 +233,7 @@ __global__ void __launch_bounds__(1024) mutual_scan_kernel(int32_t* __restrict__
   const int k0 = min(static_cast<int>(threadIdx.x) * per, nblocks);
   const int k1 = min(k0 + per, nblocks);
   int sum = 0;
+#pragma unroll 8
   for (int k = k0; k < k1; ++k) sum += block_cnt[k];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int x = sum;
@@ -408,6 +409,63 @@ __global__ void __launch_bounds__(1024) image_emit_kernel(const uint64_t* __rest
   }
 }
 
+// ---------------------------------------------- image rows of an NN12 ---
+// The ascending list of image-2 rows j in [0, n2) that some nn12[i] names:
+// flags, per-block counts (4096 rows per block, four consecutive rows per
+// thread), the shared scan, an ordered emit.
+__global__ void image_flag_kernel(const int32_t* __restrict__ nn12, int64_t n1, int64_t n2,
+                                  uint8_t* __restrict__ flag) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n1;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int32_t j = nn12[i];
+    if (j >= 0 && j < n2) flag[j] = 1;
+  }
+}
+
+__device__ __forceinline__ void image_flags4(const uint8_t* flag, int64_t n2, int64_t j,
+                                             bool (&f)[4]) {
+  if (j + 3 < n2) {
+    const uchar4 v = *reinterpret_cast<const uchar4*>(flag + j);  // j is a multiple of 4
+    f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+  } else {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) f[r] = j + r < n2 && flag[j + r];
+  }
+}
+
+__global__ void __launch_bounds__(1024) image_rows_count_kernel(const uint8_t* __restrict__ flag,
+                                                                int64_t n2,
+                                                                int32_t* __restrict__ block_cnt) {
+  __shared__ int sm[32];
+  bool f[4];
+  image_flags4(flag, n2, blockIdx.x * static_cast<int64_t>(kMutBlockRows) + 4 * threadIdx.x, f);
+  int c = (f[0] ? 1 : 0) + (f[1] ? 1 : 0) + (f[2] ? 1 : 0) + (f[3] ? 1 : 0);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+  if ((threadIdx.x & 31) == 0) sm[threadIdx.x >> 5] = c;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int t = 0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) t += sm[w];
+    block_cnt[blockIdx.x] = t;
+  }
+}
+
+__global__ void __launch_bounds__(1024) image_rows_emit_kernel(const uint8_t* __restrict__ flag,
+                                                               int64_t n2,
+                                                               const int32_t* __restrict__ off,
+                                                               int32_t* __restrict__ rows) {
+  __shared__ int sm[32];
+  const int64_t j = blockIdx.x * static_cast<int64_t>(kMutBlockRows) + 4 * threadIdx.x;
+  bool f[4];
+  image_flags4(flag, n2, j, f);
+  const int c = (f[0] ? 1 : 0) + (f[1] ? 1 : 0) + (f[2] ? 1 : 0) + (f[3] ? 1 : 0);
+  int pos = off[blockIdx.x] + block_exclusive_scan(c, sm);
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+    if (f[r]) rows[pos++] = static_cast<int32_t>(j + r);
+}
+
 // ------------------------------------------------------------ decode nn ---
 template <int DT>
 __global__ void decode_kernel(const uint64_t* __restrict__ key, int64_t n,
@@ -473,13 +531,32 @@ __device__ __forceinline__ bool mask_kept(const MaskArgs& m, int64_t g) {
   return !m.conf || __ldg(m.conf + g) >= m.threshold;
 }
 
-__global__ void __launch_bounds__(1024) mask_count_kernel(MaskArgs m) {
-  __shared__ int sm[64];
+// Kept pixels of each 1024-pixel block: 256 threads, four consecutive
+// pixels each (one 16-byte load of confidences where aligned).
+__global__ void __launch_bounds__(256) mask_count_kernel(MaskArgs m) {
+  __shared__ int sm[8];
   const int b = blockIdx.x / m.bpp, blk = blockIdx.x % m.bpp;
-  const int64_t p = static_cast<int64_t>(blk) * 1024 + threadIdx.x;
-  const bool f = p < m.N && mask_kept(m, b * m.N + p);
-  const Scan2 sc = block_scan2(f, false, sm);
-  if (threadIdx.x == 0) m.blocks[blockIdx.x] = sc.tot0;
+  const int64_t p = static_cast<int64_t>(blk) * 1024 + 4 * threadIdx.x;
+  const int64_t g = b * m.N + p;
+  int c = 0;
+  if (m.conf && p + 3 < m.N && (reinterpret_cast<uintptr_t>(m.conf + g) & 15) == 0) {
+    const float4 c4 = __ldg(reinterpret_cast<const float4*>(m.conf + g));
+    c = (c4.x >= m.threshold) + (c4.y >= m.threshold) + (c4.z >= m.threshold) +
+        (c4.w >= m.threshold);
+  } else {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) c += (p + r < m.N && mask_kept(m, g + r)) ? 1 : 0;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+  if ((threadIdx.x & 31) == 0) sm[threadIdx.x >> 5] = c;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int t = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) t += sm[w];
+    m.blocks[blockIdx.x] = t;
+  }
 }
 
 // Descriptor row (ESIZE-byte elements) into an RB-byte slot; returns max
@@ -654,7 +731,7 @@ static int launch_mask_compact_impl(const MaskArgs& m0, int dtype, cudaStream_t 
   m.bpp = mask_blocks(m.N);
   const int nb = m.batch * m.bpp;
   if (nb <= 0) return FASTNN_OK;
-  mask_count_kernel<<<nb, 1024, 0, st>>>(m);
+  mask_count_kernel<<<nb, 256, 0, st>>>(m);
   mutual_scan_kernel<<<m.batch, 1024, 0, st>>>(m.blocks, m.bpp, m.count);
   const int nbytes = m.d * elem_bytes(dtype);
   if (dtype != FASTNN_F32_L2 && nbytes % 8 == 0 && reinterpret_cast<uintptr_t>(m.src) % 16 == 0 &&
@@ -835,6 +912,20 @@ int launch_image_list(const uint64_t* k12, int64_t n1, int64_t n2, uint32_t* fir
   const int rc = launch_image_list_impl(k12, n1, n2, first, best, pos, list, list_bound, count,
                                         block_scratch, st);
   if (rc != FASTNN_OK) return rc;
+  return kernel_timer_end(slot, st);
+}
+
+int launch_image_rows(const int32_t* nn12, int64_t n1, int64_t n2, uint8_t* flag,
+                      int32_t* block_scratch, int32_t* rows, int32_t* count, cudaStream_t st) {
+  const int slot = kernel_timer_begin(st, kTimeMutual);
+  if (slot == -2) return FASTNN_ERR_CUDA;
+  const int nb = mutual_blocks(n2);
+  FASTNN_CUDA_TRY(cudaMemsetAsync(flag, 0, static_cast<size_t>(n2), st));
+  if (n1 > 0) image_flag_kernel<<<grid_for(n1, 256), 256, 0, st>>>(nn12, n1, n2, flag);
+  image_rows_count_kernel<<<nb, 1024, 0, st>>>(flag, n2, block_scratch);
+  mutual_scan_kernel<<<1, 1024, 0, st>>>(block_scratch, nb, count);
+  image_rows_emit_kernel<<<nb, 1024, 0, st>>>(flag, n2, block_scratch, rows);
+  FASTNN_CUDA_TRY(cudaGetLastError());
   return kernel_timer_end(slot, st);
 }
 

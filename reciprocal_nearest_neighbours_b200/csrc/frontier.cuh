@@ -43,6 +43,14 @@ struct RecArgs {
   int* grid_abort;       // set when any CTA gives up (zero before the launch)
   int* status;
   const int32_t* seed_cnt;  // optional [batch]: F[0] already holds this many seeds per pair
+  // Repack inside the kernel (src_nbytes > 0): the raw maps [batch * N][d]
+  // (rows of src_nbytes bytes, a multiple of 8, 8-byte aligned) are written
+  // to r.bwd.db_rows / r.fwd.db_rows (plus 256 zero rows each) by the
+  // clearing pass, before the first grid barrier.
+  const uint8_t* src1;
+  const uint8_t* src2;
+  int src_nbytes;
+  int64_t N2;
 };
 
 // Confidence-mask compaction of one map (all pairs of a batch).
@@ -111,6 +119,10 @@ int launch_chunk_boxes(const float4* rows, int64_t N, int batch, const int32_t* 
 int launch_image_list(const uint64_t* k12, int64_t n1, int64_t n2, uint32_t* first,
                       uint32_t* best, int32_t* pos, int32_t* list, uint32_t* list_bound,
                       int32_t* count, int32_t* block_scratch, cudaStream_t st);
+// Ascending list of the distinct nn12[i] in [0, n2) into rows[0 .. *count).
+// flag holds n2 bytes, block_scratch mutual_blocks(n2) ints.
+int launch_image_rows(const int32_t* nn12, int64_t n1, int64_t n2, uint8_t* flag,
+                      int32_t* block_scratch, int32_t* rows, int32_t* count, cudaStream_t st);
 int launch_mutual(const MutualSrc& m, int32_t* block_scratch, int dtype, int32_t* out_pairs,
                   void* out_score, int64_t cap, int32_t* out_count, cudaStream_t st);
 // Keys -> (index, score); pointmap scores are the squared distances the keys

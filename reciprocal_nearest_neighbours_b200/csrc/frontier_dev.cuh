@@ -111,6 +111,44 @@ __device__ __forceinline__ Scan2 block_scan_counts(int c0, int c1, int* sm) {
   return Scan2{ex & 0xFFFF, ex >> 16, tot & 0xFFFF, tot >> 16};
 }
 
+// Repack inside a persistent kernel: rows [rows][nbytes] (nbytes a multiple
+// of 8, 8-byte aligned source) into RB-byte rows zero-padded, plus pad_rows
+// zero rows; one 16-byte output chunk per thread and step of a grid-stride
+// loop (two 8-byte loads), so a warp's loads and stores cover consecutive
+// bytes. absmax (int8, optional) receives max |element| by atomicMax. The
+// stores are then ordered before the async proxy (the tensor-map loads that
+// read the rows after the next grid barrier).
+__device__ __forceinline__ void repack_in_kernel(const uint8_t* __restrict__ src, int64_t rows,
+                                                 int nbytes, int RB, uint8_t* __restrict__ dst,
+                                                 int64_t pad_rows, int* absmax, int64_t gtid,
+                                                 int64_t gsize) {
+  const int cpr = RB / 16;  // output chunks per row
+  const int64_t total = (rows + pad_rows) * cpr;
+  uint32_t amax = 0;
+  for (int64_t k = gtid; k < total; k += gsize) {
+    const int64_t row = k / cpr;
+    const int off = 16 * static_cast<int>(k - row * cpr);
+    uint2 lo = make_uint2(0, 0), hi = make_uint2(0, 0);
+    if (row < rows) {
+      const uint8_t* sr = src + row * nbytes;
+      if (off < nbytes) lo = __ldg(reinterpret_cast<const uint2*>(sr + off));
+      if (off + 8 < nbytes) hi = __ldg(reinterpret_cast<const uint2*>(sr + off + 8));
+      if (absmax)
+        amax = __vmaxu4(__vmaxu4(amax, __vabs4(lo.x)),
+                        __vmaxu4(__vmaxu4(__vabs4(lo.y), __vabs4(hi.x)), __vabs4(hi.y)));
+    }
+    reinterpret_cast<uint4*>(dst + row * RB)[off / 16] = make_uint4(lo.x, lo.y, hi.x, hi.y);
+  }
+  if (absmax) {
+    int m = static_cast<int>(max(max(amax & 0xFFu, (amax >> 8) & 0xFFu),
+                                 max((amax >> 16) & 0xFFu, amax >> 24)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31) == 0 && m > 0) atomicMax(absmax, m);
+  }
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // The round's frontier buffers (the rest of CompactArgs is fixed per call).
 struct FrontierBufs {
   const int32_t* F_cur;

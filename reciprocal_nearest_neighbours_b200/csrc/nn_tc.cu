@@ -905,7 +905,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     else
       run_phase<DT, RB, true>(&tmap_d1, r.bwd, q, L, tmem, ps);
   };
-  fast_rounds<DT>(r, pass, [] {}, &ctl->abort_flag, &ctl->grid_ok, &ctl->more, ctl->scan);
+  // The repack of both maps, when the launcher left it to the kernel, runs in
+  // the clearing pass, before the first grid barrier.
+  auto repack = [&] {
+    if (r.src_nbytes > 0) {
+      const int64_t gtid = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+      const int64_t gsize = static_cast<int64_t>(gridDim.x) * blockDim.x;
+      const int64_t pad = 256;
+      repack_in_kernel(r.src1, r.batch * r.N1, r.src_nbytes, RB, const_cast<uint8_t*>(r.bwd.db_rows),
+                       pad, DT == FASTNN_I8 ? const_cast<int*>(r.fwd.q_absmax) : nullptr, gtid,
+                       gsize);
+      repack_in_kernel(r.src2, r.batch * r.N2, r.src_nbytes, RB, const_cast<uint8_t*>(r.fwd.db_rows),
+                       pad, DT == FASTNN_I8 ? const_cast<int*>(r.fwd.db_absmax) : nullptr, gtid,
+                       gsize);
+    }
+  };
+  fast_rounds<DT>(r, pass, repack, &ctl->abort_flag, &ctl->grid_ok, &ctl->more, ctl->scan);
   pipe_teardown(ctl, tmem, r.status);
 }
 

@@ -9,11 +9,17 @@ Two ways the path shards:
   replicas only.
 * Sharded dense mutual nearest neighbours of one pair
   (``sharded_mutual_dense``). Rank r finds the nearest neighbours of its block
-  of image-1 rows (against all of image 2) and of its block of image-2 rows
-  (against all of image 1) with the tensor-core kernel. The one exchange is an
-  all-gather of the image-2 partner indices (4 bytes per pixel); each rank
-  then tests mutuality for its own image-1 rows on its GPU and emits them in
-  ascending order, so the concatenation over ranks is the dense set.
+  of image-1 rows against all of image 2 with the tensor-core kernel. A pair
+  (i, j) of the reciprocal set has j = NN12(i), so only the image-2 rows that
+  some image-1 row matches (the image of NN12) need their own nearest
+  neighbour: the forward results are all-gathered (4 bytes per image-1
+  pixel), every rank lists that image with the library (ascending, so the
+  same list everywhere), and rank r runs the backward pass on its block of
+  the list alone -- about half of image 2 on the synthetic pairs, as on one
+  GPU. The backward results are all-gathered too (4 bytes per listed row);
+  each rank then tests mutuality for its own image-1 rows on its GPU and
+  emits them in ascending order, so the concatenation over ranks is the
+  dense set.
 
 The compute steps are passed in as callables (defaulting to the CUDA library)
 so that the host-side logic -- shard bounds, padding for the collective,
@@ -84,6 +90,12 @@ def _default_nn(q, db):
     return fastnn_nn(q, db)
 
 
+def _default_image(nn12_all, n2):
+    from . import fastnn_image_rows
+    rows, count = fastnn_image_rows(nn12_all, n2)
+    return rows[: int(count[0])]
+
+
 def _default_emit(nn12, score12, i0, nn21, n1_total):
     from . import fastnn_mutual_from_nn
     pairs, score, count = fastnn_mutual_from_nn(nn12, score12, i0, nn21, n1_total)
@@ -93,11 +105,12 @@ def _default_emit(nn12, score12, i0, nn21, n1_total):
 
 def sharded_mutual_dense(desc1: torch.Tensor, desc2: torch.Tensor, group=None,
                          nn: Callable | None = None, emit: Callable | None = None,
-                         gather: bool = True):
+                         image: Callable | None = None, gather: bool = True):
     """Dense mutual nearest-neighbour pairs of one pair, rows split across ranks.
 
     ``desc1`` [n1, d] and ``desc2`` [n2, d] are the full maps on every rank.
-    ``nn(q, db) -> (idx int32, score)`` and
+    ``nn(q, db) -> (idx int32, score)``,
+    ``image(nn12_all, n2) -> rows`` (ascending image-2 rows named by NN12) and
     ``emit(nn12, score12, i0, nn21, n1_total) -> (pairs, scores)`` default to
     the CUDA library. Returns this rank's pairs (global indices, ascending
     image-1 index), or, with ``gather``, every rank's pairs in rank order --
@@ -105,14 +118,24 @@ def sharded_mutual_dense(desc1: torch.Tensor, desc2: torch.Tensor, group=None,
     """
     nn = nn or _default_nn
     emit = emit or _default_emit
+    image = image or _default_image
     rank, world = _rank_world(group)
     n1, n2 = desc1.shape[0], desc2.shape[0]
     lo1, hi1 = shard_bounds(n1, rank, world)
-    lo2, hi2 = shard_bounds(n2, rank, world)
     idx12, s12 = nn(desc1[lo1:hi1].contiguous(), desc2)
-    idx21_local, _ = nn(desc2[lo2:hi2].contiguous(), desc1)
-    idx21 = all_gather_blocks(idx21_local, n2, group)  # the one exchange: 4 B per pixel
-    pairs, scores = emit(idx12, s12, lo1, idx21, n1)
+    idx12_all = all_gather_blocks(idx12, n1, group)  # exchange 1: 4 B per image-1 pixel
+    rows = image(idx12_all, n2)  # the same ascending list on every rank
+    lo2, hi2 = shard_bounds(rows.numel(), rank, world)
+    mine = rows[lo2:hi2]
+    if mine.numel() > 0:
+        idx21_mine, _ = nn(desc2.index_select(0, mine.long()).contiguous(), desc1)
+    else:
+        idx21_mine = torch.zeros(0, dtype=torch.int32, device=desc1.device)
+    idx21_rows = all_gather_blocks(idx21_mine, rows.numel(), group)  # exchange 2: 4 B per row
+    # NN21 of every image-2 row that can be in a pair; -1 (no partner) elsewhere.
+    nn21 = torch.full((n2,), -1, dtype=torch.int32, device=desc1.device)
+    nn21[rows.long()] = idx21_rows
+    pairs, scores = emit(idx12, s12, lo1, nn21, n1)
     if gather:
         pairs = gather_varlen(pairs, group)
         scores = gather_varlen(scores, group)

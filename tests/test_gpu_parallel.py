@@ -8,8 +8,8 @@ import torch
 
 import oracle
 import synth
-from reciprocal_nearest_neighbours_b200 import (fastnn_mutual_dense, fastnn_mutual_from_nn,
-                                                fastnn_nn, parallel)
+from reciprocal_nearest_neighbours_b200 import (fastnn_image_rows, fastnn_mutual_dense,
+                                                fastnn_mutual_from_nn, fastnn_nn, parallel)
 from tests._dev import require_cuda, to_dev
 
 pytestmark = pytest.mark.gpu
@@ -57,20 +57,40 @@ def test_sharded_path_single_rank_equals_dense_kernel():
     assert np.array_equal(pairs.cpu().numpy().astype(np.int64), dm.pairs)
 
 
+def test_image_rows_are_the_sorted_distinct_partners():
+    rng = np.random.default_rng(3)
+    for n1, n2 in [(1, 1), (5000, 3000), (3000, 50000), (4097, 4097), (10, 8191)]:
+        nn12 = rng.integers(-3, n2 + 3, size=n1).astype(np.int32)  # a few out of range
+        rows, count = fastnn_image_rows(torch.from_numpy(nn12).cuda(), n2)
+        exp = np.unique(nn12[(nn12 >= 0) & (nn12 < n2)])
+        assert int(count[0]) == len(exp)
+        assert np.array_equal(rows[: len(exp)].cpu().numpy(), exp)
+    rows, count = fastnn_image_rows(torch.zeros(0, dtype=torch.int32, device="cuda"), 100)
+    assert int(count[0]) == 0
+
+
 def test_sharded_path_rank_blocks_compose_on_one_gpu():
-    """Emulate two ranks' row blocks on one GPU (no collective needed) and check
-    that the concatenated per-rank outputs form the dense set."""
+    """Emulate two ranks' row blocks on one GPU (the collectives become
+    concatenations) and check that the concatenated per-rank outputs form the
+    dense set, with the backward passes restricted to the image of NN12."""
     m = synth.warped_pair_int8(99, H=48, W=64, d=24)
     D1 = to_dev(m.desc1.reshape(-1, 24))
     D2 = to_dev(m.desc2.reshape(-1, 24))
     n1, n2 = D1.shape[0], D2.shape[0]
-    idx21 = torch.cat([fastnn_nn(D2[lo:hi].contiguous(), D1)[0]
-                       for lo, hi in (parallel.shard_bounds(n2, r, 2) for r in range(2))])
+    blocks1 = [parallel.shard_bounds(n1, r, 2) for r in range(2)]
+    fwd = [fastnn_nn(D1[lo:hi].contiguous(), D2) for lo, hi in blocks1]
+    nn12_all = torch.cat([f[0] for f in fwd])
+    rows, count = fastnn_image_rows(nn12_all, n2)
+    rows = rows[: int(count[0])]
+    assert rows.numel() < n2
+    blocks2 = [parallel.shard_bounds(rows.numel(), r, 2) for r in range(2)]
+    idx21_rows = torch.cat([fastnn_nn(D2.index_select(0, rows[lo:hi].long()).contiguous(), D1)[0]
+                            for lo, hi in blocks2])
+    nn21 = torch.full((n2,), -1, dtype=torch.int32, device="cuda")
+    nn21[rows.long()] = idx21_rows
     out = []
-    for r in range(2):
-        lo, hi = parallel.shard_bounds(n1, r, 2)
-        i12, s12 = fastnn_nn(D1[lo:hi].contiguous(), D2)
-        pr, sc, c = fastnn_mutual_from_nn(i12, s12, lo, idx21, n1)
+    for (lo, hi), (i12, s12) in zip(blocks1, fwd):
+        pr, sc, c = fastnn_mutual_from_nn(i12, s12, lo, nn21, n1)
         out.append(pr[: int(c[0])])
     ref_p, _, ref_c = fastnn_mutual_dense(D1, D2)
     assert torch.equal(torch.cat(out), ref_p[: int(ref_c[0])])

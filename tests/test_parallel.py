@@ -48,6 +48,11 @@ def _oracle_nn(q, db):
     return torch.from_numpy(r.idx.copy()), torch.from_numpy(r.score.astype(np.int32))
 
 
+def _cpu_image(nn12_all, n2):
+    v = nn12_all.numpy()
+    return torch.from_numpy(np.unique(v[(v >= 0) & (v < n2)]).astype(np.int32))
+
+
 def _cpu_emit(nn12, score12, i0, nn21, n1_total):
     i = torch.arange(nn12.numel(), dtype=torch.int64) + i0
     keep = nn21[nn12.long()].long() == i
@@ -67,8 +72,16 @@ def _worker(rank, world, port, task, out_dir):
             p = synth.warped_pair_int8(4242, H=24, W=40, d=24)
             d1 = torch.from_numpy(p.desc1.reshape(-1, 24))
             d2 = torch.from_numpy(p.desc2.reshape(-1, 24)[:777])  # n2 != n1, uneven shards
-            pairs, scores = parallel.sharded_mutual_dense(d1, d2, nn=_oracle_nn, emit=_cpu_emit)
-            torch.save((pairs, scores), os.path.join(out_dir, f"dense_{rank}.pt"))
+            backward_rows = []
+
+            def nn(q, db):
+                if db.shape[0] == d1.shape[0]:  # the backward pass: queries are image-2 rows
+                    backward_rows.append(q.shape[0])
+                return _oracle_nn(q, db)
+            pairs, scores = parallel.sharded_mutual_dense(d1, d2, nn=nn, emit=_cpu_emit,
+                                                          image=_cpu_image)
+            torch.save((pairs, scores, sum(backward_rows)),
+                       os.path.join(out_dir, f"dense_{rank}.pt"))
         else:
             pairs_in = [synth.warped_pair_int8(77 + b, H=16, W=24, d=24) for b in range(5)]
             d1 = torch.from_numpy(np.stack([q.desc1 for q in pairs_in]))
@@ -107,11 +120,16 @@ def test_sharded_dense_mutual_over_gloo_equals_single_process(world, tmp_path):
     D1 = p.desc1.reshape(-1, 24)
     D2 = p.desc2.reshape(-1, 24)[:777]
     ref = oracle.dense_mutual(D1, D2, "i8")
+    backward = 0
     for r in range(world):
-        pairs, scores = torch.load(tmp_path / f"dense_{r}.pt")
+        pairs, scores, rows = torch.load(tmp_path / f"dense_{r}.pt")
         assert np.array_equal(pairs.numpy().astype(np.int64), ref.pairs)
         assert np.array_equal(scores.numpy().astype(np.int64), ref.score)
+        backward += rows
     assert len(ref.pairs) > 50
+    # the backward passes together ran exactly the image of NN12, not all of image 2
+    image = np.unique(ref.nn12.idx)
+    assert backward == len(image) < D2.shape[0]
 
 
 def test_pair_parallel_fast_matching_over_gloo(tmp_path):
