@@ -483,38 +483,50 @@ class Runner:
             self.launches_per_step = 1 if in_kernel else 3
             self.kernels_per_step = 1
 
-    def call(self):
-        fnn, w = self.fnn, self.w
-        if w.dense:
-            fnn.fastnn_mutual_dense(self.d1, self.d2, out_pairs=self.out_pairs,
-                                    out_score=self.out_score, out_count=self.out_count,
-                                    workspace=self.ws, stream=self.stream)
-        elif self.masked:
-            fnn.fastnn_reciprocal_masked(self.d1, self.d2, w.subsample, w.max_iter, conf1=self.c1,
-                                         conf2=self.c2, threshold=w.extra["threshold"],
-                                         out_pairs=self.out_pairs, out_score=self.out_score,
-                                         out_count=self.out_count, out_iters=self.out_iters,
-                                         out_frontier=self.out_front, workspace=self.ws,
-                                         stream=self.stream)
-        else:
-            fnn.fastnn_reciprocal(self.d1, self.d2, w.subsample, w.max_iter,
-                                  out_pairs=self.out_pairs, out_score=self.out_score,
-                                  out_count=self.out_count, out_iters=self.out_iters,
-                                  out_frontier=self.out_front, workspace=self.ws,
-                                  stream=self.stream)
+    def buffers(self):
+        """The device inputs and outputs of one call."""
+        return {k: getattr(self, k, None) for k in
+                ("d1", "d2", "c1", "c2", "out_pairs", "out_score", "out_count", "out_iters",
+                 "out_front")}
 
-    def call_e2e(self):
-        """One step through the public API with host buffers: inputs copied in
-        from pinned memory, the call, every output copied back."""
-        self.d1.copy_(self.h1, non_blocking=True)
-        self.d2.copy_(self.h2, non_blocking=True)
+    def second_buffers(self):
+        """A second set of device inputs and outputs (the end-to-end pipeline's
+        double buffer)."""
+        return {k: (v.clone() if v is not None else None) for k, v in self.buffers().items()}
+
+    def call(self, buf=None, stream=None):
+        fnn, w = self.fnn, self.w
+        b = buf or self.buffers()
+        st = stream or self.stream
+        if w.dense:
+            fnn.fastnn_mutual_dense(b["d1"], b["d2"], out_pairs=b["out_pairs"],
+                                    out_score=b["out_score"], out_count=b["out_count"],
+                                    workspace=self.ws, stream=st)
+        elif self.masked:
+            fnn.fastnn_reciprocal_masked(b["d1"], b["d2"], w.subsample, w.max_iter,
+                                         conf1=b["c1"], conf2=b["c2"],
+                                         threshold=w.extra["threshold"],
+                                         out_pairs=b["out_pairs"], out_score=b["out_score"],
+                                         out_count=b["out_count"], out_iters=b["out_iters"],
+                                         out_frontier=b["out_front"], workspace=self.ws,
+                                         stream=st)
+        else:
+            fnn.fastnn_reciprocal(b["d1"], b["d2"], w.subsample, w.max_iter,
+                                  out_pairs=b["out_pairs"], out_score=b["out_score"],
+                                  out_count=b["out_count"], out_iters=b["out_iters"],
+                                  out_frontier=b["out_front"], workspace=self.ws, stream=st)
+
+    def copy_in(self, b):
+        b["d1"].copy_(self.h1, non_blocking=True)
+        b["d2"].copy_(self.h2, non_blocking=True)
         if self.masked:
-            self.c1.copy_(self.hc1, non_blocking=True)
-            self.c2.copy_(self.hc2, non_blocking=True)
-        self.call()
-        self.hp_count.copy_(self.out_count, non_blocking=True)
-        self.hp_pairs.copy_(self.out_pairs, non_blocking=True)
-        self.hp_score.copy_(self.out_score, non_blocking=True)
+            b["c1"].copy_(self.hc1, non_blocking=True)
+            b["c2"].copy_(self.hc2, non_blocking=True)
+
+    def copy_out(self, b):
+        self.hp_count.copy_(b["out_count"], non_blocking=True)
+        self.hp_pairs.copy_(b["out_pairs"], non_blocking=True)
+        self.hp_score.copy_(b["out_score"], non_blocking=True)
 
     def bytes_per_step(self):
         bin_ = (self.N1 + self.N2) * self.d * self.esize * self.B + \
@@ -537,31 +549,67 @@ class Runner:
         return int(self.out_front.cpu().sum()) * (self.N1 + self.N2), None
 
 
-def time_steps(run, K, flush, ranks, e2e=False):
+def time_steps(run, K, flush, ranks):
     """K steps, L2 flushed before each; CUDA events on the launching stream
     around each step. Returns per-step ms (max over ranks) and this rank's
     (timed kernel launches, kernel ms)."""
     torch, fnn = run.torch, run.fnn
-    if not e2e:
-        fnn.fastnn_kernel_timer_enable(K * run.kernels_per_step + 8)
+    fnn.fastnn_kernel_timer_enable(K * run.kernels_per_step + 8)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(K)]
     ranks.barrier()
     for i in range(K):
         flush.zero_()
         evs[i][0].record(run.stream)
-        if e2e:
-            run.call_e2e()
-        else:
-            run.call()
+        run.call()
         evs[i][1].record(run.stream)
     ranks.barrier()
     ms = [s.elapsed_time(e) for s, e in evs]
-    nn = (0, 0.0)
-    if not e2e:
-        nn = fnn.fastnn_kernel_timer_read()
-        fnn.fastnn_kernel_timer_enable(0)
+    nn = fnn.fastnn_kernel_timer_read()
+    fnn.fastnn_kernel_timer_enable(0)
     return ranks.max(ms), nn
+
+
+def time_end_to_end(run, K, ranks):
+    """K steps through the public API with host buffers, as a stream of pairs
+    is matched: every step copies its inputs in from pinned host memory, runs
+    the call and copies every output back. Two device buffer sets and two copy
+    streams (inputs, outputs) let step i + 1's inputs and step i - 1's outputs
+    cross the bus while step i runs; the events bracket the first copy in and
+    the last copy out. Returns the total ms (max over ranks)."""
+    torch = run.torch
+    bufs = [run.buffers(), run.second_buffers()]
+    cin, cout = torch.cuda.Stream(device=run.dev), torch.cuda.Stream(device=run.dev)
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    done = [ev(), ev()]      # compute of the last step on buffer set s finished
+    copied = [ev(), ev()]    # outputs of the last step on set s copied out
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for s in range(2):
+        done[s].record(run.stream)
+        copied[s].record(cout)
+    ranks.barrier()
+    start.record(cin)
+    for i in range(K):
+        s = i & 1
+        b = bufs[s]
+        inp = ev()
+        with torch.cuda.stream(cin):
+            cin.wait_event(done[s])  # step i - 2 no longer reads set s
+            run.copy_in(b)
+            inp.record(cin)
+        run.stream.wait_event(inp)
+        run.stream.wait_event(copied[s])  # step i - 2's outputs are out of set s
+        run.call(b)
+        done[s].record(run.stream)
+        with torch.cuda.stream(cout):
+            cout.wait_event(done[s])
+            run.copy_out(b)
+            copied[s].record(cout)
+    cout.wait_stream(cin)
+    end.record(cout)
+    ranks.barrier()
+    end.synchronize()
+    return ranks.max([start.elapsed_time(end)])[0]
 
 
 def roofline_for(run, work, image, K, nn_launches, nn_ms, total_ms):
@@ -633,7 +681,7 @@ def measure(name, K, W, rank, ranks, dev, stream, flush, sample_clocks, e2e_step
     assert run.matches() == matches
     e2e_ms = None
     if e2e_steps:
-        e2e_ms, _ = time_steps(run, e2e_steps, flush, ranks, e2e=True)
+        e2e_ms = time_end_to_end(run, e2e_steps, ranks)
         assert int(run.hp_count.sum()) == matches
     total_ms = sum(step_ms)
     nn_ms = ranks.max([nn_ms])[0]
@@ -655,9 +703,11 @@ def measure(name, K, W, rank, ranks, dev, stream, flush, sample_clocks, e2e_step
         res["frontier_per_round_pair0"] = run.out_front[0].cpu().tolist()
     if e2e_ms is not None:
         bin_, bout = run.bytes_per_step()
-        res["e2e"] = {"value": all_matches * e2e_steps / (sum(e2e_ms) / 1e3), "unit": UNIT,
+        res["e2e"] = {"value": all_matches * e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
                       "h2d_bytes_per_step": bin_, "d2h_bytes_per_step": bout,
-                      "steps": e2e_steps, "ms_per_step_percentiles": percentiles(e2e_ms)}
+                      "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps,
+                      "pipeline": "step i+1's inputs and step i-1's outputs are copied on two "
+                                  "copy streams while step i runs (two device buffer sets)"}
     res["_workload"] = run.w
     return res
 
