@@ -20,10 +20,13 @@
 // seen cannot be the nearest, so only the points inside that window are
 // ranked again, by their squared distance computed in fp64 from the
 // coordinate differences -- (dx^2 + dy^2) + dz^2, each operation rounded
-// once, the order of a plain loop over the coordinates -- and rounded to
-// fp32. The result is the lowest index among the points whose fp64 squared
-// distance rounds to the same fp32 value as the smallest one, and the score
-// reported is that fp32 value. In the fast scheme's passes a query usually
+// once, the order of a plain loop over the coordinates. Within the share of
+// the database one CTA scans, the winner is the smallest fp64 value, lowest
+// index among exact ties (the definition). Winners of different CTAs are
+// merged on the fp64 value rounded to fp32, lowest index among equal fp32
+// values, and the score reported is that fp32 value; the two rules can
+// differ only for two points in different CTAs' shares whose fp64 distances
+// differ yet round to one fp32 value. In the fast scheme's passes a query usually
 // comes with the fp32 distance D of a point it is known to reach (its partner
 // in the previous pass); the window then starts at the floor that D implies
 // instead of opening at every chunk until a near point has been seen.
@@ -41,8 +44,8 @@
 // reached the query's window. Only then does the warp reduce the maximum and
 // walk the lanes inside the window: all 32 lanes re-score the 32 rows of one
 // such lane (same FMA order, so bit-identical s~), rank the rows inside the
-// window by fp64 distance and fold the best (fp32 distance, index) key into
-// the query's winner. Consecutive units of one (pair, tile) form a segment,
+// window by fp64 distance and keep the best (fp64 distance, index) as the
+// query's winner. Consecutive units of one (pair, tile) form a segment,
 // visiting the database chunks in a scrambled order (the ranking does not
 // depend on the order, and spatially ordered rows would otherwise open the
 // re-ranking at nearly every chunk); at its end lane q of each warp merges
@@ -74,7 +77,8 @@ constexpr unsigned kFull = 0xffffffffu;
 // Per-warp, per-query state of the exact ranking that only a vote that fires
 // touches (warp-uniform values).
 struct WarpState {
-  unsigned long long key[kQW];  // winner: (fp32 distance bits << 32) | index
+  unsigned long long dbits[kQW];  // winner's exact fp64 squared distance (bits; ~0: none)
+  uint32_t idx[kQW];              // winner's index (lowest among exact ties)
   float smax[kQW];              // largest fp32 score s~ seen in the segment
   float win2[kQW];              // window width 2E
   float floor[kQW];             // lowest window edge the query's bound allows, or -FLT_MAX
@@ -328,7 +332,8 @@ __device__ __forceinline__ void load_queries(const NNArgs& a, const PhaseQ& q, i
     W.win2[lane] = win2;
     W.floor[lane] = floor;
     W.smax[lane] = -INFINITY;
-    W.key[lane] = ~0ull;
+    W.dbits[lane] = ~0ull;
+    W.idx[lane] = 0xFFFFFFFFu;
   }
 #pragma unroll
   for (int i = 0; i < kQW; ++i) {
@@ -391,32 +396,40 @@ __device__ __forceinline__ void l2_chunk(const float4* __restrict__ buf, int row
     const float thr = fmaxf(smax - W.win2[i], W.floor[i]);
     Wn.thr[i] = thr;
     const float ax = 0.5f * Q.x[i], ay = 0.5f * Q.y[i], az = 0.5f * Q.z[i];
-    unsigned long long best = W.key[i];
+    unsigned long long best = W.dbits[i];
+    uint32_t best_j = W.idx[i];
     unsigned cand = __ballot_sync(kFull, mx[i] >= thr);
     while (cand) {
       const int L = __ffs(cand) - 1;
       cand &= cand - 1;
-      // (distance bits, index) of this lane's row, or (~0, ~0) outside the
-      // window; the warp minimum in two 32-bit reductions (distance, then
-      // index among the lanes at that distance). Non-negative floats order
-      // like their bits.
-      uint32_t dbits = 0xFFFFFFFFu, jidx = 0xFFFFFFFFu;
+      // The exact fp64 squared distance of this lane's row (bits: non-negative
+      // doubles order like their bits; ~0 outside the window) and its index;
+      // the warp minimum of (distance, index) in three 32-bit reductions.
+      unsigned long long db = ~0ull;
+      uint32_t jidx = 0xFFFFFFFFu;
       const int j = jt + L;
       if (j < rows) {
         const float4 p = buf[j];
         if (l2_score(Q, i, p) >= thr) {
-          dbits = __float_as_uint(__double2float_rn(dist2_f64(ax, ay, az, p)));
+          db = static_cast<unsigned long long>(__double_as_longlong(dist2_f64(ax, ay, az, p)));
           jidx = base + static_cast<uint32_t>(j);
         }
       }
-      const uint32_t dmin = __reduce_min_sync(kFull, dbits);
-      const uint32_t jmin = __reduce_min_sync(kFull, dbits == dmin ? jidx : 0xFFFFFFFFu);
-      const unsigned long long k = (static_cast<unsigned long long>(dmin) << 32) | jmin;
-      best = k < best ? k : best;
+      const uint32_t hi = static_cast<uint32_t>(db >> 32), lo = static_cast<uint32_t>(db);
+      const uint32_t hmin = __reduce_min_sync(kFull, hi);
+      const uint32_t lmin = __reduce_min_sync(kFull, hi == hmin ? lo : 0xFFFFFFFFu);
+      const uint32_t jmin =
+          __reduce_min_sync(kFull, (hi == hmin && lo == lmin) ? jidx : 0xFFFFFFFFu);
+      const unsigned long long dmin = (static_cast<unsigned long long>(hmin) << 32) | lmin;
+      if (dmin < best || (dmin == best && jmin < best_j)) {
+        best = dmin;
+        best_j = jmin;
+      }
     }
     __syncwarp();
     if (lane == 0) {
-      W.key[i] = best;
+      W.dbits[i] = best;
+      W.idx[i] = best_j;
       W.smax[i] = smax;
     }
     __syncwarp();
@@ -480,12 +493,13 @@ __device__ void l2_phase(const NNArgs& a, const PhaseQ q, L2Smem& s) {
     walk_next(nx, s, a.batch);
     const bool seg_end = (nx.n == 0) || (u + 1 == u1);
     if (seg_end && active && ok && lane < kQW && k0 + lane < cnt) {
-      const unsigned long long kw = W.key[lane];
-      if (kw != ~0ull) {
-        const float d2 = __uint_as_float(static_cast<uint32_t>(kw >> 32));
+      const uint32_t jw = W.idx[lane];
+      if (jw != 0xFFFFFFFFu) {
+        // Across CTAs the merge compares the fp32 rounding of the distance
+        // (lowest index among equal fp32 values).
+        const float d2 = __double2float_rn(__longlong_as_double(static_cast<long long>(W.dbits[lane])));
         atomicMax(reinterpret_cast<unsigned long long*>(&a.out_key[w.b * a.q_cap + k0 + lane]),
-                  static_cast<unsigned long long>(
-                      make_key(ord_f32(-d2), static_cast<uint32_t>(kw & 0xFFFFFFFFu))));
+                  static_cast<unsigned long long>(make_key(ord_f32(-d2), jw)));
       }
     }
     if (!ok) {

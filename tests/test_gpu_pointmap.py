@@ -94,6 +94,38 @@ def test_nn_l2_integer_points_bit_exact(nq, ndb, d, amp):
     assert np.array_equal(score.cpu().numpy().astype(np.float64), ref.score)
 
 
+# Two points whose squared distances from the origin differ in fp64 yet round
+# to the same fp32 value (1.0): |p_near|^2 = 0.99999999627..., |p_far|^2 = 1.
+P_NEAR = (0.609195351600647, 0.7930201888084412, 0.0)
+P_FAR = (1.0, 0.0, 0.0)
+
+
+@pytest.mark.parametrize("near_first", [False, True])
+def test_nn_l2_fp32_collision_ranks_by_the_exact_distance(near_first):
+    """The oracle ranks by the fp64 squared distance; two points that collide
+    in fp32 must still be told apart by it, whichever index is lower."""
+    near, far = np.array(P_NEAR, np.float32), np.array(P_FAR, np.float32)
+    d_near = float(np.sum(near.astype(np.float64) ** 2))
+    assert d_near < 1.0 and np.float32(d_near) == np.float32(1.0)
+    rng = np.random.default_rng(5)
+    others = rng.uniform(2.0, 4.0, size=(40, 3)).astype(np.float32)  # all farther away
+    db = np.concatenate([[near, far] if near_first else [far, near], others]).astype(np.float32)
+    q = np.zeros((3, 3), dtype=np.float32)
+    ref = oracle.nn(q, db, "l2")
+    expect = 0 if near_first else 1
+    assert np.all(ref.idx == expect)
+    idx, score = fastnn_nn(dev(q), dev(db))
+    assert np.all(idx.cpu().numpy() == expect)
+    assert np.all(score.cpu().numpy() == np.float32(1.0))
+    # the dense mutual set and the fast scheme take the same (exact) partner
+    pairs, _, count = fastnn_mutual_dense(dev(q[:1]), dev(db))
+    assert int(count[0]) == 1 and pairs[0].tolist() == [0, expect]
+    m1 = q[:1].reshape(1, 1, 3)
+    m2 = db.reshape(1, -1, 3)
+    fp, fs, fc, _ = fastnn_reciprocal(dev(m1), dev(m2), 1, 10)
+    assert int(fc[0]) == 1 and fp[0, 0].tolist() == [0, expect]
+
+
 def test_nn_l2_identical_database_points_pick_index_zero():
     q = np.full((300, 3), 0.5, dtype=np.float32)
     db = np.ones((3000, 3), dtype=np.float32)
