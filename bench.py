@@ -720,8 +720,8 @@ STREAM_ROWS = 64 << 20  # 67,108,864 rows: inputs far larger than L2
 
 
 def measure_stream(K, ranks, dev, stream, flush, sample_clocks):
-    """Achieved HBM bandwidth of the repack, dense mutual test/emit and
-    confidence-mask compaction kernels on a 64M-row int8 map (d = 24; a few
+    """Achieved HBM bandwidth of the repack, dense mutual test/emit, image-row
+    list and confidence-mask compaction kernels on a 64M-row int8 map (d = 24; a few
     GB on the device). Each kind is timed with the library's launch timer
     restricted to that kind, inside an ordinary call:
       repack  -- fastnn_nn of the 64M-row map against a 256-row database
@@ -729,6 +729,9 @@ def measure_stream(K, ranks, dev, stream, flush, sample_clocks):
       mutual  -- fastnn_mutual_from_nn on 64M-row index arrays of a smooth
                  synthetic correspondence (count, scan and ordered emit:
                  2 x 8 B read per row, 16 B per kept pair);
+      image   -- fastnn_image_rows of the same 64M-row NN12 (the list the
+                 sharded dense backward pass runs on: 4 B read per row,
+                 4 B written per listed image-2 row);
       mask    -- fastnn_mutual_dense_masked of the 64M-row map (confidences
                  uniform in [0, 1), threshold 0.5) against a 256-row map
                  (map 1's compaction: 2 x 4 B of confidence and the 24 B row
@@ -800,7 +803,18 @@ def measure_stream(K, ranks, dev, stream, flush, sample_clocks):
     r["kind"] = "mutual test and ordered emit (mutual_count, mutual_scan, mutual_emit)"
     r["kept"] = int(cnt.item())
     out["kernels"].append(r)
-    del off, ar, nn12, nn21, miss, score, mws, pairs, pscore
+    del nn21, miss, score, pairs, pscore
+    rows = torch.empty(N, dtype=torch.int32, device=dev)
+    iws = torch.empty(fnn.fastnn_workspace_size(fnn.FASTNN_OP_IMAGE_ROWS, N, N, 1, fnn.FASTNN_I8),
+                      dtype=torch.uint8, device=dev)
+    r = timed(fnn.FASTNN_TIME_MUTUAL,
+              lambda: fnn.fastnn_image_rows(nn12, N, out_rows=rows, out_count=cnt, workspace=iws),
+              lambda: 4 * N + 4 * int(cnt.item()))
+    r["kind"] = ("image-2 rows of an NN12 (image_flag, image_rows_count, scan, "
+                 "image_rows_emit: 4 B read per image-1 row, 4 B written per listed row)")
+    r["listed"] = int(cnt.item())
+    out["kernels"].append(r)
+    del off, ar, nn12, mws, iws, rows
 
     conf = torch.rand(N, device=dev, generator=g)
     kept1 = int((conf >= 0.5).sum().item())
