@@ -112,6 +112,10 @@ struct PhaseQ {
   // to reach, so that only larger-or-equal scores need a record.
   const uint32_t* bound;
   int bstride;
+  // 1: the CTA's per-pair count cache in shared memory already holds this
+  // phase's query counts (read by the previous phase, or by the round loop's
+  // check after the compaction), so the planner skips their load.
+  int cached = 0;
 };
 
 // Counts, frontier indices and keys may have been written by other CTAs of

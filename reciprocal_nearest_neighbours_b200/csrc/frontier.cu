@@ -141,10 +141,13 @@ __global__ void __launch_bounds__(kRepackThreads)
 // scores (a row shard of image 1 checked against the full NN21 gathered from
 // every rank). Three passes keep the output in ascending i without inter-CTA
 // waiting: per-block counts, one scan block, ordered emit.
-// A block of 1024 threads covers kMutBlockRows rows; thread t takes the four
-// consecutive rows 4t .. 4t + 3, read with 16-byte loads where aligned.
-constexpr int kMutRowsPerThread = 4;
-constexpr int kMutBlockRows = 1024 * kMutRowsPerThread;
+// A block covers kMutBlockRows rows. In the mutual test thread t of
+// kMutThreads takes the eight consecutive rows 8t .. 8t + 7, two groups of
+// four read with 16-byte loads where aligned, whose gathers of the partners'
+// back-matches are in flight together.
+constexpr int kMutBlockRows = 4096;
+constexpr int kMutRowsPerThread = 8;
+constexpr int kMutThreads = kMutBlockRows / kMutRowsPerThread;
 
 // Flags (and partners) of rows i .. i + 3 (local indices). The partners'
 // back-matches are loaded together, after all four partners are known.
@@ -183,14 +186,18 @@ __device__ __forceinline__ void mutual_flags4(const MutualSrc& m, int64_t i, boo
   }
 }
 
-__global__ void __launch_bounds__(1024) mutual_count_kernel(MutualSrc m,
-                                                            int32_t* __restrict__ block_cnt) {
+__global__ void __launch_bounds__(kMutThreads) mutual_count_kernel(MutualSrc m,
+                                                                   int32_t* __restrict__ block_cnt) {
   __shared__ int sm[32];
-  const int64_t i = blockIdx.x * static_cast<int64_t>(kMutBlockRows) + 4 * threadIdx.x;
-  bool f[4];
-  uint32_t j[4];
-  mutual_flags4(m, i, f, j);
-  int c = (f[0] ? 1 : 0) + (f[1] ? 1 : 0) + (f[2] ? 1 : 0) + (f[3] ? 1 : 0);
+  const int64_t i =
+      blockIdx.x * static_cast<int64_t>(kMutBlockRows) + kMutRowsPerThread * threadIdx.x;
+  bool f[2][4];
+  uint32_t j[2][4];
+  mutual_flags4(m, i, f[0], j[0]);
+  mutual_flags4(m, i + 4, f[1], j[1]);
+  int c = 0;
+#pragma unroll
+  for (int r = 0; r < 8; ++r) c += f[r >> 2][r & 3] ? 1 : 0;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
   if ((threadIdx.x & 31) == 0) sm[threadIdx.x >> 5] = c;
@@ -220,62 +227,84 @@ __device__ __forceinline__ int block_exclusive_scan(int c, int* sm) {
 
 // Exclusive scan, in place, of the nblocks counts of segment blockIdx.x
 // (block_cnt + blockIdx.x * nblocks); the segment's total goes to
-// out_count[blockIdx.x]. Each thread scans a contiguous run of the counts;
-// one block-wide scan of the runs' totals joins them (a single pass, however
-// many counts).
+// out_count[blockIdx.x]. The counts go through shared memory in tiles of
+// kScanTile: coalesced loads, kScanPer consecutive counts per thread (the
+// index is padded by one word per 32 so that those reads are free of bank
+// conflicts), one block scan of the per-thread sums, coalesced stores; the
+// running total carries from tile to tile.
+constexpr int kScanPer = 8;
+constexpr int kScanTile = 1024 * kScanPer;
+
+__device__ __forceinline__ int scan_slot(int k) { return k + (k >> 5); }
+
 __global__ void __launch_bounds__(1024) mutual_scan_kernel(int32_t* __restrict__ block_cnt,
                                                            int nblocks,
                                                            int32_t* __restrict__ out_count) {
   block_cnt += static_cast<int64_t>(blockIdx.x) * nblocks;
   out_count += blockIdx.x;
+  __shared__ int buf[kScanTile + kScanTile / 32];
   __shared__ int sm[32];
-  const int per = (nblocks + static_cast<int>(blockDim.x) - 1) / static_cast<int>(blockDim.x);
-  const int k0 = min(static_cast<int>(threadIdx.x) * per, nblocks);
-  const int k1 = min(k0 + per, nblocks);
-  int sum = 0;
-#pragma unroll 8
-  for (int k = k0; k < k1; ++k) sum += block_cnt[k];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int x = sum;
+  __shared__ int carry_s;
+  int carry = 0;
+  for (int t0 = 0; t0 < nblocks; t0 += kScanTile) {
+    const int n = min(kScanTile, nblocks - t0);
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
+    for (int i = 0; i < kScanPer; ++i) {
+      const int k = static_cast<int>(threadIdx.x) + 1024 * i;
+      buf[scan_slot(k)] = k < n ? block_cnt[t0 + k] : 0;
+    }
+    __syncthreads();
+    int v[kScanPer];
+    int sum = 0;
+#pragma unroll
+    for (int i = 0; i < kScanPer; ++i) {
+      v[i] = buf[scan_slot(static_cast<int>(threadIdx.x) * kScanPer + i)];
+      sum += v[i];
+    }
+    int run = carry + block_exclusive_scan(sum, sm);
+#pragma unroll
+    for (int i = 0; i < kScanPer; ++i) {
+      buf[scan_slot(static_cast<int>(threadIdx.x) * kScanPer + i)] = run;
+      run += v[i];
+    }
+    if (threadIdx.x == blockDim.x - 1) carry_s = run;
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < kScanPer; ++i) {
+      const int k = static_cast<int>(threadIdx.x) + 1024 * i;
+      if (k < n) block_cnt[t0 + k] = buf[scan_slot(k)];
+    }
+    carry = carry_s;
+    __syncthreads();  // buf, sm and carry_s are reused by the next tile
   }
-  if (lane == 31) sm[warp] = x;
-  __syncthreads();
-  int woff = 0;
-  for (int w = 0; w < warp; ++w) woff += sm[w];
-  int run = woff + x - sum;  // exclusive prefix of this thread's run
-  for (int k = k0; k < k1; ++k) {
-    const int v = block_cnt[k];
-    block_cnt[k] = run;
-    run += v;
-  }
-  if (threadIdx.x == blockDim.x - 1) *out_count = run;
+  if (threadIdx.x == 0) *out_count = carry;
 }
 
 template <int DT>
-__global__ void __launch_bounds__(1024) mutual_emit_kernel(MutualSrc m,
-                                                           const int32_t* __restrict__ block_off,
-                                                           int32_t* __restrict__ out_pairs,
-                                                           void* __restrict__ out_score,
-                                                           int64_t cap) {
+__global__ void __launch_bounds__(kMutThreads) mutual_emit_kernel(
+    MutualSrc m, const int32_t* __restrict__ block_off, int32_t* __restrict__ out_pairs,
+    void* __restrict__ out_score, int64_t cap) {
   __shared__ int sm[32];
-  const int64_t i = blockIdx.x * static_cast<int64_t>(kMutBlockRows) + 4 * threadIdx.x;
-  bool f[4];
-  uint32_t j[4];
-  mutual_flags4(m, i, f, j);
-  const int c = (f[0] ? 1 : 0) + (f[1] ? 1 : 0) + (f[2] ? 1 : 0) + (f[3] ? 1 : 0);
-  int64_t pos = block_off[blockIdx.x] + block_exclusive_scan(c, sm);
+  const int64_t i =
+      blockIdx.x * static_cast<int64_t>(kMutBlockRows) + kMutRowsPerThread * threadIdx.x;
+  bool f[2][4];
+  uint32_t j[2][4];
+  mutual_flags4(m, i, f[0], j[0]);
+  mutual_flags4(m, i + 4, f[1], j[1]);
+  int c = 0;
 #pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    if (!f[r]) continue;
+  for (int r = 0; r < 8; ++r) c += f[r >> 2][r & 3] ? 1 : 0;
+  int64_t pos = block_off[blockIdx.x] + block_exclusive_scan(c, sm);
+  const bool pair8 = (reinterpret_cast<uintptr_t>(out_pairs) & 7) == 0;
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    if (!f[r >> 2][r & 3]) continue;
     if (pos < cap) {
       const int64_t ir = i + r;
+      const uint32_t jr = j[r >> 2][r & 3];
       const int32_t a = m.map1 ? m.map1[ir] : static_cast<int32_t>(m.i0 + ir);
-      const int32_t bj = m.map2 ? m.map2[j[r]] : static_cast<int32_t>(j[r]);
-      if ((reinterpret_cast<uintptr_t>(out_pairs) & 7) == 0) {
+      const int32_t bj = m.map2 ? m.map2[jr] : static_cast<int32_t>(jr);
+      if (pair8) {
         *reinterpret_cast<int2*>(out_pairs + pos * 2) = make_int2(a, bj);
       } else {
         out_pairs[pos * 2] = a;
@@ -411,59 +440,94 @@ __global__ void __launch_bounds__(1024) image_emit_kernel(const uint64_t* __rest
 
 // ---------------------------------------------- image rows of an NN12 ---
 // The ascending list of image-2 rows j in [0, n2) that some nn12[i] names:
-// flags, per-block counts (4096 rows per block, four consecutive rows per
-// thread), the shared scan, an ordered emit.
+// byte flags, per-block counts, the shared scan, an ordered emit. A block of
+// kImgThreads threads covers kMutBlockRows rows (the scan's block count is
+// the dense mutual test's); thread t takes the 16 consecutive flags
+// 16t .. 16t + 15, one 16-byte load.
+constexpr int kImgFlagsPerThread = 16;
+constexpr int kImgThreads = kMutBlockRows / kImgFlagsPerThread;
+
 __global__ void image_flag_kernel(const int32_t* __restrict__ nn12, int64_t n1, int64_t n2,
                                   uint8_t* __restrict__ flag) {
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n1;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int32_t j = nn12[i];
-    if (j >= 0 && j < n2) flag[j] = 1;
-  }
-}
-
-__device__ __forceinline__ void image_flags4(const uint8_t* flag, int64_t n2, int64_t j,
-                                             bool (&f)[4]) {
-  if (j + 3 < n2) {
-    const uchar4 v = *reinterpret_cast<const uchar4*>(flag + j);  // j is a multiple of 4
-    f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  if ((reinterpret_cast<uintptr_t>(nn12) & 15) == 0) {
+    const int64_t n4 = n1 >> 2;
+    for (int64_t q = t; q < n4; q += stride) {
+      const int4 v = *reinterpret_cast<const int4*>(nn12 + 4 * q);
+      if (v.x >= 0 && v.x < n2) flag[v.x] = 1;
+      if (v.y >= 0 && v.y < n2) flag[v.y] = 1;
+      if (v.z >= 0 && v.z < n2) flag[v.z] = 1;
+      if (v.w >= 0 && v.w < n2) flag[v.w] = 1;
+    }
+    for (int64_t i = 4 * n4 + t; i < n1; i += stride) {
+      const int32_t j = nn12[i];
+      if (j >= 0 && j < n2) flag[j] = 1;
+    }
   } else {
-#pragma unroll
-    for (int r = 0; r < 4; ++r) f[r] = j + r < n2 && flag[j + r];
+    for (int64_t i = t; i < n1; i += stride) {
+      const int32_t j = nn12[i];
+      if (j >= 0 && j < n2) flag[j] = 1;
+    }
   }
 }
 
-__global__ void __launch_bounds__(1024) image_rows_count_kernel(const uint8_t* __restrict__ flag,
-                                                                int64_t n2,
-                                                                int32_t* __restrict__ block_cnt) {
+// Bit r of the result: flag[j + r] is set (r < 16; rows at or past n2 read 0).
+__device__ __forceinline__ uint32_t image_flags16(const uint8_t* flag, int64_t n2, int64_t j) {
+  uint32_t bits = 0;
+  if (j + 15 < n2) {
+    const uint4 v = *reinterpret_cast<const uint4*>(flag + j);  // j is a multiple of 16
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int b = 0; b < 4; ++b)
+        bits |= (((w[q] >> (8 * b)) & 0xFFu) != 0u ? 1u : 0u) << (4 * q + b);
+  } else {
+    for (int r = 0; r < 16; ++r)
+      if (j + r < n2 && flag[j + r]) bits |= 1u << r;
+  }
+  return bits;
+}
+
+__global__ void __launch_bounds__(kImgThreads) image_rows_count_kernel(
+    const uint8_t* __restrict__ flag, int64_t n2, int32_t* __restrict__ block_cnt) {
   __shared__ int sm[32];
-  bool f[4];
-  image_flags4(flag, n2, blockIdx.x * static_cast<int64_t>(kMutBlockRows) + 4 * threadIdx.x, f);
-  int c = (f[0] ? 1 : 0) + (f[1] ? 1 : 0) + (f[2] ? 1 : 0) + (f[3] ? 1 : 0);
+  const int64_t j =
+      blockIdx.x * static_cast<int64_t>(kMutBlockRows) + kImgFlagsPerThread * threadIdx.x;
+  int c = __popc(image_flags16(flag, n2, j));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
   if ((threadIdx.x & 31) == 0) sm[threadIdx.x >> 5] = c;
   __syncthreads();
   if (threadIdx.x == 0) {
     int t = 0;
-    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) t += sm[w];
+    for (int w = 0; w < kImgThreads / 32; ++w) t += sm[w];
     block_cnt[blockIdx.x] = t;
   }
 }
 
-__global__ void __launch_bounds__(1024) image_rows_emit_kernel(const uint8_t* __restrict__ flag,
-                                                               int64_t n2,
-                                                               const int32_t* __restrict__ off,
-                                                               int32_t* __restrict__ rows) {
+// The block's rows are staged in shared memory in order and stored with
+// consecutive threads writing consecutive words.
+__global__ void __launch_bounds__(kImgThreads) image_rows_emit_kernel(
+    const uint8_t* __restrict__ flag, int64_t n2, const int32_t* __restrict__ off,
+    int32_t* __restrict__ rows) {
   __shared__ int sm[32];
-  const int64_t j = blockIdx.x * static_cast<int64_t>(kMutBlockRows) + 4 * threadIdx.x;
-  bool f[4];
-  image_flags4(flag, n2, j, f);
-  const int c = (f[0] ? 1 : 0) + (f[1] ? 1 : 0) + (f[2] ? 1 : 0) + (f[3] ? 1 : 0);
-  int pos = off[blockIdx.x] + block_exclusive_scan(c, sm);
-#pragma unroll
-  for (int r = 0; r < 4; ++r)
-    if (f[r]) rows[pos++] = static_cast<int32_t>(j + r);
+  __shared__ int32_t stage[kMutBlockRows];
+  const int64_t j0 = blockIdx.x * static_cast<int64_t>(kMutBlockRows);
+  const int64_t j = j0 + kImgFlagsPerThread * threadIdx.x;
+  uint32_t bits = image_flags16(flag, n2, j);
+  int p = block_exclusive_scan(__popc(bits), sm);
+  while (bits) {
+    const int r = __ffs(bits) - 1;
+    bits &= bits - 1;
+    stage[p++] = static_cast<int32_t>(j + r);
+  }
+  int total = 0;
+  for (int w = 0; w < kImgThreads / 32; ++w) total += sm[w];
+  __syncthreads();
+  int32_t* dst = rows + off[blockIdx.x];
+  for (int k = threadIdx.x; k < total; k += kImgThreads) dst[k] = stage[k];
 }
 
 // ------------------------------------------------------------ decode nn ---
@@ -857,16 +921,17 @@ static int launch_mutual_impl(const MutualSrc& m, int32_t* block_scratch, int dt
                               int32_t* out_pairs, void* out_score, int64_t cap,
                               int32_t* out_count, cudaStream_t st) {
   const int nb = mutual_blocks(m.n1);
-  mutual_count_kernel<<<nb, 1024, 0, st>>>(m, block_scratch);
+  mutual_count_kernel<<<nb, kMutThreads, 0, st>>>(m, block_scratch);
   mutual_scan_kernel<<<1, 1024, 0, st>>>(block_scratch, nb, out_count);
   if (dtype == FASTNN_I8)
-    mutual_emit_kernel<FASTNN_I8><<<nb, 1024, 0, st>>>(m, block_scratch, out_pairs, out_score, cap);
+    mutual_emit_kernel<FASTNN_I8><<<nb, kMutThreads, 0, st>>>(m, block_scratch, out_pairs,
+                                                              out_score, cap);
   else if (dtype == FASTNN_F32_L2)
-    mutual_emit_kernel<FASTNN_F32_L2><<<nb, 1024, 0, st>>>(m, block_scratch, out_pairs, out_score,
-                                                           cap);
+    mutual_emit_kernel<FASTNN_F32_L2><<<nb, kMutThreads, 0, st>>>(m, block_scratch, out_pairs,
+                                                                  out_score, cap);
   else
-    mutual_emit_kernel<FASTNN_BF16><<<nb, 1024, 0, st>>>(m, block_scratch, out_pairs, out_score,
-                                                         cap);
+    mutual_emit_kernel<FASTNN_BF16><<<nb, kMutThreads, 0, st>>>(m, block_scratch, out_pairs,
+                                                                out_score, cap);
   FASTNN_CUDA_TRY(cudaGetLastError());
   return FASTNN_OK;
 }
@@ -922,9 +987,9 @@ int launch_image_rows(const int32_t* nn12, int64_t n1, int64_t n2, uint8_t* flag
   const int nb = mutual_blocks(n2);
   FASTNN_CUDA_TRY(cudaMemsetAsync(flag, 0, static_cast<size_t>(n2), st));
   if (n1 > 0) image_flag_kernel<<<grid_for(n1, 256), 256, 0, st>>>(nn12, n1, n2, flag);
-  image_rows_count_kernel<<<nb, 1024, 0, st>>>(flag, n2, block_scratch);
+  image_rows_count_kernel<<<nb, kImgThreads, 0, st>>>(flag, n2, block_scratch);
   mutual_scan_kernel<<<1, 1024, 0, st>>>(block_scratch, nb, count);
-  image_rows_emit_kernel<<<nb, 1024, 0, st>>>(flag, n2, block_scratch, rows);
+  image_rows_emit_kernel<<<nb, kImgThreads, 0, st>>>(flag, n2, block_scratch, rows);
   FASTNN_CUDA_TRY(cudaGetLastError());
   return kernel_timer_end(slot, st);
 }

@@ -277,12 +277,16 @@ __device__ void compact_pair(const CompactArgs& c, const FrontierBufs& fb, int b
 // frontier is empty or after max_iter rounds. `nn(dir, q)` runs one
 // nearest-neighbour pass over the whole grid (dir 0: r.fwd, 1: r.bwd) and
 // ends with a CTA barrier. `cta_abort` is the CTA's own abort flag (shared
-// memory); `flag`, `more` and `scan` (66 ints) are shared scratch.
+// memory); `flag`, `more` and `scan` (66 ints) are shared scratch, and
+// `cnt_cache` (one int per pair) the planner's count cache: the backward pass
+// plans from the forward pass's counts, and each later forward pass from the
+// counts the check after the compaction read.
 // `prologue()` runs in every CTA beside the clearing of the per-call state,
 // before the first grid barrier.
 template <int DT, class NNPass, class Prologue>
 __device__ void fast_rounds(const RecArgs& r, NNPass&& nn, Prologue&& prologue,
-                            volatile int* cta_abort, int* flag, int* more, int* scan) {
+                            volatile int* cta_abort, int* flag, int* more, int* scan,
+                            int* cnt_cache) {
   uint32_t target = 0;
   const int batch = r.batch;
   const int64_t S = r.S;
@@ -343,9 +347,9 @@ __device__ void fast_rounds(const RecArgs& r, NNPass&& nn, Prologue&& prologue,
     // <D2[v], D1[u']> in the forward pass, and a match v reaches at least its
     // forward score <D1[u], D2[v]> in the backward pass (the same dot
     // product). The seeds of round 1 have none.
-    nn(0, PhaseQ{r.F[cur], r.cnt[cur], t > 1 ? r.Bd[cur] : nullptr, 1});
+    nn(0, PhaseQ{r.F[cur], r.cnt[cur], t > 1 ? r.Bd[cur] : nullptr, 1, t > 1 ? 1 : 0});
     if (!sync()) break;
-    nn(1, PhaseQ{nullptr, r.cnt[cur], reinterpret_cast<const uint32_t*>(r.cmp.fwd_key) + 1, 2});
+    nn(1, PhaseQ{nullptr, r.cnt[cur], reinterpret_cast<const uint32_t*>(r.cmp.fwd_key) + 1, 2, 1});
     if (!sync()) break;
     const FrontierBufs fb{r.F[cur], r.F[nxt], r.cnt[cur], r.cnt[nxt], r.Bd[nxt]};
     for (int b = blockIdx.x; b < batch; b += gridDim.x)
@@ -354,7 +358,11 @@ __device__ void fast_rounds(const RecArgs& r, NNPass&& nn, Prologue&& prologue,
     // Every CTA reads the same counts after the barrier: a uniform exit.
     if (threadIdx.x == 0) {
       int any = 0;
-      for (int b = 0; b < batch; ++b) any |= __ldcg(r.cnt[nxt] + b);
+      for (int b = 0; b < batch; ++b) {
+        const int c = __ldcg(r.cnt[nxt] + b);
+        cnt_cache[b] = c;
+        any |= c;
+      }
       *more = any != 0 ? 1 : 0;
     }
     __syncthreads();

@@ -224,7 +224,7 @@ __device__ void l2_plan(const NNArgs& a, const PhaseQ& q, L2Smem& s) {
   s.wait_ns = wait_limit(a.wait_ns);
   int64_t total = 0;
   for (int b = 0; b < a.batch; ++b) {
-    const int64_t c = nn_count(a, q, b);
+    const int64_t c = q.cached ? s.cnt[b] : nn_count(a, q, b);
     const int64_t rows = a.ndb_dev ? min(static_cast<int64_t>(__ldcg(a.ndb_dev + b)), a.ndb)
                                    : a.ndb;
     const int nt = static_cast<int>(rows > 0 ? (rows + kDC - 1) / kDC : 0);
@@ -589,7 +589,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto boxes = [&] {
     if (r.fwd.db_box && r.bwd.db_box) l2_boxes(r);
   };
-  fast_rounds<FASTNN_F32_L2>(r, pass, boxes, &s.abort_flag, &s.grid_ok, &s.more, s.scan);
+  fast_rounds<FASTNN_F32_L2>(r, pass, boxes, &s.abort_flag, &s.grid_ok, &s.more, s.scan, s.cnt);
   l2_teardown(s, r.status);
 }
 

@@ -50,6 +50,7 @@ constexpr int kMaxStages = 6;                   // database ring slots laid out 
 // 32- and 64-byte rows, 4 (128 KB) for 128-byte rows.
 __host__ __device__ constexpr int stages_for(int rb) { return rb == 128 ? 4 : 6; }
 constexpr int kGroupWarps = 8;                  // epilogue warps per accumulator
+constexpr int kPreTiles = 1;                    // database tiles requested before a phase's first gather
 constexpr int kEpiWarps = kAcc * kGroupWarps;
 constexpr int kProducerWarp = kEpiWarps;
 constexpr int kMmaWarp0 = kEpiWarps + 1;        // MMA issuers: warp kMmaWarp0 + g feeds accumulator g
@@ -62,6 +63,10 @@ constexpr int kMaxBatch = 1024;
 // a single segment of the same length).
 constexpr int64_t kSegCost = 8;
 constexpr int kStashBytes = kEpiWarps * 32 * 32;  // 32 B per epilogue thread
+// Segment-end partial results of the int8 epilogue (two parities); the
+// 16-bit float paths search their columns exactly and need none.
+constexpr int kPartBytes = 2 * kEpiWarps * 32 * 16;
+__host__ __device__ constexpr int part_bytes(int dtype) { return dtype == FASTNN_I8 ? kPartBytes : 0; }
 
 // Barrier slots inside the barrier block.
 constexpr int kBarBFull = 0;
@@ -105,9 +110,9 @@ __host__ __device__ constexpr size_t tile_bytes_a(int rb) { return static_cast<s
 __host__ __device__ constexpr size_t tile_bytes_b(int rb) { return static_cast<size_t>(kBN) * rb; }
 __host__ __device__ constexpr size_t ctl_bytes() { return (sizeof(Ctl) + 15) & ~static_cast<size_t>(15); }
 
-size_t smem_bytes(int rb) {
+size_t smem_bytes(int rb, int dtype) {
   return 1024 /* alignment slack */ + 2 * tile_bytes_a(rb) + stages_for(rb) * tile_bytes_b(rb) +
-         ctl_bytes() + kStashBytes;
+         ctl_bytes() + kStashBytes + part_bytes(dtype);
 }
 
 // Bounded wait on an mbarrier phase. Returns false (and raises the abort flag
@@ -385,29 +390,32 @@ __device__ __forceinline__ void fold_pack16(const uint32_t (&r)[NC][16], uint32_
 
 // The lowest column among the 16 from bidx whose int8 dot product with the
 // query equals best (one exists: the tile's tree found best in this group).
-// Rows are read from the repacked maps (L2): RB bytes of zero-padded int8; a
-// query row outside the source is the zero vector, as the query gather
-// treats it. Loads go in batches of four rows.
+// The query is row r of the segment's query tile in shared memory (RB bytes of
+// zero-padded int8, 16-byte chunks swizzled as the gather wrote them); the
+// candidate rows are read from the repacked database (L2) in batches of
+// four, a lane stopping at the batch that holds its column.
 template <int RB>
-__device__ __noinline__ uint32_t resolve_group(const uint8_t* __restrict__ qrow,
+__device__ __noinline__ uint32_t resolve_group(const uint8_t* qtile, int r,
                                                const uint8_t* __restrict__ db, uint32_t bidx,
                                                int best) {
-  constexpr int NV = RB / 16;  // 16-byte words per row
+  constexpr int NV = RB / 16;           // 16-byte words per row
+  constexpr int kRows = 4;              // candidate rows per batch of loads
+  const int swz = RB == 32 ? ((r >> 2) & 1) : ((r >> 1) & 3);
   int4 qv[NV];
 #pragma unroll
   for (int i = 0; i < NV; ++i)
-    qv[i] = qrow ? __ldg(reinterpret_cast<const int4*>(qrow) + i) : make_int4(0, 0, 0, 0);
+    qv[i] = *reinterpret_cast<const int4*>(qtile + r * RB + 16 * (i ^ swz));
   uint32_t found = 0xFFFFFFFFu;
 #pragma unroll 1
-  for (int c0 = 0; c0 < 16 && found == 0xFFFFFFFFu; c0 += 4) {
-    int4 rv[4][NV];
+  for (int c0 = 0; c0 < 16 && found == 0xFFFFFFFFu; c0 += kRows) {
+    int4 rv[kRows][NV];
 #pragma unroll
-    for (int c = 0; c < 4; ++c)
+    for (int c = 0; c < kRows; ++c)
 #pragma unroll
       for (int i = 0; i < NV; ++i)
         rv[c][i] = __ldg(reinterpret_cast<const int4*>(db + static_cast<int64_t>(bidx + c0 + c) * RB) + i);
 #pragma unroll
-    for (int c = 3; c >= 0; --c) {
+    for (int c = kRows - 1; c >= 0; --c) {
       int s = 0;
 #pragma unroll
       for (int i = 0; i < NV; ++i) {
@@ -472,6 +480,7 @@ struct SmemLayout {
   uint8_t* tileB;  // stages_for(RB) x kBN x RB database tiles
   Ctl* ctl;
   uint4* stash;    // 32 B per epilogue thread
+  uint4* part;     // 2 x kEpiWarps x 32 segment-end partial results
 };
 
 template <int RB>
@@ -484,6 +493,7 @@ __device__ __forceinline__ SmemLayout smem_layout() {
   L.tileB = base + 2 * tile_bytes_a(RB);
   L.ctl = reinterpret_cast<Ctl*>(L.tileB + stages_for(RB) * tile_bytes_b(RB));
   L.stash = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(L.ctl) + ctl_bytes());
+  L.part = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(L.stash) + kStashBytes);  // int8 only
   return L;
 }
 
@@ -492,9 +502,11 @@ __device__ __forceinline__ SmemLayout smem_layout() {
 struct PipeState {
   uint32_t ephase = 0;  // phase bit of this group's accumulator barrier
   int epar = 0;         // parity of the running unit index
+  int eseg = 0;         // parity of the running segment index (the query tile)
 };
 
 // Barrier init and TMEM allocation; ends with a CTA barrier.
+template <int DT>
 __device__ __forceinline__ void pipe_setup(Ctl* ctl) {
   if (threadIdx.x == 0) {
     ctl->abort_flag = 0;
@@ -514,7 +526,9 @@ __device__ __forceinline__ void pipe_setup(Ctl* ctl) {
     for (int i = 0; i < kNumBars; ++i) {
       uint32_t count = 1;
       if (i >= kBarAFull && i < kBarAFull + 2) count = 32;    // producer lanes
-      if (i >= kBarAEmpty && i < kBarAEmpty + 2) count = kAcc;  // one commit per MMA issuer
+      // One commit per MMA issuer; with int8 scores also one arrival per
+      // lane quarter's leader, whose column searches read the query tile.
+      if (i >= kBarAEmpty && i < kBarAEmpty + 2) count = kAcc + (DT == FASTNN_I8 ? 4 : 0);
       if (i == kBarDone) count = kAcc;
       if (i >= kBarAccEmpty && i < kBarAccEmpty + kAcc) count = kGroupWarps;
       ptx::mbar_init(ptx::smem_u32(&ctl->bars[i]), count);
@@ -546,7 +560,7 @@ __device__ void plan_phase(const NNArgs& a, const PhaseQ& q, Ctl* ctl) {
   }
   ctl->wait_ns = wait_limit(a.wait_ns);
   for (int b = 0; b < batch; ++b) {
-    const int64_t c = nn_count(a, q, b);
+    const int64_t c = q.cached ? ctl->cnt[b] : nn_count(a, q, b);
     const int64_t rows = a.ndb_dev ? min(static_cast<int64_t>(__ldcg(a.ndb_dev + b)), a.ndb)
                                    : a.ndb;
     const int64_t nt = rows > 0 ? (rows + kBN - 1) / kBN : 0;
@@ -560,6 +574,13 @@ __device__ void plan_phase(const NNArgs& a, const PhaseQ& q, Ctl* ctl) {
   // starting it (query gather, pipeline refill, result flush), so that a CTA
   // whose range starts a new segment takes that many fewer units.
   const int64_t G = gridDim.x;
+  // Quotients of non-negative values; 32-bit division when both fit (the
+  // 64-bit one is a long dependent sequence on this single thread).
+  auto div = [](int64_t x, int64_t y) -> int64_t {
+    return (x <= 0x7fffffff && y <= 0x7fffffff)
+               ? static_cast<int64_t>(static_cast<uint32_t>(x) / static_cast<uint32_t>(y))
+               : x / y;
+  };
   int64_t cost = 0;
   for (int b = 0; b < batch; ++b) cost += static_cast<int64_t>(ctl->mt[b]) * (ctl->nt[b] + kSegCost);
   // Unit index at cost position C (monotone in C; 0 at 0, total at cost).
@@ -578,7 +599,7 @@ __device__ void plan_phase(const NNArgs& a, const PhaseQ& q, Ctl* ctl) {
     m_out = n_out = 0;
     if (b >= batch) return units;
     const int64_t segc = ctl->nt[b] + kSegCost;
-    const int64_t j = (C - acc) / segc;
+    const int64_t j = div(C - acc, segc);
     const int64_t off = max(static_cast<int64_t>(0), (C - acc) - j * segc - kSegCost);
     m_out = j;
     n_out = off;
@@ -586,8 +607,8 @@ __device__ void plan_phase(const NNArgs& a, const PhaseQ& q, Ctl* ctl) {
   };
   int b, b_end;
   int64_t m0, n0, m_end, n_end;
-  ctl->u0 = unit_at(cost * blockIdx.x / G, b, m0, n0);
-  ctl->u1 = unit_at(cost * (blockIdx.x + 1) / G, b_end, m_end, n_end);
+  ctl->u0 = unit_at(div(cost * blockIdx.x, G), b, m0, n0);
+  ctl->u1 = unit_at(div(cost * (blockIdx.x + 1), G), b_end, m_end, n_end);
   ctl->b0 = b;
   ctl->m0 = m0;
   ctl->n0 = n0;
@@ -623,31 +644,41 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Pha
       Ring st;
       st.idx = ctl->p_st_idx;
       st.phase = ctl->p_st_phase;
+      // At the phase start every stage is free: the first kPreTiles database
+      // tiles are requested before the query gather, so that their latency
+      // overlaps the gather's dependent loads. (All free stages at once was
+      // measured slower: every CTA's burst of tile loads delays the gathers.)
+      auto load_b = [&](int32_t row) {
+        if (!wait_bounded(bar(kBarBEmpty + st.idx), st.phase ^ 1u, ctl, a.status)) return false;
+        ptx::mbar_arrive_expect_tx(bar(kBarBFull + st.idx), static_cast<uint32_t>(tile_bytes_b(RB)));
+        ptx::tma_load_2d(ptx::smem_u32(tileB + st.idx * tile_bytes_b(RB)), tmap_db, 0, row,
+                         bar(kBarBFull + st.idx));
+        ctl->p_last_phase[st.idx] = static_cast<int>(st.phase);
+        st.next<NS>();
+        return true;
+      };
       for (int64_t u = u0; ok && u < u1; ++seg) {
         const int len = static_cast<int>(seg_len(p, u, u1, ctl));
         const int as = static_cast<int>(seg & 1);
+        const int32_t row0 = static_cast<int32_t>(static_cast<int64_t>(p.b) * a.ndb + p.n * kBN);
+        const int pre = u == u0 ? min(len, kPreTiles) : 0;
+        if (lane == 0)
+          for (int j = 0; ok && j < pre; ++j) ok = load_b(row0 + j * kBN);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
         if (!warp_wait_bounded(bar(kBarAEmpty + as), static_cast<uint32_t>(((seg >> 1) & 1) ^ 1),
                                ctl, a.status))
           break;
-        // (Issuing the database loads of free stages before the gather was
-        // measured slower: at a pass start every CTA's burst of tile loads
-        // delays the gather's dependent loads.)
         gather_a<RB>(tileA + as * tile_bytes_a(RB), a, q, p.b, p.m, ctl->cnt[p.b], lane);
         ptx::fence_proxy_async_smem();
         ptx::mbar_arrive(bar(kBarAFull + as));
         if (lane == 0) {
-          int32_t row = static_cast<int32_t>(static_cast<int64_t>(p.b) * a.ndb + p.n * kBN);
-          for (int j = 0; j < len; ++j, row += kBN) {
-            if (!wait_bounded(bar(kBarBEmpty + st.idx), st.phase ^ 1u, ctl, a.status)) {
+          int32_t row = row0 + pre * kBN;
+          for (int j = pre; j < len; ++j, row += kBN) {
+            if (!load_b(row)) {
               ok = false;
               break;
             }
-            ptx::mbar_arrive_expect_tx(bar(kBarBFull + st.idx),
-                                       static_cast<uint32_t>(tile_bytes_b(RB)));
-            ptx::tma_load_2d(ptx::smem_u32(tileB + st.idx * tile_bytes_b(RB)), tmap_db, 0, row,
-                             bar(kBarBFull + st.idx));
-            ctl->p_last_phase[st.idx] = static_cast<int>(st.phase);
-            st.next<NS>();
           }
         }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -820,21 +851,59 @@ __device__ void run_phase(const CUtensorMap* tmap_db, const NNArgs& a, const Pha
             fold_wide<DT, 2>(r, colbase + 64, best, bidx, exact, slot);
           }
         }
-        if (!ok) break;
-        if (krow < ctl->cnt[p.b] && bidx != 0xFFFFFFFFu) {
-          if constexpr (DT == FASTNN_I8 && DEFER) {
-            if (!exact) {
-              const int64_t qr = nn_query_row(a, q, p.b, krow);
-              const uint8_t* qrow = (qr >= 0 && qr < a.q_rows_per_pair)
-                                        ? a.q_rows + (p.b * a.q_rows_per_pair + qr) * RB
-                                        : nullptr;
-              bidx = resolve_group<RB>(qrow, a.db_rows + static_cast<int64_t>(p.b) * a.ndb * RB,
-                                       bidx, best);
+        const int par = ps.eseg;
+        if constexpr (DT == FASTNN_I8) {
+          // The four warps of this lane quarter (two accumulator groups x
+          // two column halves) hold partial results for the same 32 rows over
+          // disjoint columns. They meet in shared memory (double-buffered by
+          // segment parity); the leader, warp (0, 0), keeps each row's best
+          // (higher score, then lower index: the column groups are disjoint,
+          // so a group start orders like any column in it), finds its column
+          // if it is still a 16-column group, and merges it into the global
+          // key: one column search and one atomic per row instead of four.
+          // Every warp of the quarter reaches the named barrier (all waits
+          // above are bounded), and all leave the loop together when any of
+          // them failed.
+          const bool valid = ok && krow < ctl->cnt[p.b] && bidx != 0xFFFFFFFFu;
+          uint4* part = L.part + par * (kEpiWarps * 32);
+          part[warp * 32 + lane] = make_uint4(E::ord(best), bidx, exact ? 1u : 0u,
+                                              (valid ? 1u : 0u) | (ok ? 2u : 0u));
+          ptx::named_bar_sync(1 + lg, 4 * 32);
+          const int w4[4] = {lg, kGroupWarps + lg, 4 + lg, kGroupWarps + 4 + lg};
+          bool all_ok = true;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) all_ok = all_ok && (part[w4[i] * 32 + lane].w & 2u) != 0u;
+          if (!__all_sync(0xffffffffu, all_ok)) break;
+          if (grp == 0 && h == 0) {
+            uint4 bst = part[lg * 32 + lane];
+#pragma unroll
+            for (int i = 1; i < 4; ++i) {
+              const uint4 v = part[w4[i] * 32 + lane];
+              if ((v.w & 1u) && (!(bst.w & 1u) || v.x > bst.x || (v.x == bst.x && v.y < bst.y)))
+                bst = v;
             }
+            if (bst.w & 1u) {
+              const uint32_t col =
+                  bst.z != 0u ? bst.y
+                              : resolve_group<RB>(tileA + par * tile_bytes_a(RB), lg * 32 + lane,
+                                                  a.db_rows + static_cast<int64_t>(p.b) * a.ndb * RB,
+                                                  bst.y, unord_i32(bst.x));
+              atomicMax(reinterpret_cast<unsigned long long*>(&a.out_key[p.b * a.q_cap + krow]),
+                        static_cast<unsigned long long>(make_key(bst.x, col)));
+            }
+            // The query tile may be refilled once the column searches have
+            // read their rows (one arrival per lane quarter).
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar(kBarAEmpty + par));
           }
-          atomicMax(reinterpret_cast<unsigned long long*>(&a.out_key[p.b * a.q_cap + krow]),
-                    static_cast<unsigned long long>(make_key(E::ord(best), bidx)));
+        } else {
+          // Exact columns: each warp merges its own partial results.
+          if (!ok) break;
+          if (krow < ctl->cnt[p.b] && bidx != 0xFFFFFFFFu)
+            atomicMax(reinterpret_cast<unsigned long long*>(&a.out_key[p.b * a.q_cap + krow]),
+                      static_cast<unsigned long long>(make_key(E::ord(best), bidx)));
         }
+        ps.eseg ^= 1;
         u += len;
         ps.epar ^= len & 1;
         next_segment(p, ctl, batch);
@@ -872,7 +941,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     nn_tc_kernel(const __grid_constant__ CUtensorMap tmap_db, const __grid_constant__ NNArgs a) {
   const SmemLayout L = smem_layout<RB>();
   if ((threadIdx.x >> 5) == kProducerWarp && (threadIdx.x & 31) == 0) ptx::prefetch_tmap(&tmap_db);
-  pipe_setup(L.ctl);
+  pipe_setup<DT>(L.ctl);
   const uint32_t tmem = L.ctl->tmem_base;
   PipeState ps;
   run_phase<DT, RB, true>(&tmap_db, a, PhaseQ{a.q_index, a.q_count, a.q_bound, 1}, L, tmem, ps);
@@ -896,7 +965,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::prefetch_tmap(&tmap_d1);
     ptx::prefetch_tmap(&tmap_d2);
   }
-  pipe_setup(ctl);
+  pipe_setup<DT>(ctl);
   const uint32_t tmem = ctl->tmem_base;
   PipeState ps;
   auto pass = [&](int dir, const PhaseQ& q) {
@@ -920,7 +989,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                        gsize);
     }
   };
-  fast_rounds<DT>(r, pass, repack, &ctl->abort_flag, &ctl->grid_ok, &ctl->more, ctl->scan);
+  fast_rounds<DT>(r, pass, repack, &ctl->abort_flag, &ctl->grid_ok, &ctl->more, ctl->scan,
+                  ctl->cnt);
   pipe_teardown(ctl, tmem, r.status);
 }
 
@@ -1078,7 +1148,7 @@ int launch_nn_tc(const NNArgs& a, int dtype, int64_t db_total_rows, cudaStream_t
   if (rc != FASTNN_OK) return rc;
   int sms = 0;
   if ((rc = sm_count(&sms)) != FASTNN_OK) return rc;
-  const size_t smem = smem_bytes(rb);
+  const size_t smem = smem_bytes(rb, dtype);
   FASTNN_CUDA_TRY(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem)));
   NNArgs args = a;
@@ -1102,7 +1172,7 @@ int launch_reciprocal(const RecArgs& r, int dtype, int64_t d1_rows, int64_t d2_r
   if ((rc = make_tmap(&tm1, r.bwd.db_rows, d1_rows, rb)) != FASTNN_OK) return rc;
   int sms = 0;
   if ((rc = sm_count(&sms)) != FASTNN_OK) return rc;
-  const size_t smem = smem_bytes(rb);
+  const size_t smem = smem_bytes(rb, dtype);
   FASTNN_CUDA_TRY(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem)));
   int per_sm = 0;
