@@ -12,11 +12,16 @@ namespace fastnn {
 
 // Grid-wide barrier over the co-resident CTAs of a cooperative launch: a
 // monotonic arrival counter (zero before the launch); each CTA waits, bounded
-// by limit_ns, until the counter reaches its next multiple of the grid
-// size. A CTA that arrives with cta_ok == false, or a wait that runs out,
-// raises the shared abort word so that every CTA leaves. `flag` is a shared
-// int that carries thread 0's verdict to the CTA. Returns the CTA-uniform
-// verdict.
+// by limit_ns, until the counter reaches its next multiple of the grid size.
+// Thread 0 arrives with a release add and leaves with an acquire load of the
+// counter, so the CTA's writes before the barrier are visible to every CTA
+// after it, without separate fences. A CTA that arrives with cta_ok == false,
+// or whose wait runs out, sets the counter's top bit (and the shared abort
+// word, for the record): every waiter leaves at once and the barrier fails
+// for all of them. `flag` is a shared int that carries thread 0's verdict to
+// the CTA. Returns the CTA-uniform verdict.
+constexpr uint32_t kBarrierAbortBit = 0x80000000u;
+
 __device__ __forceinline__ bool grid_barrier(uint32_t* count, int* abort_word, int* status,
                                              uint32_t& target, bool cta_ok, int* flag,
                                              uint64_t limit_ns) {
@@ -24,31 +29,23 @@ __device__ __forceinline__ bool grid_barrier(uint32_t* count, int* abort_word, i
   if (threadIdx.x == 0) {
     target += gridDim.x;
     bool ok = cta_ok;
-    if (!ok) atomicExch(abort_word, 1);
-    // Release: the CTA's writes (ordered before this thread by the barrier
-    // above) become visible to every CTA that observes the arrival.
-    ptx::fence_acq_rel_gpu();
-    atomicAdd(count, 1u);
+    if (!ok) {
+      atomicExch(abort_word, 1);
+      atomicOr(count, kBarrierAbortBit);
+    }
+    ptx::red_add_release_gpu(count, 1u);
     const uint64_t t0 = ptx::globaltimer_ns();
     for (uint32_t n = 1;; ++n) {
-      if (*reinterpret_cast<volatile uint32_t*>(count) >= target) break;
-      if ((n & 63) == 0 || n == 8) {
-        if (*reinterpret_cast<volatile int*>(abort_word)) {
-          ok = false;
-          break;
-        }
-        if (ptx::globaltimer_ns() - t0 > limit_ns) {
-          atomicOr(status, kStatusTimeout);
-          atomicExch(abort_word, 1);
-          ok = false;
-          break;
-        }
+      const uint32_t c = ptx::ld_relaxed_gpu(count);
+      if ((c & kBarrierAbortBit) || c >= target) break;
+      if ((n & 63) == 0 && ptx::globaltimer_ns() - t0 > limit_ns) {
+        atomicOr(status, kStatusTimeout);
+        atomicExch(abort_word, 1);
+        atomicOr(count, kBarrierAbortBit);
+        break;
       }
     }
-    // Acquire: every other CTA's writes before its arrival are visible to
-    // this CTA after the barrier below.
-    ptx::fence_acq_rel_gpu();
-    if (*reinterpret_cast<volatile int*>(abort_word)) ok = false;
+    if (ptx::ld_acquire_gpu(count) & kBarrierAbortBit) ok = false;
     *flag = ok ? 1 : 0;
   }
   __syncthreads();
