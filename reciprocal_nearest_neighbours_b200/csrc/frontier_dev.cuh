@@ -170,11 +170,11 @@ constexpr int kCE = 4;
 // slot's claim once the claims of that pass and of all earlier passes have
 // landed: a later slot's stamp is larger and cannot undercut it. Kept pairs
 // and pushes are compacted in slot order. The round's key slots are reset to
-// 0 for the next round's atomicMax merges. `sm` holds 66 ints.
+// 0 for the next round's atomicMax merges. `cnt` is the pair's frontier
+// count (the planner's cached copy); `sm` holds 66 ints.
 template <int DT>
 __device__ void compact_pair(const CompactArgs& c, const FrontierBufs& fb, int b, int t,
-                             bool last_round, int* sm) {
-  const int cnt = __ldcg(fb.cnt_cur + b);
+                             bool last_round, int* sm, int cnt) {
   if (cnt == 0) {
     if (threadIdx.x == 0) fb.cnt_next[b] = 0;
     return;
@@ -186,9 +186,9 @@ __device__ void compact_pair(const CompactArgs& c, const FrontierBufs& fb, int b
   const uint32_t stamp_hi = static_cast<uint32_t>(t) << 24;
   const uint32_t N1 = static_cast<uint32_t>(c.N1), N2 = static_cast<uint32_t>(c.N2);
 
-  if (threadIdx.x == 0) sm[64] = __ldcg(c.out_count + b);
-  __syncthreads();
-  int out0 = sm[64], next0 = 0;
+  // Every thread reads the output count itself: the load overlaps the first
+  // pass's loads instead of costing a round trip and a barrier of its own.
+  int out0 = __ldcg(c.out_count + b), next0 = 0;
   const int per_pass = static_cast<int>(blockDim.x) * kCE;
   for (int s = 0; s < cnt; s += per_pass) {
     const int k0 = s + static_cast<int>(threadIdx.x) * kCE;
@@ -350,7 +350,7 @@ __device__ void fast_rounds(const RecArgs& r, NNPass&& nn, Prologue&& prologue,
     if (!sync()) break;
     const FrontierBufs fb{r.F[cur], r.F[nxt], r.cnt[cur], r.cnt[nxt], r.Bd[nxt]};
     for (int b = blockIdx.x; b < batch; b += gridDim.x)
-      compact_pair<DT>(r.cmp, fb, b, t, t == r.max_iter, scan);
+      compact_pair<DT>(r.cmp, fb, b, t, t == r.max_iter, scan, cnt_cache[b]);
     if (!sync()) break;
     // Every CTA reads the same counts after the barrier: a uniform exit.
     if (threadIdx.x == 0) {
