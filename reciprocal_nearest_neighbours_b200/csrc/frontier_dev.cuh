@@ -158,7 +158,7 @@ struct FrontierBufs {
 // Slots per thread and pass of the per-pair compaction: each thread loads
 // its run of kCE consecutive slots at once, so that one pass costs a few
 // dependent L2 round trips rather than a few per slot.
-constexpr int kCE = 4;
+constexpr int kCE = 6;
 
 // Round t (1-based) of the fast scheme for pair b, run by one whole CTA.
 // Slot k holds pixel u = F[k] of image 1, its forward match v = NN(D1[u], D2)
