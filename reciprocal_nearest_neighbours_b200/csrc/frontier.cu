@@ -714,15 +714,23 @@ __global__ void __launch_bounds__(kMaskEmitThreads) mask_emit_staged_kernel(Mask
         __ldg(reinterpret_cast<const uint2*>(src + bytes - 8));
   // Four rounds of 256 pixels; in round r thread t takes pixel p0 + 256 r + t,
   // so a round's kept rows go to consecutive slots from consecutive threads.
-  // The first scan's barriers also publish the staged rows.
+  // The first scan's barriers also publish the staged rows. The four rounds'
+  // keep flags are read up front, with the staging loads.
+  constexpr int kRounds = 1024 / kMaskEmitThreads;
+  bool keep[kRounds];
+#pragma unroll
+  for (int r = 0; r < kRounds; ++r) {
+    const int lr = r * kMaskEmitThreads + tid;
+    keep[r] = lr < rows && mask_kept(m, b * m.N + p0 + lr);
+  }
   int64_t base = b * m.N + m.blocks[blockIdx.x];
   uint32_t amax = 0;  // per-byte maxima of |x| (int8)
-#pragma unroll 1
-  for (int r = 0; r < 1024 / kMaskEmitThreads; ++r) {
+#pragma unroll
+  for (int r = 0; r < kRounds; ++r) {
     const int lr = r * kMaskEmitThreads + tid;  // row within the block
     const int64_t p = p0 + lr;
     const int64_t g = b * m.N + p;
-    const bool f = lr < rows && mask_kept(m, g);
+    const bool f = keep[r];
     const Scan2 sc = block_scan2(f, false, sm);
     const int64_t slot = base + sc.ex0;
     base += sc.tot0;
@@ -763,25 +771,45 @@ int launch_mask_emit_staged(const MaskArgs& m, int nb, int nbytes, cudaStream_t 
 }
 
 // Seeds of the masked fast scheme: the kept grid pixels of each pair in grid
-// order, as compacted indices (p2c), and their count. One CTA per pair.
+// order, as compacted indices (p2c), and their count. One CTA per pair; each
+// thread takes a run of up to kSeedRun consecutive seeds per pass, all of
+// whose lookups are in flight together, and one block scan of the runs'
+// counts places them.
+constexpr int kSeedRun = 8;
+
 __global__ void __launch_bounds__(1024) masked_seeds_kernel(const int32_t* __restrict__ p2c,
                                                             int64_t N1, int W1, int sub,
                                                             int64_t S, int32_t* __restrict__ F0,
                                                             int32_t* __restrict__ seed_cnt) {
-  __shared__ int sm[64];
+  __shared__ int sm[32];
   const int b = blockIdx.x;
   const int gx = (W1 + sub - 1) / sub;
+  const int64_t per_pass = static_cast<int64_t>(blockDim.x) * kSeedRun;
+  const int64_t run = (min(S, per_pass) + blockDim.x - 1) / blockDim.x;  // seeds per thread
   int base = 0;
-  for (int64_t s0 = 0; s0 < S; s0 += blockDim.x) {
-    const int64_t k = s0 + threadIdx.x;
-    int32_t pos = -1;
-    if (k < S) {
-      const int64_t u = (k / gx) * sub * static_cast<int64_t>(W1) + (k % gx) * sub;
-      pos = __ldg(p2c + b * N1 + u);
+  for (int64_t s0 = 0; s0 < S; s0 += run * blockDim.x) {
+    const int64_t k0 = s0 + threadIdx.x * run;
+    int32_t pos[kSeedRun];
+    int c = 0;
+#pragma unroll
+    for (int i = 0; i < kSeedRun; ++i) {
+      const int64_t k = k0 + i;
+      pos[i] = -1;
+      if (i < run && k < S) {
+        const int64_t u = (k / gx) * sub * static_cast<int64_t>(W1) + (k % gx) * sub;
+        pos[i] = __ldg(p2c + b * N1 + u);
+      }
     }
-    const Scan2 sc = block_scan2(pos >= 0, false, sm);
-    if (pos >= 0) F0[b * S + base + sc.ex0] = pos;
-    base += sc.tot0;
+#pragma unroll
+    for (int i = 0; i < kSeedRun; ++i) c += pos[i] >= 0 ? 1 : 0;
+    int slot = base + block_exclusive_scan(c, sm);
+#pragma unroll
+    for (int i = 0; i < kSeedRun; ++i)
+      if (pos[i] >= 0) F0[b * S + slot++] = pos[i];
+    int total = 0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) total += sm[w];
+    base += total;
+    __syncthreads();  // sm is reused by the next pass
   }
   if (threadIdx.x == 0) seed_cnt[b] = base;
 }
