@@ -274,7 +274,7 @@ __device__ void compact_pair(const CompactArgs& c, const FrontierBufs& fb, int b
 // frontier is empty or after max_iter rounds. `nn(dir, q)` runs one
 // nearest-neighbour pass over the whole grid (dir 0: r.fwd, 1: r.bwd) and
 // ends with a CTA barrier. `cta_abort` is the CTA's own abort flag (shared
-// memory); `flag`, `more` and `scan` (66 ints) are shared scratch, and
+// memory); `flag` and `scan` (66 ints) are shared scratch, and
 // `cnt_cache` (one int per pair) the planner's count cache: the backward pass
 // plans from the forward pass's counts, and each later forward pass from the
 // counts the check after the compaction read.
@@ -282,8 +282,7 @@ __device__ void compact_pair(const CompactArgs& c, const FrontierBufs& fb, int b
 // before the first grid barrier.
 template <int DT, class NNPass, class Prologue>
 __device__ void fast_rounds(const RecArgs& r, NNPass&& nn, Prologue&& prologue,
-                            volatile int* cta_abort, int* flag, int* more, int* scan,
-                            int* cnt_cache) {
+                            volatile int* cta_abort, int* flag, int* scan, int* cnt_cache) {
   uint32_t target = 0;
   const int batch = r.batch;
   const int64_t S = r.S;
@@ -352,18 +351,15 @@ __device__ void fast_rounds(const RecArgs& r, NNPass&& nn, Prologue&& prologue,
     for (int b = blockIdx.x; b < batch; b += gridDim.x)
       compact_pair<DT>(r.cmp, fb, b, t, t == r.max_iter, scan, cnt_cache[b]);
     if (!sync()) break;
-    // Every CTA reads the same counts after the barrier: a uniform exit.
-    if (threadIdx.x == 0) {
-      int any = 0;
-      for (int b = 0; b < batch; ++b) {
-        const int c = __ldcg(r.cnt[nxt] + b);
-        cnt_cache[b] = c;
-        any |= c;
-      }
-      *more = any != 0 ? 1 : 0;
+    // Every CTA reads the same counts after the barrier: a uniform exit. The
+    // pairs' counts are read by as many threads, all loads in flight at once.
+    int any = 0;
+    for (int b = threadIdx.x; b < batch; b += blockDim.x) {
+      const int c = __ldcg(r.cnt[nxt] + b);
+      cnt_cache[b] = c;
+      any |= c;
     }
-    __syncthreads();
-    if (!*reinterpret_cast<volatile int*>(more)) break;
+    if (!__syncthreads_or(any != 0)) break;
   }
 }
 

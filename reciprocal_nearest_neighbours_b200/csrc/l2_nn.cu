@@ -95,7 +95,6 @@ struct __align__(16) L2Smem {
   int empty_cnt[kNS];       // warps done with the buffer's current chunk
   int abort_flag;
   int grid_ok;
-  int more;
   int b0;
   unsigned long long wait_ns;  // limit of the pipeline's bounded waits
   long long u0, u1, m0, n0;
@@ -589,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto boxes = [&] {
     if (r.fwd.db_box && r.bwd.db_box) l2_boxes(r);
   };
-  fast_rounds<FASTNN_F32_L2>(r, pass, boxes, &s.abort_flag, &s.grid_ok, &s.more, s.scan, s.cnt);
+  fast_rounds<FASTNN_F32_L2>(r, pass, boxes, &s.abort_flag, &s.grid_ok, s.scan, s.cnt);
   l2_teardown(s, r.status);
 }
 

@@ -95,7 +95,6 @@ struct Ctl {
   int abort_flag;
   int pack16;
   int grid_ok;
-  int more;
   uint64_t wait_ns;  // limit of the bounded waits in force (kTimeoutNs while draining)
   int scan[66];  // block-scan scratch of the per-pair compaction
   int b0;
@@ -989,8 +988,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                        gsize);
     }
   };
-  fast_rounds<DT>(r, pass, repack, &ctl->abort_flag, &ctl->grid_ok, &ctl->more, ctl->scan,
-                  ctl->cnt);
+  fast_rounds<DT>(r, pass, repack, &ctl->abort_flag, &ctl->grid_ok, ctl->scan, ctl->cnt);
   pipe_teardown(ctl, tmem, r.status);
 }
 
