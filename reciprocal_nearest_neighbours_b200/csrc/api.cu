@@ -129,7 +129,7 @@ MutLayout carve_mut(Carver& c, int64_t n1, int64_t n2, int d, int dtype) {
   L.d2rep = c.take<uint8_t>(static_cast<size_t>(n2 + kPadRows) * rb);
   L.k12 = c.take<uint64_t>(static_cast<size_t>(n1));
   L.k21 = c.take<uint64_t>(static_cast<size_t>(n2));
-  L.blocks = c.take<int32_t>(static_cast<size_t>(mutual_blocks(n1)));
+  L.blocks = c.take<int32_t>(static_cast<size_t>(mutual_scratch_ints(n1)));
   L.pos21 = c.take<int32_t>(static_cast<size_t>(n2));
   L.list21 = c.take<int32_t>(static_cast<size_t>(n2));
   L.cnt21 = c.take<int32_t>(1);
@@ -199,7 +199,7 @@ size_t fastnn_workspace_size(int op, int64_t n1, int64_t n2, int d, int dtype, i
       carve_mut(c, n1, n2, d, dtype);
       break;
     case FASTNN_OP_MUTUAL_FROM_NN:
-      c.take<int32_t>(static_cast<size_t>(mutual_blocks(n1 > 0 ? n1 : 1)));
+      c.take<int32_t>(static_cast<size_t>(mutual_scratch_ints(n1 > 0 ? n1 : 1)));
       break;
     case FASTNN_OP_IMAGE_ROWS:
       c.take<uint8_t>(static_cast<size_t>(n2));
@@ -561,7 +561,7 @@ int fastnn_mutual_from_nn(const int32_t* nn12, const void* score12, int64_t n1, 
   if (workspace_bytes < fastnn_workspace_size(FASTNN_OP_MUTUAL_FROM_NN, n1, n2, 1, dtype, 1, 0))
     return FASTNN_ERR_CAPACITY;
   Carver c{static_cast<uint8_t*>(workspace)};
-  int32_t* blocks = c.take<int32_t>(static_cast<size_t>(mutual_blocks(n1)));
+  int32_t* blocks = c.take<int32_t>(static_cast<size_t>(mutual_scratch_ints(n1)));
   MutualSrc m{};
   m.nn12 = nn12;
   m.nn21 = nn21;

@@ -149,10 +149,9 @@ constexpr int kMutBlockRows = 4096;
 constexpr int kMutRowsPerThread = 8;
 constexpr int kMutThreads = kMutBlockRows / kMutRowsPerThread;
 
-// Flags (and partners) of rows i .. i + 3 (local indices). The partners'
-// back-matches are loaded together, after all four partners are known.
-__device__ __forceinline__ void mutual_flags4(const MutualSrc& m, int64_t i, bool (&f)[4],
-                                              uint32_t (&j)[4]) {
+// Partners NN12 of rows i .. i + 3 (local indices).
+__device__ __forceinline__ void mutual_partners4(const MutualSrc& m, int64_t i,
+                                                 uint32_t (&j)[4]) {
   const bool full = i + 3 < m.n1;
   if (m.k12) {
     uint64_t k[4] = {0, 0, 0, 0};
@@ -175,6 +174,13 @@ __device__ __forceinline__ void mutual_flags4(const MutualSrc& m, int64_t i, boo
       for (int r = 0; r < 4; ++r) j[r] = i + r < m.n1 ? static_cast<uint32_t>(m.nn12[i + r]) : 0xFFFFFFFFu;
     }
   }
+}
+
+// Flags (and partners) of rows i .. i + 3. The partners' back-matches are
+// loaded together, after all four partners are known.
+__device__ __forceinline__ void mutual_flags4(const MutualSrc& m, int64_t i, bool (&f)[4],
+                                              uint32_t (&j)[4]) {
+  mutual_partners4(m, i, j);
   uint32_t back[4];
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
@@ -186,8 +192,11 @@ __device__ __forceinline__ void mutual_flags4(const MutualSrc& m, int64_t i, boo
   }
 }
 
+// The count pass also records each thread's eight keep flags as one byte, so
+// that the emit pass reads them instead of gathering the back-matches again.
 __global__ void __launch_bounds__(kMutThreads) mutual_count_kernel(MutualSrc m,
-                                                                   int32_t* __restrict__ block_cnt) {
+                                                                   int32_t* __restrict__ block_cnt,
+                                                                   uint8_t* __restrict__ keep) {
   __shared__ int sm[32];
   const int64_t i =
       blockIdx.x * static_cast<int64_t>(kMutBlockRows) + kMutRowsPerThread * threadIdx.x;
@@ -195,9 +204,11 @@ __global__ void __launch_bounds__(kMutThreads) mutual_count_kernel(MutualSrc m,
   uint32_t j[2][4];
   mutual_flags4(m, i, f[0], j[0]);
   mutual_flags4(m, i + 4, f[1], j[1]);
-  int c = 0;
+  uint32_t bits = 0;
 #pragma unroll
-  for (int r = 0; r < 8; ++r) c += f[r >> 2][r & 3] ? 1 : 0;
+  for (int r = 0; r < 8; ++r) bits |= (f[r >> 2][r & 3] ? 1u : 0u) << r;
+  keep[blockIdx.x * static_cast<int64_t>(kMutThreads) + threadIdx.x] = static_cast<uint8_t>(bits);
+  int c = __popc(bits);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
   if ((threadIdx.x & 31) == 0) sm[threadIdx.x >> 5] = c;
@@ -280,54 +291,63 @@ __global__ void __launch_bounds__(1024) mutual_scan_kernel(int32_t* __restrict__
   if (threadIdx.x == 0) *out_count = carry;
 }
 
+// The emit pass: the block's kept pairs (and scores) are placed in shared
+// memory in row order, then stored to consecutive output slots by
+// consecutive threads.
+constexpr int kMutEmitSmem = kMutBlockRows * (8 + 4);
+
 template <int DT>
 __global__ void __launch_bounds__(kMutThreads) mutual_emit_kernel(
-    MutualSrc m, const int32_t* __restrict__ block_off, int32_t* __restrict__ out_pairs,
-    void* __restrict__ out_score, int64_t cap) {
+    MutualSrc m, const int32_t* __restrict__ block_off, const uint8_t* __restrict__ keep,
+    int32_t* __restrict__ out_pairs, void* __restrict__ out_score, int64_t cap) {
+  extern __shared__ __align__(16) uint8_t mut_stage[];
+  int2* sp = reinterpret_cast<int2*>(mut_stage);
+  uint32_t* ss = reinterpret_cast<uint32_t*>(mut_stage + kMutBlockRows * 8);
   __shared__ int sm[32];
   const int64_t i =
       blockIdx.x * static_cast<int64_t>(kMutBlockRows) + kMutRowsPerThread * threadIdx.x;
-  bool f[2][4];
+  const uint32_t bits = keep[blockIdx.x * static_cast<int64_t>(kMutThreads) + threadIdx.x];
   uint32_t j[2][4];
-  mutual_flags4(m, i, f[0], j[0]);
-  mutual_flags4(m, i + 4, f[1], j[1]);
-  int c = 0;
-#pragma unroll
-  for (int r = 0; r < 8; ++r) c += f[r >> 2][r & 3] ? 1 : 0;
-  int64_t pos = block_off[blockIdx.x] + block_exclusive_scan(c, sm);
-  const bool pair8 = (reinterpret_cast<uintptr_t>(out_pairs) & 7) == 0;
+  mutual_partners4(m, i, j[0]);
+  mutual_partners4(m, i + 4, j[1]);
+  int local = block_exclusive_scan(__popc(bits), sm);
+  int total = 0;
+  for (int w = 0; w < kMutThreads / 32; ++w) total += sm[w];
 #pragma unroll
   for (int r = 0; r < 8; ++r) {
-    if (!f[r >> 2][r & 3]) continue;
-    if (pos < cap) {
-      const int64_t ir = i + r;
-      const uint32_t jr = j[r >> 2][r & 3];
-      const int32_t a = m.map1 ? m.map1[ir] : static_cast<int32_t>(m.i0 + ir);
-      const int32_t bj = m.map2 ? m.map2[jr] : static_cast<int32_t>(jr);
-      if (pair8) {
-        *reinterpret_cast<int2*>(out_pairs + pos * 2) = make_int2(a, bj);
-      } else {
-        out_pairs[pos * 2] = a;
-        out_pairs[pos * 2 + 1] = bj;
+    if (!((bits >> r) & 1u)) continue;
+    const int64_t ir = i + r;
+    const uint32_t jr = j[r >> 2][r & 3];
+    const int32_t a = m.map1 ? m.map1[ir] : static_cast<int32_t>(m.i0 + ir);
+    const int32_t bj = m.map2 ? m.map2[jr] : static_cast<int32_t>(jr);
+    sp[local] = make_int2(a, bj);
+    if (out_score) {
+      uint32_t sv = 0;
+      if (m.k12) {
+        const uint32_t h = key_score_bits(m.k12[ir]);
+        sv = DT == FASTNN_I8      ? static_cast<uint32_t>(unord_i32(h))
+             : DT == FASTNN_F32_L2 ? __float_as_uint(-unord_f32(h))
+                                   : __float_as_uint(unord_f32(h));
+      } else if (m.score12) {
+        sv = static_cast<const uint32_t*>(m.score12)[ir];
       }
-      if (out_score) {
-        if (m.k12) {
-          const uint32_t h = key_score_bits(m.k12[ir]);
-          if (DT == FASTNN_I8)
-            static_cast<int32_t*>(out_score)[pos] = unord_i32(h);
-          else if (DT == FASTNN_F32_L2)
-            static_cast<float*>(out_score)[pos] = -unord_f32(h);
-          else
-            static_cast<float*>(out_score)[pos] = unord_f32(h);
-        } else if (m.score12) {
-          if (DT == FASTNN_I8)
-            static_cast<int32_t*>(out_score)[pos] = static_cast<const int32_t*>(m.score12)[ir];
-          else
-            static_cast<float*>(out_score)[pos] = static_cast<const float*>(m.score12)[ir];
-        }
-      }
+      ss[local] = sv;
     }
-    ++pos;
+    ++local;
+  }
+  __syncthreads();
+  const int64_t base = block_off[blockIdx.x];
+  const int n = static_cast<int>(max(static_cast<int64_t>(0), min(static_cast<int64_t>(total), cap - base)));
+  const bool pair8 = (reinterpret_cast<uintptr_t>(out_pairs) & 7) == 0;
+  for (int k = threadIdx.x; k < n; k += kMutThreads) {
+    const int2 v = sp[k];
+    if (pair8) {
+      *reinterpret_cast<int2*>(out_pairs + (base + k) * 2) = v;
+    } else {
+      out_pairs[(base + k) * 2] = v.x;
+      out_pairs[(base + k) * 2 + 1] = v.y;
+    }
+    if (out_score) static_cast<uint32_t*>(out_score)[base + k] = ss[k];
   }
 }
 
@@ -454,7 +474,9 @@ __global__ void image_flag_kernel(const int32_t* __restrict__ nn12, int64_t n1, 
   if ((reinterpret_cast<uintptr_t>(nn12) & 15) == 0) {
     const int64_t n4 = n1 >> 2;
     for (int64_t q = t; q < n4; q += stride) {
-      const int4 v = *reinterpret_cast<const int4*>(nn12 + 4 * q);
+      // Streamed with the evict-first hint, so that the flag array (one byte
+      // per image-2 row) rather than NN12 stays in L2 for the passes after.
+      const int4 v = __ldcs(reinterpret_cast<const int4*>(nn12 + 4 * q));
       if (v.x >= 0 && v.x < n2) flag[v.x] = 1;
       if (v.y >= 0 && v.y < n2) flag[v.y] = 1;
       if (v.z >= 0 && v.z < n2) flag[v.z] = 1;
@@ -602,15 +624,16 @@ __global__ void __launch_bounds__(256) mask_count_kernel(MaskArgs m) {
   const int b = blockIdx.x / m.bpp, blk = blockIdx.x % m.bpp;
   const int64_t p = static_cast<int64_t>(blk) * 1024 + 4 * threadIdx.x;
   const int64_t g = b * m.N + p;
-  int c = 0;
+  uint32_t bits = 0;
   if (m.conf && p + 3 < m.N && (reinterpret_cast<uintptr_t>(m.conf + g) & 15) == 0) {
     const float4 c4 = __ldg(reinterpret_cast<const float4*>(m.conf + g));
-    c = (c4.x >= m.threshold) + (c4.y >= m.threshold) + (c4.z >= m.threshold) +
-        (c4.w >= m.threshold);
+    bits = (c4.x >= m.threshold ? 1u : 0u) | (c4.y >= m.threshold ? 2u : 0u) |
+           (c4.z >= m.threshold ? 4u : 0u) | (c4.w >= m.threshold ? 8u : 0u);
   } else {
 #pragma unroll
-    for (int r = 0; r < 4; ++r) c += (p + r < m.N && mask_kept(m, g + r)) ? 1 : 0;
+    for (int r = 0; r < 4; ++r) bits |= (p + r < m.N && mask_kept(m, g + r)) ? (1u << r) : 0u;
   }
+  int c = __popc(bits);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
   if ((threadIdx.x & 31) == 0) sm[threadIdx.x >> 5] = c;
@@ -943,23 +966,35 @@ int launch_repack(const void* src, int64_t rows, int d, int dtype, void* dst, in
 int mutual_blocks(int64_t n1) {
   return static_cast<int>((n1 + kMutBlockRows - 1) / kMutBlockRows);
 }
+int mutual_scratch_ints(int64_t n1) {
+  const int nb = mutual_blocks(n1);
+  return nb + nb * (kMutThreads / 4);  // block counts, then one keep byte per thread
+}
 int image_blocks(int64_t n1) { return static_cast<int>((n1 + 1023) / 1024); }
 
 static int launch_mutual_impl(const MutualSrc& m, int32_t* block_scratch, int dtype,
                               int32_t* out_pairs, void* out_score, int64_t cap,
                               int32_t* out_count, cudaStream_t st) {
   const int nb = mutual_blocks(m.n1);
-  mutual_count_kernel<<<nb, kMutThreads, 0, st>>>(m, block_scratch);
+  uint8_t* keep = reinterpret_cast<uint8_t*>(block_scratch + nb);
+  mutual_count_kernel<<<nb, kMutThreads, 0, st>>>(m, block_scratch, keep);
   mutual_scan_kernel<<<1, 1024, 0, st>>>(block_scratch, nb, out_count);
-  if (dtype == FASTNN_I8)
-    mutual_emit_kernel<FASTNN_I8><<<nb, kMutThreads, 0, st>>>(m, block_scratch, out_pairs,
-                                                              out_score, cap);
-  else if (dtype == FASTNN_F32_L2)
-    mutual_emit_kernel<FASTNN_F32_L2><<<nb, kMutThreads, 0, st>>>(m, block_scratch, out_pairs,
-                                                                  out_score, cap);
-  else
-    mutual_emit_kernel<FASTNN_BF16><<<nb, kMutThreads, 0, st>>>(m, block_scratch, out_pairs,
-                                                                out_score, cap);
+  if (dtype == FASTNN_I8) {
+    FASTNN_CUDA_TRY(cudaFuncSetAttribute(mutual_emit_kernel<FASTNN_I8>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kMutEmitSmem));
+    mutual_emit_kernel<FASTNN_I8><<<nb, kMutThreads, kMutEmitSmem, st>>>(
+        m, block_scratch, keep, out_pairs, out_score, cap);
+  } else if (dtype == FASTNN_F32_L2) {
+    FASTNN_CUDA_TRY(cudaFuncSetAttribute(mutual_emit_kernel<FASTNN_F32_L2>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kMutEmitSmem));
+    mutual_emit_kernel<FASTNN_F32_L2><<<nb, kMutThreads, kMutEmitSmem, st>>>(
+        m, block_scratch, keep, out_pairs, out_score, cap);
+  } else {
+    FASTNN_CUDA_TRY(cudaFuncSetAttribute(mutual_emit_kernel<FASTNN_BF16>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kMutEmitSmem));
+    mutual_emit_kernel<FASTNN_BF16><<<nb, kMutThreads, kMutEmitSmem, st>>>(
+        m, block_scratch, keep, out_pairs, out_score, cap);
+  }
   FASTNN_CUDA_TRY(cudaGetLastError());
   return FASTNN_OK;
 }

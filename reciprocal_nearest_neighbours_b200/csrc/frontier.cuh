@@ -101,6 +101,9 @@ struct MutualSrc {
 
 // Scan scratch (ints) of the mutual test over n1 rows, and of the image list.
 int mutual_blocks(int64_t n1);
+// Scratch (ints) the mutual test takes: its block counts and one keep-flag
+// byte per eight rows.
+int mutual_scratch_ints(int64_t n1);
 int image_blocks(int64_t n1);
 // Bounding box (lo, hi; xyz) of every kL2Chunk-row chunk of each pair's
 // repacked pointmap rows [batch][N]: box[(b * nchunk + c) * 2 + {0, 1}],
