@@ -15,15 +15,17 @@
 //   producer warp: gathers the 128 query rows of a tile into shared memory
 //       (swizzled, K-major) and streams kBN-row database tiles with TMA
 //       (cp.async.bulk.tensor, no multicast) into a 4- or 6-deep ring.
-//   MMA warp (one thread): tcgen05.mma kind::i8 (int8 -> int32, K = 32) or
-//       kind::f16 (bf16 -> fp32, 2 x K = 16) into the two 256-column TMEM
-//       accumulators in turn; tcgen05.commit frees the database stage and
-//       hands the accumulator to its epilogue group.
+//   MMA warps (one thread each): tcgen05.mma kind::i8 (int8 -> int32,
+//       K = 32) or kind::f16 (bf16 -> fp32, 2 x K = 16); issuer g fills
+//       TMEM accumulator g (two of 256 columns) for every other unit;
+//       tcgen05.commit frees the database stage and hands the accumulator to
+//       its epilogue group.
 // Work: units (pair, 128-query tile, kBN-row database tile) in row-major
 // order, split into contiguous ranges of equal cost over the CTAs. A run of
-// units that share a query tile is a segment; at its end the CTA merges each
-// row's partial result with one 64-bit atomicMax, which is order
-// independent. A query may come with a score it is known to reach (the fast
+// units that share a query tile is a segment; at its end the four warps that
+// share a TMEM lane quarter merge their partial results in shared memory
+// (int8), and each row's best is merged into the global key with one 64-bit
+// atomicMax, which is order independent. A query may come with a score it is known to reach (the fast
 // scheme's previous pass); its running best then starts just below that
 // score, so that only tiles reaching it search for the column.
 // Descriptors are zero-padded to 32 elements (32 B int8 rows, 64 B bf16 rows)
