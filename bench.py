@@ -729,16 +729,18 @@ def measure_stream(K, ranks, dev, stream, flush, sample_clocks):
       repack  -- fastnn_nn of the 64M-row map against a 256-row database
                  (its query map's repack: N x 24 B read, N x 32 B written);
       mutual  -- fastnn_mutual_from_nn on 64M-row index arrays of a smooth
-                 synthetic correspondence (count, scan and ordered emit:
-                 2 x 8 B read per row, 16 B per kept pair);
+                 synthetic correspondence (test and ordered emit in one pass:
+                 NN12 and the partner's NN21 read, 2 x 4 B per row; per kept
+                 pair its score read and the pair and score written, 16 B);
       image   -- fastnn_image_rows of the same 64M-row NN12 (the list the
                  sharded dense backward pass runs on: 4 B read per row,
                  4 B written per listed image-2 row);
       mask    -- fastnn_mutual_dense_masked of the 64M-row map (confidences
                  uniform in [0, 1), threshold 0.5) against a 256-row map
-                 (map 1's compaction: 2 x 4 B of confidence and the 24 B row
-                 read per pixel, 32 B repacked row + 4 B pixel index written
-                 per kept pixel).
+                 without confidences (map 1's compaction: 4 B of confidence
+                 and the 24 B row read per pixel, 32 B repacked row + 4 B
+                 pixel index written per kept pixel; map 2's: every pixel's
+                 row read and written the same way).
     Inputs are drawn on the device from a seeded generator."""
     import torch
     import reciprocal_nearest_neighbours_b200 as fnn
@@ -801,8 +803,8 @@ def measure_stream(K, ranks, dev, stream, flush, sample_clocks):
     r = timed(fnn.FASTNN_TIME_MUTUAL,
               lambda: fnn.fastnn_mutual_from_nn(nn12, score, 0, nn21, N, out_pairs=pairs,
                                                 out_score=pscore, out_count=cnt, workspace=mws),
-              lambda: 16 * N + 16 * int(cnt.item()))
-    r["kind"] = "mutual test and ordered emit (mutual_count, mutual_scan, mutual_emit)"
+              lambda: 8 * N + 16 * int(cnt.item()))
+    r["kind"] = "mutual test and ordered emit in one pass (mutual_select)"
     r["kept"] = int(cnt.item())
     out["kernels"].append(r)
     del nn21, miss, score, pairs, pscore
@@ -828,7 +830,7 @@ def measure_stream(K, ranks, dev, stream, flush, sample_clocks):
               lambda: fnn.fastnn_mutual_dense_masked(A, db, conf1=conf, threshold=0.5,
                                                      out_pairs=mp, out_score=ms_, out_count=cnt,
                                                      workspace=wsm),
-              lambda: 8 * N + N * d + kept1 * 36 + 256 * (8 + d + 36))
+              lambda: 4 * N + N * d + kept1 * 36 + 256 * (d + 36))
     r["kind"] = ("confidence-mask compaction (mask_count, scan, mask_emit) of the 64M-row map "
                  "and of the 256-row map")
     r["kept"] = kept1

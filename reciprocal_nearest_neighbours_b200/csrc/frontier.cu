@@ -192,6 +192,37 @@ __device__ __forceinline__ void mutual_flags4(const MutualSrc& m, int64_t i, boo
   }
 }
 
+// Output score bits of rows i .. i + 3, loaded whatever the keep flags say
+// (at the usual share of kept rows every sector holds some), so that the
+// loads go out with the partners' and not after the flags: the key's score in
+// the output type (the keys were just read for the partners: cache hits), or
+// score12[i] (read once: streamed), or 0 when there is neither.
+template <int DT>
+__device__ __forceinline__ void mutual_scores4(const MutualSrc& m, int64_t i, uint32_t (&sv)[4]) {
+  const bool full = i + 3 < m.n1;
+  if (m.k12) {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const uint32_t h = i + r < m.n1 ? key_score_bits(m.k12[i + r]) : 0u;
+      sv[r] = DT == FASTNN_I8      ? static_cast<uint32_t>(unord_i32(h))
+              : DT == FASTNN_F32_L2 ? __float_as_uint(-unord_f32(h))
+                                    : __float_as_uint(unord_f32(h));
+    }
+  } else if (m.score12) {
+    const uint32_t* s = static_cast<const uint32_t*>(m.score12) + i;
+    if (full && (reinterpret_cast<uintptr_t>(s) & 15) == 0) {
+      const uint4 v = __ldcs(reinterpret_cast<const uint4*>(s));
+      sv[0] = v.x; sv[1] = v.y; sv[2] = v.z; sv[3] = v.w;
+    } else {
+#pragma unroll
+      for (int r = 0; r < 4; ++r) sv[r] = i + r < m.n1 ? s[r] : 0u;
+    }
+  } else {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) sv[r] = 0u;
+  }
+}
+
 // The count pass also records each thread's eight keep flags as one byte, so
 // that the emit pass reads them instead of gathering the back-matches again.
 __global__ void __launch_bounds__(kMutThreads) mutual_count_kernel(MutualSrc m,
@@ -307,9 +338,13 @@ __global__ void __launch_bounds__(kMutThreads) mutual_emit_kernel(
   const int64_t i =
       blockIdx.x * static_cast<int64_t>(kMutBlockRows) + kMutRowsPerThread * threadIdx.x;
   const uint32_t bits = keep[blockIdx.x * static_cast<int64_t>(kMutThreads) + threadIdx.x];
-  uint32_t j[2][4];
+  uint32_t j[2][4], sv[2][4];
   mutual_partners4(m, i, j[0]);
   mutual_partners4(m, i + 4, j[1]);
+  if (out_score) {
+    mutual_scores4<DT>(m, i, sv[0]);
+    mutual_scores4<DT>(m, i + 4, sv[1]);
+  }
   int local = block_exclusive_scan(__popc(bits), sm);
   int total = 0;
   for (int w = 0; w < kMutThreads / 32; ++w) total += sm[w];
@@ -321,18 +356,7 @@ __global__ void __launch_bounds__(kMutThreads) mutual_emit_kernel(
     const int32_t a = m.map1 ? m.map1[ir] : static_cast<int32_t>(m.i0 + ir);
     const int32_t bj = m.map2 ? m.map2[jr] : static_cast<int32_t>(jr);
     sp[local] = make_int2(a, bj);
-    if (out_score) {
-      uint32_t sv = 0;
-      if (m.k12) {
-        const uint32_t h = key_score_bits(m.k12[ir]);
-        sv = DT == FASTNN_I8      ? static_cast<uint32_t>(unord_i32(h))
-             : DT == FASTNN_F32_L2 ? __float_as_uint(-unord_f32(h))
-                                   : __float_as_uint(unord_f32(h));
-      } else if (m.score12) {
-        sv = static_cast<const uint32_t*>(m.score12)[ir];
-      }
-      ss[local] = sv;
-    }
+    if (out_score) ss[local] = sv[r >> 2][r & 3];
     ++local;
   }
   __syncthreads();
