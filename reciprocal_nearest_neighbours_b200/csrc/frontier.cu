@@ -486,9 +486,9 @@ __global__ void __launch_bounds__(1024) image_emit_kernel(const uint64_t* __rest
 // The ascending list of image-2 rows j in [0, n2) that some nn12[i] names:
 // byte flags, per-block counts, the shared scan, an ordered emit. A block of
 // kImgThreads threads covers kMutBlockRows rows (the scan's block count is
-// the dense mutual test's); thread t takes the 16 consecutive flags
-// 16t .. 16t + 15, one 16-byte load.
-constexpr int kImgFlagsPerThread = 16;
+// the dense mutual test's); thread t takes the 32 consecutive flags
+// 32t .. 32t + 31, two 16-byte loads in flight together.
+constexpr int kImgFlagsPerThread = 32;
 constexpr int kImgThreads = kMutBlockRows / kImgFlagsPerThread;
 
 __global__ void image_flag_kernel(const int32_t* __restrict__ nn12, int64_t n1, int64_t n2,
@@ -518,19 +518,21 @@ __global__ void image_flag_kernel(const int32_t* __restrict__ nn12, int64_t n1, 
   }
 }
 
-// Bit r of the result: flag[j + r] is set (r < 16; rows at or past n2 read 0).
-__device__ __forceinline__ uint32_t image_flags16(const uint8_t* flag, int64_t n2, int64_t j) {
+// Bit r of the result: flag[j + r] is set (r < 32; rows at or past n2 read 0).
+__device__ __forceinline__ uint32_t image_flags32(const uint8_t* flag, int64_t n2, int64_t j) {
   uint32_t bits = 0;
-  if (j + 15 < n2) {
-    const uint4 v = *reinterpret_cast<const uint4*>(flag + j);  // j is a multiple of 16
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  if (j + 31 < n2) {
+    // j is a multiple of 32 and the flag array starts 16-byte aligned.
+    const uint4 v0 = *reinterpret_cast<const uint4*>(flag + j);
+    const uint4 v1 = *reinterpret_cast<const uint4*>(flag + j + 16);
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
+    for (int q = 0; q < 8; ++q)
 #pragma unroll
       for (int b = 0; b < 4; ++b)
         bits |= (((w[q] >> (8 * b)) & 0xFFu) != 0u ? 1u : 0u) << (4 * q + b);
   } else {
-    for (int r = 0; r < 16; ++r)
+    for (int r = 0; r < 32; ++r)
       if (j + r < n2 && flag[j + r]) bits |= 1u << r;
   }
   return bits;
@@ -541,7 +543,7 @@ __global__ void __launch_bounds__(kImgThreads) image_rows_count_kernel(
   __shared__ int sm[32];
   const int64_t j =
       blockIdx.x * static_cast<int64_t>(kMutBlockRows) + kImgFlagsPerThread * threadIdx.x;
-  int c = __popc(image_flags16(flag, n2, j));
+  int c = __popc(image_flags32(flag, n2, j));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
   if ((threadIdx.x & 31) == 0) sm[threadIdx.x >> 5] = c;
@@ -562,7 +564,7 @@ __global__ void __launch_bounds__(kImgThreads) image_rows_emit_kernel(
   __shared__ int32_t stage[kMutBlockRows];
   const int64_t j0 = blockIdx.x * static_cast<int64_t>(kMutBlockRows);
   const int64_t j = j0 + kImgFlagsPerThread * threadIdx.x;
-  uint32_t bits = image_flags16(flag, n2, j);
+  uint32_t bits = image_flags32(flag, n2, j);
   int p = block_exclusive_scan(__popc(bits), sm);
   while (bits) {
     const int r = __ffs(bits) - 1;
