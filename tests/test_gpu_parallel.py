@@ -59,7 +59,10 @@ def test_sharded_path_single_rank_equals_dense_kernel():
 
 def test_image_rows_are_the_sorted_distinct_partners():
     rng = np.random.default_rng(3)
-    for n1, n2 in [(1, 1), (5000, 3000), (3000, 50000), (4097, 4097), (10, 8191)]:
+    # The last size exceeds the flag pass's capped grid (each thread takes
+    # several groups of four rows) and spans ~2,000 blocks of the list passes.
+    for n1, n2 in [(1, 1), (5000, 3000), (3000, 50000), (4097, 4097), (10, 8191),
+                   (10_000_003, 8_000_000)]:
         nn12 = rng.integers(-3, n2 + 3, size=n1).astype(np.int32)  # a few out of range
         rows, count = fastnn_image_rows(torch.from_numpy(nn12).cuda(), n2)
         exp = np.unique(nn12[(nn12 >= 0) & (nn12 < n2)])
